@@ -1,0 +1,474 @@
+"""Benchmark of the CSA2 decode path (one JSON line on rank 0).
+
+A step = one decode token through the whole layer stack of the workload (every
+row of the hot path: quantise-append, Full scan + pool + Top-K, Reindex, Reuse,
+sparse attention) for the whole batch.  Metric: CSA2 decode layer-steps/s (a
+layer-step = one layer for the whole batch).  Default workload: batch 64 at
+context 131072, decoder stack F+4X+15U (decode_128k).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   (the CPU oracle as the reference arm)
+
+Multi-GPU (torchrun): requests are independent, so each rank runs its own batch
+with no collective on the data path (weak scaling); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode layer-steps/s; indexer+attn HBM GB/s as % of 8 TB/s"
+UNIT = "layer-steps/s"
+HBM_FALLBACK_GBS = 6650.0
+
+
+# ------------------------------------------------------------------------------------------
+# algorithmic bytes (per op and per step)
+# ------------------------------------------------------------------------------------------
+def op_bytes(wl) -> dict:
+    """Bytes the method must move, per launch of each op (whole batch)."""
+    B, Tq, d, HI, K = wl.B, wl.Tq, wl.d_I, wl.H_I, wl.top_k
+    BT = B * Tq
+    out = {}
+    for g, grp in enumerate(wl.groups):
+        N = wl.entries(g)
+        nb = (N + 7) // 8
+        q = HI * d * 2 + HI * 4
+        if grp.pool_blocks:
+            P = grp.pool_blocks
+            per = (N * (d + 4) + 4 * N + 4 * nb + 4 * nb + 8 * min(P, nb) * 4 + 4 * P + 4 * K + 4
+                   + q)
+            out[f"index_full_g{g}"] = BT * per
+            rp = 4 * P + 8 * P * (d + 4) + 8 * P * 4 * 2 + 4 * K + 4 + q
+            out[f"index_reindex_g{g}"] = BT * rp
+        else:
+            out[f"index_full_g{g}"] = BT * (N * (d + 4) + 4 * N + 4 * N + 4 * K + 4 + q)
+        out[f"append_g{g}"] = B * max(1, wl.entries(g) - wl.first_q_pos // grp.ratio) * (
+            512 * 2 + 288 + d * 2 + d + 4)
+    n_win = min(wl.swa_len, wl.first_q_pos + 1)
+    out["attn"] = BT * (K * 288 + K * 4 + n_win * 516 + wl.H * 512 * 2 + wl.H * 512 * 4 + wl.H * 4)
+    out["swa_append"] = B * Tq * (512 * 2 + 516)
+    return out
+
+
+def step_bytes(wl) -> int:
+    ob = op_bytes(wl)
+    total = 0
+    for g, grp in enumerate(wl.groups):
+        total += ob[f"append_g{g}"]
+        for m in grp.schedule:
+            total += ob["attn"] + ob["swa_append"]
+            if m == "F":
+                total += ob[f"index_full_g{g}"]
+            elif m == "X":
+                total += ob[f"index_reindex_g{g}"]
+    return total
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ------------------------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self._stop = threading.Event()
+        try:
+            import pynvml as N
+            import torch
+            N.nvmlInit()
+            p = torch.cuda.get_device_properties(device_index)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            try:
+                self.h = N.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = N.nvmlDeviceGetHandleByIndex(device_index)
+            self.N = N
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report nothing rather than guess
+            self.err = str(e)
+
+    def _run(self):
+        N = self.N
+        while not self._stop.is_set():
+            try:
+                self.samples.append(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
+                r = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self) -> dict:
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------
+# CPU oracle sample (cpu_baseline leg and the reference arm)
+# ------------------------------------------------------------------------------------------
+def oracle_sample_time(wl, requests: list[int], steps: int = 1) -> tuple[float, dict]:
+    """Time the oracle on one decode step of `requests` (caches prepared untimed).
+    Returns seconds per step for those requests and a description."""
+    import torch
+    import oracle as orc
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import oracle_ref as R
+
+    prepared = []
+    for b in requests:
+        caches = R.request_caches(wl, b, main_rows={g: np.zeros(0, np.int64)
+                                                    for g in range(len(wl.groups))})
+        for g, c in enumerate(caches):   # main KV of the whole request (state before the step)
+            N = c["N"]
+            mc, ms = orc.quantize_fp4(wl.main_kv(g, b, 0, N))
+            c["codes"], c["scales"] = mc, ms
+        rings = [R.swa_ring(wl, l, b) for l in range(len(wl.layers))]
+        inputs = dict(q=[wl.q(l, b) for l in range(len(wl.layers))],
+                      qi=[wl.q_idx(l, b) for l in range(len(wl.layers))],
+                      w=[wl.w(l, b).numpy() for l in range(len(wl.layers))],
+                      kv=[wl.main_kv(g, b, wl.entries(g) - 1, 1) for g in range(len(wl.groups))],
+                      ik=[wl.idx_k(g, b, wl.entries(g) - 1, 1) for g in range(len(wl.groups))],
+                      swa=[wl.swa(l, b, wl.ctx - 1, 1) for l in range(len(wl.layers))])
+        prepared.append((b, caches, rings, inputs))
+    q_pos = np.asarray(wl.q_positions(), np.int32)[None]
+    plan = R.reuse_sources(wl)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        for b, caches, rings, inp in prepared:
+            for g in range(len(wl.groups)):           # a1/a2: the new entry
+                orc.quantize_fp4(inp["kv"][g])
+                orc.quantize_fp8(inp["ik"][g])
+            topk, pool = {}, {}
+            for layer, (g, m, src) in enumerate(plan):
+                c, grp = caches[g], wl.groups[g]
+                orc.quantize_fp8(inp["swa"][layer])    # a2: this layer's SWA row
+                if m == "F":
+                    p, t, _ = orc.index_full(c["idx_codes"][None], c["idx_scale"][None], grp.ratio,
+                                             inp["qi"][layer][None], inp["w"][layer][None], q_pos,
+                                             grp.pool_blocks, wl.top_k)
+                    topk[layer], pool[g] = t, p
+                elif m == "X":
+                    t, _ = orc.index_reindex(c["idx_codes"][None], c["idx_scale"][None],
+                                             grp.ratio, inp["qi"][layer][None],
+                                             inp["w"][layer][None], q_pos, pool[g], wl.top_k)
+                    topk[layer] = t
+                rc, rs = rings[layer]
+                orc.attention(c["codes"][None], c["scales"][None], rc[None], rs[None],
+                              inp["q"][layer][None], q_pos, topk[src], wl.swa_len, R.SOFTMAX_SCALE)
+    dt = (time.perf_counter() - t0) / steps
+    return dt, {"requests": len(requests), "of_batch": wl.B, "steps": steps}
+
+
+def cpu_baseline(wl, requests: list[int]) -> dict:
+    import oracle as orc
+    dt, desc = oracle_sample_time(wl, requests, 1)
+    layers = len(wl.layers)
+    value = layers * len(requests) / wl.B / dt
+    return {"value": value, "unit": UNIT, "cores": orc.num_threads(), "kind": "oracle",
+            "sample": f"{len(requests)} of {wl.B} requests, 1 decode step of all {layers} layers "
+                      f"(append, index, attention) on the host; value scaled by "
+                      f"{len(requests)}/{wl.B} of a layer-step; {dt:.2f} s per sample step"}
+
+
+# ------------------------------------------------------------------------------------------
+def pack_inputs(inputs: dict, device):
+    """Copy every step input into one device buffer (views replace the tensors) and
+    return (views dict, device buffer, pinned host mirror, bytes)."""
+    import torch
+    flat = []
+
+    def visit(v):
+        if torch.is_tensor(v):
+            flat.append(v)
+        elif isinstance(v, (list, tuple)):
+            for x in v:
+                visit(x)
+    for v in inputs.values():
+        visit(v)
+    offs, off = [], 0
+    for t in flat:
+        off = (off + 255) // 256 * 256
+        offs.append(off)
+        off += t.numel() * t.element_size()
+    dbuf = torch.empty(off, dtype=torch.uint8, device=device)
+    views = {}
+    for t, o in zip(flat, offs):
+        n = t.numel() * t.element_size()
+        v = dbuf[o:o + n].view(t.dtype).view(t.shape)
+        v.copy_(t)
+        views[id(t)] = v
+
+    def rebuild(v):
+        if torch.is_tensor(v):
+            return views[id(v)]
+        if isinstance(v, list):
+            return [rebuild(x) for x in v]
+        return v
+    packed = {k: rebuild(v) for k, v in inputs.items()}
+    hbuf = torch.empty(off, dtype=torch.uint8, pin_memory=True)
+    hbuf.copy_(dbuf)
+    return packed, dbuf, hbuf, off
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from synth.workloads import WORKLOADS
+    import csa2_harness
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    dw = csa2_harness.DeviceWorkload(wl, device=dev)
+    st = dw.stack
+    inputs, dbuf, hbuf, in_bytes = pack_inputs(dw.inputs, dev)
+    full_layers = [lp.layer for lp in st.plan if lp.mode == "F"]
+    stream = torch.cuda.Stream(device=dev)
+
+    # one eager step (sets kernel attributes, checks the path), then the graph
+    with torch.cuda.stream(stream):
+        st.step(**inputs)
+    torch.cuda.synchronize(dev)
+    if st.dev_err.item() != 0:
+        raise RuntimeError(f"device error bits {st.dev_err.item()} in the warm-up step")
+
+    S = max(1, min(10, args.steps))
+    ev = [(torch.cuda.Event(enable_timing=True, external=True),
+           torch.cuda.Event(enable_timing=True, external=True)) for _ in range(S)]
+    orig_full = None
+    import fp4_kv_compressed_b200 as pkg
+
+    # wrap csa2_index_full of the Full layer with timing events (graph capture only)
+    state = {"i": 0}
+
+    def timed_full(*a, **k):
+        i = state["i"]
+        ev[i % S][0].record()
+        orig_full(*a, **k)
+        ev[i % S][1].record()
+        state["i"] = i + 1
+    import fp4_kv_compressed_b200.stack as stack_mod
+    orig_full = stack_mod.bind.csa2_index_full
+    g = torch.cuda.CUDAGraph()
+    stack_mod.bind.csa2_index_full = timed_full
+    try:
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(S):
+                st.step(**inputs)
+    finally:
+        stack_mod.bind.csa2_index_full = orig_full
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1, stream=stream):
+        st.step(**inputs)
+
+    reps = max(1, args.steps // S)
+    K = reps * S
+    for _ in range(max(args.warmup, 3)):
+        g1.replay()
+    torch.cuda.synchronize(dev)
+
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with clocks:
+        with torch.cuda.stream(stream):
+            start.record()
+            for _ in range(reps):
+                g.replay()
+            end.record()
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    full_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    if st.dev_err.item() != 0:
+        raise RuntimeError(f"device error bits {st.dev_err.item()} in the timed steps")
+
+    # ---- e2e: inputs from pinned host memory, last layer's output back to the host ----
+    last = len(st.plan) - 1
+    out_h = torch.empty_like(st.out[last], device="cpu").pin_memory()
+    lse_h = torch.empty_like(st.lse[last], device="cpu").pin_memory()
+    out_bytes = out_h.numel() * 4 + lse_h.numel() * 4
+    Ke = max(3, min(K, args.e2e_steps))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        with torch.cuda.stream(stream):
+            dbuf.copy_(hbuf, non_blocking=True)
+            g1.replay()
+            out_h.copy_(st.out[last], non_blocking=True)
+            lse_h.copy_(st.lse[last], non_blocking=True)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        e0.record()
+        for _ in range(Ke):
+            dbuf.copy_(hbuf, non_blocking=True)
+            g1.replay()
+            out_h.copy_(st.out[last], non_blocking=True)
+            lse_h.copy_(st.lse[last], non_blocking=True)
+        e1.record()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item()) / Ke
+
+    layers = len(st.plan)
+    ms_step = ms_max / K
+    value = world * layers / (ms_step / 1e3)
+    sb = step_bytes(wl)
+    ob = op_bytes(wl)
+    g_full = st.plan[full_layers[0]].group
+    full_bytes = ob[f"index_full_g{g_full}"]
+    peak, peak_src = HBM_FALLBACK_GBS, "fallback 6.65 TB/s"
+    try:
+        mp = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        peak, peak_src = float(mp["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        pass
+    achieved = full_bytes / (full_ms / 1e3) / 1e9
+    traffic = None
+    if args.traffic_bytes:
+        traffic = args.traffic_bytes
+    launches = st.launches_per_step() * K
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp32 index / bf16+fp16 MMA attention",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.ctx, "heads": wl.H,
+                   "index_heads": wl.H_I, "d_idx": wl.d_I, "top_k": wl.top_k,
+                   "pool": [g.pool_blocks for g in wl.groups],
+                   "schedule": [g.schedule for g in wl.groups], "swa": wl.swa_len,
+                   "parallelism": f"replicas x{world} (requests sharded, no collective)",
+                   "l2": "inputs larger than L2: the Full scan streams "
+                         f"{ob[f'index_full_g{g_full}'] / 1e9:.2f} GB per step",
+                   "cuda_graph": True, "step_algorithmic_bytes": sb,
+                   "step_gbps": sb / (ms_step / 1e3) / 1e9,
+                   "step_frac_of_8tbs": sb / (ms_step / 1e3) / 8e12,
+                   "token_layer_steps_per_s": value * wl.B},
+        "roofline": {"bound": "hbm", "kernel": "csa2_index_full (Full scan + pool/Top-K select)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_src,
+                     "traffic": traffic, "algorithmic_bytes_per_launch": full_bytes,
+                     "launch_ms": full_ms},
+        "e2e": {"value": world * layers / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    return line, wl
+
+
+def run_reference(args, rank, world):
+    from synth.workloads import WORKLOADS
+    import oracle as orc
+    wl = WORKLOADS[args.workload]
+    if rank != 0:
+        return None
+    K = max(1, args.steps if args.steps <= 5 else 2)
+    req = [0]
+    oracle_sample_time(wl, req, 1)            # warm-up (OpenMP pools, page-in)
+    dt, desc = oracle_sample_time(wl, req, K)
+    layers = len(wl.layers)
+    value = layers * len(req) / wl.B / dt
+    sample = (f"{len(req)} of {wl.B} requests per step, {K} timed steps of all {layers} layers "
+              f"on the host; value scaled by {len(req)}/{wl.B} of a layer-step")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": 1, "ms_per_step": dt * 1e3 * wl.B / len(req),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp32 index / fp64 attention", "data": "synthetic",
+            "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.ctx},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": orc.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode_128k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="ncu dram bytes per launch of the timed kernel, if captured")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line, wl = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(wl, [0, wl.B - 1])
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

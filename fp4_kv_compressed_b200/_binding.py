@@ -1,0 +1,158 @@
+"""ctypes binding of libcsa2.so: argument marshalling only.
+
+Every function here converts torch tensors to raw pointers and calls the C entry
+point of the same name; all computation runs in the library's CUDA kernels.
+There is no fallback: if the library is missing or fails to load, the import
+raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa2.so")
+
+CSA2_OP_INDEX_FULL = 1
+CSA2_OP_INDEX_REINDEX = 2
+CSA2_OP_SPARSE_ATTN = 3
+
+STATUS = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_CAPACITY",
+          3: "CSA2_ERR_WORKSPACE", 4: "CSA2_ERR_UNSUPPORTED", 5: "CSA2_ERR_CUDA",
+          6: "CSA2_ERR_DEVICE_BOUNDS"}
+
+DEVERR_SLOT, DEVERR_INDEX, DEVERR_NMAX, DEVERR_RANGE = 0x1, 0x2, 0x4, 0x8
+
+# every symbol declared in include/csa2.h
+EXPORTS = ("csa2_quantize_append", "csa2_workspace_size", "csa2_index_full",
+           "csa2_index_reindex", "csa2_sparse_attn_decode", "csa2_read_device_error",
+           "csa2_status_string", "csa2_abi_version")
+
+
+class Csa2Error(RuntimeError):
+    def __init__(self, fn: str, status: int, lib):
+        self.status = status
+        msg = lib.csa2_status_string(status).decode()
+        super().__init__(f"{fn} -> {STATUS.get(status, status)} ({msg})")
+
+
+class CSA2GlobalKV(C.Structure):
+    _fields_ = [("codes", C.c_void_p), ("scales", C.c_void_p), ("idx_codes", C.c_void_p),
+                ("idx_scale", C.c_void_p), ("batch", C.c_int32), ("cap", C.c_int32),
+                ("d_idx", C.c_int32), ("ratio", C.c_int32)]
+
+
+class CSA2SWA(C.Structure):
+    _fields_ = [("codes", C.c_void_p), ("scale", C.c_void_p), ("batch", C.c_int32),
+                ("window_cap", C.c_int32)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libcsa2.so (building it first only if the sources are newer)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        from .build import build
+        build()
+    L = C.CDLL(path)
+    P, i32, sz = C.c_void_p, C.c_int32, C.c_size_t
+    L.csa2_quantize_append.argtypes = [P, P, P, i32, P, P, P, i32, P, P, P]
+    L.csa2_workspace_size.argtypes = [i32] * 7
+    L.csa2_workspace_size.restype = sz
+    L.csa2_index_full.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, P, P, P, P, sz, P, P]
+    L.csa2_index_reindex.argtypes = [P, P, P, P, i32, i32, P, i32, i32, P, P, P, sz, P, P]
+    L.csa2_sparse_attn_decode.argtypes = [P, P, P, P, i32, i32, P, i32, i32, C.c_float, P, P, P,
+                                          sz, P, P]
+    L.csa2_read_device_error.argtypes = [P, P, P]
+    L.csa2_status_string.argtypes = [C.c_int]
+    L.csa2_status_string.restype = C.c_char_p
+    L.csa2_abi_version.restype = i32
+    for fn in ("csa2_quantize_append", "csa2_index_full", "csa2_index_reindex",
+               "csa2_sparse_attn_decode", "csa2_read_device_error"):
+        getattr(L, fn).restype = C.c_int
+    _lib = L
+    return L
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    assert t.is_contiguous(), "tensors passed to libcsa2 must be contiguous"
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> C.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise Csa2Error(fn, status, load_library())
+
+
+def csa2_workspace_size(op: int, B: int, Tq: int, n_max: int, H: int, top_k: int,
+                        pool_blocks: int) -> int:
+    return load_library().csa2_workspace_size(op, B, Tq, n_max, H, top_k, pool_blocks)
+
+
+def csa2_quantize_append(kv: CSA2GlobalKV | None, kv_bf16, idxk_bf16, T_kv: int, kv_start,
+                         swa: CSA2SWA | None, swa_bf16, T_swa: int, swa_start, dev_err=None,
+                         stream=None):
+    L = load_library()
+    st = L.csa2_quantize_append(C.byref(kv) if kv is not None else None, _ptr(kv_bf16),
+                                _ptr(idxk_bf16), T_kv, _ptr(kv_start),
+                                C.byref(swa) if swa is not None else None, _ptr(swa_bf16),
+                                T_swa, _ptr(swa_start), _ptr(dev_err), _stream(stream))
+    _check("csa2_quantize_append", st)
+
+
+def csa2_index_full(kv: CSA2GlobalKV, q_idx, w, q_pos, Tq: int, H_I: int, n_max: int,
+                    pool_blocks: int, top_k: int, pool_out, topk_out, topk_count, workspace,
+                    dev_err=None, stream=None):
+    L = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = L.csa2_index_full(C.byref(kv), _ptr(q_idx), _ptr(w), _ptr(q_pos), Tq, H_I, n_max,
+                           pool_blocks, top_k, _ptr(pool_out), _ptr(topk_out), _ptr(topk_count),
+                           _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream))
+    _check("csa2_index_full", st)
+
+
+def csa2_index_reindex(kv: CSA2GlobalKV, q_idx, w, q_pos, Tq: int, H_I: int, pool,
+                       pool_blocks: int, top_k: int, topk_out, topk_count, workspace,
+                       dev_err=None, stream=None):
+    L = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = L.csa2_index_reindex(C.byref(kv), _ptr(q_idx), _ptr(w), _ptr(q_pos), Tq, H_I,
+                              _ptr(pool), pool_blocks, top_k, _ptr(topk_out), _ptr(topk_count),
+                              _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream))
+    _check("csa2_index_reindex", st)
+
+
+def csa2_sparse_attn_decode(kv: CSA2GlobalKV, swa: CSA2SWA | None, q, q_pos, Tq: int, H: int,
+                            topk, top_k: int, swa_len: int, softmax_scale: float, out, lse,
+                            workspace=None, dev_err=None, stream=None):
+    L = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = L.csa2_sparse_attn_decode(C.byref(kv), C.byref(swa) if swa is not None else None,
+                                   _ptr(q), _ptr(q_pos), Tq, H, _ptr(topk), top_k, swa_len,
+                                   softmax_scale, _ptr(out), _ptr(lse), _ptr(workspace),
+                                   ws_bytes, _ptr(dev_err), _stream(stream))
+    _check("csa2_sparse_attn_decode", st)
+
+
+def csa2_read_device_error(dev_err, stream=None) -> int:
+    """Synchronises the stream; returns the device error bits (0 = none) and resets them."""
+    L = load_library()
+    bits = C.c_int32(0)
+    st = L.csa2_read_device_error(_ptr(dev_err), C.byref(bits), _stream(stream))
+    if st not in (0, 6):
+        _check("csa2_read_device_error", st)
+    return bits.value

@@ -1,0 +1,307 @@
+// csa2_api.cu -- the extern "C" entry points of libcsa2: host-side validation,
+// workspace layout and kernel launches.  No allocation, no state, no exceptions.
+#include <stdint.h>
+#include <string.h>
+
+#include "csa2.h"
+#include "csa2_internal.h"
+
+using namespace csa2;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// Workspace layout of csa2_index_full: scores [BT][score_stride] fp32, then
+// (hierarchical only) block maxima [BT][bmax_stride] fp32.
+struct FullLayout {
+    int64_t score_stride, bmax_stride;
+    size_t bmax_off, total;
+};
+
+FullLayout full_layout(int64_t BT, int64_t n_max, int32_t pool_blocks) {
+    FullLayout L;
+    L.score_stride = (int64_t)align_up((size_t)(n_max > 0 ? n_max : 1), 64);
+    L.bmax_stride = (int64_t)align_up((size_t)((n_max + 7) / 8 > 0 ? (n_max + 7) / 8 : 1), 64);
+    L.bmax_off = align_up((size_t)BT * L.score_stride * sizeof(float), kAlign);
+    L.total = L.bmax_off;
+    if (pool_blocks > 0) L.total += align_up((size_t)BT * L.bmax_stride * sizeof(float), kAlign);
+    return L;
+}
+
+size_t reindex_ws(int64_t BT, int32_t pool_blocks) {
+    return align_up((size_t)BT * pool_blocks * 8 * sizeof(float), kAlign);
+}
+
+csa2_status check_kv(const csa2_global_kv *kv, bool need_index) {
+    if (!kv || !kv->codes || !kv->scales) return CSA2_ERR_INVALID_ARG;
+    if (kv->batch <= 0 || kv->cap <= 0 || kv->ratio < 1 || kv->ratio > 64) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(kv->codes, 16) || !aligned(kv->scales, 16)) return CSA2_ERR_INVALID_ARG;
+    if (need_index) {
+        if (!kv->idx_codes || !kv->idx_scale) return CSA2_ERR_INVALID_ARG;
+        if (kv->d_idx != 64 && kv->d_idx != 128) return CSA2_ERR_UNSUPPORTED;
+        if (!aligned(kv->idx_codes, 16) || !aligned(kv->idx_scale, 4)) return CSA2_ERR_INVALID_ARG;
+    }
+    return CSA2_OK;
+}
+
+csa2_status launched(cudaError_t e) {
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return CSA2_ERR_CUDA;
+    }
+    return CSA2_OK;
+}
+
+bool hi_supported(int32_t H_I) {
+    return H_I == 1 || H_I == 2 || H_I == 4 || H_I == 8 || H_I == 16;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t csa2_abi_version(void) { return 100; }
+
+const char *csa2_status_string(csa2_status st) {
+    switch (st) {
+        case CSA2_OK: return "ok";
+        case CSA2_ERR_INVALID_ARG: return "invalid argument";
+        case CSA2_ERR_CAPACITY: return "cache or window capacity too small";
+        case CSA2_ERR_WORKSPACE: return "workspace missing or too small";
+        case CSA2_ERR_UNSUPPORTED: return "shape not supported by the kernels";
+        case CSA2_ERR_CUDA: return "CUDA launch or runtime error";
+        case CSA2_ERR_DEVICE_BOUNDS: return "device-side bounds check failed";
+    }
+    return "unknown status";
+}
+
+size_t csa2_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t n_max, int32_t H,
+                           int32_t top_k, int32_t pool_blocks) {
+    (void)H;
+    (void)top_k;
+    if (B <= 0 || Tq <= 0) return 0;
+    const int64_t BT = (int64_t)B * Tq;
+    switch (op) {
+        case CSA2_OP_INDEX_FULL:
+            return n_max > 0 ? full_layout(BT, n_max, pool_blocks).total : 0;
+        case CSA2_OP_INDEX_REINDEX:
+            return pool_blocks > 0 ? reindex_ws(BT, pool_blocks) : 0;
+        case CSA2_OP_SPARSE_ATTN:
+            return 0;
+        default:
+            return 0;
+    }
+}
+
+csa2_status csa2_quantize_append(const csa2_global_kv *kv, const void *kv_bf16,
+                                 const void *idxk_bf16, int32_t T_kv, const int32_t *kv_start,
+                                 const csa2_swa *swa, const void *swa_bf16, int32_t T_swa,
+                                 const int32_t *swa_start, int32_t *dev_err,
+                                 csa2_stream_t stream) {
+    QuantArgs a;
+    memset(&a, 0, sizeof(a));
+    a.dev_err = dev_err;
+    if (T_kv < 0 || T_swa < 0) return CSA2_ERR_INVALID_ARG;
+    int32_t B = -1;
+    if (T_kv > 0 && (kv_bf16 || idxk_bf16)) {
+        csa2_status st = check_kv(kv, idxk_bf16 != nullptr);
+        if (st != CSA2_OK) return st;
+        if (!kv_start) return CSA2_ERR_INVALID_ARG;
+        if (kv_bf16 && !aligned(kv_bf16, 16)) return CSA2_ERR_INVALID_ARG;
+        if (idxk_bf16 && !aligned(idxk_bf16, 8)) return CSA2_ERR_INVALID_ARG;
+        if (T_kv > kv->cap) return CSA2_ERR_CAPACITY;
+        B = kv->batch;
+        a.codes = kv->codes;
+        a.scales = kv->scales;
+        a.idx_codes = kv->idx_codes;
+        a.idx_scale = kv->idx_scale;
+        a.cap = kv->cap;
+        a.d_idx = kv->d_idx;
+        a.kv_bf16 = (const uint16_t *)kv_bf16;
+        a.idxk_bf16 = (const uint16_t *)idxk_bf16;
+        a.T_kv = T_kv;
+        a.kv_start = kv_start;
+        a.n_main = kv_bf16 ? (int64_t)B * T_kv : 0;
+        a.n_idx = idxk_bf16 ? (int64_t)B * T_kv : 0;
+    }
+    if (T_swa > 0 && swa_bf16) {
+        if (!swa || !swa->codes || !swa->scale || !swa_start) return CSA2_ERR_INVALID_ARG;
+        if (swa->batch <= 0 || swa->window_cap <= 0) return CSA2_ERR_INVALID_ARG;
+        if (B >= 0 && swa->batch != B) return CSA2_ERR_INVALID_ARG;
+        if (!aligned(swa->codes, 16) || !aligned(swa->scale, 4) || !aligned(swa_bf16, 16))
+            return CSA2_ERR_INVALID_ARG;
+        if (T_swa > swa->window_cap) return CSA2_ERR_CAPACITY;
+        a.swa_codes = swa->codes;
+        a.swa_scale = swa->scale;
+        a.wcap = swa->window_cap;
+        a.swa_bf16 = (const uint16_t *)swa_bf16;
+        a.T_swa = T_swa;
+        a.swa_start = swa_start;
+        a.n_swa = (int64_t)swa->batch * T_swa;
+    }
+    return launched(launch_quantize_append(a, (cudaStream_t)stream));
+}
+
+csa2_status csa2_index_full(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
+                            const int32_t *q_pos, int32_t Tq, int32_t H_I, int32_t n_max,
+                            int32_t pool_blocks, int32_t top_k, int32_t *pool_out,
+                            int32_t *topk_out, int32_t *topk_count, void *workspace,
+                            size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
+    csa2_status st = check_kv(kv, true);
+    if (st != CSA2_OK) return st;
+    if (!q_idx_bf16 || !w || !q_pos || !topk_out || !topk_count) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(q_idx_bf16, 4) || !aligned(w, 4)) return CSA2_ERR_INVALID_ARG;
+    if (Tq <= 0 || n_max < 0) return CSA2_ERR_INVALID_ARG;
+    if (!hi_supported(H_I)) return CSA2_ERR_UNSUPPORTED;
+    if (top_k < 1 || top_k > CSA2_TOPK_MAX) return CSA2_ERR_UNSUPPORTED;
+    if (pool_blocks != 0 && (pool_blocks < top_k || pool_blocks > CSA2_POOL_MAX))
+        return CSA2_ERR_UNSUPPORTED;
+    const int64_t BT = (int64_t)kv->batch * Tq;
+    if (BT > 65535) return CSA2_ERR_UNSUPPORTED;   // grid.y limit
+    const FullLayout L = full_layout(BT, n_max, pool_blocks);
+    if (n_max > 0 && (!workspace || ws_bytes < L.total || !aligned(workspace, kAlign)))
+        return CSA2_ERR_WORKSPACE;
+
+    IndexArgs a;
+    memset(&a, 0, sizeof(a));
+    a.idx_codes = kv->idx_codes;
+    a.idx_scale = kv->idx_scale;
+    a.cap = kv->cap;
+    a.d_idx = kv->d_idx;
+    a.ratio = kv->ratio;
+    a.q_idx = (const uint16_t *)q_idx_bf16;
+    a.w = w;
+    a.q_pos = q_pos;
+    a.Tq = Tq;
+    a.H_I = H_I;
+    a.n_max = n_max;
+    a.scores = (float *)workspace;
+    a.score_stride = L.score_stride;
+    a.bmax = pool_blocks > 0 && workspace ? (float *)((uint8_t *)workspace + L.bmax_off) : nullptr;
+    a.bmax_stride = L.bmax_stride;
+    a.pool_blocks = pool_blocks;
+    a.pool_out = pool_out;
+    a.top_k = top_k;
+    a.topk_out = topk_out;
+    a.topk_count = topk_count;
+    a.dev_err = dev_err;
+    cudaStream_t s = (cudaStream_t)stream;
+    st = launched(launch_index_scan(a, (int)BT, s));
+    if (st != CSA2_OK) return st;
+    return launched(launch_select_full(a, (int)BT, s));
+}
+
+csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
+                               const int32_t *q_pos, int32_t Tq, int32_t H_I,
+                               const int32_t *pool, int32_t pool_blocks, int32_t top_k,
+                               int32_t *topk_out, int32_t *topk_count, void *workspace,
+                               size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
+    csa2_status st = check_kv(kv, true);
+    if (st != CSA2_OK) return st;
+    if (!q_idx_bf16 || !w || !q_pos || !pool || !topk_out || !topk_count) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(q_idx_bf16, 4) || !aligned(w, 4)) return CSA2_ERR_INVALID_ARG;
+    if (Tq <= 0) return CSA2_ERR_INVALID_ARG;
+    if (!hi_supported(H_I)) return CSA2_ERR_UNSUPPORTED;
+    if (top_k < 1 || top_k > CSA2_TOPK_MAX) return CSA2_ERR_UNSUPPORTED;
+    if (pool_blocks < 1 || pool_blocks > CSA2_POOL_MAX) return CSA2_ERR_UNSUPPORTED;
+    const int64_t BT = (int64_t)kv->batch * Tq;
+    if (BT > 65535) return CSA2_ERR_UNSUPPORTED;   // grid.y limit
+    if (!workspace || ws_bytes < reindex_ws(BT, pool_blocks) || !aligned(workspace, kAlign))
+        return CSA2_ERR_WORKSPACE;
+
+    IndexArgs a;
+    memset(&a, 0, sizeof(a));
+    a.idx_codes = kv->idx_codes;
+    a.idx_scale = kv->idx_scale;
+    a.cap = kv->cap;
+    a.d_idx = kv->d_idx;
+    a.ratio = kv->ratio;
+    a.q_idx = (const uint16_t *)q_idx_bf16;
+    a.w = w;
+    a.q_pos = q_pos;
+    a.Tq = Tq;
+    a.H_I = H_I;
+    a.scores = (float *)workspace;
+    a.score_stride = (int64_t)pool_blocks * 8;
+    a.pool = pool;
+    a.pool_blocks = pool_blocks;
+    a.top_k = top_k;
+    a.topk_out = topk_out;
+    a.topk_count = topk_count;
+    a.dev_err = dev_err;
+    cudaStream_t s = (cudaStream_t)stream;
+    st = launched(launch_reindex_score(a, (int)BT, s));
+    if (st != CSA2_OK) return st;
+    return launched(launch_select_reindex(a, (int)BT, s));
+}
+
+csa2_status csa2_sparse_attn_decode(const csa2_global_kv *kv, const csa2_swa *swa,
+                                    const void *q_bf16, const int32_t *q_pos, int32_t Tq,
+                                    int32_t H, const int32_t *topk, int32_t top_k,
+                                    int32_t swa_len, float softmax_scale, float *out,
+                                    float *lse, void *workspace, size_t ws_bytes,
+                                    int32_t *dev_err, csa2_stream_t stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    csa2_status st = check_kv(kv, false);
+    if (st != CSA2_OK) return st;
+    if (!q_bf16 || !q_pos || !out || !lse) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(q_bf16, 4) || !aligned(out, 8)) return CSA2_ERR_INVALID_ARG;
+    if (Tq <= 0 || H < 16 || H % 16 != 0) return CSA2_ERR_UNSUPPORTED;
+    if (top_k < 0 || top_k > CSA2_TOPK_MAX) return CSA2_ERR_UNSUPPORTED;
+    if (top_k > 0 && !topk) return CSA2_ERR_INVALID_ARG;
+    if (swa_len < 0) return CSA2_ERR_INVALID_ARG;
+    if (swa_len > 0) {
+        if (!swa || !swa->codes || !swa->scale || swa->window_cap <= 0) return CSA2_ERR_INVALID_ARG;
+        if (swa->batch != kv->batch) return CSA2_ERR_INVALID_ARG;
+        if (!aligned(swa->codes, 16) || !aligned(swa->scale, 4)) return CSA2_ERR_INVALID_ARG;
+        if ((int64_t)swa_len + Tq - 1 > swa->window_cap) return CSA2_ERR_CAPACITY;
+    }
+    const int64_t BT = (int64_t)kv->batch * Tq;
+    if (BT > 65535) return CSA2_ERR_UNSUPPORTED;   // grid.y limit of the attention kernel
+
+    AttnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.codes = kv->codes;
+    a.scales = kv->scales;
+    a.cap = kv->cap;
+    a.ratio = kv->ratio;
+    if (swa_len > 0) {
+        a.swa_codes = swa->codes;
+        a.swa_scale = swa->scale;
+        a.wcap = swa->window_cap;
+    } else {
+        a.wcap = 1;
+    }
+    a.q = (const uint16_t *)q_bf16;
+    a.q_pos = q_pos;
+    a.Tq = Tq;
+    a.H = H;
+    a.topk = topk;
+    a.top_k = top_k;
+    a.swa_len = swa_len;
+    a.softmax_scale = softmax_scale;
+    a.out = out;
+    a.lse = lse;
+    a.dev_err = dev_err;
+    return launched(launch_sparse_attn(a, (int)BT, (cudaStream_t)stream));
+}
+
+csa2_status csa2_read_device_error(int32_t *dev_err, int32_t *bits_out, csa2_stream_t stream) {
+    if (!dev_err) return CSA2_ERR_INVALID_ARG;
+    int32_t bits = 0;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(&bits, dev_err, sizeof(bits), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return launched(cudaErrorUnknown);
+    if (cudaMemsetAsync(dev_err, 0, sizeof(int32_t), s) != cudaSuccess) return launched(cudaErrorUnknown);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return launched(cudaErrorUnknown);
+    if (bits_out) *bits_out = bits;
+    return bits ? CSA2_ERR_DEVICE_BOUNDS : CSA2_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,110 @@
+// csa2_common.cuh -- shared device helpers of libcsa2 (number formats, order keys).
+//
+// Formats (DeepSeek V4.1 Flash study notes, section 4; myzaker "cache precision
+// and tiering"): the main KV is E2M1 with one E4M3 scale per 16 channels; the
+// SWA window and the indexer K are E4M3 with one fp32 scale per token.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "csa2.h"
+
+namespace csa2 {
+
+constexpr int kDim = CSA2_KV_DIM;          // 512-channel K=V entry
+constexpr int kCodeBytes = kDim / 2;       // 256 B of E2M1 codes per entry
+constexpr int kScaleBytes = kDim / 16;     // 32 E4M3 scales per entry
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) {
+    return __uint_as_float(h << 16);
+}
+
+// Eight fp32 values -> four bytes of E2M1 codes, round-to-nearest-even with
+// saturation; value 2j goes to the low nibble of byte j.  (cvt puts its first
+// source in the upper half.)
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float *v) {
+    uint32_t out;
+    asm("{\n.reg .b8 b0, b1, b2, b3;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n"
+        "mov.b32 %0, {b0, b1, b2, b3};\n}"
+        : "=r"(out)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+          "f"(v[7]));
+    return out;
+}
+
+// Two fp32 values -> two E4M3 bytes (lo in the low byte), RNE, saturating.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(out) : "f"(lo), "f"(hi));
+    return out;
+}
+
+// Exact E4M3 -> fp32.  The code's 7 magnitude bits placed at fp32 bit 20 give
+// the value times 2^-120 (the E4M3 subnormals land on fp32 subnormals), so one
+// exact multiply by 2^120 finishes it.  Needs denormals preserved (no FTZ).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+    uint32_t bits = ((b & 0x7Fu) << 20) | ((b & 0x80u) << 24);
+    return __uint_as_float(bits) * 0x1p120f;
+}
+
+// Two E4M3 bytes (low 16 bits of w) -> f16x2, exact (low byte -> low half).
+__device__ __forceinline__ uint32_t cvt_e4m3x2_f16x2(uint32_t w) {
+    uint32_t out;
+    uint16_t in = (uint16_t)w;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(out) : "h"(in));
+    return out;
+}
+
+// Four bytes of E2M1 codes -> four f16x2 words (exact), byte j -> word j.
+__device__ __forceinline__ void cvt_e2m1x8_f16x2(uint32_t w, uint32_t *out) {
+    asm("{\n.reg .b8 b0, b1, b2, b3;\n"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+        : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3])
+        : "r"(w));
+}
+
+// d = a * b + c on two fp32 lanes, each lane an IEEE fma (round to nearest even).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(reinterpret_cast<unsigned long long &>(d))
+        : "l"(reinterpret_cast<unsigned long long &>(a)),
+          "l"(reinterpret_cast<unsigned long long &>(b)),
+          "l"(reinterpret_cast<unsigned long long &>(c)));
+    return d;
+}
+
+// Order key of a score: larger score -> larger key; -0 == +0; NaN -> 1 (below
+// every number); 0 is reserved for "not a candidate".
+__device__ __forceinline__ uint32_t score_key(float f) {
+    if (f != f) return 1u;
+    uint32_t u = __float_as_uint(f == 0.0f ? 0.0f : f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_to_score(uint32_t k) {
+    uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+    return __uint_as_float(u);
+}
+
+__device__ __forceinline__ void set_dev_err(int32_t *dev_err, int bit) {
+    if (dev_err) atomicOr(dev_err, bit);
+}
+
+__device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+__device__ __forceinline__ int64_t visible_entries(int32_t t, int32_t ratio) {
+    return t < 0 ? 0 : ((int64_t)t + 1) / ratio;
+}
+
+}  // namespace csa2

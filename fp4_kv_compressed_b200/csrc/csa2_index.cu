@@ -1,0 +1,537 @@
+// csa2_index.cu -- Full-layer index scan, pool / Top-K selection, Reindex (sm_100a).
+//
+// DeepSeek V4.1 Flash study notes, section 2 (report Figure 5) and myzaker
+// "CSA2 attention": the first Full layer scans all causally visible positions,
+// scores them block by block and builds a shared candidate pool of at most
+// 2048 blocks x 8 positions; it picks at most 512 positions; later Reindex
+// layers re-score with their own index query only inside the pool.
+//
+// Score (fixed for this build): score(s) = sum_h w_h * relu(q_h . k_s), k_s the
+// FP8 indexer K of entry s times its per-entry scale, evaluated in this fp32
+// order so that Top-K membership is reproducible bit for bit:
+//   per head: (even, odd) = fma chains over channel pairs (2j, 2j+1), one
+//             packed fma.rn.f32x2 per pair; a_h = even + odd
+//   t = fma chain over h of (w_h, max(a_h, 0));  score = t * sigma_s
+// Selection order: score descending, ties to the lower position.
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "csa2_common.cuh"
+#include "csa2_internal.h"
+
+namespace csa2 {
+
+// ------------------------------------------------------------------------------
+// Scoring core: one CTA scores a tile of kTileRows rows staged in shared memory.
+// ------------------------------------------------------------------------------
+constexpr int kScoreThreads = 128;
+constexpr int kRowsPerThread = 4;
+constexpr int kTileRows = kScoreThreads * kRowsPerThread;   // 512 positions per CTA
+
+// 16-byte unit u of row r lives at unit swz(r, u): a quarter-warp reading unit
+// u of 8 consecutive rows hits 8 different 16-byte bank groups.
+template <int D>
+__device__ __forceinline__ int swz(int r, int u) {
+    if constexpr (D == 128)
+        return u ^ (r & 7);
+    else
+        return u ^ ((r >> 1) & 3);
+}
+
+template <int D, int HI>
+struct ScoreSmem {
+    uint8_t rows[kTileRows * D];
+    float2 q[D / 2][HI];     // q pairs (q[h][2j], q[h][2j+1]) as fp32
+    float w[HI];
+};
+
+// Stage q (bf16 [HI][D]) and w into shared memory as fp32.
+template <int D, int HI>
+__device__ __forceinline__ void load_query(ScoreSmem<D, HI> &s, const uint16_t *q, const float *w) {
+    for (int e = threadIdx.x; e < HI * D / 2; e += blockDim.x) {
+        int h = e / (D / 2), j = e % (D / 2);
+        uint32_t two = *reinterpret_cast<const uint32_t *>(q + h * D + 2 * j);
+        s.q[j][h] = make_float2(bf16_bits_to_f32(two & 0xFFFFu), bf16_bits_to_f32(two >> 16));
+    }
+    if (threadIdx.x < HI) s.w[threadIdx.x] = w[threadIdx.x];
+}
+
+// Copy one 16-byte unit global -> shared (bypassing L1).
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
+// Scores of the thread's rows r_s = threadIdx.x + 128 s (s < kRowsPerThread), before
+// the per-entry scale.  Rows must be staged; invalid rows produce garbage the
+// caller discards.
+template <int D, int HI>
+__device__ __forceinline__ void score_rows(const ScoreSmem<D, HI> &s, float out[kRowsPerThread]) {
+    float2 acc[kRowsPerThread][HI];
+#pragma unroll
+    for (int r = 0; r < kRowsPerThread; ++r)
+#pragma unroll
+        for (int h = 0; h < HI; ++h) acc[r][h] = make_float2(0.0f, 0.0f);
+
+#pragma unroll
+    for (int u = 0; u < D / 16; ++u) {          // 16 channels = 8 pairs per unit
+        float2 qv[8][HI];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int h = 0; h < HI; ++h) qv[j][h] = s.q[8 * u + j][h];
+#pragma unroll
+        for (int r = 0; r < kRowsPerThread; ++r) {
+            int row = threadIdx.x + kScoreThreads * r;
+            uint4 kw = *reinterpret_cast<const uint4 *>(s.rows + row * D + 16 * swz<D>(row, u));
+            uint32_t wv[4] = {kw.x, kw.y, kw.z, kw.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t h01 = cvt_e4m3x2_f16x2(wv[i] & 0xFFFFu);
+                uint32_t h23 = cvt_e4m3x2_f16x2(wv[i] >> 16);
+                float2 k01 = __half22float2(*reinterpret_cast<__half2 *>(&h01));
+                float2 k23 = __half22float2(*reinterpret_cast<__half2 *>(&h23));
+#pragma unroll
+                for (int h = 0; h < HI; ++h) {
+                    acc[r][h] = fma2(qv[2 * i][h], k01, acc[r][h]);
+                    acc[r][h] = fma2(qv[2 * i + 1][h], k23, acc[r][h]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < kRowsPerThread; ++r) {
+        float t = 0.0f;
+#pragma unroll
+        for (int h = 0; h < HI; ++h) {
+            float a = __fadd_rn(acc[r][h].x, acc[r][h].y);
+            t = __fmaf_rn(s.w[h], a > 0.0f ? a : 0.0f, t);
+        }
+        out[r] = t;
+    }
+}
+
+// ------------------------------------------------------------------------------
+// a3: Full scan.  grid (ceil(n_max / 512), B*Tq), 128 threads.
+// ------------------------------------------------------------------------------
+template <int D, int HI>
+__global__ void __launch_bounds__(kScoreThreads)
+index_scan_kernel(IndexArgs a) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    ScoreSmem<D, HI> &s = *reinterpret_cast<ScoreSmem<D, HI> *>(smem_raw);
+    const int qi = blockIdx.y;
+    const int b = qi / a.Tq;
+    int64_t N = visible_entries(a.q_pos[qi], a.ratio);
+    if (N > a.n_max || N > a.cap) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_NMAX);
+        N = min64(min64(N, a.n_max), a.cap);
+    }
+    const int64_t p0 = (int64_t)blockIdx.x * kTileRows;
+    if (p0 >= N) return;
+    const int rows = (int)min64(kTileRows, N - p0);
+
+    const uint8_t *src = a.idx_codes + ((int64_t)b * a.cap + p0) * D;
+    constexpr int U = D / 16;
+    for (int e = threadIdx.x; e < rows * U; e += kScoreThreads) {
+        int r = e / U, u = e % U;
+        cp_async16(s.rows + r * D + 16 * swz<D>(r, u), src + (int64_t)e * 16);
+    }
+    cp_async_commit();
+    load_query<D, HI>(s, a.q_idx + (int64_t)qi * HI * D, a.w + (int64_t)qi * HI);
+    cp_async_wait_all();
+    __syncthreads();
+
+    float sc[kRowsPerThread];
+    score_rows<D, HI>(s, sc);
+
+    float *scores = a.scores + (int64_t)qi * a.score_stride;
+    const float *sig = a.idx_scale + (int64_t)b * a.cap;
+#pragma unroll
+    for (int r = 0; r < kRowsPerThread; ++r) {
+        int row = threadIdx.x + kScoreThreads * r;
+        int64_t p = p0 + row;
+        float v = -INFINITY;
+        if (row < rows) {
+            v = __fmul_rn(sc[r], sig[p]);
+            scores[p] = v;
+        }
+        if (a.bmax) {
+            // block of 8 positions = 8 consecutive lanes
+            float m = v;
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+            if ((row & 7) == 0 && row < rows) a.bmax[(int64_t)qi * a.bmax_stride + p / 8] = m;
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------
+// a6: Reindex scoring of the pool.  grid (ceil(pool_blocks / 64), B*Tq), 128 thr.
+// Candidate c = 8 * slot + r of the pool (slot < pool_blocks, r < 8) is position
+// 8 * pool[slot] + r; its score goes to scores[qi][c].
+// ------------------------------------------------------------------------------
+template <int D, int HI>
+__global__ void __launch_bounds__(kScoreThreads)
+reindex_score_kernel(IndexArgs a) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    ScoreSmem<D, HI> &s = *reinterpret_cast<ScoreSmem<D, HI> *>(smem_raw);
+    __shared__ int valid_row[kTileRows];
+    __shared__ int pos_row[kTileRows];
+    const int qi = blockIdx.y;
+    const int b = qi / a.Tq;
+    int64_t N = visible_entries(a.q_pos[qi], a.ratio);
+    N = min64(N, a.cap);
+    const int slot0 = blockIdx.x * (kTileRows / 8);
+    const int32_t *pool = a.pool + (int64_t)qi * a.pool_blocks;
+
+    for (int r = threadIdx.x; r < kTileRows; r += kScoreThreads) {
+        int slot = slot0 + r / 8;
+        int blk = slot < a.pool_blocks ? pool[slot] : -1;
+        int64_t p = (int64_t)blk * 8 + (r & 7);
+        bool ok = blk >= 0 && p < N;
+        if (blk >= 0 && (int64_t)blk * 8 >= N && (r & 7) == 0) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
+        valid_row[r] = ok;
+        pos_row[r] = ok ? (int)p : 0;
+    }
+    __syncthreads();
+    const uint8_t *base = a.idx_codes + (int64_t)b * a.cap * D;
+    constexpr int U = D / 16;
+    for (int e = threadIdx.x; e < kTileRows * U; e += kScoreThreads) {
+        int r = e / U, u = e % U;
+        if (valid_row[r])
+            cp_async16(s.rows + r * D + 16 * swz<D>(r, u), base + (int64_t)pos_row[r] * D + 16 * u);
+    }
+    cp_async_commit();
+    load_query<D, HI>(s, a.q_idx + (int64_t)qi * HI * D, a.w + (int64_t)qi * HI);
+    cp_async_wait_all();
+    __syncthreads();
+
+    float sc[kRowsPerThread];
+    score_rows<D, HI>(s, sc);
+    const float *sig = a.idx_scale + (int64_t)b * a.cap;
+    float *out = a.scores + (int64_t)qi * a.score_stride + (int64_t)slot0 * 8;
+#pragma unroll
+    for (int r = 0; r < kRowsPerThread; ++r) {
+        int row = threadIdx.x + kScoreThreads * r;
+        if (slot0 + row / 8 < a.pool_blocks)
+            out[row] = valid_row[row] ? __fmul_rn(sc[r], sig[pos_row[row]]) : 0.0f;
+    }
+}
+
+// ------------------------------------------------------------------------------
+// Block-wide Top-K selection (one CTA per query).
+// Radix select over 32-bit order keys, most significant byte first, then a
+// compaction in index order: every key above the threshold, plus the
+// lowest-indexed keys equal to it.  Candidate index order == position order.
+// ------------------------------------------------------------------------------
+constexpr int kSelThreads = 1024;
+constexpr int kSelStageMax = 16384;   // keys staged in shared memory up to this count
+
+struct SelSmem {
+    uint32_t hist[256];
+    int warp_tot[32];
+    int bcast[4];
+    int pool[CSA2_POOL_MAX];
+    uint32_t keys[kSelStageMax];
+};
+
+__device__ __forceinline__ int block_excl_scan(bool flag, int &total, SelSmem &s) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t bal = __ballot_sync(0xFFFFFFFFu, flag);
+    int excl = __popc(bal & ((1u << lane) - 1u));
+    if (lane == 0) s.warp_tot[warp] = __popc(bal);
+    __syncthreads();
+    if (warp == 0) {
+        int v = s.warp_tot[lane];
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        s.warp_tot[lane] = incl - v;
+        if (lane == 31) s.bcast[3] = incl;
+    }
+    __syncthreads();
+    int r = s.warp_tot[warp] + excl;
+    total = s.bcast[3];
+    __syncthreads();
+    return r;
+}
+
+// Threshold key T and the number of keys equal to T to take, so that
+// #(key > T) + take == k.  Keys equal to 0 are never candidates.  1 <= k <= #valid.
+template <class KeyAt>
+__device__ void radix_threshold(KeyAt key_at, int n, int k, SelSmem &s, uint32_t &T, int &take) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t prefix = 0;
+    int rem = k;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) s.hist[i] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            uint32_t key = key_at(i);
+            bool match = key != 0u && (pass == 0 || ((key ^ prefix) >> (shift + 8)) == 0u);
+            if (match) {
+                uint32_t bin = (key >> shift) & 255u;
+                uint32_t peers = __match_any_sync(__activemask(), bin);
+                if (lane == __ffs(peers) - 1) atomicAdd(&s.hist[bin], (uint32_t)__popc(peers));
+            }
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // lane l owns bins 255-8l .. 248-8l, visited in descending order
+            uint32_t c[8], sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) { c[i] = s.hist[255 - 8 * lane - i]; sum += c[i]; }
+            uint32_t incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            uint32_t run = incl - sum;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (run < (uint32_t)rem && (uint32_t)rem <= run + c[i]) {
+                    s.bcast[0] = 255 - 8 * lane - i;
+                    s.bcast[1] = (int)run;
+                }
+                run += c[i];
+            }
+        }
+        __syncthreads();
+        prefix |= (uint32_t)s.bcast[0] << shift;
+        rem -= s.bcast[1];
+        __syncthreads();
+    }
+    T = prefix;
+    take = rem;
+}
+
+// Writes the selected candidates' ids, ascending, to out[0..k); returns k.
+template <class KeyAt, class IdAt>
+__device__ int compact_selected(KeyAt key_at, IdAt id_at, int n, uint32_t T, int take,
+                                int *out, SelSmem &s) {
+    int base_sel = 0, base_eq = 0;
+    for (int start = 0; start < n; start += blockDim.x) {
+        int i = start + threadIdx.x;
+        uint32_t key = i < n ? key_at(i) : 0u;
+        bool eq = key != 0u && key == T;
+        int eq_tot;
+        int eq_rank = block_excl_scan(eq, eq_tot, s);
+        bool sel = key > T || (eq && base_eq + eq_rank < take);
+        int sel_tot;
+        int sel_rank = block_excl_scan(sel, sel_tot, s);
+        if (sel) out[base_sel + sel_rank] = id_at(i);
+        base_sel += sel_tot;
+        base_eq += eq_tot;
+    }
+    return base_sel;
+}
+
+// Top-k of n candidates (keys from key_at, 0 = not a candidate) -> ascending ids
+// in out[0..cnt), cnt = min(k, #valid) returned.
+template <class KeyAt, class IdAt>
+__device__ int block_topk(KeyAt key_at, IdAt id_at, int n, int k, int *out, SelSmem &s) {
+    // number of valid candidates
+    int local = 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) local += key_at(i) != 0u;
+    local = __reduce_add_sync(0xFFFFFFFFu, local);
+    if ((threadIdx.x & 31) == 0) s.warp_tot[threadIdx.x >> 5] = local;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        int v = (threadIdx.x < (blockDim.x >> 5)) ? s.warp_tot[threadIdx.x] : 0;
+        v = __reduce_add_sync(0xFFFFFFFFu, v);
+        if (threadIdx.x == 0) s.bcast[2] = v;
+    }
+    __syncthreads();
+    const int nvalid = s.bcast[2];
+    __syncthreads();
+    const int kk = min(k, nvalid);
+    if (kk == 0) return 0;
+    uint32_t T;
+    int take;
+    radix_threshold(key_at, n, kk, s, T, take);
+    return compact_selected(key_at, id_at, n, T, take, out, s);
+}
+
+// a4 + a5: one CTA per query.  Hierarchical: pool from block maxima, then Top-K
+// inside the pool's positions (equal to Top-K over all positions because every
+// pool block's best position outranks any position outside the pool, and
+// pool_blocks >= top_k).  Flat: Top-K over all visible positions.
+__global__ void __launch_bounds__(kSelThreads)
+select_full_kernel(IndexArgs a) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    SelSmem &s = *reinterpret_cast<SelSmem *>(smem_raw);
+    __shared__ int sel_out[CSA2_TOPK_MAX];
+    const int qi = blockIdx.x;
+    int64_t N64 = visible_entries(a.q_pos[qi], a.ratio);
+    N64 = min64(min64(N64, a.n_max), a.cap);
+    const int N = (int)N64;
+    const float *scores = a.scores + (int64_t)qi * a.score_stride;
+    int cnt;
+    if (a.pool_blocks > 0) {
+        const int nb = (N + 7) / 8;
+        const float *bm = a.bmax + (int64_t)qi * a.bmax_stride;
+        const bool staged = nb <= kSelStageMax;
+        if (staged) {
+            for (int i = threadIdx.x; i < nb; i += blockDim.x) s.keys[i] = score_key(bm[i]);
+            __syncthreads();
+        }
+        auto bkey = [&](int i) -> uint32_t { return staged ? s.keys[i] : score_key(bm[i]); };
+        auto bid = [&](int i) -> int { return i; };
+        int np = block_topk(bkey, bid, nb, a.pool_blocks, s.pool, s);
+        __syncthreads();
+        int32_t *pool_out = a.pool_out ? a.pool_out + (int64_t)qi * a.pool_blocks : nullptr;
+        if (pool_out)
+            for (int i = threadIdx.x; i < a.pool_blocks; i += blockDim.x)
+                pool_out[i] = i < np ? s.pool[i] : -1;
+        // candidates: the pool's positions, in ascending order
+        const int nc = np * 8;
+        for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+            int64_t p = (int64_t)s.pool[i >> 3] * 8 + (i & 7);
+            s.keys[i] = p < N ? score_key(scores[p]) : 0u;
+        }
+        __syncthreads();
+        auto ckey = [&](int i) -> uint32_t { return s.keys[i]; };
+        auto cid = [&](int i) -> int { return s.pool[i >> 3] * 8 + (i & 7); };
+        cnt = block_topk(ckey, cid, nc, a.top_k, sel_out, s);
+    } else {
+        const bool staged = N <= kSelStageMax;
+        if (staged) {
+            for (int i = threadIdx.x; i < N; i += blockDim.x) s.keys[i] = score_key(scores[i]);
+            __syncthreads();
+        }
+        auto key = [&](int i) -> uint32_t { return staged ? s.keys[i] : score_key(scores[i]); };
+        auto id = [&](int i) -> int { return i; };
+        cnt = block_topk(key, id, N, a.top_k, sel_out, s);
+    }
+    __syncthreads();
+    int32_t *topk = a.topk_out + (int64_t)qi * a.top_k;
+    for (int i = threadIdx.x; i < a.top_k; i += blockDim.x) topk[i] = i < cnt ? sel_out[i] : -1;
+    if (threadIdx.x == 0) a.topk_count[qi] = cnt;
+}
+
+// a6 selection: Top-K of the scored pool candidates.
+__global__ void __launch_bounds__(kSelThreads)
+select_reindex_kernel(IndexArgs a) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    SelSmem &s = *reinterpret_cast<SelSmem *>(smem_raw);
+    __shared__ int sel_out[CSA2_TOPK_MAX];
+    const int qi = blockIdx.x;
+    int64_t N = min64(visible_entries(a.q_pos[qi], a.ratio), a.cap);
+    const int32_t *pool = a.pool + (int64_t)qi * a.pool_blocks;
+    const float *sc = a.scores + (int64_t)qi * a.score_stride;
+    const int nc = a.pool_blocks * 8;
+    for (int i = threadIdx.x; i < a.pool_blocks; i += blockDim.x) {
+        s.pool[i] = pool[i];
+        if (i > 0 && pool[i] >= 0 && pool[i - 1] >= pool[i]) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+        int blk = s.pool[i >> 3];
+        int64_t p = (int64_t)blk * 8 + (i & 7);
+        s.keys[i] = (blk >= 0 && p < N) ? score_key(sc[i]) : 0u;
+    }
+    __syncthreads();
+    auto key = [&](int i) -> uint32_t { return s.keys[i]; };
+    auto id = [&](int i) -> int { return s.pool[i >> 3] * 8 + (i & 7); };
+    int cnt = block_topk(key, id, nc, a.top_k, sel_out, s);
+    __syncthreads();
+    int32_t *topk = a.topk_out + (int64_t)qi * a.top_k;
+    for (int i = threadIdx.x; i < a.top_k; i += blockDim.x) topk[i] = i < cnt ? sel_out[i] : -1;
+    if (threadIdx.x == 0) a.topk_count[qi] = cnt;
+}
+
+// ------------------------------------------------------------------------------
+// Host launchers
+// ------------------------------------------------------------------------------
+template <int D, int HI>
+static cudaError_t launch_scan_t(const IndexArgs &a, int grid_x, int BT, cudaStream_t st) {
+    size_t smem = sizeof(ScoreSmem<D, HI>);
+    static bool attr_set = false;  // once per process and instantiation
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(index_scan_kernel<D, HI>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    index_scan_kernel<D, HI><<<dim3(grid_x, BT), kScoreThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <int D, int HI>
+static cudaError_t launch_reindex_t(const IndexArgs &a, int BT, cudaStream_t st) {
+    size_t smem = sizeof(ScoreSmem<D, HI>);
+    static bool attr_set = false;  // once per process and instantiation
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(reindex_score_kernel<D, HI>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    int gx = (a.pool_blocks + kTileRows / 8 - 1) / (kTileRows / 8);
+    reindex_score_kernel<D, HI><<<dim3(gx, BT), kScoreThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+#define CSA2_DISPATCH_HI(D, FN, ...)                                          \
+    switch (a.H_I) {                                                          \
+        case 1: return FN<D, 1>(__VA_ARGS__);                                 \
+        case 2: return FN<D, 2>(__VA_ARGS__);                                 \
+        case 4: return FN<D, 4>(__VA_ARGS__);                                 \
+        case 8: return FN<D, 8>(__VA_ARGS__);                                 \
+        case 16: return FN<D, 16>(__VA_ARGS__);                               \
+        default: return cudaErrorInvalidValue;                                \
+    }
+
+cudaError_t launch_index_scan(const IndexArgs &a, int BT, cudaStream_t st) {
+    int grid_x = (int)((a.n_max + kTileRows - 1) / kTileRows);
+    if (grid_x == 0) return cudaSuccess;
+    if (a.d_idx == 128) { CSA2_DISPATCH_HI(128, launch_scan_t, a, grid_x, BT, st) }
+    CSA2_DISPATCH_HI(64, launch_scan_t, a, grid_x, BT, st)
+}
+
+cudaError_t launch_reindex_score(const IndexArgs &a, int BT, cudaStream_t st) {
+    if (a.d_idx == 128) { CSA2_DISPATCH_HI(128, launch_reindex_t, a, BT, st) }
+    CSA2_DISPATCH_HI(64, launch_reindex_t, a, BT, st)
+}
+
+cudaError_t launch_select_full(const IndexArgs &a, int BT, cudaStream_t st) {
+    size_t smem = sizeof(SelSmem);
+    static bool attr_set = false;  // once per process (one device per process)
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(select_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    select_full_kernel<<<BT, kSelThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select_reindex(const IndexArgs &a, int BT, cudaStream_t st) {
+    size_t smem = sizeof(SelSmem);
+    static bool attr_set = false;  // once per process (one device per process)
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(select_reindex_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    select_reindex_kernel<<<BT, kSelThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+size_t score_smem_bytes(int d_idx, int H_I) {
+    if (d_idx == 128) return kTileRows * 128 + (128 / 2) * H_I * 8 + 64;
+    return kTileRows * 64 + (64 / 2) * H_I * 8 + 64;
+}
+
+}  // namespace csa2

@@ -1,0 +1,86 @@
+// csa2_internal.h -- kernel argument blocks and launchers shared by the .cu files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace csa2 {
+
+struct QuantArgs {
+    // main KV group (FP4 + FP8 indexer K)
+    uint8_t *codes;
+    uint8_t *scales;
+    uint8_t *idx_codes;
+    float *idx_scale;
+    int32_t cap;
+    int32_t d_idx;
+    const uint16_t *kv_bf16;
+    const uint16_t *idxk_bf16;
+    int32_t T_kv;
+    const int32_t *kv_start;
+    // SWA ring
+    uint8_t *swa_codes;
+    float *swa_scale;
+    int32_t wcap;
+    const uint16_t *swa_bf16;
+    int32_t T_swa;
+    const int32_t *swa_start;
+    // work split: warps of each kind
+    int64_t n_main, n_idx, n_swa;
+    int32_t *dev_err;
+};
+
+struct IndexArgs {
+    const uint8_t *idx_codes;
+    const float *idx_scale;
+    int32_t cap;
+    int32_t d_idx;
+    int32_t ratio;
+    const uint16_t *q_idx;   // [BT][H_I][d_idx] bf16 bits
+    const float *w;          // [BT][H_I]
+    const int32_t *q_pos;    // [BT]
+    int32_t Tq;
+    int32_t H_I;
+    int64_t n_max;
+    float *scores;           // workspace [BT][score_stride]
+    int64_t score_stride;
+    float *bmax;             // workspace [BT][bmax_stride] or null
+    int64_t bmax_stride;
+    const int32_t *pool;     // reindex input [BT][pool_blocks]
+    int32_t pool_blocks;
+    int32_t *pool_out;       // full output [BT][pool_blocks] or null
+    int32_t top_k;
+    int32_t *topk_out;
+    int32_t *topk_count;
+    int32_t *dev_err;
+};
+
+struct AttnArgs {
+    const uint8_t *codes;
+    const uint8_t *scales;
+    int32_t cap;
+    int32_t ratio;
+    const uint8_t *swa_codes;
+    const float *swa_scale;
+    int32_t wcap;
+    const uint16_t *q;       // [BT][H][512] bf16 bits
+    const int32_t *q_pos;
+    int32_t Tq;
+    int32_t H;
+    const int32_t *topk;     // [BT][top_k]
+    int32_t top_k;
+    int32_t swa_len;
+    float softmax_scale;
+    float *out;
+    float *lse;
+    int32_t *dev_err;
+};
+
+cudaError_t launch_quantize_append(const QuantArgs &a, cudaStream_t st);
+cudaError_t launch_index_scan(const IndexArgs &a, int BT, cudaStream_t st);
+cudaError_t launch_select_full(const IndexArgs &a, int BT, cudaStream_t st);
+cudaError_t launch_reindex_score(const IndexArgs &a, int BT, cudaStream_t st);
+cudaError_t launch_select_reindex(const IndexArgs &a, int BT, cudaStream_t st);
+cudaError_t launch_sparse_attn(const AttnArgs &a, int BT, cudaStream_t st);
+
+}  // namespace csa2

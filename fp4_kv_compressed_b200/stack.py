@@ -1,0 +1,192 @@
+"""CSA2 layer-stack driver: caches, per-layer buffers and the Full/Reindex/Reuse schedule.
+
+DeepSeek V4.1 Flash study notes, section 2 ("many layers share one global KV"):
+every CSA2 layer is statically Full, Reindex or Reuse; the decoder is 1 Full +
+4 Reindex + 15 Reuse layers sharing one global KV, each encoder group 1 Full +
+5 Reuse.  A Reuse layer takes the most recent selection of its group (nothing
+is recomputed); every layer keeps its own query and its own SWA window.  The
+decoder order "F U U U X U U U X ..." is this build's reading of the
+"Reindex-led groups" of myzaker's CSA2 section.
+
+This module only owns device buffers (allocated through PyTorch) and decides
+which library call runs for which layer; every step runs in libcsa2's kernels.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import _binding as bind
+
+KV_DIM = 512
+
+
+@dataclass(frozen=True)
+class LayerPlan:
+    layer: int        # global layer index, execution order
+    group: int        # global-KV group
+    mode: str         # "F" full, "X" reindex, "U" reuse
+    source: int       # layer whose Top-K this layer attends with
+
+
+def plan_layers(schedules: list[str]) -> list[LayerPlan]:
+    """Execution plan of a stack of groups; Reuse points at the nearest preceding
+    Full/Reindex layer of its own group.  Raises on a schedule that cannot run
+    (a Reindex or Reuse layer with no selection before it)."""
+    out: list[LayerPlan] = []
+    layer = 0
+    for g, sched in enumerate(schedules):
+        last_sel = None
+        have_pool = False
+        for m in sched:
+            if m == "F":
+                last_sel, have_pool = layer, True
+            elif m == "X":
+                if not have_pool:
+                    raise ValueError(f"group {g}: Reindex layer {layer} before any Full layer")
+                last_sel = layer
+            elif m == "U":
+                if last_sel is None:
+                    raise ValueError(f"group {g}: Reuse layer {layer} with nothing to reuse")
+            else:
+                raise ValueError(f"unknown layer mode {m!r}")
+            out.append(LayerPlan(layer, g, m, last_sel))
+            layer += 1
+    return out
+
+
+@dataclass(frozen=True)
+class GroupSpec:
+    ratio: int
+    schedule: str
+    pool_blocks: int      # 0 = flat indexer
+    cap: int              # entries per request
+
+
+class GlobalKV:
+    """Device planes of one global-KV group (FP4 main KV + FP8 indexer K)."""
+
+    def __init__(self, B: int, cap: int, d_idx: int, ratio: int, device):
+        self.B, self.cap, self.d_idx, self.ratio = B, cap, d_idx, ratio
+        self.codes = torch.zeros(B, cap, KV_DIM // 2, dtype=torch.uint8, device=device)
+        self.scales = torch.zeros(B, cap, KV_DIM // 16, dtype=torch.uint8, device=device)
+        self.idx_codes = torch.zeros(B, cap, d_idx, dtype=torch.uint8, device=device)
+        self.idx_scale = torch.zeros(B, cap, dtype=torch.float32, device=device)
+        self.struct = bind.CSA2GlobalKV(self.codes.data_ptr(), self.scales.data_ptr(),
+                                        self.idx_codes.data_ptr(), self.idx_scale.data_ptr(),
+                                        B, cap, d_idx, ratio)
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in
+                   (self.codes, self.scales, self.idx_codes, self.idx_scale))
+
+
+class SwaRing:
+    """One layer's FP8 SWA window ring: token p lives in slot p % window_cap."""
+
+    def __init__(self, B: int, window_cap: int, device):
+        self.B, self.window_cap = B, window_cap
+        self.codes = torch.zeros(B, window_cap, KV_DIM, dtype=torch.uint8, device=device)
+        self.scale = torch.zeros(B, window_cap, dtype=torch.float32, device=device)
+        self.struct = bind.CSA2SWA(self.codes.data_ptr(), self.scale.data_ptr(), B, window_cap)
+
+
+class DecodeStack:
+    """All device state of a CSA2 stack for a batch of B requests, Tq queries each."""
+
+    def __init__(self, B: int, H: int, H_I: int, d_idx: int, top_k: int, swa_len: int,
+                 groups: list[GroupSpec], Tq: int = 1, window_cap: int | None = None,
+                 device="cuda"):
+        self.B, self.H, self.H_I, self.d_idx = B, H, H_I, d_idx
+        self.top_k, self.swa_len, self.Tq = top_k, swa_len, Tq
+        self.groups = groups
+        self.device = torch.device(device)
+        self.window_cap = window_cap or (swa_len + Tq - 1)
+        self.plan = plan_layers([g.schedule for g in groups])
+        self.kv = [GlobalKV(B, g.cap, d_idx, g.ratio, device) for g in groups]
+        self.swa = [SwaRing(B, self.window_cap, device) for _ in self.plan]
+        BT = B * Tq
+        dev = self.device
+        self.topk = {}
+        self.count = {}
+        for lp in self.plan:
+            if lp.mode in "FX":
+                self.topk[lp.layer] = torch.full((B, Tq, top_k), -1, dtype=torch.int32, device=dev)
+                self.count[lp.layer] = torch.zeros(B, Tq, dtype=torch.int32, device=dev)
+        self.pool = {g: torch.full((B, Tq, max(spec.pool_blocks, 1)), -1, dtype=torch.int32,
+                                   device=dev)
+                     for g, spec in enumerate(groups)}
+        self.out = [torch.zeros(B, Tq, H, KV_DIM, dtype=torch.float32, device=dev)
+                    for _ in self.plan]
+        self.lse = [torch.zeros(B, Tq, H, dtype=torch.float32, device=dev) for _ in self.plan]
+        ws = 256
+        for spec in groups:
+            ws = max(ws, bind.csa2_workspace_size(bind.CSA2_OP_INDEX_FULL, B, Tq, spec.cap, H,
+                                                  top_k, spec.pool_blocks))
+            if spec.pool_blocks:
+                ws = max(ws, bind.csa2_workspace_size(bind.CSA2_OP_INDEX_REINDEX, B, Tq, 0, H,
+                                                      top_k, spec.pool_blocks))
+        ws = max(ws, bind.csa2_workspace_size(bind.CSA2_OP_SPARSE_ATTN, B, Tq, 0, H, top_k, 0))
+        self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+        self.dev_err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.softmax_scale = KV_DIM ** -0.5
+
+    def topk_of(self, layer: int) -> torch.Tensor:
+        return self.topk[self.plan[layer].source]
+
+    def cache_bytes(self) -> int:
+        return sum(g.nbytes() for g in self.kv) + sum(
+            r.codes.numel() + r.scale.numel() * 4 for r in self.swa)
+
+    # -----------------------------------------------------------------------------------
+    def step(self, *, q_pos, n_max, q, q_idx, w, swa_bf16, swa_start, kv_bf16=None,
+             idxk_bf16=None, kv_start=None, stream=None):
+        """Run every layer of the stack once, in order.
+
+        q_pos [B][Tq] int32 token positions; n_max[g] >= visible entries of any query of
+        group g; q[l] bf16 [B][Tq][H][512]; q_idx[l] bf16 [B][Tq][H_I][d_idx] and w[l]
+        fp32 [B][Tq][H_I] for Full/Reindex layers; swa_bf16[l] bf16 [B][T_swa][512] new
+        SWA rows at token positions swa_start [B]; kv_bf16[g] / idxk_bf16[g] bf16
+        [B][T_kv][...] new entries of group g at entry slots kv_start[g] [B] (None =
+        nothing to append).
+        """
+        first_of_group = {}
+        for lp in self.plan:
+            first_of_group.setdefault(lp.group, lp.layer)
+        T_swa = swa_bf16[0].shape[1] if swa_bf16[0] is not None else 0
+        for lp in self.plan:
+            g, l = lp.group, lp.layer
+            kv = self.kv[g]
+            if l == first_of_group[g] and kv_bf16 is not None and kv_bf16[g] is not None:
+                T_kv = kv_bf16[g].shape[1]
+                bind.csa2_quantize_append(kv.struct, kv_bf16[g], idxk_bf16[g], T_kv, kv_start[g],
+                                       self.swa[l].struct, swa_bf16[l], T_swa, swa_start,
+                                       self.dev_err, stream)
+            elif swa_bf16[l] is not None:
+                bind.csa2_quantize_append(None, None, None, 0, None, self.swa[l].struct,
+                                       swa_bf16[l], T_swa, swa_start, self.dev_err, stream)
+            spec = self.groups[g]
+            if lp.mode == "F":
+                bind.csa2_index_full(kv.struct, q_idx[l], w[l], q_pos, self.Tq, self.H_I, n_max[g],
+                                  spec.pool_blocks, self.top_k,
+                                  self.pool[g] if spec.pool_blocks else None, self.topk[l],
+                                  self.count[l], self.workspace, self.dev_err, stream)
+            elif lp.mode == "X":
+                bind.csa2_index_reindex(kv.struct, q_idx[l], w[l], q_pos, self.Tq, self.H_I,
+                                     self.pool[g], spec.pool_blocks, self.top_k, self.topk[l],
+                                     self.count[l], self.workspace, self.dev_err, stream)
+            bind.csa2_sparse_attn_decode(kv.struct, self.swa[l].struct, q[l], q_pos, self.Tq, self.H,
+                                      self.topk_of(l), self.top_k, self.swa_len,
+                                      self.softmax_scale, self.out[l], self.lse[l],
+                                      self.workspace, self.dev_err, stream)
+
+    def launches_per_step(self, append: bool = True) -> int:
+        """Kernels one step() launches."""
+        n = 0
+        for lp in self.plan:
+            n += 1                     # quantise-append (SWA row, plus the group's entry)
+            n += {"F": 2, "X": 2, "U": 0}[lp.mode]
+            n += 1                     # attention
+        return n
+

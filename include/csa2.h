@@ -1,0 +1,220 @@
+/*
+ * csa2.h -- C ABI of the CSA2 global-attention decode path over an FP4 KV cache
+ * (libcsa2.so, sm_100a).
+ *
+ * The method: DeepSeek V4.1 Flash's CSA2 attention as described in
+ *   "DeepSeek V4.1 Flash: architecture study notes" (macin.top), sections 1-4, and
+ *   "DeepSeek V4.1 Flash goes online" (myzaker), sections "CSA2 attention" and
+ *   "cache precision and tiering".
+ * Every layer is statically Full, Reindex or Reuse.  A Full layer scans all
+ * visible global entries, builds a shared candidate pool of at most 2048 blocks
+ * of 8 positions and picks at most 512 entries; a Reindex layer re-scores only
+ * inside that pool with its own index query; a Reuse layer takes the most recent
+ * selection as is.  Each layer then attends, with its own query, over the
+ * selected FP4 entries together with its own 128-token FP8 SWA window.
+ *
+ * Conventions (all entry points):
+ *  - Every pointer is DEVICE memory owned by the caller unless stated otherwise.
+ *    The library allocates nothing, keeps no state between calls and is
+ *    re-entrant; calls on one stream execute in order.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  The returned status reports host-side validation
+ *    (null pointers, sizes, capacities) and launch errors (CSA2_ERR_CUDA).
+ *  - Bounds the host cannot see (device-resident positions, indices) are checked
+ *    in the kernels: a violating row / index is skipped and a CSA2_DEVERR_* bit
+ *    is OR-ed into `*dev_err` (an int32 in device memory, may be NULL).  Read it
+ *    with csa2_read_device_error().  Kernels never trap and never spin.
+ *  - bf16 inputs are row-major and contiguous; "B" is the request count, "Tq"
+ *    the number of query tokens per request (1 = decode, >1 = prefill chunk).
+ *  - Numbers are finite: NaN/Inf inputs are outside the contract.
+ */
+#ifndef CSA2_H_
+#define CSA2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSA2_API __attribute__((visibility("default")))
+#else
+#define CSA2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *csa2_stream_t; /* same handle as cudaStream_t */
+
+typedef enum csa2_status {
+    CSA2_OK = 0,
+    CSA2_ERR_INVALID_ARG = 1,   /* null pointer, bad size or shape */
+    CSA2_ERR_CAPACITY = 2,      /* a cache or ring too small for the request */
+    CSA2_ERR_WORKSPACE = 3,     /* workspace pointer null or smaller than required */
+    CSA2_ERR_UNSUPPORTED = 4,   /* shape outside what the kernels implement */
+    CSA2_ERR_CUDA = 5,          /* a CUDA launch or runtime call failed */
+    CSA2_ERR_DEVICE_BOUNDS = 6  /* csa2_read_device_error found a device-side bit */
+} csa2_status;
+
+/* Device-side error bits OR-ed into *dev_err. */
+#define CSA2_DEVERR_SLOT 0x1      /* append slot >= cap */
+#define CSA2_DEVERR_INDEX 0x2     /* a Top-K or pool id outside the visible range */
+#define CSA2_DEVERR_NMAX 0x4      /* a query sees more entries than n_max */
+#define CSA2_DEVERR_RANGE 0x8     /* a dequantised SWA value beyond the fp16 range */
+
+/* Limits of the kernels. */
+#define CSA2_KV_DIM 512           /* shared K=V latent width (MQA) */
+#define CSA2_GROUP 16             /* channels per E4M3 scale */
+#define CSA2_TOPK_MAX 512         /* at most 512 selected entries per query */
+#define CSA2_BLOCK 8              /* positions per pool block */
+#define CSA2_POOL_MAX 2048        /* at most 2048 pool blocks = 16384 positions */
+
+/*
+ * One global-KV group (shared by the Full layer and its Reindex / Reuse layers).
+ * Main KV (FP4, study notes section 4: 4-bit E2M1 values, one 8-bit E4M3 scale
+ * per 16 channels, 4 + 8/16 = 4.5 bits per value, no second-level scale):
+ *   codes   uint8 [batch][cap][256]  two E2M1 codes per byte, even channel in
+ *                                    the low nibble
+ *   scales  uint8 [batch][cap][32]   E4M3, scale j covers channels 16j..16j+15
+ * Indexer K (FP8 E4M3, one fp32 scale per entry; projected from the main KV
+ * entry, myzaker "CSA2 attention"):
+ *   idx_codes uint8 [batch][cap][d_idx],  idx_scale float [batch][cap]
+ * Entry e covers tokens [ratio*e, ratio*e + ratio) (ratio 1 decoder, 2 encoder
+ * groups, study notes section 3); the token at position t sees entries
+ * 0 .. (t+1)/ratio - 1.
+ */
+typedef struct csa2_global_kv {
+    uint8_t *codes;
+    uint8_t *scales;
+    uint8_t *idx_codes;
+    float *idx_scale;
+    int32_t batch;
+    int32_t cap;
+    int32_t d_idx;   /* 64 or 128 */
+    int32_t ratio;   /* 1 or 2 */
+} csa2_global_kv;
+
+/*
+ * One layer's SWA window (FP8 E4M3 with one fp32 scale per token; study notes
+ * sections 1 and 4: a 128-token local window per layer, kept in FP8).
+ * Token position p lives in ring slot p % window_cap.
+ *   codes uint8 [batch][window_cap][512],  scale float [batch][window_cap]
+ */
+typedef struct csa2_swa {
+    uint8_t *codes;
+    float *scale;
+    int32_t batch;
+    int32_t window_cap;
+} csa2_swa;
+
+/*
+ * a1/a2 quantise-append.  Main KV entries are quantised to FP4 after RoPE
+ * (myzaker "cache precision": the quantisation point is after RoPE, so the
+ * inputs here are post-RoPE): per 16 channels, scale = E4M3(amax / 6) and
+ * code = E2M1(x / scale), both round-to-nearest-even with saturation.  The
+ * indexer-K and SWA rows are quantised to E4M3 with sigma = amax / 448.
+ *
+ *   kv, kv_bf16 [B][T_kv][512], idxk_bf16 [B][T_kv][d_idx], kv_start [B]:
+ *       entry i of request b goes to slot kv_start[b] + i.  kv may be NULL
+ *       (then T_kv must be 0); kv_bf16 / idxk_bf16 may each be NULL to skip
+ *       that plane.
+ *   swa, swa_bf16 [B][T_swa][512], swa_start [B]:
+ *       token i of request b is token position swa_start[b] + i, stored in
+ *       ring slot (swa_start[b] + i) % window_cap.  swa may be NULL (T_swa 0).
+ * Errors: CSA2_ERR_INVALID_ARG for bad pointers/sizes; slots >= cap are
+ * skipped with CSA2_DEVERR_SLOT.
+ */
+CSA2_API csa2_status csa2_quantize_append(const csa2_global_kv *kv, const void *kv_bf16,
+                                 const void *idxk_bf16, int32_t T_kv, const int32_t *kv_start,
+                                 const csa2_swa *swa, const void *swa_bf16, int32_t T_swa,
+                                 const int32_t *swa_start, int32_t *dev_err,
+                                 csa2_stream_t stream);
+
+/* Operation ids for csa2_workspace_size. */
+#define CSA2_OP_INDEX_FULL 1
+#define CSA2_OP_INDEX_REINDEX 2
+#define CSA2_OP_SPARSE_ATTN 3
+
+/* Bytes of workspace an operation needs (0 if none).  n_max: the largest number
+ * of visible entries of any query of the call; H: attention heads; pool_blocks
+ * as passed to the call.  Returns 0 for an unknown op. */
+CSA2_API size_t csa2_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t n_max, int32_t H,
+                           int32_t top_k, int32_t pool_blocks);
+
+/*
+ * a3-a5 Full layer: for every query, score every visible entry s with
+ *   score(s) = sum_h w_h * relu(q_h . k_s)          (k_s: dequantised FP8 indexer K)
+ * in the fixed fp32 order: per head an fma chain over even channels and one over
+ * odd channels, added; then an fma chain over heads of (w_h, relu(a_h)); then
+ * times the entry's scale.  Then
+ *   pool_blocks > 0 (hierarchical, decoder): pool = the min(pool_blocks,
+ *       ceil(N/8)) blocks of 8 positions with the largest block score (max over
+ *       the block's visible positions), ascending ids, -1 padded; and Top-K =
+ *       the top_k highest-scoring visible positions (taken inside the pool,
+ *       which holds them all because pool_blocks >= top_k);
+ *   pool_blocks == 0 (flat, encoder groups): Top-K over all visible entries.
+ * Order: score descending, ties to the lower index.  Outputs ascending, -1 padded.
+ *   q_idx_bf16 [B][Tq][H_I][d_idx], w [B][Tq][H_I] fp32, q_pos [B][Tq] token
+ *   positions, n_max >= the visible count of every query, H_I in 1..16,
+ *   top_k in 1..512, pool_blocks 0 or top_k..2048.
+ *   pool_out [B][Tq][pool_blocks] (may be NULL when pool_blocks == 0),
+ *   topk_out [B][Tq][top_k], topk_count [B][Tq].
+ * Workspace: csa2_workspace_size(CSA2_OP_INDEX_FULL, B, Tq, n_max, 0, top_k,
+ * pool_blocks) bytes, 256-byte aligned.
+ */
+CSA2_API csa2_status csa2_index_full(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
+                            const int32_t *q_pos, int32_t Tq, int32_t H_I, int32_t n_max,
+                            int32_t pool_blocks, int32_t top_k, int32_t *pool_out,
+                            int32_t *topk_out, int32_t *topk_count, void *workspace,
+                            size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream);
+
+/*
+ * a6 Reindex layer: the same score with this layer's own q_idx / w, over the
+ * visible positions of the pool's blocks only, then Top-K (same order, same
+ * output form).  pool [B][Tq][pool_blocks] as written by csa2_index_full
+ * (-1 = unused slot).  Workspace: csa2_workspace_size(CSA2_OP_INDEX_REINDEX,
+ * B, Tq, 0, 0, top_k, pool_blocks).
+ */
+CSA2_API csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
+                               const int32_t *q_pos, int32_t Tq, int32_t H_I,
+                               const int32_t *pool, int32_t pool_blocks, int32_t top_k,
+                               int32_t *topk_out, int32_t *topk_count, void *workspace,
+                               size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream);
+
+/*
+ * a8 sparse attention.  For each query (request b, token position t = q_pos)
+ * and head h:
+ *   o_h = sum_j softmax_j(softmax_scale * q_h . v_j) v_j,  K = V = the entry,
+ * over j in {topk entries (FP4, dequantised)} U {SWA tokens max(0,t-swa_len+1)..t
+ * (FP8, dequantised)}, one softmax, no de-duplication.  A Reuse layer passes the
+ * topk buffer of the layer it reuses.
+ *   q_bf16 [B][Tq][H][512], topk [B][Tq][top_k] entry ids (-1 skipped; ids
+ *   must be visible to the query, else skipped with CSA2_DEVERR_INDEX),
+ *   swa_len in 0..window_cap-Tq+1, H a multiple of 16, top_k in 0..512.
+ *   out [B][Tq][H][512] fp32, lse [B][Tq][H] fp32 (natural log; a query with
+ *   no key gets o = 0 and lse = -inf).
+ * Precondition: dequantised SWA values lie within +-65504 (else
+ * CSA2_DEVERR_RANGE).  Workspace: csa2_workspace_size(CSA2_OP_SPARSE_ATTN, ...).
+ */
+CSA2_API csa2_status csa2_sparse_attn_decode(const csa2_global_kv *kv, const csa2_swa *swa,
+                                    const void *q_bf16, const int32_t *q_pos, int32_t Tq,
+                                    int32_t H, const int32_t *topk, int32_t top_k,
+                                    int32_t swa_len, float softmax_scale, float *out,
+                                    float *lse, void *workspace, size_t ws_bytes,
+                                    int32_t *dev_err, csa2_stream_t stream);
+
+/* Synchronise `stream`, read *dev_err (device int32) into *bits_out (host),
+ * reset it to 0, and return CSA2_ERR_DEVICE_BOUNDS if any bit was set. */
+CSA2_API csa2_status csa2_read_device_error(int32_t *dev_err, int32_t *bits_out, csa2_stream_t stream);
+
+/* Static description of a status code (never NULL). */
+CSA2_API const char *csa2_status_string(csa2_status status);
+
+/* ABI version: 100 * major + minor. */
+CSA2_API int32_t csa2_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA2_H_ */

@@ -78,16 +78,32 @@ EXPORT int csa2o_e2m1_encode(float r) {
     return sign | best;
 }
 
+/* E4M3 values of codes 0..255, filled once from csa2o_e4m3_value (speed only). */
+static double E4M3_TAB[256];
+static int e4m3_tab_ready = 0;
+
+static void e4m3_tab_init(void) {
+    if (e4m3_tab_ready) return;
+#pragma omp critical(csa2o_e4m3_tab)
+    {
+        if (!e4m3_tab_ready) {
+            for (int c = 0; c < 256; ++c) E4M3_TAB[c] = csa2o_e4m3_value(c);
+            e4m3_tab_ready = 1;
+        }
+    }
+}
+
 /* Round-to-nearest-even into E4M3 with saturation to +-448; sign kept. */
 EXPORT int csa2o_e4m3_encode(float x) {
     if (isnan(x)) return 0x7F;
+    e4m3_tab_init();
     int sign = signbit(x) ? 0x80 : 0;
     double a = fabs((double)x);
     if (a >= 448.0) return sign | 0x7E;
     int best = 0;
     double bd = a;
     for (int c = 1; c <= 0x7E; ++c) {
-        double d = fabs(a - csa2o_e4m3_value(c));
+        double d = fabs(a - E4M3_TAB[c]);
         if (d < bd || (d == bd && (c & 1) == 0)) { best = c; bd = d; }
     }
     return sign | best;
@@ -105,6 +121,8 @@ EXPORT int csa2o_e4m3_encode(float x) {
  * x: bf16 bits [rows][width]; codes [rows][width/2]; scales [rows][width/16]. */
 EXPORT void csa2o_quantize_fp4(const uint16_t *x, int64_t rows, int width,
                                uint8_t *codes, uint8_t *scales) {
+    e4m3_tab_init();
+#pragma omp parallel for schedule(static) if (rows > 256)
     for (int64_t r = 0; r < rows; ++r) {
         const uint16_t *xr = x + r * width;
         for (int g = 0; g < width / 16; ++g) {
@@ -138,6 +156,8 @@ EXPORT void csa2o_quantize_fp4(const uint16_t *x, int64_t rows, int width,
  * a zero sigma stores codes 0x00. */
 EXPORT void csa2o_quantize_fp8(const uint16_t *x, int64_t rows, int width,
                                uint8_t *codes, float *scale) {
+    e4m3_tab_init();
+#pragma omp parallel for schedule(static) if (rows > 256)
     for (int64_t r = 0; r < rows; ++r) {
         const uint16_t *xr = x + r * width;
         float amax = 0.0f;
@@ -208,8 +228,12 @@ EXPORT int64_t csa2o_visible(int64_t t, int ratio) {
 EXPORT void csa2o_scores(const uint8_t *kc, const float *ks, int d, const int32_t *pos,
                          int64_t n, const uint16_t *q, const float *w, int H_I, float *out) {
     float qf[16][256];
+    float kval[256];
+    e4m3_tab_init();
+    for (int c = 0; c < 256; ++c) kval[c] = (float)E4M3_TAB[c];
     for (int h = 0; h < H_I; ++h)
         for (int c = 0; c < d; ++c) qf[h][c] = csa2o_bf16_to_f32(q[h * d + c]);
+#pragma omp parallel for schedule(static) if (n > 65536)
     for (int64_t i = 0; i < n; ++i) {
         int64_t s = pos ? pos[i] : i;
         const uint8_t *row = kc + s * (int64_t)d;
@@ -217,8 +241,8 @@ EXPORT void csa2o_scores(const uint8_t *kc, const float *ks, int d, const int32_
         for (int h = 0; h < H_I; ++h) {
             float e = 0.0f, o = 0.0f;
             for (int c = 0; c < d; c += 2) {
-                e = fmaf(qf[h][c], (float)csa2o_e4m3_value(row[c]), e);
-                o = fmaf(qf[h][c + 1], (float)csa2o_e4m3_value(row[c + 1]), o);
+                e = fmaf(qf[h][c], kval[row[c]], e);
+                o = fmaf(qf[h][c + 1], kval[row[c + 1]], o);
             }
             float a = e + o;
             float r = (a > 0.0f) ? a : 0.0f;

@@ -211,3 +211,64 @@ def small_variant(w: Workload, *, B=None, ctx=None, H=None, Tq=None, name=None) 
         d["Tq"] = Tq
     d["name"] = name or (w.name + "_small")
     return Workload(**d)
+
+
+# ---- batched row generation (all requests at once, same bits as the per-request calls) ----
+def batch_rows_normal_bf16(seed: int, name: str, B: int, start: int, count: int, width: int,
+                           device="cpu", stride: int = POS_STRIDE) -> torch.Tensor:
+    """[B][count][width] bf16; row (b, start+i) equals rows_normal_bf16(..., b, start, ...)[i]."""
+    b = torch.arange(B, dtype=torch.int64, device=device).view(B, 1, 1)
+    p = (start + torch.arange(count, dtype=torch.int64, device=device)).view(1, count, 1)
+    c = torch.arange(width, dtype=torch.int64, device=device).view(1, 1, width)
+    idx = (b * stride + p) * width + c
+    return normal_bf16(seed, name, idx)
+
+
+def _main_kv_batch(self: Workload, g: int, start: int, count: int, device="cpu"):
+    x = batch_rows_normal_bf16(self.seed, f"g{g}.kv", self.B, start, count, KV_DIM, device)
+    return self._apply_scale(x)
+
+
+def _idx_k_batch(self: Workload, g: int, start: int, count: int, device="cpu"):
+    x = batch_rows_normal_bf16(self.seed, f"g{g}.idxk", self.B, start, count, self.d_I, device)
+    if self.planted and g == self.decoder_group:
+        for b in range(self.B):
+            pos, rows = self.planted_rows(b)
+            for p, r in zip(pos, rows):
+                if start <= p < start + count:
+                    x[b, p - start] = r.to(device)
+    return x
+
+
+def _swa_batch(self: Workload, layer: int, start: int, count: int, device="cpu"):
+    x = batch_rows_normal_bf16(self.seed, f"L{layer}.swa", self.B, start, count, KV_DIM, device)
+    return self._apply_scale(x)
+
+
+def _q_batch(self: Workload, layer: int, device="cpu"):
+    x = batch_rows_normal_bf16(self.seed, f"L{layer}.q", self.B, 0, self.Tq * self.H, KV_DIM,
+                               device, stride=Q_STRIDE)
+    return x.view(self.B, self.Tq, self.H, KV_DIM)
+
+
+def _q_idx_batch(self: Workload, layer: int, device="cpu"):
+    x = batch_rows_normal_bf16(self.seed, f"L{layer}.qidx", self.B, 0, self.Tq * self.H_I,
+                               self.d_I, device, stride=Q_STRIDE)
+    return x.view(self.B, self.Tq, self.H_I, self.d_I)
+
+
+def _w_batch(self: Workload, layer: int, device="cpu"):
+    from . import uniform_f32
+    b = torch.arange(self.B, dtype=torch.int64, device=device).view(self.B, 1, 1)
+    r = torch.arange(self.Tq, dtype=torch.int64, device=device).view(1, self.Tq, 1)
+    c = torch.arange(self.H_I, dtype=torch.int64, device=device).view(1, 1, self.H_I)
+    idx = (b * Q_STRIDE + r) * self.H_I + c
+    return uniform_f32(self.seed, f"L{layer}.w", idx)
+
+
+Workload.main_kv_batch = _main_kv_batch
+Workload.idx_k_batch = _idx_k_batch
+Workload.swa_batch = _swa_batch
+Workload.q_batch = _q_batch
+Workload.q_idx_batch = _q_idx_batch
+Workload.w_batch = _w_batch

@@ -1,0 +1,144 @@
+"""GPU parity of sparse attention (a8) and of whole stack steps (a1-a9) against
+the oracle: Top-K bit-exact, attention within 2e-3 (norm-wise per head row)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle_ref as R
+import synth
+from synth.workloads import WORKLOADS, small_variant
+
+pytestmark = pytest.mark.gpu
+
+ATTN_TOL = 2e-3      # max_c |o - o_ref| / max_c |o_ref| per (request, query, head)
+LSE_TOL = 1e-3       # absolute, natural-log units
+
+
+@pytest.fixture(scope="module")
+def pkg():
+    import fp4_kv_compressed_b200 as p
+    assert torch.cuda.is_available()
+    return p
+
+
+def _attn_case(pkg, orc, *, B, H, cap, W, q_pos, topk, swa_len, seed):
+    kv = pkg.GlobalKV(B, cap, 128, 1, "cuda")
+    ring = pkg.SwaRing(B, W, "cuda")
+    x = torch.stack([synth.rows_normal_bf16(seed, "kv", b, 0, cap, 512) for b in range(B)])
+    s = torch.stack([(synth.rows_normal_bf16(seed, "swa", b, 0, W, 512).float() * 3)
+                     .to(torch.bfloat16) for b in range(B)])
+    z = torch.zeros(B, dtype=torch.int32, device="cuda")
+    pkg.csa2_quantize_append(kv.struct, x.cuda(), None, cap, z, ring.struct, s.cuda(), W, z)
+    Tq = q_pos.shape[1]
+    q = torch.stack([synth.rows_normal_bf16(seed, "q", b, 0, Tq * H, 512, stride=synth.Q_STRIDE)
+                     for b in range(B)]).view(B, Tq, H, 512)
+    out = torch.zeros(B, Tq, H, 512, device="cuda")
+    lse = torch.zeros(B, Tq, H, device="cuda")
+    dev_err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    top_k = topk.shape[-1]
+    pkg.csa2_sparse_attn_decode(kv.struct, ring.struct if swa_len else None, q.cuda(),
+                                q_pos.cuda(), Tq, H, topk.cuda() if top_k else None, top_k,
+                                swa_len, 1 / math.sqrt(512), out, lse, None, dev_err)
+    bits = pkg.csa2_read_device_error(dev_err)
+    mc, ms = orc.quantize_fp4(x)
+    sc, ss = orc.quantize_fp8(s)
+    tk = topk.numpy() if top_k else np.full((B, Tq, 1), -1, np.int32)
+    o_ref, l_ref = orc.attention(mc, ms, sc, ss, q, q_pos.numpy(), tk, swa_len, 1 / math.sqrt(512))
+    return out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, bits
+
+
+def _assert_close(o, l, o_ref, l_ref):
+    err = R.rel_err_rows(o, o_ref)
+    assert err.max() <= ATTN_TOL, f"max row error {err.max():.3e}"
+    fin = np.isfinite(l_ref)
+    assert np.array_equal(np.isfinite(l), fin)
+    assert np.abs(l[fin] - l_ref[fin]).max(initial=0) <= LSE_TOL
+
+
+@pytest.mark.parametrize("H", [16, 64])
+def test_attention_random_sets(pkg, orc, H):
+    B, cap, W = 2, 700, 128
+    g = torch.Generator().manual_seed(H)
+    q_pos = torch.tensor([[699], [450]], dtype=torch.int32)
+    topk = torch.randint(-1, 451, (B, 1, 96), generator=g, dtype=torch.int32)
+    topk[0, 0, :10] = torch.arange(690, 700, dtype=torch.int32)      # recent entries, duplicates w/ window
+    o, l, o_ref, l_ref, bits = _attn_case(pkg, orc, B=B, H=H, cap=cap, W=W, q_pos=q_pos,
+                                          topk=topk, swa_len=128, seed=H)
+    assert bits == 0
+    _assert_close(o, l, o_ref, l_ref)
+
+
+def test_attention_edges(pkg, orc):
+    B, cap, W = 2, 300, 130
+    # window only, early position (window clipped at 0), ring wider than the window
+    q_pos = torch.tensor([[5], [200]], dtype=torch.int32)
+    o, l, o_ref, l_ref, _ = _attn_case(pkg, orc, B=B, H=16, cap=cap, W=W, q_pos=q_pos,
+                                       topk=torch.zeros(B, 1, 0, dtype=torch.int32),
+                                       swa_len=128, seed=1)
+    _assert_close(o, l, o_ref, l_ref)
+    # selected entries only (no window), with -1 padding
+    topk = torch.full((B, 1, 64), -1, dtype=torch.int32)
+    topk[0, 0, :3] = torch.tensor([0, 1, 5])
+    topk[1, 0, :40] = torch.arange(100, 140)
+    o, l, o_ref, l_ref, _ = _attn_case(pkg, orc, B=B, H=32, cap=cap, W=W, q_pos=q_pos,
+                                       topk=topk, swa_len=0, seed=2)
+    _assert_close(o, l, o_ref, l_ref)
+    # nothing at all: o = 0, lse = -inf
+    topk = torch.full((B, 1, 8), -1, dtype=torch.int32)
+    o, l, o_ref, l_ref, _ = _attn_case(pkg, orc, B=B, H=16, cap=cap, W=W, q_pos=q_pos,
+                                       topk=topk, swa_len=0, seed=3)
+    assert not o.any() and np.isneginf(l).all()
+    # an id past the visible range is skipped and flagged
+    topk = torch.full((B, 1, 8), 250, dtype=torch.int32)
+    _, _, _, _, bits = _attn_case(pkg, orc, B=B, H=16, cap=cap, W=W, q_pos=q_pos,
+                                  topk=topk, swa_len=4, seed=4)
+    assert bits & pkg.DEVERR_INDEX
+
+
+def _stack_check(wl, requests, layers=None):
+    import csa2_harness
+    dw = csa2_harness.DeviceWorkload(wl)
+    dw.step()
+    torch.cuda.synchronize()
+    assert dw.stack.dev_err.item() == 0
+    plan = R.reuse_sources(wl)
+    for b in requests:
+        gpu = dw.request_state(b)
+        # main rows needed: every selected entry of every selector layer
+        rows = {g: [] for g in range(len(wl.groups))}
+        for layer, t in gpu["topk"].items():
+            rows[plan[layer][0]].append(t.ravel())
+        rows = {g: np.concatenate(v) if v else np.zeros(0, np.int64) for g, v in rows.items()}
+        caches = R.request_caches(wl, b, main_rows=rows)
+        for g, c in enumerate(caches):
+            assert np.array_equal(gpu["kv"][g]["codes"][c["rows"]], c["codes"][c["rows"]])
+            assert np.array_equal(gpu["kv"][g]["scales"][c["rows"]], c["scales"][c["rows"]])
+        ref = R.index_layers(wl, b, caches)
+        for layer, t in ref["topk"].items():
+            assert np.array_equal(gpu["topk"][layer], t), f"request {b} layer {layer}"
+        for layer in (range(len(plan)) if layers is None else layers):
+            src = plan[layer][2]
+            o_ref, l_ref = R.attention_layer(wl, b, layer, caches, ref["topk"][src])
+            _assert_close(gpu["out"][layer], gpu["lse"][layer], o_ref, l_ref)
+
+
+def test_stack_decoder_group(pkg):
+    """Decoder group (F + 4X + 15U) on 2 requests at N = 20000, every layer."""
+    _stack_check(small_variant(WORKLOADS["decoder_group_32k"], B=2, ctx=20000), [0, 1])
+
+
+def test_stack_tiny(pkg):
+    _stack_check(WORKLOADS["tiny_full_layer"], [0])
+
+
+def test_stack_prefill_chunk(pkg):
+    """Encoder group, ratio 2, 64 causal queries sharing the cache, every layer."""
+    _stack_check(small_variant(WORKLOADS["prefill_chunk_enc"], B=1, ctx=3000 + 64, Tq=64), [0])
+
+
+def test_stack_scaled_channels(pkg):
+    """Per-channel log-uniform scales on the main KV and SWA (the 128K workload's inputs)."""
+    _stack_check(small_variant(WORKLOADS["decode_128k"], B=2, ctx=5000), [1],
+                 layers=[0, 3, 4, 19])
