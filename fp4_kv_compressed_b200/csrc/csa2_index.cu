@@ -317,7 +317,7 @@ __device__ void radix_threshold(KeyAt key_at, int n, int k, SelSmem &s, uint32_t
 // Writes the selected candidates' ids, ascending, to out[0..k); returns k.
 template <class KeyAt, class IdAt>
 __device__ int compact_selected(KeyAt key_at, IdAt id_at, int n, uint32_t T, int take,
-                                int *out, SelSmem &s) {
+                                int *out, int max_out, SelSmem &s) {
     int base_sel = 0, base_eq = 0;
     for (int start = 0; start < n; start += blockDim.x) {
         int i = start + threadIdx.x;
@@ -328,11 +328,11 @@ __device__ int compact_selected(KeyAt key_at, IdAt id_at, int n, uint32_t T, int
         bool sel = key > T || (eq && base_eq + eq_rank < take);
         int sel_tot;
         int sel_rank = block_excl_scan(sel, sel_tot, s);
-        if (sel) out[base_sel + sel_rank] = id_at(i);
+        if (sel && base_sel + sel_rank < max_out) out[base_sel + sel_rank] = id_at(i);
         base_sel += sel_tot;
         base_eq += eq_tot;
     }
-    return base_sel;
+    return min(base_sel, max_out);
 }
 
 // Top-k of n candidates (keys from key_at, 0 = not a candidate) -> ascending ids
@@ -358,7 +358,7 @@ __device__ int block_topk(KeyAt key_at, IdAt id_at, int n, int k, int *out, SelS
     uint32_t T;
     int take;
     radix_threshold(key_at, n, kk, s, T, take);
-    return compact_selected(key_at, id_at, n, T, take, out, s);
+    return compact_selected(key_at, id_at, n, T, take, out, kk, s);
 }
 
 // a4 + a5: one CTA per query.  Hierarchical: pool from block maxima, then Top-K
