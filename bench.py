@@ -250,6 +250,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = WORKLOADS[args.workload]
+    if args.batch:
+        from synth.workloads import small_variant
+        wl = small_variant(wl, B=args.batch, name=f"{wl.name}_b{args.batch}")
     dw = csa2_harness.DeviceWorkload(wl, device=dev)
     st = dw.stack
     inputs, dbuf, hbuf, in_bytes = pack_inputs(dw.inputs, dev)
@@ -327,34 +330,36 @@ def run_ours(args, rank, world, local_rank):
     out_h = torch.empty_like(st.out[last], device="cpu").pin_memory()
     lse_h = torch.empty_like(st.lse[last], device="cpu").pin_memory()
     out_bytes = out_h.numel() * 4 + lse_h.numel() * 4
-    Ke = max(3, min(K, args.e2e_steps))
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    for _ in range(2):
+    Ke = 0 if args.no_e2e else max(3, min(K, args.e2e_steps))
+    e2e_ms = None
+    if Ke:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+
+        def e2e_step():
+            dbuf.copy_(hbuf, non_blocking=True)          # this step's inputs, host -> device
+            g1.replay()
+            out_h.copy_(st.out[last], non_blocking=True)  # the step's result, device -> host
+            lse_h.copy_(st.lse[last], non_blocking=True)
         with torch.cuda.stream(stream):
-            dbuf.copy_(hbuf, non_blocking=True)
-            g1.replay()
-            out_h.copy_(st.out[last], non_blocking=True)
-            lse_h.copy_(st.lse[last], non_blocking=True)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    with torch.cuda.stream(stream):
-        e0.record()
-        for _ in range(Ke):
-            dbuf.copy_(hbuf, non_blocking=True)
-            g1.replay()
-            out_h.copy_(st.out[last], non_blocking=True)
-            lse_h.copy_(st.lse[last], non_blocking=True)
-        e1.record()
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item()) / Ke
+            for _ in range(2):
+                e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            e0.record()
+            for _ in range(Ke):
+                e2e_step()
+            e1.record()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te.item()) / Ke
 
     layers = len(st.plan)
     ms_step = ms_max / K
@@ -395,9 +400,9 @@ def run_ours(args, rank, world, local_rank):
                      "frac": achieved / peak, "peak_source": peak_src,
                      "traffic": traffic, "algorithmic_bytes_per_launch": full_bytes,
                      "launch_ms": full_ms},
-        "e2e": {"value": world * layers / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes,
-                "ms_per_step": e2e_ms},
+        "e2e": ({"value": world * layers / (e2e_ms / 1e3), "unit": UNIT,
+                 "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes,
+                 "ms_per_step": e2e_ms} if Ke else None),
         "gpu_launches": launches,
         "clocks": clocks.summary(),
     }
@@ -438,6 +443,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (small cases for profiling)")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="ncu dram bytes per launch of the timed kernel, if captured")
     args = ap.parse_args()
