@@ -27,8 +27,8 @@ DEVERR_SLOT, DEVERR_INDEX, DEVERR_NMAX, DEVERR_RANGE = 0x1, 0x2, 0x4, 0x8
 
 # every symbol declared in include/csa2.h
 EXPORTS = ("csa2_quantize_append", "csa2_workspace_size", "csa2_index_full",
-           "csa2_index_reindex", "csa2_sparse_attn_decode", "csa2_read_device_error",
-           "csa2_status_string", "csa2_abi_version")
+           "csa2_index_full_noalloc", "csa2_index_reindex", "csa2_sparse_attn_decode",
+           "csa2_read_device_error", "csa2_status_string", "csa2_abi_version")
 
 
 class Csa2Error(RuntimeError):

@@ -169,6 +169,33 @@ CSA2_API csa2_status csa2_index_full(const csa2_global_kv *kv, const void *q_idx
                             size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream);
 
 /*
+ * csa2_index_full without a workspace argument, for callers that cannot allocate
+ * device memory -- for example a backend plugin that runs inside a host
+ * framework's execute callback where the framework owns all device memory, or a
+ * latency-critical loop that cannot take cudaMalloc's device-wide sync.  The
+ * pages have no counterpart: this is an interface convenience, not part of the
+ * method.
+ * Same arguments, results and errors as csa2_index_full; the scores and block
+ * maxima live in a fixed array of CSA2_NOALLOC_SCRATCH_BYTES inside the library,
+ * allocated on every GPU that loads the library and held until the process
+ * exits.  A call that would need more than that (see csa2_workspace_size with
+ * CSA2_OP_INDEX_FULL) returns CSA2_ERR_WORKSPACE and launches nothing.
+ * The first call on a device looks up the array's device address (one-time
+ * set-up, guarded by a mutex); make that first call before any stream capture.
+ * Every call on a device shares the one array: calls that can overlap on the GPU
+ * (different streams without ordering, or several host threads) race on it, so
+ * order them.  Nothing in the array has to start at zero: each call writes all
+ * the scratch it reads.
+ */
+#define CSA2_NOALLOC_SCRATCH_BYTES (16u << 20)
+CSA2_API csa2_status csa2_index_full_noalloc(const csa2_global_kv *kv, const void *q_idx_bf16,
+                                             const float *w, const int32_t *q_pos, int32_t Tq,
+                                             int32_t H_I, int32_t n_max, int32_t pool_blocks,
+                                             int32_t top_k, int32_t *pool_out,
+                                             int32_t *topk_out, int32_t *topk_count,
+                                             int32_t *dev_err, csa2_stream_t stream);
+
+/*
  * a6 Reindex layer: the same score with this layer's own q_idx / w, over the
  * visible positions of the pool's blocks only, then Top-K (same order, same
  * output form).  pool [B][Tq][pool_blocks] as written by csa2_index_full
