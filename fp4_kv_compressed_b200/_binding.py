@@ -23,7 +23,7 @@ STATUS = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_CAPACITY",
           3: "CSA2_ERR_WORKSPACE", 4: "CSA2_ERR_UNSUPPORTED", 5: "CSA2_ERR_CUDA",
           6: "CSA2_ERR_DEVICE_BOUNDS"}
 
-DEVERR_SLOT, DEVERR_INDEX, DEVERR_NMAX, DEVERR_RANGE = 0x1, 0x2, 0x4, 0x8
+DEVERR_SLOT, DEVERR_INDEX, DEVERR_NMAX, DEVERR_RANGE, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
 
 # every symbol declared in include/csa2.h
 EXPORTS = ("csa2_quantize_append", "csa2_workspace_size", "csa2_index_full",

@@ -263,7 +263,6 @@ csa2_status csa2_sparse_attn_decode(const csa2_global_kv *kv, const csa2_swa *sw
         if ((int64_t)swa_len + Tq - 1 > swa->window_cap) return CSA2_ERR_CAPACITY;
     }
     const int64_t BT = (int64_t)kv->batch * Tq;
-    if (BT > 65535) return CSA2_ERR_UNSUPPORTED;   // grid.y limit of the attention kernel
 
     AttnArgs a;
     memset(&a, 0, sizeof(a));

@@ -61,6 +61,7 @@ typedef enum csa2_status {
 #define CSA2_DEVERR_INDEX 0x2     /* a Top-K or pool id outside the visible range */
 #define CSA2_DEVERR_NMAX 0x4      /* a query sees more entries than n_max */
 #define CSA2_DEVERR_RANGE 0x8     /* a dequantised SWA value beyond the fp16 range */
+#define CSA2_DEVERR_TIMEOUT 0x10  /* a kernel's bounded wait gave up (internal error) */
 
 /* Limits of the kernels. */
 #define CSA2_KV_DIM 512           /* shared K=V latent width (MQA) */
