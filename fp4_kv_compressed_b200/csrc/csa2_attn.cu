@@ -6,7 +6,9 @@
 // together with its own 128-token FP8 SWA window; one softmax over the union.
 // K = V = the 512-channel entry (MQA, fixed for this build).
 //
-// One CTA per (query, group of 64 heads); 16 warps, specialised:
+// A 2-CTA cluster per (query, group of 64 heads); each CTA takes half of the
+// query's key tiles and the two partial results are merged through distributed
+// shared memory (each CTA writes half of the output channels).  16 warps, specialised:
 //   warp 0      TMEM allocation + the single MMA-issuing thread;
 //   warps 4-7   softmax, one per TMEM lane quadrant (warp w reads lanes 32(w%4)..);
 //   warps 8-15  producers: gather the tile's rows (FP4 entry or FP8 SWA row) into
@@ -22,8 +24,9 @@
 // layout), the two S buffers (64 x 64 fp32) at lane offset 16, columns 0..127.
 // Online softmax in the log2 domain with lazy rescaling: O is rescaled only when
 // a head's running max grows by more than 8 (p stays <= 2^8, safe in fp16).
-// Every wait is bounded: on timeout the kernel flags CSA2_DEVERR_TIMEOUT, drains
-// its MMAs, frees TMEM and returns.
+// The MMA thread issues S(i+1) and P V(i) as soon as each is ready.  Every wait is
+// bounded: on timeout the kernel flags CSA2_DEVERR_TIMEOUT, drains its MMAs, frees
+// TMEM and returns.
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -47,10 +50,10 @@ struct __align__(1024) Smem {
     float sig[2][kTK];               // per-key scale of each stage (1 FP4, sigma SWA, 0 none)
     uint64_t kv_full[2], kv_empty[2], s_full[2], p_full, pv_done, drain;
     uint32_t tmem_base;
-    int32_t n_sel;
     int32_t abort;
-    float qmax[16];
-    int32_t warp_cnt[16];
+    float wred[16];
+    int32_t wcnt[16];
+    float cm[kHeads], cl[kHeads];    // this CTA's partial softmax max / sum per head
 };
 
 // ---- small PTX wrappers ---------------------------------------------------------------
@@ -182,12 +185,13 @@ struct Raw {
     int kind;        // 0 none, 1 FP4 entry, 2 SWA row
 };
 
-__device__ __forceinline__ void load_raw(Raw &r, const AttnArgs &a, const Smem &s, int b,
-                                         int64_t w0, int n_keys, int tile, int row, int quarter) {
+__device__ __forceinline__ void load_raw(Raw &r, const AttnArgs &a, const int32_t *ids, int n_sel,
+                                         int b, int64_t w0, int n_keys, int tile, int row,
+                                         int quarter) {
     const int kg = tile * kTK + row;
     r.kind = 0;
-    if (kg < s.n_sel) {
-        const int e = s.ids[kg];
+    if (kg < n_sel) {
+        const int e = ids[kg];
         const int64_t off = (int64_t)b * a.cap + e;
         const uint4 *src = reinterpret_cast<const uint4 *>(a.codes + off * kCodeBytes + 64 * quarter);
 #pragma unroll
@@ -195,7 +199,7 @@ __device__ __forceinline__ void load_raw(Raw &r, const AttnArgs &a, const Smem &
         r.s = __ldg(reinterpret_cast<const uint2 *>(a.scales + off * kScaleBytes + 8 * quarter));
         r.kind = 1;
     } else if (kg < n_keys) {
-        const int64_t pos = w0 + (kg - s.n_sel);
+        const int64_t pos = w0 + (kg - n_sel);
         const int64_t slot = (int64_t)b * a.wcap + pos % a.wcap;
         const uint4 *src = reinterpret_cast<const uint4 *>(a.swa_codes + slot * kDim + 128 * quarter);
 #pragma unroll
@@ -214,16 +218,22 @@ __device__ __forceinline__ void store_dequant(const Raw &r, uint8_t *tile, int r
                                  r.c[1].z, r.c[1].w, r.c[2].x, r.c[2].y, r.c[2].z, r.c[2].w,
                                  r.c[3].x, r.c[3].y, r.c[3].z, r.c[3].w};
         const uint32_t sc[2] = {r.s.x, r.s.y};
+        uint32_t scale2[8];                            // one f16x2 scale per 16 channels
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const uint32_t pair = (sc[g >> 1] >> (16 * (g & 1))) & 0xFFFFu;   // scales 2g, 2g+1
+            const uint32_t h = cvt_e4m3x2_f16x2(pair);
+            scale2[2 * g] = (h & 0xFFFFu) * 0x10001u;
+            scale2[2 * g + 1] = (h >> 16) * 0x10001u;
+        }
 #pragma unroll
         for (int u = 0; u < 16; ++u) {                 // 8 channels per 32-bit code word
-            const uint32_t sb = (sc[u >> 3] >> (8 * ((u >> 1) & 3))) & 0xFFu;
-            const uint32_t sh = cvt_e4m3x2_f16x2(sb | (sb << 8));
-            const __half2 scale2 = *reinterpret_cast<const __half2 *>(&sh);
+            const __half2 sv = *reinterpret_cast<const __half2 *>(&scale2[u >> 1]);
             uint32_t v[4];
             cvt_e2m1x8_f16x2(cw[u], v);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                __half2 x = __hmul2(*reinterpret_cast<__half2 *>(&v[j]), scale2);
+                __half2 x = __hmul2(*reinterpret_cast<__half2 *>(&v[j]), sv);
                 v[j] = *reinterpret_cast<uint32_t *>(&x);
             }
             *reinterpret_cast<uint4 *>(tile + tile_off(row, ch0 + 8 * u)) =
@@ -250,12 +260,55 @@ __device__ __forceinline__ void store_dequant(const Raw &r, uint8_t *tile, int r
     }
 }
 
+// ---- cluster helpers (2 CTAs per query split its keys; partials combine via DSMEM) ----
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t peer_addr(const void *local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float ld_peer(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_peer4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c),
+                 "f"(d)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n.reg .pred p;\n"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done)
+        : "r"(smem_u32(b)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+attn_tc_kernel(AttnArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem &s = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qi = blockIdx.x;
+    const uint32_t rank = cluster_rank();
+    const int qi = blockIdx.x >> 1;
     const int b = qi / a.Tq;
     const int h0 = blockIdx.y * kHeads;
     const int hcta = min(kHeads, a.H - h0);
@@ -264,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
     const int n_win = a.swa_len > 0 ? (int)(t - w0 + 1) : 0;
     const int64_t n_vis = min64(visible_entries((int32_t)t, a.ratio), a.cap);
 
-    // ---- set-up ------------------------------------------------------------------------
+    // ---- set-up (all threads) -------------------------------------------------------------
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.kv_full[i], 8);
@@ -283,155 +336,144 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
                      "r"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
-    // compact the valid selected ids (ids must be visible entries), warps 8-15
-    if (warp >= 8) {
-        const int pt = threadIdx.x - 256;                     // 0..255, two ids each
-        const int32_t *src = a.topk + (int64_t)qi * a.top_k;
-        int e0 = (2 * pt < a.top_k) ? src[2 * pt] : -1;
-        int e1 = (2 * pt + 1 < a.top_k) ? src[2 * pt + 1] : -1;
-        const bool ok0 = e0 >= 0 && e0 < n_vis, ok1 = e1 >= 0 && e1 < n_vis;
-        if ((e0 >= 0 && !ok0) || (e1 >= 0 && !ok1)) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
-        const int mine = (int)ok0 + (int)ok1;
-        int incl = mine;
+    // selected ids: thread t checks topk[t]; valid ids are compacted in order
+    const int32_t *tk = a.topk + (int64_t)qi * a.top_k;
+    const int e_id = (int)threadIdx.x < a.top_k ? tk[threadIdx.x] : -1;
+    const bool e_ok = e_id >= 0 && e_id < n_vis;
+    if (e_id >= 0 && !e_ok) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, e_ok);
+    // Q chunks of 8 channels: thread t holds chunks t + 512 j
+    const uint16_t *q = a.q + ((int64_t)qi * a.H + h0) * kDim;
+    uint4 qv[8];
+    float qm = 0.0f;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        if (lane == 31) s.warp_cnt[warp - 8] = incl;
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        int base = 0;
-        for (int w = 0; w < warp - 8; ++w) base += s.warp_cnt[w];
-        int pos = base + incl - mine;
-        if (ok0) s.ids[pos++] = e0;
-        if (ok1) s.ids[pos] = e1;
-        if (threadIdx.x == 511) s.n_sel = base + incl;
-        // Q: max |q| over the CTA's heads, then fp16 with a power-of-two scale
-        const uint16_t *q = a.q + ((int64_t)qi * a.H + h0) * kDim;
-        float m = 0.0f;
-        for (int i = pt; i < hcta * kDim / 8; i += 256) {
-            uint4 v = __ldg(reinterpret_cast<const uint4 *>(q) + i);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int j = 0; j < 8; ++j) {
+        const int i = threadIdx.x + kThreads * j;
+        qv[j] = (i / 64 < hcta) ? __ldg(reinterpret_cast<const uint4 *>(q) + i) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t w[4] = {qv[j].x, qv[j].y, qv[j].z, qv[j].w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu)),
-                                   fabsf(bf16_bits_to_f32(w[j] >> 16))));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-        if (lane == 0) s.qmax[warp - 8] = m;
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        float qm = 0.0f;
-        for (int w = 0; w < 8; ++w) qm = fmaxf(qm, s.qmax[w]);
-        const int e = qm > 0.0f ? max(0, ilogbf(qm) - 14) : 0;
-        const float inv = exp2f((float)-e);
-        for (int i = pt; i < kHeads * kDim / 8; i += 256) {
-            const int row = i / 64, ch = (i % 64) * 8;
-            uint4 o = make_uint4(0u, 0u, 0u, 0u);
-            if (row < hcta) {
-                uint4 v = __ldg(reinterpret_cast<const uint4 *>(q) + i);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                uint32_t h[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    h[j] = pack_h2(bf16_bits_to_f32(w[j] & 0xFFFFu) * inv,
-                                   bf16_bits_to_f32(w[j] >> 16) * inv);
-                o = make_uint4(h[0], h[1], h[2], h[3]);
-            }
-            *reinterpret_cast<uint4 *>(s.q + tile_off(row, ch)) = o;
-        }
-        if (threadIdx.x == 256) s.qmax[8] = (float)e;
-        fence_async_smem();
+        for (int k = 0; k < 4; ++k)
+            qm = fmaxf(qm, fmaxf(fabsf(bf16_bits_to_f32(w[k] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[k] >> 16))));
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) qm = fmaxf(qm, __shfl_xor_sync(0xFFFFFFFFu, qm, o));
+    if (lane == 0) {
+        s.wcnt[warp] = __popc(bal);
+        s.wred[warp] = qm;
+    }
+    __syncthreads();
+    int base = 0, n_sel = 0;
+    float qmax = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 16; ++w) {
+        base += w < warp ? s.wcnt[w] : 0;
+        n_sel += s.wcnt[w];
+        qmax = fmaxf(qmax, s.wred[w]);
+    }
+    if (e_ok) s.ids[base + __popc(bal & ((1u << lane) - 1u))] = e_id;
+    const int qexp = qmax > 0.0f ? max(0, ilogbf(qmax) - 14) : 0;   // max|q| * 2^-qexp < 2^15
+    {
+        const float inv = exp2f((float)-qexp);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = threadIdx.x + kThreads * j;
+            const uint32_t w[4] = {qv[j].x, qv[j].y, qv[j].z, qv[j].w};
+            uint32_t h[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                h[k] = pack_h2(bf16_bits_to_f32(w[k] & 0xFFFFu) * inv, bf16_bits_to_f32(w[k] >> 16) * inv);
+            *reinterpret_cast<uint4 *>(s.q + tile_off(i / 64, (i % 64) * 8)) = make_uint4(h[0], h[1], h[2], h[3]);
+        }
+    }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
-    const int n_sel = s.n_sel;
     const int n_keys = n_sel + n_win;
-    const int n_tiles = (n_keys + kTK - 1) / kTK;
+    const int n_all = (n_keys + kTK - 1) / kTK;            // tiles of the query
+    const int t_split = (n_all + 1) / 2;
+    const int tile_lo = rank == 0 ? 0 : t_split;
+    const int nt = (rank == 0 ? t_split : n_all) - tile_lo; // tiles of this CTA
     const uint32_t tmem = s.tmem_base;
     const uint32_t idesc_s = (1u << 4) | ((uint32_t)(kTK >> 3) << 17) | ((uint32_t)(kHeads >> 4) << 24);
     const uint32_t idesc_pv = (1u << 4) | (1u << 16) | (32u << 17) | ((uint32_t)(kHeads >> 4) << 24);
+    const int qd = warp & 3;
+    const int head = 16 * qd + (lane & 15);
+    const int half = lane >> 4;
+    float m_run = -INFINITY, l_run = 0.0f;
+    bool sm_ok = true;
 
     if (warp == 0) {
         // ---------------- MMA issuer ----------------
-        if (lane == 0 && n_tiles > 0) {
-            const uint32_t q_base = smem_u32(s.q);
-            const uint32_t p_base = smem_u32(s.p);
-            bool ok = true;
-            auto issue_s = [&](int i) {
-                const uint32_t kv = smem_u32(s.kv[i & 1]);
-                const uint32_t d = tmem + (16u << 16) + (uint32_t)(i & 1) * kTK;
-#pragma unroll
-                for (int kk = 0; kk < 32; ++kk) {
-                    const uint32_t off = (uint32_t)(kk >> 2) * 8192u + (uint32_t)(kk & 3) * 32u;
-                    mma_f16(d, sw128_desc(q_base + off, 16, 1024), sw128_desc(kv + off, 16, 1024),
-                            idesc_s, kk > 0);
-                }
-                mma_commit(&s.s_full[i & 1]);
-            };
-            ok = mbar_wait(&s.kv_full[0], 0);
-            if (ok) {
-                tc_fence_after();
-                issue_s(0);
-            }
-            for (int i = 0; ok && i < n_tiles; ++i) {
-                if (i + 1 < n_tiles) {
-                    ok = mbar_wait(&s.kv_full[(i + 1) & 1], ((i + 1) >> 1) & 1);
-                    if (!ok) break;
+        if (lane == 0 && nt > 0) {
+            const uint64_t qd0 = sw128_desc(smem_u32(s.q), 16, 1024);
+            const uint64_t pd0 = sw128_desc(smem_u32(s.p), 16, 1024);
+            const uint64_t kd0 = sw128_desc(smem_u32(s.kv[0]), 16, 1024);
+            const uint64_t kd1 = sw128_desc(smem_u32(s.kv[1]), 16, 1024);
+            const uint64_t vd0 = sw128_desc(smem_u32(s.kv[0]), 8192, 1024);
+            const uint64_t vd1 = sw128_desc(smem_u32(s.kv[1]), 8192, 1024);
+            int s_next = 0, pv_next = 0;
+            uint32_t idle = 0;
+            while (pv_next < nt && idle < (1u << 26)) {
+                bool progressed = false;
+                if (s_next < nt && s_next <= pv_next + 1 && mbar_test(&s.kv_full[s_next & 1], (s_next >> 1) & 1)) {
                     tc_fence_after();
-                    issue_s(i + 1);
+                    const uint32_t d = tmem + (16u << 16) + (uint32_t)(s_next & 1) * kTK;
+                    const uint64_t kb = (s_next & 1) ? kd1 : kd0;
+#pragma unroll
+                    for (int kk = 0; kk < 32; ++kk) {
+                        const uint64_t off = (uint64_t)((kk >> 2) * 512 + (kk & 3) * 2);  // 16-byte units
+                        mma_f16(d, qd0 + off, kb + off, idesc_s, kk > 0);
+                    }
+                    mma_commit(&s.s_full[s_next & 1]);
+                    ++s_next;
+                    progressed = true;
                 }
-                ok = mbar_wait(&s.p_full, i & 1);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t kv = smem_u32(s.kv[i & 1]);
+                if (pv_next < s_next && mbar_test(&s.p_full, pv_next & 1)) {
+                    tc_fence_after();
+                    const uint64_t vb = (pv_next & 1) ? vd1 : vd0;
 #pragma unroll
-                for (int nh = 0; nh < 2; ++nh)
+                    for (int nh = 0; nh < 2; ++nh)
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(tmem + 256u * nh, sw128_desc(p_base + 32u * ks, 16, 1024),
-                                sw128_desc(kv + 4u * 8192u * nh + 2048u * ks, 8192, 1024),
-                                idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
-                mma_commit(&s.kv_empty[i & 1]);
-                mma_commit(&s.pv_done);
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_f16(tmem + 256u * nh, pd0 + (uint64_t)(2 * ks),
+                                    vb + (uint64_t)(nh * 2048 + ks * 128), idesc_pv,
+                                    (pv_next > 0 || ks > 0) ? 1u : 0u);
+                    mma_commit(&s.kv_empty[pv_next & 1]);
+                    mma_commit(&s.pv_done);
+                    ++pv_next;
+                    progressed = true;
+                }
+                idle = progressed ? 0u : idle + 1u;
             }
-            if (!ok) {
+            if (pv_next < nt) {
                 atomicExch(&s.abort, 1);
                 set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
             }
-            // drain: every MMA issued so far has completed once this barrier flips
-            mma_commit(&s.drain);
+            mma_commit(&s.drain);          // completes once every MMA issued above has
             mbar_wait(&s.drain, 0);
         }
         __syncwarp();
     } else if (warp >= 4 && warp < 8) {
         // ---------------- softmax (TMEM quadrant warp % 4) ----------------
-        const int qd = warp & 3;
-        const int head = 16 * qd + (lane & 15);
-        const int half = lane >> 4;
-        const float c = a.softmax_scale * 1.4426950408889634f * exp2f(s.qmax[8]);
-        float m_run = -INFINITY, l_run = 0.0f;
-        bool ok = true;
+        const float c = a.softmax_scale * 1.4426950408889634f * exp2f((float)qexp);
         const uint32_t s_lane = tmem + ((uint32_t)(32 * qd + 16) << 16);
         const uint32_t o_lane = tmem + ((uint32_t)(32 * qd) << 16);
-        for (int i = 0; i < n_tiles; ++i) {
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.s_full[i & 1], (i >> 1) & 1) && !aborted(s));
+        bool ok = true;
+        for (int i = 0; i < nt; ++i) {
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.s_full[i & 1], (i >> 1) & 1) &&
+                                             mbar_wait(&s.kv_full[i & 1], (i >> 1) & 1) && !aborted(s));
             if (!ok) break;
             tc_fence_after();
-            // the stage's per-key scales: kv_full of this tile has completed (the
-            // MMA waited on it) and cannot advance before this warp releases P
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.kv_full[i & 1], (i >> 1) & 1));
-            if (!ok) break;
             float x[32], sg[32];
             tmem_ld16x32<32>(s_lane + (uint32_t)(i & 1) * kTK, x);
+            const int key0 = (tile_lo + i) * kTK + 32 * half;
             float mt = -INFINITY;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const int key = i * kTK + 32 * half + j;
                 sg[j] = s.sig[i & 1][32 * half + j];
-                x[j] = (key < n_keys && sg[j] > 0.0f) ? x[j] * (c * sg[j]) : -INFINITY;
+                x[j] = (key0 + j < n_keys && sg[j] > 0.0f) ? x[j] * (c * sg[j]) : -INFINITY;
                 mt = fmaxf(mt, x[j]);
             }
             mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, 16));
@@ -444,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
             if (i == 0) {
                 m_run = mt;
             } else if (mt > m_run + 8.0f) {
-                alpha = exp2f(m_run - mt);
+                alpha = ex2(m_run - mt);
                 m_run = mt;
                 l_run *= alpha;
             }
@@ -463,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
             uint32_t pk[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const float p0 = exp2f(x[2 * j] - m_run), p1 = exp2f(x[2 * j + 1] - m_run);
+                const float p0 = ex2(x[2 * j] - m_run), p1 = ex2(x[2 * j + 1] - m_run);
                 ps += p0 + p1;
                 pk[j] = pack_h2(p0 * sg[2 * j], p1 * sg[2 * j + 1]);   // V = code, so P carries sigma
             }
@@ -479,48 +521,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.p_full);
         }
-        if (ok && n_tiles > 0) {
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.pv_done, (n_tiles - 1) & 1) && !aborted(s));
+        if (ok && nt > 0) {
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.pv_done, (nt - 1) & 1) && !aborted(s));
             tc_fence_after();
         }
         if (!ok) {
             atomicExch(&s.abort, 1);
             set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
         }
-        const float l_tot = l_run + __shfl_xor_sync(0xFFFFFFFFu, l_run, 16);
-        const bool valid = ok && n_tiles > 0 && head < hcta && l_tot > 0.0f;
-        const float inv = valid ? 1.0f / l_tot : 0.0f;
-        float *orow = a.out + ((int64_t)qi * a.H + h0 + head) * kDim;
-        if (ok && n_tiles > 0) {
-#pragma unroll 1
-            for (int cc = 0; cc < 256; cc += 32) {
-                float o[32];
-                tmem_ld16x32<256>(o_lane + (uint32_t)cc, o);
-                if (head < hcta) {
-                    float4 *dst = reinterpret_cast<float4 *>(orow + 256 * half + cc);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        dst[j] = make_float4(o[4 * j] * inv, o[4 * j + 1] * inv,
-                                             o[4 * j + 2] * inv, o[4 * j + 3] * inv);
-                }
-            }
-        } else if (head < hcta) {
-            for (int cc = 0; cc < 256; ++cc) orow[256 * half + cc] = 0.0f;
+        sm_ok = ok;
+        l_run += __shfl_xor_sync(0xFFFFFFFFu, l_run, 16);
+        if (half == 0) {
+            s.cm[head] = (ok && nt > 0) ? m_run : -INFINITY;
+            s.cl[head] = (ok && nt > 0) ? l_run : 0.0f;
         }
-        if (half == 0 && head < hcta)
-            a.lse[(int64_t)qi * a.H + h0 + head] =
-                valid ? (m_run + log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
-        tc_fence_before();
     } else if (warp >= 8) {
         // ---------------- producers ----------------
         const int pt = threadIdx.x - 256;
         const int row = pt >> 2, quarter = pt & 3;
         Raw cur, nxt;
-        if (n_tiles > 0) load_raw(nxt, a, s, b, w0, n_keys, 0, row, quarter);
+        if (nt > 0) load_raw(nxt, a, s.ids, n_sel, b, w0, n_keys, tile_lo, row, quarter);
         bool ok = true;
-        for (int i = 0; i < n_tiles; ++i) {
+        for (int i = 0; i < nt; ++i) {
             cur = nxt;
-            if (i + 1 < n_tiles) load_raw(nxt, a, s, b, w0, n_keys, i + 1, row, quarter);
+            if (i + 1 < nt) load_raw(nxt, a, s.ids, n_sel, b, w0, n_keys, tile_lo + i + 1, row, quarter);
             if (i >= 2) {
                 ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.kv_empty[i & 1], ((i >> 1) - 1) & 1) && !aborted(s));
                 if (!ok) break;
@@ -538,6 +562,77 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(AttnArgs a) {
         }
     }
 
+    // ---- combine the two key halves of the query through distributed shared memory ----
+    // CTA r outputs channels [256 r, 256 r + 256); a softmax thread (head, half) holds
+    // O[head][256 half .. +256) of its CTA in TMEM.
+    tc_fence_before();
+    cluster_sync();                        // partial stats published; all MMAs of both CTAs done
+    tc_fence_after();
+    // Both CTAs derive the same weights; each softmax thread scales its half-row of
+    // O and stores it either into its own CTA's staging half (the channels this CTA
+    // writes) or into the peer's; then all threads add the two and write coalesced.
+    float *own = reinterpret_cast<float *>(s.kv[1]);       // [64 heads][256] this CTA's part
+    float *recv = reinterpret_cast<float *>(s.kv[0]);      // [64 heads][256] the peer's part
+    const bool smx = warp >= 4 && warp < 8;
+    if (smx) {
+        const uint32_t peer = rank ^ 1u;
+        const float m_self = s.cm[head], l_self = s.cl[head];
+        const float m_peer = ld_peer(peer_addr(&s.cm[head], peer));
+        const float l_peer = ld_peer(peer_addr(&s.cl[head], peer));
+        const float m_all = fmaxf(m_self, m_peer);
+        float f_self = 0.0f, f_peer = 0.0f;
+        if (m_all != -INFINITY) {
+            f_self = m_self == -INFINITY ? 0.0f : ex2(m_self - m_all);
+            f_peer = m_peer == -INFINITY ? 0.0f : ex2(m_peer - m_all);
+        }
+        const float l_all = l_self * f_self + l_peer * f_peer;
+        const bool valid = head < hcta && l_all > 0.0f;
+        const float w = valid ? f_self / l_all : 0.0f;
+        const uint32_t o_lane = tmem + ((uint32_t)(32 * qd) << 16);
+        const bool keep = (uint32_t)half == rank;
+        float *dst_own = own + head * 256;
+        const uint32_t dst_peer = peer_addr(recv + head * 256, peer);
+#pragma unroll 1
+        for (int cc = 0; cc < 256; cc += 32) {
+            float o[32];
+            if (nt > 0 && sm_ok) {
+                tmem_ld16x32<256>(o_lane + (uint32_t)cc, o);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) o[j] *= w;
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) o[j] = 0.0f;
+            }
+            if (keep) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    reinterpret_cast<float4 *>(dst_own + cc)[j] =
+                        make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    st_peer4(dst_peer + 4u * (cc + 4 * j), o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+            }
+        }
+        if (keep && rank == 0 && head < hcta)
+            a.lse[(int64_t)qi * a.H + h0 + head] =
+                valid ? (m_all + log2f(l_all)) * 0.6931471805599453f : -INFINITY;
+    }
+    cluster_sync();                        // the peer's part has landed in recv
+    {
+        const float4 *o4 = reinterpret_cast<const float4 *>(own);
+        const float4 *r4 = reinterpret_cast<const float4 *>(recv);
+        float *obase = a.out + ((int64_t)qi * a.H + h0) * kDim + 256 * rank;
+#pragma unroll 2
+        for (int i = threadIdx.x; i < kHeads * 64; i += kThreads) {
+            const int hh = i >> 6, c4 = i & 63;
+            if (hh < hcta) {
+                const float4 x = o4[i], y = r4[i];
+                reinterpret_cast<float4 *>(obase + (int64_t)hh * kDim)[c4] =
+                    make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w);
+            }
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -558,7 +653,7 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, int BT, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    dim3 grid(BT, (a.H + tc::kHeads - 1) / tc::kHeads);
+    dim3 grid(2 * BT, (a.H + tc::kHeads - 1) / tc::kHeads);   // 2-CTA clusters
     tc::attn_tc_kernel<<<grid, tc::kThreads, smem, st>>>(a);
     return cudaGetLastError();
 }

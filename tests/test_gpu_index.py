@@ -136,3 +136,35 @@ def test_device_bounds_flags(harness):
                            st.dev_err)
     assert pkg.csa2_read_device_error(st.dev_err) & pkg.DEVERR_INDEX
     assert st.count[L][0].item() == 0
+
+
+@pytest.mark.parametrize("qscale", [1.0, 300.0])
+def test_scores_wide_dynamic_range(harness, orc, qscale):
+    """Index-K rows whose magnitudes span about 40 binades (so the E4M3 codes reach
+    the subnormals and the top of the range) against a small and a large query:
+    the fp32 scores match the oracle's bit for bit."""
+    import fp4_kv_compressed_b200 as pkg
+    import synth
+    N, d, H_I = 3000, 128, 4
+    kv = pkg.GlobalKV(1, N, d, 1, "cuda")
+    g = torch.Generator().manual_seed(9)
+    mags = torch.exp2(torch.randint(-30, 12, (N, 1), generator=g).float())
+    rows = (synth.rows_normal_bf16(4, "k", 0, 0, N, d).float() * mags).to(torch.bfloat16)
+    z = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkg.csa2_quantize_append(kv.struct, None, rows.view(1, N, d).cuda(), N, z, None, None, 0, None)
+    q = (synth.rows_normal_bf16(5, "q", 0, 0, H_I, d).float() * qscale).to(torch.bfloat16)
+    q[1, 7] = -q[1, 7]
+    w = synth.rows_uniform_f32(6, "w", 0, 0, 1, H_I)
+    topk = torch.zeros(1, 1, 64, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(1, 1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(pkg.csa2_workspace_size(pkg.CSA2_OP_INDEX_FULL, 1, 1, N, 0, 64, 0),
+                     dtype=torch.uint8, device="cuda")
+    qpos = torch.tensor([[N - 1]], dtype=torch.int32, device="cuda")
+    pkg.csa2_index_full(kv.struct, q.view(1, 1, H_I, d).cuda(), w.view(1, 1, H_I).cuda(), qpos, 1,
+                        H_I, N, 0, 64, None, topk, cnt, ws)
+    torch.cuda.synchronize()
+    kc, ks = orc.quantize_fp8(rows)
+    ref = orc.scores(kc, ks, q, w[0].numpy(), n=N)
+    got = ws.view(torch.float32)[:N].cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    assert np.array_equal(topk[0, 0].cpu().numpy(), orc.select_topk(ref, 64))
