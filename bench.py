@@ -63,6 +63,79 @@ def op_bytes(wl) -> dict:
     return out
 
 
+def attn_flops(wl) -> int:
+    """Q K^T and P V over the selection and the window: 4 * H * 512 flop per key."""
+    n_win = min(wl.swa_len, wl.first_q_pos + 1)
+    return wl.B * wl.Tq * 4 * wl.H * 512 * (wl.top_k + n_win)
+
+
+# DRAM bytes (read + write) per launch from one ncu capture of each op's kernels:
+# (bytes, batch of the captured launch, kernel sources, sha256[:16] of those sources at
+# capture time).  Reported (scaled to the batch) only while the sources are unchanged.
+NCU_TRAFFIC = {
+    "csa2_sparse_attn_decode": (21_178_624, 64, ("csa2_attn.cu",), "c5d128b41c2558b3"),
+}
+
+
+def _sources_hash(files) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "fp4_kv_compressed_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    out = {"hbm_gbs": HBM_FALLBACK_GBS, "tflops": 1400.0, "source": "fallback (6.65 TB/s, 1.4 PF/s)"}
+    try:
+        mp = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        out = {"hbm_gbs": float(mp["hbm_gbs"]), "tflops": float(mp["bf16_tflops_sustained"]),
+               "source": "of measured (MEASURED_PEAKS.json: hbm_gbs; bf16_tflops_sustained, "
+                         "the kernels being timed inside a long step)"}
+    except Exception:
+        pass
+    return out
+
+
+def op_rooflines(wl, plan, op_ms: dict, ms_step: float) -> dict:
+    """Per timed op: algorithmic bytes (and flops) per launch over the live launch time."""
+    ob = op_bytes(wl)
+    pk = measured_peaks()
+    modes = [lp.mode for lp in plan]
+    dec = plan[[lp.layer for lp in plan if lp.mode == "F"][-1]].group
+    spec = {"csa2_index_full": (ob[f"index_full_g{dec}"], modes.count("F"),
+                                "index_scan_kernel + select_full_kernel"),
+            "csa2_index_reindex": (ob.get(f"index_reindex_g{dec}", 0), modes.count("X"),
+                                   "reindex_score_kernel + select_reindex_kernel"),
+            "csa2_sparse_attn_decode": (ob["attn"], len(modes), "attn_tc_kernel")}
+    out = {}
+    for name, ms in op_ms.items():
+        nbytes, n, kernels = spec[name]
+        if not nbytes or not n:
+            continue
+        gbs = nbytes / (ms / 1e3) / 1e9
+        traffic = None
+        if name in NCU_TRAFFIC:
+            tb, tbatch, files, sha = NCU_TRAFFIC[name]
+            if _sources_hash(files) == sha:
+                traffic = tb * wl.B / tbatch
+        e = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+             "frac": gbs / pk["hbm_gbs"], "traffic": traffic, "kernels": kernels,
+             "algorithmic_bytes_per_launch": nbytes, "launch_ms": ms, "launches_per_step": n,
+             "share_of_step": n * ms / ms_step, "peak_source": pk["source"]}
+        if name == "csa2_sparse_attn_decode":
+            fl = attn_flops(wl)
+            tfs = fl / (ms / 1e3) / 1e12
+            e["tensor"] = {"achieved": tfs, "peak": pk["tflops"], "unit": "TFLOP/s",
+                           "frac": tfs / pk["tflops"], "flops_per_launch": fl}
+            if fl / (pk["tflops"] * 1e12) > nbytes / (pk["hbm_gbs"] * 1e9):
+                e.update(bound="tensor", achieved=tfs, peak=pk["tflops"], unit="TFLOP/s",
+                         frac=tfs / pk["tflops"])
+        out[name] = e
+    return out
+
+
 def step_bytes(wl) -> int:
     ob = op_bytes(wl)
     total = 0
@@ -75,6 +148,31 @@ def step_bytes(wl) -> int:
             elif m == "X":
                 total += ob[f"index_reindex_g{g}"]
     return total
+
+
+# ------------------------------------------------------------------------------------------
+# ranks: disjoint requests per rank, time = max over ranks
+# ------------------------------------------------------------------------------------------
+def rank_workload(wl, rank: int):
+    """Rank r holds global requests r*B .. r*B + B - 1 (requests are independent: weak
+    scaling with no collective on the data path)."""
+    from synth.workloads import small_variant
+    return small_variant(wl, b0=wl.b0 + rank * wl.B, name=wl.name) if rank else wl
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, layers: int, ms_step: float) -> float:
+    """Whole-job layer-steps/s: every rank runs `layers` layer-steps per step."""
+    return world * layers / (ms_step / 1e3)
 
 
 # ------------------------------------------------------------------------------------------
@@ -253,6 +351,7 @@ def run_ours(args, rank, world, local_rank):
     if args.batch:
         from synth.workloads import small_variant
         wl = small_variant(wl, B=args.batch, name=f"{wl.name}_b{args.batch}")
+    wl = rank_workload(wl, rank)
     dw = csa2_harness.DeviceWorkload(wl, device=dev)
     st = dw.stack
     inputs, dbuf, hbuf, in_bytes = pack_inputs(dw.inputs, dev)
@@ -267,30 +366,47 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device error bits {st.dev_err.item()} in the warm-up step")
 
     S = max(1, min(10, args.steps))
-    ev = [(torch.cuda.Event(enable_timing=True, external=True),
-           torch.cuda.Event(enable_timing=True, external=True)) for _ in range(S)]
-    orig_full = None
-    import fp4_kv_compressed_b200 as pkg
-
-    # wrap csa2_index_full of the Full layer with timing events (graph capture only)
-    state = {"i": 0}
-
-    def timed_full(*a, **k):
-        i = state["i"]
-        ev[i % S][0].record()
-        orig_full(*a, **k)
-        ev[i % S][1].record()
-        state["i"] = i + 1
     import fp4_kv_compressed_b200.stack as stack_mod
-    orig_full = stack_mod.bind.csa2_index_full
+
+    # Timing events around one call per step of each op, recorded on the launching
+    # stream inside the timed graph: the Full op, the first Reindex op and the last
+    # layer's attention.
+    modes = [lp.mode for lp in st.plan]
+    picks = {"csa2_index_full": (modes.count("F"), 0),
+             "csa2_index_reindex": (modes.count("X"), 0),
+             "csa2_sparse_attn_decode": (len(modes), len(modes) - 1)}
+    op_events = {name: [] for name in picks}
+    originals = {name: getattr(stack_mod.bind, name) for name in picks}
+
+    def make_timed(name):
+        per_step, pick = picks[name]
+        orig = originals[name]
+        count = [0]
+
+        def f(*a, **k):
+            i = count[0]
+            count[0] += 1
+            if per_step and i % per_step == pick:
+                e0 = torch.cuda.Event(enable_timing=True, external=True)
+                e1 = torch.cuda.Event(enable_timing=True, external=True)
+                e0.record()
+                orig(*a, **k)
+                e1.record()
+                op_events[name].append((e0, e1))
+            else:
+                orig(*a, **k)
+        return f
+
     g = torch.cuda.CUDAGraph()
-    stack_mod.bind.csa2_index_full = timed_full
+    for name in picks:
+        setattr(stack_mod.bind, name, make_timed(name))
     try:
         with torch.cuda.graph(g, stream=stream):
             for _ in range(S):
                 st.step(**inputs)
     finally:
-        stack_mod.bind.csa2_index_full = orig_full
+        for name, orig in originals.items():
+            setattr(stack_mod.bind, name, orig)
     g1 = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g1, stream=stream):
         st.step(**inputs)
@@ -317,11 +433,9 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     ms = start.elapsed_time(end)
-    full_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    op_ms = {name: statistics.mean(a.elapsed_time(b) for a, b in evs)
+             for name, evs in op_events.items() if evs}
+    ms_max = max_over_ranks(ms, world, dev)
     if st.dev_err.item() != 0:
         raise RuntimeError(f"device error bits {st.dev_err.item()} in the timed steps")
 
@@ -356,28 +470,16 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te.item()) / Ke
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / Ke
 
     layers = len(st.plan)
     ms_step = ms_max / K
-    value = world * layers / (ms_step / 1e3)
+    value = job_value(world, layers, ms_step)
     sb = step_bytes(wl)
     ob = op_bytes(wl)
     g_full = st.plan[full_layers[0]].group
-    full_bytes = ob[f"index_full_g{g_full}"]
-    peak, peak_src = HBM_FALLBACK_GBS, "fallback 6.65 TB/s"
-    try:
-        mp = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
-        peak, peak_src = float(mp["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
-    except Exception:
-        pass
-    achieved = full_bytes / (full_ms / 1e3) / 1e9
-    traffic = None
-    if args.traffic_bytes:
-        traffic = args.traffic_bytes
+    ops = op_rooflines(wl, st.plan, op_ms, ms_step)
+    dominant = max(ops, key=lambda n: ops[n]["share_of_step"])
     launches = st.launches_per_step() * K
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -395,12 +497,9 @@ def run_ours(args, rank, world, local_rank):
                    "step_gbps": sb / (ms_step / 1e3) / 1e9,
                    "step_frac_of_8tbs": sb / (ms_step / 1e3) / 8e12,
                    "token_layer_steps_per_s": value * wl.B},
-        "roofline": {"bound": "hbm", "kernel": "csa2_index_full (Full scan + pool/Top-K select)",
-                     "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_source": peak_src,
-                     "traffic": traffic, "algorithmic_bytes_per_launch": full_bytes,
-                     "launch_ms": full_ms},
-        "e2e": ({"value": world * layers / (e2e_ms / 1e3), "unit": UNIT,
+        "roofline": dict(ops[dominant], op=dominant),
+        "roofline_ops": ops,
+        "e2e": ({"value": job_value(world, layers, e2e_ms), "unit": UNIT,
                  "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes,
                  "ms_per_step": e2e_ms} if Ke else None),
         "gpu_launches": launches,
@@ -446,8 +545,6 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (small cases for profiling)")
-    ap.add_argument("--traffic-bytes", type=float, default=None,
-                    help="ncu dram bytes per launch of the timed kernel, if captured")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

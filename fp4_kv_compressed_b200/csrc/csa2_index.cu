@@ -140,6 +140,14 @@ index_scan_kernel(IndexArgs a) {
     }
     cp_async_commit();
     load_query<D, HI>(s, a.q_idx + (int64_t)qi * HI * D, a.w + (int64_t)qi * HI);
+    // the rows' scales, fetched while the tile is in flight
+    const float *sig = a.idx_scale + (int64_t)b * a.cap;
+    float sgv[kRowsPerThread];
+#pragma unroll
+    for (int r = 0; r < kRowsPerThread; ++r) {
+        const int row = threadIdx.x + kScoreThreads * r;
+        sgv[r] = row < rows ? __ldg(sig + p0 + row) : 0.0f;
+    }
     cp_async_wait_all();
     __syncthreads();
 
@@ -147,14 +155,13 @@ index_scan_kernel(IndexArgs a) {
     score_rows<D, HI>(s, sc);
 
     float *scores = a.scores + (int64_t)qi * a.score_stride;
-    const float *sig = a.idx_scale + (int64_t)b * a.cap;
 #pragma unroll
     for (int r = 0; r < kRowsPerThread; ++r) {
         int row = threadIdx.x + kScoreThreads * r;
         int64_t p = p0 + row;
         float v = -INFINITY;
         if (row < rows) {
-            v = __fmul_rn(sc[r], sig[p]);
+            v = __fmul_rn(sc[r], sgv[r]);
             scores[p] = v;
         }
         if (a.bmax) {
@@ -186,8 +193,11 @@ reindex_score_kernel(IndexArgs a) {
     N = min64(N, a.cap);
     const int slot0 = blockIdx.x * (kTileRows / 8);
     const int32_t *pool = a.pool + (int64_t)qi * a.pool_blocks;
-
-    for (int r = threadIdx.x; r < kTileRows; r += kScoreThreads) {
+    const float *sig = a.idx_scale + (int64_t)b * a.cap;
+    float sgv[kRowsPerThread];   // row threadIdx.x + 128 i is handled by this thread below
+#pragma unroll
+    for (int i = 0; i < kRowsPerThread; ++i) {
+        const int r = threadIdx.x + kScoreThreads * i;
         int slot = slot0 + r / 8;
         int blk = slot < a.pool_blocks ? pool[slot] : -1;
         int64_t p = (int64_t)blk * 8 + (r & 7);
@@ -195,6 +205,7 @@ reindex_score_kernel(IndexArgs a) {
         if (blk >= 0 && (int64_t)blk * 8 >= N && (r & 7) == 0) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
         valid_row[r] = ok;
         pos_row[r] = ok ? (int)p : 0;
+        sgv[i] = ok ? __ldg(sig + p) : 0.0f;
     }
     __syncthreads();
     const uint8_t *base = a.idx_codes + (int64_t)b * a.cap * D;
@@ -211,154 +222,217 @@ reindex_score_kernel(IndexArgs a) {
 
     float sc[kRowsPerThread];
     score_rows<D, HI>(s, sc);
-    const float *sig = a.idx_scale + (int64_t)b * a.cap;
     float *out = a.scores + (int64_t)qi * a.score_stride + (int64_t)slot0 * 8;
 #pragma unroll
     for (int r = 0; r < kRowsPerThread; ++r) {
         int row = threadIdx.x + kScoreThreads * r;
         if (slot0 + row / 8 < a.pool_blocks)
-            out[row] = valid_row[row] ? __fmul_rn(sc[r], sig[pos_row[row]]) : 0.0f;
+            out[row] = valid_row[row] ? __fmul_rn(sc[r], sgv[r]) : 0.0f;
     }
 }
 
 // ------------------------------------------------------------------------------
 // Block-wide Top-K selection (one CTA per query).
-// Radix select over 32-bit order keys, most significant byte first, then a
-// compaction in index order: every key above the threshold, plus the
-// lowest-indexed keys equal to it.  Candidate index order == position order.
+// Keys are 32-bit order keys (0 = not a candidate).  Radix select, most significant
+// digit first, over the bits where the valid keys differ: the digits start at the
+// highest bit in which the smallest and largest valid keys differ (scores share
+// their sign and most exponent bits, which would otherwise pile every key into a
+// few bins), 11 bits per pass, stopping as soon as the remaining demand equals
+// the population of the chosen bin.  The result is a masked threshold (T, mask)
+// and a count `take`: selected = every key whose masked value exceeds T, plus
+// the `take` lowest-indexed keys whose masked value equals T.  A compaction over
+// per-warp contiguous segments then writes the selected ids in index order.
 // ------------------------------------------------------------------------------
 constexpr int kSelThreads = 1024;
+constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelStageMax = 16384;   // keys staged in shared memory up to this count
+constexpr int kSelDigit = 11;         // bits per radix pass
 
 struct SelSmem {
-    uint32_t hist[256];
-    int warp_tot[32];
+    uint32_t hist[1 << kSelDigit];
+    int wa[kSelWarps], wb[kSelWarps];
+    uint32_t wmin[kSelWarps], wmax[kSelWarps];
     int bcast[4];
     int pool[CSA2_POOL_MAX];
     uint32_t keys[kSelStageMax];
 };
 
-__device__ __forceinline__ int block_excl_scan(bool flag, int &total, SelSmem &s) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t bal = __ballot_sync(0xFFFFFFFFu, flag);
-    int excl = __popc(bal & ((1u << lane) - 1u));
-    if (lane == 0) s.warp_tot[warp] = __popc(bal);
-    __syncthreads();
-    if (warp == 0) {
-        int v = s.warp_tot[lane];
-        int incl = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-            if (lane >= o) incl += t;
-        }
-        s.warp_tot[lane] = incl - v;
-        if (lane == 31) s.bcast[3] = incl;
-    }
-    __syncthreads();
-    int r = s.warp_tot[warp] + excl;
-    total = s.bcast[3];
-    __syncthreads();
-    return r;
-}
-
-// Threshold key T and the number of keys equal to T to take, so that
-// #(key > T) + take == k.  Keys equal to 0 are never candidates.  1 <= k <= #valid.
-template <class KeyAt>
-__device__ void radix_threshold(KeyAt key_at, int n, int k, SelSmem &s, uint32_t &T, int &take) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t prefix = 0;
-    int rem = k;
-#pragma unroll 1
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) s.hist[i] = 0;
-        __syncthreads();
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            uint32_t key = key_at(i);
-            bool match = key != 0u && (pass == 0 || ((key ^ prefix) >> (shift + 8)) == 0u);
-            if (match) {
-                uint32_t bin = (key >> shift) & 255u;
-                uint32_t peers = __match_any_sync(__activemask(), bin);
-                if (lane == __ffs(peers) - 1) atomicAdd(&s.hist[bin], (uint32_t)__popc(peers));
-            }
-        }
-        __syncthreads();
-        if (warp == 0) {
-            // lane l owns bins 255-8l .. 248-8l, visited in descending order
-            uint32_t c[8], sum = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) { c[i] = s.hist[255 - 8 * lane - i]; sum += c[i]; }
-            uint32_t incl = sum;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-                if (lane >= o) incl += t;
-            }
-            uint32_t run = incl - sum;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                if (run < (uint32_t)rem && (uint32_t)rem <= run + c[i]) {
-                    s.bcast[0] = 255 - 8 * lane - i;
-                    s.bcast[1] = (int)run;
-                }
-                run += c[i];
-            }
-        }
-        __syncthreads();
-        prefix |= (uint32_t)s.bcast[0] << shift;
-        rem -= s.bcast[1];
-        __syncthreads();
-    }
-    T = prefix;
-    take = rem;
-}
-
-// Writes the selected candidates' ids, ascending, to out[0..k); returns k.
-template <class KeyAt, class IdAt>
-__device__ int compact_selected(KeyAt key_at, IdAt id_at, int n, uint32_t T, int take,
-                                int *out, int max_out, SelSmem &s) {
-    int base_sel = 0, base_eq = 0;
-    for (int start = 0; start < n; start += blockDim.x) {
-        int i = start + threadIdx.x;
-        uint32_t key = i < n ? key_at(i) : 0u;
-        bool eq = key != 0u && key == T;
-        int eq_tot;
-        int eq_rank = block_excl_scan(eq, eq_tot, s);
-        bool sel = key > T || (eq && base_eq + eq_rank < take);
-        int sel_tot;
-        int sel_rank = block_excl_scan(sel, sel_tot, s);
-        if (sel && base_sel + sel_rank < max_out) out[base_sel + sel_rank] = id_at(i);
-        base_sel += sel_tot;
-        base_eq += eq_tot;
-    }
-    return min(base_sel, max_out);
-}
-
-// Top-k of n candidates (keys from key_at, 0 = not a candidate) -> ascending ids
-// in out[0..cnt), cnt = min(k, #valid) returned.
-template <class KeyAt, class IdAt>
-__device__ int block_topk(KeyAt key_at, IdAt id_at, int n, int k, int *out, SelSmem &s) {
-    // number of valid candidates
-    int local = 0;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) local += key_at(i) != 0u;
-    local = __reduce_add_sync(0xFFFFFFFFu, local);
-    if ((threadIdx.x & 31) == 0) s.warp_tot[threadIdx.x >> 5] = local;
+// Exclusive scans (in warp order) of s.wa and s.wb; totals in s.bcast[0], s.bcast[1].
+// Call with every warp's entry written; ends with a barrier.
+__device__ __forceinline__ void sel_scan_warps(SelSmem &s) {
     __syncthreads();
     if (threadIdx.x < 32) {
-        int v = (threadIdx.x < (blockDim.x >> 5)) ? s.warp_tot[threadIdx.x] : 0;
-        v = __reduce_add_sync(0xFFFFFFFFu, v);
-        if (threadIdx.x == 0) s.bcast[2] = v;
+        const int lane = threadIdx.x;
+        const int a = s.wa[lane], b = s.wb[lane];
+        int ia = a, ib = b;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int ta = __shfl_up_sync(0xFFFFFFFFu, ia, o), tb = __shfl_up_sync(0xFFFFFFFFu, ib, o);
+            if (lane >= o) { ia += ta; ib += tb; }
+        }
+        s.wa[lane] = ia - a;
+        s.wb[lane] = ib - b;
+        if (lane == 31) { s.bcast[0] = ia; s.bcast[1] = ib; }
     }
     __syncthreads();
-    const int nvalid = s.bcast[2];
+}
+
+// The bin (of nbins, visited from the top) holding the rem-th largest counted key:
+// bin, number of counted keys in higher bins, population of the bin.
+__device__ __forceinline__ void sel_find_bin(SelSmem &s, int nbins, int rem, int &bin, int &above,
+                                             int &cnt) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int per = (nbins + kSelThreads - 1) / kSelThreads;   // 1 or 2 bins per thread
+    int c[2] = {0, 0}, sum = 0;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int bb = nbins - 1 - (threadIdx.x * per + j);
+        if (j < per && bb >= 0) c[j] = (int)s.hist[bb];
+        sum += c[j];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) s.wa[warp] = incl;
+    s.wb[warp] = 0;
+    sel_scan_warps(s);
+    int run = s.wa[warp] + incl - sum;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        if (c[j] > 0 && run < rem && rem <= run + c[j]) {
+            s.bcast[2] = nbins - 1 - (threadIdx.x * per + j);
+            s.bcast[3] = run;
+            s.wmin[0] = (uint32_t)c[j];
+        }
+        run += c[j];
+    }
+    __syncthreads();
+    bin = s.bcast[2];
+    above = s.bcast[3];
+    cnt = (int)s.wmin[0];
+    __syncthreads();
+}
+
+// Top-k of n candidates (keys from key_at, 0 = not a candidate) -> ascending ids in
+// out[0..cnt), cnt = min(k, #valid) returned.
+template <class KeyAt, class IdAt>
+__device__ int block_topk(KeyAt key_at, IdAt id_at, int n, int k, int *out, SelSmem &s) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // valid count, smallest and largest valid key
+    int nv = 0;
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int i = threadIdx.x; i < n; i += kSelThreads) {
+        const uint32_t key = key_at(i);
+        if (key != 0u) {
+            ++nv;
+            kmin = min(kmin, key);
+            kmax = max(kmax, key);
+        }
+    }
+    nv = __reduce_add_sync(0xFFFFFFFFu, nv);
+    kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
+    kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+    if (lane == 0) {
+        s.wa[warp] = nv;
+        s.wmin[warp] = kmin;
+        s.wmax[warp] = kmax;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int v = __reduce_add_sync(0xFFFFFFFFu, s.wa[lane]);
+        const uint32_t mn = __reduce_min_sync(0xFFFFFFFFu, s.wmin[lane]);
+        const uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, s.wmax[lane]);
+        if (lane == 0) {
+            s.bcast[0] = v;
+            s.bcast[1] = (int)mn;
+            s.bcast[2] = (int)mx;
+        }
+    }
+    __syncthreads();
+    const int nvalid = s.bcast[0];
+    kmin = (uint32_t)s.bcast[1];
+    kmax = (uint32_t)s.bcast[2];
     __syncthreads();
     const int kk = min(k, nvalid);
     if (kk == 0) return 0;
-    uint32_t T;
+
+    // ---- threshold ----
+    uint32_t T, mask;
     int take;
-    radix_threshold(key_at, n, kk, s, T, take);
-    return compact_selected(key_at, id_at, n, T, take, out, kk, s);
+    if (kk == nvalid) {                 // everything valid is selected
+        T = 0u;
+        mask = 0u;
+        take = kk;
+    } else if (kmin == kmax) {          // all valid keys equal: the first kk in index order
+        T = kmax;
+        mask = 0xFFFFFFFFu;
+        take = kk;
+    } else {
+        const int hi = 31 - __clz(kmin ^ kmax);
+        uint32_t pmask = ~((2u << hi) - 1u);      // bits above hi are common to every valid key
+        uint32_t prefix = kmax & pmask;
+        int rem = kk, lo_bit = hi + 1;
+        while (lo_bit > 0) {
+            const int bits = min(kSelDigit, lo_bit), shift = lo_bit - bits, nbins = 1 << bits;
+            for (int i = threadIdx.x; i < nbins; i += kSelThreads) s.hist[i] = 0u;
+            __syncthreads();
+            for (int i = threadIdx.x; i < n; i += kSelThreads) {
+                const uint32_t key = key_at(i);
+                if (key != 0u && (key & pmask) == prefix)
+                    atomicAdd(&s.hist[(key >> shift) & (uint32_t)(nbins - 1)], 1u);
+            }
+            __syncthreads();
+            int bin, above, cnt;
+            sel_find_bin(s, nbins, rem, bin, above, cnt);
+            prefix |= (uint32_t)bin << shift;
+            pmask |= (uint32_t)(nbins - 1) << shift;
+            rem -= above;
+            lo_bit = shift;
+            if (cnt == rem) break;            // the whole bin is taken
+        }
+        T = prefix;
+        mask = pmask;
+        take = rem;
+    }
+
+    // ---- compaction in index order: warp w owns keys [w*seg, (w+1)*seg) ----
+    const int seg = ((n + kSelThreads - 1) / kSelThreads) * 32;
+    const int lo = warp * seg, hi_i = min(n, lo + seg);
+    int ngt = 0, neq = 0;
+    for (int i0 = lo; i0 < hi_i; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t key = i < hi_i ? key_at(i) : 0u;
+        const uint32_t km = key & mask;
+        ngt += __popc(__ballot_sync(0xFFFFFFFFu, key != 0u && km > T));
+        neq += __popc(__ballot_sync(0xFFFFFFFFu, key != 0u && km == T));
+    }
+    if (lane == 0) {
+        s.wa[warp] = ngt;
+        s.wb[warp] = neq;
+    }
+    sel_scan_warps(s);
+    int gt_run = s.wa[warp], eq_run = s.wb[warp];
+    const int total = s.bcast[0] + min(take, s.bcast[1]);
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int i0 = lo; i0 < hi_i; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t key = i < hi_i ? key_at(i) : 0u;
+        const uint32_t km = key & mask;
+        const bool gt = key != 0u && km > T, eq = key != 0u && km == T;
+        const uint32_t bgt = __ballot_sync(0xFFFFFFFFu, gt), beq = __ballot_sync(0xFFFFFFFFu, eq);
+        const int gt_before = gt_run + __popc(bgt & lt), eq_before = eq_run + __popc(beq & lt);
+        if (gt || (eq && eq_before < take)) {
+            const int r = gt_before + min(take, eq_before);
+            if (r < kk) out[r] = id_at(i);
+        }
+        gt_run += __popc(bgt);
+        eq_run += __popc(beq);
+    }
+    __syncthreads();
+    return min(total, kk);
 }
 
 // a4 + a5: one CTA per query.  Hierarchical: pool from block maxima, then Top-K

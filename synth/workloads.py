@@ -49,6 +49,7 @@ class Workload:
     chan_scale: bool = False  # per-channel log-uniform [0.25, 4] scale on main KV and SWA
     planted: int = 0          # planted high-score index positions per request
     description: str = ""
+    b0: int = 0               # global index of request 0 (ranks hold disjoint requests)
 
     # ---- derived shapes -------------------------------------------------------------------
     @property
@@ -97,12 +98,13 @@ class Workload:
 
     def main_kv(self, g: int, b: int, start: int, count: int, device="cpu") -> torch.Tensor:
         """bf16 [count][512] post-RoPE main KV entries of group g, request b."""
-        x = rows_normal_bf16(self.seed, f"g{g}.kv", b, start, count, KV_DIM, device)
+        x = rows_normal_bf16(self.seed, f"g{g}.kv", self.b0 + b, start, count, KV_DIM, device)
         return self._apply_scale(x)
 
     def idx_k(self, g: int, b: int, start: int, count: int, device="cpu") -> torch.Tensor:
         """bf16 [count][d_I] indexer-K rows of group g, request b (planted rows included)."""
-        x = rows_normal_bf16(self.seed, f"g{g}.idxk", b, start, count, self.d_I, device)
+        x = rows_normal_bf16(self.seed, f"g{g}.idxk", self.b0 + b, start, count, self.d_I,
+                             device)
         if self.planted and g == self.decoder_group:
             pos, rows = self.planted_rows(b)
             for p, r in zip(pos, rows):
@@ -112,24 +114,25 @@ class Workload:
 
     def swa(self, layer: int, b: int, start: int, count: int, device="cpu") -> torch.Tensor:
         """bf16 [count][512] SWA rows of one layer for token positions [start, start+count)."""
-        x = rows_normal_bf16(self.seed, f"L{layer}.swa", b, start, count, KV_DIM, device)
+        x = rows_normal_bf16(self.seed, f"L{layer}.swa", self.b0 + b, start, count, KV_DIM,
+                             device)
         return self._apply_scale(x)
 
     def q(self, layer: int, b: int, device="cpu") -> torch.Tensor:
         """bf16 [Tq][H][512] attention queries of one layer."""
-        x = rows_normal_bf16(self.seed, f"L{layer}.q", b, 0, self.Tq * self.H, KV_DIM, device,
-                             stride=Q_STRIDE)
+        x = rows_normal_bf16(self.seed, f"L{layer}.q", self.b0 + b, 0, self.Tq * self.H, KV_DIM,
+                             device, stride=Q_STRIDE)
         return x.view(self.Tq, self.H, KV_DIM)
 
     def q_idx(self, layer: int, b: int, device="cpu") -> torch.Tensor:
         """bf16 [Tq][H_I][d_I] index queries of one layer."""
-        x = rows_normal_bf16(self.seed, f"L{layer}.qidx", b, 0, self.Tq * self.H_I, self.d_I,
-                             device, stride=Q_STRIDE)
+        x = rows_normal_bf16(self.seed, f"L{layer}.qidx", self.b0 + b, 0, self.Tq * self.H_I,
+                             self.d_I, device, stride=Q_STRIDE)
         return x.view(self.Tq, self.H_I, self.d_I)
 
     def w(self, layer: int, b: int, device="cpu") -> torch.Tensor:
         """fp32 [Tq][H_I] index-head weights, U(0,1)."""
-        x = rows_uniform_f32(self.seed, f"L{layer}.w", b, 0, self.Tq, self.H_I, device)
+        x = rows_uniform_f32(self.seed, f"L{layer}.w", self.b0 + b, 0, self.Tq, self.H_I, device)
         return x.view(self.Tq, self.H_I)
 
     # ---- structure ------------------------------------------------------------------------
@@ -156,7 +159,8 @@ class Workload:
         pos: list[int] = []
         j = 0
         while len(pos) < self.planted:
-            h = int(hash_u32(torch.tensor([b * 4096 + j], dtype=torch.int64), keys)[0])
+            h = int(hash_u32(torch.tensor([(self.b0 + b) * 4096 + j], dtype=torch.int64),
+                             keys)[0])
             p = h % n
             if p not in pos:
                 pos.append(p)
@@ -198,9 +202,13 @@ WORKLOADS = {
 }
 
 
-def small_variant(w: Workload, *, B=None, ctx=None, H=None, Tq=None, name=None) -> Workload:
-    """A reduced copy of a workload (same structure and seeds) for oracle-sized tests."""
+def small_variant(w: Workload, *, B=None, ctx=None, H=None, Tq=None, name=None,
+                  b0=None) -> Workload:
+    """A reduced copy of a workload (same structure and seeds) for oracle-sized tests;
+    b0 selects which global requests the copy holds."""
     d = dict(w.__dict__)
+    if b0 is not None:
+        d["b0"] = b0
     if B is not None:
         d["B"] = B
     if ctx is not None:
@@ -215,9 +223,10 @@ def small_variant(w: Workload, *, B=None, ctx=None, H=None, Tq=None, name=None) 
 
 # ---- batched row generation (all requests at once, same bits as the per-request calls) ----
 def batch_rows_normal_bf16(seed: int, name: str, B: int, start: int, count: int, width: int,
-                           device="cpu", stride: int = POS_STRIDE) -> torch.Tensor:
-    """[B][count][width] bf16; row (b, start+i) equals rows_normal_bf16(..., b, start, ...)[i]."""
-    b = torch.arange(B, dtype=torch.int64, device=device).view(B, 1, 1)
+                           device="cpu", stride: int = POS_STRIDE, b0: int = 0) -> torch.Tensor:
+    """[B][count][width] bf16; row (b, start+i) equals rows_normal_bf16(..., b0 + b, start,
+    ...)[i]."""
+    b = (b0 + torch.arange(B, dtype=torch.int64, device=device)).view(B, 1, 1)
     p = (start + torch.arange(count, dtype=torch.int64, device=device)).view(1, count, 1)
     c = torch.arange(width, dtype=torch.int64, device=device).view(1, 1, width)
     idx = (b * stride + p) * width + c
@@ -225,12 +234,14 @@ def batch_rows_normal_bf16(seed: int, name: str, B: int, start: int, count: int,
 
 
 def _main_kv_batch(self: Workload, g: int, start: int, count: int, device="cpu"):
-    x = batch_rows_normal_bf16(self.seed, f"g{g}.kv", self.B, start, count, KV_DIM, device)
+    x = batch_rows_normal_bf16(self.seed, f"g{g}.kv", self.B, start, count, KV_DIM, device,
+                               b0=self.b0)
     return self._apply_scale(x)
 
 
 def _idx_k_batch(self: Workload, g: int, start: int, count: int, device="cpu"):
-    x = batch_rows_normal_bf16(self.seed, f"g{g}.idxk", self.B, start, count, self.d_I, device)
+    x = batch_rows_normal_bf16(self.seed, f"g{g}.idxk", self.B, start, count, self.d_I, device,
+                               b0=self.b0)
     if self.planted and g == self.decoder_group:
         for b in range(self.B):
             pos, rows = self.planted_rows(b)
@@ -241,25 +252,26 @@ def _idx_k_batch(self: Workload, g: int, start: int, count: int, device="cpu"):
 
 
 def _swa_batch(self: Workload, layer: int, start: int, count: int, device="cpu"):
-    x = batch_rows_normal_bf16(self.seed, f"L{layer}.swa", self.B, start, count, KV_DIM, device)
+    x = batch_rows_normal_bf16(self.seed, f"L{layer}.swa", self.B, start, count, KV_DIM, device,
+                               b0=self.b0)
     return self._apply_scale(x)
 
 
 def _q_batch(self: Workload, layer: int, device="cpu"):
     x = batch_rows_normal_bf16(self.seed, f"L{layer}.q", self.B, 0, self.Tq * self.H, KV_DIM,
-                               device, stride=Q_STRIDE)
+                               device, stride=Q_STRIDE, b0=self.b0)
     return x.view(self.B, self.Tq, self.H, KV_DIM)
 
 
 def _q_idx_batch(self: Workload, layer: int, device="cpu"):
     x = batch_rows_normal_bf16(self.seed, f"L{layer}.qidx", self.B, 0, self.Tq * self.H_I,
-                               self.d_I, device, stride=Q_STRIDE)
+                               self.d_I, device, stride=Q_STRIDE, b0=self.b0)
     return x.view(self.B, self.Tq, self.H_I, self.d_I)
 
 
 def _w_batch(self: Workload, layer: int, device="cpu"):
     from . import uniform_f32
-    b = torch.arange(self.B, dtype=torch.int64, device=device).view(self.B, 1, 1)
+    b = (self.b0 + torch.arange(self.B, dtype=torch.int64, device=device)).view(self.B, 1, 1)
     r = torch.arange(self.Tq, dtype=torch.int64, device=device).view(1, self.Tq, 1)
     c = torch.arange(self.H_I, dtype=torch.int64, device=device).view(1, 1, self.H_I)
     idx = (b * Q_STRIDE + r) * self.H_I + c

@@ -68,39 +68,48 @@ def swa_ring(wl: Workload, layer: int, b: int):
     return codes, scale
 
 
-def index_layers(wl: Workload, b: int, caches, q_pos: np.ndarray | None = None):
-    """Pool / Top-K / count of every Full and Reindex layer of request b."""
+def index_layers(wl: Workload, b: int, caches, q_pos: np.ndarray | None = None,
+                 qsel: np.ndarray | None = None):
+    """Pool / Top-K / count of every Full and Reindex layer of request b (of the query
+    tokens qsel only, when given: queries are independent given the caches)."""
     q_pos = np.asarray(wl.q_positions() if q_pos is None else q_pos, np.int32)
+    sel = slice(None) if qsel is None else np.asarray(qsel)
+    q_pos = np.ascontiguousarray(q_pos[sel])
     res = {"topk": {}, "count": {}, "pool": {}}
     pool = {}
     for layer, (g, m, src) in enumerate(reuse_sources(wl)):
         grp = wl.groups[g]
         c = caches[g]
+        if m in "FX":
+            qi = wl.q_idx(layer, b)[sel].contiguous()
+            w = np.ascontiguousarray(wl.w(layer, b)[sel].numpy())
         if m == "F":
             p, t, n = orc.index_full(c["idx_codes"][None], c["idx_scale"][None], grp.ratio,
-                                     wl.q_idx(layer, b)[None], wl.w(layer, b)[None].numpy(),
-                                     q_pos[None], grp.pool_blocks, wl.top_k)
+                                     qi[None], w[None], q_pos[None], grp.pool_blocks, wl.top_k)
             if p is not None:
                 pool[g] = p
                 res["pool"][g] = p[0]
             res["topk"][layer], res["count"][layer] = t[0], n[0]
         elif m == "X":
             t, n = orc.index_reindex(c["idx_codes"][None], c["idx_scale"][None], grp.ratio,
-                                     wl.q_idx(layer, b)[None], wl.w(layer, b)[None].numpy(),
-                                     q_pos[None], pool[g], wl.top_k)
+                                     qi[None], w[None], q_pos[None], pool[g], wl.top_k)
             res["topk"][layer], res["count"][layer] = t[0], n[0]
     return res
 
 
 def attention_layer(wl: Workload, b: int, layer: int, caches, topk: np.ndarray,
-                    q_pos: np.ndarray | None = None):
+                    q_pos: np.ndarray | None = None, qsel: np.ndarray | None = None):
+    """Attention of one layer for request b (query tokens qsel only, when given; topk
+    then holds those queries' selections)."""
     q_pos = np.asarray(wl.q_positions() if q_pos is None else q_pos, np.int32)
+    sel = slice(None) if qsel is None else np.asarray(qsel)
+    q_pos = np.ascontiguousarray(q_pos[sel])
     g = reuse_sources(wl)[layer][0]
     c = caches[g]
     ring_c, ring_s = swa_ring(wl, layer, b)
     o, lse = orc.attention(c["codes"][None], c["scales"][None], ring_c[None], ring_s[None],
-                           wl.q(layer, b)[None], q_pos[None], topk[None], wl.swa_len,
-                           SOFTMAX_SCALE)
+                           wl.q(layer, b)[sel].contiguous()[None], q_pos[None],
+                           np.ascontiguousarray(topk)[None], wl.swa_len, SOFTMAX_SCALE)
     return o[0], lse[0]
 
 

@@ -1,0 +1,116 @@
+"""Host-side logic of bench.py: the multi-rank path on two gloo ranks (CPU), the
+algorithmic byte counts, and the reference arm's output line."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from synth.workloads import WORKLOADS  # noqa: E402
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        ms = bench.max_over_ranks(10.0 + 5.0 * rank, world, "cpu")
+        wl = bench.rank_workload(WORKLOADS["decode_128k"], rank)
+        first = wl.q_idx_batch(0)[0, 0, 0, :8].view(torch.int16).tolist()
+        out.put((rank, ms, wl.b0, wl.B, wl.name, first,
+                 bench.job_value(world, len(wl.layers), ms)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_max_time_and_disjoint_requests():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, ms0, b00, B0, n0, f0, v0), (r1, ms1, b01, B1, n1, f1, v1) = res
+    assert ms0 == ms1 == 15.0                  # both ranks time the slowest rank
+    assert (b00, b01) == (0, 64) and B0 == B1 == 64 and n0 == n1 == "decode_128k"
+    # rank 1's first request is global request 64, not a copy of rank 0's
+    ref = WORKLOADS["decode_128k"]
+    assert f1 == ref.q_idx(0, 64)[0, 0, :8].view(torch.int16).tolist()
+    assert f0 != f1
+    assert v0 == v1 == 2 * 20 / 0.015          # whole-job layer-steps/s
+
+
+def test_algorithmic_bytes_at_128k():
+    """Per-unit costs: 132 B of indexer K + 4 B score written + 4 B read back + block
+    max per visible position; 288 B per selected entry and 516 B per window row."""
+    wl = WORKLOADS["decode_128k"]
+    ob = bench.op_bytes(wl)
+    N, B = 131072, 64
+    nb = N // 8
+    per_q = (N * 132 + 4 * N + 4 * nb + 4 * nb + 8 * 2048 * 4 + 4 * 2048 + 4 * 512 + 4
+             + 4 * 128 * 2 + 4 * 4)
+    assert ob["index_full_g0"] == B * per_q == 1_154_155_776
+    attn = 512 * 288 + 512 * 4 + 128 * 516 + 64 * 512 * 2 + 64 * 512 * 4 + 64 * 4
+    assert ob["attn"] == B * attn
+    assert bench.step_bytes(wl) == 2_274_219_520
+
+
+def test_reference_arm_line():
+    """`--impl reference` times the CPU oracle and prints one line with impl=reference."""
+    env = dict(os.environ, OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny_full_layer", "--steps", "1", "--warmup", "1"],
+                       capture_output=True, text=True, timeout=600, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["unit"] == bench.UNIT
+
+
+def test_reference_arm_other_ranks_do_nothing():
+    class A:
+        workload = "decode_128k"
+        steps = 1
+    assert bench.run_reference(A(), 1, 2) is None
+
+
+def test_op_rooflines_dominant_and_traffic():
+    """Per-op roofline entries: bytes / live time, share of the step, ncu traffic only
+    while the captured kernel's sources are unchanged, dominant op by share."""
+    from fp4_kv_compressed_b200.stack import plan_layers
+    wl = WORKLOADS["decode_128k"]
+    plan = plan_layers([g.schedule for g in wl.groups])
+    op_ms = {"csa2_index_full": 0.4, "csa2_index_reindex": 0.1, "csa2_sparse_attn_decode": 0.03}
+    ops = bench.op_rooflines(wl, plan, op_ms, ms_step=1.5)
+    f = ops["csa2_index_full"]
+    assert f["launches_per_step"] == 1 and f["bound"] == "hbm"
+    assert abs(f["achieved"] - 1_154_155_776 / 0.4e-3 / 1e9) < 1e-6
+    assert abs(f["share_of_step"] - 0.4 / 1.5) < 1e-12
+    a = ops["csa2_sparse_attn_decode"]
+    assert a["launches_per_step"] == 20 and abs(a["share_of_step"] - 0.4) < 1e-12
+    assert a["tensor"]["flops_per_launch"] == 64 * 4 * 64 * 512 * 640
+    assert ops["csa2_index_reindex"]["launches_per_step"] == 4
+    tb, tbatch, files, sha = bench.NCU_TRAFFIC["csa2_sparse_attn_decode"]
+    expect = tb * wl.B / tbatch if bench._sources_hash(files) == sha else None
+    assert a["traffic"] == expect
+    assert max(ops, key=lambda n: ops[n]["share_of_step"]) == "csa2_sparse_attn_decode"

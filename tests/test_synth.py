@@ -39,3 +39,20 @@ def test_workload_shapes():
     assert w3.window_cap >= 128 + 2048 - 1
     s = w4._scale("cpu")
     assert float(s.min()) >= 0.25 and float(s.max()) <= 4.0
+
+
+def test_request_offset_selects_global_requests():
+    """A workload copy with b0 = k holds global requests k.. : its batch rows, per-request
+    rows and planted rows equal those of the first workload's requests k.."""
+    from synth.workloads import WORKLOADS, small_variant
+    base = small_variant(WORKLOADS["decoder_group_32k"], B=4, ctx=2000)
+    part = small_variant(base, B=2, b0=2)
+    assert torch.equal(part.main_kv_batch(0, 10, 3), base.main_kv_batch(0, 10, 3)[2:])
+    assert torch.equal(part.idx_k_batch(0, 0, 2000), base.idx_k_batch(0, 0, 2000)[2:])
+    assert torch.equal(part.q_batch(4), base.q_batch(4)[2:])
+    assert torch.equal(part.q_idx_batch(0), base.q_idx_batch(0)[2:])
+    assert torch.equal(part.w_batch(4), base.w_batch(4)[2:])
+    assert torch.equal(part.swa_batch(7, 5, 4), base.swa_batch(7, 5, 4)[2:])
+    assert torch.equal(part.idx_k(0, 1, 0, 2000), base.idx_k(0, 3, 0, 2000))
+    assert part.planted_rows(1)[0] == base.planted_rows(3)[0]
+    assert part.planted_rows(0)[0] != base.planted_rows(0)[0]
