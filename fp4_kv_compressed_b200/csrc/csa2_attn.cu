@@ -21,7 +21,9 @@
 // logit and folded into P for the P V product.  Q is converted to fp16 after an exact
 // power-of-two scaling that keeps max|q| below 2^15.
 // TMEM (512 columns): O = 64 x 512 fp32 in lanes 0-15 of each quadrant (M = 64
-// layout), the two S buffers (64 x 64 fp32) at lane offset 16, columns 0..127.
+// layout); at lane offset 16, the two S buffers, each as 4 partial 64 x 64 fp32
+// accumulators over channel quarters (independent MMA chains that the tensor pipe
+// overlaps; the softmax adds them), columns 0..511.
 // Online softmax in the log2 domain with lazy rescaling: O is rescaled only when
 // a head's running max grows by more than 8 (p stays <= 2^8, safe in fp16).
 // The MMA thread issues S(i+1) and P V(i) as soon as each is ready.  Every wait is
@@ -40,7 +42,9 @@ constexpr int kThreads = 512;
 constexpr int kTK = 64;                        // keys per tile
 constexpr int kHeads = 64;                     // heads per CTA (MMA M)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSpinLimit = 1u << 24;      // polls per wait before giving up
+constexpr int kSPart = 4;                      // partial S accumulators per tile (K split)
+constexpr uint32_t kXferBytes = 64 * 256 * 4;  // one CTA's O for the peer's channel half
+constexpr uint64_t kWaitLimitNs = 500000000ull; // a wait gives up after 0.5 s of wall time
 
 struct __align__(1024) Smem {
     uint8_t q[64 * 1024];            // Q fp16, [8 cb][64 heads][128 B] swizzled
@@ -48,7 +52,7 @@ struct __align__(1024) Smem {
     uint8_t p[kHeads * 128];         // P fp16, [64 heads][64 keys] swizzled (K-major)
     int32_t ids[CSA2_TOPK_MAX];      // compacted selected entry ids
     float sig[2][kTK];               // per-key scale of each stage (1 FP4, sigma SWA, 0 none)
-    uint64_t kv_full[2], kv_empty[2], s_full[2], p_full, pv_done, drain;
+    uint64_t kv_full[2], kv_empty[2], s_full[2], p_full, pv_done, drain, xfer;
     uint32_t tmem_base;
     int32_t abort;
     float wred[16];
@@ -69,10 +73,18 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *b) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
 }
 
-// Bounded wait for the phase with the given parity; returns false on timeout.
+__device__ __forceinline__ uint64_t wall_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait for the phase with the given parity: false once kWaitLimitNs of wall
+// time has passed without it completing.
 __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity) {
-    uint32_t addr = smem_u32(b);
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    const uint32_t addr = smem_u32(b);
+    const uint64_t t0 = wall_ns();
+    while (true) {
         uint32_t done;
         asm volatile(
             "{\n.reg .pred p;\n"
@@ -82,8 +94,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity) {
             : "r"(addr), "r"(parity)
             : "memory");
         if (done) return true;
+        if (wall_ns() - t0 > kWaitLimitNs) return false;
     }
-    return false;
 }
 
 __device__ __forceinline__ bool aborted(const Smem &s) {
@@ -98,6 +110,22 @@ __device__ __forceinline__ void tc_fence_before() {
 }
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+                 : "memory");
+}
+
+// Asynchronous bulk copy from this CTA's shared memory into another CTA's of the
+// cluster (dst and bar are shared::cluster addresses); bar receives complete_tx.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void *src, uint32_t bytes,
+                                                  uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "r"(smem_u32(src)), "r"(bytes), "r"(bar)
+        : "memory");
 }
 
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -117,6 +145,17 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
         "setp.ne.b32 p, %4, 0;\n"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
         "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+// One lane of a converged warp (the same lane on every call).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n.reg .pred p;\n.reg .b32 r;\n"
+        "elect.sync r|p, 0xffffffff;\n"
+        "selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(pred));
+    return pred != 0;
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t *b) {
@@ -144,6 +183,21 @@ __device__ __forceinline__ void tmem_ld16x32(uint32_t taddr, float *v) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int HALF>
+__device__ __forceinline__ void tmem_ld16x16(uint32_t taddr, float *v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], %17;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr), "n"(HALF));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 template <int HALF>
@@ -327,6 +381,7 @@ attn_tc_kernel(AttnArgs a) {
         mbar_init(&s.p_full, 4);
         mbar_init(&s.pv_done, 1);
         mbar_init(&s.drain, 1);
+        mbar_init(&s.xfer, 1);
         s.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -402,11 +457,12 @@ attn_tc_kernel(AttnArgs a) {
     const int head = 16 * qd + (lane & 15);
     const int half = lane >> 4;
     float m_run = -INFINITY, l_run = 0.0f;
-    bool sm_ok = true;
 
     if (warp == 0) {
         // ---------------- MMA issuer ----------------
-        if (lane == 0 && nt > 0) {
+        // The whole warp runs the loop (warp-uniform control flow and descriptors);
+        // one elected lane issues the MMAs and commits.
+        if (nt > 0) {
             const uint64_t qd0 = sw128_desc(smem_u32(s.q), 16, 1024);
             const uint64_t pd0 = sw128_desc(smem_u32(s.p), 16, 1024);
             const uint64_t kd0 = sw128_desc(smem_u32(s.kv[0]), 16, 1024);
@@ -414,45 +470,68 @@ attn_tc_kernel(AttnArgs a) {
             const uint64_t vd0 = sw128_desc(smem_u32(s.kv[0]), 8192, 1024);
             const uint64_t vd1 = sw128_desc(smem_u32(s.kv[1]), 8192, 1024);
             int s_next = 0, pv_next = 0;
-            uint32_t idle = 0;
-            while (pv_next < nt && idle < (1u << 26)) {
+            uint64_t idle_since = wall_ns();
+            bool stalled = false;
+            while (pv_next < nt && !stalled) {
                 bool progressed = false;
-                if (s_next < nt && s_next <= pv_next + 1 && mbar_test(&s.kv_full[s_next & 1], (s_next >> 1) & 1)) {
-                    tc_fence_after();
-                    const uint32_t d = tmem + (16u << 16) + (uint32_t)(s_next & 1) * kTK;
-                    const uint64_t kb = (s_next & 1) ? kd1 : kd0;
-#pragma unroll
-                    for (int kk = 0; kk < 32; ++kk) {
-                        const uint64_t off = (uint64_t)((kk >> 2) * 512 + (kk & 3) * 2);  // 16-byte units
-                        mma_f16(d, qd0 + off, kb + off, idesc_s, kk > 0);
-                    }
-                    mma_commit(&s.s_full[s_next & 1]);
-                    ++s_next;
-                    progressed = true;
-                }
-                if (pv_next < s_next && mbar_test(&s.p_full, pv_next & 1)) {
+                // P V first: it frees a K/V stage for the producers and O for the softmax
+                int go = 0;
+                if (lane == 0) go = pv_next < s_next && mbar_test(&s.p_full, pv_next & 1);
+                if (__shfl_sync(0xFFFFFFFFu, go, 0)) {
                     tc_fence_after();
                     const uint64_t vb = (pv_next & 1) ? vd1 : vd0;
-#pragma unroll
-                    for (int nh = 0; nh < 2; ++nh)
+                    if (elect_one()) {
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks)
-                            mma_f16(tmem + 256u * nh, pd0 + (uint64_t)(2 * ks),
-                                    vb + (uint64_t)(nh * 2048 + ks * 128), idesc_pv,
-                                    (pv_next > 0 || ks > 0) ? 1u : 0u);
-                    mma_commit(&s.kv_empty[pv_next & 1]);
-                    mma_commit(&s.pv_done);
+#pragma unroll
+                            for (int nh = 0; nh < 2; ++nh)
+                                mma_f16(tmem + 256u * nh, pd0 + (uint64_t)(2 * ks),
+                                        vb + (uint64_t)(nh * 2048 + ks * 128), idesc_pv,
+                                        (pv_next > 0 || ks > 0) ? 1u : 0u);
+                        mma_commit(&s.kv_empty[pv_next & 1]);
+                        mma_commit(&s.pv_done);
+                    }
+                    __syncwarp();
                     ++pv_next;
                     progressed = true;
                 }
-                idle = progressed ? 0u : idle + 1u;
+                go = 0;
+                if (lane == 0)
+                    go = s_next < nt && s_next <= pv_next + 1 &&
+                         mbar_test(&s.kv_full[s_next & 1], (s_next >> 1) & 1);
+                if (__shfl_sync(0xFFFFFFFFu, go, 0)) {
+                    tc_fence_after();
+                    // S as kSPart independent partial sums over channel slices, issued
+                    // round-robin so that consecutive MMAs never share an accumulator
+                    const uint32_t d = tmem + (16u << 16) + (uint32_t)(s_next & 1) * (kSPart * kTK);
+                    const uint64_t kb = (s_next & 1) ? kd1 : kd0;
+                    if (elect_one()) {
+#pragma unroll
+                        for (int kk = 0; kk < 32 / kSPart; ++kk)
+#pragma unroll
+                            for (int pp = 0; pp < kSPart; ++pp) {
+                                const int k16 = pp * (32 / kSPart) + kk;      // K-step of 16 channels
+                                const uint64_t off = (uint64_t)((k16 >> 2) * 512 + (k16 & 3) * 2);  // 16-byte units
+                                mma_f16(d + (uint32_t)(pp * kTK), qd0 + off, kb + off, idesc_s, kk > 0);
+                            }
+                        mma_commit(&s.s_full[s_next & 1]);
+                    }
+                    __syncwarp();
+                    ++s_next;
+                    progressed = true;
+                }
+                if (progressed)
+                    idle_since = wall_ns();
+                else
+                    stalled = __shfl_sync(0xFFFFFFFFu, (int)(wall_ns() - idle_since > kWaitLimitNs), 0) != 0;
             }
-            if (pv_next < nt) {
+            if (pv_next < nt && lane == 0) {
                 atomicExch(&s.abort, 1);
                 set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
             }
-            mma_commit(&s.drain);          // completes once every MMA issued above has
-            mbar_wait(&s.drain, 0);
+            if (elect_one()) mma_commit(&s.drain);   // completes once every MMA issued above has
+            __syncwarp();
+            if (lane == 0) mbar_wait(&s.drain, 0);
         }
         __syncwarp();
     } else if (warp >= 4 && warp < 8) {
@@ -467,7 +546,20 @@ attn_tc_kernel(AttnArgs a) {
             if (!ok) break;
             tc_fence_after();
             float x[32], sg[32];
-            tmem_ld16x32<32>(s_lane + (uint32_t)(i & 1) * kTK, x);
+            {
+                const uint32_t sb = s_lane + (uint32_t)(i & 1) * (kSPart * kTK);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    tmem_ld16x16<32>(sb + (uint32_t)(16 * c), x + 16 * c);
+#pragma unroll
+                    for (int pp = 1; pp < kSPart; ++pp) {
+                        float y[16];
+                        tmem_ld16x16<32>(sb + (uint32_t)(pp * kTK + 16 * c), y);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) x[16 * c + j] += y[j];
+                    }
+                }
+            }
             const int key0 = (tile_lo + i) * kTK + 32 * half;
             float mt = -INFINITY;
 #pragma unroll
@@ -529,7 +621,6 @@ attn_tc_kernel(AttnArgs a) {
             atomicExch(&s.abort, 1);
             set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
         }
-        sm_ok = ok;
         l_run += __shfl_xor_sync(0xFFFFFFFFu, l_run, 16);
         if (half == 0) {
             s.cm[head] = (ok && nt > 0) ? m_run : -INFINITY;
@@ -565,20 +656,26 @@ attn_tc_kernel(AttnArgs a) {
     // ---- combine the two key halves of the query through distributed shared memory ----
     // CTA r outputs channels [256 r, 256 r + 256); a softmax thread (head, half) holds
     // O[head][256 half .. +256) of its CTA in TMEM.
+    __syncwarp();                          // converged warps for the cluster barrier
+    if (threadIdx.x == 0) mbar_expect_tx(&s.xfer, kXferBytes);   // the peer's part, armed early
     tc_fence_before();
     cluster_sync();                        // partial stats published; all MMAs of both CTAs done
     tc_fence_after();
-    // Both CTAs derive the same weights; each softmax thread scales its half-row of
-    // O and stores it either into its own CTA's staging half (the channels this CTA
-    // writes) or into the peer's; then all threads add the two and write coalesced.
-    float *own = reinterpret_cast<float *>(s.kv[1]);       // [64 heads][256] this CTA's part
-    float *recv = reinterpret_cast<float *>(s.kv[0]);      // [64 heads][256] the peer's part
-    const bool smx = warp >= 4 && warp < 8;
-    if (smx) {
-        const uint32_t peer = rank ^ 1u;
-        const float m_self = s.cm[head], l_self = s.cl[head];
-        const float m_peer = ld_peer(peer_addr(&s.cm[head], peer));
-        const float l_peer = ld_peer(peer_addr(&s.cl[head], peer));
+    // Both CTAs derive the same weights.  Every thread scales a 64-column piece of one
+    // head's half-row of O (TMEM quadrant warp % 4, column quarter warp / 4) and stores
+    // it into local staging: `own` for the channels this CTA writes, `send` for the
+    // peer's.  One bulk copy moves `send` into the peer's `recv`; then all threads add
+    // own + recv and write coalesced.
+    float *own = reinterpret_cast<float *>(s.q);           // [64 heads][256] this CTA's part
+    float *send = reinterpret_cast<float *>(s.kv[1]);      // [64 heads][256] for the peer
+    float *recv = reinterpret_cast<float *>(s.kv[0]);      // [64 heads][256] from the peer
+    const uint32_t peer = rank ^ 1u;
+    {
+        const int qw = warp & 3, sub = warp >> 2;
+        const int hd = 16 * qw + (lane & 15), hf = lane >> 4;
+        const float m_self = s.cm[hd], l_self = s.cl[hd];
+        const float m_peer = ld_peer(peer_addr(&s.cm[hd], peer));
+        const float l_peer = ld_peer(peer_addr(&s.cl[hd], peer));
         const float m_all = fmaxf(m_self, m_peer);
         float f_self = 0.0f, f_peer = 0.0f;
         if (m_all != -INFINITY) {
@@ -586,16 +683,18 @@ attn_tc_kernel(AttnArgs a) {
             f_peer = m_peer == -INFINITY ? 0.0f : ex2(m_peer - m_all);
         }
         const float l_all = l_self * f_self + l_peer * f_peer;
-        const bool valid = head < hcta && l_all > 0.0f;
+        const bool valid = hd < hcta && l_all > 0.0f;
         const float w = valid ? f_self / l_all : 0.0f;
-        const uint32_t o_lane = tmem + ((uint32_t)(32 * qd) << 16);
-        const bool keep = (uint32_t)half == rank;
-        float *dst_own = own + head * 256;
-        const uint32_t dst_peer = peer_addr(recv + head * 256, peer);
+        // warp-uniform: tcgen05.ld is a whole-warp instruction (lanes 0-15 read the low
+        // half-row, lanes 16-31 the high one)
+        const bool have = __shfl_sync(0xFFFFFFFFu, (int)(nt > 0 && !aborted(s)), 0) != 0;
+        const uint32_t o_lane = tmem + ((uint32_t)(32 * qw) << 16);
+        const bool keep = (uint32_t)hf == rank;
+        float4 *dst = reinterpret_cast<float4 *>((keep ? own : send) + hd * 256);
 #pragma unroll 1
-        for (int cc = 0; cc < 256; cc += 32) {
+        for (int cc = 64 * sub; cc < 64 * sub + 64; cc += 32) {
             float o[32];
-            if (nt > 0 && sm_ok) {
+            if (have) {
                 tmem_ld16x32<256>(o_lane + (uint32_t)cc, o);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) o[j] *= w;
@@ -603,22 +702,28 @@ attn_tc_kernel(AttnArgs a) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j) o[j] = 0.0f;
             }
-            if (keep) {
+            // float4 f of head hd's row is stored at f ^ (hd % 16): the 16 heads of a
+            // quarter-warp then hit different bank groups
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    reinterpret_cast<float4 *>(dst_own + cc)[j] =
-                        make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    st_peer4(dst_peer + 4u * (cc + 4 * j), o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-            }
+            for (int j = 0; j < 8; ++j)
+                dst[(cc / 4 + j) ^ (hd & 15)] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
         }
-        if (keep && rank == 0 && head < hcta)
-            a.lse[(int64_t)qi * a.H + h0 + head] =
+        if (keep && sub == 0 && rank == 0 && hd < hcta)
+            a.lse[(int64_t)qi * a.H + h0 + hd] =
                 valid ? (m_all + log2f(l_all)) * 0.6931471805599453f : -INFINITY;
     }
-    cluster_sync();                        // the peer's part has landed in recv
+    fence_async_smem();                    // generic-proxy writes of `send` -> the bulk copy
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t dst = peer_addr(recv, peer), bar = peer_addr(&s.xfer, peer);
+#pragma unroll
+        for (int part = 0; part < 4; ++part)
+            bulk_copy_to_peer(dst + part * (kXferBytes / 4), reinterpret_cast<uint8_t *>(send) + part * (kXferBytes / 4),
+                              kXferBytes / 4, bar);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    const bool got = __syncthreads_and(mbar_wait(&s.xfer, 0)) != 0;   // the peer's part landed
+    if (!got && threadIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
     {
         const float4 *o4 = reinterpret_cast<const float4 *>(own);
         const float4 *r4 = reinterpret_cast<const float4 *>(recv);
@@ -627,12 +732,16 @@ attn_tc_kernel(AttnArgs a) {
         for (int i = threadIdx.x; i < kHeads * 64; i += kThreads) {
             const int hh = i >> 6, c4 = i & 63;
             if (hh < hcta) {
-                const float4 x = o4[i], y = r4[i];
+                const int f = hh * 64 + (c4 ^ (hh & 15));
+                const float4 x = o4[f];
+                const float4 y = got ? r4[f] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                 reinterpret_cast<float4 *>(obase + (int64_t)hh * kDim)[c4] =
                     make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w);
             }
         }
     }
+    // this CTA's outgoing copy has finished reading `send` before the CTA may exit
+    if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -650,6 +759,8 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, int BT, cudaStream_t st) {
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        e = prefer_max_smem(tc::attn_tc_kernel);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }

@@ -22,11 +22,13 @@
 namespace csa2 {
 
 // ------------------------------------------------------------------------------
-// Scoring core: one CTA scores a tile of kTileRows rows staged in shared memory.
+// Scoring core: one CTA of kScoreThreads threads scores a tile of kTileRows rows
+// staged in shared memory (thread t: rows t + kScoreThreads r, r < 4).  Small CTAs
+// (a 256-row, 32 KB tile) keep many tiles in flight per SM.
 // ------------------------------------------------------------------------------
-constexpr int kScoreThreads = 128;
+constexpr int kScoreThreads = 64;
 constexpr int kRowsPerThread = 4;
-constexpr int kTileRows = kScoreThreads * kRowsPerThread;   // 512 positions per CTA
+constexpr int kTileRows = kScoreThreads * kRowsPerThread;   // 256 positions per CTA
 
 // 16-byte unit u of row r lives at unit swz(r, u): a quarter-warp reading unit
 // u of 8 consecutive rows hits 8 different 16-byte bank groups.
@@ -64,7 +66,7 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
-// Scores of the thread's rows r_s = threadIdx.x + 128 s (s < kRowsPerThread), before
+// Scores of the thread's rows r_s = threadIdx.x + kScoreThreads s (s < kRowsPerThread), before
 // the per-entry scale.  Rows must be staged; invalid rows produce garbage the
 // caller discards.
 template <int D, int HI>
@@ -114,7 +116,7 @@ __device__ __forceinline__ void score_rows(const ScoreSmem<D, HI> &s, float out[
 }
 
 // ------------------------------------------------------------------------------
-// a3: Full scan.  grid (ceil(n_max / 512), B*Tq), 128 threads.
+// a3: Full scan.  grid (ceil(n_max / kTileRows), B*Tq), kScoreThreads threads.
 // ------------------------------------------------------------------------------
 template <int D, int HI>
 __global__ void __launch_bounds__(kScoreThreads)
@@ -176,7 +178,8 @@ index_scan_kernel(IndexArgs a) {
 }
 
 // ------------------------------------------------------------------------------
-// a6: Reindex scoring of the pool.  grid (ceil(pool_blocks / 64), B*Tq), 128 thr.
+// a6: Reindex scoring of the pool.  grid (ceil(8 pool_blocks / kTileRows), B*Tq),
+// kScoreThreads threads.
 // Candidate c = 8 * slot + r of the pool (slot < pool_blocks, r < 8) is position
 // 8 * pool[slot] + r; its score goes to scores[qi][c].
 // ------------------------------------------------------------------------------
@@ -194,7 +197,7 @@ reindex_score_kernel(IndexArgs a) {
     const int slot0 = blockIdx.x * (kTileRows / 8);
     const int32_t *pool = a.pool + (int64_t)qi * a.pool_blocks;
     const float *sig = a.idx_scale + (int64_t)b * a.cap;
-    float sgv[kRowsPerThread];   // row threadIdx.x + 128 i is handled by this thread below
+    float sgv[kRowsPerThread];   // row threadIdx.x + kScoreThreads i is handled by this thread below
 #pragma unroll
     for (int i = 0; i < kRowsPerThread; ++i) {
         const int r = threadIdx.x + kScoreThreads * i;
@@ -534,6 +537,8 @@ static cudaError_t launch_scan_t(const IndexArgs &a, int grid_x, int BT, cudaStr
         cudaError_t e = cudaFuncSetAttribute(index_scan_kernel<D, HI>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
+        e = prefer_max_smem(index_scan_kernel<D, HI>);
+        if (e != cudaSuccess) return e;
         attr_set = true;
     }
     index_scan_kernel<D, HI><<<dim3(grid_x, BT), kScoreThreads, smem, st>>>(a);
@@ -547,6 +552,8 @@ static cudaError_t launch_reindex_t(const IndexArgs &a, int BT, cudaStream_t st)
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(reindex_score_kernel<D, HI>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        e = prefer_max_smem(reindex_score_kernel<D, HI>);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -584,6 +591,8 @@ cudaError_t launch_select_full(const IndexArgs &a, int BT, cudaStream_t st) {
         cudaError_t e = cudaFuncSetAttribute(select_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
+        e = prefer_max_smem(select_full_kernel);
+        if (e != cudaSuccess) return e;
         attr_set = true;
     }
     select_full_kernel<<<BT, kSelThreads, smem, st>>>(a);
@@ -596,6 +605,8 @@ cudaError_t launch_select_reindex(const IndexArgs &a, int BT, cudaStream_t st) {
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(select_reindex_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
+        if (e != cudaSuccess) return e;
+        e = prefer_max_smem(select_reindex_kernel);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }

@@ -76,6 +76,14 @@ struct AttnArgs {
     int32_t *dev_err;
 };
 
+// Every kernel of the library asks for the largest shared-memory carveout, so that
+// consecutive kernels of a step never make an SM re-partition L1 and shared memory.
+template <class Kernel>
+inline cudaError_t prefer_max_smem(Kernel kernel) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                (int)cudaSharedmemCarveoutMaxShared);
+}
+
 cudaError_t launch_quantize_append(const QuantArgs &a, cudaStream_t st);
 cudaError_t launch_index_scan(const IndexArgs &a, int BT, cudaStream_t st);
 cudaError_t launch_select_full(const IndexArgs &a, int BT, cudaStream_t st);

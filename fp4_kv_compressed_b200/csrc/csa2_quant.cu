@@ -144,6 +144,12 @@ cudaError_t launch_quantize_append(const QuantArgs &a, cudaStream_t st) {
     int64_t warps = a.n_main + a.n_idx + a.n_swa;
     if (warps == 0) return cudaSuccess;
     int64_t blocks = (warps * 32 + 255) / 256;
+    static bool attr_set = false;  // once per process (one device per process)
+    if (!attr_set) {
+        cudaError_t e = prefer_max_smem(quantize_append_kernel);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
     quantize_append_kernel<<<(unsigned)blocks, 256, 0, st>>>(a);
     return cudaGetLastError();
 }
