@@ -69,11 +69,16 @@ def attn_flops(wl) -> int:
     return wl.B * wl.Tq * 4 * wl.H * 512 * (wl.top_k + n_win)
 
 
-# DRAM bytes (read + write) per launch from one ncu capture of each op's kernels:
-# (bytes, batch of the captured launch, kernel sources, sha256[:16] of those sources at
-# capture time).  Reported (scaled to the batch) only while the sources are unchanged.
+# DRAM bytes (read + write) per launch from one ncu capture of each of an op's kernels:
+# ([(bytes, batch of the captured launch), ...], kernel sources, sha256[:16] of those
+# sources at capture time).  Reported, each kernel scaled to the batch, only while the
+# sources are unchanged.  Captures: profiles/*.md.
 NCU_TRAFFIC = {
-    "csa2_sparse_attn_decode": (21_178_624, 64, ("csa2_attn.cu",), "c5d128b41c2558b3"),
+    "csa2_sparse_attn_decode": ([(21_173_504 + 512, 64)], ("csa2_attn.cu",), "0bf47515333277dc"),
+    "csa2_index_full": ([(138_471_168 + 5_096_448, 8), (18_140_160, 64)], ("csa2_index.cu",),
+                        "9ad48d8576b5b662"),
+    "csa2_index_reindex": ([(18_626_560, 8), (4_748_544, 64)], ("csa2_index.cu",),
+                           "9ad48d8576b5b662"),
 }
 
 
@@ -117,9 +122,9 @@ def op_rooflines(wl, plan, op_ms: dict, ms_step: float) -> dict:
         gbs = nbytes / (ms / 1e3) / 1e9
         traffic = None
         if name in NCU_TRAFFIC:
-            tb, tbatch, files, sha = NCU_TRAFFIC[name]
+            caps, files, sha = NCU_TRAFFIC[name]
             if _sources_hash(files) == sha:
-                traffic = tb * wl.B / tbatch
+                traffic = sum(tb * wl.B / tbatch for tb, tbatch in caps)
         e = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
              "frac": gbs / pk["hbm_gbs"], "traffic": traffic, "kernels": kernels,
              "algorithmic_bytes_per_launch": nbytes, "launch_ms": ms, "launches_per_step": n,

@@ -110,7 +110,8 @@ def test_op_rooflines_dominant_and_traffic():
     assert a["launches_per_step"] == 20 and abs(a["share_of_step"] - 0.4) < 1e-12
     assert a["tensor"]["flops_per_launch"] == 64 * 4 * 64 * 512 * 640
     assert ops["csa2_index_reindex"]["launches_per_step"] == 4
-    tb, tbatch, files, sha = bench.NCU_TRAFFIC["csa2_sparse_attn_decode"]
-    expect = tb * wl.B / tbatch if bench._sources_hash(files) == sha else None
-    assert a["traffic"] == expect
+    for name, e in ops.items():
+        caps, files, sha = bench.NCU_TRAFFIC[name]
+        expect = sum(tb * wl.B / b for tb, b in caps) if bench._sources_hash(files) == sha else None
+        assert e["traffic"] == expect
     assert max(ops, key=lambda n: ops[n]["share_of_step"]) == "csa2_sparse_attn_decode"
