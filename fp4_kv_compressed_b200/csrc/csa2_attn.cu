@@ -43,7 +43,7 @@ constexpr int kTK = 64;                        // keys per tile
 constexpr int kHeads = 64;                     // heads per CTA (MMA M)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSPart = 4;                      // partial S accumulators per tile (K split)
-constexpr uint32_t kXferBytes = 64 * 256 * 4;  // one CTA's O for the peer's channel half
+constexpr uint32_t kXferBytes = 32 * 256 * 4;  // half (32 heads) of one CTA's O for the peer
 constexpr uint64_t kWaitLimitNs = 500000000ull; // a wait gives up after 0.5 s of wall time
 
 struct __align__(1024) Smem {
@@ -52,7 +52,7 @@ struct __align__(1024) Smem {
     uint8_t p[kHeads * 128];         // P fp16, [64 heads][64 keys] swizzled (K-major)
     int32_t ids[CSA2_TOPK_MAX];      // compacted selected entry ids
     float sig[2][kTK];               // per-key scale of each stage (1 FP4, sigma SWA, 0 none)
-    uint64_t kv_full[2], kv_empty[2], s_full[2], p_full, pv_done, drain, xfer;
+    uint64_t kv_full[2], kv_empty[2], s_full[2], p_full, pv_done, drain, xfer[2];
     uint32_t tmem_base;
     int32_t abort;
     float wred[16];
@@ -366,11 +366,6 @@ attn_tc_kernel(AttnArgs a) {
     const int b = qi / a.Tq;
     const int h0 = blockIdx.y * kHeads;
     const int hcta = min(kHeads, a.H - h0);
-    const int64_t t = a.q_pos[qi];
-    const int64_t w0 = max64(0, t - a.swa_len + 1);
-    const int n_win = a.swa_len > 0 ? (int)(t - w0 + 1) : 0;
-    const int64_t n_vis = min64(visible_entries((int32_t)t, a.ratio), a.cap);
-
     // ---- set-up (all threads) -------------------------------------------------------------
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -381,7 +376,8 @@ attn_tc_kernel(AttnArgs a) {
         mbar_init(&s.p_full, 4);
         mbar_init(&s.pv_done, 1);
         mbar_init(&s.drain, 1);
-        mbar_init(&s.xfer, 1);
+        mbar_init(&s.xfer[0], 1);
+        mbar_init(&s.xfer[1], 1);
         s.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -391,6 +387,13 @@ attn_tc_kernel(AttnArgs a) {
                      "r"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
+    // barriers and TMEM above touch no global memory; everything below may read what the
+    // previous kernel of the stream wrote
+    grid_dep_wait();
+    const int64_t t = a.q_pos[qi];
+    const int64_t w0 = max64(0, t - a.swa_len + 1);
+    const int n_win = a.swa_len > 0 ? (int)(t - w0 + 1) : 0;
+    const int64_t n_vis = min64(visible_entries((int32_t)t, a.ratio), a.cap);
     // selected ids: thread t checks topk[t]; valid ids are compacted in order
     const int32_t *tk = a.topk + (int64_t)qi * a.top_k;
     const int e_id = (int)threadIdx.x < a.top_k ? tk[threadIdx.x] : -1;
@@ -657,10 +660,14 @@ attn_tc_kernel(AttnArgs a) {
     // CTA r outputs channels [256 r, 256 r + 256); a softmax thread (head, half) holds
     // O[head][256 half .. +256) of its CTA in TMEM.
     __syncwarp();                          // converged warps for the cluster barrier
-    if (threadIdx.x == 0) mbar_expect_tx(&s.xfer, kXferBytes);   // the peer's part, armed early
+    if (threadIdx.x == 0) {                // the peer's part, two halves of 32 heads, armed early
+        mbar_expect_tx(&s.xfer[0], kXferBytes);
+        mbar_expect_tx(&s.xfer[1], kXferBytes);
+    }
     tc_fence_before();
     cluster_sync();                        // partial stats published; all MMAs of both CTAs done
     tc_fence_after();
+    grid_dep_launch();
     // Both CTAs derive the same weights.  Every thread scales a 64-column piece of one
     // head's half-row of O (TMEM quadrant warp % 4, column quarter warp / 4) and stores
     // it into local staging: `own` for the channels this CTA writes, `send` for the
@@ -715,27 +722,31 @@ attn_tc_kernel(AttnArgs a) {
     fence_async_smem();                    // generic-proxy writes of `send` -> the bulk copy
     __syncthreads();
     if (threadIdx.x == 0) {
-        const uint32_t dst = peer_addr(recv, peer), bar = peer_addr(&s.xfer, peer);
 #pragma unroll
-        for (int part = 0; part < 4; ++part)
-            bulk_copy_to_peer(dst + part * (kXferBytes / 4), reinterpret_cast<uint8_t *>(send) + part * (kXferBytes / 4),
-                              kXferBytes / 4, bar);
+        for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t dst = peer_addr(recv + hh * 32 * 256, peer), bar = peer_addr(&s.xfer[hh], peer);
+            bulk_copy_to_peer(dst, send + hh * 32 * 256, kXferBytes / 2, bar);
+            bulk_copy_to_peer(dst + kXferBytes / 2, reinterpret_cast<uint8_t *>(send + hh * 32 * 256) + kXferBytes / 2,
+                              kXferBytes / 2, bar);
+        }
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     }
-    const bool got = __syncthreads_and(mbar_wait(&s.xfer, 0)) != 0;   // the peer's part landed
-    if (!got && threadIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
-    {
-        const float4 *o4 = reinterpret_cast<const float4 *>(own);
-        const float4 *r4 = reinterpret_cast<const float4 *>(recv);
-        float *obase = a.out + ((int64_t)qi * a.H + h0) * kDim + 256 * rank;
+    // add the peer's part as each half of the heads lands; write coalesced
+    const float4 *o4 = reinterpret_cast<const float4 *>(own);
+    const float4 *r4 = reinterpret_cast<const float4 *>(recv);
+    float *obase = a.out + ((int64_t)qi * a.H + h0) * kDim + 256 * rank;
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {
+        const bool got = __syncthreads_and(mbar_wait(&s.xfer[hh], 0)) != 0;
+        if (!got && threadIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
 #pragma unroll 2
-        for (int i = threadIdx.x; i < kHeads * 64; i += kThreads) {
-            const int hh = i >> 6, c4 = i & 63;
-            if (hh < hcta) {
-                const int f = hh * 64 + (c4 ^ (hh & 15));
+        for (int i = hh * 32 * 64 + threadIdx.x; i < (hh + 1) * 32 * 64; i += kThreads) {
+            const int h = i >> 6, c4 = i & 63;
+            if (h < hcta) {
+                const int f = h * 64 + (c4 ^ (h & 15));
                 const float4 x = o4[f];
                 const float4 y = got ? r4[f] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                reinterpret_cast<float4 *>(obase + (int64_t)hh * kDim)[c4] =
+                reinterpret_cast<float4 *>(obase + (int64_t)h * kDim)[c4] =
                     make_float4(x.x + y.x, x.y + y.y, x.z + y.z, x.w + y.w);
             }
         }
@@ -765,8 +776,8 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, int BT, cudaStream_t st) {
         attr_set = true;
     }
     dim3 grid(2 * BT, (a.H + tc::kHeads - 1) / tc::kHeads);   // 2-CTA clusters
-    tc::attn_tc_kernel<<<grid, tc::kThreads, smem, st>>>(a);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(tc::attn_tc_kernel, grid, dim3(tc::kThreads), smem, st, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace csa2

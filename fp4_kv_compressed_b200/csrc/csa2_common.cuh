@@ -96,6 +96,14 @@ __device__ __forceinline__ float key_to_score(uint32_t k) {
     return __uint_as_float(u);
 }
 
+// Programmatic dependent launch.  Every kernel of the library is launched so that the
+// next kernel of the stream may be scheduled while it finishes: grid_dep_wait() blocks
+// until the previous grid has completed with its memory visible (each kernel calls it
+// before its first global memory access), grid_dep_launch() lets the next grid start
+// launching (called once a CTA's main work is done).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void set_dev_err(int32_t *dev_err, int bit) {
     if (dev_err) atomicOr(dev_err, bit);
 }

@@ -22,13 +22,13 @@
 namespace csa2 {
 
 // ------------------------------------------------------------------------------
-// Scoring core: one CTA of kScoreThreads threads scores a tile of kTileRows rows
-// staged in shared memory (thread t: rows t + kScoreThreads r, r < 4).  Small CTAs
-// (a 256-row, 32 KB tile) keep many tiles in flight per SM.
+// Scoring core: one CTA of kScoreThreads threads scores a tile of kScoreThreads * R rows
+// staged in shared memory (thread t: rows t + kScoreThreads r, r < R).  Small CTAs
+// keep many tiles in flight per SM; the Reindex gather prefers the smaller tile.
 // ------------------------------------------------------------------------------
 constexpr int kScoreThreads = 64;
-constexpr int kRowsPerThread = 4;
-constexpr int kTileRows = kScoreThreads * kRowsPerThread;   // 256 positions per CTA
+constexpr int kScanRows = 4;       // rows per thread, Full scan (256-row, 32 KB tiles)
+constexpr int kReindexRows = 2;    // rows per thread, Reindex gather (128-row, 16 KB tiles)
 
 // 16-byte unit u of row r lives at unit swz(r, u): a quarter-warp reading unit
 // u of 8 consecutive rows hits 8 different 16-byte bank groups.
@@ -40,16 +40,16 @@ __device__ __forceinline__ int swz(int r, int u) {
         return u ^ ((r >> 1) & 3);
 }
 
-template <int D, int HI>
+template <int D, int HI, int R>
 struct ScoreSmem {
-    uint8_t rows[kTileRows * D];
+    uint8_t rows[kScoreThreads * R * D];
     float2 q[D / 2][HI];     // q pairs (q[h][2j], q[h][2j+1]) as fp32
     float w[HI];
 };
 
 // Stage q (bf16 [HI][D]) and w into shared memory as fp32.
-template <int D, int HI>
-__device__ __forceinline__ void load_query(ScoreSmem<D, HI> &s, const uint16_t *q, const float *w) {
+template <int D, int HI, int R>
+__device__ __forceinline__ void load_query(ScoreSmem<D, HI, R> &s, const uint16_t *q, const float *w) {
     for (int e = threadIdx.x; e < HI * D / 2; e += blockDim.x) {
         int h = e / (D / 2), j = e % (D / 2);
         uint32_t two = *reinterpret_cast<const uint32_t *>(q + h * D + 2 * j);
@@ -66,45 +66,50 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
-// Scores of the thread's rows r_s = threadIdx.x + kScoreThreads s (s < kRowsPerThread), before
+// Scores of the thread's rows r_s = threadIdx.x + kScoreThreads s (s < R), before
 // the per-entry scale.  Rows must be staged; invalid rows produce garbage the
 // caller discards.
-template <int D, int HI>
-__device__ __forceinline__ void score_rows(const ScoreSmem<D, HI> &s, float out[kRowsPerThread]) {
-    float2 acc[kRowsPerThread][HI];
+template <int D, int HI, int R>
+__device__ __forceinline__ void score_rows(const ScoreSmem<D, HI, R> &s, float out[R]) {
+    float2 acc[R][HI];
 #pragma unroll
-    for (int r = 0; r < kRowsPerThread; ++r)
+    for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int h = 0; h < HI; ++h) acc[r][h] = make_float2(0.0f, 0.0f);
 
 #pragma unroll
     for (int u = 0; u < D / 16; ++u) {          // 16 channels = 8 pairs per unit
-        float2 qv[8][HI];
+        uint32_t wv[R][4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int r = 0; r < R; ++r) {
+            const int row = threadIdx.x + kScoreThreads * r;
+            const uint4 kw = *reinterpret_cast<const uint4 *>(s.rows + row * D + 16 * swz<D>(row, u));
+            wv[r][0] = kw.x; wv[r][1] = kw.y; wv[r][2] = kw.z; wv[r][3] = kw.w;
+        }
 #pragma unroll
-            for (int h = 0; h < HI; ++h) qv[j][h] = s.q[8 * u + j][h];
+        for (int i = 0; i < 4; ++i) {           // one 32-bit word = channel pairs 2i, 2i+1 of the unit
+            float2 qa[HI], qb[HI];              // q is read per word: few live registers
 #pragma unroll
-        for (int r = 0; r < kRowsPerThread; ++r) {
-            int row = threadIdx.x + kScoreThreads * r;
-            uint4 kw = *reinterpret_cast<const uint4 *>(s.rows + row * D + 16 * swz<D>(row, u));
-            uint32_t wv[4] = {kw.x, kw.y, kw.z, kw.w};
+            for (int h = 0; h < HI; ++h) {
+                qa[h] = s.q[8 * u + 2 * i][h];
+                qb[h] = s.q[8 * u + 2 * i + 1][h];
+            }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint32_t h01 = cvt_e4m3x2_f16x2(wv[i] & 0xFFFFu);
-                uint32_t h23 = cvt_e4m3x2_f16x2(wv[i] >> 16);
+            for (int r = 0; r < R; ++r) {
+                uint32_t h01 = cvt_e4m3x2_f16x2(wv[r][i] & 0xFFFFu);
+                uint32_t h23 = cvt_e4m3x2_f16x2(wv[r][i] >> 16);
                 float2 k01 = __half22float2(*reinterpret_cast<__half2 *>(&h01));
                 float2 k23 = __half22float2(*reinterpret_cast<__half2 *>(&h23));
 #pragma unroll
                 for (int h = 0; h < HI; ++h) {
-                    acc[r][h] = fma2(qv[2 * i][h], k01, acc[r][h]);
-                    acc[r][h] = fma2(qv[2 * i + 1][h], k23, acc[r][h]);
+                    acc[r][h] = fma2(qa[h], k01, acc[r][h]);
+                    acc[r][h] = fma2(qb[h], k23, acc[r][h]);
                 }
             }
         }
     }
 #pragma unroll
-    for (int r = 0; r < kRowsPerThread; ++r) {
+    for (int r = 0; r < R; ++r) {
         float t = 0.0f;
 #pragma unroll
         for (int h = 0; h < HI; ++h) {
@@ -121,8 +126,10 @@ __device__ __forceinline__ void score_rows(const ScoreSmem<D, HI> &s, float out[
 template <int D, int HI>
 __global__ void __launch_bounds__(kScoreThreads)
 index_scan_kernel(IndexArgs a) {
+    constexpr int R = kScanRows, kTileRows = kScoreThreads * R;
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    ScoreSmem<D, HI> &s = *reinterpret_cast<ScoreSmem<D, HI> *>(smem_raw);
+    ScoreSmem<D, HI, R> &s = *reinterpret_cast<ScoreSmem<D, HI, R> *>(smem_raw);
+    grid_dep_wait();
     const int qi = blockIdx.y;
     const int b = qi / a.Tq;
     int64_t N = visible_entries(a.q_pos[qi], a.ratio);
@@ -144,21 +151,22 @@ index_scan_kernel(IndexArgs a) {
     load_query<D, HI>(s, a.q_idx + (int64_t)qi * HI * D, a.w + (int64_t)qi * HI);
     // the rows' scales, fetched while the tile is in flight
     const float *sig = a.idx_scale + (int64_t)b * a.cap;
-    float sgv[kRowsPerThread];
+    float sgv[R];
 #pragma unroll
-    for (int r = 0; r < kRowsPerThread; ++r) {
+    for (int r = 0; r < R; ++r) {
         const int row = threadIdx.x + kScoreThreads * r;
         sgv[r] = row < rows ? __ldg(sig + p0 + row) : 0.0f;
     }
     cp_async_wait_all();
     __syncthreads();
 
-    float sc[kRowsPerThread];
-    score_rows<D, HI>(s, sc);
+    float sc[R];
+    score_rows<D, HI, R>(s, sc);
+    grid_dep_launch();
 
     float *scores = a.scores + (int64_t)qi * a.score_stride;
 #pragma unroll
-    for (int r = 0; r < kRowsPerThread; ++r) {
+    for (int r = 0; r < R; ++r) {
         int row = threadIdx.x + kScoreThreads * r;
         int64_t p = p0 + row;
         float v = -INFINITY;
@@ -179,17 +187,19 @@ index_scan_kernel(IndexArgs a) {
 
 // ------------------------------------------------------------------------------
 // a6: Reindex scoring of the pool.  grid (ceil(8 pool_blocks / kTileRows), B*Tq),
-// kScoreThreads threads.
+// kScoreThreads threads, kTileRows = kScoreThreads * kReindexRows.
 // Candidate c = 8 * slot + r of the pool (slot < pool_blocks, r < 8) is position
 // 8 * pool[slot] + r; its score goes to scores[qi][c].
 // ------------------------------------------------------------------------------
 template <int D, int HI>
 __global__ void __launch_bounds__(kScoreThreads)
 reindex_score_kernel(IndexArgs a) {
+    constexpr int R = kReindexRows, kTileRows = kScoreThreads * R;
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    ScoreSmem<D, HI> &s = *reinterpret_cast<ScoreSmem<D, HI> *>(smem_raw);
+    ScoreSmem<D, HI, R> &s = *reinterpret_cast<ScoreSmem<D, HI, R> *>(smem_raw);
     __shared__ int valid_row[kTileRows];
     __shared__ int pos_row[kTileRows];
+    grid_dep_wait();
     const int qi = blockIdx.y;
     const int b = qi / a.Tq;
     int64_t N = visible_entries(a.q_pos[qi], a.ratio);
@@ -197,9 +207,9 @@ reindex_score_kernel(IndexArgs a) {
     const int slot0 = blockIdx.x * (kTileRows / 8);
     const int32_t *pool = a.pool + (int64_t)qi * a.pool_blocks;
     const float *sig = a.idx_scale + (int64_t)b * a.cap;
-    float sgv[kRowsPerThread];   // row threadIdx.x + kScoreThreads i is handled by this thread below
+    float sgv[R];   // row threadIdx.x + kScoreThreads i is handled by this thread below
 #pragma unroll
-    for (int i = 0; i < kRowsPerThread; ++i) {
+    for (int i = 0; i < R; ++i) {
         const int r = threadIdx.x + kScoreThreads * i;
         int slot = slot0 + r / 8;
         int blk = slot < a.pool_blocks ? pool[slot] : -1;
@@ -223,11 +233,12 @@ reindex_score_kernel(IndexArgs a) {
     cp_async_wait_all();
     __syncthreads();
 
-    float sc[kRowsPerThread];
-    score_rows<D, HI>(s, sc);
+    float sc[R];
+    score_rows<D, HI, R>(s, sc);
+    grid_dep_launch();
     float *out = a.scores + (int64_t)qi * a.score_stride + (int64_t)slot0 * 8;
 #pragma unroll
-    for (int r = 0; r < kRowsPerThread; ++r) {
+    for (int r = 0; r < R; ++r) {
         int row = threadIdx.x + kScoreThreads * r;
         if (slot0 + row / 8 < a.pool_blocks)
             out[row] = valid_row[row] ? __fmul_rn(sc[r], sgv[r]) : 0.0f;
@@ -447,6 +458,7 @@ select_full_kernel(IndexArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     SelSmem &s = *reinterpret_cast<SelSmem *>(smem_raw);
     __shared__ int sel_out[CSA2_TOPK_MAX];
+    grid_dep_wait();
     const int qi = blockIdx.x;
     int64_t N64 = visible_entries(a.q_pos[qi], a.ratio);
     N64 = min64(min64(N64, a.n_max), a.cap);
@@ -490,6 +502,7 @@ select_full_kernel(IndexArgs a) {
         cnt = block_topk(key, id, N, a.top_k, sel_out, s);
     }
     __syncthreads();
+    grid_dep_launch();
     int32_t *topk = a.topk_out + (int64_t)qi * a.top_k;
     for (int i = threadIdx.x; i < a.top_k; i += blockDim.x) topk[i] = i < cnt ? sel_out[i] : -1;
     if (threadIdx.x == 0) a.topk_count[qi] = cnt;
@@ -501,26 +514,28 @@ select_reindex_kernel(IndexArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     SelSmem &s = *reinterpret_cast<SelSmem *>(smem_raw);
     __shared__ int sel_out[CSA2_TOPK_MAX];
+    grid_dep_wait();
     const int qi = blockIdx.x;
     int64_t N = min64(visible_entries(a.q_pos[qi], a.ratio), a.cap);
     const int32_t *pool = a.pool + (int64_t)qi * a.pool_blocks;
     const float *sc = a.scores + (int64_t)qi * a.score_stride;
     const int nc = a.pool_blocks * 8;
-    for (int i = threadIdx.x; i < a.pool_blocks; i += blockDim.x) {
-        s.pool[i] = pool[i];
-        if (i > 0 && pool[i] >= 0 && pool[i - 1] >= pool[i]) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
-    }
-    __syncthreads();
+    // candidate c's score and its pool block are read together (no dependent round trip)
     for (int i = threadIdx.x; i < nc; i += blockDim.x) {
-        int blk = s.pool[i >> 3];
-        int64_t p = (int64_t)blk * 8 + (i & 7);
-        s.keys[i] = (blk >= 0 && p < N) ? score_key(sc[i]) : 0u;
+        const int blk = __ldg(pool + (i >> 3));
+        const int64_t p = (int64_t)blk * 8 + (i & 7);
+        s.keys[i] = (blk >= 0 && p < N) ? score_key(__ldg(sc + i)) : 0u;
+        if ((i & 7) == 0) {
+            s.pool[i >> 3] = blk;
+            if (i > 0 && blk >= 0 && __ldg(pool + (i >> 3) - 1) >= blk) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
+        }
     }
     __syncthreads();
     auto key = [&](int i) -> uint32_t { return s.keys[i]; };
     auto id = [&](int i) -> int { return s.pool[i >> 3] * 8 + (i & 7); };
     int cnt = block_topk(key, id, nc, a.top_k, sel_out, s);
     __syncthreads();
+    grid_dep_launch();
     int32_t *topk = a.topk_out + (int64_t)qi * a.top_k;
     for (int i = threadIdx.x; i < a.top_k; i += blockDim.x) topk[i] = i < cnt ? sel_out[i] : -1;
     if (threadIdx.x == 0) a.topk_count[qi] = cnt;
@@ -531,7 +546,7 @@ select_reindex_kernel(IndexArgs a) {
 // ------------------------------------------------------------------------------
 template <int D, int HI>
 static cudaError_t launch_scan_t(const IndexArgs &a, int grid_x, int BT, cudaStream_t st) {
-    size_t smem = sizeof(ScoreSmem<D, HI>);
+    size_t smem = sizeof(ScoreSmem<D, HI, kScanRows>);
     static bool attr_set = false;  // once per process and instantiation
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(index_scan_kernel<D, HI>,
@@ -541,13 +556,13 @@ static cudaError_t launch_scan_t(const IndexArgs &a, int grid_x, int BT, cudaStr
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    index_scan_kernel<D, HI><<<dim3(grid_x, BT), kScoreThreads, smem, st>>>(a);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(index_scan_kernel<D, HI>, dim3(grid_x, BT), dim3(kScoreThreads), smem, st, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int D, int HI>
 static cudaError_t launch_reindex_t(const IndexArgs &a, int BT, cudaStream_t st) {
-    size_t smem = sizeof(ScoreSmem<D, HI>);
+    size_t smem = sizeof(ScoreSmem<D, HI, kReindexRows>);
     static bool attr_set = false;  // once per process and instantiation
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(reindex_score_kernel<D, HI>,
@@ -557,9 +572,10 @@ static cudaError_t launch_reindex_t(const IndexArgs &a, int BT, cudaStream_t st)
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    int gx = (a.pool_blocks + kTileRows / 8 - 1) / (kTileRows / 8);
-    reindex_score_kernel<D, HI><<<dim3(gx, BT), kScoreThreads, smem, st>>>(a);
-    return cudaGetLastError();
+    constexpr int kBlocksPerTile = kScoreThreads * kReindexRows / 8;
+    int gx = (a.pool_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
+    cudaError_t e = launch_pdl(reindex_score_kernel<D, HI>, dim3(gx, BT), dim3(kScoreThreads), smem, st, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 #define CSA2_DISPATCH_HI(D, FN, ...)                                          \
@@ -573,6 +589,7 @@ static cudaError_t launch_reindex_t(const IndexArgs &a, int BT, cudaStream_t st)
     }
 
 cudaError_t launch_index_scan(const IndexArgs &a, int BT, cudaStream_t st) {
+    constexpr int kTileRows = kScoreThreads * kScanRows;
     int grid_x = (int)((a.n_max + kTileRows - 1) / kTileRows);
     if (grid_x == 0) return cudaSuccess;
     if (a.d_idx == 128) { CSA2_DISPATCH_HI(128, launch_scan_t, a, grid_x, BT, st) }
@@ -595,8 +612,8 @@ cudaError_t launch_select_full(const IndexArgs &a, int BT, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    select_full_kernel<<<BT, kSelThreads, smem, st>>>(a);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(select_full_kernel, dim3(BT), dim3(kSelThreads), smem, st, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_select_reindex(const IndexArgs &a, int BT, cudaStream_t st) {
@@ -610,13 +627,8 @@ cudaError_t launch_select_reindex(const IndexArgs &a, int BT, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    select_reindex_kernel<<<BT, kSelThreads, smem, st>>>(a);
-    return cudaGetLastError();
-}
-
-size_t score_smem_bytes(int d_idx, int H_I) {
-    if (d_idx == 128) return kTileRows * 128 + (128 / 2) * H_I * 8 + 64;
-    return kTileRows * 64 + (64 / 2) * H_I * 8 + 64;
+    cudaError_t e = launch_pdl(select_reindex_kernel, dim3(BT), dim3(kSelThreads), smem, st, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace csa2

@@ -84,6 +84,23 @@ inline cudaError_t prefer_max_smem(Kernel kernel) {
                                 (int)cudaSharedmemCarveoutMaxShared);
 }
 
+// Launch with programmatic stream serialisation (see grid_dep_wait / grid_dep_launch).
+template <class... KArgs, class... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 cudaError_t launch_quantize_append(const QuantArgs &a, cudaStream_t st);
 cudaError_t launch_index_scan(const IndexArgs &a, int BT, cudaStream_t st);
 cudaError_t launch_select_full(const IndexArgs &a, int BT, cudaStream_t st);

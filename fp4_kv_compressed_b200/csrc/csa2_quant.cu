@@ -105,6 +105,8 @@ __device__ void quant_fp8_row(const uint16_t *src, uint8_t *dst_codes, float *ds
 }
 
 __global__ void __launch_bounds__(256) quantize_append_kernel(QuantArgs a) {
+    grid_dep_wait();
+    grid_dep_launch();
     int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp < a.n_main) {
@@ -150,8 +152,8 @@ cudaError_t launch_quantize_append(const QuantArgs &a, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    quantize_append_kernel<<<(unsigned)blocks, 256, 0, st>>>(a);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(quantize_append_kernel, dim3((unsigned)blocks), dim3(256), 0, st, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace csa2
