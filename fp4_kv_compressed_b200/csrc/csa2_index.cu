@@ -48,14 +48,26 @@ struct ScoreSmem {
 };
 
 // Stage q (bf16 [HI][D]) and w into shared memory as fp32.
+// All of a thread's loads are issued before any is used (one memory round trip).
 template <int D, int HI, int R>
 __device__ __forceinline__ void load_query(ScoreSmem<D, HI, R> &s, const uint16_t *q, const float *w) {
-    for (int e = threadIdx.x; e < HI * D / 2; e += blockDim.x) {
-        int h = e / (D / 2), j = e % (D / 2);
-        uint32_t two = *reinterpret_cast<const uint32_t *>(q + h * D + 2 * j);
-        s.q[j][h] = make_float2(bf16_bits_to_f32(two & 0xFFFFu), bf16_bits_to_f32(two >> 16));
+    constexpr int kPer = (HI * D / 2 + kScoreThreads - 1) / kScoreThreads;
+    uint32_t two[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int e = threadIdx.x + k * kScoreThreads;
+        two[k] = e < HI * D / 2 ? __ldg(reinterpret_cast<const uint32_t *>(q) + e) : 0u;
     }
-    if (threadIdx.x < HI) s.w[threadIdx.x] = w[threadIdx.x];
+    const float wv = threadIdx.x < HI ? __ldg(w + threadIdx.x) : 0.0f;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int e = threadIdx.x + k * kScoreThreads;
+        if (e < HI * D / 2) {
+            const int h = e / (D / 2), j = e % (D / 2);
+            s.q[j][h] = make_float2(bf16_bits_to_f32(two[k] & 0xFFFFu), bf16_bits_to_f32(two[k] >> 16));
+        }
+    }
+    if (threadIdx.x < HI) s.w[threadIdx.x] = wv;
 }
 
 // Copy one 16-byte unit global -> shared (bypassing L1).
@@ -155,7 +167,7 @@ index_scan_kernel(IndexArgs a) {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
         const int row = threadIdx.x + kScoreThreads * r;
-        sgv[r] = row < rows ? __ldg(sig + p0 + row) : 0.0f;
+        sgv[r] = __ldg(sig + p0 + min(row, rows - 1));   // branch-free: all R loads in flight
     }
     cp_async_wait_all();
     __syncthreads();
@@ -212,13 +224,14 @@ reindex_score_kernel(IndexArgs a) {
     for (int i = 0; i < R; ++i) {
         const int r = threadIdx.x + kScoreThreads * i;
         int slot = slot0 + r / 8;
-        int blk = slot < a.pool_blocks ? pool[slot] : -1;
+        int blk = __ldg(pool + min(slot, a.pool_blocks - 1));
+        if (slot >= a.pool_blocks) blk = -1;
         int64_t p = (int64_t)blk * 8 + (r & 7);
         bool ok = blk >= 0 && p < N;
         if (blk >= 0 && (int64_t)blk * 8 >= N && (r & 7) == 0) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
         valid_row[r] = ok;
         pos_row[r] = ok ? (int)p : 0;
-        sgv[i] = ok ? __ldg(sig + p) : 0.0f;
+        sgv[i] = __ldg(sig + (ok ? p : 0));   // branch-free (row 0 always exists)
     }
     __syncthreads();
     const uint8_t *base = a.idx_codes + (int64_t)b * a.cap * D;
@@ -273,6 +286,26 @@ struct SelSmem {
 
 // Exclusive scans (in warp order) of s.wa and s.wb; totals in s.bcast[0], s.bcast[1].
 // Call with every warp's entry written; ends with a barrier.
+// keys[i] = make(i, load(i)) for i < n, where load(i) is a branch-free global load
+// (its index clamped into [0, n)) and make applies the validity rules: a thread
+// issues the loads of kStageBatch strides before using any, so its 16 keys cost
+// about one memory round trip instead of sixteen.
+constexpr int kStageBatch = 16;
+template <class Raw, class Load, class Make>
+__device__ __forceinline__ void stage_keys(uint32_t *keys, int n, Load load, Make make) {
+    for (int base = 0; base < n; base += kSelThreads * kStageBatch) {
+        Raw v[kStageBatch];
+#pragma unroll
+        for (int j = 0; j < kStageBatch; ++j)
+            v[j] = load(min(base + j * kSelThreads + (int)threadIdx.x, n - 1));
+#pragma unroll
+        for (int j = 0; j < kStageBatch; ++j) {
+            const int i = base + j * kSelThreads + (int)threadIdx.x;
+            if (i < n) keys[i] = make(i, v[j]);
+        }
+    }
+}
+
 __device__ __forceinline__ void sel_scan_warps(SelSmem &s) {
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -470,7 +503,8 @@ select_full_kernel(IndexArgs a) {
         const float *bm = a.bmax + (int64_t)qi * a.bmax_stride;
         const bool staged = nb <= kSelStageMax;
         if (staged) {
-            for (int i = threadIdx.x; i < nb; i += blockDim.x) s.keys[i] = score_key(bm[i]);
+            stage_keys<float>(s.keys, nb, [&](int i) { return __ldg(bm + i); },
+                              [&](int, float v) { return score_key(v); });
             __syncthreads();
         }
         auto bkey = [&](int i) -> uint32_t { return staged ? s.keys[i] : score_key(bm[i]); };
@@ -483,10 +517,15 @@ select_full_kernel(IndexArgs a) {
                 pool_out[i] = i < np ? s.pool[i] : -1;
         // candidates: the pool's positions, in ascending order
         const int nc = np * 8;
-        for (int i = threadIdx.x; i < nc; i += blockDim.x) {
-            int64_t p = (int64_t)s.pool[i >> 3] * 8 + (i & 7);
-            s.keys[i] = p < N ? score_key(scores[p]) : 0u;
-        }
+        stage_keys<float>(s.keys, nc,
+            [&](int i) {   // a position past N (the pool's last block) is clamped, then dropped
+                const int64_t p = (int64_t)s.pool[i >> 3] * 8 + (i & 7);
+                return __ldg(scores + min64(p, (int64_t)N - 1));
+            },
+            [&](int i, float v) {
+                const int64_t p = (int64_t)s.pool[i >> 3] * 8 + (i & 7);
+                return p < N ? score_key(v) : 0u;
+            });
         __syncthreads();
         auto ckey = [&](int i) -> uint32_t { return s.keys[i]; };
         auto cid = [&](int i) -> int { return s.pool[i >> 3] * 8 + (i & 7); };
@@ -494,7 +533,8 @@ select_full_kernel(IndexArgs a) {
     } else {
         const bool staged = N <= kSelStageMax;
         if (staged) {
-            for (int i = threadIdx.x; i < N; i += blockDim.x) s.keys[i] = score_key(scores[i]);
+            stage_keys<float>(s.keys, N, [&](int i) { return __ldg(scores + i); },
+                              [&](int, float v) { return score_key(v); });
             __syncthreads();
         }
         auto key = [&](int i) -> uint32_t { return staged ? s.keys[i] : score_key(scores[i]); };
@@ -520,16 +560,19 @@ select_reindex_kernel(IndexArgs a) {
     const int32_t *pool = a.pool + (int64_t)qi * a.pool_blocks;
     const float *sc = a.scores + (int64_t)qi * a.score_stride;
     const int nc = a.pool_blocks * 8;
-    // candidate c's score and its pool block are read together (no dependent round trip)
-    for (int i = threadIdx.x; i < nc; i += blockDim.x) {
-        const int blk = __ldg(pool + (i >> 3));
-        const int64_t p = (int64_t)blk * 8 + (i & 7);
-        s.keys[i] = (blk >= 0 && p < N) ? score_key(__ldg(sc + i)) : 0u;
-        if ((i & 7) == 0) {
-            s.pool[i >> 3] = blk;
-            if (i > 0 && blk >= 0 && __ldg(pool + (i >> 3) - 1) >= blk) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
-        }
+    for (int i = threadIdx.x; i < a.pool_blocks; i += blockDim.x) {
+        const int blk = __ldg(pool + i);
+        s.pool[i] = blk;
+        if (i > 0 && blk >= 0 && __ldg(pool + i - 1) >= blk) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
     }
+    // candidate c's score and its pool block are read together (no dependent round trip)
+    stage_keys<float2>(s.keys, nc,
+        [&](int i) { return make_float2(__int_as_float(__ldg(pool + (i >> 3))), __ldg(sc + i)); },
+        [&](int i, float2 r) {
+            const int blk = __float_as_int(r.x);
+            const int64_t p = (int64_t)blk * 8 + (i & 7);
+            return (blk >= 0 && p < N) ? score_key(r.y) : 0u;
+        });
     __syncthreads();
     auto key = [&](int i) -> uint32_t { return s.keys[i]; };
     auto id = [&](int i) -> int { return s.pool[i >> 3] * 8 + (i & 7); };
