@@ -280,30 +280,22 @@ struct SelSmem {
     int wa[kSelWarps], wb[kSelWarps];
     uint32_t wmin[kSelWarps], wmax[kSelWarps];
     int bcast[4];
-    int pool[CSA2_POOL_MAX];
-    uint32_t keys[kSelStageMax];
+    alignas(16) int pool[CSA2_POOL_MAX];
+    alignas(16) uint32_t keys[kSelStageMax];
 };
 
 // Exclusive scans (in warp order) of s.wa and s.wb; totals in s.bcast[0], s.bcast[1].
 // Call with every warp's entry written; ends with a barrier.
-// keys[i] = make(i, load(i)) for i < n, where load(i) is a branch-free global load
-// (its index clamped into [0, n)) and make applies the validity rules: a thread
-// issues the loads of kStageBatch strides before using any, so its 16 keys cost
-// about one memory round trip instead of sixteen.
-constexpr int kStageBatch = 16;
-template <class Raw, class Load, class Make>
-__device__ __forceinline__ void stage_keys(uint32_t *keys, int n, Load load, Make make) {
-    for (int base = 0; base < n; base += kSelThreads * kStageBatch) {
-        Raw v[kStageBatch];
-#pragma unroll
-        for (int j = 0; j < kStageBatch; ++j)
-            v[j] = load(min(base + j * kSelThreads + (int)threadIdx.x, n - 1));
-#pragma unroll
-        for (int j = 0; j < kStageBatch; ++j) {
-            const int i = base + j * kSelThreads + (int)threadIdx.x;
-            if (i < n) keys[i] = make(i, v[j]);
-        }
-    }
+// dst[0..n) = the raw 32-bit words src[0..n), copied into shared memory with 16-byte
+// cp.async (src 16-byte aligned, as every workspace row is) so that no register or
+// dependent round trip is involved; the caller converts in place after a barrier.
+__device__ __forceinline__ void stage_raw(uint32_t *dst, const void *src, int n) {
+    const uint32_t *s32 = reinterpret_cast<const uint32_t *>(src);
+    const int n4 = n / 4;
+    for (int c = threadIdx.x; c < n4; c += kSelThreads) cp_async16(dst + 4 * c, s32 + 4 * c);
+    for (int i = 4 * n4 + (int)threadIdx.x; i < n; i += kSelThreads) dst[i] = __ldg(s32 + i);
+    cp_async_commit();
+    cp_async_wait_all();
 }
 
 __device__ __forceinline__ void sel_scan_warps(SelSmem &s) {
@@ -503,8 +495,9 @@ select_full_kernel(IndexArgs a) {
         const float *bm = a.bmax + (int64_t)qi * a.bmax_stride;
         const bool staged = nb <= kSelStageMax;
         if (staged) {
-            stage_keys<float>(s.keys, nb, [&](int i) { return __ldg(bm + i); },
-                              [&](int, float v) { return score_key(v); });
+            stage_raw(s.keys, bm, nb);
+            __syncthreads();
+            for (int i = threadIdx.x; i < nb; i += kSelThreads) s.keys[i] = score_key(__uint_as_float(s.keys[i]));
             __syncthreads();
         }
         auto bkey = [&](int i) -> uint32_t { return staged ? s.keys[i] : score_key(bm[i]); };
@@ -517,15 +510,17 @@ select_full_kernel(IndexArgs a) {
                 pool_out[i] = i < np ? s.pool[i] : -1;
         // candidates: the pool's positions, in ascending order
         const int nc = np * 8;
-        stage_keys<float>(s.keys, nc,
-            [&](int i) {   // a position past N (the pool's last block) is clamped, then dropped
-                const int64_t p = (int64_t)s.pool[i >> 3] * 8 + (i & 7);
-                return __ldg(scores + min64(p, (int64_t)N - 1));
-            },
-            [&](int i, float v) {
-                const int64_t p = (int64_t)s.pool[i >> 3] * 8 + (i & 7);
-                return p < N ? score_key(v) : 0u;
-            });
+        // gather the 8 scores of each pool block (32 B, inside the query's row even for
+        // the last, partial block), then convert; positions past N are dropped
+        for (int c = threadIdx.x; c < 2 * np; c += kSelThreads)
+            cp_async16(s.keys + 4 * c, scores + (int64_t)s.pool[c >> 1] * 8 + 4 * (c & 1));
+        cp_async_commit();
+        cp_async_wait_all();
+        __syncthreads();
+        for (int i = threadIdx.x; i < nc; i += kSelThreads) {
+            const int64_t p = (int64_t)s.pool[i >> 3] * 8 + (i & 7);
+            s.keys[i] = p < N ? score_key(__uint_as_float(s.keys[i])) : 0u;
+        }
         __syncthreads();
         auto ckey = [&](int i) -> uint32_t { return s.keys[i]; };
         auto cid = [&](int i) -> int { return s.pool[i >> 3] * 8 + (i & 7); };
@@ -533,8 +528,9 @@ select_full_kernel(IndexArgs a) {
     } else {
         const bool staged = N <= kSelStageMax;
         if (staged) {
-            stage_keys<float>(s.keys, N, [&](int i) { return __ldg(scores + i); },
-                              [&](int, float v) { return score_key(v); });
+            stage_raw(s.keys, scores, N);
+            __syncthreads();
+            for (int i = threadIdx.x; i < N; i += kSelThreads) s.keys[i] = score_key(__uint_as_float(s.keys[i]));
             __syncthreads();
         }
         auto key = [&](int i) -> uint32_t { return staged ? s.keys[i] : score_key(scores[i]); };
@@ -560,19 +556,23 @@ select_reindex_kernel(IndexArgs a) {
     const int32_t *pool = a.pool + (int64_t)qi * a.pool_blocks;
     const float *sc = a.scores + (int64_t)qi * a.score_stride;
     const int nc = a.pool_blocks * 8;
-    for (int i = threadIdx.x; i < a.pool_blocks; i += blockDim.x) {
-        const int blk = __ldg(pool + i);
-        s.pool[i] = blk;
-        if (i > 0 && blk >= 0 && __ldg(pool + i - 1) >= blk) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
+    // candidate scores and the pool, copied together, then converted in place
+    {
+        const uint32_t *p32 = reinterpret_cast<const uint32_t *>(pool);
+        const int n4 = (reinterpret_cast<uintptr_t>(pool) & 15) == 0 ? a.pool_blocks / 4 : 0;
+        for (int c = threadIdx.x; c < n4; c += kSelThreads)
+            cp_async16(reinterpret_cast<uint32_t *>(s.pool) + 4 * c, p32 + 4 * c);
+        for (int i = 4 * n4 + (int)threadIdx.x; i < a.pool_blocks; i += kSelThreads) s.pool[i] = __ldg(pool + i);
     }
-    // candidate c's score and its pool block are read together (no dependent round trip)
-    stage_keys<float2>(s.keys, nc,
-        [&](int i) { return make_float2(__int_as_float(__ldg(pool + (i >> 3))), __ldg(sc + i)); },
-        [&](int i, float2 r) {
-            const int blk = __float_as_int(r.x);
-            const int64_t p = (int64_t)blk * 8 + (i & 7);
-            return (blk >= 0 && p < N) ? score_key(r.y) : 0u;
-        });
+    stage_raw(s.keys, sc, nc);
+    __syncthreads();
+    for (int i = threadIdx.x; i < nc; i += kSelThreads) {
+        const int blk = s.pool[i >> 3];
+        const int64_t p = (int64_t)blk * 8 + (i & 7);
+        s.keys[i] = (blk >= 0 && p < N) ? score_key(__uint_as_float(s.keys[i])) : 0u;
+        if ((i & 7) == 0 && i > 0 && blk >= 0 && s.pool[(i >> 3) - 1] >= blk)
+            set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
+    }
     __syncthreads();
     auto key = [&](int i) -> uint32_t { return s.keys[i]; };
     auto id = [&](int i) -> int { return s.pool[i >> 3] * 8 + (i & 7); };
