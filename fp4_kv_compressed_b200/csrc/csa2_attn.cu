@@ -52,7 +52,7 @@ struct __align__(1024) Smem {
     uint8_t p[kHeads * 128];         // P fp16, [64 heads][64 keys] swizzled (K-major)
     int32_t ids[CSA2_TOPK_MAX];      // compacted selected entry ids
     float sig[2][kTK];               // per-key scale of each stage (1 FP4, sigma SWA, 0 none)
-    uint64_t kv_full[2], kv_empty[2], s_full[2], p_full, pv_done, drain, xfer[2];
+    uint64_t kv_lo[2], kv_hi[2], kv_empty[2], s_full[2], p_full, pv_done, drain, xfer[2];
     uint32_t tmem_base;
     int32_t abort;
     float wred[16];
@@ -232,9 +232,13 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 }
 
 // ---- producer: raw rows in registers -------------------------------------------------
+// Producer thread (row, quarter q) handles channels [64q, 64q + 64) of the low half
+// (channels 0-255) and [256 + 64q, 256 + 64q + 64) of the high half of one key, so
+// that a tile's low half can be complete (and its S MMAs start) before the high half.
 struct Raw {
-    uint4 c[8];      // FP4: c[0..3] = 64 code bytes (128 channels); SWA: 128 code bytes
-    uint2 s;         // FP4: 8 scale bytes of the 128 channels
+    uint4 c[8];      // FP4: c[0..1] low-half codes, c[2..3] high-half codes (32 B each);
+                     // SWA: c[0..3] low-half codes, c[4..7] high-half codes (64 B each)
+    uint2 s;         // FP4: 4 scale bytes of each half (x low, y high)
     float sigma;     // SWA scale
     int kind;        // 0 none, 1 FP4 entry, 2 SWA row
 };
@@ -247,41 +251,49 @@ __device__ __forceinline__ void load_raw(Raw &r, const AttnArgs &a, const int32_
     if (kg < n_sel) {
         const int e = ids[kg];
         const int64_t off = (int64_t)b * a.cap + e;
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.codes + off * kCodeBytes + 64 * quarter);
+        const uint8_t *codes = a.codes + off * kCodeBytes;
+        const uint8_t *scales = a.scales + off * kScaleBytes;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) r.c[i] = __ldg(src + i);
-        r.s = __ldg(reinterpret_cast<const uint2 *>(a.scales + off * kScaleBytes + 8 * quarter));
+        for (int h = 0; h < 2; ++h) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(codes + 128 * h + 32 * quarter);
+            r.c[2 * h] = __ldg(src);
+            r.c[2 * h + 1] = __ldg(src + 1);
+        }
+        r.s.x = __ldg(reinterpret_cast<const uint32_t *>(scales + 4 * quarter));
+        r.s.y = __ldg(reinterpret_cast<const uint32_t *>(scales + 16 + 4 * quarter));
         r.kind = 1;
     } else if (kg < n_keys) {
         const int64_t pos = w0 + (kg - n_sel);
         const int64_t slot = (int64_t)b * a.wcap + pos % a.wcap;
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.swa_codes + slot * kDim + 128 * quarter);
+        const uint8_t *codes = a.swa_codes + slot * kDim;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) r.c[i] = __ldg(src + i);
+        for (int h = 0; h < 2; ++h) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(codes + 256 * h + 64 * quarter);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) r.c[4 * h + i] = __ldg(src + i);
+        }
         r.sigma = __ldg(a.swa_scale + slot);
         r.kind = 2;
     }
 }
 
-// Dequantise the thread's 128 channels of one key into the fp16 tile.
-__device__ __forceinline__ void store_dequant(const Raw &r, uint8_t *tile, int row, int quarter,
-                                              int32_t *dev_err) {
-    const int ch0 = 128 * quarter;
+// Dequantise the thread's 64 channels of half h of one key into the fp16 tile.
+__device__ __forceinline__ void store_dequant_half(const Raw &r, uint8_t *tile, int row, int quarter,
+                                                   int h, int32_t *dev_err) {
+    const int ch0 = 256 * h + 64 * quarter;
     if (r.kind == 1) {
-        const uint32_t cw[16] = {r.c[0].x, r.c[0].y, r.c[0].z, r.c[0].w, r.c[1].x, r.c[1].y,
-                                 r.c[1].z, r.c[1].w, r.c[2].x, r.c[2].y, r.c[2].z, r.c[2].w,
-                                 r.c[3].x, r.c[3].y, r.c[3].z, r.c[3].w};
-        const uint32_t sc[2] = {r.s.x, r.s.y};
-        uint32_t scale2[8];                            // one f16x2 scale per 16 channels
+        const uint4 c0 = r.c[2 * h], c1 = r.c[2 * h + 1];
+        const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const uint32_t sw = h ? r.s.y : r.s.x;         // scales of channel groups 0..3 (16 each)
+        uint32_t scale2[4];                            // one f16x2 scale per 16 channels
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-            const uint32_t pair = (sc[g >> 1] >> (16 * (g & 1))) & 0xFFFFu;   // scales 2g, 2g+1
-            const uint32_t h = cvt_e4m3x2_f16x2(pair);
-            scale2[2 * g] = (h & 0xFFFFu) * 0x10001u;
-            scale2[2 * g + 1] = (h >> 16) * 0x10001u;
+        for (int g = 0; g < 2; ++g) {
+            const uint32_t hh = cvt_e4m3x2_f16x2((sw >> (16 * g)) & 0xFFFFu);
+            scale2[2 * g] = (hh & 0xFFFFu) * 0x10001u;
+            scale2[2 * g + 1] = (hh >> 16) * 0x10001u;
         }
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {                 // 8 channels per 32-bit code word
+        for (int u = 0; u < 8; ++u) {                  // 8 channels per 32-bit code word
             const __half2 sv = *reinterpret_cast<const __half2 *>(&scale2[u >> 1]);
             uint32_t v[4];
             cvt_e2m1x8_f16x2(cw[u], v);
@@ -290,15 +302,15 @@ __device__ __forceinline__ void store_dequant(const Raw &r, uint8_t *tile, int r
                 __half2 x = __hmul2(*reinterpret_cast<__half2 *>(&v[j]), sv);
                 v[j] = *reinterpret_cast<uint32_t *>(&x);
             }
-            *reinterpret_cast<uint4 *>(tile + tile_off(row, ch0 + 8 * u)) =
-                make_uint4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<uint4 *>(tile + tile_off(row, ch0 + 8 * u)) = make_uint4(v[0], v[1], v[2], v[3]);
         }
     } else if (r.kind == 2) {
         // exact E4M3 codes; the row scale is applied in fp32 on the logit and on P
-        if (quarter == 0 && r.sigma * 256.0f > 65504.0f) set_dev_err(dev_err, CSA2_DEVERR_RANGE);
+        if (h == 0 && quarter == 0 && r.sigma * 256.0f > 65504.0f) set_dev_err(dev_err, CSA2_DEVERR_RANGE);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t w4[4] = {r.c[i].x, r.c[i].y, r.c[i].z, r.c[i].w};
+        for (int i = 0; i < 4; ++i) {
+            const uint4 cv = r.c[4 * h + i];
+            const uint32_t w4[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
             for (int hu = 0; hu < 2; ++hu) {           // 8 channels
                 const uint32_t w0 = w4[2 * hu], w1 = w4[2 * hu + 1];
@@ -310,7 +322,7 @@ __device__ __forceinline__ void store_dequant(const Raw &r, uint8_t *tile, int r
     } else {
         const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) *reinterpret_cast<uint4 *>(tile + tile_off(row, ch0 + 8 * u)) = z;
+        for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4 *>(tile + tile_off(row, ch0 + 8 * u)) = z;
     }
 }
 
@@ -369,7 +381,8 @@ attn_tc_kernel(AttnArgs a) {
     // ---- set-up (all threads) -------------------------------------------------------------
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s.kv_full[i], 8);
+            mbar_init(&s.kv_lo[i], 8);
+            mbar_init(&s.kv_hi[i], 8);
             mbar_init(&s.kv_empty[i], 1);
             mbar_init(&s.s_full[i], 1);
         }
@@ -472,7 +485,7 @@ attn_tc_kernel(AttnArgs a) {
             const uint64_t kd1 = sw128_desc(smem_u32(s.kv[1]), 16, 1024);
             const uint64_t vd0 = sw128_desc(smem_u32(s.kv[0]), 8192, 1024);
             const uint64_t vd1 = sw128_desc(smem_u32(s.kv[1]), 8192, 1024);
-            int s_next = 0, pv_next = 0;
+            int s_next = 0, pv_next = 0, s_half = 0;
             uint64_t idle_since = wall_ns();
             bool stalled = false;
             while (pv_next < nt && !stalled) {
@@ -498,13 +511,15 @@ attn_tc_kernel(AttnArgs a) {
                     ++pv_next;
                     progressed = true;
                 }
+                // S(s_next) in two halves: channel quarters 0-1 once the tile's low half
+                // has landed, quarters 2-3 once its high half has
                 go = 0;
                 if (lane == 0)
                     go = s_next < nt && s_next <= pv_next + 1 &&
-                         mbar_test(&s.kv_full[s_next & 1], (s_next >> 1) & 1);
+                         mbar_test(s_half ? &s.kv_hi[s_next & 1] : &s.kv_lo[s_next & 1], (s_next >> 1) & 1);
                 if (__shfl_sync(0xFFFFFFFFu, go, 0)) {
                     tc_fence_after();
-                    // S as kSPart independent partial sums over channel slices, issued
+                    // S as kSPart independent partial sums over channel quarters, issued
                     // round-robin so that consecutive MMAs never share an accumulator
                     const uint32_t d = tmem + (16u << 16) + (uint32_t)(s_next & 1) * (kSPart * kTK);
                     const uint64_t kb = (s_next & 1) ? kd1 : kd0;
@@ -512,15 +527,17 @@ attn_tc_kernel(AttnArgs a) {
 #pragma unroll
                         for (int kk = 0; kk < 32 / kSPart; ++kk)
 #pragma unroll
-                            for (int pp = 0; pp < kSPart; ++pp) {
+                            for (int p2 = 0; p2 < kSPart / 2; ++p2) {
+                                const int pp = (kSPart / 2) * s_half + p2;
                                 const int k16 = pp * (32 / kSPart) + kk;      // K-step of 16 channels
                                 const uint64_t off = (uint64_t)((k16 >> 2) * 512 + (k16 & 3) * 2);  // 16-byte units
                                 mma_f16(d + (uint32_t)(pp * kTK), qd0 + off, kb + off, idesc_s, kk > 0);
                             }
-                        mma_commit(&s.s_full[s_next & 1]);
+                        if (s_half) mma_commit(&s.s_full[s_next & 1]);
                     }
                     __syncwarp();
-                    ++s_next;
+                    if (s_half) ++s_next;
+                    s_half ^= 1;
                     progressed = true;
                 }
                 if (progressed)
@@ -545,7 +562,7 @@ attn_tc_kernel(AttnArgs a) {
         bool ok = true;
         for (int i = 0; i < nt; ++i) {
             ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.s_full[i & 1], (i >> 1) & 1) &&
-                                             mbar_wait(&s.kv_full[i & 1], (i >> 1) & 1) && !aborted(s));
+                                             mbar_wait(&s.kv_hi[i & 1], (i >> 1) & 1) && !aborted(s));
             if (!ok) break;
             tc_fence_after();
             float x[32], sg[32];
@@ -643,12 +660,16 @@ attn_tc_kernel(AttnArgs a) {
                 ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.kv_empty[i & 1], ((i >> 1) - 1) & 1) && !aborted(s));
                 if (!ok) break;
             }
-            store_dequant(cur, s.kv[i & 1], row, quarter, a.dev_err);
+            store_dequant_half(cur, s.kv[i & 1], row, quarter, 0, a.dev_err);
             if (quarter == 0)
                 s.sig[i & 1][row] = cur.kind == 1 ? 1.0f : (cur.kind == 2 ? cur.sigma : 0.0f);
             fence_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s.kv_full[i & 1]);
+            if (lane == 0) mbar_arrive(&s.kv_lo[i & 1]);      // channels 0-255 of the tile ready
+            store_dequant_half(cur, s.kv[i & 1], row, quarter, 1, a.dev_err);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.kv_hi[i & 1]);      // channels 256-511 ready
         }
         if (!ok) {
             atomicExch(&s.abort, 1);
