@@ -21,9 +21,10 @@
 // logit and folded into P for the P V product.  Q is converted to fp16 after an exact
 // power-of-two scaling that keeps max|q| below 2^15.
 // TMEM (512 columns): O = 64 x 512 fp32 in lanes 0-15 of each quadrant (M = 64
-// layout); at lane offset 16, the two S buffers, each as 4 partial 64 x 64 fp32
-// accumulators over channel quarters (independent MMA chains that the tensor pipe
-// overlaps; the softmax adds them), columns 0..511.
+// layout); at lane offset 16, the two S buffers, each as 2 partial 64 x 64 fp32
+// accumulators over channel halves (the low half's MMAs start as soon as the
+// producers have written channels 0-255 of the tile; the softmax adds the two),
+// columns 0..255.
 // Online softmax in the log2 domain with lazy rescaling: O is rescaled only when
 // a head's running max grows by more than 8 (p stays <= 2^8, safe in fp16).
 // The MMA thread issues S(i+1) and P V(i) as soon as each is ready.  Every wait is
@@ -42,7 +43,7 @@ constexpr int kThreads = 512;
 constexpr int kTK = 64;                        // keys per tile
 constexpr int kHeads = 64;                     // heads per CTA (MMA M)
 constexpr uint32_t kTmemCols = 512;
-constexpr int kSPart = 4;                      // partial S accumulators per tile (K split)
+constexpr int kSPart = 2;                      // partial S accumulators per tile (K split)
 constexpr uint32_t kXferBytes = 32 * 256 * 4;  // half (32 heads) of one CTA's O for the peer
 constexpr uint64_t kWaitLimitNs = 500000000ull; // a wait gives up after 0.5 s of wall time
 
@@ -184,6 +185,20 @@ __device__ __forceinline__ void tmem_ld16x32(uint32_t taddr, float *v) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+
+// The same 16-column load without the wait: the caller issues several, then calls
+// tmem_wait_ld() once before reading any of the registers.
+template <int HALF>
+__device__ __forceinline__ void tmem_ld16x16_nw(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], %17;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr), "n"(HALF));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 template <int HALF>
 __device__ __forceinline__ void tmem_ld16x16(uint32_t taddr, float *v) {
@@ -511,16 +526,16 @@ attn_tc_kernel(AttnArgs a) {
                     ++pv_next;
                     progressed = true;
                 }
-                // S(s_next) in two halves: channel quarters 0-1 once the tile's low half
-                // has landed, quarters 2-3 once its high half has
+                // S(s_next) in two halves: the accumulators of channels 0-255 once the
+                // tile's low half has landed, those of channels 256-511 once its high half has
                 go = 0;
                 if (lane == 0)
                     go = s_next < nt && s_next <= pv_next + 1 &&
                          mbar_test(s_half ? &s.kv_hi[s_next & 1] : &s.kv_lo[s_next & 1], (s_next >> 1) & 1);
                 if (__shfl_sync(0xFFFFFFFFu, go, 0)) {
                     tc_fence_after();
-                    // S as kSPart independent partial sums over channel quarters, issued
-                    // round-robin so that consecutive MMAs never share an accumulator
+                    // S as kSPart partial sums over channel slices (kSPart / 2 per half),
+                    // issued round-robin over the half's accumulators
                     const uint32_t d = tmem + (16u << 16) + (uint32_t)(s_next & 1) * (kSPart * kTK);
                     const uint64_t kb = (s_next & 1) ? kd1 : kd0;
                     if (elect_one()) {
@@ -567,24 +582,32 @@ attn_tc_kernel(AttnArgs a) {
             tc_fence_after();
             float x[32], sg[32];
             {
+                // all partial sums of 16 columns are loaded, then waited for once
                 const uint32_t sb = s_lane + (uint32_t)(i & 1) * (kSPart * kTK);
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
-                    tmem_ld16x16<32>(sb + (uint32_t)(16 * c), x + 16 * c);
+                    uint32_t y[kSPart][16];
 #pragma unroll
-                    for (int pp = 1; pp < kSPart; ++pp) {
-                        float y[16];
-                        tmem_ld16x16<32>(sb + (uint32_t)(pp * kTK + 16 * c), y);
+                    for (int pp = 0; pp < kSPart; ++pp) tmem_ld16x16_nw<32>(sb + (uint32_t)(pp * kTK + 16 * c), y[pp]);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) x[16 * c + j] += y[j];
+                    for (int j = 0; j < 16; ++j) {
+                        float v = __uint_as_float(y[0][j]);
+#pragma unroll
+                        for (int pp = 1; pp < kSPart; ++pp) v += __uint_as_float(y[pp][j]);
+                        x[16 * c + j] = v;
                     }
                 }
             }
             const int key0 = (tile_lo + i) * kTK + 32 * half;
             float mt = -INFINITY;
 #pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+                const float4 g4 = reinterpret_cast<const float4 *>(&s.sig[i & 1][32 * half])[j4];
+                sg[4 * j4] = g4.x; sg[4 * j4 + 1] = g4.y; sg[4 * j4 + 2] = g4.z; sg[4 * j4 + 3] = g4.w;
+            }
+#pragma unroll
             for (int j = 0; j < 32; ++j) {
-                sg[j] = s.sig[i & 1][32 * half + j];
                 x[j] = (key0 + j < n_keys && sg[j] > 0.0f) ? x[j] * (c * sg[j]) : -INFINITY;
                 mt = fmaxf(mt, x[j]);
             }
