@@ -74,11 +74,11 @@ def attn_flops(wl) -> int:
 # sources at capture time).  Reported, each kernel scaled to the batch, only while the
 # sources are unchanged.  Captures: profiles/*.md.
 NCU_TRAFFIC = {
-    "csa2_sparse_attn_decode": ([(21_173_504 + 512, 64)], ("csa2_attn.cu",), "0bf47515333277dc"),
-    "csa2_index_full": ([(138_471_168 + 5_096_448, 8), (18_140_160, 64)], ("csa2_index.cu",),
-                        "9ad48d8576b5b662"),
-    "csa2_index_reindex": ([(18_626_560, 8), (4_748_544, 64)], ("csa2_index.cu",),
-                           "9ad48d8576b5b662"),
+    "csa2_sparse_attn_decode": ([(21_172_480 + 512, 64)], ("csa2_attn.cu",), "ae6bef53bbe04b82"),
+    "csa2_index_full": ([(138_484_992 + 4_945_664, 8), (18_141_952, 64)], ("csa2_index.cu",),
+                        "4bd071bde104eeff"),
+    "csa2_index_reindex": ([(18_606_080, 8), (4_754_432, 64)], ("csa2_index.cu",),
+                           "4bd071bde104eeff"),
 }
 
 
