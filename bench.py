@@ -75,6 +75,8 @@ def attn_flops(wl) -> int:
 # sources are unchanged.  Captures: profiles/*.md.
 NCU_TRAFFIC = {
     "csa2_sparse_attn_decode": ([(21_172_480 + 512, 64)], ("csa2_attn.cu",), "ae6bef53bbe04b82"),
+    "csa2_sparse_attn_decode_append": ([(21_172_480 + 512, 64)], ("csa2_attn.cu",),
+                                       "ae6bef53bbe04b82"),
     "csa2_index_full": ([(138_484_992 + 4_945_664, 8), (18_141_952, 64)], ("csa2_index.cu",),
                         "4bd071bde104eeff"),
     "csa2_index_reindex": ([(18_606_080, 8), (4_754_432, 64)], ("csa2_index.cu",),
@@ -113,7 +115,12 @@ def op_rooflines(wl, plan, op_ms: dict, ms_step: float) -> dict:
                                 "index_scan_kernel + select_full_kernel"),
             "csa2_index_reindex": (ob.get(f"index_reindex_g{dec}", 0), modes.count("X"),
                                    "reindex_score_kernel + select_reindex_kernel"),
-            "csa2_sparse_attn_decode": (ob["attn"], len(modes), "attn_tc_kernel")}
+            "csa2_sparse_attn_decode": (ob["attn"], len(modes), "attn_tc_kernel"),
+            # decode: every layer but a group's first appends its SWA row inside the
+            # attention launch
+            "csa2_sparse_attn_decode_append": (ob["attn"] + ob["swa_append"],
+                                               len(modes) - len({lp.group for lp in plan}),
+                                               "attn_tc_kernel (with the SWA append)")}
     out = {}
     for name, ms in op_ms.items():
         nbytes, n, kernels = spec[name]
@@ -129,7 +136,7 @@ def op_rooflines(wl, plan, op_ms: dict, ms_step: float) -> dict:
              "frac": gbs / pk["hbm_gbs"], "traffic": traffic, "kernels": kernels,
              "algorithmic_bytes_per_launch": nbytes, "launch_ms": ms, "launches_per_step": n,
              "share_of_step": n * ms / ms_step, "peak_source": pk["source"]}
-        if name == "csa2_sparse_attn_decode":
+        if name.startswith("csa2_sparse_attn_decode"):
             fl = attn_flops(wl)
             tfs = fl / (ms / 1e3) / 1e12
             e["tensor"] = {"achieved": tfs, "peak": pk["tflops"], "unit": "TFLOP/s",
@@ -377,9 +384,15 @@ def run_ours(args, rank, world, local_rank):
     # stream inside the timed graph: the Full op, the first Reindex op and the last
     # layer's attention.
     modes = [lp.mode for lp in st.plan]
+    # the last layer's attention: the fused SWA append + attention call in decode
+    if st._fuse_swa(wl.Tq):
+        n_attn = len(modes) - len({lp.group for lp in st.plan})
+        attn_pick = ("csa2_sparse_attn_decode_append", (n_attn, n_attn - 1))
+    else:
+        attn_pick = ("csa2_sparse_attn_decode", (len(modes), len(modes) - 1))
     picks = {"csa2_index_full": (modes.count("F"), 0),
              "csa2_index_reindex": (modes.count("X"), 0),
-             "csa2_sparse_attn_decode": (len(modes), len(modes) - 1)}
+             attn_pick[0]: attn_pick[1]}
     op_events = {name: [] for name in picks}
     originals = {name: getattr(stack_mod.bind, name) for name in picks}
 

@@ -28,7 +28,8 @@ DEVERR_SLOT, DEVERR_INDEX, DEVERR_NMAX, DEVERR_RANGE, DEVERR_TIMEOUT = 0x1, 0x2,
 # every symbol declared in include/csa2.h
 EXPORTS = ("csa2_quantize_append", "csa2_workspace_size", "csa2_index_full",
            "csa2_index_full_noalloc", "csa2_index_reindex", "csa2_sparse_attn_decode",
-           "csa2_read_device_error", "csa2_status_string", "csa2_abi_version")
+           "csa2_sparse_attn_decode_append", "csa2_read_device_error", "csa2_status_string",
+           "csa2_abi_version")
 
 
 class Csa2Error(RuntimeError):
@@ -69,12 +70,15 @@ def load_library(path: str = LIB_PATH):
     L.csa2_index_reindex.argtypes = [P, P, P, P, i32, i32, P, i32, i32, P, P, P, sz, P, P]
     L.csa2_sparse_attn_decode.argtypes = [P, P, P, P, i32, i32, P, i32, i32, C.c_float, P, P, P,
                                           sz, P, P]
+    L.csa2_sparse_attn_decode_append.argtypes = [P, P, P, P, P, i32, i32, P, i32, i32, C.c_float,
+                                                 P, P, P, sz, P, P]
     L.csa2_read_device_error.argtypes = [P, P, P]
     L.csa2_status_string.argtypes = [C.c_int]
     L.csa2_status_string.restype = C.c_char_p
     L.csa2_abi_version.restype = i32
     for fn in ("csa2_quantize_append", "csa2_index_full", "csa2_index_reindex",
-               "csa2_sparse_attn_decode", "csa2_read_device_error"):
+               "csa2_sparse_attn_decode", "csa2_sparse_attn_decode_append",
+               "csa2_read_device_error"):
         getattr(L, fn).restype = C.c_int
     _lib = L
     return L
@@ -146,6 +150,19 @@ def csa2_sparse_attn_decode(kv: CSA2GlobalKV, swa: CSA2SWA | None, q, q_pos, Tq:
                                    softmax_scale, _ptr(out), _ptr(lse), _ptr(workspace),
                                    ws_bytes, _ptr(dev_err), _stream(stream))
     _check("csa2_sparse_attn_decode", st)
+
+
+def csa2_sparse_attn_decode_append(kv: CSA2GlobalKV, swa: CSA2SWA, swa_bf16, q, q_pos, Tq: int,
+                                   H: int, topk, top_k: int, swa_len: int, softmax_scale: float,
+                                   out, lse, workspace=None, dev_err=None, stream=None):
+    """SWA append of the query token (Tq = 1) fused with csa2_sparse_attn_decode."""
+    L = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = L.csa2_sparse_attn_decode_append(C.byref(kv), C.byref(swa) if swa is not None else None,
+                                          _ptr(swa_bf16), _ptr(q), _ptr(q_pos), Tq, H, _ptr(topk),
+                                          top_k, swa_len, softmax_scale, _ptr(out), _ptr(lse),
+                                          _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream))
+    _check("csa2_sparse_attn_decode_append", st)
 
 
 def csa2_read_device_error(dev_err, stream=None) -> int:

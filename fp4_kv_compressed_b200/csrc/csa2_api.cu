@@ -240,14 +240,11 @@ csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16,
     return launched(launch_select_reindex(a, (int)BT, s));
 }
 
-csa2_status csa2_sparse_attn_decode(const csa2_global_kv *kv, const csa2_swa *swa,
-                                    const void *q_bf16, const int32_t *q_pos, int32_t Tq,
-                                    int32_t H, const int32_t *topk, int32_t top_k,
-                                    int32_t swa_len, float softmax_scale, float *out,
-                                    float *lse, void *workspace, size_t ws_bytes,
-                                    int32_t *dev_err, csa2_stream_t stream) {
-    (void)workspace;
-    (void)ws_bytes;
+static csa2_status sparse_attn(const csa2_global_kv *kv, const csa2_swa *swa, const void *swa_new_bf16,
+                               const void *q_bf16, const int32_t *q_pos, int32_t Tq, int32_t H,
+                               const int32_t *topk, int32_t top_k, int32_t swa_len,
+                               float softmax_scale, float *out, float *lse, int32_t *dev_err,
+                               csa2_stream_t stream) {
     csa2_status st = check_kv(kv, false);
     if (st != CSA2_OK) return st;
     if (!q_bf16 || !q_pos || !out || !lse) return CSA2_ERR_INVALID_ARG;
@@ -285,10 +282,39 @@ csa2_status csa2_sparse_attn_decode(const csa2_global_kv *kv, const csa2_swa *sw
     a.top_k = top_k;
     a.swa_len = swa_len;
     a.softmax_scale = softmax_scale;
+    a.swa_new = (const uint16_t *)swa_new_bf16;
     a.out = out;
     a.lse = lse;
     a.dev_err = dev_err;
     return launched(launch_sparse_attn(a, (int)BT, (cudaStream_t)stream));
+}
+
+csa2_status csa2_sparse_attn_decode(const csa2_global_kv *kv, const csa2_swa *swa,
+                                    const void *q_bf16, const int32_t *q_pos, int32_t Tq,
+                                    int32_t H, const int32_t *topk, int32_t top_k,
+                                    int32_t swa_len, float softmax_scale, float *out,
+                                    float *lse, void *workspace, size_t ws_bytes,
+                                    int32_t *dev_err, csa2_stream_t stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    return sparse_attn(kv, swa, nullptr, q_bf16, q_pos, Tq, H, topk, top_k, swa_len, softmax_scale,
+                       out, lse, dev_err, stream);
+}
+
+csa2_status csa2_sparse_attn_decode_append(const csa2_global_kv *kv, const csa2_swa *swa,
+                                           const void *swa_bf16, const void *q_bf16,
+                                           const int32_t *q_pos, int32_t Tq, int32_t H,
+                                           const int32_t *topk, int32_t top_k, int32_t swa_len,
+                                           float softmax_scale, float *out, float *lse,
+                                           void *workspace, size_t ws_bytes, int32_t *dev_err,
+                                           csa2_stream_t stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    if (Tq != 1) return CSA2_ERR_UNSUPPORTED;
+    if (swa_len <= 0 || !swa || !swa_bf16) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(swa_bf16, 16)) return CSA2_ERR_INVALID_ARG;
+    return sparse_attn(kv, swa, swa_bf16, q_bf16, q_pos, Tq, H, topk, top_k, swa_len, softmax_scale,
+                       out, lse, dev_err, stream);
 }
 
 csa2_status csa2_read_device_error(int32_t *dev_err, int32_t *bits_out, csa2_stream_t stream) {

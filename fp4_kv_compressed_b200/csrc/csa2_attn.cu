@@ -53,6 +53,8 @@ struct __align__(1024) Smem {
     uint8_t p[kHeads * 128];         // P fp16, [64 heads][64 keys] swizzled (K-major)
     int32_t ids[CSA2_TOPK_MAX];      // compacted selected entry ids
     float sig[2][kTK];               // per-key scale of each stage (1 FP4, sigma SWA, 0 none)
+    alignas(16) uint8_t swa_new[kDim];   // fused append: the query token's new SWA row (E4M3)
+    float swa_new_sigma;
     uint64_t kv_lo[2], kv_hi[2], kv_empty[2], s_full[2], p_full, pv_done, drain, xfer[2];
     uint32_t tmem_base;
     int32_t abort;
@@ -258,9 +260,11 @@ struct Raw {
     int kind;        // 0 none, 1 FP4 entry, 2 SWA row
 };
 
+// new_row / new_sigma: the window's newest row already quantised in shared memory
+// (fused append), or null.
 __device__ __forceinline__ void load_raw(Raw &r, const AttnArgs &a, const int32_t *ids, int n_sel,
                                          int b, int64_t w0, int n_keys, int tile, int row,
-                                         int quarter) {
+                                         int quarter, const uint8_t *new_row, float new_sigma) {
     const int kg = tile * kTK + row;
     r.kind = 0;
     if (kg < n_sel) {
@@ -277,6 +281,15 @@ __device__ __forceinline__ void load_raw(Raw &r, const AttnArgs &a, const int32_
         r.s.x = __ldg(reinterpret_cast<const uint32_t *>(scales + 4 * quarter));
         r.s.y = __ldg(reinterpret_cast<const uint32_t *>(scales + 16 + 4 * quarter));
         r.kind = 1;
+    } else if (kg < n_keys && new_row != nullptr && kg == n_keys - 1) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(new_row + 256 * h + 64 * quarter);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) r.c[4 * h + i] = src[i];
+        }
+        r.sigma = new_sigma;
+        r.kind = 2;
     } else if (kg < n_keys) {
         const int64_t pos = w0 + (kg - n_sel);
         const int64_t slot = (int64_t)b * a.wcap + pos % a.wcap;
@@ -428,6 +441,14 @@ attn_tc_kernel(AttnArgs a) {
     const bool e_ok = e_id >= 0 && e_id < n_vis;
     if (e_id >= 0 && !e_ok) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
     const uint32_t bal = __ballot_sync(0xFFFFFFFFu, e_ok);
+    // fused SWA append (decode, Tq = 1): warp 1 reads the token's new bf16 row now
+    const bool fuse = a.swa_new != nullptr && n_win > 0;
+    float xnew[16];
+    if (fuse && warp == 1) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.swa_new + (int64_t)qi * kDim + 16 * lane);
+        unpack_bf16x8(__ldg(src), xnew);
+        unpack_bf16x8(__ldg(src + 1), xnew + 8);
+    }
     // Q chunks of 8 channels: thread t holds chunks t + 512 j
     const uint16_t *q = a.q + ((int64_t)qi * a.H + h0) * kDim;
     uint4 qv[8];
@@ -457,6 +478,22 @@ attn_tc_kernel(AttnArgs a) {
         qmax = fmaxf(qmax, s.wred[w]);
     }
     if (e_ok) s.ids[base + __popc(bal & ((1u << lane) - 1u))] = e_id;
+    if (fuse && warp == 1) {
+        // The same FP8 row quantiser as csa2_quantize_append: codes and sigma go to
+        // shared memory (this CTA's producers read the window's newest key from there)
+        // and, from head group 0's CTA that owns that key, to the ring slot t % wcap.
+        quant_fp8_lanes<kDim>(xnew, s.swa_new, &s.swa_new_sigma, lane);
+        const int last_tile = (n_sel + n_win - 1) / kTK;
+        const int n_all0 = (n_sel + n_win + kTK - 1) / kTK;
+        const uint32_t owner = last_tile < (n_all0 + 1) / 2 ? 0u : 1u;
+        __syncwarp();
+        if (blockIdx.y == 0 && rank == owner) {
+            const int64_t slot = (int64_t)b * a.wcap + t % a.wcap;
+            reinterpret_cast<uint4 *>(a.swa_codes + slot * kDim)[lane] =
+                reinterpret_cast<const uint4 *>(s.swa_new)[lane];
+            if (lane == 0) a.swa_scale[slot] = s.swa_new_sigma;
+        }
+    }
     const int qexp = qmax > 0.0f ? max(0, ilogbf(qmax) - 14) : 0;   // max|q| * 2^-qexp < 2^15
     {
         const float inv = exp2f((float)-qexp);
@@ -674,11 +711,13 @@ attn_tc_kernel(AttnArgs a) {
         const int pt = threadIdx.x - 256;
         const int row = pt >> 2, quarter = pt & 3;
         Raw cur, nxt;
-        if (nt > 0) load_raw(nxt, a, s.ids, n_sel, b, w0, n_keys, tile_lo, row, quarter);
+        const uint8_t *new_row = fuse ? s.swa_new : nullptr;
+        const float new_sigma = fuse ? s.swa_new_sigma : 0.0f;
+        if (nt > 0) load_raw(nxt, a, s.ids, n_sel, b, w0, n_keys, tile_lo, row, quarter, new_row, new_sigma);
         bool ok = true;
         for (int i = 0; i < nt; ++i) {
             cur = nxt;
-            if (i + 1 < nt) load_raw(nxt, a, s.ids, n_sel, b, w0, n_keys, tile_lo + i + 1, row, quarter);
+            if (i + 1 < nt) load_raw(nxt, a, s.ids, n_sel, b, w0, n_keys, tile_lo + i + 1, row, quarter, new_row, new_sigma);
             if (i >= 2) {
                 ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.kv_empty[i & 1], ((i >> 1) - 1) & 1) && !aborted(s));
                 if (!ok) break;

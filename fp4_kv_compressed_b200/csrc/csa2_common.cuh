@@ -96,6 +96,72 @@ __device__ __forceinline__ float key_to_score(uint32_t k) {
     return __uint_as_float(u);
 }
 
+__device__ __forceinline__ void unpack_bf16x8(uint4 v, float *x) {
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
+        x[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+    }
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+// FP8 row of WIDTH channels (64, 128 or 512), one warp: sigma = amax / 448 (IEEE
+// division), codes = E4M3_RNE_satfinite(x / sigma), a zero row stores zero codes.
+// quant_fp8_lanes takes the lane's PER = WIDTH / 32 consecutive channels already in
+// registers (lane l holds channels PER l ..); quant_fp8_row loads them first.
+template <int WIDTH>
+__device__ void quant_fp8_lanes(const float *x, uint8_t *dst_codes, float *dst_scale, int lane) {
+    constexpr int PER = WIDTH / 32;      // channels per lane: 2, 4 or 16
+    float amax = 0.0f;
+#pragma unroll
+    for (int c = 0; c < PER; ++c) amax = fmaxf(amax, fabsf(x[c]));
+    amax = warp_max(amax);
+    const float sigma = __fdiv_rn(amax, 448.0f);
+    uint32_t pk[PER / 2];
+#pragma unroll
+    for (int j = 0; j < PER / 2; ++j)
+        pk[j] = sigma != 0.0f ? cvt_e4m3x2(__fdiv_rn(x[2 * j], sigma), __fdiv_rn(x[2 * j + 1], sigma))
+                              : 0u;
+    if constexpr (PER == 16) {
+        uint4 o = make_uint4(pk[0] | (pk[1] << 16), pk[2] | (pk[3] << 16), pk[4] | (pk[5] << 16),
+                             pk[6] | (pk[7] << 16));
+        reinterpret_cast<uint4 *>(dst_codes)[lane] = o;
+    } else if constexpr (PER == 4) {
+        reinterpret_cast<uint32_t *>(dst_codes)[lane] = pk[0] | (pk[1] << 16);
+    } else {
+        reinterpret_cast<uint16_t *>(dst_codes)[lane] = (uint16_t)pk[0];
+    }
+    if (lane == 0) *dst_scale = sigma;
+}
+
+template <int WIDTH>
+__device__ void quant_fp8_row(const uint16_t *src, uint8_t *dst_codes, float *dst_scale, int lane) {
+    constexpr int PER = WIDTH / 32;      // channels per lane: 2, 4 or 16
+    float x[PER];
+    if constexpr (PER == 16) {
+        const uint4 *s4 = reinterpret_cast<const uint4 *>(src + 16 * lane);
+        unpack_bf16x8(s4[0], x);
+        unpack_bf16x8(s4[1], x + 8);
+    } else if constexpr (PER == 4) {
+        uint2 v = reinterpret_cast<const uint2 *>(src)[lane];
+        x[0] = bf16_bits_to_f32(v.x & 0xFFFFu);
+        x[1] = bf16_bits_to_f32(v.x >> 16);
+        x[2] = bf16_bits_to_f32(v.y & 0xFFFFu);
+        x[3] = bf16_bits_to_f32(v.y >> 16);
+    } else {
+        uint32_t v = reinterpret_cast<const uint32_t *>(src)[lane];
+        x[0] = bf16_bits_to_f32(v & 0xFFFFu);
+        x[1] = bf16_bits_to_f32(v >> 16);
+    }
+    quant_fp8_lanes<WIDTH>(x, dst_codes, dst_scale, lane);
+}
+
 // Programmatic dependent launch.  Every kernel of the library is launched so that the
 // next kernel of the stream may be scheduled while it finishes: grid_dep_wait() blocks
 // until the previous grid has completed with its memory visible (each kernel calls it

@@ -60,9 +60,10 @@ struct AttnArgs {
     const uint8_t *scales;
     int32_t cap;
     int32_t ratio;
-    const uint8_t *swa_codes;
-    const float *swa_scale;
+    uint8_t *swa_codes;      // written only by the fused append (swa_new != null)
+    float *swa_scale;
     int32_t wcap;
+    const uint16_t *swa_new; // fused append: [BT][512] bf16 new SWA row per query (Tq = 1), or null
     const uint16_t *q;       // [BT][H][512] bf16 bits
     const int32_t *q_pos;
     int32_t Tq;

@@ -163,7 +163,7 @@ class DecodeStack:
                 bind.csa2_quantize_append(kv.struct, kv_bf16[g], idxk_bf16[g], T_kv, kv_start[g],
                                        self.swa[l].struct, swa_bf16[l], T_swa, swa_start,
                                        self.dev_err, stream)
-            elif swa_bf16[l] is not None:
+            elif swa_bf16[l] is not None and not self._fuse_swa(T_swa):
                 bind.csa2_quantize_append(None, None, None, 0, None, self.swa[l].struct,
                                        swa_bf16[l], T_swa, swa_start, self.dev_err, stream)
             spec = self.groups[g]
@@ -176,17 +176,34 @@ class DecodeStack:
                 bind.csa2_index_reindex(kv.struct, q_idx[l], w[l], q_pos, self.Tq, self.H_I,
                                      self.pool[g], spec.pool_blocks, self.top_k, self.topk[l],
                                      self.count[l], self.workspace, self.dev_err, stream)
-            bind.csa2_sparse_attn_decode(kv.struct, self.swa[l].struct, q[l], q_pos, self.Tq, self.H,
-                                      self.topk_of(l), self.top_k, self.swa_len,
-                                      self.softmax_scale, self.out[l], self.lse[l],
-                                      self.workspace, self.dev_err, stream)
+            fused = (l != first_of_group[g] or kv_bf16 is None or kv_bf16[g] is None) \
+                and swa_bf16[l] is not None and self._fuse_swa(T_swa)
+            if fused:       # the layer's SWA row is appended inside the attention launch
+                bind.csa2_sparse_attn_decode_append(
+                    kv.struct, self.swa[l].struct, swa_bf16[l], q[l], q_pos, self.Tq, self.H,
+                    self.topk_of(l), self.top_k, self.swa_len, self.softmax_scale, self.out[l],
+                    self.lse[l], self.workspace, self.dev_err, stream)
+            else:
+                bind.csa2_sparse_attn_decode(kv.struct, self.swa[l].struct, q[l], q_pos, self.Tq,
+                                          self.H, self.topk_of(l), self.top_k, self.swa_len,
+                                          self.softmax_scale, self.out[l], self.lse[l],
+                                          self.workspace, self.dev_err, stream)
+
+    def _fuse_swa(self, T_swa: int) -> bool:
+        """Decode (one query token, its own SWA row): the append runs inside the
+        attention launch (csa2_sparse_attn_decode_append)."""
+        return self.Tq == 1 and T_swa == 1 and self.swa_len > 0
 
     def launches_per_step(self, append: bool = True) -> int:
-        """Kernels one step() launches."""
+        """Kernels one step() launches (with new entries appended)."""
         n = 0
+        first = {}
         for lp in self.plan:
-            n += 1                     # quantise-append (SWA row, plus the group's entry)
+            first.setdefault(lp.group, lp.layer)
+        for lp in self.plan:
+            if lp.layer == first[lp.group] or not self._fuse_swa(self.Tq):
+                n += 1                 # quantise-append (the group's entry and/or SWA rows)
             n += {"F": 2, "X": 2, "U": 0}[lp.mode]
-            n += 1                     # attention
+            n += 1                     # attention (with the fused SWA append in decode)
         return n
 

@@ -231,6 +231,28 @@ CSA2_API csa2_status csa2_sparse_attn_decode(const csa2_global_kv *kv, const csa
                                     float *lse, void *workspace, size_t ws_bytes,
                                     int32_t *dev_err, csa2_stream_t stream);
 
+/*
+ * a2 + a8 fused for decode (Tq = 1): the SWA append of the query token followed by
+ * the sparse attention, in one launch.  Equivalent to
+ *   csa2_quantize_append(NULL, ..., swa, swa_bf16, 1, q_pos, ...)   (the ring row of
+ *       token t = q_pos[b] at slot t % window_cap, FP8 with sigma = amax / 448)
+ *   csa2_sparse_attn_decode(kv, swa, q_bf16, q_pos, 1, ...)
+ * with the same ring bytes and the same outputs bit for bit (the kernel quantises the
+ * row with the same routine and uses it directly as the window's newest key).  The
+ * SWA row is the layer's own (DeepSeek V4.1 Flash study notes, section 1: each
+ * layer keeps its own 128-token window); the pages define no fused form.
+ *   swa_bf16 [B][512] bf16 (16-byte aligned), Tq must be 1 (else
+ *   CSA2_ERR_UNSUPPORTED), swa_len >= 1 and swa non-NULL (else CSA2_ERR_INVALID_ARG);
+ *   every other argument as for csa2_sparse_attn_decode.
+ */
+CSA2_API csa2_status csa2_sparse_attn_decode_append(const csa2_global_kv *kv, const csa2_swa *swa,
+                                           const void *swa_bf16, const void *q_bf16,
+                                           const int32_t *q_pos, int32_t Tq, int32_t H,
+                                           const int32_t *topk, int32_t top_k, int32_t swa_len,
+                                           float softmax_scale, float *out, float *lse,
+                                           void *workspace, size_t ws_bytes, int32_t *dev_err,
+                                           csa2_stream_t stream);
+
 /* Synchronise `stream`, read *dev_err (device int32) into *bits_out (host),
  * reset it to 0, and return CSA2_ERR_DEVICE_BOUNDS if any bit was set. */
 CSA2_API csa2_status csa2_read_device_error(int32_t *dev_err, int32_t *bits_out, csa2_stream_t stream);

@@ -71,6 +71,16 @@ def test_validation_rejects_before_launch(pkg):
                                        C.c_float(0.04), qbuf, qbuf, None, 0, None, None) == 4
     assert lib.csa2_sparse_attn_decode(C.byref(kv), C.byref(swa), qbuf, qbuf, 4, 64, qbuf, 8, 128,
                                        C.c_float(0.04), qbuf, qbuf, None, 0, None, None) == 2
+    # fused append + attention: decode only (Tq = 1), needs the ring and the new row
+    assert lib.csa2_sparse_attn_decode_append(C.byref(kv), C.byref(swa), qbuf, qbuf, qbuf, 2, 64,
+                                              qbuf, 8, 128, C.c_float(0.04), qbuf, qbuf, None, 0,
+                                              None, None) == 4
+    assert lib.csa2_sparse_attn_decode_append(C.byref(kv), None, qbuf, qbuf, qbuf, 1, 64, qbuf,
+                                              8, 128, C.c_float(0.04), qbuf, qbuf, None, 0, None,
+                                              None) == 1
+    assert lib.csa2_sparse_attn_decode_append(C.byref(kv), C.byref(swa), C.c_void_p(4100), qbuf,
+                                              qbuf, 1, 64, qbuf, 8, 128, C.c_float(0.04), qbuf,
+                                              qbuf, None, 0, None, None) == 1
     # append: slot count beyond the cache
     assert lib.csa2_quantize_append(C.byref(kv), qbuf, None, 101, qbuf, None, None, 0, None,
                                     None, None) == 2

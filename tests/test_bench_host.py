@@ -100,18 +100,20 @@ def test_op_rooflines_dominant_and_traffic():
     from fp4_kv_compressed_b200.stack import plan_layers
     wl = WORKLOADS["decode_128k"]
     plan = plan_layers([g.schedule for g in wl.groups])
-    op_ms = {"csa2_index_full": 0.4, "csa2_index_reindex": 0.1, "csa2_sparse_attn_decode": 0.03}
+    op_ms = {"csa2_index_full": 0.4, "csa2_index_reindex": 0.1,
+             "csa2_sparse_attn_decode_append": 0.03}
     ops = bench.op_rooflines(wl, plan, op_ms, ms_step=1.5)
     f = ops["csa2_index_full"]
     assert f["launches_per_step"] == 1 and f["bound"] == "hbm"
     assert abs(f["achieved"] - 1_154_155_776 / 0.4e-3 / 1e9) < 1e-6
     assert abs(f["share_of_step"] - 0.4 / 1.5) < 1e-12
-    a = ops["csa2_sparse_attn_decode"]
-    assert a["launches_per_step"] == 20 and abs(a["share_of_step"] - 0.4) < 1e-12
+    a = ops["csa2_sparse_attn_decode_append"]
+    assert a["launches_per_step"] == 19 and abs(a["share_of_step"] - 19 * 0.03 / 1.5) < 1e-12
+    assert a["algorithmic_bytes_per_launch"] == bench.op_bytes(wl)["attn"] + 64 * (1024 + 516)
     assert a["tensor"]["flops_per_launch"] == 64 * 4 * 64 * 512 * 640
     assert ops["csa2_index_reindex"]["launches_per_step"] == 4
     for name, e in ops.items():
         caps, files, sha = bench.NCU_TRAFFIC[name]
         expect = sum(tb * wl.B / b for tb, b in caps) if bench._sources_hash(files) == sha else None
         assert e["traffic"] == expect
-    assert max(ops, key=lambda n: ops[n]["share_of_step"]) == "csa2_sparse_attn_decode"
+    assert max(ops, key=lambda n: ops[n]["share_of_step"]) == "csa2_sparse_attn_decode_append"

@@ -142,3 +142,50 @@ def test_stack_scaled_channels(pkg):
     """Per-channel log-uniform scales on the main KV and SWA (the 128K workload's inputs)."""
     _stack_check(small_variant(WORKLOADS["decode_128k"], B=2, ctx=5000), [1],
                  layers=[0, 3, 4, 19])
+
+
+def test_fused_swa_append_matches_separate(pkg):
+    """csa2_sparse_attn_decode_append == csa2_quantize_append (SWA row) followed by
+    csa2_sparse_attn_decode: the same ring bytes and the same outputs, bit for bit,
+    for H = 64 and H = 128 (two head groups), and at a position where the window is
+    still filling (t < swa_len - 1)."""
+    import synth
+    for H, t_last in ((64, 2999), (128, 2999), (64, 40)):
+        B, cap, W = 3, 3000, 160
+        kv = pkg.GlobalKV(B, cap, 128, 1, "cuda")
+        x = torch.stack([synth.rows_normal_bf16(31, "kv", b, 0, cap, 512) for b in range(B)])
+        z = torch.zeros(B, dtype=torch.int32, device="cuda")
+        pkg.csa2_quantize_append(kv.struct, x.cuda(), None, cap, z, None, None, 0, None)
+        rings = [pkg.SwaRing(B, W, "cuda") for _ in range(2)]
+        n_old = min(t_last, W - 1)          # the ring holds the previous W - 1 tokens
+        p_old = t_last - n_old
+        old = torch.stack([synth.rows_normal_bf16(32, "swa", b, p_old, n_old, 512) for b in range(B)])
+        s_old = torch.full((B,), p_old, dtype=torch.int32, device="cuda")
+        if n_old > 0:
+            for r in rings:
+                pkg.csa2_quantize_append(None, None, None, 0, None, r.struct, old.cuda(), n_old, s_old)
+        new = torch.stack([synth.rows_normal_bf16(33, "new", b, 0, 1, 512) for b in range(B)]).cuda()
+        q = torch.stack([synth.rows_normal_bf16(34, "q", b, 0, H, 512, stride=synth.Q_STRIDE)
+                         for b in range(B)]).view(B, 1, H, 512).cuda()
+        q_pos = torch.full((B, 1), t_last, dtype=torch.int32, device="cuda")
+        g = torch.Generator().manual_seed(35)
+        vis = min(t_last + 1, cap)
+        topk = torch.stack([torch.sort(torch.randperm(vis, generator=g)[:min(512, vis)]).values
+                            for _ in range(B)]).view(B, 1, -1).int().cuda()
+        K = topk.shape[-1]
+        outs = [torch.zeros(B, 1, H, 512, device="cuda") for _ in range(2)]
+        lses = [torch.zeros(B, 1, H, device="cuda") for _ in range(2)]
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        start = torch.full((B,), t_last, dtype=torch.int32, device="cuda")
+        pkg.csa2_quantize_append(None, None, None, 0, None, rings[0].struct, new.view(B, 1, 512), 1,
+                                 start, err)
+        pkg.csa2_sparse_attn_decode(kv.struct, rings[0].struct, q, q_pos, 1, H, topk, K, 128,
+                                    512 ** -0.5, outs[0], lses[0], None, err)
+        pkg.csa2_sparse_attn_decode_append(kv.struct, rings[1].struct, new, q, q_pos, 1, H, topk, K,
+                                           128, 512 ** -0.5, outs[1], lses[1], None, err)
+        torch.cuda.synchronize()
+        assert pkg.csa2_read_device_error(err) == 0
+        assert torch.equal(rings[0].codes, rings[1].codes)
+        assert torch.equal(rings[0].scale.view(torch.int32), rings[1].scale.view(torch.int32))
+        assert torch.equal(outs[0].view(torch.int32), outs[1].view(torch.int32))
+        assert torch.equal(lses[0].view(torch.int32), lses[1].view(torch.int32))
