@@ -431,32 +431,41 @@ attn_tc_kernel(AttnArgs a) {
     // barriers and TMEM above touch no global memory; everything below may read what the
     // previous kernel of the stream wrote
     grid_dep_wait();
-    const int64_t t = a.q_pos[qi];
-    const int64_t w0 = max64(0, t - a.swa_len + 1);
-    const int n_win = a.swa_len > 0 ? (int)(t - w0 + 1) : 0;
-    const int64_t n_vis = min64(visible_entries((int32_t)t, a.ratio), a.cap);
-    // selected ids: thread t checks topk[t]; valid ids are compacted in order
+    // every independent global load first (one memory round trip): the position, this
+    // thread's Top-K entry, its Q chunks and (warp 1, fused append) the new SWA row
+    const int32_t t32 = a.q_pos[qi];
     const int32_t *tk = a.topk + (int64_t)qi * a.top_k;
     const int e_id = (int)threadIdx.x < a.top_k ? tk[threadIdx.x] : -1;
-    const bool e_ok = e_id >= 0 && e_id < n_vis;
-    if (e_id >= 0 && !e_ok) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
-    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, e_ok);
-    // fused SWA append (decode, Tq = 1): warp 1 reads the token's new bf16 row now
-    const bool fuse = a.swa_new != nullptr && n_win > 0;
-    float xnew[16];
-    if (fuse && warp == 1) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.swa_new + (int64_t)qi * kDim + 16 * lane);
-        unpack_bf16x8(__ldg(src), xnew);
-        unpack_bf16x8(__ldg(src + 1), xnew + 8);
-    }
     // Q chunks of 8 channels: thread t holds chunks t + 512 j
     const uint16_t *q = a.q + ((int64_t)qi * a.H + h0) * kDim;
     uint4 qv[8];
-    float qm = 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int i = threadIdx.x + kThreads * j;
         qv[j] = (i / 64 < hcta) ? __ldg(reinterpret_cast<const uint4 *>(q) + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    uint4 xraw[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+    if (a.swa_new != nullptr && warp == 1) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.swa_new + (int64_t)qi * kDim + 16 * lane);
+        xraw[0] = __ldg(src);
+        xraw[1] = __ldg(src + 1);
+    }
+    const int64_t t = t32;
+    const int64_t w0 = max64(0, t - a.swa_len + 1);
+    const int n_win = a.swa_len > 0 ? (int)(t - w0 + 1) : 0;
+    const int64_t n_vis = min64(visible_entries((int32_t)t, a.ratio), a.cap);
+    // selected ids: thread t checks topk[t]; valid ids are compacted in order
+    const bool e_ok = e_id >= 0 && e_id < n_vis;
+    if (e_id >= 0 && !e_ok) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
+    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, e_ok);
+    // fused SWA append (decode, Tq = 1): the token's new bf16 row, read above by warp 1
+    const bool fuse = a.swa_new != nullptr && n_win > 0;
+    float xnew[16];
+    unpack_bf16x8(xraw[0], xnew);
+    unpack_bf16x8(xraw[1], xnew + 8);
+    float qm = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
         const uint32_t w[4] = {qv[j].x, qv[j].y, qv[j].z, qv[j].w};
 #pragma unroll
         for (int k = 0; k < 4; ++k)
