@@ -74,9 +74,8 @@ def attn_flops(wl) -> int:
 # sources at capture time).  Reported, each kernel scaled to the batch, only while the
 # sources are unchanged.  Captures: profiles/*.md.
 NCU_TRAFFIC = {
-    "csa2_sparse_attn_decode": ([(21_172_480 + 512, 64)], ("csa2_attn.cu",), "ae6bef53bbe04b82"),
-    "csa2_sparse_attn_decode_append": ([(21_172_480 + 512, 64)], ("csa2_attn.cu",),
-                                       "ae6bef53bbe04b82"),
+    "csa2_sparse_attn_decode": ([(21_212_416, 64)], ("csa2_attn.cu",), "c63fd92c20f73652"),
+    "csa2_sparse_attn_decode_append": ([(21_212_416, 64)], ("csa2_attn.cu",), "c63fd92c20f73652"),
     "csa2_index_full": ([(138_484_992 + 4_945_664, 8), (18_141_952, 64)], ("csa2_index.cu",),
                         "4bd071bde104eeff"),
     "csa2_index_reindex": ([(18_606_080, 8), (4_754_432, 64)], ("csa2_index.cu",),
