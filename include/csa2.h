@@ -23,7 +23,12 @@
  *  - Bounds the host cannot see (device-resident positions, indices) are checked
  *    in the kernels: a violating row / index is skipped and a CSA2_DEVERR_* bit
  *    is OR-ed into `*dev_err` (an int32 in device memory, may be NULL).  Read it
- *    with csa2_read_device_error().  Kernels never trap and never spin.
+ *    with csa2_read_device_error().  Kernels never trap; their internal waits
+ *    are bounded (0.5 s of wall time) and report CSA2_DEVERR_TIMEOUT.
+ *  - Kernels are launched with programmatic dependent launch: each may be
+ *    scheduled while the previous kernel of the stream finishes, but waits for it
+ *    (completion and memory visibility) before its first global memory access, so
+ *    results are stream-ordered exactly as with ordinary launches.
  *  - bf16 inputs are row-major and contiguous; "B" is the request count, "Tq"
  *    the number of query tokens per request (1 = decode, >1 = prefill chunk).
  *  - Numbers are finite: NaN/Inf inputs are outside the contract.
