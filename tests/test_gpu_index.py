@@ -168,3 +168,75 @@ def test_scores_wide_dynamic_range(harness, orc, qscale):
     got = ws.view(torch.float32)[:N].cpu().numpy()
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
     assert np.array_equal(topk[0, 0].cpu().numpy(), orc.select_topk(ref, 64))
+
+
+def _index_case(pkg, orc, rows, ratio, q_pos, pool_blocks, top_k, H_I=4, seed=41):
+    """Runs csa2_index_full over per-request index-K rows [B][N][d] and compares pool,
+    Top-K and counts with the oracle, bit for bit."""
+    import synth
+    B, N, d = rows.shape
+    kv = pkg.GlobalKV(B, N, d, ratio, "cuda")
+    z = torch.zeros(B, dtype=torch.int32, device="cuda")
+    pkg.csa2_quantize_append(kv.struct, None, rows.cuda(), N, z, None, None, 0, None)
+    q = torch.stack([synth.rows_normal_bf16(seed, "q", b, 0, H_I, d) for b in range(B)]).view(B, 1, H_I, d)
+    w = torch.stack([synth.rows_uniform_f32(seed, "w", b, 0, 1, H_I) for b in range(B)]).view(B, 1, H_I)
+    qp = torch.tensor(q_pos, dtype=torch.int32).view(B, 1)
+    P = max(pool_blocks, 1)
+    pool = torch.full((B, 1, P), -1, dtype=torch.int32, device="cuda")
+    topk = torch.full((B, 1, top_k), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((B, 1), -7, dtype=torch.int32, device="cuda")
+    ws = torch.empty(pkg.csa2_workspace_size(pkg.CSA2_OP_INDEX_FULL, B, 1, N, 0, top_k, pool_blocks),
+                     dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkg.csa2_index_full(kv.struct, q.cuda(), w.cuda(), qp.cuda(), 1, H_I, N, pool_blocks, top_k,
+                        pool if pool_blocks else None, topk, cnt, ws, err)
+    torch.cuda.synchronize()
+    assert pkg.csa2_read_device_error(err) == 0
+    kc, ks = orc.quantize_fp8(rows.reshape(B * N, d))
+    p_ref, t_ref, n_ref = orc.index_full(kc.reshape(B, N, d), ks.reshape(B, N), ratio, q, w.numpy(),
+                                         qp.numpy(), pool_blocks, top_k)
+    assert np.array_equal(topk.cpu().numpy(), t_ref)
+    assert np.array_equal(cnt.cpu().numpy(), n_ref)
+    if pool_blocks:
+        assert np.array_equal(pool.cpu().numpy(), p_ref)
+    return topk.cpu().numpy(), cnt.cpu().numpy(), (pool.cpu().numpy() if pool_blocks else None)
+
+
+@pytest.mark.parametrize("N,pool_blocks", [(5000, 0), (5000, 2048), (20000, 2048)])
+def test_exact_ties_take_the_lowest_positions(harness, orc, N, pool_blocks):
+    """Every index-K row identical, so every score and every block maximum is equal: the
+    selection falls back to the position order (lowest first), flat and hierarchical,
+    including a pool smaller than the block count."""
+    import fp4_kv_compressed_b200 as pkg
+    import synth
+    row = synth.rows_normal_bf16(40, "row", 0, 0, 1, 128)
+    rows = row.expand(2, N, 128).contiguous()
+    topk, cnt, pool = _index_case(pkg, orc, rows, 1, [N - 1, N - 1], pool_blocks, 512)
+    assert (topk[:, 0] == np.arange(512)).all() and (cnt == 512).all()
+    if pool_blocks:
+        nb = (N + 7) // 8
+        assert (pool[:, 0, :min(nb, 2048)] == np.arange(min(nb, 2048))).all()
+
+
+def test_zero_scores_and_mixed(harness, orc):
+    """A third of the rows are zero (sigma 0, score exactly 0) and tie below every
+    positive score; the rest include scores clipped to 0 by the relu."""
+    import fp4_kv_compressed_b200 as pkg
+    import synth
+    N = 3000
+    rows = synth.rows_normal_bf16(42, "rows", 0, 0, N, 128).view(1, N, 128).clone()
+    rows[0, ::3] = 0
+    _index_case(pkg, orc, rows, 1, [N - 1], 0, 512)
+    t, c, _ = _index_case(pkg, orc, rows, 1, [N - 1], 2048, 2048 // 4)
+    assert c[0, 0] == 512
+
+
+def test_ratio2_earliest_positions(harness, orc):
+    """Ratio-2 entries at the first token positions: t = 0 sees no entry, t = 1 and 2 one,
+    t = 3 two; counts and padded Top-K match the oracle."""
+    import fp4_kv_compressed_b200 as pkg
+    import synth
+    rows = torch.stack([synth.rows_normal_bf16(43, "rows", b, 0, 8, 128) for b in range(4)])
+    topk, cnt, _ = _index_case(pkg, orc, rows, 2, [0, 1, 2, 3], 0, 16)
+    assert cnt[:, 0].tolist() == [0, 1, 1, 2]
+    assert (topk[0, 0] == -1).all() and (topk[3, 0, 2:] == -1).all()
