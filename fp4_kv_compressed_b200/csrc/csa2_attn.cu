@@ -1,4 +1,5 @@
-// csa2_attn_tc.cu -- a8 sparse decode attention on the 5th-generation tensor cores.
+// csa2_attn.cu -- a8 sparse decode attention on the 5th-generation tensor cores
+// (and, for decode, the a2 append of the layer's SWA row, fused in).
 //
 // DeepSeek V4.1 Flash study notes, sections 1, 2 and 4: each layer attends, with
 // its own query, over at most 512 selected global entries (FP4, dequantised on
@@ -9,10 +10,12 @@
 // A 2-CTA cluster per (query, group of 64 heads); each CTA takes half of the
 // query's key tiles and the two partial results are merged through distributed
 // shared memory (each CTA writes half of the output channels).  16 warps, specialised:
-//   warp 0      TMEM allocation + the single MMA-issuing thread;
+//   warp 0      TMEM allocation + the MMA loop (whole warp, one elected lane issues);
+//   warp 1      fused append only: quantises the query token's new SWA row;
 //   warps 4-7   softmax, one per TMEM lane quadrant (warp w reads lanes 32(w%4)..);
 //   warps 8-15  producers: gather the tile's rows (FP4 entry or FP8 SWA row) into
-//               registers one tile ahead, dequantise to fp16 into shared memory.
+//               registers one tile ahead, dequantise to fp16 into shared memory,
+//               channels 0-255 first (own mbarrier), then 256-511.
 // Data layout: one fp16 tile of 64 keys x 512 channels serves both MMAs -- as the
 // K-major B operand of S = Q K^T and as the MN-major B operand of O = P V -- in
 // the 128-byte-swizzled layout [channel block of 64][key][128 B].  fp16 holds the
@@ -27,9 +30,10 @@
 // columns 0..255.
 // Online softmax in the log2 domain with lazy rescaling: O is rescaled only when
 // a head's running max grows by more than 8 (p stays <= 2^8, safe in fp16).
-// The MMA thread issues S(i+1) and P V(i) as soon as each is ready.  Every wait is
-// bounded: on timeout the kernel flags CSA2_DEVERR_TIMEOUT, drains its MMAs, frees
-// TMEM and returns.
+// The MMA warp issues P V(i) and S(i+1) as soon as each is ready.  The combine
+// moves the peer's half of O with bulk copies between the two CTAs' shared memory.
+// Every wait is bounded: on timeout the kernel flags CSA2_DEVERR_TIMEOUT, drains its
+// MMAs, frees TMEM and returns.
 #include <cuda_fp16.h>
 #include <stdint.h>
 
