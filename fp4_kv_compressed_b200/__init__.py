@@ -8,6 +8,7 @@ device buffers.  Importing it loads the library and raises if it is missing.
 from ._binding import (CSA2_OP_INDEX_FULL, CSA2_OP_INDEX_REINDEX, CSA2_OP_SPARSE_ATTN,
                        CSA2GlobalKV, CSA2SWA, Csa2Error, DEVERR_INDEX, DEVERR_NMAX,
                        DEVERR_RANGE, DEVERR_SLOT, EXPORTS, LIB_PATH, csa2_index_full,
+                       csa2_index_full_tc,
                        csa2_index_reindex, csa2_quantize_append, csa2_read_device_error,
                        csa2_sparse_attn_decode, csa2_sparse_attn_decode_append,
                        csa2_workspace_size, load_library)
@@ -18,7 +19,7 @@ load_library()
 __all__ = [
     "CSA2_OP_INDEX_FULL", "CSA2_OP_INDEX_REINDEX", "CSA2_OP_SPARSE_ATTN", "CSA2GlobalKV",
     "CSA2SWA", "Csa2Error", "DEVERR_INDEX", "DEVERR_NMAX", "DEVERR_RANGE", "DEVERR_SLOT",
-    "EXPORTS", "LIB_PATH", "csa2_index_full", "csa2_index_reindex", "csa2_quantize_append",
+    "EXPORTS", "LIB_PATH", "csa2_index_full", "csa2_index_full_tc", "csa2_index_reindex", "csa2_quantize_append",
     "csa2_read_device_error", "csa2_sparse_attn_decode", "csa2_sparse_attn_decode_append",
     "csa2_workspace_size",
     "load_library", "DecodeStack", "GlobalKV", "GroupSpec", "LayerPlan", "SwaRing",

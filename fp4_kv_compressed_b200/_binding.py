@@ -27,7 +27,7 @@ DEVERR_SLOT, DEVERR_INDEX, DEVERR_NMAX, DEVERR_RANGE, DEVERR_TIMEOUT = 0x1, 0x2,
 
 # every symbol declared in include/csa2.h
 EXPORTS = ("csa2_quantize_append", "csa2_workspace_size", "csa2_index_full",
-           "csa2_index_full_noalloc", "csa2_index_reindex", "csa2_sparse_attn_decode",
+           "csa2_index_full_tc", "csa2_index_full_noalloc", "csa2_index_reindex", "csa2_sparse_attn_decode",
            "csa2_sparse_attn_decode_append", "csa2_read_device_error", "csa2_status_string",
            "csa2_abi_version")
 
@@ -67,6 +67,7 @@ def load_library(path: str = LIB_PATH):
     L.csa2_workspace_size.argtypes = [i32] * 7
     L.csa2_workspace_size.restype = sz
     L.csa2_index_full.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, P, P, P, P, sz, P, P]
+    L.csa2_index_full_tc.argtypes = L.csa2_index_full.argtypes
     L.csa2_index_reindex.argtypes = [P, P, P, P, i32, i32, P, i32, i32, P, P, P, sz, P, P]
     L.csa2_sparse_attn_decode.argtypes = [P, P, P, P, i32, i32, P, i32, i32, C.c_float, P, P, P,
                                           sz, P, P]
@@ -76,7 +77,7 @@ def load_library(path: str = LIB_PATH):
     L.csa2_status_string.argtypes = [C.c_int]
     L.csa2_status_string.restype = C.c_char_p
     L.csa2_abi_version.restype = i32
-    for fn in ("csa2_quantize_append", "csa2_index_full", "csa2_index_reindex",
+    for fn in ("csa2_quantize_append", "csa2_index_full", "csa2_index_full_tc", "csa2_index_reindex",
                "csa2_sparse_attn_decode", "csa2_sparse_attn_decode_append",
                "csa2_read_device_error"):
         getattr(L, fn).restype = C.c_int
@@ -127,6 +128,19 @@ def csa2_index_full(kv: CSA2GlobalKV, q_idx, w, q_pos, Tq: int, H_I: int, n_max:
                            pool_blocks, top_k, _ptr(pool_out), _ptr(topk_out), _ptr(topk_count),
                            _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream))
     _check("csa2_index_full", st)
+
+
+def csa2_index_full_tc(kv: CSA2GlobalKV, q_idx, w, q_pos, Tq: int, H_I: int, n_max: int,
+                       pool_blocks: int, top_k: int, pool_out, topk_out, topk_count, workspace,
+                       dev_err=None, stream=None):
+    """csa2_index_full with the scan on the tensor cores (prefill chunks)."""
+    L = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = L.csa2_index_full_tc(C.byref(kv), _ptr(q_idx), _ptr(w), _ptr(q_pos), Tq, H_I, n_max,
+                              pool_blocks, top_k, _ptr(pool_out), _ptr(topk_out),
+                              _ptr(topk_count), _ptr(workspace), ws_bytes, _ptr(dev_err),
+                              _stream(stream))
+    _check("csa2_index_full_tc", st)
 
 
 def csa2_index_reindex(kv: CSA2GlobalKV, q_idx, w, q_pos, Tq: int, H_I: int, pool,

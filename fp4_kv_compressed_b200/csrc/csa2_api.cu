@@ -147,15 +147,16 @@ csa2_status csa2_quantize_append(const csa2_global_kv *kv, const void *kv_bf16,
     return launched(launch_quantize_append(a, (cudaStream_t)stream));
 }
 
-csa2_status csa2_index_full(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
-                            const int32_t *q_pos, int32_t Tq, int32_t H_I, int32_t n_max,
-                            int32_t pool_blocks, int32_t top_k, int32_t *pool_out,
-                            int32_t *topk_out, int32_t *topk_count, void *workspace,
-                            size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
+// Full layer: scan (exact CUDA-core order, or tensor cores) then pool / Top-K.
+static csa2_status index_full(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
+                              const int32_t *q_pos, int32_t Tq, int32_t H_I, int32_t n_max,
+                              int32_t pool_blocks, int32_t top_k, int32_t *pool_out,
+                              int32_t *topk_out, int32_t *topk_count, void *workspace,
+                              size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream, bool tc) {
     csa2_status st = check_kv(kv, true);
     if (st != CSA2_OK) return st;
     if (!q_idx_bf16 || !w || !q_pos || !topk_out || !topk_count) return CSA2_ERR_INVALID_ARG;
-    if (!aligned(q_idx_bf16, 4) || !aligned(w, 4)) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(q_idx_bf16, tc ? 16 : 4) || !aligned(w, 4)) return CSA2_ERR_INVALID_ARG;
     if (Tq <= 0 || n_max < 0) return CSA2_ERR_INVALID_ARG;
     if (!hi_supported(H_I)) return CSA2_ERR_UNSUPPORTED;
     if (top_k < 1 || top_k > CSA2_TOPK_MAX) return CSA2_ERR_UNSUPPORTED;
@@ -191,9 +192,27 @@ csa2_status csa2_index_full(const csa2_global_kv *kv, const void *q_idx_bf16, co
     a.topk_count = topk_count;
     a.dev_err = dev_err;
     cudaStream_t s = (cudaStream_t)stream;
-    st = launched(launch_index_scan(a, (int)BT, s));
+    st = launched(tc ? launch_index_scan_tc(a, (int)kv->batch, s) : launch_index_scan(a, (int)BT, s));
     if (st != CSA2_OK) return st;
     return launched(launch_select_full(a, (int)BT, s));
+}
+
+csa2_status csa2_index_full(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
+                            const int32_t *q_pos, int32_t Tq, int32_t H_I, int32_t n_max,
+                            int32_t pool_blocks, int32_t top_k, int32_t *pool_out,
+                            int32_t *topk_out, int32_t *topk_count, void *workspace,
+                            size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
+    return index_full(kv, q_idx_bf16, w, q_pos, Tq, H_I, n_max, pool_blocks, top_k, pool_out,
+                      topk_out, topk_count, workspace, ws_bytes, dev_err, stream, false);
+}
+
+csa2_status csa2_index_full_tc(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
+                               const int32_t *q_pos, int32_t Tq, int32_t H_I, int32_t n_max,
+                               int32_t pool_blocks, int32_t top_k, int32_t *pool_out,
+                               int32_t *topk_out, int32_t *topk_count, void *workspace,
+                               size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
+    return index_full(kv, q_idx_bf16, w, q_pos, Tq, H_I, n_max, pool_blocks, top_k, pool_out,
+                      topk_out, topk_count, workspace, ws_bytes, dev_err, stream, true);
 }
 
 csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,

@@ -175,6 +175,29 @@ CSA2_API csa2_status csa2_index_full(const csa2_global_kv *kv, const void *q_idx
                             size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream);
 
 /*
+ * a3-a5 Full layer with the scan on the tensor cores, for prefill chunks (Tq in
+ * the hundreds or thousands), where the scan is Tq * N * H_I * d_idx
+ * multiply-adds (DeepSeek V4.1 Flash study notes, section 2; myzaker "CSA2
+ * attention": the same score as csa2_index_full).  The products q_h . k_s run
+ * as bf16 tensor-core MMAs with fp32 accumulation: the E4M3 codes are exact in
+ * bf16 and every product is exact in fp32, but the order of the fp32 sums over
+ * channels and heads is the hardware's, not csa2_index_full's fixed order.  So
+ * each score equals the exactly rounded one to within a few fp32 ulps of
+ * sum_h w_h * |q_h| . |k_s| and the Top-K can differ from csa2_index_full's
+ * only between positions whose scores lie within that bound of each other.
+ * Arguments, outputs, workspace and errors are those of csa2_index_full, plus:
+ * q_idx_bf16 must be 16-byte aligned (else CSA2_ERR_INVALID_ARG).  One CTA
+ * takes 128 / H_I query tokens of one request against up to 2048 entries; Tq
+ * = 1 works but wastes the tile -- decode should call csa2_index_full.
+ */
+CSA2_API csa2_status csa2_index_full_tc(const csa2_global_kv *kv, const void *q_idx_bf16,
+                                        const float *w, const int32_t *q_pos, int32_t Tq,
+                                        int32_t H_I, int32_t n_max, int32_t pool_blocks,
+                                        int32_t top_k, int32_t *pool_out, int32_t *topk_out,
+                                        int32_t *topk_count, void *workspace, size_t ws_bytes,
+                                        int32_t *dev_err, csa2_stream_t stream);
+
+/*
  * csa2_index_full without a workspace argument, for callers that cannot allocate
  * device memory -- for example a backend plugin that runs inside a host
  * framework's execute callback where the framework owns all device memory, or a

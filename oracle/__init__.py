@@ -37,6 +37,7 @@ def lib():
             "csa2o_dequant_fp8": (None, [P, P, i64, C.c_int, P]),
             "csa2o_visible": (i64, [i64, C.c_int]),
             "csa2o_scores": (None, [P, P, C.c_int, P, i64, P, P, C.c_int, P]),
+            "csa2o_scores_f64": (None, [P, P, C.c_int, P, i64, P, P, C.c_int, P, P]),
             "csa2o_block_max": (None, [P, i64, P]),
             "csa2o_select_topk": (i64, [P, P, i64, i64, P]),
             "csa2o_index_full_one": (i32, [P, P, C.c_int, i64, P, P, C.c_int, C.c_int, C.c_int,
@@ -156,6 +157,25 @@ def scores(kc: np.ndarray, ks: np.ndarray, q, w: np.ndarray, pos: np.ndarray | N
     out = np.zeros(n, np.float32)
     lib().csa2o_scores(_p(kc), _p(ks), d, _p(pos), n, _p(qb), _p(w), H_I, _p(out))
     return out
+
+
+def scores_f64(kc: np.ndarray, ks: np.ndarray, q, w: np.ndarray, pos: np.ndarray | None = None,
+               n: int | None = None) -> tuple[np.ndarray, np.ndarray]:
+    """Index scores without fp32 rounding, for one query: (score f64 [n], magnitude
+    f64 [n]), magnitude = sigma_s * sum_h w_h * sum_c |q_hc * k_sc|, which bounds the
+    rounding error of any fp32 summation order of the score."""
+    kc = np.ascontiguousarray(kc, np.uint8)
+    ks = np.ascontiguousarray(ks, np.float32)
+    qb = as_bf16_bits(q)
+    w = np.ascontiguousarray(w, np.float32)
+    H_I, d = qb.shape
+    if pos is not None:
+        pos = np.ascontiguousarray(pos, np.int32)
+        n = len(pos)
+    out = np.zeros(n, np.float64)
+    mag = np.zeros(n, np.float64)
+    lib().csa2o_scores_f64(_p(kc), _p(ks), d, _p(pos), n, _p(qb), _p(w), H_I, _p(out), _p(mag))
+    return out, mag
 
 
 def block_max(sc: np.ndarray) -> np.ndarray:

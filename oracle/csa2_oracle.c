@@ -252,6 +252,42 @@ EXPORT void csa2o_scores(const uint8_t *kc, const float *ks, int d, const int32_
     }
 }
 
+/* The same score without fp32 rounding, for a scan that sums in another order
+ * (the tensor-core scan of prefill chunks): every product q_hc * k_sc and the
+ * sums over channels and heads in fp64, then times sigma_s.  A bf16 times an
+ * E4M3 value has at most 12 significant bits, so the products are exact and the
+ * fp64 sums lose at most d * 2^-53 of the magnitude below -- far under any fp32
+ * rounding.  mag_out[i] = sigma_s * sum_h w_h * sum_c |q_hc * k_sc|: the
+ * magnitude that bounds the rounding error of any fp32 evaluation order of the
+ * score (each of the d + H_I + 1 roundings costs at most 2^-24 of it, relative,
+ * for round-to-nearest).  Same arguments as csa2o_scores. */
+EXPORT void csa2o_scores_f64(const uint8_t *kc, const float *ks, int d, const int32_t *pos,
+                             int64_t n, const uint16_t *q, const float *w, int H_I,
+                             double *out, double *mag_out) {
+    double qf[16][256];
+    e4m3_tab_init();
+    for (int h = 0; h < H_I; ++h)
+        for (int c = 0; c < d; ++c) qf[h][c] = (double)csa2o_bf16_to_f32(q[h * d + c]);
+#pragma omp parallel for schedule(static) if (n > 65536)
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t s = pos ? pos[i] : i;
+        const uint8_t *row = kc + s * (int64_t)d;
+        double t = 0.0, m = 0.0;
+        for (int h = 0; h < H_I; ++h) {
+            double a = 0.0, am = 0.0;
+            for (int c = 0; c < d; ++c) {
+                double pr = qf[h][c] * E4M3_TAB[row[c]];
+                a += pr;
+                am += fabs(pr);
+            }
+            t += (double)w[h] * (a > 0.0 ? a : 0.0);
+            m += (double)w[h] * am;
+        }
+        out[i] = t * (double)ks[s];
+        if (mag_out) mag_out[i] = m * (double)ks[s];
+    }
+}
+
 /* Block key for the hierarchical pool: the maximum score over the visible
  * positions of block b = [8b, 8b+8) (blocks of 8 positions, study notes
  * section 2 / report Figure 5; max over the block as fixed for this build). */

@@ -61,6 +61,13 @@ def test_validation_rejects_before_launch(pkg):
     # workspace too small
     assert lib.csa2_index_full(C.byref(kv), qbuf, qbuf, qbuf, 1, 4, 100, 0, 8, None, qbuf, qbuf,
                                qbuf, 16, None, None) == 3
+    # tensor-core Full scan: same checks, and q_idx must be 16-byte aligned
+    assert lib.csa2_index_full_tc(C.byref(kv), qbuf, qbuf, qbuf, 1, 3, 10, 0, 8, None, qbuf,
+                                  qbuf, qbuf, 1 << 20, None, None) == 4
+    assert lib.csa2_index_full_tc(C.byref(kv), qbuf, qbuf, qbuf, 1, 4, 100, 0, 8, None, qbuf,
+                                  qbuf, qbuf, 16, None, None) == 3
+    assert lib.csa2_index_full_tc(C.byref(kv), C.c_void_p(4104), qbuf, qbuf, 1, 4, 10, 0, 8, None,
+                                  qbuf, qbuf, qbuf, 1 << 20, None, None) == 1
     # bad d_idx
     kv2 = pkg.CSA2GlobalKV(256, 256, 256, 256, 1, 100, 96, 1)
     assert lib.csa2_index_reindex(C.byref(kv2), qbuf, qbuf, qbuf, 1, 4, qbuf, 64, 64, qbuf, qbuf,

@@ -81,6 +81,39 @@ def test_score_formula_fp64_bound_and_one_hot(orc):
             assert s == max(float(q[h, c]), 0.0)
 
 
+def test_scores_f64_exact_rational_and_bound(orc):
+    """The unrounded score (used for scans that sum in another order) equals the
+    exact rational score of the definition, its magnitude equals the exact sum of
+    |products|, and the canonical fp32 score lies within (d + H_I + 1) * 2^-24 of
+    that magnitude from it."""
+    d, H_I, n = 64, 4, 16
+    k = random_index_rows(n, d, 24, 3.0)
+    kc, ks = orc.quantize_fp8(k)
+    q = synth.rows_normal_bf16(25, "q", 0, 0, H_I, d)
+    q[2, 5] = -q[2, 5]
+    w = synth.rows_uniform_f32(26, "w", 0, 0, 1, H_I)[0].numpy()
+    sc, mag = orc.scores_f64(kc, ks, q, w, n=n)
+    qf = q.float().numpy()
+    for s in range(n):
+        t = Fraction(0)
+        m = Fraction(0)
+        for h in range(H_I):
+            prods = [f(qf[h, c]) * e4m3_exact(int(kc[s, c])) for c in range(d)]
+            a = sum(prods, Fraction(0))
+            t += f(w[h]) * max(a, Fraction(0))
+            m += f(w[h]) * sum((abs(p) for p in prods), Fraction(0))
+        t *= f(ks[s])
+        m *= f(ks[s])
+        assert abs(Fraction(float(sc[s])) - t) <= abs(t) * Fraction(1, 2 ** 50), s
+        assert abs(Fraction(float(mag[s])) - m) <= m * Fraction(1, 2 ** 50), s
+    sc32 = orc.scores(kc, ks, q, w, n=n).astype(np.float64)
+    assert np.all(np.abs(sc32 - sc) <= (d + H_I + 1) * 2.0 ** -24 * mag * 1.001 + 1e-300)
+    # a subset of positions gives the same values
+    pos = np.array([15, 0, 7], np.int32)
+    sp, mp = orc.scores_f64(kc, ks, q, w, pos=pos)
+    assert np.array_equal(sp, sc[pos]) and np.array_equal(mp, mag[pos])
+
+
 def test_block_max(orc):
     sc = np.random.default_rng(1).standard_normal(83).astype(np.float32)
     bm = orc.block_max(sc)
