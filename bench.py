@@ -8,6 +8,8 @@ context 131072, decoder stack F+4X+15U (decode_128k).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   (the CPU oracle as the reference arm)
+  python bench.py --workload prefill_chunk_enc --index-scan tc
+      (a 2048-token prefill chunk; the Full scan on the tensor cores)
 
 Multi-GPU (torchrun): requests are independent, so each rank runs its own batch
 with no collective on the data path (weak scaling); timing is the max over ranks.
@@ -55,12 +57,21 @@ def op_bytes(wl) -> dict:
             out[f"index_reindex_g{g}"] = BT * rp
         else:
             out[f"index_full_g{g}"] = BT * (N * (d + 4) + 4 * N + 4 * N + 4 * K + 4 + q)
+        if Tq > 1:
+            # the query tokens of a request share its index cache: read it once
+            out[f"index_full_g{g}"] -= (BT - B) * N * (d + 4)
         out[f"append_g{g}"] = B * max(1, wl.entries(g) - wl.first_q_pos // grp.ratio) * (
             512 * 2 + 288 + d * 2 + d + 4)
     n_win = min(wl.swa_len, wl.first_q_pos + 1)
     out["attn"] = BT * (K * 288 + K * 4 + n_win * 516 + wl.H * 512 * 2 + wl.H * 512 * 4 + wl.H * 4)
     out["swa_append"] = B * Tq * (512 * 2 + 516)
     return out
+
+
+def index_scan_flops(wl, g: int) -> int:
+    """Score products of a Full scan: 2 * H_I * d_idx flop per (query, visible entry)."""
+    vis = sum(min((t + 1) // wl.groups[g].ratio, wl.entries(g)) for t in wl.q_positions())
+    return wl.B * vis * 2 * wl.H_I * wl.d_I
 
 
 def attn_flops(wl) -> int:
@@ -70,26 +81,34 @@ def attn_flops(wl) -> int:
 
 
 # DRAM bytes (read + write) per launch from one ncu capture of each of an op's kernels:
-# ([(bytes, batch of the captured launch), ...], kernel sources, sha256[:16] of those
+# ([(bytes, batch of the captured launch), ...], kernel sources, code_hash of those
 # sources at capture time).  Reported, each kernel scaled to the batch, only while the
-# sources are unchanged.  Captures: profiles/*.md.
+# code is unchanged.  Captures: profiles/*.md.
 NCU_TRAFFIC = {
-    "csa2_sparse_attn_decode": ([(21_212_416, 64)], ("csa2_attn.cu",), "c63fd92c20f73652"),
-    "csa2_sparse_attn_decode_append": ([(21_212_416, 64)], ("csa2_attn.cu",), "c63fd92c20f73652"),
+    "csa2_sparse_attn_decode": ([(21_212_416, 64)], ("csa2_attn.cu",), "139e5cf6f85cdcdd"),
+    "csa2_sparse_attn_decode_append": ([(21_212_416, 64)], ("csa2_attn.cu",), "139e5cf6f85cdcdd"),
     "csa2_index_full": ([(138_484_992 + 4_945_664, 8), (18_141_952, 64)], ("csa2_index.cu",),
-                        "4bd071bde104eeff"),
+                        "33472cf35d49fbf2"),
     "csa2_index_reindex": ([(18_606_080, 8), (4_754_432, 64)], ("csa2_index.cu",),
-                           "4bd071bde104eeff"),
+                           "33472cf35d49fbf2"),
 }
 
 
-def _sources_hash(files) -> str:
+def code_hash(text: bytes) -> str:
+    """sha256[:16] of a source with its // comments and blank lines removed, so that
+    the key changes with the code but not with its comments."""
     import hashlib
     h = hashlib.sha256()
-    for f in files:
-        with open(os.path.join(ROOT, "fp4_kv_compressed_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    for ln in text.decode().splitlines():
+        code = ln.split("//", 1)[0].rstrip()
+        if code:
+            h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
+
+
+def _sources_hash(files) -> str:
+    return code_hash(b"".join(open(os.path.join(ROOT, "fp4_kv_compressed_b200", "csrc", f), "rb").read()
+                              for f in files))
 
 
 def measured_peaks() -> dict:
@@ -112,6 +131,8 @@ def op_rooflines(wl, plan, op_ms: dict, ms_step: float) -> dict:
     dec = plan[[lp.layer for lp in plan if lp.mode == "F"][-1]].group
     spec = {"csa2_index_full": (ob[f"index_full_g{dec}"], modes.count("F"),
                                 "index_scan_kernel + select_full_kernel"),
+            "csa2_index_full_tc": (ob[f"index_full_g{dec}"], modes.count("F"),
+                                   "index_scan_tc_kernel + select_full_kernel"),
             "csa2_index_reindex": (ob.get(f"index_reindex_g{dec}", 0), modes.count("X"),
                                    "reindex_score_kernel + select_reindex_kernel"),
             "csa2_sparse_attn_decode": (ob["attn"], len(modes), "attn_tc_kernel"),
@@ -135,8 +156,12 @@ def op_rooflines(wl, plan, op_ms: dict, ms_step: float) -> dict:
              "frac": gbs / pk["hbm_gbs"], "traffic": traffic, "kernels": kernels,
              "algorithmic_bytes_per_launch": nbytes, "launch_ms": ms, "launches_per_step": n,
              "share_of_step": n * ms / ms_step, "peak_source": pk["source"]}
+        fl = None
         if name.startswith("csa2_sparse_attn_decode"):
             fl = attn_flops(wl)
+        elif name == "csa2_index_full_tc":
+            fl = index_scan_flops(wl, dec)
+        if fl:
             tfs = fl / (ms / 1e3) / 1e12
             e["tensor"] = {"achieved": tfs, "peak": pk["tflops"], "unit": "TFLOP/s",
                            "frac": tfs / pk["tflops"], "flops_per_launch": fl}
@@ -363,7 +388,7 @@ def run_ours(args, rank, world, local_rank):
         from synth.workloads import small_variant
         wl = small_variant(wl, B=args.batch, name=f"{wl.name}_b{args.batch}")
     wl = rank_workload(wl, rank)
-    dw = csa2_harness.DeviceWorkload(wl, device=dev)
+    dw = csa2_harness.DeviceWorkload(wl, device=dev, index_scan=args.index_scan)
     st = dw.stack
     inputs, dbuf, hbuf, in_bytes = pack_inputs(dw.inputs, dev)
     full_layers = [lp.layer for lp in st.plan if lp.mode == "F"]
@@ -389,7 +414,8 @@ def run_ours(args, rank, world, local_rank):
         attn_pick = ("csa2_sparse_attn_decode_append", (n_attn, n_attn - 1))
     else:
         attn_pick = ("csa2_sparse_attn_decode", (len(modes), len(modes) - 1))
-    picks = {"csa2_index_full": (modes.count("F"), 0),
+    full_name = "csa2_index_full_tc" if args.index_scan == "tc" else "csa2_index_full"
+    picks = {full_name: (modes.count("F"), 0),
              "csa2_index_reindex": (modes.count("X"), 0),
              attn_pick[0]: attn_pick[1]}
     op_events = {name: [] for name in picks}
@@ -501,12 +527,15 @@ def run_ours(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "fp32 index / bf16+fp16 MMA attention",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": ("bf16 MMA index (fp32 accumulate)" if args.index_scan == "tc" else "fp32 index")
+                 + " / bf16+fp16 MMA attention",
         "data": "synthetic",
         "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.ctx, "heads": wl.H,
                    "index_heads": wl.H_I, "d_idx": wl.d_I, "top_k": wl.top_k,
                    "pool": [g.pool_blocks for g in wl.groups],
                    "schedule": [g.schedule for g in wl.groups], "swa": wl.swa_len,
+                   "query_tokens": wl.Tq, "index_scan": args.index_scan,
                    "parallelism": f"replicas x{world} (requests sharded, no collective)",
                    "l2": "inputs larger than L2: the Full scan streams "
                          f"{ob[f'index_full_g{g_full}'] / 1e9:.2f} GB per step",
@@ -557,6 +586,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="decode_128k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--index-scan", default="exact", choices=["exact", "tc"],
+                    help="Full-layer scan: fixed fp32 order, or tensor cores (prefill chunks)")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

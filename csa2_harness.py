@@ -22,13 +22,15 @@ from synth.workloads import Workload
 
 
 class DeviceWorkload:
-    def __init__(self, wl: Workload, device="cuda", chunk_elems: int = 1 << 25, fill=True):
+    def __init__(self, wl: Workload, device="cuda", chunk_elems: int = 1 << 25, fill=True,
+                 index_scan: str = "exact"):
         self.wl = wl
         self.device = torch.device(device)
         self.groups = [GroupSpec(g.ratio, g.schedule, g.pool_blocks, wl.entries(i))
                        for i, g in enumerate(wl.groups)]
         self.stack = DecodeStack(wl.B, wl.H, wl.H_I, wl.d_I, wl.top_k, wl.swa_len, self.groups,
-                                 Tq=wl.Tq, window_cap=wl.window_cap, device=device)
+                                 Tq=wl.Tq, window_cap=wl.window_cap, device=device,
+                                 index_scan=index_scan)
         self.t0 = wl.first_q_pos
         self.chunk_elems = chunk_elems
         if fill:

@@ -5,21 +5,24 @@
 // Full layer scores every causally visible entry with
 //   score(s) = sigma_s * sum_h w_h * relu(q_h . c_s)
 // (c_s the entry's E4M3 indexer-K codes, sigma_s its scale).  With Tq query tokens
-// per request the scan is Tq * N * H_I * d_idx multiply-adds, which the CUDA cores
-// of the exact scan (csa2_index.cu) take ~1000x longer to do than this tensor-core
-// form: the products q_h . c_s of 128 / H_I query tokens (M = 128 rows = tokens x
-// heads) against 256 entries (N = 256) at a time are one tcgen05 MMA chain over the
-// d_idx channels (K).  Operands are bf16: the bf16 query is used as is and the E4M3
-// codes are exact in bf16, so every product is exact; only the fp32 accumulation
-// order differs from the fixed order of the exact scan, so scores agree to a few
-// fp32 ulps and Top-K membership can differ only between near-tied positions.
+// per request the scan is Tq * N * H_I * d_idx multiply-adds, a dense contraction:
+// the products c_s . q_h of 128 entries (MMA M = 128, one TMEM lane per entry)
+// against 256 / H_I query tokens x H_I heads (MMA N = 256 columns) are one tcgen05
+// MMA chain over the d_idx channels (K).  Operands are bf16: the bf16 query is used
+// as is and the E4M3 codes are exact in bf16, so every product is exact; only the
+// fp32 accumulation order differs from the fixed order of the exact scan
+// (csa2_index.cu), so scores agree to a few fp32 ulps and Top-K membership can
+// differ only between near-tied positions.
 //
-// One CTA (512 threads) = one request's block of 128 / H_I query tokens and up to
-// kTilesPerCta tiles of 256 entries.  Per tile: every thread converts a share of
-// the tile's codes to bf16 into a 128-byte-swizzled K-major tile (double-buffered),
-// one elected thread issues the MMAs into one of two TMEM accumulators, and while
-// they run all 16 warps take the previous tile's accumulator: relu, w_h, the sum
-// over the H_I rows of a token (lane shuffles), sigma, the causal mask; scores and
+// Persistent: one CTA (512 threads) per SM takes a contiguous range of work items
+// (request, block of 256 / H_I query tokens, tile of 128 entries), so the query
+// block -- the MMA's B operand, kept in shared memory -- changes at most a few
+// times per CTA.  Per tile: every thread converts a share of the tile's codes to
+// bf16 into a 128-byte-swizzled K-major A tile (double-buffered), one elected
+// thread issues the MMAs into one of two TMEM accumulators, and while they run all
+// 16 warps take the previous tile's accumulator: thread = entry, so relu, w_h and
+// the sum over a token's heads stay in registers, then sigma and the causal mask;
+// a warp stores 32 consecutive entries of a token (128 bytes).  Scores and
 // 8-position block maxima go to the same workspace as the exact scan, whose
 // selection kernel then runs unchanged.  Every wait is bounded (0.5 s).
 #include <cuda_bf16.h>
@@ -33,19 +36,17 @@ namespace csa2 {
 namespace itc {
 
 constexpr int kThreads = 512;
-constexpr int kM = 128;                  // MMA rows: query tokens x index heads
-constexpr int kN = 256;                  // entries per tile (MMA N)
-constexpr int kTilesPerCta = 8;
+constexpr int kM = 128;                  // entries per tile (MMA M, TMEM lanes)
+constexpr int kN = 256;                  // query tokens x index heads (MMA N)
 constexpr uint32_t kTmemCols = 512;      // two 256-column fp32 accumulators
 constexpr uint64_t kWaitLimitNs = 500000000ull;
 
 template <int D>
 struct __align__(1024) Smem {
-    uint8_t a[D / 64][kM * 128];         // q, bf16, [channel block][row][128 B] swizzled
-    uint8_t b[2][D / 64][kN * 128];      // entry codes as bf16, same layout, 2 buffers
-    float sig[3][kN];                    // entry scales of tile i in sig[i % 3] (see the loop)
-    float w[kM];                         // w of each row (token, head)
-    int32_t nvis[kM];                    // visible entries of each row's token (-1: no token)
+    uint8_t q[D / 64][kN * 128];         // B: query rows (token, head), bf16, [channel block][row][128 B]
+    uint8_t a[2][D / 64][kM * 128];      // A: entry codes as bf16, same layout, 2 buffers
+    alignas(16) float w[kN];             // w of each column (token, head)
+    int32_t nvis[kN];                    // visible entries of each token of the block (-1: none)
     uint64_t mma_done[2];
     uint32_t tmem_base;
 };
@@ -137,15 +138,19 @@ __device__ __forceinline__ uint32_t e4m3x2_bf16x2(uint32_t two) {
     return *reinterpret_cast<const uint32_t *>(&b);
 }
 
+// Work item it = (by, tile), by = b * n_qblk + y: request b, query block y (tokens
+// y * QB ..), entry tile (entries tile * 128 ..).  CTA c takes items
+// [c * W / G, (c + 1) * W / G).
 template <int D, int HI>
-__global__ void __launch_bounds__(kThreads, 1) index_scan_tc_kernel(IndexArgs a) {
-    constexpr int QB = kM / HI;          // query tokens per CTA
+__global__ void __launch_bounds__(kThreads, 1) index_scan_tc_kernel(IndexArgs a, int B, int n_qblk,
+                                                                    int n_tiles) {
+    constexpr int QB = kN / HI;          // query tokens per block
     constexpr int CB = D / 64;           // 64-channel blocks
+    constexpr int TPC = 32 / HI;         // tokens per 32-column TMEM load
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem<D> &s = *reinterpret_cast<Smem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = blockIdx.z;
-    const int tq0 = blockIdx.y * QB;     // first query token of the block
+    const int my_ent = 32 * (warp & 3) + lane;   // this thread's entry (TMEM lane) in a tile
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&s.mma_done[i])));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -156,148 +161,173 @@ __global__ void __launch_bounds__(kThreads, 1) index_scan_tc_kernel(IndexArgs a)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
         asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     }
-    grid_dep_wait();
-    // rows r = token * HI + head; tokens past Tq are zero rows whose scores are dropped
-    if (threadIdx.x < kM) {
-        const int r = threadIdx.x, tk = tq0 + r / HI, h = r % HI;
-        int nv = -1;
-        float wv = 0.0f;
-        if (tk < a.Tq) {
-            const int qi = b * a.Tq + tk;
-            int64_t N = visible_entries(a.q_pos[qi], a.ratio);
-            if (N > a.n_max || N > a.cap) {
-                if (h == 0) set_dev_err(a.dev_err, CSA2_DEVERR_NMAX);
-                N = min64(min64(N, a.n_max), a.cap);
-            }
-            nv = (int)N;
-            wv = __ldg(a.w + (int64_t)qi * HI + h);
-        }
-        s.nvis[r] = nv;
-        s.w[r] = wv;
-    }
-    // q rows into the A operand (bf16 as is): unit (row, cb, u) of 8 channels
-    for (int e = threadIdx.x; e < kM * CB * 8; e += kThreads) {
-        const int r = e / (CB * 8), cb = (e / 8) % CB, u = e % 8;
-        const int tk = tq0 + r / HI, h = r % HI;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (tk < a.Tq)
-            v = __ldg(reinterpret_cast<const uint4 *>(a.q_idx + ((int64_t)(b * a.Tq + tk) * HI + h) * D + cb * 64 + u * 8));
-        *reinterpret_cast<uint4 *>(s.a[cb] + swz_off(r, u)) = v;
-    }
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    // tiles past the largest visible count of the block's tokens are skipped
-    int hi_vis = 0;
-    for (int r = 0; r < kM; r += HI) hi_vis = max(hi_vis, s.nvis[r]);
-    const int n_tiles_vis = (hi_vis + kN - 1) / kN;
-    const int t_begin = blockIdx.x * kTilesPerCta;
-    const int t_end = min(n_tiles_vis, t_begin + kTilesPerCta);
-    const int nt = max(0, t_end - t_begin);
     const uint32_t tmem = s.tmem_base;
+    grid_dep_wait();
     // kind::f16 instruction descriptor: F32 accumulator, bf16 A and B, both K-major
     const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kN >> 3) << 17) |
                            ((uint32_t)(kM >> 4) << 24);
-    const uint8_t *codes = a.idx_codes + (int64_t)b * a.cap * D;
-    const float *sigma = a.idx_scale + (int64_t)b * a.cap;
+    const int64_t total = (int64_t)B * n_qblk * n_tiles;
+    const int64_t lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
+
+    int cur_by = -1, b = 0, tq0 = 0, hi_vis = 0;
+    uint32_t n_issued = 0;               // MMA groups issued: buffer = n & 1, use = n >> 1
+    int pend = -1;                       // issue number of the tile awaiting its epilogue
+    int64_t pend_e0 = 0;
+    float pend_sig = 0.0f;
     bool ok = true;
-    // tile i: convert into buffer i & 1, issue its MMAs, then the epilogue of tile i - 1
-    for (int i = 0; i <= nt; ++i) {
-        if (i < nt) {
-            const int64_t e0 = (int64_t)(t_begin + i) * kN;
-            // entry row n, 16-byte unit of 16 codes -> two bf16 units of 8 channels
-            for (int e = threadIdx.x; e < kN * (D / 16); e += kThreads) {
-                const int n = e / (D / 16), g = e % (D / 16);
-                const int64_t ent = e0 + n;
-                uint4 c = make_uint4(0u, 0u, 0u, 0u);
-                if (ent < a.cap) c = __ldg(reinterpret_cast<const uint4 *>(codes + ent * D + g * 16));
-                const uint32_t w4[4] = {c.x, c.y, c.z, c.w};
-                uint32_t o[8];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    o[2 * k] = e4m3x2_bf16x2(w4[k] & 0xFFFFu);
-                    o[2 * k + 1] = e4m3x2_bf16x2(w4[k] >> 16);
-                }
-                const int ch = g * 16, cb = ch / 64, u = (ch % 64) / 8;
-                uint8_t *blk = s.b[i & 1][cb];
-                *reinterpret_cast<uint4 *>(blk + swz_off(n, u)) = make_uint4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<uint4 *>(blk + swz_off(n, u + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
-            }
-            // three scale buffers: a thread here has passed the barrier that ends tile i - 3's
-            // epilogue, while warps with no rows to write may still be in tile i - 2's
-            for (int n = threadIdx.x; n < kN; n += kThreads)
-                s.sig[i % 3][n] = e0 + n < a.cap ? __ldg(sigma + e0 + n) : 0.0f;
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-            __syncthreads();
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            if (warp == 0) {
-                if (elect_one()) {
-                    const uint32_t d = tmem + (uint32_t)((i & 1) * kN);
-#pragma unroll
-                    for (int k16 = 0; k16 < D / 16; ++k16) {
-                        const int cb = k16 / 4, kk = k16 % 4;
-                        const uint64_t ad = sw128_desc(smem_u32(s.a[cb])) + (uint64_t)(2 * kk);
-                        const uint64_t bd = sw128_desc(smem_u32(s.b[i & 1][cb])) + (uint64_t)(2 * kk);
-                        mma_bf16(d, ad, bd, idesc, k16 > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&s.mma_done[i & 1]);
-                }
-                __syncwarp();
-            }
-        }
-        if (i > 0) {
-            // epilogue of tile j = i - 1: warp w reads TMEM lanes 32 (w % 4) .. (rows) and
-            // columns 64 (w / 4) .. +64 (entries)
-            const int j = i - 1;
-            ok = __syncthreads_and(ok && mbar_wait(&s.mma_done[j & 1], (j >> 1) & 1)) != 0;
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            if (!ok) break;
-            const int r = 32 * (warp & 3) + lane;
-            const int c0 = 64 * (warp >> 2);
-            const int tk = tq0 + r / HI, h = r % HI;
-            const int nv = s.nvis[r];
-            const float wr = s.w[r];
-            const int64_t e0 = (int64_t)(t_begin + j) * kN;
-            const bool writer = h == 0 && tk < a.Tq;
-            const int qi = b * a.Tq + tk;
-            float *srow = a.scores + (int64_t)qi * a.score_stride;
+
+    // epilogue of the pending tile: scores of entries pend_e0 + my_ent for every token
+    auto epilogue = [&]() {
+        const uint32_t buf = (uint32_t)pend & 1u;
+        ok = __syncthreads_and(ok && mbar_wait(&s.mma_done[buf], ((uint32_t)pend >> 1) & 1u)) != 0;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        if (!ok) return;
+        const int64_t ent = pend_e0 + my_ent;
+        const int col0 = 64 * (warp >> 2);
 #pragma unroll 1
-            for (int cc = 0; cc < 64; cc += 32) {
-                float v[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)((j & 1) * kN + c0 + cc), v);
+        for (int cc = 0; cc < 64; cc += 32) {
+            float v[32];
+            tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + buf * kN + (uint32_t)(col0 + cc), v);
 #pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                    float t = wr * fmaxf(v[x], 0.0f);
+            for (int u = 0; u < TPC; ++u) {
+                const int c = col0 + cc + u * HI;            // first column of the token
+                float wt[HI];
+                if constexpr (HI >= 4) {
 #pragma unroll
-                    for (int o = 1; o < HI; o <<= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
-                    v[x] = t;
+                    for (int h = 0; h < HI; h += 4) {
+                        const float4 w4 = *reinterpret_cast<const float4 *>(&s.w[c + h]);
+                        wt[h] = w4.x; wt[h + 1] = w4.y; wt[h + 2] = w4.z; wt[h + 3] = w4.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < HI; ++h) wt[h] = s.w[c + h];
                 }
-                if (writer) {
-                    float sc[32];
+                float t = 0.0f;
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) {
-                        const int64_t ent = e0 + c0 + cc + x;
-                        sc[x] = ent < nv ? __fmul_rn(v[x], s.sig[j % 3][c0 + cc + x]) : -INFINITY;
-                    }
-#pragma unroll
-                    for (int x = 0; x < 32; x += 4)
-                        if (e0 + c0 + cc + x + 3 < a.score_stride)
-                            *reinterpret_cast<float4 *>(srow + e0 + c0 + cc + x) =
-                                make_float4(sc[x], sc[x + 1], sc[x + 2], sc[x + 3]);
-                    if (a.bmax) {
-#pragma unroll
-                        for (int x = 0; x < 32; x += 8) {
-                            float m = sc[x];
-#pragma unroll
-                            for (int y = 1; y < 8; ++y) m = fmaxf(m, sc[x + y]);
-                            const int64_t blk = (e0 + c0 + cc + x) / 8;
-                            if (blk * 8 < nv) a.bmax[(int64_t)qi * a.bmax_stride + blk] = m;
-                        }
-                    }
+                for (int h = 0; h < HI; ++h) t = fmaf(wt[h], fmaxf(v[u * HI + h], 0.0f), t);
+                const int tl = c / HI, tk = tq0 + tl;
+                const int nv = s.nvis[tl];
+                const bool vis = ent < nv;
+                const float sc = __fmul_rn(t, pend_sig);
+                const int64_t qi = (int64_t)b * a.Tq + tk;
+                if (vis) a.scores[qi * a.score_stride + ent] = sc;
+                if (a.bmax) {
+                    float m = vis ? sc : -INFINITY;
+                    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+                    if ((lane & 7) == 0 && vis) a.bmax[qi * a.bmax_stride + ent / 8] = m;
                 }
             }
-            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
         }
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        pend = -1;
+    };
+
+    for (int64_t it = lo; ok; ++it) {
+        const bool have = it < hi;
+        const int by = have ? (int)(it / n_tiles) : -1;
+        if (have && by == cur_by && (int64_t)(it % n_tiles) * kM >= hi_vis) {
+            it = (int64_t)(by + 1) * n_tiles - 1;            // the rest of this block is not visible
+            continue;
+        }
+        if (!have || by != cur_by) {
+            if (pend >= 0) epilogue();
+            if (!have || !ok) break;
+            // new query block: rows n = token * HI + head are consecutive rows of q_idx
+            __syncthreads();
+            cur_by = by;
+            b = by / n_qblk;
+            tq0 = (by % n_qblk) * QB;
+            if (threadIdx.x < kN) {
+                const int tl = threadIdx.x / HI, h = threadIdx.x % HI, tk = tq0 + tl;
+                int nv = -1;
+                float wv = 0.0f;
+                if (tk < a.Tq) {
+                    const int64_t qi = (int64_t)b * a.Tq + tk;
+                    int64_t N = visible_entries(a.q_pos[qi], a.ratio);
+                    if (N > a.n_max || N > a.cap) {
+                        if (h == 0) set_dev_err(a.dev_err, CSA2_DEVERR_NMAX);
+                        N = min64(min64(N, a.n_max), a.cap);
+                    }
+                    nv = (int)N;
+                    wv = __ldg(a.w + qi * HI + h);
+                }
+                s.nvis[tl] = nv;
+                s.w[threadIdx.x] = wv;
+            }
+            const uint16_t *qsrc = a.q_idx + ((int64_t)b * a.Tq + tq0) * HI * D;
+            const int rows_valid = min(kN, (a.Tq - tq0) * HI);
+            for (int e = threadIdx.x; e < kN * CB * 8; e += kThreads) {
+                const int r = e / (CB * 8), cb = (e / 8) % CB, u = e % 8;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (r < rows_valid) v = __ldg(reinterpret_cast<const uint4 *>(qsrc + (int64_t)r * D + cb * 64 + u * 8));
+                *reinterpret_cast<uint4 *>(s.q[cb] + swz_off(r, u)) = v;
+            }
+            __syncthreads();
+            hi_vis = 0;
+            for (int tl = 0; tl < QB; ++tl) hi_vis = max(hi_vis, s.nvis[tl]);
+            if ((int64_t)(it % n_tiles) * kM >= hi_vis) {
+                it = (int64_t)(by + 1) * n_tiles - 1;
+                continue;
+            }
+        }
+        // tile (by, it % n_tiles): convert into buffer n_issued & 1, issue its MMAs
+        const int64_t e0 = (it % n_tiles) * kM;
+        const uint8_t *codes = a.idx_codes + ((int64_t)b * a.cap + e0) * D;
+        const uint32_t buf = n_issued & 1u;
+        const int64_t my_e = e0 + my_ent;
+        const float sig = my_e < a.cap ? __ldg(a.idx_scale + (int64_t)b * a.cap + my_e) : 0.0f;
+        constexpr int kUnits = kM * (D / 16) / kThreads;   // 16-code units per thread
+        uint4 cu[kUnits];
+#pragma unroll
+        for (int k = 0; k < kUnits; ++k) {                  // all loads in flight together
+            const int e = threadIdx.x + k * kThreads, n = e / (D / 16), g = e % (D / 16);
+            cu[k] = make_uint4(0u, 0u, 0u, 0u);
+            if (e0 + n < a.cap) cu[k] = __ldg(reinterpret_cast<const uint4 *>(codes + (int64_t)n * D + g * 16));
+        }
+#pragma unroll
+        for (int k = 0; k < kUnits; ++k) {
+            const int e = threadIdx.x + k * kThreads, n = e / (D / 16), g = e % (D / 16);
+            // 16 channels = units u, u + 1 of channel block cb; which of the two is stored
+            // first alternates so that a quarter-warp's stores hit 8 different bank groups
+            const int cb = g / 4, u = (g % 4) * 2;
+            const int first = (g ^ (g >> 2)) & 1;
+            const uint32_t w0 = first ? cu[k].z : cu[k].x, w1 = first ? cu[k].w : cu[k].y;
+            const uint32_t w2 = first ? cu[k].x : cu[k].z, w3 = first ? cu[k].y : cu[k].w;
+            uint8_t *blk = s.a[buf][cb];
+            *reinterpret_cast<uint4 *>(blk + swz_off(n, u + first)) =
+                make_uint4(e4m3x2_bf16x2(w0 & 0xFFFFu), e4m3x2_bf16x2(w0 >> 16),
+                           e4m3x2_bf16x2(w1 & 0xFFFFu), e4m3x2_bf16x2(w1 >> 16));
+            *reinterpret_cast<uint4 *>(blk + swz_off(n, u + 1 - first)) =
+                make_uint4(e4m3x2_bf16x2(w2 & 0xFFFFu), e4m3x2_bf16x2(w2 >> 16),
+                           e4m3x2_bf16x2(w3 & 0xFFFFu), e4m3x2_bf16x2(w3 >> 16));
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncthreads();
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        if (warp == 0) {
+            if (elect_one()) {
+                const uint32_t d = tmem + buf * kN;
+#pragma unroll
+                for (int k16 = 0; k16 < D / 16; ++k16) {
+                    const int cb = k16 / 4, kk = k16 % 4;
+                    const uint64_t ad = sw128_desc(smem_u32(s.a[buf][cb])) + (uint64_t)(2 * kk);
+                    const uint64_t bd = sw128_desc(smem_u32(s.q[cb])) + (uint64_t)(2 * kk);
+                    mma_bf16(d, ad, bd, idesc, k16 > 0 ? 1u : 0u);
+                }
+                mma_commit(&s.mma_done[buf]);
+            }
+            __syncwarp();
+        }
+        const int issued = (int)n_issued++;
+        if (pend >= 0) epilogue();
+        pend = issued;
+        pend_e0 = e0;
+        pend_sig = sig;
     }
     if (!ok && threadIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
     grid_dep_launch();
@@ -305,6 +335,17 @@ __global__ void __launch_bounds__(kThreads, 1) index_scan_tc_kernel(IndexArgs a)
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+}
+
+static int sm_count() {
+    static int n = 0;   // once per process (one device per process)
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    }
+    return n;
 }
 
 template <int D, int HI>
@@ -319,10 +360,13 @@ static cudaError_t launch_t(const IndexArgs &a, int B, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    const int n_tiles = (int)((a.n_max + kN - 1) / kN);
-    const dim3 grid((n_tiles + kTilesPerCta - 1) / kTilesPerCta, (a.Tq + kM / HI - 1) / (kM / HI), B);
-    if (grid.x == 0) return cudaSuccess;
-    cudaError_t e = launch_pdl(index_scan_tc_kernel<D, HI>, grid, dim3(kThreads), smem, st, a);
+    const int n_tiles = (int)((a.n_max + kM - 1) / kM);
+    const int n_qblk = (a.Tq + kN / HI - 1) / (kN / HI);
+    const int64_t total = (int64_t)B * n_qblk * n_tiles;
+    if (total == 0) return cudaSuccess;
+    const int grid = (int)(total < sm_count() ? total : sm_count());
+    cudaError_t e = launch_pdl(index_scan_tc_kernel<D, HI>, dim3(grid), dim3(kThreads), smem, st, a,
+                               B, n_qblk, n_tiles);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
@@ -331,11 +375,11 @@ static cudaError_t launch_t(const IndexArgs &a, int B, cudaStream_t st) {
 cudaError_t launch_index_scan_tc(const IndexArgs &a, int B, cudaStream_t st) {
 #define CSA2_TC_HI(D)                                                   \
     switch (a.H_I) {                                                    \
-        case 1: return itc::launch_t<D, 1>(a, B, st);                   \
-        case 2: return itc::launch_t<D, 2>(a, B, st);                   \
-        case 4: return itc::launch_t<D, 4>(a, B, st);                   \
-        case 8: return itc::launch_t<D, 8>(a, B, st);                   \
-        case 16: return itc::launch_t<D, 16>(a, B, st);                 \
+        case 1: return itc::launch_t<D, 1>(a, B, st);                       \
+        case 2: return itc::launch_t<D, 2>(a, B, st);                       \
+        case 4: return itc::launch_t<D, 4>(a, B, st);                       \
+        case 8: return itc::launch_t<D, 8>(a, B, st);                       \
+        case 16: return itc::launch_t<D, 16>(a, B, st);                     \
         default: return cudaErrorInvalidValue;                          \
     }
     if (a.d_idx == 128) { CSA2_TC_HI(128) }

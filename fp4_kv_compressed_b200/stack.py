@@ -97,7 +97,12 @@ class DecodeStack:
 
     def __init__(self, B: int, H: int, H_I: int, d_idx: int, top_k: int, swa_len: int,
                  groups: list[GroupSpec], Tq: int = 1, window_cap: int | None = None,
-                 device="cuda"):
+                 device="cuda", index_scan: str = "exact"):
+        if index_scan not in ("exact", "tc"):
+            raise ValueError(f"index_scan must be 'exact' or 'tc', not {index_scan!r}")
+        # "exact": the fixed fp32 score order (reproducible Top-K); "tc": the tensor-core
+        # scan for prefill chunks (relaxed summation order, see csa2_index_full_tc)
+        self.index_scan = index_scan
         self.B, self.H, self.H_I, self.d_idx = B, H, H_I, d_idx
         self.top_k, self.swa_len, self.Tq = top_k, swa_len, Tq
         self.groups = groups
@@ -168,10 +173,10 @@ class DecodeStack:
                                        swa_bf16[l], T_swa, swa_start, self.dev_err, stream)
             spec = self.groups[g]
             if lp.mode == "F":
-                bind.csa2_index_full(kv.struct, q_idx[l], w[l], q_pos, self.Tq, self.H_I, n_max[g],
-                                  spec.pool_blocks, self.top_k,
-                                  self.pool[g] if spec.pool_blocks else None, self.topk[l],
-                                  self.count[l], self.workspace, self.dev_err, stream)
+                full = bind.csa2_index_full_tc if self.index_scan == "tc" else bind.csa2_index_full
+                full(kv.struct, q_idx[l], w[l], q_pos, self.Tq, self.H_I, n_max[g],
+                     spec.pool_blocks, self.top_k, self.pool[g] if spec.pool_blocks else None,
+                     self.topk[l], self.count[l], self.workspace, self.dev_err, stream)
             elif lp.mode == "X":
                 bind.csa2_index_reindex(kv.struct, q_idx[l], w[l], q_pos, self.Tq, self.H_I,
                                      self.pool[g], spec.pool_blocks, self.top_k, self.topk[l],

@@ -117,3 +117,12 @@ def test_op_rooflines_dominant_and_traffic():
         expect = sum(tb * wl.B / b for tb, b in caps) if bench._sources_hash(files) == sha else None
         assert e["traffic"] == expect
     assert max(ops, key=lambda n: ops[n]["share_of_step"]) == "csa2_sparse_attn_decode_append"
+
+
+def test_code_hash_ignores_comments_only():
+    """The traffic key follows the code, not its comments."""
+    import bench
+    a = b"int f(int x) {  // doubles\n    return 2 * x;\n}\n"
+    b = b"// a new header line\nint f(int x) {  // twice x\n\n    return 2 * x;\n}\n"
+    c = b"int f(int x) {\n    return 3 * x;\n}\n"
+    assert bench.code_hash(a) == bench.code_hash(b) != bench.code_hash(c)

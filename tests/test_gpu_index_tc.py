@@ -167,3 +167,45 @@ def test_tc_full_size_prefill_chunk_sampled(pkg, orc):
     q_pos = [[wl.ctx - Tq + t for t in range(Tq)]]
     check = [(0, t) for t in (0, 1, 31, 32, 1000, 2047)]
     _tc_case(pkg, orc, rows, 2, q_pos, 0, 512, H_I, 60, check=check)
+
+
+def test_tc_stack_prefill_chunk(pkg, orc):
+    """The encoder stack (ratio 2, F + 5 U) on a 64-token prefill chunk with the
+    tensor-core scan: every query's Top-K is valid against the unrounded scores (a
+    position is left out only for one within the error bound of it), and every layer's
+    attention over the kernel's own selection matches the oracle."""
+    import csa2_harness
+    import oracle_ref as R
+    from synth.workloads import WORKLOADS, small_variant
+    wl = small_variant(WORKLOADS["prefill_chunk_enc"], B=1, ctx=3000 + 64, Tq=64)
+    dw = csa2_harness.DeviceWorkload(wl, index_scan="tc")
+    dw.step()
+    torch.cuda.synchronize()
+    assert dw.stack.dev_err.item() == 0
+    gpu = dw.request_state(0)
+    plan = R.reuse_sources(wl)
+    L = [layer for layer, (_, m, _) in enumerate(plan) if m == "F"][0]
+    caches = R.request_caches(wl, 0, main_rows={0: gpu["topk"][L].ravel()})
+    c = caches[0]
+    d = wl.d_I
+    for t, pos in enumerate(wl.q_positions()):
+        n = orc.visible(pos, wl.groups[0].ratio)
+        ex, mag = orc.scores_f64(c["idx_codes"], c["idx_scale"], wl.q_idx(L, 0)[t],
+                                 wl.w(L, 0)[t].numpy(), n=n)
+        tol = (d + wl.H_I + 2) * 2.0 ** -23 * mag
+        got = gpu["topk"][L][t]
+        k = min(n, wl.top_k)
+        assert gpu["count"][L][t] == k and (got[k:] == -1).all()
+        chosen = got[:k]
+        assert (np.diff(chosen) > 0).all() and chosen.min(initial=0) >= 0 and chosen.max(initial=0) < n
+        left = np.setdiff1d(np.arange(n), chosen)
+        if len(left):
+            # every left-out position scores at most the lowest chosen one, up to the bound
+            i = np.argmin(ex[chosen] + tol[chosen])
+            assert (ex[left] - tol[left] <= ex[chosen][i] + tol[chosen][i]).all(), t
+    for layer in range(len(plan)):
+        o_ref, l_ref = R.attention_layer(wl, 0, layer, caches, gpu["topk"][plan[layer][2]])
+        assert R.rel_err_rows(gpu["out"][layer], o_ref).max() <= 2e-3
+        fin = np.isfinite(l_ref)
+        assert np.array_equal(np.isfinite(gpu["lse"][layer]), fin)
+        assert np.abs(gpu["lse"][layer][fin] - l_ref[fin]).max(initial=0) <= 1e-3
