@@ -10,6 +10,7 @@ context 131072, decoder stack F+4X+15U (decode_128k).
   python bench.py --impl reference ...   (the CPU oracle as the reference arm)
   python bench.py --workload prefill_chunk_enc --index-scan tc
       (a 2048-token prefill chunk; the Full scan on the tensor cores)
+  python bench.py --rope   (pre-RoPE rows, rotated inside the append launches)
 
 Multi-GPU (torchrun): requests are independent, so each rank runs its own batch
 with no collective on the data path (weak scaling); timing is the max over ranks.
@@ -65,6 +66,9 @@ def op_bytes(wl) -> dict:
     n_win = min(wl.swa_len, wl.first_q_pos + 1)
     out["attn"] = BT * (K * 288 + K * 4 + n_win * 516 + wl.H * 512 * 2 + wl.H * 512 * 4 + wl.H * 4)
     out["swa_append"] = B * Tq * (512 * 2 + 516)
+    # RoPE inside the append: one (cos, sin) fp32 row of the table per rotated row
+    from synth.workloads import ROPE_PAIRS
+    out["rope_row"] = B * Tq * ROPE_PAIRS * 8
     return out
 
 
@@ -140,7 +144,12 @@ def op_rooflines(wl, plan, op_ms: dict, ms_step: float) -> dict:
             # attention launch
             "csa2_sparse_attn_decode_append": (ob["attn"] + ob["swa_append"],
                                                len(modes) - len({lp.group for lp in plan}),
-                                               "attn_tc_kernel (with the SWA append)")}
+                                               "attn_tc_kernel (with the SWA append)"),
+            # the same, the new row rotated first: its (cos, sin) row is read too
+            "csa2_sparse_attn_decode_append_rope": (
+                ob["attn"] + ob["swa_append"] + ob["rope_row"],
+                len(modes) - len({lp.group for lp in plan}),
+                "attn_tc_kernel (with the RoPE + SWA append)")}
     out = {}
     for name, ms in op_ms.items():
         nbytes, n, kernels = spec[name]
@@ -388,7 +397,7 @@ def run_ours(args, rank, world, local_rank):
         from synth.workloads import small_variant
         wl = small_variant(wl, B=args.batch, name=f"{wl.name}_b{args.batch}")
     wl = rank_workload(wl, rank)
-    dw = csa2_harness.DeviceWorkload(wl, device=dev, index_scan=args.index_scan)
+    dw = csa2_harness.DeviceWorkload(wl, device=dev, index_scan=args.index_scan, rope=args.rope)
     st = dw.stack
     inputs, dbuf, hbuf, in_bytes = pack_inputs(dw.inputs, dev)
     full_layers = [lp.layer for lp in st.plan if lp.mode == "F"]
@@ -411,7 +420,8 @@ def run_ours(args, rank, world, local_rank):
     # the last layer's attention: the fused SWA append + attention call in decode
     if st._fuse_swa(wl.Tq):
         n_attn = len(modes) - len({lp.group for lp in st.plan})
-        attn_pick = ("csa2_sparse_attn_decode_append", (n_attn, n_attn - 1))
+        attn_pick = ("csa2_sparse_attn_decode_append" + ("_rope" if args.rope else ""),
+                     (n_attn, n_attn - 1))
     else:
         attn_pick = ("csa2_sparse_attn_decode", (len(modes), len(modes) - 1))
     full_name = "csa2_index_full_tc" if args.index_scan == "tc" else "csa2_index_full"
@@ -536,6 +546,10 @@ def run_ours(args, rank, world, local_rank):
                    "pool": [g.pool_blocks for g in wl.groups],
                    "schedule": [g.schedule for g in wl.groups], "swa": wl.swa_len,
                    "query_tokens": wl.Tq, "index_scan": args.index_scan,
+                   "rope": ({"start": csa2_harness.ROPE_START,
+                             "pairs": csa2_harness.ROPE_PAIRS,
+                             "rows": "main KV and SWA, rotated inside the append launches"}
+                            if args.rope else None),
                    "parallelism": f"replicas x{world} (requests sharded, no collective)",
                    "l2": "inputs larger than L2: the Full scan streams "
                          f"{ob[f'index_full_g{g_full}'] / 1e9:.2f} GB per step",
@@ -588,6 +602,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--index-scan", default="exact", choices=["exact", "tc"],
                     help="Full-layer scan: fixed fp32 order, or tensor cores (prefill chunks)")
+    ap.add_argument("--rope", action="store_true",
+                    help="pass pre-RoPE rows and rotate them inside the append launches")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")

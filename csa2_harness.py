@@ -17,20 +17,24 @@ from __future__ import annotations
 
 import torch
 
-from fp4_kv_compressed_b200 import DecodeStack, GroupSpec, csa2_quantize_append
-from synth.workloads import Workload
+import synth
+from fp4_kv_compressed_b200 import (DecodeStack, GroupSpec, Rope, csa2_quantize_append,
+                                    csa2_quantize_append_rope)
+from synth.workloads import ROPE_PAIRS, ROPE_START, Workload
 
 
 class DeviceWorkload:
     def __init__(self, wl: Workload, device="cuda", chunk_elems: int = 1 << 25, fill=True,
-                 index_scan: str = "exact"):
+                 index_scan: str = "exact", rope: bool = False):
         self.wl = wl
         self.device = torch.device(device)
+        self.rope = (Rope(synth.rope_table(wl.ctx, ROPE_PAIRS), ROPE_START, ROPE_PAIRS, device)
+                     if rope else None)
         self.groups = [GroupSpec(g.ratio, g.schedule, g.pool_blocks, wl.entries(i))
                        for i, g in enumerate(wl.groups)]
         self.stack = DecodeStack(wl.B, wl.H, wl.H_I, wl.d_I, wl.top_k, wl.swa_len, self.groups,
                                  Tq=wl.Tq, window_cap=wl.window_cap, device=device,
-                                 index_scan=index_scan)
+                                 index_scan=index_scan, rope=self.rope)
         self.t0 = wl.first_q_pos
         self.chunk_elems = chunk_elems
         if fill:
@@ -48,17 +52,21 @@ class DeviceWorkload:
                 kv = wl.main_kv_batch(g, s, c, dev).contiguous()
                 ik = wl.idx_k_batch(g, s, c, dev).contiguous()
                 start = torch.full((wl.B,), s, dtype=torch.int32, device=dev)
-                csa2_quantize_append(st.kv[g].struct, kv, ik, c, start, None, None, 0, None,
-                                     st.dev_err)
+                self._append(st.kv[g].struct, kv, ik, c, start, None, None, 0, None)
         p0 = max(0, self.t0 - (wl.swa_len - 1))
         cnt = self.t0 - p0
         if cnt > 0:
             start = torch.full((wl.B,), p0, dtype=torch.int32, device=dev)
             for lp in st.plan:
                 rows = wl.swa_batch(lp.layer, p0, cnt, dev).contiguous()
-                csa2_quantize_append(None, None, None, 0, None, st.swa[lp.layer].struct, rows,
-                                     cnt, start, st.dev_err)
+                self._append(None, None, None, 0, None, st.swa[lp.layer].struct, rows, cnt, start)
         torch.cuda.synchronize(dev)
+
+    def _append(self, *args):
+        if self.rope is None:
+            csa2_quantize_append(*args, self.stack.dev_err)
+        else:
+            csa2_quantize_append_rope(*args, self.rope.struct, self.stack.dev_err)
 
     def step_inputs(self, device=None) -> dict:
         wl = self.wl

@@ -6,21 +6,23 @@ the C names (argument marshalling only) and the layer-stack driver that owns the
 device buffers.  Importing it loads the library and raises if it is missing.
 """
 from ._binding import (CSA2_OP_INDEX_FULL, CSA2_OP_INDEX_REINDEX, CSA2_OP_SPARSE_ATTN,
-                       CSA2GlobalKV, CSA2SWA, Csa2Error, DEVERR_INDEX, DEVERR_NMAX,
-                       DEVERR_RANGE, DEVERR_SLOT, EXPORTS, LIB_PATH, csa2_index_full,
-                       csa2_index_full_tc,
-                       csa2_index_reindex, csa2_quantize_append, csa2_read_device_error,
+                       CSA2GlobalKV, CSA2Rope, CSA2SWA, Csa2Error, DEVERR_INDEX, DEVERR_NMAX,
+                       DEVERR_RANGE, DEVERR_ROPE, DEVERR_SLOT, EXPORTS, LIB_PATH, Rope,
+                       csa2_index_full, csa2_index_full_tc, csa2_index_reindex,
+                       csa2_quantize_append, csa2_quantize_append_rope, csa2_read_device_error,
                        csa2_sparse_attn_decode, csa2_sparse_attn_decode_append,
-                       csa2_workspace_size, load_library)
+                       csa2_sparse_attn_decode_append_rope, csa2_workspace_size, load_library)
 from .stack import DecodeStack, GlobalKV, GroupSpec, LayerPlan, SwaRing, plan_layers
 
 load_library()
 
 __all__ = [
     "CSA2_OP_INDEX_FULL", "CSA2_OP_INDEX_REINDEX", "CSA2_OP_SPARSE_ATTN", "CSA2GlobalKV",
-    "CSA2SWA", "Csa2Error", "DEVERR_INDEX", "DEVERR_NMAX", "DEVERR_RANGE", "DEVERR_SLOT",
-    "EXPORTS", "LIB_PATH", "csa2_index_full", "csa2_index_full_tc", "csa2_index_reindex", "csa2_quantize_append",
-    "csa2_read_device_error", "csa2_sparse_attn_decode", "csa2_sparse_attn_decode_append",
+    "CSA2Rope", "CSA2SWA", "Csa2Error", "DEVERR_INDEX", "DEVERR_NMAX", "DEVERR_RANGE",
+    "DEVERR_ROPE", "DEVERR_SLOT", "EXPORTS", "LIB_PATH", "Rope", "csa2_index_full",
+    "csa2_index_full_tc", "csa2_index_reindex", "csa2_quantize_append",
+    "csa2_quantize_append_rope", "csa2_read_device_error", "csa2_sparse_attn_decode",
+    "csa2_sparse_attn_decode_append", "csa2_sparse_attn_decode_append_rope",
     "csa2_workspace_size",
     "load_library", "DecodeStack", "GlobalKV", "GroupSpec", "LayerPlan", "SwaRing",
     "plan_layers",

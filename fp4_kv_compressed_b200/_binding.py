@@ -24,12 +24,14 @@ STATUS = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_CAPACITY",
           6: "CSA2_ERR_DEVICE_BOUNDS"}
 
 DEVERR_SLOT, DEVERR_INDEX, DEVERR_NMAX, DEVERR_RANGE, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
+DEVERR_ROPE = 0x20
 
 # every symbol declared in include/csa2.h
-EXPORTS = ("csa2_quantize_append", "csa2_workspace_size", "csa2_index_full",
-           "csa2_index_full_tc", "csa2_index_full_noalloc", "csa2_index_reindex", "csa2_sparse_attn_decode",
-           "csa2_sparse_attn_decode_append", "csa2_read_device_error", "csa2_status_string",
-           "csa2_abi_version")
+EXPORTS = ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_workspace_size",
+           "csa2_index_full", "csa2_index_full_tc", "csa2_index_full_noalloc",
+           "csa2_index_reindex", "csa2_sparse_attn_decode", "csa2_sparse_attn_decode_append",
+           "csa2_sparse_attn_decode_append_rope", "csa2_read_device_error",
+           "csa2_status_string", "csa2_abi_version")
 
 
 class Csa2Error(RuntimeError):
@@ -50,6 +52,22 @@ class CSA2SWA(C.Structure):
                 ("window_cap", C.c_int32)]
 
 
+class CSA2Rope(C.Structure):
+    _fields_ = [("cos_sin", C.c_void_p), ("n_pos", C.c_int32), ("start", C.c_int32),
+                ("pairs", C.c_int32)]
+
+
+class Rope:
+    """A RoPE table on the device ([n_pos][pairs][2] fp32 (cos, sin)) with its channel
+    range, and the csa2_rope descriptor that points at it (kept alive together)."""
+
+    def __init__(self, cos_sin, start: int, pairs: int, device="cuda"):
+        t = torch.as_tensor(cos_sin, dtype=torch.float32).to(device).contiguous()
+        assert t.dim() == 3 and t.shape[1] == pairs and t.shape[2] == 2
+        self.table = t
+        self.struct = CSA2Rope(t.data_ptr(), t.shape[0], start, pairs)
+
+
 _lib = None
 
 
@@ -64,6 +82,7 @@ def load_library(path: str = LIB_PATH):
     L = C.CDLL(path)
     P, i32, sz = C.c_void_p, C.c_int32, C.c_size_t
     L.csa2_quantize_append.argtypes = [P, P, P, i32, P, P, P, i32, P, P, P]
+    L.csa2_quantize_append_rope.argtypes = [P, P, P, i32, P, P, P, i32, P, P, P, P]
     L.csa2_workspace_size.argtypes = [i32] * 7
     L.csa2_workspace_size.restype = sz
     L.csa2_index_full.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, P, P, P, P, sz, P, P]
@@ -73,12 +92,15 @@ def load_library(path: str = LIB_PATH):
                                           sz, P, P]
     L.csa2_sparse_attn_decode_append.argtypes = [P, P, P, P, P, i32, i32, P, i32, i32, C.c_float,
                                                  P, P, P, sz, P, P]
+    L.csa2_sparse_attn_decode_append_rope.argtypes = [P, P, P, P, P, i32, i32, P, i32, i32,
+                                                      C.c_float, P, P, P, P, sz, P, P]
     L.csa2_read_device_error.argtypes = [P, P, P]
     L.csa2_status_string.argtypes = [C.c_int]
     L.csa2_status_string.restype = C.c_char_p
     L.csa2_abi_version.restype = i32
-    for fn in ("csa2_quantize_append", "csa2_index_full", "csa2_index_full_tc", "csa2_index_reindex",
-               "csa2_sparse_attn_decode", "csa2_sparse_attn_decode_append",
+    for fn in ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_index_full",
+               "csa2_index_full_tc", "csa2_index_reindex", "csa2_sparse_attn_decode",
+               "csa2_sparse_attn_decode_append", "csa2_sparse_attn_decode_append_rope",
                "csa2_read_device_error"):
         getattr(L, fn).restype = C.c_int
     _lib = L
@@ -117,6 +139,20 @@ def csa2_quantize_append(kv: CSA2GlobalKV | None, kv_bf16, idxk_bf16, T_kv: int,
                                 C.byref(swa) if swa is not None else None, _ptr(swa_bf16),
                                 T_swa, _ptr(swa_start), _ptr(dev_err), _stream(stream))
     _check("csa2_quantize_append", st)
+
+
+def csa2_quantize_append_rope(kv: CSA2GlobalKV | None, kv_bf16, idxk_bf16, T_kv: int, kv_start,
+                              swa: CSA2SWA | None, swa_bf16, T_swa: int, swa_start,
+                              rope: CSA2Rope | None, dev_err=None, stream=None):
+    """csa2_quantize_append with RoPE applied to the main-KV and SWA rows first."""
+    L = load_library()
+    st = L.csa2_quantize_append_rope(C.byref(kv) if kv is not None else None, _ptr(kv_bf16),
+                                     _ptr(idxk_bf16), T_kv, _ptr(kv_start),
+                                     C.byref(swa) if swa is not None else None, _ptr(swa_bf16),
+                                     T_swa, _ptr(swa_start),
+                                     C.byref(rope) if rope is not None else None, _ptr(dev_err),
+                                     _stream(stream))
+    _check("csa2_quantize_append_rope", st)
 
 
 def csa2_index_full(kv: CSA2GlobalKV, q_idx, w, q_pos, Tq: int, H_I: int, n_max: int,
@@ -187,3 +223,17 @@ def csa2_read_device_error(dev_err, stream=None) -> int:
     if st not in (0, 6):
         _check("csa2_read_device_error", st)
     return bits.value
+
+
+def csa2_sparse_attn_decode_append_rope(kv: CSA2GlobalKV, swa: CSA2SWA, swa_bf16, q, q_pos,
+                                        Tq: int, H: int, topk, top_k: int, swa_len: int,
+                                        softmax_scale: float, rope: CSA2Rope | None, out, lse,
+                                        workspace=None, dev_err=None, stream=None):
+    """csa2_sparse_attn_decode_append with RoPE applied to the new SWA row first."""
+    L = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = L.csa2_sparse_attn_decode_append_rope(
+        C.byref(kv), C.byref(swa), _ptr(swa_bf16), _ptr(q), _ptr(q_pos), Tq, H, _ptr(topk), top_k,
+        swa_len, softmax_scale, C.byref(rope) if rope is not None else None, _ptr(out), _ptr(lse),
+        _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream))
+    _check("csa2_sparse_attn_decode_append_rope", st)

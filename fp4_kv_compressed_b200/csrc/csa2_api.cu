@@ -65,7 +65,7 @@ bool hi_supported(int32_t H_I) {
 
 extern "C" {
 
-int32_t csa2_abi_version(void) { return 100; }
+int32_t csa2_abi_version(void) { return 101; }
 
 const char *csa2_status_string(csa2_status st) {
     switch (st) {
@@ -98,14 +98,31 @@ size_t csa2_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t n_max, int
     }
 }
 
-csa2_status csa2_quantize_append(const csa2_global_kv *kv, const void *kv_bf16,
-                                 const void *idxk_bf16, int32_t T_kv, const int32_t *kv_start,
-                                 const csa2_swa *swa, const void *swa_bf16, int32_t T_swa,
-                                 const int32_t *swa_start, int32_t *dev_err,
-                                 csa2_stream_t stream) {
+// RoPE descriptor -> kernel arguments (nullptr: no rotation).
+static csa2_status rope_args(const csa2_rope *rope, RopeArgs *out) {
+    memset(out, 0, sizeof(*out));
+    if (!rope) return CSA2_OK;
+    if (!rope->cos_sin || !aligned(rope->cos_sin, 8) || rope->n_pos < 1) return CSA2_ERR_INVALID_ARG;
+    if (rope->start < 0 || rope->start % 2 != 0 || rope->pairs < 1 ||
+        (int64_t)rope->start + 2 * (int64_t)rope->pairs > CSA2_KV_DIM)
+        return CSA2_ERR_INVALID_ARG;
+    out->cs = reinterpret_cast<const float2 *>(rope->cos_sin);
+    out->n_pos = rope->n_pos;
+    out->start = rope->start;
+    out->pairs = rope->pairs;
+    return CSA2_OK;
+}
+
+static csa2_status quantize_append(const csa2_global_kv *kv, const void *kv_bf16,
+                                   const void *idxk_bf16, int32_t T_kv, const int32_t *kv_start,
+                                   const csa2_swa *swa, const void *swa_bf16, int32_t T_swa,
+                                   const int32_t *swa_start, const csa2_rope *rope,
+                                   int32_t *dev_err, csa2_stream_t stream) {
     QuantArgs a;
     memset(&a, 0, sizeof(a));
     a.dev_err = dev_err;
+    csa2_status rs = rope_args(rope, &a.rope);
+    if (rs != CSA2_OK) return rs;
     if (T_kv < 0 || T_swa < 0) return CSA2_ERR_INVALID_ARG;
     int32_t B = -1;
     if (T_kv > 0 && (kv_bf16 || idxk_bf16)) {
@@ -122,6 +139,7 @@ csa2_status csa2_quantize_append(const csa2_global_kv *kv, const void *kv_bf16,
         a.idx_scale = kv->idx_scale;
         a.cap = kv->cap;
         a.d_idx = kv->d_idx;
+        a.ratio = kv->ratio;
         a.kv_bf16 = (const uint16_t *)kv_bf16;
         a.idxk_bf16 = (const uint16_t *)idxk_bf16;
         a.T_kv = T_kv;
@@ -145,6 +163,25 @@ csa2_status csa2_quantize_append(const csa2_global_kv *kv, const void *kv_bf16,
         a.n_swa = (int64_t)swa->batch * T_swa;
     }
     return launched(launch_quantize_append(a, (cudaStream_t)stream));
+}
+
+csa2_status csa2_quantize_append(const csa2_global_kv *kv, const void *kv_bf16,
+                                 const void *idxk_bf16, int32_t T_kv, const int32_t *kv_start,
+                                 const csa2_swa *swa, const void *swa_bf16, int32_t T_swa,
+                                 const int32_t *swa_start, int32_t *dev_err,
+                                 csa2_stream_t stream) {
+    return quantize_append(kv, kv_bf16, idxk_bf16, T_kv, kv_start, swa, swa_bf16, T_swa, swa_start,
+                           nullptr, dev_err, stream);
+}
+
+csa2_status csa2_quantize_append_rope(const csa2_global_kv *kv, const void *kv_bf16,
+                                      const void *idxk_bf16, int32_t T_kv,
+                                      const int32_t *kv_start, const csa2_swa *swa,
+                                      const void *swa_bf16, int32_t T_swa,
+                                      const int32_t *swa_start, const csa2_rope *rope,
+                                      int32_t *dev_err, csa2_stream_t stream) {
+    return quantize_append(kv, kv_bf16, idxk_bf16, T_kv, kv_start, swa, swa_bf16, T_swa, swa_start,
+                           rope, dev_err, stream);
 }
 
 // Full layer: scan (exact CUDA-core order, or tensor cores) then pool / Top-K.
@@ -262,8 +299,8 @@ csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16,
 static csa2_status sparse_attn(const csa2_global_kv *kv, const csa2_swa *swa, const void *swa_new_bf16,
                                const void *q_bf16, const int32_t *q_pos, int32_t Tq, int32_t H,
                                const int32_t *topk, int32_t top_k, int32_t swa_len,
-                               float softmax_scale, float *out, float *lse, int32_t *dev_err,
-                               csa2_stream_t stream) {
+                               float softmax_scale, const csa2_rope *rope, float *out,
+                               float *lse, int32_t *dev_err, csa2_stream_t stream) {
     csa2_status st = check_kv(kv, false);
     if (st != CSA2_OK) return st;
     if (!q_bf16 || !q_pos || !out || !lse) return CSA2_ERR_INVALID_ARG;
@@ -302,6 +339,8 @@ static csa2_status sparse_attn(const csa2_global_kv *kv, const csa2_swa *swa, co
     a.swa_len = swa_len;
     a.softmax_scale = softmax_scale;
     a.swa_new = (const uint16_t *)swa_new_bf16;
+    st = rope_args(rope, &a.rope);
+    if (st != CSA2_OK) return st;
     a.out = out;
     a.lse = lse;
     a.dev_err = dev_err;
@@ -317,7 +356,7 @@ csa2_status csa2_sparse_attn_decode(const csa2_global_kv *kv, const csa2_swa *sw
     (void)workspace;
     (void)ws_bytes;
     return sparse_attn(kv, swa, nullptr, q_bf16, q_pos, Tq, H, topk, top_k, swa_len, softmax_scale,
-                       out, lse, dev_err, stream);
+                       nullptr, out, lse, dev_err, stream);
 }
 
 csa2_status csa2_sparse_attn_decode_append(const csa2_global_kv *kv, const csa2_swa *swa,
@@ -327,13 +366,23 @@ csa2_status csa2_sparse_attn_decode_append(const csa2_global_kv *kv, const csa2_
                                            float softmax_scale, float *out, float *lse,
                                            void *workspace, size_t ws_bytes, int32_t *dev_err,
                                            csa2_stream_t stream) {
+    return csa2_sparse_attn_decode_append_rope(kv, swa, swa_bf16, q_bf16, q_pos, Tq, H, topk, top_k,
+                                               swa_len, softmax_scale, nullptr, out, lse, workspace,
+                                               ws_bytes, dev_err, stream);
+}
+
+csa2_status csa2_sparse_attn_decode_append_rope(
+    const csa2_global_kv *kv, const csa2_swa *swa, const void *swa_bf16, const void *q_bf16,
+    const int32_t *q_pos, int32_t Tq, int32_t H, const int32_t *topk, int32_t top_k,
+    int32_t swa_len, float softmax_scale, const csa2_rope *rope, float *out, float *lse,
+    void *workspace, size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
     (void)workspace;
     (void)ws_bytes;
     if (Tq != 1) return CSA2_ERR_UNSUPPORTED;
     if (swa_len <= 0 || !swa || !swa_bf16) return CSA2_ERR_INVALID_ARG;
     if (!aligned(swa_bf16, 16)) return CSA2_ERR_INVALID_ARG;
     return sparse_attn(kv, swa, swa_bf16, q_bf16, q_pos, Tq, H, topk, top_k, swa_len, softmax_scale,
-                       out, lse, dev_err, stream);
+                       rope, out, lse, dev_err, stream);
 }
 
 csa2_status csa2_read_device_error(int32_t *dev_err, int32_t *bits_out, csa2_stream_t stream) {

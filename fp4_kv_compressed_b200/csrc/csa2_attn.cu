@@ -495,6 +495,9 @@ attn_tc_kernel(AttnArgs a) {
         // The same FP8 row quantiser as csa2_quantize_append: codes and sigma go to
         // shared memory (this CTA's producers read the window's newest key from there)
         // and, from head group 0's CTA that owns that key, to the ring slot t % wcap.
+        if (!rope_lane16(xnew, lane, a.rope.cs, a.rope.n_pos, a.rope.start, a.rope.pairs, t) &&
+            lane == 0)
+            set_dev_err(a.dev_err, CSA2_DEVERR_ROPE);
         quant_fp8_lanes<kDim>(xnew, s.swa_new, &s.swa_new_sigma, lane);
         const int last_tile = (n_sel + n_win - 1) / kTK;
         const int n_all0 = (n_sel + n_win + kTK - 1) / kTK;

@@ -6,6 +6,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 #include "csa2.h"
@@ -160,6 +161,38 @@ __device__ void quant_fp8_row(const uint16_t *src, uint8_t *dst_codes, float *ds
         x[1] = bf16_bits_to_f32(v >> 16);
     }
     quant_fp8_lanes<WIDTH>(x, dst_codes, dst_scale, lane);
+}
+
+// RoPE of one 512-channel row inside the append (csa2_rope): lane l holds channels
+// [16 l, 16 l + 16) as fp32 in x; the rotated pairs among them become
+//   y0 = fma(x0, c, -(x1 * s)),  y1 = fma(x0, s, x1 * c),
+// with (c, s) = cs[pos][i] for pair i = (channel - start) / 2, each rounded to bf16.
+// cs == nullptr rotates nothing; a position outside [0, n_pos) rotates nothing and
+// returns false.
+__device__ __forceinline__ bool rope_lane16(float *x, int lane, const float2 *cs, int n_pos,
+                                            int start, int pairs, int64_t pos) {
+    if (cs == nullptr) return true;
+    if (pos < 0 || pos >= n_pos) return false;
+    const float2 *row = cs + pos * pairs;
+    float2 t[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {             // every table load in flight together
+        const int ch = 16 * lane + 2 * k;
+        t[k] = ch >= start && ch < start + 2 * pairs ? __ldg(row + ((ch - start) >> 1))
+                                                      : make_float2(1.0f, 0.0f);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int ch = 16 * lane + 2 * k;
+        if (ch >= start && ch < start + 2 * pairs) {
+            const float x0 = x[2 * k], x1 = x[2 * k + 1];
+            const float y0 = fmaf(x0, t[k].x, -__fmul_rn(x1, t[k].y));
+            const float y1 = fmaf(x0, t[k].y, __fmul_rn(x1, t[k].x));
+            x[2 * k] = __bfloat162float(__float2bfloat16_rn(y0));
+            x[2 * k + 1] = __bfloat162float(__float2bfloat16_rn(y1));
+        }
+    }
+    return true;
 }
 
 // Programmatic dependent launch.  Every kernel of the library is launched so that the

@@ -6,6 +6,14 @@
 
 namespace csa2 {
 
+// RoPE table of the _rope calls (cs == nullptr: no rotation); see csa2_rope.
+struct RopeArgs {
+    const float2 *cs;        // [n_pos][pairs] (cos, sin)
+    int32_t n_pos;
+    int32_t start;
+    int32_t pairs;
+};
+
 struct QuantArgs {
     // main KV group (FP4 + FP8 indexer K)
     uint8_t *codes;
@@ -14,6 +22,8 @@ struct QuantArgs {
     float *idx_scale;
     int32_t cap;
     int32_t d_idx;
+    int32_t ratio;           // main entry in slot e sits at token position ratio * e + ratio - 1
+    RopeArgs rope;
     const uint16_t *kv_bf16;
     const uint16_t *idxk_bf16;
     int32_t T_kv;
@@ -64,6 +74,7 @@ struct AttnArgs {
     float *swa_scale;
     int32_t wcap;
     const uint16_t *swa_new; // fused append: [BT][512] bf16 new SWA row per query (Tq = 1), or null
+    RopeArgs rope;           // fused append: RoPE of the new row at its token position
     const uint16_t *q;       // [BT][H][512] bf16 bits
     const int32_t *q_pos;
     int32_t Tq;

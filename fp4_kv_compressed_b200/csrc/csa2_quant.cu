@@ -8,6 +8,10 @@
 // E2M1_RNE(x / scale) with saturation (a zero scale stores zero codes); FP8 rows
 // use sigma = amax / 448 and codes = E4M3_RNE(x / sigma).
 //
+// With a RoPE table (csa2_quantize_append_rope) the main and SWA rows are rotated in
+// registers first (rope_lane16), the rotated values rounded to bf16, so the codes are
+// those of the plain call given the rotated rows.
+//
 // One warp per row.  FP4 entry: lane l owns scale group l (16 channels, two
 // 16-byte loads) and writes 8 code bytes + 1 scale byte, so a warp writes the
 // entry's 256 + 32 bytes with coalesced stores.
@@ -29,6 +33,9 @@ __device__ void quant_fp4_entry(const QuantArgs &a, int64_t row, int lane) {
     float x[16];
     unpack_bf16x8(src[0], x);
     unpack_bf16x8(src[1], x + 8);
+    if (!rope_lane16(x, lane, a.rope.cs, a.rope.n_pos, a.rope.start, a.rope.pairs,
+                     slot * a.ratio + a.ratio - 1) && lane == 0)
+        set_dev_err(a.dev_err, CSA2_DEVERR_ROPE);
     float amax = 0.0f;
 #pragma unroll
     for (int c = 0; c < 16; ++c) amax = fmaxf(amax, fabsf(x[c]));
@@ -81,7 +88,14 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(QuantArgs a) {
             return;
         }
         const int64_t e = (int64_t)b * a.wcap + pos % a.wcap;
-        quant_fp8_row<512>(a.swa_bf16 + warp * kDim, a.swa_codes + e * kDim, a.swa_scale + e, lane);
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.swa_bf16 + warp * kDim + 16 * lane);
+        float x[16];
+        unpack_bf16x8(src[0], x);
+        unpack_bf16x8(src[1], x + 8);
+        if (!rope_lane16(x, lane, a.rope.cs, a.rope.n_pos, a.rope.start, a.rope.pairs, pos) &&
+            lane == 0)
+            set_dev_err(a.dev_err, CSA2_DEVERR_ROPE);
+        quant_fp8_lanes<512>(x, a.swa_codes + e * kDim, a.swa_scale + e, lane);
     }
 }
 

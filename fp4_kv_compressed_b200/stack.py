@@ -97,12 +97,15 @@ class DecodeStack:
 
     def __init__(self, B: int, H: int, H_I: int, d_idx: int, top_k: int, swa_len: int,
                  groups: list[GroupSpec], Tq: int = 1, window_cap: int | None = None,
-                 device="cuda", index_scan: str = "exact"):
+                 device="cuda", index_scan: str = "exact", rope=None):
         if index_scan not in ("exact", "tc"):
             raise ValueError(f"index_scan must be 'exact' or 'tc', not {index_scan!r}")
         # "exact": the fixed fp32 score order (reproducible Top-K); "tc": the tensor-core
         # scan for prefill chunks (relaxed summation order, see csa2_index_full_tc)
         self.index_scan = index_scan
+        # a _binding.Rope: the main-KV and SWA rows are passed before RoPE and rotated
+        # inside the append launches (csa2_quantize_append_rope and the fused attention)
+        self.rope = rope
         self.B, self.H, self.H_I, self.d_idx = B, H, H_I, d_idx
         self.top_k, self.swa_len, self.Tq = top_k, swa_len, Tq
         self.groups = groups
@@ -160,17 +163,23 @@ class DecodeStack:
         for lp in self.plan:
             first_of_group.setdefault(lp.group, lp.layer)
         T_swa = swa_bf16[0].shape[1] if swa_bf16[0] is not None else 0
+        rope = self.rope.struct if self.rope is not None else None
+
+        def append(*args):
+            if rope is None:
+                bind.csa2_quantize_append(*args, self.dev_err, stream)
+            else:
+                bind.csa2_quantize_append_rope(*args, rope, self.dev_err, stream)
+
         for lp in self.plan:
             g, l = lp.group, lp.layer
             kv = self.kv[g]
             if l == first_of_group[g] and kv_bf16 is not None and kv_bf16[g] is not None:
                 T_kv = kv_bf16[g].shape[1]
-                bind.csa2_quantize_append(kv.struct, kv_bf16[g], idxk_bf16[g], T_kv, kv_start[g],
-                                       self.swa[l].struct, swa_bf16[l], T_swa, swa_start,
-                                       self.dev_err, stream)
+                append(kv.struct, kv_bf16[g], idxk_bf16[g], T_kv, kv_start[g], self.swa[l].struct,
+                       swa_bf16[l], T_swa, swa_start)
             elif swa_bf16[l] is not None and not self._fuse_swa(T_swa):
-                bind.csa2_quantize_append(None, None, None, 0, None, self.swa[l].struct,
-                                       swa_bf16[l], T_swa, swa_start, self.dev_err, stream)
+                append(None, None, None, 0, None, self.swa[l].struct, swa_bf16[l], T_swa, swa_start)
             spec = self.groups[g]
             if lp.mode == "F":
                 full = bind.csa2_index_full_tc if self.index_scan == "tc" else bind.csa2_index_full
@@ -183,7 +192,12 @@ class DecodeStack:
                                      self.count[l], self.workspace, self.dev_err, stream)
             fused = (l != first_of_group[g] or kv_bf16 is None or kv_bf16[g] is None) \
                 and swa_bf16[l] is not None and self._fuse_swa(T_swa)
-            if fused:       # the layer's SWA row is appended inside the attention launch
+            if fused and rope is not None:
+                bind.csa2_sparse_attn_decode_append_rope(
+                    kv.struct, self.swa[l].struct, swa_bf16[l], q[l], q_pos, self.Tq, self.H,
+                    self.topk_of(l), self.top_k, self.swa_len, self.softmax_scale, rope,
+                    self.out[l], self.lse[l], self.workspace, self.dev_err, stream)
+            elif fused:     # the layer's SWA row is appended inside the attention launch
                 bind.csa2_sparse_attn_decode_append(
                     kv.struct, self.swa[l].struct, swa_bf16[l], q[l], q_pos, self.Tq, self.H,
                     self.topk_of(l), self.top_k, self.swa_len, self.softmax_scale, self.out[l],

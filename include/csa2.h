@@ -67,6 +67,7 @@ typedef enum csa2_status {
 #define CSA2_DEVERR_NMAX 0x4      /* a query sees more entries than n_max */
 #define CSA2_DEVERR_RANGE 0x8     /* a dequantised SWA value beyond the fp16 range */
 #define CSA2_DEVERR_TIMEOUT 0x10  /* a kernel's bounded wait gave up (internal error) */
+#define CSA2_DEVERR_ROPE 0x20     /* a row's position lies outside the RoPE table */
 
 /* Limits of the kernels. */
 #define CSA2_KV_DIM 512           /* shared K=V latent width (MQA) */
@@ -114,6 +115,32 @@ typedef struct csa2_swa {
 } csa2_swa;
 
 /*
+ * RoPE applied inside the append (the _rope calls below).  The quantisation point
+ * is after RoPE (myzaker "cache precision and tiering"), so a caller holding
+ * pre-RoPE rows can rotate and quantise in one pass.  The pages give neither the
+ * rotated channels nor the frequencies, so both are inputs:
+ *   cos_sin  float [n_pos][pairs][2]: (cos, sin) of the angle of pair i at token
+ *            position p, 8-byte aligned;
+ *   start    first rotated channel of the 512-channel latent (even);
+ *   pairs    rotated channel pairs (2i, 2i+1) = start + 2i, start + 2i + 1, with
+ *            start + 2 * pairs <= 512.
+ * A pair (x0, x1) at position p becomes, in fp32,
+ *   y0 = fma(x0, c, -(x1 * s)),  y1 = fma(x0, s, x1 * c)   (products rounded first)
+ * and each of y0, y1 is rounded to bf16 (nearest, ties to even), so the stored
+ * codes equal those of the plain call given the rotated bf16 rows.  Channels
+ * outside the range pass unchanged.  The position of an SWA row is its token
+ * position; that of a main entry in slot e is ratio * e + ratio - 1 (its last
+ * token).  Indexer-K rows are taken as given (not rotated).  A row whose
+ * position is outside [0, n_pos) is stored unrotated and flags CSA2_DEVERR_ROPE.
+ */
+typedef struct csa2_rope {
+    const float *cos_sin;
+    int32_t n_pos;
+    int32_t start;
+    int32_t pairs;
+} csa2_rope;
+
+/*
  * a1/a2 quantise-append.  Main KV entries are quantised to FP4 after RoPE
  * (myzaker "cache precision": the quantisation point is after RoPE, so the
  * inputs here are post-RoPE): per 16 channels, scale = E4M3(amax / 6) and
@@ -135,6 +162,17 @@ CSA2_API csa2_status csa2_quantize_append(const csa2_global_kv *kv, const void *
                                  const csa2_swa *swa, const void *swa_bf16, int32_t T_swa,
                                  const int32_t *swa_start, int32_t *dev_err,
                                  csa2_stream_t stream);
+
+/* csa2_quantize_append with RoPE applied to the main-KV and SWA rows first (see
+ * csa2_rope; rope NULL = csa2_quantize_append).  Invalid rope fields (NULL table,
+ * n_pos < 1, odd or negative start, pairs < 1, start + 2 * pairs > 512, a table
+ * not 8-byte aligned) return CSA2_ERR_INVALID_ARG. */
+CSA2_API csa2_status csa2_quantize_append_rope(const csa2_global_kv *kv, const void *kv_bf16,
+                                               const void *idxk_bf16, int32_t T_kv,
+                                               const int32_t *kv_start, const csa2_swa *swa,
+                                               const void *swa_bf16, int32_t T_swa,
+                                               const int32_t *swa_start, const csa2_rope *rope,
+                                               int32_t *dev_err, csa2_stream_t stream);
 
 /* Operation ids for csa2_workspace_size. */
 #define CSA2_OP_INDEX_FULL 1
@@ -280,6 +318,15 @@ CSA2_API csa2_status csa2_sparse_attn_decode_append(const csa2_global_kv *kv, co
                                            float softmax_scale, float *out, float *lse,
                                            void *workspace, size_t ws_bytes, int32_t *dev_err,
                                            csa2_stream_t stream);
+
+/* csa2_sparse_attn_decode_append with RoPE applied to the new SWA row (at its
+ * token position q_pos) before it is quantised; rope NULL = the plain call.  Same
+ * rope checks as csa2_quantize_append_rope. */
+CSA2_API csa2_status csa2_sparse_attn_decode_append_rope(
+    const csa2_global_kv *kv, const csa2_swa *swa, const void *swa_bf16, const void *q_bf16,
+    const int32_t *q_pos, int32_t Tq, int32_t H, const int32_t *topk, int32_t top_k,
+    int32_t swa_len, float softmax_scale, const csa2_rope *rope, float *out, float *lse,
+    void *workspace, size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream);
 
 /* Synchronise `stream`, read *dev_err (device int32) into *bits_out (host),
  * reset it to 0, and return CSA2_ERR_DEVICE_BOUNDS if any bit was set. */

@@ -27,6 +27,8 @@ def lib():
         i32, i64, f32, f64 = C.c_int32, C.c_int64, C.c_float, C.c_double
         sig = {
             "csa2o_bf16_to_f32": (f32, [C.c_uint16]),
+            "csa2o_f32_to_bf16": (C.c_uint16, [f32]),
+            "csa2o_rope_rows": (i64, [P, i64, C.c_int, P, P, i64, C.c_int, C.c_int, P]),
             "csa2o_e2m1_value": (f64, [C.c_int]),
             "csa2o_e4m3_value": (f64, [C.c_int]),
             "csa2o_e2m1_encode": (C.c_int, [f32]),
@@ -94,6 +96,27 @@ def e2m1_encode(r: float) -> int:
 
 def e4m3_encode(x: float) -> int:
     return lib().csa2o_e4m3_encode(x)
+
+
+def f32_to_bf16(v: float) -> int:
+    return lib().csa2o_f32_to_bf16(v)
+
+
+def rope_rows(x, pos, cos_sin: np.ndarray, start: int, pairs: int) -> tuple[np.ndarray, int]:
+    """bf16 rows [..., W] at token positions pos [...] -> (rotated bf16 rows as uint16,
+    number of rows whose position is outside the table and stay unrotated)."""
+    xb = as_bf16_bits(x)
+    shape = xb.shape
+    W = shape[-1]
+    xb = np.ascontiguousarray(xb.reshape(-1, W))
+    pos = np.ascontiguousarray(np.asarray(pos, np.int64).reshape(-1))
+    assert len(pos) == xb.shape[0]
+    cs = np.ascontiguousarray(cos_sin, np.float32)
+    assert cs.shape[1:] == (pairs, 2)
+    out = np.zeros_like(xb)
+    n_out = lib().csa2o_rope_rows(_p(xb), xb.shape[0], W, _p(pos), _p(cs), cs.shape[0], start,
+                                  pairs, _p(out))
+    return out.reshape(shape), n_out
 
 
 # ---- a1 / a2 --------------------------------------------------------------------------------

@@ -39,6 +39,17 @@ EXPORT float csa2o_bf16_to_f32(uint16_t h) {
     return f;
 }
 
+/* fp32 -> bf16, round to nearest with ties to even (NaN stays a quiet NaN).  On the
+ * bit pattern: add half of the dropped range minus one, plus the kept lsb, then
+ * drop the low 16 bits. */
+EXPORT uint16_t csa2o_f32_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((u >> 16) | 0x0040u);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
 /* E2M1 (study notes, section 4 "main KV from FP8 to FP4": 4-bit E2M1 values).
  * Code = sign(1) | exponent(2) | mantissa(1); magnitudes by code 0..7. */
 static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
@@ -193,6 +204,45 @@ EXPORT void csa2o_dequant_fp8(const uint8_t *codes, const float *scale, int64_t 
     for (int64_t r = 0; r < rows; ++r)
         for (int c = 0; c < width; ++c)
             out[r * width + c] = csa2o_e4m3_value(codes[r * width + c]) * (double)scale[r];
+}
+
+/* ------------------------------------------------------------------------ */
+/* RoPE inside the append                                                    */
+/* ------------------------------------------------------------------------ */
+/* The main KV is quantised after RoPE (myzaker "cache precision and tiering").
+ * The pages give neither the rotated channels nor the angles, so both are
+ * inputs: cs [n_pos][pairs][2] holds (cos, sin) of pair i at token position p;
+ * pair i is channels start + 2i, start + 2i + 1 of a width-channel bf16 row.
+ * Reading fixed for this build: a pair (x0, x1) becomes, in fp32 with the
+ * products rounded first, y0 = fma(x0, c, -(x1 s)) and y1 = fma(x0, s, x1 c),
+ * each rounded to bf16 -- the rows a separate RoPE step would store before the
+ * append.  Other channels are copied.  pos[r] is row r's token position; a row
+ * whose position is outside [0, n_pos) is copied unrotated.  Returns the number
+ * of such rows. */
+EXPORT int64_t csa2o_rope_rows(const uint16_t *x, int64_t rows, int width, const int64_t *pos,
+                               const float *cs, int64_t n_pos, int start, int pairs,
+                               uint16_t *out) {
+    int64_t outside = 0;
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t *xr = x + r * width;
+        uint16_t *yr = out + r * width;
+        memcpy(yr, xr, sizeof(uint16_t) * (size_t)width);
+        int64_t p = pos[r];
+        if (p < 0 || p >= n_pos) {
+            ++outside;
+            continue;
+        }
+        for (int i = 0; i < pairs; ++i) {
+            int j = start + 2 * i;
+            float x0 = csa2o_bf16_to_f32(xr[j]), x1 = csa2o_bf16_to_f32(xr[j + 1]);
+            float c = cs[(p * pairs + i) * 2], sn = cs[(p * pairs + i) * 2 + 1];
+            float m0 = x1 * sn;
+            float m1 = x1 * c;
+            yr[j] = csa2o_f32_to_bf16(fmaf(x0, c, -m0));
+            yr[j + 1] = csa2o_f32_to_bf16(fmaf(x0, sn, m1));
+        }
+    }
+    return outside;
 }
 
 /* ------------------------------------------------------------------------ */

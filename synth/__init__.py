@@ -135,3 +135,13 @@ def rows_uniform_f32(seed: int, name: str, b: int, start: int, count: int, width
                      device="cpu", stride: int = Q_STRIDE) -> torch.Tensor:
     idx = row_indices(b, start, count, width, stride, device)
     return uniform_f32(seed, name, idx).view(count, width)
+
+
+def rope_table(n_pos: int, pairs: int, base: float = 10000.0) -> np.ndarray:
+    """A RoPE angle table as the _rope calls take it: fp32 [n_pos][pairs][2] holding
+    (cos, sin) of p * base^(-i / pairs).  The pages give no frequencies; this is the
+    common geometric choice, used as a synthetic input (the library applies any table)."""
+    p = np.arange(n_pos, dtype=np.float64)[:, None]
+    inv = base ** (-np.arange(pairs, dtype=np.float64) / pairs)
+    ang = p * inv[None, :]
+    return np.ascontiguousarray(np.stack([np.cos(ang), np.sin(ang)], -1).astype(np.float32))

@@ -23,6 +23,10 @@ from . import POS_STRIDE, Q_STRIDE, row_indices, rows_normal_bf16, rows_uniform_
 KV_DIM = 512            # shared K=V latent width
 DECODER_SCHEDULE = "FUUUXUUUXUUUXUUUXUUU"   # 1 Full + 4 Reindex + 15 Reuse
 ENCODER_SCHEDULE = "FUUUUU"                 # 1 Full + 5 Reuse, flat indexer
+# RoPE runs (pre-RoPE rows rotated inside the append): the last 64 of the 512 latent
+# channels.  The pages give neither the rotated channels nor the angles; the angles
+# come from synth.rope_table.
+ROPE_START, ROPE_PAIRS = 448, 32
 
 
 @dataclass(frozen=True)

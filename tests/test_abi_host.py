@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol(pkg):
     assert set(names) == set(pkg.EXPORTS)
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.csa2_abi_version() == 100
+    assert lib.csa2_abi_version() == 101      # 1.1: the _rope calls and the tensor-core scan
     for st in range(7):
         assert lib.csa2_status_string(st)
 
@@ -88,6 +88,16 @@ def test_validation_rejects_before_launch(pkg):
     assert lib.csa2_sparse_attn_decode_append(C.byref(kv), C.byref(swa), C.c_void_p(4100), qbuf,
                                               qbuf, 1, 64, qbuf, 8, 128, C.c_float(0.04), qbuf,
                                               qbuf, None, 0, None, None) == 1
+    # RoPE descriptors: null table, odd start, range past channel 511, no pairs, no rows,
+    # misaligned table -- each rejected before any launch, in both _rope calls
+    for bad in [(0, 8, 0, 4), (4096, 8, 3, 4), (4096, 8, 500, 8), (4096, 8, 0, 0),
+                (4096, 0, 0, 4), (4100, 8, 0, 4)]:
+        rope = pkg.CSA2Rope(*bad)
+        assert lib.csa2_quantize_append_rope(None, None, None, 0, None, C.byref(swa), qbuf, 1, qbuf,
+                                             C.byref(rope), None, None) == 1, bad
+        assert lib.csa2_sparse_attn_decode_append_rope(
+            C.byref(kv), C.byref(swa), qbuf, qbuf, qbuf, 1, 64, qbuf, 8, 128, C.c_float(0.04),
+            C.byref(rope), qbuf, qbuf, None, 0, None, None) == 1, bad
     # append: slot count beyond the cache
     assert lib.csa2_quantize_append(C.byref(kv), qbuf, None, 101, qbuf, None, None, 0, None,
                                     None, None) == 2
