@@ -400,6 +400,9 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // ---------------------------------------------------------------------------------------
+// kRope: the fused append rotates the new SWA row first (a separate instantiation, so
+// that the plain kernel carries none of its code).
+template <bool kRope>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 attn_tc_kernel(AttnArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -495,9 +498,11 @@ attn_tc_kernel(AttnArgs a) {
         // The same FP8 row quantiser as csa2_quantize_append: codes and sigma go to
         // shared memory (this CTA's producers read the window's newest key from there)
         // and, from head group 0's CTA that owns that key, to the ring slot t % wcap.
-        if (!rope_lane16(xnew, lane, a.rope.cs, a.rope.n_pos, a.rope.start, a.rope.pairs, t) &&
-            lane == 0)
-            set_dev_err(a.dev_err, CSA2_DEVERR_ROPE);
+        if constexpr (kRope) {
+            if (!rope_lane16(xnew, lane, a.rope.cs, a.rope.n_pos, a.rope.start, a.rope.pairs, t) &&
+                lane == 0)
+                set_dev_err(a.dev_err, CSA2_DEVERR_ROPE);
+        }
         quant_fp8_lanes<kDim>(xnew, s.swa_new, &s.swa_new_sigma, lane);
         const int last_tile = (n_sel + n_win - 1) / kTK;
         const int n_all0 = (n_sel + n_win + kTK - 1) / kTK;
@@ -863,20 +868,26 @@ attn_tc_kernel(AttnArgs a) {
 
 size_t attn_tc_smem_bytes() { return sizeof(tc::Smem) + 1024; }
 
-cudaError_t launch_sparse_attn(const AttnArgs &a, int BT, cudaStream_t st) {
+template <bool kRope>
+static cudaError_t launch_attn_t(const AttnArgs &a, int BT, cudaStream_t st) {
     const size_t smem = attn_tc_smem_bytes();
-    static bool attr_set = false;  // once per process (one device per process)
+    static bool attr_set = false;  // once per process and instantiation (one device per process)
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel,
+        cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel<kRope>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        e = prefer_max_smem(tc::attn_tc_kernel);
+        e = prefer_max_smem(tc::attn_tc_kernel<kRope>);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
     dim3 grid(2 * BT, (a.H + tc::kHeads - 1) / tc::kHeads);   // 2-CTA clusters
-    cudaError_t e = launch_pdl(tc::attn_tc_kernel, grid, dim3(tc::kThreads), smem, st, a);
+    cudaError_t e = launch_pdl(tc::attn_tc_kernel<kRope>, grid, dim3(tc::kThreads), smem, st, a);
     return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_sparse_attn(const AttnArgs &a, int BT, cudaStream_t st) {
+    return a.swa_new != nullptr && a.rope.cs != nullptr ? launch_attn_t<true>(a, BT, st)
+                                                         : launch_attn_t<false>(a, BT, st);
 }
 
 }  // namespace csa2
