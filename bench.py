@@ -89,8 +89,8 @@ def attn_flops(wl) -> int:
 # sources at capture time).  Reported, each kernel scaled to the batch, only while the
 # code is unchanged.  Captures: profiles/*.md.
 NCU_TRAFFIC = {
-    "csa2_sparse_attn_decode": ([(21_212_416, 64)], ("csa2_attn.cu",), "139e5cf6f85cdcdd"),
-    "csa2_sparse_attn_decode_append": ([(21_212_416, 64)], ("csa2_attn.cu",), "139e5cf6f85cdcdd"),
+    "csa2_sparse_attn_decode": ([(21_211_392, 64)], ("csa2_attn.cu",), "f8a8dd610b4ba7ac"),
+    "csa2_sparse_attn_decode_append": ([(21_211_392, 64)], ("csa2_attn.cu",), "f8a8dd610b4ba7ac"),
     "csa2_index_full": ([(138_484_992 + 4_945_664, 8), (18_141_952, 64)], ("csa2_index.cu",),
                         "33472cf35d49fbf2"),
     "csa2_index_reindex": ([(18_606_080, 8), (4_754_432, 64)], ("csa2_index.cu",),
