@@ -273,16 +273,22 @@ reindex_score_kernel(IndexArgs a) {
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelStageMax = 16384;   // keys staged in shared memory up to this count
+// Flat selections over more keys (prefill chunks, long encoder groups) use a second
+// instantiation that stages up to kSelStageWide keys (192 KB, one CTA per SM) and so
+// reads its row from HBM once instead of once per radix pass.
+constexpr int kSelStageWide = 49152;
 constexpr int kSelDigit = 11;         // bits per radix pass
 
-struct SelSmem {
+template <int kCap>
+struct SelSmemT {
     uint32_t hist[1 << kSelDigit];
     int wa[kSelWarps], wb[kSelWarps];
     uint32_t wmin[kSelWarps], wmax[kSelWarps];
     int bcast[4];
     alignas(16) int pool[CSA2_POOL_MAX];
-    alignas(16) uint32_t keys[kSelStageMax];
+    alignas(16) uint32_t keys[kCap];
 };
+using SelSmem = SelSmemT<kSelStageMax>;
 
 // Exclusive scans (in warp order) of s.wa and s.wb; totals in s.bcast[0], s.bcast[1].
 // Call with every warp's entry written; ends with a barrier.
@@ -298,7 +304,8 @@ __device__ __forceinline__ void stage_raw(uint32_t *dst, const void *src, int n)
     cp_async_wait_all();
 }
 
-__device__ __forceinline__ void sel_scan_warps(SelSmem &s) {
+template <class S>
+__device__ __forceinline__ void sel_scan_warps(S &s) {
     __syncthreads();
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
@@ -318,7 +325,8 @@ __device__ __forceinline__ void sel_scan_warps(SelSmem &s) {
 
 // The bin (of nbins, visited from the top) holding the rem-th largest counted key:
 // bin, number of counted keys in higher bins, population of the bin.
-__device__ __forceinline__ void sel_find_bin(SelSmem &s, int nbins, int rem, int &bin, int &above,
+template <class S>
+__device__ __forceinline__ void sel_find_bin(S &s, int nbins, int rem, int &bin, int &above,
                                              int &cnt) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int per = (nbins + kSelThreads - 1) / kSelThreads;   // 1 or 2 bins per thread
@@ -357,8 +365,8 @@ __device__ __forceinline__ void sel_find_bin(SelSmem &s, int nbins, int rem, int
 
 // Top-k of n candidates (keys from key_at, 0 = not a candidate) -> ascending ids in
 // out[0..cnt), cnt = min(k, #valid) returned.
-template <class KeyAt, class IdAt>
-__device__ int block_topk(KeyAt key_at, IdAt id_at, int n, int k, int *out, SelSmem &s) {
+template <class KeyAt, class IdAt, class S>
+__device__ int block_topk(KeyAt key_at, IdAt id_at, int n, int k, int *out, S &s) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // valid count, smallest and largest valid key
     int nv = 0;
@@ -478,10 +486,11 @@ __device__ int block_topk(KeyAt key_at, IdAt id_at, int n, int k, int *out, SelS
 // inside the pool's positions (equal to Top-K over all positions because every
 // pool block's best position outranks any position outside the pool, and
 // pool_blocks >= top_k).  Flat: Top-K over all visible positions.
+template <int kCap>
 __global__ void __launch_bounds__(kSelThreads)
 select_full_kernel(IndexArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    SelSmem &s = *reinterpret_cast<SelSmem *>(smem_raw);
+    SelSmemT<kCap> &s = *reinterpret_cast<SelSmemT<kCap> *>(smem_raw);
     __shared__ int sel_out[CSA2_TOPK_MAX];
     grid_dep_wait();
     const int qi = blockIdx.x;
@@ -493,7 +502,7 @@ select_full_kernel(IndexArgs a) {
     if (a.pool_blocks > 0) {
         const int nb = (N + 7) / 8;
         const float *bm = a.bmax + (int64_t)qi * a.bmax_stride;
-        const bool staged = nb <= kSelStageMax;
+        const bool staged = nb <= kCap;
         if (staged) {
             stage_raw(s.keys, bm, nb);
             __syncthreads();
@@ -526,7 +535,7 @@ select_full_kernel(IndexArgs a) {
         auto cid = [&](int i) -> int { return s.pool[i >> 3] * 8 + (i & 7); };
         cnt = block_topk(ckey, cid, nc, a.top_k, sel_out, s);
     } else {
-        const bool staged = N <= kSelStageMax;
+        const bool staged = N <= kCap;
         if (staged) {
             stage_raw(s.keys, scores, N);
             __syncthreads();
@@ -644,19 +653,26 @@ cudaError_t launch_reindex_score(const IndexArgs &a, int BT, cudaStream_t st) {
     CSA2_DISPATCH_HI(64, launch_reindex_t, a, BT, st)
 }
 
-cudaError_t launch_select_full(const IndexArgs &a, int BT, cudaStream_t st) {
-    size_t smem = sizeof(SelSmem);
-    static bool attr_set = false;  // once per process (one device per process)
+template <int kCap>
+static cudaError_t launch_select_full_t(const IndexArgs &a, int BT, cudaStream_t st) {
+    size_t smem = sizeof(SelSmemT<kCap>);
+    static bool attr_set = false;  // once per process and instantiation (one device per process)
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(select_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(select_full_kernel<kCap>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        e = prefer_max_smem(select_full_kernel);
+        e = prefer_max_smem(select_full_kernel<kCap>);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    cudaError_t e = launch_pdl(select_full_kernel, dim3(BT), dim3(kSelThreads), smem, st, a);
+    cudaError_t e = launch_pdl(select_full_kernel<kCap>, dim3(BT), dim3(kSelThreads), smem, st, a);
     return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_select_full(const IndexArgs &a, int BT, cudaStream_t st) {
+    // flat rows longer than the default stage: the wide stage, if they fit
+    if (a.pool_blocks == 0 && a.n_max > kSelStageMax) return launch_select_full_t<kSelStageWide>(a, BT, st);
+    return launch_select_full_t<kSelStageMax>(a, BT, st);
 }
 
 cudaError_t launch_select_reindex(const IndexArgs &a, int BT, cudaStream_t st) {

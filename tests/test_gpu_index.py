@@ -80,10 +80,12 @@ def test_flat_ratio2_prefill_causal(harness):
     _check_request_index(dw, 0)
 
 
-def test_flat_unstaged_and_hierarchical_million_shape(harness):
-    """Encoder groups with N = 20000 (> 16384: selection streams keys from global
-    memory) next to a decoder group with N = 40000."""
-    wl = small_variant(WORKLOADS["decode_1m"], B=2, ctx=40000)
+@pytest.mark.parametrize("ctx", [40000, 110000])
+def test_flat_unstaged_and_hierarchical_million_shape(harness, ctx):
+    """Encoder groups (flat) with N = ctx / 2 next to a decoder group with N = ctx:
+    20000 keys (> 16384: the wide shared-memory stage) and 55000 keys (> 49152: the
+    selection streams its keys from global memory in every radix pass)."""
+    wl = small_variant(WORKLOADS["decode_1m"], B=2, ctx=ctx)
     dw = harness.DeviceWorkload(wl)
     dw.step()
     assert dw.stack.dev_err.item() == 0
