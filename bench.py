@@ -84,17 +84,18 @@ def attn_flops(wl) -> int:
     return wl.B * wl.Tq * 4 * wl.H * 512 * (wl.top_k + n_win)
 
 
-# DRAM bytes (read + write) per launch from one ncu capture of each of an op's kernels:
-# ([(bytes, batch of the captured launch), ...], kernel sources, code_hash of those
-# sources at capture time).  Reported, each kernel scaled to the batch, only while the
-# code is unchanged.  Captures: profiles/*.md.
+# DRAM bytes (read + write) per launch from one ncu capture of each of an op's kernels
+# in decode (one query token per request): ([(bytes, batch of the captured launch), ...],
+# kernel sources, code_hash of those sources at capture time).  Reported, each kernel
+# scaled to the batch, only for decode workloads and while the code is unchanged.
+# Captures: profiles/*.md.
 NCU_TRAFFIC = {
     "csa2_sparse_attn_decode": ([(21_211_392, 64)], ("csa2_attn.cu",), "f8a8dd610b4ba7ac"),
     "csa2_sparse_attn_decode_append": ([(21_211_392, 64)], ("csa2_attn.cu",), "f8a8dd610b4ba7ac"),
-    "csa2_index_full": ([(138_484_992 + 4_945_664, 8), (18_141_952, 64)], ("csa2_index.cu",),
-                        "33472cf35d49fbf2"),
-    "csa2_index_reindex": ([(18_606_080, 8), (4_754_432, 64)], ("csa2_index.cu",),
-                           "33472cf35d49fbf2"),
+    "csa2_index_full": ([(138_466_304 + 4_205_312, 8), (2_321_920, 8)], ("csa2_index.cu",),
+                        "c6711e4c46445f50"),
+    "csa2_index_reindex": ([(18_607_872, 8), (625_920, 8)], ("csa2_index.cu",),
+                           "c6711e4c46445f50"),
 }
 
 
@@ -159,7 +160,7 @@ def op_rooflines(wl, plan, op_ms: dict, ms_step: float) -> dict:
         traffic = None
         if name in NCU_TRAFFIC:
             caps, files, sha = NCU_TRAFFIC[name]
-            if _sources_hash(files) == sha:
+            if _sources_hash(files) == sha and wl.Tq == 1:
                 traffic = sum(tb * wl.B / tbatch for tb, tbatch in caps)
         e = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
              "frac": gbs / pk["hbm_gbs"], "traffic": traffic, "kernels": kernels,
