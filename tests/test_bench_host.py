@@ -126,3 +126,32 @@ def test_code_hash_ignores_comments_only():
     b = b"// a new header line\nint f(int x) {  // twice x\n\n    return 2 * x;\n}\n"
     c = b"int f(int x) {\n    return 3 * x;\n}\n"
     assert bench.code_hash(a) == bench.code_hash(b) != bench.code_hash(c)
+
+
+def test_prefill_and_rope_op_rooflines():
+    """The prefill chunk's tensor-core Full op: the index cache is read once per request
+    (not once per query token), its tensor flops are 2 * H_I * d per (query, visible
+    entry), and no decode traffic capture is scaled onto it.  The RoPE attention op adds
+    one (cos, sin) table row per query."""
+    from fp4_kv_compressed_b200.stack import plan_layers
+    from synth.workloads import ROPE_PAIRS
+    wl = WORKLOADS["prefill_chunk_enc"]
+    N, d, HI, Tq = wl.entries(0), wl.d_I, wl.H_I, wl.Tq
+    ob = bench.op_bytes(wl)
+    assert ob["index_full_g0"] == N * (d + 4) + Tq * (8 * N + 4 * wl.top_k + 4 + HI * d * 2 + HI * 4)
+    vis = sum((t + 1) // 2 for t in range(wl.ctx - Tq, wl.ctx))
+    assert bench.index_scan_flops(wl, 0) == vis * 2 * HI * d
+    plan = plan_layers([g.schedule for g in wl.groups])
+    ops = bench.op_rooflines(wl, plan, {"csa2_index_full_tc": 0.6, "csa2_sparse_attn_decode": 0.7},
+                             ms_step=4.7)
+    tc = ops["csa2_index_full_tc"]
+    assert tc["traffic"] is None and ops["csa2_sparse_attn_decode"]["traffic"] is None
+    assert abs(tc["tensor"]["achieved"] - vis * 2 * HI * d / 0.6e-3 / 1e12) < 1e-9
+    assert tc["bound"] == "hbm"          # the score round trip outweighs the MMAs
+    dec = WORKLOADS["decode_128k"]
+    plan = plan_layers([g.schedule for g in dec.groups])
+    r = bench.op_rooflines(dec, plan, {"csa2_sparse_attn_decode_append_rope": 0.033}, 1.12)
+    e = r["csa2_sparse_attn_decode_append_rope"]
+    assert e["algorithmic_bytes_per_launch"] == (bench.op_bytes(dec)["attn"] + 64 * (1024 + 516)
+                                                 + 64 * ROPE_PAIRS * 8)
+    assert e["launches_per_step"] == 19 and e["traffic"] is None
