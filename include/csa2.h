@@ -21,8 +21,9 @@
  *    default stream).  The returned status reports host-side validation
  *    (null pointers, sizes, capacities) and launch errors (CSA2_ERR_CUDA).
  *  - Bounds the host cannot see (device-resident positions, indices) are checked
- *    in the kernels: a violating row / index is skipped and a CSA2_DEVERR_* bit
- *    is OR-ed into `*dev_err` (an int32 in device memory, may be NULL).  Read it
+ *    in the kernels: a violating row / index is skipped (a row outside a RoPE
+ *    table is stored unrotated) and a CSA2_DEVERR_* bit is OR-ed into `*dev_err`
+ *    (an int32 in device memory, may be NULL).  Read it
  *    with csa2_read_device_error().  Kernels never trap; their internal waits
  *    are bounded (0.5 s of wall time) and report CSA2_DEVERR_TIMEOUT.
  *  - Kernels are launched with programmatic dependent launch: each may be
@@ -224,9 +225,9 @@ CSA2_API csa2_status csa2_index_full(const csa2_global_kv *kv, const void *q_idx
  * sum_h w_h * |q_h| . |k_s| and the Top-K can differ from csa2_index_full's
  * only between positions whose scores lie within that bound of each other.
  * Arguments, outputs, workspace and errors are those of csa2_index_full, plus:
- * q_idx_bf16 must be 16-byte aligned (else CSA2_ERR_INVALID_ARG).  One CTA
- * takes 128 / H_I query tokens of one request against up to 2048 entries; Tq
- * = 1 works but wastes the tile -- decode should call csa2_index_full.
+ * q_idx_bf16 must be 16-byte aligned (else CSA2_ERR_INVALID_ARG).  An MMA
+ * tile is 128 entries against 256 / H_I query tokens of one request, so Tq = 1
+ * works but wastes most of it: decode should call csa2_index_full.
  */
 CSA2_API csa2_status csa2_index_full_tc(const csa2_global_kv *kv, const void *q_idx_bf16,
                                         const float *w, const int32_t *q_pos, int32_t Tq,
