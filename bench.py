@@ -88,7 +88,6 @@ def attn_flops(wl) -> int:
 # in decode (one query token per request): ([(bytes, batch of the captured launch), ...],
 # kernel sources, code_hash of those sources at capture time).  Reported, each kernel
 # scaled to the batch, only for decode workloads and while the code is unchanged.
-# Captures: profiles/*.md.
 NCU_TRAFFIC = {
     "csa2_sparse_attn_decode": ([(21_211_392, 64)], ("csa2_attn.cu",), "f8a8dd610b4ba7ac"),
     "csa2_sparse_attn_decode_append": ([(21_211_392, 64)], ("csa2_attn.cu",), "f8a8dd610b4ba7ac"),
@@ -286,8 +285,7 @@ def oracle_sample_time(wl, requests: list[int], steps: int = 1) -> tuple[float, 
     Returns seconds per step for those requests and a description."""
     import torch
     import oracle as orc
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    import oracle_ref as R
+    from oracle import workload_ref as R
 
     prepared = []
     for b in requests:
@@ -542,22 +540,10 @@ def run_ours(args, rank, world, local_rank):
         "dtype": ("bf16 MMA index (fp32 accumulate)" if args.index_scan == "tc" else "fp32 index")
                  + " / bf16+fp16 MMA attention",
         "data": "synthetic",
-        "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.ctx, "heads": wl.H,
-                   "index_heads": wl.H_I, "d_idx": wl.d_I, "top_k": wl.top_k,
-                   "pool": [g.pool_blocks for g in wl.groups],
-                   "schedule": [g.schedule for g in wl.groups], "swa": wl.swa_len,
-                   "query_tokens": wl.Tq, "index_scan": args.index_scan,
-                   "rope": ({"start": csa2_harness.ROPE_START,
-                             "pairs": csa2_harness.ROPE_PAIRS,
-                             "rows": "main KV and SWA, rotated inside the append launches"}
-                            if args.rope else None),
-                   "parallelism": f"replicas x{world} (requests sharded, no collective)",
-                   "l2": "inputs larger than L2: the Full scan streams "
-                         f"{ob[f'index_full_g{g_full}'] / 1e9:.2f} GB per step",
-                   "cuda_graph": True, "step_algorithmic_bytes": sb,
-                   "step_gbps": sb / (ms_step / 1e3) / 1e9,
-                   "step_frac_of_8tbs": sb / (ms_step / 1e3) / 8e12,
-                   "token_layer_steps_per_s": value * wl.B},
+        "config": workload_config(wl, args, world),
+        "step": {"cuda_graph": True, "algorithmic_bytes": sb,
+                 "gbps": sb / (ms_step / 1e3) / 1e9, "frac_of_8tbs": sb / (ms_step / 1e3) / 8e12,
+                 "token_layer_steps_per_s": value * wl.B},
         "roofline": dict(ops[dominant], op=dominant),
         "roofline_ops": ops,
         "e2e": ({"value": job_value(world, layers, e2e_ms), "unit": UNIT,
@@ -567,6 +553,25 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks.summary(),
     }
     return line, wl
+
+
+def workload_config(wl, args, world: int) -> dict:
+    """The `config` of a bench line: the workload and how it is run (the same for
+    both arms)."""
+    from synth.workloads import ROPE_PAIRS, ROPE_START
+    ob = op_bytes(wl)
+    g_full = next(g for g, grp in enumerate(wl.groups) if "F" in grp.schedule)
+    return {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.ctx, "heads": wl.H,
+            "index_heads": wl.H_I, "d_idx": wl.d_I, "top_k": wl.top_k,
+            "pool": [g.pool_blocks for g in wl.groups],
+            "schedule": [g.schedule for g in wl.groups], "swa": wl.swa_len,
+            "query_tokens": wl.Tq, "index_scan": args.index_scan,
+            "rope": ({"start": ROPE_START, "pairs": ROPE_PAIRS,
+                      "rows": "main KV and SWA, rotated inside the append launches"}
+                     if args.rope else None),
+            "parallelism": f"replicas x{world} (requests sharded, no collective)",
+            "l2": "inputs larger than L2: the Full scan streams "
+                  f"{ob[f'index_full_g{g_full}'] / 1e9:.2f} GB per step"}
 
 
 def run_reference(args, rank, world):
@@ -584,10 +589,10 @@ def run_reference(args, rank, world):
     sample = (f"{len(req)} of {wl.B} requests per step, {K} timed steps of all {layers} layers "
               f"on the host; value scaled by {len(req)}/{wl.B} of a layer-step")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": K, "warmup": 1, "ms_per_step": dt * 1e3 * wl.B / len(req),
+            "steps": K, "warmup": 1, "ms_per_step": dt * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "fp32 index / fp64 attention", "data": "synthetic",
-            "config": {"workload": wl.name, "batch_per_gpu": wl.B, "context": wl.ctx},
+            "config": workload_config(wl, args, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": orc.num_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,

@@ -19,8 +19,13 @@ NVCC_FLAGS = [
     "--expt-relaxed-constexpr",
     # IEEE division / sqrt and preserved denormals: the quantisers and the score
     # order are defined in exact fp32 arithmetic.
-    "-prec-div=true", "-prec-sqrt=true", "-ftz=false", "-fmad=false",
+    "-prec-div=true", "-prec-sqrt=true", "-ftz=false",
 ]
+# The quantisers and the exact-order scan spell every rounding out with intrinsics
+# (__fdiv_rn, __fmaf_rn, fma.rn.f32x2, ...); no contraction of a plain a * b + c is
+# allowed in those two files either, as a guard.  The other kernels keep fmad.
+NO_FMAD = {"csa2_quant.cu", "csa2_index.cu"}
+BUILD_DIR = os.path.join(ROOT, "_build", "csa2")
 
 
 def sources() -> list[str]:
@@ -43,14 +48,29 @@ def nvcc() -> str:
     return "nvcc"
 
 
+def _compile(src: str, verbose: bool) -> str:
+    obj = os.path.join(BUILD_DIR, os.path.basename(src)[:-3] + ".o")
+    flags = list(NVCC_FLAGS)
+    if os.path.basename(src) in NO_FMAD:
+        flags.append("-fmad=false")
+    cmd = [nvcc(), *flags, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+    if verbose:
+        cmd.insert(1, "-Xptxas=-v")
+        print(" ".join(cmd), flush=True)
+    subprocess.run(cmd, check=True)
+    return obj
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not _stale():
         return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, "-shared", "-I", INCLUDE, "-I", CSRC, *sources(),
+    from concurrent.futures import ThreadPoolExecutor
+    os.makedirs(BUILD_DIR, exist_ok=True)
+    srcs = sources()
+    with ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
+        objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
+    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *objs,
            "-o", LIB + ".tmp"]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-        print(" ".join(cmd))
     subprocess.run(cmd, check=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB

@@ -871,14 +871,10 @@ size_t attn_tc_smem_bytes() { return sizeof(tc::Smem) + 1024; }
 template <bool kRope>
 static cudaError_t launch_attn_t(const AttnArgs &a, int BT, cudaStream_t st) {
     const size_t smem = attn_tc_smem_bytes();
-    static bool attr_set = false;  // once per process and instantiation (one device per process)
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel<kRope>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<uint64_t> configured{0};   // per device
+    {
+        cudaError_t e = config_kernel_once(tc::attn_tc_kernel<kRope>, smem, configured);
         if (e != cudaSuccess) return e;
-        e = prefer_max_smem(tc::attn_tc_kernel<kRope>);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     dim3 grid(2 * BT, (a.H + tc::kHeads - 1) / tc::kHeads);   // 2-CTA clusters
     cudaError_t e = launch_pdl(tc::attn_tc_kernel<kRope>, grid, dim3(tc::kThreads), smem, st, a);

@@ -599,14 +599,10 @@ select_reindex_kernel(IndexArgs a) {
 template <int D, int HI>
 static cudaError_t launch_scan_t(const IndexArgs &a, int grid_x, int BT, cudaStream_t st) {
     size_t smem = sizeof(ScoreSmem<D, HI, kScanRows>);
-    static bool attr_set = false;  // once per process and instantiation
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(index_scan_kernel<D, HI>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<uint64_t> configured{0};   // per device
+    {
+        cudaError_t e = config_kernel_once(index_scan_kernel<D, HI>, smem, configured);
         if (e != cudaSuccess) return e;
-        e = prefer_max_smem(index_scan_kernel<D, HI>);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     cudaError_t e = launch_pdl(index_scan_kernel<D, HI>, dim3(grid_x, BT), dim3(kScoreThreads), smem, st, a);
     return e != cudaSuccess ? e : cudaGetLastError();
@@ -615,14 +611,10 @@ static cudaError_t launch_scan_t(const IndexArgs &a, int grid_x, int BT, cudaStr
 template <int D, int HI>
 static cudaError_t launch_reindex_t(const IndexArgs &a, int BT, cudaStream_t st) {
     size_t smem = sizeof(ScoreSmem<D, HI, kReindexRows>);
-    static bool attr_set = false;  // once per process and instantiation
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(reindex_score_kernel<D, HI>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<uint64_t> configured{0};   // per device
+    {
+        cudaError_t e = config_kernel_once(reindex_score_kernel<D, HI>, smem, configured);
         if (e != cudaSuccess) return e;
-        e = prefer_max_smem(reindex_score_kernel<D, HI>);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     constexpr int kBlocksPerTile = kScoreThreads * kReindexRows / 8;
     int gx = (a.pool_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
@@ -656,14 +648,10 @@ cudaError_t launch_reindex_score(const IndexArgs &a, int BT, cudaStream_t st) {
 template <int kCap>
 static cudaError_t launch_select_full_t(const IndexArgs &a, int BT, cudaStream_t st) {
     size_t smem = sizeof(SelSmemT<kCap>);
-    static bool attr_set = false;  // once per process and instantiation (one device per process)
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(select_full_kernel<kCap>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<uint64_t> configured{0};   // per device
+    {
+        cudaError_t e = config_kernel_once(select_full_kernel<kCap>, smem, configured);
         if (e != cudaSuccess) return e;
-        e = prefer_max_smem(select_full_kernel<kCap>);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     cudaError_t e = launch_pdl(select_full_kernel<kCap>, dim3(BT), dim3(kSelThreads), smem, st, a);
     return e != cudaSuccess ? e : cudaGetLastError();
@@ -677,14 +665,10 @@ cudaError_t launch_select_full(const IndexArgs &a, int BT, cudaStream_t st) {
 
 cudaError_t launch_select_reindex(const IndexArgs &a, int BT, cudaStream_t st) {
     size_t smem = sizeof(SelSmem);
-    static bool attr_set = false;  // once per process (one device per process)
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(select_reindex_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+    static std::atomic<uint64_t> configured{0};   // per device
+    {
+        cudaError_t e = config_kernel_once(select_reindex_kernel, smem, configured);
         if (e != cudaSuccess) return e;
-        e = prefer_max_smem(select_reindex_kernel);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     cudaError_t e = launch_pdl(select_reindex_kernel, dim3(BT), dim3(kSelThreads), smem, st, a);
     return e != cudaSuccess ? e : cudaGetLastError();

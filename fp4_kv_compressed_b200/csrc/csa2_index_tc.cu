@@ -337,34 +337,19 @@ __global__ void __launch_bounds__(kThreads, 1) index_scan_tc_kernel(IndexArgs a,
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
-static int sm_count() {
-    static int n = 0;   // once per process (one device per process)
-    if (n == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-    }
-    return n;
-}
-
 template <int D, int HI>
 static cudaError_t launch_t(const IndexArgs &a, int B, cudaStream_t st) {
     const size_t smem = sizeof(Smem<D>) + 1024;
-    static bool attr_set = false;   // once per process and instantiation
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(index_scan_tc_kernel<D, HI>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<uint64_t> configured{0};   // per device
+    {
+        cudaError_t e = config_kernel_once(index_scan_tc_kernel<D, HI>, smem, configured);
         if (e != cudaSuccess) return e;
-        e = prefer_max_smem(index_scan_tc_kernel<D, HI>);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     const int n_tiles = (int)((a.n_max + kM - 1) / kM);
     const int n_qblk = (a.Tq + kN / HI - 1) / (kN / HI);
     const int64_t total = (int64_t)B * n_qblk * n_tiles;
     if (total == 0) return cudaSuccess;
-    const int grid = (int)(total < sm_count() ? total : sm_count());
+    const int grid = (int)(total < device_sm_count() ? total : device_sm_count());
     cudaError_t e = launch_pdl(index_scan_tc_kernel<D, HI>, dim3(grid), dim3(kThreads), smem, st, a,
                                B, n_qblk, n_tiles);
     return e != cudaSuccess ? e : cudaGetLastError();

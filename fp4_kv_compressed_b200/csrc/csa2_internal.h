@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace csa2 {
 
 // RoPE table of the _rope calls (cs == nullptr: no rotation); see csa2_rope.
@@ -94,6 +96,39 @@ template <class Kernel>
 inline cudaError_t prefer_max_smem(Kernel kernel) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                 (int)cudaSharedmemCarveoutMaxShared);
+}
+
+// Kernel attributes (dynamic shared-memory limit, carveout) belong to a device: a
+// launcher sets its kernel's attributes once on every device it launches on.
+// `done` holds one bit per device ordinal 0..63 (beyond that the attributes are set
+// on every launch).  Two host threads may both set them the first time; that is
+// harmless, the calls being idempotent.
+template <class Kernel>
+inline cudaError_t config_kernel_once(Kernel kernel, size_t dyn_smem, std::atomic<uint64_t> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t)1 << dev : 0;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    if (dyn_smem > 0) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn_smem);
+        if (e != cudaSuccess) return e;
+    }
+    e = prefer_max_smem(kernel);
+    if (e != cudaSuccess) return e;
+    done.fetch_or(bit, std::memory_order_acq_rel);
+    return cudaSuccess;
+}
+
+// Number of SMs of the current device (148 on B200 if the query fails).
+inline int device_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        (void)cudaGetLastError();
+        n = 148;
+    }
+    return n;
 }
 
 // Launch with programmatic stream serialisation (see grid_dep_wait / grid_dep_launch).

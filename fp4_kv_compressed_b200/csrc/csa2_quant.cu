@@ -103,11 +103,10 @@ cudaError_t launch_quantize_append(const QuantArgs &a, cudaStream_t st) {
     int64_t warps = a.n_main + a.n_idx + a.n_swa;
     if (warps == 0) return cudaSuccess;
     int64_t blocks = (warps * 32 + 255) / 256;
-    static bool attr_set = false;  // once per process (one device per process)
-    if (!attr_set) {
-        cudaError_t e = prefer_max_smem(quantize_append_kernel);
+    static std::atomic<uint64_t> configured{0};   // per device
+    {
+        cudaError_t e = config_kernel_once(quantize_append_kernel, 0, configured);
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     cudaError_t e = launch_pdl(quantize_append_kernel, dim3((unsigned)blocks), dim3(256), 0, st, a);
     return e != cudaSuccess ? e : cudaGetLastError();

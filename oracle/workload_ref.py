@@ -1,5 +1,8 @@
 """Oracle-side reference of one request of a workload (host only).
 
+TEST INFRASTRUCTURE, like the rest of this package: only the tests, the smoke
+check and the benchmark's CPU baseline leg / reference arm use it.
+
 Regenerates the request's bf16 inputs with the seeded generator and runs the
 CPU oracle on them: caches, every selector layer's pool / Top-K, and the
 attention of the requested layers.  Imports nothing of the CUDA path.
@@ -120,3 +123,16 @@ def rel_err_rows(o: np.ndarray, ref: np.ndarray) -> np.ndarray:
     den = np.abs(ref).max(-1)
     num = np.abs(o - ref).max(-1)
     return np.where(den > 0, num / np.where(den > 0, den, 1), num)
+
+
+def rel_err_elems(o: np.ndarray, ref: np.ndarray) -> float:
+    """Largest elementwise relative error |o - ref| / |ref| over the elements whose
+    |ref| is at least the RMS of their row (the companion figure of the norm-wise
+    error; rows = leading dims).  0.0 when no element qualifies."""
+    o = o.reshape(-1, o.shape[-1]).astype(np.float64)
+    ref = ref.reshape(-1, ref.shape[-1]).astype(np.float64)
+    rms = np.sqrt((ref * ref).mean(-1, keepdims=True))
+    big = (np.abs(ref) >= rms) & (rms > 0)
+    if not big.any():
+        return 0.0
+    return float((np.abs(o - ref)[big] / np.abs(ref)[big]).max())

@@ -4,7 +4,7 @@ import numpy as np
 import pytest
 import torch
 
-import oracle_ref as R
+from oracle import workload_ref as R
 from synth.workloads import WORKLOADS, small_variant
 
 pytestmark = pytest.mark.gpu

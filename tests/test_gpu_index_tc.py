@@ -175,7 +175,7 @@ def test_tc_stack_prefill_chunk(pkg, orc):
     position is left out only for one within the error bound of it), and every layer's
     attention over the kernel's own selection matches the oracle."""
     import csa2_harness
-    import oracle_ref as R
+    from oracle import workload_ref as R
     from synth.workloads import WORKLOADS, small_variant
     wl = small_variant(WORKLOADS["prefill_chunk_enc"], B=1, ctx=3000 + 64, Tq=64)
     dw = csa2_harness.DeviceWorkload(wl, index_scan="tc")
