@@ -24,6 +24,7 @@ STATUS = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_CAPACITY",
           6: "CSA2_ERR_DEVICE_BOUNDS"}
 
 DEVERR_SLOT, DEVERR_INDEX, DEVERR_NMAX, DEVERR_RANGE, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
+DEFAULT_WAIT_LIMIT_NS = 500_000_000
 DEVERR_ROPE = 0x20
 
 # every symbol declared in include/csa2.h
@@ -31,7 +32,7 @@ EXPORTS = ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_workspace_
            "csa2_index_full", "csa2_index_full_tc", "csa2_index_full_noalloc",
            "csa2_index_reindex", "csa2_sparse_attn_decode", "csa2_sparse_attn_decode_append",
            "csa2_sparse_attn_decode_append_rope", "csa2_read_device_error",
-           "csa2_status_string", "csa2_abi_version")
+           "csa2_status_string", "csa2_abi_version", "csa2_debug_set_waits")
 
 
 class Csa2Error(RuntimeError):
@@ -98,6 +99,8 @@ def load_library(path: str = LIB_PATH):
     L.csa2_status_string.argtypes = [C.c_int]
     L.csa2_status_string.restype = C.c_char_p
     L.csa2_abi_version.restype = i32
+    L.csa2_debug_set_waits.argtypes = [C.c_uint64, i32]
+    L.csa2_debug_set_waits.restype = None
     for fn in ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_index_full",
                "csa2_index_full_tc", "csa2_index_reindex", "csa2_sparse_attn_decode",
                "csa2_sparse_attn_decode_append", "csa2_sparse_attn_decode_append_rope",
@@ -213,6 +216,11 @@ def csa2_sparse_attn_decode_append(kv: CSA2GlobalKV, swa: CSA2SWA, swa_bf16, q, 
                                           top_k, swa_len, softmax_scale, _ptr(out), _ptr(lse),
                                           _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream))
     _check("csa2_sparse_attn_decode_append", st)
+
+
+def csa2_debug_set_waits(limit_ns: int, stuck_wait: bool) -> None:
+    """Test hook of the kernels' bounded waits (see include/csa2.h)."""
+    load_library().csa2_debug_set_waits(int(limit_ns), 1 if stuck_wait else 0)
 
 
 def csa2_read_device_error(dev_err, stream=None) -> int:

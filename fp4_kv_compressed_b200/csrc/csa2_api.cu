@@ -3,10 +3,27 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "csa2.h"
 #include "csa2_internal.h"
 
 using namespace csa2;
+
+namespace csa2 {
+
+// The process-wide wait settings of csa2_debug_set_waits.
+static std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
+static std::atomic<int32_t> g_stuck_wait{0};
+
+WaitCfg current_wait_cfg() {
+    WaitCfg w;
+    w.limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+    w.stuck = g_stuck_wait.load(std::memory_order_relaxed);
+    return w;
+}
+
+}  // namespace csa2
 
 namespace {
 
@@ -65,7 +82,12 @@ bool hi_supported(int32_t H_I) {
 
 extern "C" {
 
-int32_t csa2_abi_version(void) { return 101; }
+int32_t csa2_abi_version(void) { return 102; }
+
+void csa2_debug_set_waits(uint64_t limit_ns, int32_t stuck_wait) {
+    g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+    g_stuck_wait.store(stuck_wait ? 1 : 0, std::memory_order_relaxed);
+}
 
 const char *csa2_status_string(csa2_status st) {
     switch (st) {
@@ -228,6 +250,7 @@ static csa2_status index_full(const csa2_global_kv *kv, const void *q_idx_bf16, 
     a.topk_out = topk_out;
     a.topk_count = topk_count;
     a.dev_err = dev_err;
+    a.wait = current_wait_cfg();
     cudaStream_t s = (cudaStream_t)stream;
     st = launched(tc ? launch_index_scan_tc(a, (int)kv->batch, s) : launch_index_scan(a, (int)BT, s));
     if (st != CSA2_OK) return st;
@@ -290,6 +313,7 @@ csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16,
     a.topk_out = topk_out;
     a.topk_count = topk_count;
     a.dev_err = dev_err;
+    a.wait = current_wait_cfg();
     cudaStream_t s = (cudaStream_t)stream;
     st = launched(launch_reindex_score(a, (int)BT, s));
     if (st != CSA2_OK) return st;
@@ -344,6 +368,7 @@ static csa2_status sparse_attn(const csa2_global_kv *kv, const csa2_swa *swa, co
     a.out = out;
     a.lse = lse;
     a.dev_err = dev_err;
+    a.wait = current_wait_cfg();
     return launched(launch_sparse_attn(a, (int)BT, (cudaStream_t)stream));
 }
 

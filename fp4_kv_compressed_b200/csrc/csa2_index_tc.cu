@@ -24,7 +24,9 @@
 // the sum over a token's heads stay in registers, then sigma and the causal mask;
 // a warp stores 32 consecutive entries of a token (128 bytes).  Scores and
 // 8-position block maxima go to the same workspace as the exact scan, whose
-// selection kernel then runs unchanged.  Every wait is bounded (0.5 s).
+// selection kernel then runs unchanged.  Every wait is bounded (WaitCfg); a CTA whose
+// wait runs out flags CSA2_DEVERR_TIMEOUT, waits for the MMAs it has issued, frees its
+// TMEM and returns.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -39,7 +41,6 @@ constexpr int kThreads = 512;
 constexpr int kM = 128;                  // entries per tile (MMA M, TMEM lanes)
 constexpr int kN = 256;                  // query tokens x index heads (MMA N)
 constexpr uint32_t kTmemCols = 512;      // two 256-column fp32 accumulators
-constexpr uint64_t kWaitLimitNs = 500000000ull;
 
 template <int D>
 struct __align__(1024) Smem {
@@ -48,6 +49,8 @@ struct __align__(1024) Smem {
     alignas(16) float w[kN];             // w of each column (token, head)
     int32_t nvis[kN];                    // visible entries of each token of the block (-1: none)
     uint64_t mma_done[2];
+    uint64_t drain;                      // abort path: completes once every issued MMA has
+    uint64_t never;                      // test hook (WaitCfg::stuck): never signalled
     uint32_t tmem_base;
 };
 
@@ -59,7 +62,7 @@ __device__ __forceinline__ uint64_t wall_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, uint64_t limit_ns) {
     const uint32_t addr = smem_u32(b);
     const uint64_t t0 = wall_ns();
     while (true) {
@@ -72,7 +75,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity) {
             : "r"(addr), "r"(parity)
             : "memory");
         if (done) return true;
-        if (wall_ns() - t0 > kWaitLimitNs) return false;
+        if (wall_ns() - t0 > limit_ns) return false;
     }
 }
 // 128-byte-swizzled K-major operand descriptor (SBO = 8 rows x 128 B).
@@ -153,6 +156,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_scan_tc_kernel(IndexArgs a,
     const int my_ent = 32 * (warp & 3) + lane;   // this thread's entry (TMEM lane) in a tile
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&s.mma_done[i])));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&s.drain)));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&s.never)));
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -177,11 +182,15 @@ __global__ void __launch_bounds__(kThreads, 1) index_scan_tc_kernel(IndexArgs a,
     int64_t pend_e0 = 0;
     float pend_sig = 0.0f;
     bool ok = true;
+    bool stuck = a.wait.stuck != 0;      // test hook: the first wait never completes
 
     // epilogue of the pending tile: scores of entries pend_e0 + my_ent for every token
     auto epilogue = [&]() {
         const uint32_t buf = (uint32_t)pend & 1u;
-        ok = __syncthreads_and(ok && mbar_wait(&s.mma_done[buf], ((uint32_t)pend >> 1) & 1u)) != 0;
+        ok = __syncthreads_and(ok && (stuck ? mbar_wait(&s.never, 0, a.wait.limit_ns)
+                                            : mbar_wait(&s.mma_done[buf], ((uint32_t)pend >> 1) & 1u,
+                                                        a.wait.limit_ns))) != 0;
+        stuck = false;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         if (!ok) return;
         const int64_t ent = pend_e0 + my_ent;
@@ -329,8 +338,19 @@ __global__ void __launch_bounds__(kThreads, 1) index_scan_tc_kernel(IndexArgs a,
         pend_e0 = e0;
         pend_sig = sig;
     }
-    if (!ok && threadIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+    if (!ok) {
+        // a wait ran out: the MMAs issued so far may still be running.  The issuing
+        // thread commits once more; that arrival comes after all of them.
+        if (threadIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+        if (warp == 0) {
+            if (elect_one()) mma_commit(&s.drain);
+            __syncwarp();
+        }
+        const bool drained = mbar_wait(&s.drain, 0, kDrainLimitNs);
+        (void)drained;
+    }
     grid_dep_launch();
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (warp == 0)

@@ -8,6 +8,20 @@
 
 namespace csa2 {
 
+// Bounded waits.  Every spin of a kernel on an mbarrier gives up after `limit_ns` of
+// wall time (%globaltimer); the kernel then flags CSA2_DEVERR_TIMEOUT, waits (bounded
+// by kDrainLimitNs) for the tensor-core work and copies it has in flight, frees its
+// TMEM and returns.  `stuck` is a test hook: with it set, the instrumented kernels'
+// first wait of every CTA is on a barrier that nothing ever signals, so that wait
+// always runs out.  Both come from csa2_debug_set_waits (defaults 0.5 s, off).
+struct WaitCfg {
+    uint64_t limit_ns;
+    int32_t stuck;
+};
+constexpr uint64_t kDefaultWaitLimitNs = 500000000ull;
+constexpr uint64_t kDrainLimitNs = 500000000ull;
+WaitCfg current_wait_cfg();
+
 // RoPE table of the _rope calls (cs == nullptr: no rotation); see csa2_rope.
 struct RopeArgs {
     const float2 *cs;        // [n_pos][pairs] (cos, sin)
@@ -65,6 +79,7 @@ struct IndexArgs {
     int32_t *topk_out;
     int32_t *topk_count;
     int32_t *dev_err;
+    WaitCfg wait;
 };
 
 struct AttnArgs {
@@ -88,6 +103,7 @@ struct AttnArgs {
     float *out;
     float *lse;
     int32_t *dev_err;
+    WaitCfg wait;
 };
 
 // Every kernel of the library asks for the largest shared-memory carveout, so that

@@ -15,8 +15,9 @@
  *
  * Conventions (all entry points):
  *  - Every pointer is DEVICE memory owned by the caller unless stated otherwise.
- *    The library allocates nothing, keeps no state between calls and is
- *    re-entrant; calls on one stream execute in order.
+ *    The library allocates nothing, keeps no state between calls (apart from
+ *    the csa2_debug_set_waits test setting) and is re-entrant; calls on one
+ *    stream execute in order.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *    default stream).  The returned status reports host-side validation
  *    (null pointers, sizes, capacities) and launch errors (CSA2_ERR_CUDA).
@@ -67,7 +68,8 @@ typedef enum csa2_status {
 #define CSA2_DEVERR_INDEX 0x2     /* a Top-K or pool id outside the visible range */
 #define CSA2_DEVERR_NMAX 0x4      /* a query sees more entries than n_max */
 #define CSA2_DEVERR_RANGE 0x8     /* a dequantised SWA value beyond the fp16 range */
-#define CSA2_DEVERR_TIMEOUT 0x10  /* a kernel's bounded wait gave up (internal error) */
+#define CSA2_DEVERR_TIMEOUT 0x10  /* a kernel's bounded wait gave up (internal error, or
+                                     the csa2_debug_set_waits test hook) */
 #define CSA2_DEVERR_ROPE 0x20     /* a row's position lies outside the RoPE table */
 
 /* Limits of the kernels. */
@@ -338,6 +340,21 @@ CSA2_API const char *csa2_status_string(csa2_status status);
 
 /* ABI version: 100 * major + minor. */
 CSA2_API int32_t csa2_abi_version(void);
+
+/*
+ * Test hook for the kernels' bounded waits; the pages have no counterpart (it is
+ * not part of the method).  Every spin of a kernel on an mbarrier gives up after
+ * limit_ns of wall time: the kernel then sets CSA2_DEVERR_TIMEOUT in *dev_err,
+ * waits (bounded) for its own tensor-core work and copies in flight, frees its
+ * tensor memory and returns, so that the CUDA context stays usable.
+ * stuck_wait != 0 makes the first wait of every CTA of the tensor-core kernels
+ * (the scan of csa2_index_full_tc and the sparse attention) wait on a barrier that
+ * nothing signals, so that it always runs out: a test can drive the timeout path
+ * without faulting or hanging a GPU.  The setting is process-wide and read by each
+ * call when it launches; defaults: limit_ns = 500000000 (0.5 s), stuck_wait = 0.
+ * Results of calls made with stuck_wait set are undefined (only the error bit is).
+ */
+CSA2_API void csa2_debug_set_waits(uint64_t limit_ns, int32_t stuck_wait);
 
 #ifdef __cplusplus
 }

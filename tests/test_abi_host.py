@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol(pkg):
     assert set(names) == set(pkg.EXPORTS)
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.csa2_abi_version() == 101      # 1.1: the _rope calls and the tensor-core scan
+    assert lib.csa2_abi_version() == 102      # 1.2: csa2_debug_set_waits
     for st in range(7):
         assert lib.csa2_status_string(st)
 
