@@ -54,7 +54,9 @@ def op_bytes(wl) -> dict:
             per = (N * (d + 4) + 4 * N + 4 * nb + 4 * nb + 8 * min(P, nb) * 4 + 4 * P + 4 * K + 4
                    + q)
             out[f"index_full_g{g}"] = BT * per
-            rp = 4 * P + 8 * P * (d + 4) + 8 * P * 4 * 2 + 4 * K + 4 + q
+            # the pool, its entries' index K and scales, the Top-K out (the scores stay
+            # on chip)
+            rp = 4 * P + 8 * P * (d + 4) + 4 * K + 4 + q
             out[f"index_reindex_g{g}"] = BT * rp
         else:
             out[f"index_full_g{g}"] = BT * (N * (d + 4) + 4 * N + 4 * N + 4 * K + 4 + q)
@@ -89,12 +91,11 @@ def attn_flops(wl) -> int:
 # kernel sources, code_hash of those sources at capture time).  Reported, each kernel
 # scaled to the batch, only for decode workloads and while the code is unchanged.
 NCU_TRAFFIC = {
-    "csa2_sparse_attn_decode": ([(21_211_392, 64)], ("csa2_attn.cu",), "f8a8dd610b4ba7ac"),
-    "csa2_sparse_attn_decode_append": ([(21_211_392, 64)], ("csa2_attn.cu",), "f8a8dd610b4ba7ac"),
+    "csa2_sparse_attn_decode": ([], ("csa2_attn.cu",), ""),
+    "csa2_sparse_attn_decode_append": ([], ("csa2_attn.cu",), ""),
     "csa2_index_full": ([(138_466_304 + 4_205_312, 8), (2_321_920, 8)], ("csa2_index.cu",),
                         "c6711e4c46445f50"),
-    "csa2_index_reindex": ([(18_607_872, 8), (625_920, 8)], ("csa2_index.cu",),
-                           "c6711e4c46445f50"),
+    "csa2_index_reindex": ([], ("csa2_index.cu",), ""),
 }
 
 
@@ -138,7 +139,7 @@ def op_rooflines(wl, plan, op_ms: dict, ms_step: float) -> dict:
             "csa2_index_full_tc": (ob[f"index_full_g{dec}"], modes.count("F"),
                                    "index_scan_tc_kernel + select_full_kernel"),
             "csa2_index_reindex": (ob.get(f"index_reindex_g{dec}", 0), modes.count("X"),
-                                   "reindex_score_kernel + select_reindex_kernel"),
+                                   "reindex_fused_kernel"),
             "csa2_sparse_attn_decode": (ob["attn"], len(modes), "attn_tc_kernel"),
             # decode: every layer but a group's first appends its SWA row inside the
             # attention launch

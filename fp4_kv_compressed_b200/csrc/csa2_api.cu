@@ -50,10 +50,6 @@ FullLayout full_layout(int64_t BT, int64_t n_max, int32_t pool_blocks) {
     return L;
 }
 
-size_t reindex_ws(int64_t BT, int32_t pool_blocks) {
-    return align_up((size_t)BT * pool_blocks * 8 * sizeof(float), kAlign);
-}
-
 csa2_status check_kv(const csa2_global_kv *kv, bool need_index) {
     if (!kv || !kv->codes || !kv->scales) return CSA2_ERR_INVALID_ARG;
     if (kv->batch <= 0 || kv->cap <= 0 || kv->ratio < 1 || kv->ratio > 64) return CSA2_ERR_INVALID_ARG;
@@ -112,7 +108,7 @@ size_t csa2_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t n_max, int
         case CSA2_OP_INDEX_FULL:
             return n_max > 0 ? full_layout(BT, n_max, pool_blocks).total : 0;
         case CSA2_OP_INDEX_REINDEX:
-            return pool_blocks > 0 ? reindex_ws(BT, pool_blocks) : 0;
+            return 0;   // the scores stay in shared memory
         case CSA2_OP_SPARSE_ATTN:
             return 0;
         default:
@@ -290,8 +286,8 @@ csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16,
     if (pool_blocks < 1 || pool_blocks > CSA2_POOL_MAX) return CSA2_ERR_UNSUPPORTED;
     const int64_t BT = (int64_t)kv->batch * Tq;
     if (BT > 65535) return CSA2_ERR_UNSUPPORTED;   // grid.y limit
-    if (!workspace || ws_bytes < reindex_ws(BT, pool_blocks) || !aligned(workspace, kAlign))
-        return CSA2_ERR_WORKSPACE;
+    (void)workspace;
+    (void)ws_bytes;
 
     IndexArgs a;
     memset(&a, 0, sizeof(a));
@@ -305,8 +301,6 @@ csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16,
     a.q_pos = q_pos;
     a.Tq = Tq;
     a.H_I = H_I;
-    a.scores = (float *)workspace;
-    a.score_stride = (int64_t)pool_blocks * 8;
     a.pool = pool;
     a.pool_blocks = pool_blocks;
     a.top_k = top_k;
@@ -315,9 +309,7 @@ csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16,
     a.dev_err = dev_err;
     a.wait = current_wait_cfg();
     cudaStream_t s = (cudaStream_t)stream;
-    st = launched(launch_reindex_score(a, (int)BT, s));
-    if (st != CSA2_OK) return st;
-    return launched(launch_select_reindex(a, (int)BT, s));
+    return launched(launch_reindex_fused(a, (int)BT, s));
 }
 
 static csa2_status sparse_attn(const csa2_global_kv *kv, const csa2_swa *swa, const void *swa_new_bf16,

@@ -269,8 +269,11 @@ CSA2_API csa2_status csa2_index_full_noalloc(const csa2_global_kv *kv, const voi
  * a6 Reindex layer: the same score with this layer's own q_idx / w, over the
  * visible positions of the pool's blocks only, then Top-K (same order, same
  * output form).  pool [B][Tq][pool_blocks] as written by csa2_index_full
- * (-1 = unused slot).  Workspace: csa2_workspace_size(CSA2_OP_INDEX_REINDEX,
- * B, Tq, 0, 0, top_k, pool_blocks).
+ * (-1 = unused slot; the used slots ascending).  One launch: a cluster of CTAs
+ * per query scores its share of the pool into shared memory, selects a local
+ * Top-K, and the cluster merges the local lists.  No workspace is needed:
+ * csa2_workspace_size(CSA2_OP_INDEX_REINDEX, ...) is 0 and `workspace` may be
+ * NULL (it is ignored).
  */
 CSA2_API csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
                                const int32_t *q_pos, int32_t Tq, int32_t H_I,

@@ -39,7 +39,7 @@ def test_workspace_sizes(pkg):
     assert full >= 64 * 131072 * 4 + 64 * 16384 * 4 and full % 256 == 0
     flat = ws(pkg.CSA2_OP_INDEX_FULL, 64, 1, 131072, 64, 512, 0)
     assert flat >= 64 * 131072 * 4 and flat < full
-    assert ws(pkg.CSA2_OP_INDEX_REINDEX, 64, 1, 0, 64, 512, 2048) >= 64 * 16384 * 4
+    assert ws(pkg.CSA2_OP_INDEX_REINDEX, 64, 1, 0, 64, 512, 2048) == 0   # scores on chip
     assert ws(pkg.CSA2_OP_SPARSE_ATTN, 64, 1, 0, 64, 512, 0) == 0
     assert ws(99, 1, 1, 1, 1, 1, 1) == 0
 

@@ -71,7 +71,11 @@ def test_algorithmic_bytes_at_128k():
     assert ob["index_full_g0"] == B * per_q == 1_154_155_776
     attn = 512 * 288 + 512 * 4 + 128 * 516 + 64 * 512 * 2 + 64 * 512 * 4 + 64 * 4
     assert ob["attn"] == B * attn
-    assert bench.step_bytes(wl) == 2_274_219_520
+    # Reindex: the pool, 8 entries of index K (128 B codes + 4 B scale) per pool block,
+    # the Top-K out; the scores stay on chip
+    rx = 4 * 2048 + 8 * 2048 * 132 + 4 * 512 + 4 + 4 * 128 * 2 + 4 * 4
+    assert ob["index_reindex_g0"] == B * rx == 139_134_208
+    assert bench.step_bytes(wl) == 2_240_665_088
 
 
 def test_reference_arm_line():
