@@ -33,20 +33,28 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
-// Workspace layout of csa2_index_full: scores [BT][score_stride] fp32, then
-// (hierarchical only) block maxima [BT][bmax_stride] fp32.
+// Workspace layout of csa2_index_full: scores [BT][score_stride] fp32, then block
+// maxima of 8 positions [BT][bmax_stride] (hierarchical rows, and flat rows longer than
+// kFlatDirect), then maxima of 64 positions [BT][bmax64_stride] (rows longer than
+// kFlatDirect).  The selection of a long row goes through the block maxima.
+constexpr int64_t kFlatDirect = 16384;
+
 struct FullLayout {
-    int64_t score_stride, bmax_stride;
-    size_t bmax_off, total;
+    int64_t score_stride, bmax_stride, bmax64_stride;
+    size_t bmax_off, bmax64_off, total;
+    bool bmax, bmax64;
 };
 
 FullLayout full_layout(int64_t BT, int64_t n_max, int32_t pool_blocks) {
     FullLayout L;
     L.score_stride = (int64_t)align_up((size_t)(n_max > 0 ? n_max : 1), 64);
     L.bmax_stride = (int64_t)align_up((size_t)((n_max + 7) / 8 > 0 ? (n_max + 7) / 8 : 1), 64);
+    L.bmax64_stride = (int64_t)align_up((size_t)((n_max + 63) / 64 > 0 ? (n_max + 63) / 64 : 1), 64);
+    L.bmax = pool_blocks > 0 || n_max > kFlatDirect;
+    L.bmax64 = n_max > kFlatDirect;
     L.bmax_off = align_up((size_t)BT * L.score_stride * sizeof(float), kAlign);
-    L.total = L.bmax_off;
-    if (pool_blocks > 0) L.total += align_up((size_t)BT * L.bmax_stride * sizeof(float), kAlign);
+    L.bmax64_off = L.bmax_off + (L.bmax ? align_up((size_t)BT * L.bmax_stride * sizeof(float), kAlign) : 0);
+    L.total = L.bmax64_off + (L.bmax64 ? align_up((size_t)BT * L.bmax64_stride * sizeof(float), kAlign) : 0);
     return L;
 }
 
@@ -238,8 +246,12 @@ static csa2_status index_full(const csa2_global_kv *kv, const void *q_idx_bf16, 
     a.n_max = n_max;
     a.scores = (float *)workspace;
     a.score_stride = L.score_stride;
-    a.bmax = pool_blocks > 0 && workspace ? (float *)((uint8_t *)workspace + L.bmax_off) : nullptr;
+    // the tensor-core scan writes 8-position maxima for the pool only; the exact scan
+    // writes both kinds whenever the layout has them
+    a.bmax = workspace && (tc ? pool_blocks > 0 : L.bmax) ? (float *)((uint8_t *)workspace + L.bmax_off) : nullptr;
     a.bmax_stride = L.bmax_stride;
+    a.bmax64 = workspace && !tc && L.bmax64 ? (float *)((uint8_t *)workspace + L.bmax64_off) : nullptr;
+    a.bmax64_stride = L.bmax64_stride;
     a.pool_blocks = pool_blocks;
     a.pool_out = pool_out;
     a.top_k = top_k;

@@ -45,6 +45,7 @@ struct ScoreSmem {
     uint8_t rows[kScoreThreads * R * D];
     float2 q[D / 2][HI];     // q pairs (q[h][2j], q[h][2j+1]) as fp32
     float w[HI];
+    float m64[kScoreThreads / 32][R];   // per warp and row group: max of its 32 rows
 };
 
 // Stage q (bf16 [HI][D]) and w into shared memory as fp32.
@@ -203,7 +204,19 @@ index_scan_kernel(IndexArgs a) {
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
             if ((row & 7) == 0 && row < rows) a.bmax[(int64_t)qi * a.bmax_stride + p / 8] = m;
+            if (a.bmax64) {
+                // super-block of 64 positions = rows 64 r .. 64 r + 63 = both warps' r-th rows
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 8));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
+                if ((threadIdx.x & 31) == 0) s.m64[threadIdx.x >> 5][r] = m;
+            }
         }
+    }
+    if (a.bmax64) {
+        __syncthreads();
+        if (threadIdx.x < R && 64 * (int)threadIdx.x < rows)
+            a.bmax64[(int64_t)qi * a.bmax64_stride + p0 / 64 + threadIdx.x] =
+                fmaxf(s.m64[0][threadIdx.x], s.m64[1][threadIdx.x]);
     }
 }
 
@@ -227,6 +240,8 @@ constexpr int kSelStageMax = 16384;   // keys staged in shared memory up to this
 // reads its row from HBM once instead of once per radix pass.
 constexpr int kSelStageWide = 49152;
 constexpr int kSelDigit = 11;         // bits per radix pass
+// Flat rows longer than this select through the 64- and 8-position block maxima.
+constexpr int kSelFlatDirect = 16384;
 
 template <int kCap>
 struct SelSmemT {
@@ -235,6 +250,7 @@ struct SelSmemT {
     uint32_t wmin[kSelWarps], wmax[kSelWarps];
     int bcast[4];
     alignas(16) int pool[CSA2_POOL_MAX];
+    int sup[CSA2_POOL_MAX];               // multi-level selection: the chosen super-blocks
     alignas(16) uint32_t keys[kCap];
 };
 using SelSmem = SelSmemT<kSelStageMax>;
@@ -431,58 +447,124 @@ __device__ int block_topk(KeyAt key_at, IdAt id_at, int n, int k, int *out, S &s
     return min(total, kk);
 }
 
-// a4 + a5: one CTA per query.  Hierarchical: pool from block maxima, then Top-K
-// inside the pool's positions (equal to Top-K over all positions because every
-// pool block's best position outranks any position outside the pool, and
-// pool_blocks >= top_k).  Flat: Top-K over all visible positions.
+// keys[8 i + j] = order key of src[8 ids[i] + j] (i < n, j < 8), 0 for the entries at or
+// past `limit`.  src rows are 32-byte aligned and long enough for whole groups of 8.
+__device__ __forceinline__ void gather8_keys(uint32_t *keys, const float *src, const int *ids, int n,
+                                             int64_t limit) {
+    for (int c = threadIdx.x; c < 2 * n; c += kSelThreads)
+        cp_async16(keys + 4 * c, src + (int64_t)ids[c >> 1] * 8 + 4 * (c & 1));
+    cp_async_commit();
+    cp_async_wait_all();
+    __syncthreads();
+    for (int i = threadIdx.x; i < 8 * n; i += kSelThreads) {
+        const int64_t p = (int64_t)ids[i >> 3] * 8 + (i & 7);
+        keys[i] = p < limit ? score_key(__uint_as_float(keys[i])) : 0u;
+    }
+    __syncthreads();
+}
+
+// a4 + a5: one CTA per query.
+// Lemma (the pages' pool argument, for any k and any partition into contiguous groups):
+// the k best items by (value desc, index asc) all lie in the k best groups by (group max
+// desc, group asc) -- an item of another group is preceded by the maxima of k groups,
+// each of which precedes it.  So:
+//   Hierarchical: pool = the pool_blocks best 8-position blocks (from the 64-position
+//     super-blocks first when there are more blocks than the stage holds); Top-K = the
+//     top_k best positions of the top_k best pool blocks (top_k <= pool_blocks).
+//   Flat: Top-K over all visible positions; for long rows from the top_k best
+//     super-blocks, then their top_k best blocks, then those blocks' positions.
+// Outputs ascending.
 template <int kCap>
 __global__ void __launch_bounds__(kSelThreads)
 select_full_kernel(IndexArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     SelSmemT<kCap> &s = *reinterpret_cast<SelSmemT<kCap> *>(smem_raw);
     __shared__ int sel_out[CSA2_TOPK_MAX];
+    __shared__ int sub[CSA2_TOPK_MAX];
     grid_dep_wait();
     const int qi = blockIdx.x;
     int64_t N64 = visible_entries(a.q_pos[qi], a.ratio);
     N64 = min64(min64(N64, a.n_max), a.cap);
     const int N = (int)N64;
+    const int nb = (N + 7) / 8, nb64 = (N + 63) / 64;
     const float *scores = a.scores + (int64_t)qi * a.score_stride;
+    const float *bm = a.bmax ? a.bmax + (int64_t)qi * a.bmax_stride : nullptr;
+    const float *bm64 = a.bmax64 ? a.bmax64 + (int64_t)qi * a.bmax64_stride : nullptr;
+    // the top_k best 8-blocks among the candidate blocks ids[0..n) (ascending), into
+    // sub[]; keys from bm
+    auto best_blocks = [&](const int *ids, int n) -> int {
+        for (int i = threadIdx.x; i < n; i += kSelThreads) s.keys[i] = score_key(__ldg(bm + ids[i]));
+        __syncthreads();
+        auto k = [&](int i) -> uint32_t { return s.keys[i]; };
+        auto id = [&](int i) -> int { return ids[i]; };
+        return block_topk(k, id, n, a.top_k, sub, s);
+    };
+    // Top-K over the positions of blocks sub[0..n) (ascending)
+    auto best_positions = [&](int n) -> int {
+        gather8_keys(s.keys, scores, sub, n, N);
+        auto k = [&](int i) -> uint32_t { return s.keys[i]; };
+        auto id = [&](int i) -> int { return sub[i >> 3] * 8 + (i & 7); };
+        return block_topk(k, id, 8 * n, a.top_k, sel_out, s);
+    };
     int cnt;
     if (a.pool_blocks > 0) {
-        const int nb = (N + 7) / 8;
-        const float *bm = a.bmax + (int64_t)qi * a.bmax_stride;
-        const bool staged = nb <= kCap;
-        if (staged) {
+        int np;
+        if (nb <= kCap) {
             stage_raw(s.keys, bm, nb);
             __syncthreads();
             for (int i = threadIdx.x; i < nb; i += kSelThreads) s.keys[i] = score_key(__uint_as_float(s.keys[i]));
             __syncthreads();
+            auto bkey = [&](int i) -> uint32_t { return s.keys[i]; };
+            auto bid = [&](int i) -> int { return i; };
+            np = block_topk(bkey, bid, nb, a.pool_blocks, s.pool, s);
+        } else if (bm64 != nullptr && nb64 <= kCap) {
+            // the pool_blocks best super-blocks, then the best 8-blocks inside them
+            stage_raw(s.keys, bm64, nb64);
+            __syncthreads();
+            for (int i = threadIdx.x; i < nb64; i += kSelThreads) s.keys[i] = score_key(__uint_as_float(s.keys[i]));
+            __syncthreads();
+            auto gkey = [&](int i) -> uint32_t { return s.keys[i]; };
+            auto gid = [&](int i) -> int { return i; };
+            const int ns = block_topk(gkey, gid, nb64, a.pool_blocks, s.pool, s);
+            __syncthreads();
+            gather8_keys(s.keys, bm, s.pool, ns, nb);
+            for (int i = threadIdx.x; i < ns; i += kSelThreads) s.sup[i] = s.pool[i];
+            __syncthreads();
+            auto ckey = [&](int i) -> uint32_t { return s.keys[i]; };
+            auto cid = [&](int i) -> int { return s.sup[i >> 3] * 8 + (i & 7); };
+            np = block_topk(ckey, cid, 8 * ns, a.pool_blocks, s.pool, s);
+        } else {
+            auto bkey = [&](int i) -> uint32_t { return score_key(bm[i]); };
+            auto bid = [&](int i) -> int { return i; };
+            np = block_topk(bkey, bid, nb, a.pool_blocks, s.pool, s);
         }
-        auto bkey = [&](int i) -> uint32_t { return staged ? s.keys[i] : score_key(bm[i]); };
-        auto bid = [&](int i) -> int { return i; };
-        int np = block_topk(bkey, bid, nb, a.pool_blocks, s.pool, s);
         __syncthreads();
         int32_t *pool_out = a.pool_out ? a.pool_out + (int64_t)qi * a.pool_blocks : nullptr;
         if (pool_out)
             for (int i = threadIdx.x; i < a.pool_blocks; i += blockDim.x)
                 pool_out[i] = i < np ? s.pool[i] : -1;
-        // candidates: the pool's positions, in ascending order
-        const int nc = np * 8;
-        // gather the 8 scores of each pool block (32 B, inside the query's row even for
-        // the last, partial block), then convert; positions past N are dropped
-        for (int c = threadIdx.x; c < 2 * np; c += kSelThreads)
-            cp_async16(s.keys + 4 * c, scores + (int64_t)s.pool[c >> 1] * 8 + 4 * (c & 1));
-        cp_async_commit();
-        cp_async_wait_all();
+        // the top_k best pool blocks hold the Top-K; their positions
+        const int ns = best_blocks(s.pool, np);
         __syncthreads();
-        for (int i = threadIdx.x; i < nc; i += kSelThreads) {
-            const int64_t p = (int64_t)s.pool[i >> 3] * 8 + (i & 7);
-            s.keys[i] = p < N ? score_key(__uint_as_float(s.keys[i])) : 0u;
-        }
+        cnt = best_positions(ns);
+    } else if (N > kSelFlatDirect && bm != nullptr && bm64 != nullptr && nb64 <= kCap) {
+        stage_raw(s.keys, bm64, nb64);
+        __syncthreads();
+        for (int i = threadIdx.x; i < nb64; i += kSelThreads) s.keys[i] = score_key(__uint_as_float(s.keys[i]));
+        __syncthreads();
+        auto gkey = [&](int i) -> uint32_t { return s.keys[i]; };
+        auto gid = [&](int i) -> int { return i; };
+        const int ns = block_topk(gkey, gid, nb64, a.top_k, s.pool, s);
+        __syncthreads();
+        // the blocks of those super-blocks, their top_k best, then their positions
+        gather8_keys(s.keys, bm, s.pool, ns, nb);
+        for (int i = threadIdx.x; i < ns; i += kSelThreads) s.sup[i] = s.pool[i];
         __syncthreads();
         auto ckey = [&](int i) -> uint32_t { return s.keys[i]; };
-        auto cid = [&](int i) -> int { return s.pool[i >> 3] * 8 + (i & 7); };
-        cnt = block_topk(ckey, cid, nc, a.top_k, sel_out, s);
+        auto cid = [&](int i) -> int { return s.sup[i >> 3] * 8 + (i & 7); };
+        const int nsb = block_topk(ckey, cid, 8 * ns, a.top_k, sub, s);
+        __syncthreads();
+        cnt = best_positions(nsb);
     } else {
         const bool staged = N <= kCap;
         if (staged) {
@@ -742,8 +824,10 @@ static cudaError_t launch_select_full_t(const IndexArgs &a, int BT, cudaStream_t
 }
 
 cudaError_t launch_select_full(const IndexArgs &a, int BT, cudaStream_t st) {
-    // flat rows longer than the default stage: the wide stage, if they fit
-    if (a.pool_blocks == 0 && a.n_max > kSelStageMax) return launch_select_full_t<kSelStageWide>(a, BT, st);
+    // flat rows longer than the default stage and without 64-position maxima (the
+    // tensor-core scan): the wide stage, if they fit
+    if (a.pool_blocks == 0 && a.n_max > kSelStageMax && a.bmax64 == nullptr)
+        return launch_select_full_t<kSelStageWide>(a, BT, st);
     return launch_select_full_t<kSelStageMax>(a, BT, st);
 }
 

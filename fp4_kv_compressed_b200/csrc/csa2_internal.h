@@ -70,8 +70,10 @@ struct IndexArgs {
     int64_t n_max;
     float *scores;           // workspace [BT][score_stride]
     int64_t score_stride;
-    float *bmax;             // workspace [BT][bmax_stride] or null
+    float *bmax;             // workspace [BT][bmax_stride] or null: max of each 8 positions
     int64_t bmax_stride;
+    float *bmax64;           // workspace [BT][bmax64_stride] or null: max of each 64 positions
+    int64_t bmax64_stride;
     const int32_t *pool;     // reindex input [BT][pool_blocks]
     int32_t pool_blocks;
     int32_t *pool_out;       // full output [BT][pool_blocks] or null
