@@ -128,54 +128,84 @@ def measured_peaks() -> dict:
     return out
 
 
-def op_rooflines(wl, plan, op_ms: dict, ms_step: float) -> dict:
-    """Per timed op: algorithmic bytes (and flops) per launch over the live launch time."""
+OP_KERNELS = {
+    "csa2_quantize_append": "quantize_append_kernel",
+    "csa2_quantize_append_rope": "quantize_append_kernel",
+    "csa2_index_full": "index_scan_kernel + select_full_kernel",
+    "csa2_index_full_tc": "index_scan_tc_kernel + select_full_kernel",
+    "csa2_index_reindex": "reindex_fused_kernel",
+    "csa2_sparse_attn_decode": "attn_kernel",
+    "csa2_sparse_attn_decode_append": "attn_kernel (with the SWA append)",
+    "csa2_sparse_attn_decode_append_rope": "attn_kernel (with the RoPE + SWA append)",
+}
+
+
+def op_step_bytes(wl, plan, rope: bool = False, index_scan: str = "exact") -> dict:
+    """Per library call name: (algorithmic bytes per step, launches per step), walking the
+    layer plan the way DecodeStack.step issues its calls."""
     ob = op_bytes(wl)
-    pk = measured_peaks()
-    modes = [lp.mode for lp in plan]
-    dec = plan[[lp.layer for lp in plan if lp.mode == "F"][-1]].group
-    spec = {"csa2_index_full": (ob[f"index_full_g{dec}"], modes.count("F"),
-                                "index_scan_kernel + select_full_kernel"),
-            "csa2_index_full_tc": (ob[f"index_full_g{dec}"], modes.count("F"),
-                                   "index_scan_tc_kernel + select_full_kernel"),
-            "csa2_index_reindex": (ob.get(f"index_reindex_g{dec}", 0), modes.count("X"),
-                                   "reindex_fused_kernel"),
-            "csa2_sparse_attn_decode": (ob["attn"], len(modes), "attn_tc_kernel"),
-            # decode: every layer but a group's first appends its SWA row inside the
-            # attention launch
-            "csa2_sparse_attn_decode_append": (ob["attn"] + ob["swa_append"],
-                                               len(modes) - len({lp.group for lp in plan}),
-                                               "attn_tc_kernel (with the SWA append)"),
-            # the same, the new row rotated first: its (cos, sin) row is read too
-            "csa2_sparse_attn_decode_append_rope": (
-                ob["attn"] + ob["swa_append"] + ob["rope_row"],
-                len(modes) - len({lp.group for lp in plan}),
-                "attn_tc_kernel (with the RoPE + SWA append)")}
+    fused = wl.Tq == 1 and wl.swa_len > 0          # decode: SWA append inside the attention
+    first = {}
+    for lp in plan:
+        first.setdefault(lp.group, lp.layer)
+    app = "csa2_quantize_append_rope" if rope else "csa2_quantize_append"
+    full = "csa2_index_full_tc" if index_scan == "tc" else "csa2_index_full"
     out = {}
-    for name, ms in op_ms.items():
-        nbytes, n, kernels = spec[name]
-        if not nbytes or not n:
+
+    def add(name, nbytes):
+        b, n = out.get(name, (0, 0))
+        out[name] = (b + nbytes, n + 1)
+    for lp in plan:
+        g = lp.group
+        if lp.layer == first[g]:
+            add(app, ob[f"append_g{g}"] + ob["swa_append"])
+        elif not fused:
+            add(app, ob["swa_append"])
+        if lp.mode == "F":
+            add(full, ob[f"index_full_g{g}"])
+        elif lp.mode == "X":
+            add("csa2_index_reindex", ob[f"index_reindex_g{g}"])
+        if fused and lp.layer != first[g]:
+            name = "csa2_sparse_attn_decode_append" + ("_rope" if rope else "")
+            add(name, ob["attn"] + ob["swa_append"] + (ob["rope_row"] if rope else 0))
+        else:
+            add("csa2_sparse_attn_decode", ob["attn"])
+    return out
+
+
+def op_rooflines(wl, plan, op_ms: dict, ms_step: float, rope: bool = False,
+                 index_scan: str = "exact") -> dict:
+    """Per library call: algorithmic bytes (and flops) per step over its measured time per
+    step.  op_ms[name] = (total ms per step of the calls of that name, calls per step)."""
+    pk = measured_peaks()
+    per = op_step_bytes(wl, plan, rope, index_scan)
+    modes = [lp.mode for lp in plan]
+    out = {}
+    for name, (tot_ms, n) in op_ms.items():
+        nbytes_step, n_plan = per.get(name, (0, 0))
+        if not nbytes_step or not n:
             continue
-        gbs = nbytes / (ms / 1e3) / 1e9
+        ms = tot_ms / n
+        gbs = nbytes_step / (tot_ms / 1e3) / 1e9
         traffic = None
         if name in NCU_TRAFFIC:
             caps, files, sha = NCU_TRAFFIC[name]
-            if _sources_hash(files) == sha and wl.Tq == 1:
+            if caps and _sources_hash(files) == sha and wl.Tq == 1:
                 traffic = sum(tb * wl.B / tbatch for tb, tbatch in caps)
         e = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-             "frac": gbs / pk["hbm_gbs"], "traffic": traffic, "kernels": kernels,
-             "algorithmic_bytes_per_launch": nbytes, "launch_ms": ms, "launches_per_step": n,
-             "share_of_step": n * ms / ms_step, "peak_source": pk["source"]}
+             "frac": gbs / pk["hbm_gbs"], "traffic": traffic, "kernels": OP_KERNELS.get(name, name),
+             "algorithmic_bytes_per_launch": nbytes_step / n_plan, "launch_ms": ms,
+             "launches_per_step": n, "share_of_step": tot_ms / ms_step, "peak_source": pk["source"]}
         fl = None
         if name.startswith("csa2_sparse_attn_decode"):
-            fl = attn_flops(wl)
+            fl = attn_flops(wl) * n
         elif name == "csa2_index_full_tc":
-            fl = index_scan_flops(wl, dec)
+            fl = sum(index_scan_flops(wl, lp.group) for lp in plan if lp.mode == "F")
         if fl:
-            tfs = fl / (ms / 1e3) / 1e12
+            tfs = fl / (tot_ms / 1e3) / 1e12
             e["tensor"] = {"achieved": tfs, "peak": pk["tflops"], "unit": "TFLOP/s",
-                           "frac": tfs / pk["tflops"], "flops_per_launch": fl}
-            if fl / (pk["tflops"] * 1e12) > nbytes / (pk["hbm_gbs"] * 1e9):
+                           "frac": tfs / pk["tflops"], "flops_per_launch": fl / n}
+            if fl / (pk["tflops"] * 1e12) > nbytes_step / (pk["hbm_gbs"] * 1e9):
                 e.update(bound="tensor", achieved=tfs, peak=pk["tflops"], unit="TFLOP/s",
                          frac=tfs / pk["tflops"])
         out[name] = e
@@ -413,56 +443,47 @@ def run_ours(args, rank, world, local_rank):
     S = max(1, min(10, args.steps))
     import fp4_kv_compressed_b200.stack as stack_mod
 
-    # Timing events around one call per step of each op, recorded on the launching
-    # stream inside the timed graph: the Full op, the first Reindex op and the last
-    # layer's attention.
-    modes = [lp.mode for lp in st.plan]
-    # the last layer's attention: the fused SWA append + attention call in decode
-    if st._fuse_swa(wl.Tq):
-        n_attn = len(modes) - len({lp.group for lp in st.plan})
-        attn_pick = ("csa2_sparse_attn_decode_append" + ("_rope" if args.rope else ""),
-                     (n_attn, n_attn - 1))
-    else:
-        attn_pick = ("csa2_sparse_attn_decode", (len(modes), len(modes) - 1))
-    full_name = "csa2_index_full_tc" if args.index_scan == "tc" else "csa2_index_full"
-    picks = {full_name: (modes.count("F"), 0),
-             "csa2_index_reindex": (modes.count("X"), 0),
-             attn_pick[0]: attn_pick[1]}
-    op_events = {name: [] for name in picks}
-    originals = {name: getattr(stack_mod.bind, name) for name in picks}
-
-    def make_timed(name):
-        per_step, pick = picks[name]
-        orig = originals[name]
-        count = [0]
-
-        def f(*a, **k):
-            i = count[0]
-            count[0] += 1
-            if per_step and i % per_step == pick:
-                e0 = torch.cuda.Event(enable_timing=True, external=True)
-                e1 = torch.cuda.Event(enable_timing=True, external=True)
-                e0.record()
-                orig(*a, **k)
-                e1.record()
-                op_events[name].append((e0, e1))
-            else:
-                orig(*a, **k)
-        return f
-
+    # The headline graph holds S steps and no events.  A second graph holds one step
+    # with a CUDA event recorded on the launching stream after every library call (and
+    # one before the first): consecutive events partition the step, so each call's
+    # time is the interval between its two events and the calls' times add up to the
+    # step.  It is replayed after the timed region, with the same warm-up and
+    # synchronisation, for the per-op figures (roofline, shares).
     g = torch.cuda.CUDAGraph()
-    for name in picks:
-        setattr(stack_mod.bind, name, make_timed(name))
-    try:
-        with torch.cuda.graph(g, stream=stream):
-            for _ in range(S):
-                st.step(**inputs)
-    finally:
-        for name, orig in originals.items():
-            setattr(stack_mod.bind, name, orig)
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(S):
+            st.step(**inputs)
     g1 = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g1, stream=stream):
         st.step(**inputs)
+    op_names = [n for n in ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_index_full",
+                            "csa2_index_full_tc", "csa2_index_reindex", "csa2_sparse_attn_decode",
+                            "csa2_sparse_attn_decode_append", "csa2_sparse_attn_decode_append_rope")
+                if hasattr(stack_mod.bind, n)]
+    originals = {name: getattr(stack_mod.bind, name) for name in op_names}
+    marks = []                       # (op name, event after the call)
+
+    def make_marked(name):
+        orig = originals[name]
+
+        def f(*a, **k):
+            orig(*a, **k)
+            e = torch.cuda.Event(enable_timing=True, external=True)
+            e.record()
+            marks.append((name, e))
+        return f
+
+    g_ops = torch.cuda.CUDAGraph()
+    for name in op_names:
+        setattr(stack_mod.bind, name, make_marked(name))
+    try:
+        with torch.cuda.graph(g_ops, stream=stream):
+            e_first = torch.cuda.Event(enable_timing=True, external=True)
+            e_first.record()
+            st.step(**inputs)
+    finally:
+        for name, orig in originals.items():
+            setattr(stack_mod.bind, name, orig)
 
     reps = max(1, args.steps // S)
     K = reps * S
@@ -486,8 +507,25 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     ms = start.elapsed_time(end)
-    op_ms = {name: statistics.mean(a.elapsed_time(b) for a, b in evs)
-             for name, evs in op_events.items() if evs}
+    # per-op figures from the partitioned graph (replayed after the timed region)
+    op_sum, op_n, ops_step = {}, {}, []
+    for _ in range(max(args.warmup, 3)):
+        g_ops.replay()
+    torch.cuda.synchronize(dev)
+    for _ in range(max(3, min(20, reps))):
+        with torch.cuda.stream(stream):
+            g_ops.replay()
+        torch.cuda.synchronize(dev)
+        prev, tot = e_first, 0.0
+        for name, e in marks:
+            dt = prev.elapsed_time(e)
+            op_sum[name] = op_sum.get(name, 0.0) + dt
+            op_n[name] = op_n.get(name, 0) + 1
+            prev, tot = e, tot + dt
+        ops_step.append(tot)
+    n_rep = len(ops_step)
+    op_ms = {name: (op_sum[name] / n_rep, op_n[name] // n_rep) for name in op_sum}
+    ops_step_ms = statistics.mean(ops_step)
     ms_max = max_over_ranks(ms, world, dev)
     if st.dev_err.item() != 0:
         raise RuntimeError(f"device error bits {st.dev_err.item()} in the timed steps")
@@ -531,7 +569,7 @@ def run_ours(args, rank, world, local_rank):
     sb = step_bytes(wl)
     ob = op_bytes(wl)
     g_full = st.plan[full_layers[0]].group
-    ops = op_rooflines(wl, st.plan, op_ms, ms_step)
+    ops = op_rooflines(wl, st.plan, op_ms, ops_step_ms, rope=args.rope, index_scan=args.index_scan)
     dominant = max(ops, key=lambda n: ops[n]["share_of_step"])
     launches = st.launches_per_step() * K
     line = {
@@ -543,6 +581,7 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": workload_config(wl, args, world),
         "step": {"cuda_graph": True, "algorithmic_bytes": sb,
+                 "ms_with_op_events": ops_step_ms,
                  "gbps": sb / (ms_step / 1e3) / 1e9, "frac_of_8tbs": sb / (ms_step / 1e3) / 8e12,
                  "token_layer_steps_per_s": value * wl.B},
         "roofline": dict(ops[dominant], op=dominant),

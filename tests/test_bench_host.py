@@ -99,26 +99,35 @@ def test_reference_arm_other_ranks_do_nothing():
 
 
 def test_op_rooflines_dominant_and_traffic():
-    """Per-op roofline entries: bytes / live time, share of the step, ncu traffic only
-    while the captured kernel's sources are unchanged, dominant op by share."""
+    """Per-op roofline entries: algorithmic bytes per step over the op's measured time per
+    step (the per-call intervals partition the step, so the shares add up to 1), ncu
+    traffic only while the captured kernel's sources are unchanged, dominant op by share."""
     from fp4_kv_compressed_b200.stack import plan_layers
     wl = WORKLOADS["decode_128k"]
     plan = plan_layers([g.schedule for g in wl.groups])
-    op_ms = {"csa2_index_full": 0.4, "csa2_index_reindex": 0.1,
-             "csa2_sparse_attn_decode_append": 0.03}
-    ops = bench.op_rooflines(wl, plan, op_ms, ms_step=1.5)
+    per = bench.op_step_bytes(wl, plan)
+    assert per["csa2_quantize_append"][1] == 1 and per["csa2_index_full"][1] == 1
+    assert per["csa2_index_reindex"][1] == 4 and per["csa2_sparse_attn_decode"][1] == 1
+    assert per["csa2_sparse_attn_decode_append"][1] == 19
+    assert sum(b for b, _ in per.values()) == bench.step_bytes(wl)
+    op_ms = {"csa2_quantize_append": (0.005, 1), "csa2_index_full": (0.4, 1),
+             "csa2_index_reindex": (0.4, 4), "csa2_sparse_attn_decode": (0.03, 1),
+             "csa2_sparse_attn_decode_append": (0.665, 19)}
+    ms_step = sum(t for t, _ in op_ms.values())
+    ops = bench.op_rooflines(wl, plan, op_ms, ms_step=ms_step)
+    assert abs(sum(e["share_of_step"] for e in ops.values()) - 1.0) < 1e-12
     f = ops["csa2_index_full"]
     assert f["launches_per_step"] == 1 and f["bound"] == "hbm"
     assert abs(f["achieved"] - 1_154_155_776 / 0.4e-3 / 1e9) < 1e-6
-    assert abs(f["share_of_step"] - 0.4 / 1.5) < 1e-12
     a = ops["csa2_sparse_attn_decode_append"]
-    assert a["launches_per_step"] == 19 and abs(a["share_of_step"] - 19 * 0.03 / 1.5) < 1e-12
+    assert a["launches_per_step"] == 19 and abs(a["launch_ms"] - 0.035) < 1e-12
     assert a["algorithmic_bytes_per_launch"] == bench.op_bytes(wl)["attn"] + 64 * (1024 + 516)
     assert a["tensor"]["flops_per_launch"] == 64 * 4 * 64 * 512 * 640
     assert ops["csa2_index_reindex"]["launches_per_step"] == 4
     for name, e in ops.items():
-        caps, files, sha = bench.NCU_TRAFFIC[name]
-        expect = sum(tb * wl.B / b for tb, b in caps) if bench._sources_hash(files) == sha else None
+        caps, files, sha = bench.NCU_TRAFFIC.get(name, ([], (), ""))
+        expect = (sum(tb * wl.B / b for tb, b in caps)
+                  if caps and bench._sources_hash(files) == sha else None)
         assert e["traffic"] == expect
     assert max(ops, key=lambda n: ops[n]["share_of_step"]) == "csa2_sparse_attn_decode_append"
 
@@ -146,15 +155,17 @@ def test_prefill_and_rope_op_rooflines():
     vis = sum((t + 1) // 2 for t in range(wl.ctx - Tq, wl.ctx))
     assert bench.index_scan_flops(wl, 0) == vis * 2 * HI * d
     plan = plan_layers([g.schedule for g in wl.groups])
-    ops = bench.op_rooflines(wl, plan, {"csa2_index_full_tc": 0.6, "csa2_sparse_attn_decode": 0.7},
-                             ms_step=4.7)
+    ops = bench.op_rooflines(wl, plan, {"csa2_index_full_tc": (0.6, 1),
+                                        "csa2_sparse_attn_decode": (4.2, 6)},
+                             ms_step=4.7, index_scan="tc")
     tc = ops["csa2_index_full_tc"]
     assert tc["traffic"] is None and ops["csa2_sparse_attn_decode"]["traffic"] is None
     assert abs(tc["tensor"]["achieved"] - vis * 2 * HI * d / 0.6e-3 / 1e12) < 1e-9
     assert tc["bound"] == "hbm"          # the score round trip outweighs the MMAs
     dec = WORKLOADS["decode_128k"]
     plan = plan_layers([g.schedule for g in dec.groups])
-    r = bench.op_rooflines(dec, plan, {"csa2_sparse_attn_decode_append_rope": 0.033}, 1.12)
+    r = bench.op_rooflines(dec, plan, {"csa2_sparse_attn_decode_append_rope": (19 * 0.033, 19)}, 1.12,
+                           rope=True)
     e = r["csa2_sparse_attn_decode_append_rope"]
     assert e["algorithmic_bytes_per_launch"] == (bench.op_bytes(dec)["attn"] + 64 * (1024 + 516)
                                                  + 64 * ROPE_PAIRS * 8)
