@@ -9,7 +9,8 @@ from ._binding import (CSA2_OP_INDEX_FULL, CSA2_OP_INDEX_REINDEX, CSA2_OP_SPARSE
                        CSA2GlobalKV, CSA2Rope, CSA2SWA, Csa2Error, DEFAULT_WAIT_LIMIT_NS,
                        DEVERR_INDEX, DEVERR_NMAX, DEVERR_RANGE, DEVERR_ROPE, DEVERR_SLOT,
                        DEVERR_TIMEOUT, EXPORTS, LIB_PATH, Rope, csa2_debug_set_waits,
-                       csa2_index_full, csa2_index_full_tc, csa2_index_reindex,
+                       csa2_attn_combine, csa2_index_full, csa2_index_full_slice, csa2_index_full_tc,
+                       csa2_index_merge, csa2_index_reindex,
                        csa2_quantize_append, csa2_quantize_append_rope, csa2_read_device_error,
                        csa2_sparse_attn_decode, csa2_sparse_attn_decode_append,
                        csa2_sparse_attn_decode_append_rope, csa2_workspace_size, load_library)
@@ -22,7 +23,8 @@ __all__ = [
     "CSA2Rope", "CSA2SWA", "Csa2Error", "DEFAULT_WAIT_LIMIT_NS", "DEVERR_TIMEOUT",
     "csa2_debug_set_waits", "DEVERR_INDEX", "DEVERR_NMAX", "DEVERR_RANGE",
     "DEVERR_ROPE", "DEVERR_SLOT", "EXPORTS", "LIB_PATH", "Rope", "csa2_index_full",
-    "csa2_index_full_tc", "csa2_index_reindex", "csa2_quantize_append",
+    "csa2_index_full_tc", "csa2_index_reindex", "csa2_attn_combine", "csa2_index_full_slice",
+    "csa2_index_merge", "csa2_quantize_append",
     "csa2_quantize_append_rope", "csa2_read_device_error", "csa2_sparse_attn_decode",
     "csa2_sparse_attn_decode_append", "csa2_sparse_attn_decode_append_rope",
     "csa2_workspace_size",

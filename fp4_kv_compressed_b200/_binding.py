@@ -32,7 +32,8 @@ EXPORTS = ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_workspace_
            "csa2_index_full", "csa2_index_full_tc", "csa2_index_full_noalloc",
            "csa2_index_reindex", "csa2_sparse_attn_decode", "csa2_sparse_attn_decode_append",
            "csa2_sparse_attn_decode_append_rope", "csa2_read_device_error",
-           "csa2_status_string", "csa2_abi_version", "csa2_debug_set_waits")
+           "csa2_status_string", "csa2_abi_version", "csa2_debug_set_waits",
+           "csa2_index_full_slice", "csa2_index_merge", "csa2_attn_combine")
 
 
 class Csa2Error(RuntimeError):
@@ -101,6 +102,12 @@ def load_library(path: str = LIB_PATH):
     L.csa2_abi_version.restype = i32
     L.csa2_debug_set_waits.argtypes = [C.c_uint64, i32]
     L.csa2_debug_set_waits.restype = None
+    i64 = C.c_int64
+    L.csa2_index_full_slice.argtypes = [P, i64, P, P, P, i32, i32, i32, i32, i32, P, P, P, sz, P, P]
+    L.csa2_index_merge.argtypes = [P, i32, i32, i32, i32, i64, i64, P, P, P, P]
+    L.csa2_attn_combine.argtypes = [P, P, i32, i64, P, P, P]
+    for fn in ("csa2_index_full_slice", "csa2_index_merge", "csa2_attn_combine"):
+        getattr(L, fn).restype = C.c_int
     for fn in ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_index_full",
                "csa2_index_full_tc", "csa2_index_reindex", "csa2_sparse_attn_decode",
                "csa2_sparse_attn_decode_append", "csa2_sparse_attn_decode_append_rope",
@@ -180,6 +187,36 @@ def csa2_index_full_tc(kv: CSA2GlobalKV, q_idx, w, q_pos, Tq: int, H_I: int, n_m
                               _ptr(topk_count), _ptr(workspace), ws_bytes, _ptr(dev_err),
                               _stream(stream))
     _check("csa2_index_full_tc", st)
+
+
+def csa2_index_full_slice(kv: CSA2GlobalKV, entry_lo: int, q_idx, w, q_pos, Tq: int, H_I: int,
+                          n_max: int, pool_blocks: int, top_k: int, pool_keys_out, topk_keys_out,
+                          workspace, dev_err=None, stream=None):
+    """Context parallel: the Full layer on a slice of the entries, its local selections
+    as candidate keys."""
+    L = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = L.csa2_index_full_slice(C.byref(kv), entry_lo, _ptr(q_idx), _ptr(w), _ptr(q_pos), Tq, H_I,
+                                 n_max, pool_blocks, top_k, _ptr(pool_keys_out), _ptr(topk_keys_out),
+                                 _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream))
+    _check("csa2_index_full_slice", st)
+
+
+def csa2_index_merge(lists, BT: int, n_lists: int, list_len: int, k: int, local_lo: int,
+                     local_hi: int, ids_out, count_out, local_out, stream=None):
+    """Context parallel: the exact selection from the shards' candidate lists."""
+    L = load_library()
+    st = L.csa2_index_merge(_ptr(lists), BT, n_lists, list_len, k, local_lo, local_hi,
+                            _ptr(ids_out), _ptr(count_out), _ptr(local_out), _stream(stream))
+    _check("csa2_index_merge", st)
+
+
+def csa2_attn_combine(o_parts, lse_parts, n_parts: int, rows: int, out, lse_out, stream=None):
+    """Context parallel: one softmax from the shards' partial attention results."""
+    L = load_library()
+    st = L.csa2_attn_combine(_ptr(o_parts), _ptr(lse_parts), n_parts, rows, _ptr(out),
+                             _ptr(lse_out), _stream(stream))
+    _check("csa2_attn_combine", st)
 
 
 def csa2_index_reindex(kv: CSA2GlobalKV, q_idx, w, q_pos, Tq: int, H_I: int, pool,

@@ -86,7 +86,7 @@ bool hi_supported(int32_t H_I) {
 
 extern "C" {
 
-int32_t csa2_abi_version(void) { return 102; }
+int32_t csa2_abi_version(void) { return 103; }
 
 void csa2_debug_set_waits(uint64_t limit_ns, int32_t stuck_wait) {
     g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
@@ -215,10 +215,13 @@ static csa2_status index_full(const csa2_global_kv *kv, const void *q_idx_bf16, 
                               const int32_t *q_pos, int32_t Tq, int32_t H_I, int32_t n_max,
                               int32_t pool_blocks, int32_t top_k, int32_t *pool_out,
                               int32_t *topk_out, int32_t *topk_count, void *workspace,
-                              size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream, bool tc) {
+                              size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream, bool tc,
+                              int64_t entry_lo = 0, uint64_t *pool_keys_out = nullptr,
+                              uint64_t *topk_keys_out = nullptr) {
     csa2_status st = check_kv(kv, true);
     if (st != CSA2_OK) return st;
-    if (!q_idx_bf16 || !w || !q_pos || !topk_out || !topk_count) return CSA2_ERR_INVALID_ARG;
+    if (!q_idx_bf16 || !w || !q_pos) return CSA2_ERR_INVALID_ARG;
+    if (topk_keys_out == nullptr && (!topk_out || !topk_count)) return CSA2_ERR_INVALID_ARG;
     if (!aligned(q_idx_bf16, tc ? 16 : 4) || !aligned(w, 4)) return CSA2_ERR_INVALID_ARG;
     if (Tq <= 0 || n_max < 0) return CSA2_ERR_INVALID_ARG;
     if (!hi_supported(H_I)) return CSA2_ERR_UNSUPPORTED;
@@ -259,6 +262,9 @@ static csa2_status index_full(const csa2_global_kv *kv, const void *q_idx_bf16, 
     a.topk_count = topk_count;
     a.dev_err = dev_err;
     a.wait = current_wait_cfg();
+    a.entry_lo = entry_lo;
+    a.pool_keys_out = pool_keys_out;
+    a.topk_keys_out = topk_keys_out;
     cudaStream_t s = (cudaStream_t)stream;
     st = launched(tc ? launch_index_scan_tc(a, (int)kv->batch, s) : launch_index_scan(a, (int)BT, s));
     if (st != CSA2_OK) return st;
@@ -281,6 +287,41 @@ csa2_status csa2_index_full_tc(const csa2_global_kv *kv, const void *q_idx_bf16,
                                size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
     return index_full(kv, q_idx_bf16, w, q_pos, Tq, H_I, n_max, pool_blocks, top_k, pool_out,
                       topk_out, topk_count, workspace, ws_bytes, dev_err, stream, true);
+}
+
+csa2_status csa2_index_full_slice(const csa2_global_kv *kv, int64_t entry_lo,
+                                  const void *q_idx_bf16, const float *w, const int32_t *q_pos,
+                                  int32_t Tq, int32_t H_I, int32_t n_max, int32_t pool_blocks,
+                                  int32_t top_k, uint64_t *pool_keys_out, uint64_t *topk_keys_out,
+                                  void *workspace, size_t ws_bytes, int32_t *dev_err,
+                                  csa2_stream_t stream) {
+    if (entry_lo < 0 || entry_lo % 64 != 0 || !topk_keys_out) return CSA2_ERR_INVALID_ARG;
+    if (pool_blocks > 0 && !pool_keys_out) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(topk_keys_out, 8) || (pool_keys_out && !aligned(pool_keys_out, 8))) return CSA2_ERR_INVALID_ARG;
+    if (kv && entry_lo / 8 + (int64_t)kv->cap / 8 + 1 > INT32_MAX / 2) return CSA2_ERR_UNSUPPORTED;
+    return index_full(kv, q_idx_bf16, w, q_pos, Tq, H_I, n_max, pool_blocks, top_k, nullptr, nullptr,
+                      nullptr, workspace, ws_bytes, dev_err, stream, false, entry_lo,
+                      pool_blocks > 0 ? pool_keys_out : nullptr, topk_keys_out);
+}
+
+csa2_status csa2_index_merge(const uint64_t *lists, int32_t BT, int32_t n_lists, int32_t list_len,
+                             int32_t k, int64_t local_lo, int64_t local_hi, int32_t *ids_out,
+                             int32_t *count_out, int32_t *local_out, csa2_stream_t stream) {
+    if (!lists || BT <= 0 || n_lists <= 0 || list_len <= 0 || k <= 0) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(lists, 8)) return CSA2_ERR_INVALID_ARG;
+    if (!ids_out && !local_out) return CSA2_ERR_INVALID_ARG;
+    if (k > CSA2_POOL_MAX || (int64_t)n_lists * list_len > 16384) return CSA2_ERR_UNSUPPORTED;
+    if (BT > 65535 * 32) return CSA2_ERR_UNSUPPORTED;
+    return launched(launch_index_merge(lists, BT, n_lists, list_len, k, local_lo, local_hi, ids_out,
+                                       count_out, local_out, (cudaStream_t)stream));
+}
+
+csa2_status csa2_attn_combine(const float *o_parts, const float *lse_parts, int32_t n_parts, int64_t rows,
+                              float *out, float *lse_out, csa2_stream_t stream) {
+    if (!o_parts || !lse_parts || !out || !lse_out || n_parts <= 0 || rows < 0) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(o_parts, 16) || !aligned(out, 16)) return CSA2_ERR_INVALID_ARG;
+    return launched(launch_attn_combine(o_parts, lse_parts, n_parts, rows, out, lse_out,
+                                        (cudaStream_t)stream));
 }
 
 csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,

@@ -155,7 +155,7 @@ index_scan_kernel(IndexArgs a) {
     grid_dep_wait();
     const int qi = blockIdx.y;
     const int b = qi / a.Tq;
-    int64_t N = visible_entries(a.q_pos[qi], a.ratio);
+    int64_t N = max64(0, visible_entries(a.q_pos[qi], a.ratio) - a.entry_lo);   // of this cache
     if (N > a.n_max || N > a.cap) {
         if (threadIdx.x == 0 && blockIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_NMAX);
         N = min64(min64(N, a.n_max), a.cap);
@@ -483,7 +483,7 @@ select_full_kernel(IndexArgs a) {
     __shared__ int sub[CSA2_TOPK_MAX];
     grid_dep_wait();
     const int qi = blockIdx.x;
-    int64_t N64 = visible_entries(a.q_pos[qi], a.ratio);
+    int64_t N64 = max64(0, visible_entries(a.q_pos[qi], a.ratio) - a.entry_lo);
     N64 = min64(min64(N64, a.n_max), a.cap);
     const int N = (int)N64;
     const int nb = (N + 7) / 8, nb64 = (N + 63) / 64;
@@ -543,6 +543,13 @@ select_full_kernel(IndexArgs a) {
         if (pool_out)
             for (int i = threadIdx.x; i < a.pool_blocks; i += blockDim.x)
                 pool_out[i] = i < np ? s.pool[i] : -1;
+        if (a.pool_keys_out) {
+            uint64_t *pk = a.pool_keys_out + (int64_t)qi * a.pool_blocks;
+            for (int i = threadIdx.x; i < a.pool_blocks; i += blockDim.x)
+                pk[i] = i < np ? ((uint64_t)score_key(__ldg(bm + s.pool[i])) << 32) |
+                                     (uint32_t)~(uint32_t)(s.pool[i] + a.entry_lo / 8)
+                               : 0ull;
+        }
         // the top_k best pool blocks hold the Top-K; their positions
         const int ns = best_blocks(s.pool, np);
         __syncthreads();
@@ -579,9 +586,70 @@ select_full_kernel(IndexArgs a) {
     }
     __syncthreads();
     grid_dep_launch();
-    int32_t *topk = a.topk_out + (int64_t)qi * a.top_k;
-    for (int i = threadIdx.x; i < a.top_k; i += blockDim.x) topk[i] = i < cnt ? sel_out[i] : -1;
-    if (threadIdx.x == 0) a.topk_count[qi] = cnt;
+    if (a.topk_keys_out) {
+        // slice form: the selected entries' candidate keys, global ids
+        uint64_t *tk = a.topk_keys_out + (int64_t)qi * a.top_k;
+        for (int i = threadIdx.x; i < a.top_k; i += blockDim.x)
+            tk[i] = i < cnt ? ((uint64_t)score_key(__ldg(scores + sel_out[i])) << 32) |
+                                  (uint32_t)~(uint32_t)(sel_out[i] + a.entry_lo)
+                            : 0ull;
+    }
+    if (a.topk_out) {
+        int32_t *topk = a.topk_out + (int64_t)qi * a.top_k;
+        for (int i = threadIdx.x; i < a.top_k; i += blockDim.x) topk[i] = i < cnt ? sel_out[i] : -1;
+    }
+    if (threadIdx.x == 0 && a.topk_count) a.topk_count[qi] = cnt;
+}
+
+// ------------------------------------------------------------------------------
+// Context parallel: merge of the shards' candidate lists.  One CTA per query; the lists
+// [n_lists][BT][list_len] of candidate keys (order key << 32 | ~global id, 0 = empty;
+// shard-major, as an all-gather lays them out) are given in ascending slice order and
+// each is ascending in id, so candidate index order
+// is id order and block_topk's (key desc, index asc) order is the (key desc, id asc)
+// order.  Every item of the global Top-k is in its own shard's local Top-k, so the
+// result is exact.  Outputs ascending ids, -1 padded; with local_out, also the ids in
+// [lo, hi) shifted by -lo (others -1).
+// ------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kSelThreads)
+index_merge_kernel(const uint64_t *lists, int n_lists, int list_len, int k, int64_t lo, int64_t hi,
+                   int32_t *ids_out, int32_t *count_out, int32_t *local_out) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    SelSmem &s = *reinterpret_cast<SelSmem *>(smem_raw);
+    __shared__ int sel_out[CSA2_POOL_MAX];
+    grid_dep_wait();
+    const int qi = blockIdx.x, BT = gridDim.x;
+    const int n = n_lists * list_len;
+    auto at = [&](int i) -> const uint64_t * {
+        return lists + ((int64_t)(i / list_len) * BT + qi) * list_len + i % list_len;
+    };
+    for (int i = threadIdx.x; i < n; i += kSelThreads) s.keys[i] = (uint32_t)(__ldg(at(i)) >> 32);
+    __syncthreads();
+    auto key = [&](int i) -> uint32_t { return s.keys[i]; };
+    auto id = [&](int i) -> int { return (int)~(uint32_t)__ldg(at(i)); };
+    const int cnt = block_topk(key, id, n, k, sel_out, s);
+    __syncthreads();
+    grid_dep_launch();
+    for (int i = threadIdx.x; i < k; i += kSelThreads) {
+        const int g = i < cnt ? sel_out[i] : -1;
+        if (ids_out) ids_out[(int64_t)qi * k + i] = g;
+        if (local_out) local_out[(int64_t)qi * k + i] = g >= 0 && g >= lo && g < hi ? (int)(g - lo) : -1;
+    }
+    if (threadIdx.x == 0 && count_out) count_out[qi] = cnt;
+}
+
+cudaError_t launch_index_merge(const uint64_t *lists, int BT, int n_lists, int list_len, int k,
+                               int64_t lo, int64_t hi, int32_t *ids_out, int32_t *count_out,
+                               int32_t *local_out, cudaStream_t st) {
+    const size_t smem = sizeof(SelSmem);
+    static std::atomic<uint64_t> configured{0};   // per device
+    {
+        cudaError_t e = config_kernel_once(index_merge_kernel, smem, configured);
+        if (e != cudaSuccess) return e;
+    }
+    cudaError_t e = launch_pdl(index_merge_kernel, dim3(BT), dim3(kSelThreads), smem, st, lists, n_lists,
+                               list_len, k, lo, hi, ids_out, count_out, local_out);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // ------------------------------------------------------------------------------

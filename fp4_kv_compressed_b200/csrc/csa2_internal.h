@@ -82,6 +82,12 @@ struct IndexArgs {
     int32_t *topk_count;
     int32_t *dev_err;
     WaitCfg wait;
+    // slice form (context parallel): the cache holds entries [entry_lo, entry_lo + cap)
+    // of each request (entry_lo a multiple of 64; 0 otherwise), and the selections are
+    // written as candidate keys (order key << 32 | ~global id) instead of ids
+    int64_t entry_lo;
+    uint64_t *pool_keys_out;   // [BT][pool_blocks] or null
+    uint64_t *topk_keys_out;   // [BT][top_k] or null
 };
 
 struct AttnArgs {
@@ -172,5 +178,10 @@ cudaError_t launch_index_scan_tc(const IndexArgs &a, int B, cudaStream_t st);
 cudaError_t launch_select_full(const IndexArgs &a, int BT, cudaStream_t st);
 cudaError_t launch_reindex_fused(const IndexArgs &a, int BT, cudaStream_t st);
 cudaError_t launch_sparse_attn(const AttnArgs &a, int BT, cudaStream_t st);
+cudaError_t launch_index_merge(const uint64_t *lists, int BT, int n_lists, int list_len, int k,
+                               int64_t lo, int64_t hi, int32_t *ids_out, int32_t *count_out,
+                               int32_t *local_out, cudaStream_t st);
+cudaError_t launch_attn_combine(const float *o_parts, const float *lse_parts, int n_parts, int64_t rows,
+                                float *out, float *lse_out, cudaStream_t st);
 
 }  // namespace csa2

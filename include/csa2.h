@@ -266,6 +266,70 @@ CSA2_API csa2_status csa2_index_full_noalloc(const csa2_global_kv *kv, const voi
                                              int32_t *dev_err, csa2_stream_t stream);
 
 /*
+ * Context parallel: a single request too long for one GPU is split by entry range
+ * across shards (DeepSeek V4.1 Flash study notes, section 2 with report Figure 5: the
+ * Full-layer scan is the only per-query cost that grows with the context).  Each
+ * shard holds entries [entry_lo, entry_lo + cap) of every request in an ordinary
+ * csa2_global_kv.  The steps, in order:
+ *   1. csa2_index_full_slice on every shard: the Full scan of its slice and its local
+ *      pool and Top-K, written as candidate keys;
+ *   2. an all-gather of those lists (the caller's collective, e.g. NCCL), shard-major;
+ *   3. csa2_index_merge: the exact global pool / Top-K (every item of the global
+ *      selection is in its own shard's local selection, so the merge is exact), and
+ *      each shard's own part of it as slice-local ids;
+ *   4. csa2_sparse_attn_decode on every shard over its part (the shard holding the
+ *      query's window passes swa_len, the others 0), then an all-gather of the
+ *      partial outputs and lse, and csa2_attn_combine.
+ * The pages define no API for this; these calls restate the same score, selection
+ * order and softmax over a split cache.
+ *
+ * csa2_index_full_slice: csa2_index_full on a slice.  entry_lo >= 0, a multiple of 64
+ * (so that blocks of 8 and 64 positions fall inside one slice); the query at token
+ * position t sees the local entries e with entry_lo + e < (t + 1) / ratio; n_max >= the
+ * local visible count of every query (<= cap).  Outputs, ascending in id:
+ *   pool_keys_out [B][Tq][pool_blocks] (pool_blocks > 0): the slice's best blocks,
+ *   topk_keys_out [B][Tq][top_k]: the slice's best entries,
+ * each as the candidate key (order key << 32) | (0xFFFFFFFF - global id), where the
+ * order key is larger for a larger score (equal scores equal keys) and 0 marks an
+ * empty slot.  Block ids are global entry ids / 8.  Workspace and errors as for
+ * csa2_index_full (with the local n_max); both outputs 8-byte aligned.
+ */
+CSA2_API csa2_status csa2_index_full_slice(const csa2_global_kv *kv, int64_t entry_lo,
+                                           const void *q_idx_bf16, const float *w,
+                                           const int32_t *q_pos, int32_t Tq, int32_t H_I,
+                                           int32_t n_max, int32_t pool_blocks, int32_t top_k,
+                                           uint64_t *pool_keys_out, uint64_t *topk_keys_out,
+                                           void *workspace, size_t ws_bytes, int32_t *dev_err,
+                                           csa2_stream_t stream);
+
+/*
+ * csa2_index_merge: the best k candidates by (score desc, id asc) of each query from
+ * n_lists lists of candidate keys, lists [n_lists][BT][list_len] (shard-major, as an
+ * all-gather lays them out), given in ascending slice order, each ascending in id
+ * (as csa2_index_full_slice writes them).  n_lists * list_len <= 16384, k <= 2048.
+ *   ids_out [BT][k] (or NULL): the global ids, ascending, -1 padded;
+ *   count_out [BT] (or NULL): how many;
+ *   local_out [BT][k] (or NULL): the same ids minus local_lo where local_lo <= id <
+ *       local_hi, else -1 (a shard's own part, as ids of its slice).
+ * For a pool, ids are block ids and local_lo / local_hi are block bounds.
+ */
+CSA2_API csa2_status csa2_index_merge(const uint64_t *lists, int32_t BT, int32_t n_lists,
+                                      int32_t list_len, int32_t k, int64_t local_lo,
+                                      int64_t local_hi, int32_t *ids_out, int32_t *count_out,
+                                      int32_t *local_out, csa2_stream_t stream);
+
+/*
+ * csa2_attn_combine: one softmax over the union of the shards' keys from their
+ * normalised partial results.  o_parts [n_parts][rows][512] fp32 (16-byte aligned),
+ * lse_parts [n_parts][rows] (natural log, -inf = no key):
+ *   lse = log sum_p exp(lse_p),  out = sum_p exp(lse_p - lse) o_p
+ * (out 0 and lse -inf when every part is -inf).  rows = B * Tq * H.
+ */
+CSA2_API csa2_status csa2_attn_combine(const float *o_parts, const float *lse_parts, int32_t n_parts,
+                                       int64_t rows, float *out, float *lse_out,
+                                       csa2_stream_t stream);
+
+/*
  * a6 Reindex layer: the same score with this layer's own q_idx / w, over the
  * visible positions of the pool's blocks only, then Top-K (same order, same
  * output form).  pool [B][Tq][pool_blocks] as written by csa2_index_full
