@@ -26,6 +26,7 @@ STATUS = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_CAPACITY",
 DEVERR_SLOT, DEVERR_INDEX, DEVERR_NMAX, DEVERR_RANGE, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
 DEFAULT_WAIT_LIMIT_NS = 500_000_000
 DEVERR_ROPE = 0x20
+DEVERR_PAGE = 0x40
 
 # every symbol declared in include/csa2.h
 EXPORTS = ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_workspace_size",
@@ -33,7 +34,9 @@ EXPORTS = ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_workspace_
            "csa2_index_reindex", "csa2_sparse_attn_decode", "csa2_sparse_attn_decode_append",
            "csa2_sparse_attn_decode_append_rope", "csa2_read_device_error",
            "csa2_status_string", "csa2_abi_version", "csa2_debug_set_waits",
-           "csa2_index_full_slice", "csa2_index_merge", "csa2_attn_combine")
+           "csa2_index_full_slice", "csa2_index_merge", "csa2_attn_combine",
+           "csa2_quantize_append_paged", "csa2_index_full_paged", "csa2_index_reindex_paged",
+           "csa2_sparse_attn_decode_paged")
 
 
 class Csa2Error(RuntimeError):
@@ -52,6 +55,13 @@ class CSA2GlobalKV(C.Structure):
 class CSA2SWA(C.Structure):
     _fields_ = [("codes", C.c_void_p), ("scale", C.c_void_p), ("batch", C.c_int32),
                 ("window_cap", C.c_int32)]
+
+
+class CSA2PagedKV(C.Structure):
+    _fields_ = [("codes", C.c_void_p), ("scales", C.c_void_p), ("idx_codes", C.c_void_p),
+                ("idx_scale", C.c_void_p), ("block_table", C.c_void_p), ("batch", C.c_int32),
+                ("max_pages", C.c_int32), ("page_size", C.c_int32), ("n_pages", C.c_int32),
+                ("d_idx", C.c_int32), ("ratio", C.c_int32)]
 
 
 class CSA2Rope(C.Structure):
@@ -107,6 +117,14 @@ def load_library(path: str = LIB_PATH):
     L.csa2_index_merge.argtypes = [P, i32, i32, i32, i32, i64, i64, P, P, P, P]
     L.csa2_attn_combine.argtypes = [P, P, i32, i64, P, P, P]
     for fn in ("csa2_index_full_slice", "csa2_index_merge", "csa2_attn_combine"):
+        getattr(L, fn).restype = C.c_int
+    L.csa2_quantize_append_paged.argtypes = [P, P, P, i32, P, P, P, i32, P, P, P, P]
+    L.csa2_index_full_paged.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, P, P, P, P, sz, P, P]
+    L.csa2_index_reindex_paged.argtypes = [P, P, P, P, i32, i32, P, i32, i32, P, P, P, P]
+    L.csa2_sparse_attn_decode_paged.argtypes = [P, P, P, P, P, i32, i32, P, i32, i32, C.c_float,
+                                                P, P, P, P, P]
+    for fn in ("csa2_quantize_append_paged", "csa2_index_full_paged", "csa2_index_reindex_paged",
+               "csa2_sparse_attn_decode_paged"):
         getattr(L, fn).restype = C.c_int
     for fn in ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_index_full",
                "csa2_index_full_tc", "csa2_index_reindex", "csa2_sparse_attn_decode",
@@ -217,6 +235,57 @@ def csa2_attn_combine(o_parts, lse_parts, n_parts: int, rows: int, out, lse_out,
     st = L.csa2_attn_combine(_ptr(o_parts), _ptr(lse_parts), n_parts, rows, _ptr(out),
                              _ptr(lse_out), _stream(stream))
     _check("csa2_attn_combine", st)
+
+
+def csa2_quantize_append_paged(kv: CSA2PagedKV | None, kv_bf16, idxk_bf16, T_kv: int, kv_start,
+                               swa: CSA2SWA | None, swa_bf16, T_swa: int, swa_start, rope=None,
+                               dev_err=None, stream=None):
+    """csa2_quantize_append(_rope) on a paged cache."""
+    L = load_library()
+    st = L.csa2_quantize_append_paged(C.byref(kv) if kv is not None else None, _ptr(kv_bf16),
+                                      _ptr(idxk_bf16), T_kv, _ptr(kv_start),
+                                      C.byref(swa) if swa is not None else None, _ptr(swa_bf16),
+                                      T_swa, _ptr(swa_start),
+                                      C.byref(rope) if rope is not None else None, _ptr(dev_err),
+                                      _stream(stream))
+    _check("csa2_quantize_append_paged", st)
+
+
+def csa2_index_full_paged(kv: CSA2PagedKV, q_idx, w, q_pos, Tq: int, H_I: int, n_max: int,
+                          pool_blocks: int, top_k: int, pool_out, topk_out, topk_count, workspace,
+                          dev_err=None, stream=None):
+    """csa2_index_full on a paged cache."""
+    L = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = L.csa2_index_full_paged(C.byref(kv), _ptr(q_idx), _ptr(w), _ptr(q_pos), Tq, H_I, n_max,
+                                 pool_blocks, top_k, _ptr(pool_out), _ptr(topk_out),
+                                 _ptr(topk_count), _ptr(workspace), ws_bytes, _ptr(dev_err),
+                                 _stream(stream))
+    _check("csa2_index_full_paged", st)
+
+
+def csa2_index_reindex_paged(kv: CSA2PagedKV, q_idx, w, q_pos, Tq: int, H_I: int, pool,
+                             pool_blocks: int, top_k: int, topk_out, topk_count, dev_err=None,
+                             stream=None):
+    """csa2_index_reindex on a paged cache."""
+    L = load_library()
+    st = L.csa2_index_reindex_paged(C.byref(kv), _ptr(q_idx), _ptr(w), _ptr(q_pos), Tq, H_I,
+                                    _ptr(pool), pool_blocks, top_k, _ptr(topk_out),
+                                    _ptr(topk_count), _ptr(dev_err), _stream(stream))
+    _check("csa2_index_reindex_paged", st)
+
+
+def csa2_sparse_attn_decode_paged(kv: CSA2PagedKV, swa: CSA2SWA | None, swa_bf16, q, q_pos,
+                                  Tq: int, H: int, topk, top_k: int, swa_len: int,
+                                  softmax_scale: float, rope, out, lse, dev_err=None, stream=None):
+    """csa2_sparse_attn_decode (swa_bf16 None) or its fused-append form on a paged cache."""
+    L = load_library()
+    st = L.csa2_sparse_attn_decode_paged(C.byref(kv), C.byref(swa) if swa is not None else None,
+                                         _ptr(swa_bf16), _ptr(q), _ptr(q_pos), Tq, H, _ptr(topk),
+                                         top_k, swa_len, softmax_scale,
+                                         C.byref(rope) if rope is not None else None, _ptr(out),
+                                         _ptr(lse), _ptr(dev_err), _stream(stream))
+    _check("csa2_sparse_attn_decode_paged", st)
 
 
 def csa2_index_reindex(kv: CSA2GlobalKV, q_idx, w, q_pos, Tq: int, H_I: int, pool,

@@ -58,7 +58,42 @@ FullLayout full_layout(int64_t BT, int64_t n_max, int32_t pool_blocks) {
     return L;
 }
 
-csa2_status check_kv(const csa2_global_kv *kv, bool need_index) {
+// A global-KV group as the kernels see it: the planes, the logical shape and the page
+// map (contiguous for csa2_global_kv, a block table for csa2_paged_kv).
+struct KvView {
+    uint8_t *codes, *scales, *idx_codes;
+    float *idx_scale;
+    int32_t batch, cap, d_idx, ratio;
+    PageMap pm;
+};
+
+const KvView *view_of(const csa2_global_kv *kv, KvView *v) {
+    if (!kv) return nullptr;
+    *v = KvView{kv->codes, kv->scales, kv->idx_codes, kv->idx_scale, kv->batch, kv->cap, kv->d_idx,
+                kv->ratio, PageMap{nullptr, 0, 0, 0}};
+    return v;
+}
+
+// Paged view: pages of page_size entries (a power of two >= 256, so that scan tiles, pool
+// blocks and 64-position blocks never straddle a page), block table [batch][max_pages].
+csa2_status paged_view(const csa2_paged_kv *kv, KvView *v, const KvView **out) {
+    *out = nullptr;
+    if (!kv) return CSA2_OK;
+    if (!kv->block_table || !aligned(kv->block_table, 4)) return CSA2_ERR_INVALID_ARG;
+    if (kv->page_size < 256 || kv->page_size > (1 << 20) || (kv->page_size & (kv->page_size - 1)))
+        return CSA2_ERR_UNSUPPORTED;
+    if (kv->max_pages < 1 || kv->n_pages < 1 || kv->batch < 1) return CSA2_ERR_INVALID_ARG;
+    const int64_t cap = (int64_t)kv->max_pages * kv->page_size;
+    if (cap > INT32_MAX || (int64_t)kv->n_pages * kv->page_size > ((int64_t)1 << 40)) return CSA2_ERR_UNSUPPORTED;
+    int shift = 0;
+    while ((1 << shift) < kv->page_size) ++shift;
+    *v = KvView{kv->codes, kv->scales, kv->idx_codes, kv->idx_scale, kv->batch, (int32_t)cap, kv->d_idx,
+                kv->ratio, PageMap{kv->block_table, shift, kv->max_pages, kv->n_pages}};
+    *out = v;
+    return CSA2_OK;
+}
+
+csa2_status check_kv(const KvView *kv, bool need_index) {
     if (!kv || !kv->codes || !kv->scales) return CSA2_ERR_INVALID_ARG;
     if (kv->batch <= 0 || kv->cap <= 0 || kv->ratio < 1 || kv->ratio > 64) return CSA2_ERR_INVALID_ARG;
     if (!aligned(kv->codes, 16) || !aligned(kv->scales, 16)) return CSA2_ERR_INVALID_ARG;
@@ -86,7 +121,7 @@ bool hi_supported(int32_t H_I) {
 
 extern "C" {
 
-int32_t csa2_abi_version(void) { return 103; }
+int32_t csa2_abi_version(void) { return 104; }
 
 void csa2_debug_set_waits(uint64_t limit_ns, int32_t stuck_wait) {
     g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
@@ -139,7 +174,7 @@ static csa2_status rope_args(const csa2_rope *rope, RopeArgs *out) {
     return CSA2_OK;
 }
 
-static csa2_status quantize_append(const csa2_global_kv *kv, const void *kv_bf16,
+static csa2_status quantize_append(const KvView *kv, const void *kv_bf16,
                                    const void *idxk_bf16, int32_t T_kv, const int32_t *kv_start,
                                    const csa2_swa *swa, const void *swa_bf16, int32_t T_swa,
                                    const int32_t *swa_start, const csa2_rope *rope,
@@ -166,6 +201,7 @@ static csa2_status quantize_append(const csa2_global_kv *kv, const void *kv_bf16
         a.cap = kv->cap;
         a.d_idx = kv->d_idx;
         a.ratio = kv->ratio;
+        a.pm = kv->pm;
         a.kv_bf16 = (const uint16_t *)kv_bf16;
         a.idxk_bf16 = (const uint16_t *)idxk_bf16;
         a.T_kv = T_kv;
@@ -196,8 +232,9 @@ csa2_status csa2_quantize_append(const csa2_global_kv *kv, const void *kv_bf16,
                                  const csa2_swa *swa, const void *swa_bf16, int32_t T_swa,
                                  const int32_t *swa_start, int32_t *dev_err,
                                  csa2_stream_t stream) {
-    return quantize_append(kv, kv_bf16, idxk_bf16, T_kv, kv_start, swa, swa_bf16, T_swa, swa_start,
-                           nullptr, dev_err, stream);
+    KvView v;
+    return quantize_append(view_of(kv, &v), kv_bf16, idxk_bf16, T_kv, kv_start, swa, swa_bf16, T_swa,
+                           swa_start, nullptr, dev_err, stream);
 }
 
 csa2_status csa2_quantize_append_rope(const csa2_global_kv *kv, const void *kv_bf16,
@@ -206,12 +243,13 @@ csa2_status csa2_quantize_append_rope(const csa2_global_kv *kv, const void *kv_b
                                       const void *swa_bf16, int32_t T_swa,
                                       const int32_t *swa_start, const csa2_rope *rope,
                                       int32_t *dev_err, csa2_stream_t stream) {
-    return quantize_append(kv, kv_bf16, idxk_bf16, T_kv, kv_start, swa, swa_bf16, T_swa, swa_start,
-                           rope, dev_err, stream);
+    KvView v;
+    return quantize_append(view_of(kv, &v), kv_bf16, idxk_bf16, T_kv, kv_start, swa, swa_bf16, T_swa,
+                           swa_start, rope, dev_err, stream);
 }
 
 // Full layer: scan (exact CUDA-core order, or tensor cores) then pool / Top-K.
-static csa2_status index_full(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
+static csa2_status index_full(const KvView *kv, const void *q_idx_bf16, const float *w,
                               const int32_t *q_pos, int32_t Tq, int32_t H_I, int32_t n_max,
                               int32_t pool_blocks, int32_t top_k, int32_t *pool_out,
                               int32_t *topk_out, int32_t *topk_count, void *workspace,
@@ -263,6 +301,7 @@ static csa2_status index_full(const csa2_global_kv *kv, const void *q_idx_bf16, 
     a.dev_err = dev_err;
     a.wait = current_wait_cfg();
     a.entry_lo = entry_lo;
+    a.pm = kv->pm;
     a.pool_keys_out = pool_keys_out;
     a.topk_keys_out = topk_keys_out;
     cudaStream_t s = (cudaStream_t)stream;
@@ -276,7 +315,8 @@ csa2_status csa2_index_full(const csa2_global_kv *kv, const void *q_idx_bf16, co
                             int32_t pool_blocks, int32_t top_k, int32_t *pool_out,
                             int32_t *topk_out, int32_t *topk_count, void *workspace,
                             size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
-    return index_full(kv, q_idx_bf16, w, q_pos, Tq, H_I, n_max, pool_blocks, top_k, pool_out,
+    KvView v;
+    return index_full(view_of(kv, &v), q_idx_bf16, w, q_pos, Tq, H_I, n_max, pool_blocks, top_k, pool_out,
                       topk_out, topk_count, workspace, ws_bytes, dev_err, stream, false);
 }
 
@@ -285,7 +325,8 @@ csa2_status csa2_index_full_tc(const csa2_global_kv *kv, const void *q_idx_bf16,
                                int32_t pool_blocks, int32_t top_k, int32_t *pool_out,
                                int32_t *topk_out, int32_t *topk_count, void *workspace,
                                size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
-    return index_full(kv, q_idx_bf16, w, q_pos, Tq, H_I, n_max, pool_blocks, top_k, pool_out,
+    KvView v;
+    return index_full(view_of(kv, &v), q_idx_bf16, w, q_pos, Tq, H_I, n_max, pool_blocks, top_k, pool_out,
                       topk_out, topk_count, workspace, ws_bytes, dev_err, stream, true);
 }
 
@@ -299,8 +340,9 @@ csa2_status csa2_index_full_slice(const csa2_global_kv *kv, int64_t entry_lo,
     if (pool_blocks > 0 && !pool_keys_out) return CSA2_ERR_INVALID_ARG;
     if (!aligned(topk_keys_out, 8) || (pool_keys_out && !aligned(pool_keys_out, 8))) return CSA2_ERR_INVALID_ARG;
     if (kv && entry_lo / 8 + (int64_t)kv->cap / 8 + 1 > INT32_MAX / 2) return CSA2_ERR_UNSUPPORTED;
-    return index_full(kv, q_idx_bf16, w, q_pos, Tq, H_I, n_max, pool_blocks, top_k, nullptr, nullptr,
-                      nullptr, workspace, ws_bytes, dev_err, stream, false, entry_lo,
+    KvView v;
+    return index_full(view_of(kv, &v), q_idx_bf16, w, q_pos, Tq, H_I, n_max, pool_blocks, top_k, nullptr,
+                      nullptr, nullptr, workspace, ws_bytes, dev_err, stream, false, entry_lo,
                       pool_blocks > 0 ? pool_keys_out : nullptr, topk_keys_out);
 }
 
@@ -324,11 +366,11 @@ csa2_status csa2_attn_combine(const float *o_parts, const float *lse_parts, int3
                                         (cudaStream_t)stream));
 }
 
-csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
-                               const int32_t *q_pos, int32_t Tq, int32_t H_I,
-                               const int32_t *pool, int32_t pool_blocks, int32_t top_k,
-                               int32_t *topk_out, int32_t *topk_count, void *workspace,
-                               size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
+static csa2_status index_reindex(const KvView *kv, const void *q_idx_bf16, const float *w,
+                                 const int32_t *q_pos, int32_t Tq, int32_t H_I,
+                                 const int32_t *pool, int32_t pool_blocks, int32_t top_k,
+                                 int32_t *topk_out, int32_t *topk_count, void *workspace,
+                                 size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
     csa2_status st = check_kv(kv, true);
     if (st != CSA2_OK) return st;
     if (!q_idx_bf16 || !w || !q_pos || !pool || !topk_out || !topk_count) return CSA2_ERR_INVALID_ARG;
@@ -361,11 +403,22 @@ csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16,
     a.topk_count = topk_count;
     a.dev_err = dev_err;
     a.wait = current_wait_cfg();
+    a.pm = kv->pm;
     cudaStream_t s = (cudaStream_t)stream;
     return launched(launch_reindex_fused(a, (int)BT, s));
 }
 
-static csa2_status sparse_attn(const csa2_global_kv *kv, const csa2_swa *swa, const void *swa_new_bf16,
+csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
+                               const int32_t *q_pos, int32_t Tq, int32_t H_I,
+                               const int32_t *pool, int32_t pool_blocks, int32_t top_k,
+                               int32_t *topk_out, int32_t *topk_count, void *workspace,
+                               size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
+    KvView v;
+    return index_reindex(view_of(kv, &v), q_idx_bf16, w, q_pos, Tq, H_I, pool, pool_blocks, top_k,
+                         topk_out, topk_count, workspace, ws_bytes, dev_err, stream);
+}
+
+static csa2_status sparse_attn(const KvView *kv, const csa2_swa *swa, const void *swa_new_bf16,
                                const void *q_bf16, const int32_t *q_pos, int32_t Tq, int32_t H,
                                const int32_t *topk, int32_t top_k, int32_t swa_len,
                                float softmax_scale, const csa2_rope *rope, float *out,
@@ -392,6 +445,7 @@ static csa2_status sparse_attn(const csa2_global_kv *kv, const csa2_swa *swa, co
     a.scales = kv->scales;
     a.cap = kv->cap;
     a.ratio = kv->ratio;
+    a.pm = kv->pm;
     if (swa_len > 0) {
         a.swa_codes = swa->codes;
         a.swa_scale = swa->scale;
@@ -425,8 +479,9 @@ csa2_status csa2_sparse_attn_decode(const csa2_global_kv *kv, const csa2_swa *sw
                                     int32_t *dev_err, csa2_stream_t stream) {
     (void)workspace;
     (void)ws_bytes;
-    return sparse_attn(kv, swa, nullptr, q_bf16, q_pos, Tq, H, topk, top_k, swa_len, softmax_scale,
-                       nullptr, out, lse, dev_err, stream);
+    KvView v;
+    return sparse_attn(view_of(kv, &v), swa, nullptr, q_bf16, q_pos, Tq, H, topk, top_k, swa_len,
+                       softmax_scale, nullptr, out, lse, dev_err, stream);
 }
 
 csa2_status csa2_sparse_attn_decode_append(const csa2_global_kv *kv, const csa2_swa *swa,
@@ -451,7 +506,68 @@ csa2_status csa2_sparse_attn_decode_append_rope(
     if (Tq != 1) return CSA2_ERR_UNSUPPORTED;
     if (swa_len <= 0 || !swa || !swa_bf16) return CSA2_ERR_INVALID_ARG;
     if (!aligned(swa_bf16, 16)) return CSA2_ERR_INVALID_ARG;
-    return sparse_attn(kv, swa, swa_bf16, q_bf16, q_pos, Tq, H, topk, top_k, swa_len, softmax_scale,
+    KvView v;
+    return sparse_attn(view_of(kv, &v), swa, swa_bf16, q_bf16, q_pos, Tq, H, topk, top_k, swa_len,
+                       softmax_scale, rope, out, lse, dev_err, stream);
+}
+
+// ---- paged cache: the same calls over a csa2_paged_kv ----------------------------------
+csa2_status csa2_quantize_append_paged(const csa2_paged_kv *kv, const void *kv_bf16,
+                                       const void *idxk_bf16, int32_t T_kv, const int32_t *kv_start,
+                                       const csa2_swa *swa, const void *swa_bf16, int32_t T_swa,
+                                       const int32_t *swa_start, const csa2_rope *rope,
+                                       int32_t *dev_err, csa2_stream_t stream) {
+    KvView v;
+    const KvView *pv;
+    csa2_status st = paged_view(kv, &v, &pv);
+    if (st != CSA2_OK) return st;
+    return quantize_append(pv, kv_bf16, idxk_bf16, T_kv, kv_start, swa, swa_bf16, T_swa, swa_start,
+                           rope, dev_err, stream);
+}
+
+csa2_status csa2_index_full_paged(const csa2_paged_kv *kv, const void *q_idx_bf16, const float *w,
+                                  const int32_t *q_pos, int32_t Tq, int32_t H_I, int32_t n_max,
+                                  int32_t pool_blocks, int32_t top_k, int32_t *pool_out,
+                                  int32_t *topk_out, int32_t *topk_count, void *workspace,
+                                  size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
+    KvView v;
+    const KvView *pv;
+    csa2_status st = paged_view(kv, &v, &pv);
+    if (st != CSA2_OK) return st;
+    return index_full(pv, q_idx_bf16, w, q_pos, Tq, H_I, n_max, pool_blocks, top_k, pool_out, topk_out,
+                      topk_count, workspace, ws_bytes, dev_err, stream, false);
+}
+
+csa2_status csa2_index_reindex_paged(const csa2_paged_kv *kv, const void *q_idx_bf16, const float *w,
+                                     const int32_t *q_pos, int32_t Tq, int32_t H_I, const int32_t *pool,
+                                     int32_t pool_blocks, int32_t top_k, int32_t *topk_out,
+                                     int32_t *topk_count, int32_t *dev_err, csa2_stream_t stream) {
+    KvView v;
+    const KvView *pv;
+    csa2_status st = paged_view(kv, &v, &pv);
+    if (st != CSA2_OK) return st;
+    return index_reindex(pv, q_idx_bf16, w, q_pos, Tq, H_I, pool, pool_blocks, top_k, topk_out,
+                         topk_count, nullptr, 0, dev_err, stream);
+}
+
+csa2_status csa2_sparse_attn_decode_paged(const csa2_paged_kv *kv, const csa2_swa *swa,
+                                          const void *swa_bf16, const void *q_bf16,
+                                          const int32_t *q_pos, int32_t Tq, int32_t H,
+                                          const int32_t *topk, int32_t top_k, int32_t swa_len,
+                                          float softmax_scale, const csa2_rope *rope, float *out,
+                                          float *lse, int32_t *dev_err, csa2_stream_t stream) {
+    KvView v;
+    const KvView *pv;
+    csa2_status st = paged_view(kv, &v, &pv);
+    if (st != CSA2_OK) return st;
+    if (swa_bf16) {
+        if (Tq != 1) return CSA2_ERR_UNSUPPORTED;
+        if (swa_len <= 0 || !swa) return CSA2_ERR_INVALID_ARG;
+        if (!aligned(swa_bf16, 16)) return CSA2_ERR_INVALID_ARG;
+    } else if (rope) {
+        return CSA2_ERR_INVALID_ARG;
+    }
+    return sparse_attn(pv, swa, swa_bf16, q_bf16, q_pos, Tq, H, topk, top_k, swa_len, softmax_scale,
                        rope, out, lse, dev_err, stream);
 }
 

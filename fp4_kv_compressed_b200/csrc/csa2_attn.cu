@@ -280,7 +280,7 @@ struct KeyMap {      // this CTA's keys and where each comes from
     int64_t w0;      // first window position
     int n_keys;      // keys of the query (selection + window)
     int k_end;       // end of this CTA's key range
-    int64_t slot_base;
+    int64_t b;
     int64_t ring_base;
     const uint8_t *new_row;   // fused append: the newest window key is this row (smem)
     float new_sigma;
@@ -291,7 +291,7 @@ __device__ __forceinline__ void load_stage(Raw &r, const AttnArgs &a, const KeyM
     r.kind = zrow ? 0 : -1;
     if (kg < km.k_end) {
         if (kg < km.n_sel) {
-            const int64_t off = km.slot_base + km.ids[kg];
+            const int64_t off = cache_row(a.pm, a.cap, km.b, km.ids[kg]);   // checked when compacted
             const uint4 *src = reinterpret_cast<const uint4 *>(a.codes + off * kCodeBytes + 64 * j);
 #pragma unroll
             for (int u = 0; u < 4; ++u) r.c[u] = __ldg(src + u);
@@ -443,8 +443,12 @@ attn_kernel(AttnArgs a) {
     const int64_t w0 = max64(0, t - a.swa_len + 1);
     const int n_win = a.swa_len > 0 ? (int)(t - w0 + 1) : 0;
     const int64_t n_vis = min64(visible_entries((int32_t)t, a.ratio), a.cap);
-    const bool e_ok = e_id >= 0 && e_id < n_vis;
+    bool e_ok = e_id >= 0 && e_id < n_vis;
     if (e_id >= 0 && !e_ok) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
+    if (e_ok && a.pm.table != nullptr && cache_row(a.pm, a.cap, b, e_id) < 0) {
+        set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
+        e_ok = false;
+    }
     const uint32_t bal = __ballot_sync(0xFFFFFFFFu, e_ok);
     float qm = 0.0f;
 #pragma unroll
@@ -582,10 +586,9 @@ attn_kernel(AttnArgs a) {
         }
     } else if (warp == 2) {
         // ---------------- L2 prefetch of every row this CTA gathers ----------------
-        const int64_t slot_base = (int64_t)b * a.cap;
         for (int kg = k0 + lane; kg < k1; kg += 32) {
             if (kg < n_sel) {
-                const int64_t off = slot_base + s.ids[kg];
+                const int64_t off = cache_row(a.pm, a.cap, b, s.ids[kg]);
                 prefetch_l2(a.codes + off * kCodeBytes, kCodeBytes);
                 prefetch_l2(a.scales + off * kScaleBytes, kScaleBytes);
             } else if (!(fuse && kg == n_keys - 1)) {
@@ -722,7 +725,7 @@ attn_kernel(AttnArgs a) {
         km.w0 = w0;
         km.n_keys = n_keys;
         km.k_end = k1;
-        km.slot_base = (int64_t)b * a.cap;
+        km.b = b;
         km.ring_base = (int64_t)b * a.wcap;
         km.new_row = fuse && rank == owner ? s.swa_new : nullptr;
         km.new_sigma = fuse && rank == owner ? s.swa_new_sigma : 0.0f;

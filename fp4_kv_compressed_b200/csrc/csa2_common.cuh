@@ -210,6 +210,16 @@ __device__ __forceinline__ void set_dev_err(int32_t *dev_err, int bit) {
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 
+// Row of entry e of request b in the cache planes (see PageMap): -1 when the block
+// table names a page outside [0, n_pages) (the caller skips the entry and flags it).
+template <class PM>
+__device__ __forceinline__ int64_t cache_row(const PM &pm, int64_t cap, int64_t b, int64_t e) {
+    if (pm.table == nullptr) return b * cap + e;
+    const int32_t pg = __ldg(pm.table + b * pm.max_pages + (e >> pm.shift));
+    if (pg < 0 || pg >= pm.n_pages) return -1;
+    return ((int64_t)pg << pm.shift) | (e & (((int64_t)1 << pm.shift) - 1));
+}
+
 __device__ __forceinline__ int64_t visible_entries(int32_t t, int32_t ratio) {
     return t < 0 ? 0 : ((int64_t)t + 1) / ratio;
 }

@@ -164,7 +164,13 @@ index_scan_kernel(IndexArgs a) {
     if (p0 >= N) return;
     const int rows = (int)min64(kTileRows, N - p0);
 
-    const uint8_t *src = a.idx_codes + ((int64_t)b * a.cap + p0) * D;
+    // the tile's rows are consecutive cache rows (a page holds whole tiles)
+    const int64_t row0 = cache_row(a.pm, a.cap, b, p0);
+    if (row0 < 0) {
+        if (threadIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
+        return;
+    }
+    const uint8_t *src = a.idx_codes + row0 * D;
     constexpr int U = D / 16;
     for (int e = threadIdx.x; e < rows * U; e += kScoreThreads) {
         int r = e / U, u = e % U;
@@ -173,12 +179,12 @@ index_scan_kernel(IndexArgs a) {
     cp_async_commit();
     load_query<D, HI>(s, a.q_idx + (int64_t)qi * HI * D, a.w + (int64_t)qi * HI);
     // the rows' scales, fetched while the tile is in flight
-    const float *sig = a.idx_scale + (int64_t)b * a.cap;
+    const float *sig = a.idx_scale + row0;
     float sgv[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
         const int row = threadIdx.x + kScoreThreads * r;
-        sgv[r] = __ldg(sig + p0 + min(row, rows - 1));   // branch-free: all R loads in flight
+        sgv[r] = __ldg(sig + min(row, rows - 1));   // branch-free: all R loads in flight
     }
     cp_async_wait_all();
     __syncthreads();
@@ -684,6 +690,7 @@ struct RfSmem {
     float2 q[D / 2][HI];
     float w[HI];
     int32_t pool[kRfMaxCand / 8];
+    int64_t prow[kRfMaxCand / 8];                        // first cache row of each pool block
     // selection state (block_topk)
     uint32_t hist[1 << kSelDigit];
     int wa[kSelWarps], wb[kSelWarps];
@@ -738,6 +745,13 @@ reindex_fused_kernel(IndexArgs a, int C) {
         if (blk >= 0 && (int64_t)blk * 8 >= N) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
         if (i > 0 && blk >= 0 && __ldg(pool + i - 1) >= blk) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
         s.pool[i] = blk >= 0 && (int64_t)blk * 8 < N ? blk : -1;
+        // the block's first cache row (a page holds whole blocks); -1: not scored
+        int64_t row = -1;
+        if (s.pool[i] >= 0) {
+            row = cache_row(a.pm, a.cap, b, (int64_t)s.pool[i] * 8);
+            if (row < 0) set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
+        }
+        s.prow[i] = row;
     }
     if (threadIdx.x < kSelThreads / 2) {
         // q and w of the query (the scoring core's layout)
@@ -756,27 +770,26 @@ reindex_fused_kernel(IndexArgs a, int C) {
     const int n_stages = (ncand + SR - 1) / SR;
     if (threadIdx.x < kRfScoreThreads) {
         const int t = threadIdx.x;
-        const uint8_t *codes = a.idx_codes + (int64_t)b * a.cap * D;
-        const float *sigb = a.idx_scale + (int64_t)b * a.cap;
         auto issue = [&](int st) {
             const int buf = st & 1;
             constexpr int U = D / 16;
             for (int e = t; e < SR * U; e += kRfScoreThreads) {
                 const int r = e / U, u = e % U, c = st * SR + r;
                 if (c < ncand) {
-                    const int blk = s.pool[c >> 3];
+                    const int blk = s.prow[c >> 3] >= 0 ? s.pool[c >> 3] : -1;
                     const int64_t p = (int64_t)blk * 8 + (c & 7);
                     if (blk >= 0 && p < N)
-                        cp_async16(s.rows[buf] + r * D + 16 * swz<D>(r, u), codes + p * D + 16 * u);
+                        cp_async16(s.rows[buf] + r * D + 16 * swz<D>(r, u),
+                                   a.idx_codes + (s.prow[c >> 3] + (c & 7)) * D + 16 * u);
                 }
             }
             // the entries' scales (4 bytes each; visible positions only)
             for (int r = t; r < SR; r += kRfScoreThreads) {
                 const int c = st * SR + r;
                 if (c < ncand) {
-                    const int blk = s.pool[c >> 3];
+                    const int blk = s.prow[c >> 3] >= 0 ? s.pool[c >> 3] : -1;
                     const int64_t p = (int64_t)blk * 8 + (c & 7);
-                    if (blk >= 0 && p < N) cp_async4(&s.sig[buf][r], sigb + p);
+                    if (blk >= 0 && p < N) cp_async4(&s.sig[buf][r], a.idx_scale + s.prow[c >> 3] + (c & 7));
                 }
             }
             cp_async_commit();
@@ -796,7 +809,7 @@ reindex_fused_kernel(IndexArgs a, int C) {
             for (int r = 0; r < R; ++r) {
                 const int row = t + kRfScoreThreads * r, c = st * SR + row;
                 if (c < ncand) {
-                    const int blk = s.pool[c >> 3];
+                    const int blk = s.prow[c >> 3] >= 0 ? s.pool[c >> 3] : -1;
                     const int64_t p = (int64_t)blk * 8 + (c & 7);
                     s.keys[c] = (blk >= 0 && p < N) ? score_key(__fmul_rn(sc[r], s.sig[buf][row])) : 0u;
                 }

@@ -285,10 +285,17 @@ __global__ void __launch_bounds__(kThreads, 1) index_scan_tc_kernel(IndexArgs a,
         }
         // tile (by, it % n_tiles): convert into buffer n_issued & 1, issue its MMAs
         const int64_t e0 = (it % n_tiles) * kM;
-        const uint8_t *codes = a.idx_codes + ((int64_t)b * a.cap + e0) * D;
+        // the tile's entries are consecutive cache rows (a page holds whole tiles); a
+        // bad page reads the request's first page instead and flags it (scores invalid)
+        int64_t row0 = cache_row(a.pm, a.cap, b, e0);
+        if (row0 < 0) {
+            if (threadIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
+            row0 = 0;
+        }
+        const uint8_t *codes = a.idx_codes + row0 * D;
         const uint32_t buf = n_issued & 1u;
         const int64_t my_e = e0 + my_ent;
-        const float sig = my_e < a.cap ? __ldg(a.idx_scale + (int64_t)b * a.cap + my_e) : 0.0f;
+        const float sig = my_e < a.cap ? __ldg(a.idx_scale + row0 + my_ent) : 0.0f;
         constexpr int kUnits = kM * (D / 16) / kThreads;   // 16-code units per thread
         uint4 cu[kUnits];
 #pragma unroll

@@ -8,6 +8,16 @@
 
 namespace csa2 {
 
+// Paged cache: entry e of request b lives in row table[b][e >> shift] << shift |
+// (e & (2^shift - 1)) of the planes (pages of 2^shift entries); table == nullptr is the
+// contiguous layout, row b * cap + e.
+struct PageMap {
+    const int32_t *table;     // [batch][max_pages] page ids, or null
+    int32_t shift;
+    int32_t max_pages;
+    int32_t n_pages;
+};
+
 // Bounded waits.  Every spin of a kernel on an mbarrier gives up after `limit_ns` of
 // wall time (%globaltimer); the kernel then flags CSA2_DEVERR_TIMEOUT, waits (bounded
 // by kDrainLimitNs) for the tensor-core work and copies it has in flight, frees its
@@ -54,6 +64,7 @@ struct QuantArgs {
     // work split: warps of each kind
     int64_t n_main, n_idx, n_swa;
     int32_t *dev_err;
+    PageMap pm;
 };
 
 struct IndexArgs {
@@ -88,6 +99,7 @@ struct IndexArgs {
     int64_t entry_lo;
     uint64_t *pool_keys_out;   // [BT][pool_blocks] or null
     uint64_t *topk_keys_out;   // [BT][top_k] or null
+    PageMap pm;
 };
 
 struct AttnArgs {
@@ -112,6 +124,7 @@ struct AttnArgs {
     float *lse;
     int32_t *dev_err;
     WaitCfg wait;
+    PageMap pm;
 };
 
 // Every kernel of the library asks for the largest shared-memory carveout, so that

@@ -49,7 +49,11 @@ __device__ void quant_fp4_entry(const QuantArgs &a, int64_t row, int lane) {
         codes.x = cvt_e2m1x8(r);
         codes.y = cvt_e2m1x8(r + 8);
     }
-    const int64_t e = (int64_t)b * a.cap + slot;
+    const int64_t e = cache_row(a.pm, a.cap, b, slot);
+    if (e < 0) {
+        if (lane == 0) set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
+        return;
+    }
     reinterpret_cast<uint2 *>(a.codes + e * kCodeBytes)[lane] = codes;
     a.scales[e * kScaleBytes + lane] = (uint8_t)s8;
 }
@@ -71,7 +75,11 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(QuantArgs a) {
             if (lane == 0) set_dev_err(a.dev_err, CSA2_DEVERR_SLOT);
             return;
         }
-        const int64_t e = (int64_t)b * a.cap + slot;
+        const int64_t e = cache_row(a.pm, a.cap, b, slot);
+        if (e < 0) {
+            if (lane == 0) set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
+            return;
+        }
         const uint16_t *src = a.idxk_bf16 + warp * a.d_idx;
         if (a.d_idx == 128)
             quant_fp8_row<128>(src, a.idx_codes + e * 128, a.idx_scale + e, lane);

@@ -82,6 +82,33 @@ class GlobalKV:
                    (self.codes, self.scales, self.idx_codes, self.idx_scale))
 
 
+class PagedKV:
+    """Device planes of one global-KV group in pages (serving layout): a pool of n_pages
+    pages of page_size entries and a block table [B][max_pages] of page ids."""
+
+    def __init__(self, B: int, max_pages: int, page_size: int, n_pages: int, d_idx: int,
+                 ratio: int, block_table: torch.Tensor, device):
+        if block_table.shape != (B, max_pages) or block_table.dtype != torch.int32:
+            raise ValueError("block_table must be int32 [B][max_pages]")
+        self.B, self.max_pages, self.page_size, self.n_pages = B, max_pages, page_size, n_pages
+        self.d_idx, self.ratio = d_idx, ratio
+        rows = n_pages * page_size
+        self.codes = torch.zeros(rows, KV_DIM // 2, dtype=torch.uint8, device=device)
+        self.scales = torch.zeros(rows, KV_DIM // 16, dtype=torch.uint8, device=device)
+        self.idx_codes = torch.zeros(rows, d_idx, dtype=torch.uint8, device=device)
+        self.idx_scale = torch.zeros(rows, dtype=torch.float32, device=device)
+        self.block_table = block_table.to(device).contiguous()
+        self.struct = bind.CSA2PagedKV(self.codes.data_ptr(), self.scales.data_ptr(),
+                                       self.idx_codes.data_ptr(), self.idx_scale.data_ptr(),
+                                       self.block_table.data_ptr(), B, max_pages, page_size,
+                                       n_pages, d_idx, ratio)
+
+    def rows_of(self, b: int, n: int) -> torch.Tensor:
+        """Pool rows of entries 0..n-1 of request b."""
+        e = torch.arange(n, device=self.block_table.device)
+        return self.block_table[b][e // self.page_size].long() * self.page_size + e % self.page_size
+
+
 class SwaRing:
     """One layer's FP8 SWA window ring: token p lives in slot p % window_cap."""
 

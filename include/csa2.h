@@ -71,6 +71,7 @@ typedef enum csa2_status {
 #define CSA2_DEVERR_TIMEOUT 0x10  /* a kernel's bounded wait gave up (internal error, or
                                      the csa2_debug_set_waits test hook) */
 #define CSA2_DEVERR_ROPE 0x20     /* a row's position lies outside the RoPE table */
+#define CSA2_DEVERR_PAGE 0x40     /* a block table entry names a page outside the pool */
 
 /* Limits of the kernels. */
 #define CSA2_KV_DIM 512           /* shared K=V latent width (MQA) */
@@ -397,6 +398,73 @@ CSA2_API csa2_status csa2_sparse_attn_decode_append_rope(
     const int32_t *q_pos, int32_t Tq, int32_t H, const int32_t *topk, int32_t top_k,
     int32_t swa_len, float softmax_scale, const csa2_rope *rope, float *out, float *lse,
     void *workspace, size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream);
+
+/*
+ * Paged global KV (serving: requests of different lengths share one pool of pages;
+ * the pages' cache is the one global KV of study notes section 5 / myzaker "cache
+ * precision and tiering", here laid out in fixed-size pages).  The planes hold
+ * n_pages pages of page_size entries each, in the same per-entry formats as
+ * csa2_global_kv:
+ *   codes [n_pages * page_size][256], scales [n_pages * page_size][32],
+ *   idx_codes [n_pages * page_size][d_idx], idx_scale [n_pages * page_size];
+ * entry e of request b lives in row
+ *   block_table[b][e / page_size] * page_size + e % page_size
+ * (block_table int32 [batch][max_pages], device).  The logical capacity of a request
+ * is max_pages * page_size entries; its length is set by its query positions, as for
+ * csa2_global_kv.  page_size is a power of two >= 256 (so that a scan tile, a pool
+ * block and a 64-position block never straddle a page; else CSA2_ERR_UNSUPPORTED).
+ * A table entry outside [0, n_pages) met by a kernel is skipped and flags
+ * CSA2_DEVERR_PAGE (results are then undefined).  The pages define no paging: this is
+ * the serving layout of the same cache.
+ */
+typedef struct csa2_paged_kv {
+    uint8_t *codes;
+    uint8_t *scales;
+    uint8_t *idx_codes;
+    float *idx_scale;
+    const int32_t *block_table;
+    int32_t batch;
+    int32_t max_pages;
+    int32_t page_size;
+    int32_t n_pages;
+    int32_t d_idx;   /* 64 or 128 */
+    int32_t ratio;   /* 1 or 2 */
+} csa2_paged_kv;
+
+/* csa2_quantize_append(_rope) on a paged cache (rope NULL = no rotation). */
+CSA2_API csa2_status csa2_quantize_append_paged(const csa2_paged_kv *kv, const void *kv_bf16,
+                                                const void *idxk_bf16, int32_t T_kv,
+                                                const int32_t *kv_start, const csa2_swa *swa,
+                                                const void *swa_bf16, int32_t T_swa,
+                                                const int32_t *swa_start, const csa2_rope *rope,
+                                                int32_t *dev_err, csa2_stream_t stream);
+
+/* csa2_index_full on a paged cache (same arguments, workspace and results). */
+CSA2_API csa2_status csa2_index_full_paged(const csa2_paged_kv *kv, const void *q_idx_bf16,
+                                           const float *w, const int32_t *q_pos, int32_t Tq,
+                                           int32_t H_I, int32_t n_max, int32_t pool_blocks,
+                                           int32_t top_k, int32_t *pool_out, int32_t *topk_out,
+                                           int32_t *topk_count, void *workspace, size_t ws_bytes,
+                                           int32_t *dev_err, csa2_stream_t stream);
+
+/* csa2_index_reindex on a paged cache (no workspace). */
+CSA2_API csa2_status csa2_index_reindex_paged(const csa2_paged_kv *kv, const void *q_idx_bf16,
+                                              const float *w, const int32_t *q_pos, int32_t Tq,
+                                              int32_t H_I, const int32_t *pool,
+                                              int32_t pool_blocks, int32_t top_k,
+                                              int32_t *topk_out, int32_t *topk_count,
+                                              int32_t *dev_err, csa2_stream_t stream);
+
+/* csa2_sparse_attn_decode on a paged cache.  swa_bf16 non-NULL = the fused decode
+ * append of csa2_sparse_attn_decode_append (Tq = 1), rope non-NULL (with swa_bf16) =
+ * its RoPE form; both NULL = the plain call. */
+CSA2_API csa2_status csa2_sparse_attn_decode_paged(const csa2_paged_kv *kv, const csa2_swa *swa,
+                                                   const void *swa_bf16, const void *q_bf16,
+                                                   const int32_t *q_pos, int32_t Tq, int32_t H,
+                                                   const int32_t *topk, int32_t top_k,
+                                                   int32_t swa_len, float softmax_scale,
+                                                   const csa2_rope *rope, float *out, float *lse,
+                                                   int32_t *dev_err, csa2_stream_t stream);
 
 /* Synchronise `stream`, read *dev_err (device int32) into *bits_out (host),
  * reset it to 0, and return CSA2_ERR_DEVICE_BOUNDS if any bit was set. */
