@@ -67,3 +67,44 @@ def test_tc_scan_wait_runs_out_then_recovers(pkg):
         assert bits2 == 0
         for a, b in zip(ref, got):
             assert torch.equal(a, b)
+
+
+def test_attention_wait_runs_out_then_recovers(pkg):
+    """The same for the sparse attention: a stuck wait in every CTA of every 2-CTA
+    cluster (after the first score MMAs were issued) must end the call with the timeout
+    bit, both CTAs still meeting at the cluster barriers of the combine, and leave the
+    tensor memory free for the next call."""
+    import math
+    B, cap, H, W = 3, 1500, 64, 128
+    kv = pkg.GlobalKV(B, cap, 128, 1, "cuda")
+    ring = pkg.SwaRing(B, W, "cuda")
+    x = torch.stack([synth.rows_normal_bf16(83, "kv", b, 0, cap, 512) for b in range(B)]).cuda()
+    sw = torch.stack([synth.rows_normal_bf16(83, "swa", b, 0, W, 512) for b in range(B)]).cuda()
+    z = torch.zeros(B, dtype=torch.int32, device="cuda")
+    pkg.csa2_quantize_append(kv.struct, x, None, cap, z, ring.struct, sw, W, z)
+    g = torch.Generator().manual_seed(84)
+    topk = torch.stack([torch.sort(torch.randperm(cap, generator=g)[:512]).values
+                        for _ in range(B)]).to(torch.int32).view(B, 1, 512).cuda()
+    q = torch.stack([synth.rows_normal_bf16(85, "q", b, 0, H, 512, stride=synth.Q_STRIDE)
+                     for b in range(B)]).view(B, 1, H, 512).cuda()
+    qp = torch.full((B, 1), cap - 1, dtype=torch.int32, device="cuda")
+
+    def run():
+        o = torch.full((B, 1, H, 512), 7.0, device="cuda")
+        l = torch.full((B, 1, H), 7.0, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        pkg.csa2_sparse_attn_decode(kv.struct, ring.struct, q, qp, 1, H, topk, 512, W,
+                                    1 / math.sqrt(512), o, l, None, err)
+        return pkg.csa2_read_device_error(err), o.cpu(), l.cpu()
+
+    bits0, o0, l0 = run()
+    assert bits0 == 0
+    pkg.csa2_debug_set_waits(LIMIT_NS, True)
+    try:
+        bits1, _, _ = run()
+    finally:
+        pkg.csa2_debug_set_waits(pkg.DEFAULT_WAIT_LIMIT_NS, False)
+    assert bits1 & pkg.DEVERR_TIMEOUT, f"device error bits {bits1:#x}: the wait did not run out"
+    for _ in range(2):
+        bits2, o2, l2 = run()
+        assert bits2 == 0 and torch.equal(o2, o0) and torch.equal(l2, l0)
