@@ -27,7 +27,8 @@
 // 16 warps, specialised:
 //   warp 0       TMEM allocation + the MMA issue loop (one elected lane issues);
 //   warp 1       fused append only: quantises the query token's new SWA row;
-//   warp 2       prefetches every row this CTA will gather into L2 (bulk prefetch);
+//   (set-up: every thread prefetches its selected entry into L2 -- the two CTAs take
+//    alternate entries -- and one thread the request's SWA ring)
 //   warps 4-11   softmax: warp w reads TMEM lane quadrant w % 4 (32 keys) and the
 //                32 heads of half (w - 4) / 4;
 //   warps 12-15  producers: thread = key of the tile; dequantise one 128-channel stage
@@ -445,9 +446,24 @@ attn_kernel(AttnArgs a) {
     const int64_t n_vis = min64(visible_entries((int32_t)t, a.ratio), a.cap);
     bool e_ok = e_id >= 0 && e_id < n_vis;
     if (e_id >= 0 && !e_ok) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
-    if (e_ok && a.pm.table != nullptr && cache_row(a.pm, a.cap, b, e_id) < 0) {
-        set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
-        e_ok = false;
+    if (e_ok) {
+        const int64_t row = cache_row(a.pm, a.cap, b, e_id);
+        if (row < 0) {
+            set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
+            e_ok = false;
+        } else if ((threadIdx.x & 1) == rank) {
+            // the two CTAs of the cluster prefetch alternate entries into L2 while the
+            // set-up goes on; the producers then gather from L2
+            prefetch_l2(a.codes + row * kCodeBytes, kCodeBytes);
+            prefetch_l2(a.scales + row * kScaleBytes, kScaleBytes);
+        }
+    }
+    if (threadIdx.x == 32 * 3 && a.swa_len > 0 && rank == 0) {
+        // the request's whole SWA ring (rows are contiguous) and its scales
+        prefetch_l2(a.swa_codes + (int64_t)b * a.wcap * kDim, (uint32_t)a.wcap * kDim);
+        const float *sg = a.swa_scale + (int64_t)b * a.wcap;   // only whole 16-byte units
+        if ((reinterpret_cast<uintptr_t>(sg) & 15) == 0 && (a.wcap & 3) == 0)
+            prefetch_l2(sg, (uint32_t)a.wcap * 4);
     }
     const uint32_t bal = __ballot_sync(0xFFFFFFFFu, e_ok);
     float qm = 0.0f;
@@ -583,18 +599,6 @@ attn_kernel(AttnArgs a) {
             __syncwarp();
             const bool drained = mbar_wait<false>(&s.drain, 0, kDrainLimitNs, s);
             (void)drained;
-        }
-    } else if (warp == 2) {
-        // ---------------- L2 prefetch of every row this CTA gathers ----------------
-        for (int kg = k0 + lane; kg < k1; kg += 32) {
-            if (kg < n_sel) {
-                const int64_t off = cache_row(a.pm, a.cap, b, s.ids[kg]);
-                prefetch_l2(a.codes + off * kCodeBytes, kCodeBytes);
-                prefetch_l2(a.scales + off * kScaleBytes, kScaleBytes);
-            } else if (!(fuse && kg == n_keys - 1)) {
-                const int64_t slot = (int64_t)b * a.wcap + (w0 + (kg - n_sel)) % a.wcap;
-                prefetch_l2(a.swa_codes + slot * kDim, kDim);
-            }
         }
     } else if (warp >= kSoftWarp0 && warp < kProdWarp0) {
         // ---------------- softmax: keys 32 qd .. (TMEM lanes), heads 32 hh .. ----------------
