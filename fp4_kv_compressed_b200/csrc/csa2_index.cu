@@ -156,6 +156,7 @@ index_scan_kernel(IndexArgs a) {
     const int qi = blockIdx.y;
     const int b = qi / a.Tq;
     int64_t N = max64(0, visible_entries(a.q_pos[qi], a.ratio) - a.entry_lo);   // of this cache
+    if (a.topk_keys_out) N = min64(N, a.cap);     // a slice: the query sees past its end
     if (N > a.n_max || N > a.cap) {
         if (threadIdx.x == 0 && blockIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_NMAX);
         N = min64(min64(N, a.n_max), a.cap);

@@ -40,12 +40,12 @@ def _layouts(pkg, lens, page, d=128, ratio=1, seed=71, spare=7):
     for b, n in enumerate(lens):
         rows = synth.rows_normal_bf16(seed, "kv", b, 0, n, 512).view(1, n, 512).cuda()
         ik = synth.rows_normal_bf16(seed, "ik", b, 0, n, d).view(1, n, d).cuda()
-        # one request at a time: the others' kv_start points past... each call appends
-        # request b's rows; the other requests get T_kv rows too, so give them all
+        # one request at a time: the call appends T_kv rows to every request, so the
+        # others start past any capacity and are skipped (CSA2_DEVERR_SLOT)
         full = torch.zeros(B, n, 512, dtype=torch.bfloat16, device=dev)
         fik = torch.zeros(B, n, d, dtype=torch.bfloat16, device=dev)
         full[b], fik[b] = rows[0], ik[0]
-        start = torch.full((B,), cap, dtype=torch.int32, device=dev)   # past the cap: skipped
+        start = torch.full((B,), 1 << 30, dtype=torch.int32, device=dev)   # past any cap: skipped
         start[b] = 0
         pkg.csa2_quantize_append(kv.struct, full, fik, n, start, None, None, 0, None, err)
         pkg.csa2_quantize_append_paged(pk.struct, full, fik, n, start, None, None, 0, None, None, err)
