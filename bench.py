@@ -54,9 +54,9 @@ def op_bytes(wl) -> dict:
             per = (N * (d + 4) + 4 * N + 4 * nb + 4 * nb + 8 * min(P, nb) * 4 + 4 * P + 4 * K + 4
                    + q)
             out[f"index_full_g{g}"] = BT * per
-            # the pool, its entries' index K and scales, the Top-K out (the scores stay
-            # on chip)
-            rp = 4 * P + 8 * P * (d + 4) + 4 * K + 4 + q
+            # the pool, its entries' index K and scales, the scores and slot maxima
+            # written, the chosen slots' scores read back, the Top-K out
+            rp = 4 * P + 8 * P * (d + 4) + 8 * P * 4 + 4 * P + 4 * P + 8 * K * 4 + 4 * K + 4 + q
             out[f"index_reindex_g{g}"] = BT * rp
         else:
             out[f"index_full_g{g}"] = BT * (N * (d + 4) + 4 * N + 4 * N + 4 * K + 4 + q)
@@ -133,7 +133,7 @@ OP_KERNELS = {
     "csa2_quantize_append_rope": "quantize_append_kernel",
     "csa2_index_full": "index_scan_kernel + select_full_kernel",
     "csa2_index_full_tc": "index_scan_tc_kernel + select_full_kernel",
-    "csa2_index_reindex": "reindex_fused_kernel",
+    "csa2_index_reindex": "reindex_score_kernel + select_reindex_kernel",
     "csa2_sparse_attn_decode": "attn_kernel",
     "csa2_sparse_attn_decode_append": "attn_kernel (with the SWA append)",
     "csa2_sparse_attn_decode_append_rope": "attn_kernel (with the RoPE + SWA append)",

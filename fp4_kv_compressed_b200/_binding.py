@@ -120,7 +120,7 @@ def load_library(path: str = LIB_PATH):
         getattr(L, fn).restype = C.c_int
     L.csa2_quantize_append_paged.argtypes = [P, P, P, i32, P, P, P, i32, P, P, P, P]
     L.csa2_index_full_paged.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, P, P, P, P, sz, P, P]
-    L.csa2_index_reindex_paged.argtypes = [P, P, P, P, i32, i32, P, i32, i32, P, P, P, P]
+    L.csa2_index_reindex_paged.argtypes = [P, P, P, P, i32, i32, P, i32, i32, P, P, P, sz, P, P]
     L.csa2_sparse_attn_decode_paged.argtypes = [P, P, P, P, P, i32, i32, P, i32, i32, C.c_float,
                                                 P, P, P, P, P]
     for fn in ("csa2_quantize_append_paged", "csa2_index_full_paged", "csa2_index_reindex_paged",
@@ -265,13 +265,15 @@ def csa2_index_full_paged(kv: CSA2PagedKV, q_idx, w, q_pos, Tq: int, H_I: int, n
 
 
 def csa2_index_reindex_paged(kv: CSA2PagedKV, q_idx, w, q_pos, Tq: int, H_I: int, pool,
-                             pool_blocks: int, top_k: int, topk_out, topk_count, dev_err=None,
-                             stream=None):
+                             pool_blocks: int, top_k: int, topk_out, topk_count, workspace,
+                             dev_err=None, stream=None):
     """csa2_index_reindex on a paged cache."""
     L = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = L.csa2_index_reindex_paged(C.byref(kv), _ptr(q_idx), _ptr(w), _ptr(q_pos), Tq, H_I,
                                     _ptr(pool), pool_blocks, top_k, _ptr(topk_out),
-                                    _ptr(topk_count), _ptr(dev_err), _stream(stream))
+                                    _ptr(topk_count), _ptr(workspace), ws_bytes, _ptr(dev_err),
+                                    _stream(stream))
     _check("csa2_index_reindex_paged", st)
 
 

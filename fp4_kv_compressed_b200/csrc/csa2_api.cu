@@ -93,6 +93,18 @@ csa2_status paged_view(const csa2_paged_kv *kv, KvView *v, const KvView **out) {
     return CSA2_OK;
 }
 
+// Workspace of csa2_index_reindex: scores [BT][8 pool_blocks] fp32, then the maximum of
+// each pool slot [BT][pool_blocks] fp32.
+struct ReindexLayout {
+    size_t bmax_off, total;
+};
+ReindexLayout reindex_layout(int64_t BT, int32_t pool_blocks) {
+    ReindexLayout L;
+    L.bmax_off = align_up((size_t)BT * pool_blocks * 8 * sizeof(float), kAlign);
+    L.total = L.bmax_off + align_up((size_t)BT * pool_blocks * sizeof(float), kAlign);
+    return L;
+}
+
 csa2_status check_kv(const KvView *kv, bool need_index) {
     if (!kv || !kv->codes || !kv->scales) return CSA2_ERR_INVALID_ARG;
     if (kv->batch <= 0 || kv->cap <= 0 || kv->ratio < 1 || kv->ratio > 64) return CSA2_ERR_INVALID_ARG;
@@ -151,7 +163,7 @@ size_t csa2_workspace_size(int32_t op, int32_t B, int32_t Tq, int32_t n_max, int
         case CSA2_OP_INDEX_FULL:
             return n_max > 0 ? full_layout(BT, n_max, pool_blocks).total : 0;
         case CSA2_OP_INDEX_REINDEX:
-            return 0;   // the scores stay in shared memory
+            return pool_blocks > 0 ? reindex_layout(BT, pool_blocks).total : 0;
         case CSA2_OP_SPARSE_ATTN:
             return 0;
         default:
@@ -381,8 +393,8 @@ static csa2_status index_reindex(const KvView *kv, const void *q_idx_bf16, const
     if (pool_blocks < 1 || pool_blocks > CSA2_POOL_MAX) return CSA2_ERR_UNSUPPORTED;
     const int64_t BT = (int64_t)kv->batch * Tq;
     if (BT > 65535) return CSA2_ERR_UNSUPPORTED;   // grid.y limit
-    (void)workspace;
-    (void)ws_bytes;
+    const ReindexLayout L = reindex_layout(BT, pool_blocks);
+    if (!workspace || ws_bytes < L.total || !aligned(workspace, kAlign)) return CSA2_ERR_WORKSPACE;
 
     IndexArgs a;
     memset(&a, 0, sizeof(a));
@@ -396,6 +408,10 @@ static csa2_status index_reindex(const KvView *kv, const void *q_idx_bf16, const
     a.q_pos = q_pos;
     a.Tq = Tq;
     a.H_I = H_I;
+    a.scores = (float *)workspace;
+    a.score_stride = (int64_t)pool_blocks * 8;
+    a.bmax = (float *)((uint8_t *)workspace + L.bmax_off);
+    a.bmax_stride = pool_blocks;
     a.pool = pool;
     a.pool_blocks = pool_blocks;
     a.top_k = top_k;
@@ -405,7 +421,9 @@ static csa2_status index_reindex(const KvView *kv, const void *q_idx_bf16, const
     a.wait = current_wait_cfg();
     a.pm = kv->pm;
     cudaStream_t s = (cudaStream_t)stream;
-    return launched(launch_reindex_fused(a, (int)BT, s));
+    st = launched(launch_reindex_score(a, (int)BT, s));
+    if (st != CSA2_OK) return st;
+    return launched(launch_select_reindex(a, (int)BT, s));
 }
 
 csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
@@ -541,13 +559,14 @@ csa2_status csa2_index_full_paged(const csa2_paged_kv *kv, const void *q_idx_bf1
 csa2_status csa2_index_reindex_paged(const csa2_paged_kv *kv, const void *q_idx_bf16, const float *w,
                                      const int32_t *q_pos, int32_t Tq, int32_t H_I, const int32_t *pool,
                                      int32_t pool_blocks, int32_t top_k, int32_t *topk_out,
-                                     int32_t *topk_count, int32_t *dev_err, csa2_stream_t stream) {
+                                     int32_t *topk_count, void *workspace, size_t ws_bytes,
+                                     int32_t *dev_err, csa2_stream_t stream) {
     KvView v;
     const KvView *pv;
     csa2_status st = paged_view(kv, &v, &pv);
     if (st != CSA2_OK) return st;
     return index_reindex(pv, q_idx_bf16, w, q_pos, Tq, H_I, pool, pool_blocks, top_k, topk_out,
-                         topk_count, nullptr, 0, dev_err, stream);
+                         topk_count, workspace, ws_bytes, dev_err, stream);
 }
 
 csa2_status csa2_sparse_attn_decode_paged(const csa2_paged_kv *kv, const csa2_swa *swa,

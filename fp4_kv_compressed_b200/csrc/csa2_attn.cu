@@ -27,8 +27,8 @@
 // 16 warps, specialised:
 //   warp 0       TMEM allocation + the MMA issue loop (one elected lane issues);
 //   warp 1       fused append only: quantises the query token's new SWA row;
-//   (set-up: every thread prefetches its selected entry into L2 -- the two CTAs take
-//    alternate entries -- and one thread the request's SWA ring)
+//   warp 2       prefetches the entries of this CTA's later tiles into L2 (bulk prefetch;
+//                the set-up prefetches the request's SWA ring);
 //   warps 4-11   softmax: warp w reads TMEM lane quadrant w % 4 (32 keys) and the
 //                32 heads of half (w - 4) / 4;
 //   warps 12-15  producers: thread = key of the tile; dequantise one 128-channel stage
@@ -83,6 +83,8 @@ struct __align__(1024) Smem {
     float pm[kHeads], pl[kHeads];              // the peer's, written by the peer
     float wself[kHeads];                       // combine: weight of this CTA's partial
     uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], p_full, pv_done, drain, never;
+    uint64_t new_ready;                        // fused append: the new SWA row is in smem
+    uint64_t xfer;                             // combine: the peer's part has landed
     uint32_t tmem_base;
     int32_t abort;
     float wred[16];
@@ -233,6 +235,18 @@ __device__ __forceinline__ bool group_any(int hh, bool pred) {
         : "memory");
     return r != 0;
 }
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+                 : "memory");
+}
+// Bulk copy from this CTA's shared memory into the peer CTA's (dst and bar are
+// shared::cluster addresses; completes as bytes on bar).  No multicast.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "r"(smem_u32(src)), "r"(bytes), "r"(bar)
+        : "memory");
+}
 // L2 prefetch of [p, p + bytes) (p 16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
@@ -284,7 +298,10 @@ struct KeyMap {      // this CTA's keys and where each comes from
     int64_t b;
     int64_t ring_base;
     const uint8_t *new_row;   // fused append: the newest window key is this row (smem)
-    float new_sigma;
+    const float *new_sigma;
+    uint64_t *new_ready;      // ... written once this completes
+    bool *new_ok;
+    const Smem *smem;
 };
 
 __device__ __forceinline__ void load_stage(Raw &r, const AttnArgs &a, const KeyMap &km, int kg, bool zrow,
@@ -299,10 +316,18 @@ __device__ __forceinline__ void load_stage(Raw &r, const AttnArgs &a, const KeyM
             r.sc = __ldg(reinterpret_cast<const uint2 *>(a.scales + off * kScaleBytes + 8 * j));
             r.kind = 1;
         } else if (km.new_row != nullptr && kg == km.n_keys - 1) {
+            if (!*km.new_ok) {
+                *km.new_ok = mbar_wait(km.new_ready, 0, a.wait.limit_ns, *km.smem);
+                if (!*km.new_ok) {
+                    set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+                    r.kind = 0;
+                    return;
+                }
+            }
             const uint4 *src = reinterpret_cast<const uint4 *>(km.new_row + 128 * j);
 #pragma unroll
             for (int u = 0; u < 8; ++u) r.c[u] = src[u];
-            r.sigma = km.new_sigma;
+            r.sigma = *km.new_sigma;
             r.kind = 2;
         } else {
             const int64_t pos = km.w0 + (kg - km.n_sel);
@@ -411,6 +436,8 @@ attn_kernel(AttnArgs a) {
         mbar_init(&s.pv_done, 1);
         mbar_init(&s.drain, 1);
         mbar_init(&s.never, 1);
+        mbar_init(&s.new_ready, 1);
+        mbar_init(&s.xfer, 1);
         s.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -451,11 +478,6 @@ attn_kernel(AttnArgs a) {
         if (row < 0) {
             set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
             e_ok = false;
-        } else if ((threadIdx.x & 1) == rank) {
-            // the two CTAs of the cluster prefetch alternate entries into L2 while the
-            // set-up goes on; the producers then gather from L2
-            prefetch_l2(a.codes + row * kCodeBytes, kCodeBytes);
-            prefetch_l2(a.scales + row * kScaleBytes, kScaleBytes);
         }
     }
     if (threadIdx.x == 32 * 3 && a.swa_len > 0 && rank == 0) {
@@ -496,27 +518,6 @@ attn_kernel(AttnArgs a) {
     const int nt = (k1 - k0 + kTK - 1) / kTK;
     const bool fuse = a.swa_new != nullptr && n_win > 0;
     const uint32_t owner = (n_keys - 1) < k_split ? 0u : 1u;   // the CTA holding the newest key
-    if (fuse && warp == 1 && rank == owner) {
-        // The same FP8 row quantiser as csa2_quantize_append: codes and sigma go to
-        // shared memory (this CTA's producers read the window's newest key from there)
-        // and, from head group 0, to the ring slot t % wcap.
-        float xnew[16];
-        unpack_bf16x8(xraw[0], xnew);
-        unpack_bf16x8(xraw[1], xnew + 8);
-        if constexpr (kRope) {
-            if (!rope_lane16(xnew, lane, a.rope.cs, a.rope.n_pos, a.rope.start, a.rope.pairs, t) &&
-                lane == 0)
-                set_dev_err(a.dev_err, CSA2_DEVERR_ROPE);
-        }
-        quant_fp8_lanes<kDim>(xnew, s.swa_new, &s.swa_new_sigma, lane);
-        __syncwarp();
-        if (blockIdx.y == 0) {
-            const int64_t slot = (int64_t)b * a.wcap + t % a.wcap;
-            reinterpret_cast<uint4 *>(a.swa_codes + slot * kDim)[lane] =
-                reinterpret_cast<const uint4 *>(s.swa_new)[lane];
-            if (lane == 0) a.swa_scale[slot] = s.swa_new_sigma;
-        }
-    }
     const int qexp = qmax > 0.0f ? max(0, ilogbf(qmax) - 14) : 0;   // max|q| * 2^-qexp < 2^15
     {
         const float inv = exp2f((float)-qexp);
@@ -599,6 +600,37 @@ attn_kernel(AttnArgs a) {
             __syncwarp();
             const bool drained = mbar_wait<false>(&s.drain, 0, kDrainLimitNs, s);
             (void)drained;
+        }
+    } else if (warp == 1) {
+        if (fuse && rank == owner) {
+            // The same FP8 row quantiser as csa2_quantize_append: codes and sigma go to
+            // shared memory (this CTA's producers read the window's newest key from there,
+            // after new_ready) and, from head group 0, to the ring slot t % wcap.
+            float xnew[16];
+            unpack_bf16x8(xraw[0], xnew);
+            unpack_bf16x8(xraw[1], xnew + 8);
+            if constexpr (kRope) {
+                if (!rope_lane16(xnew, lane, a.rope.cs, a.rope.n_pos, a.rope.start, a.rope.pairs, t) &&
+                    lane == 0)
+                    set_dev_err(a.dev_err, CSA2_DEVERR_ROPE);
+            }
+            quant_fp8_lanes<kDim>(xnew, s.swa_new, &s.swa_new_sigma, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.new_ready);
+            if (blockIdx.y == 0) {
+                const int64_t slot = (int64_t)b * a.wcap + t % a.wcap;
+                reinterpret_cast<uint4 *>(a.swa_codes + slot * kDim)[lane] =
+                    reinterpret_cast<const uint4 *>(s.swa_new)[lane];
+                if (lane == 0) a.swa_scale[slot] = s.swa_new_sigma;
+            }
+        }
+    } else if (warp == 2) {
+        // L2 prefetch of the entries of this CTA's later tiles (tile 0 the producers fetch
+        // at once)
+        for (int kg = k0 + kTK + lane; kg < min(k1, n_sel); kg += 32) {
+            const int64_t row = cache_row(a.pm, a.cap, b, s.ids[kg]);
+            prefetch_l2(a.codes + row * kCodeBytes, kCodeBytes);
+            prefetch_l2(a.scales + row * kScaleBytes, kScaleBytes);
         }
     } else if (warp >= kSoftWarp0 && warp < kProdWarp0) {
         // ---------------- softmax: keys 32 qd .. (TMEM lanes), heads 32 hh .. ----------------
@@ -731,8 +763,12 @@ attn_kernel(AttnArgs a) {
         km.k_end = k1;
         km.b = b;
         km.ring_base = (int64_t)b * a.wcap;
+        bool new_ok = false;
         km.new_row = fuse && rank == owner ? s.swa_new : nullptr;
-        km.new_sigma = fuse && rank == owner ? s.swa_new_sigma : 0.0f;
+        km.new_sigma = &s.swa_new_sigma;
+        km.new_ready = &s.new_ready;
+        km.new_ok = &new_ok;
+        km.smem = &s;
         // rows of the tile's last 16-key group of valid keys are read by the output MMAs
         // and so written (zeros past the keys); rows after that group are not written
         auto zrow_of = [&](int i) { return r < ((min(kTK, k1 - k0 - i * kTK) + 15) / 16) * 16; };
@@ -773,16 +809,18 @@ attn_kernel(AttnArgs a) {
 
     // ---- combine the two key halves of the query through distributed shared memory ----
     // CTA r writes channels [256 r, 256 r + 256) = O^T blocks 2 r, 2 r + 1.  Every thread
-    // of both CTAs takes both cluster barriers, whatever happened above.
+    // of both CTAs takes every cluster barrier, whatever happened above.
     __syncwarp();
     tc_fence_before();
     __syncthreads();                       // stats written; this CTA's MMAs have completed
     tc_fence_after();
     const uint32_t peer = rank ^ 1u;
+    constexpr uint32_t kXfer = 2 * kTK * kHeads * 4;    // the peer's two blocks, fp32
     if (threadIdx.x < kHeads) {
         st_peer(peer_addr(&s.pm[threadIdx.x], peer), s.cm[threadIdx.x]);
         st_peer(peer_addr(&s.pl[threadIdx.x], peer), s.cl[threadIdx.x]);
     }
+    if (threadIdx.x == 0) mbar_expect_tx(&s.xfer, kXfer);   // armed before the peer can send
     cluster_sync();                        // stats exchanged; both CTAs' tiles are free
     grid_dep_launch();
     if (threadIdx.x < kHeads) {
@@ -802,56 +840,66 @@ attn_kernel(AttnArgs a) {
     }
     __syncthreads();
     // Warp w: TMEM lane quadrant w % 4 (channels 32 (w % 4) .. of a block), head half
-    // (w >> 2) & 1, block pair member w >> 3.  First the peer's blocks, scaled, into the
-    // peer's shared memory (its tiles, [2 blocks][128 channels][64 heads] fp32, float4
-    // slots swizzled by channel); then own blocks + what the peer sent, to global memory.
+    // (w >> 2) & 1, block pair member w >> 3.  The peer's blocks, scaled, are staged in
+    // local shared memory (`send`, [2 blocks][128 channels][64 heads] fp32, float4 slots
+    // swizzled by channel) and moved by one bulk copy into the peer's `recv`; own blocks
+    // wait in registers.
     const bool have = __shfl_sync(0xFFFFFFFFu, (int)(nt > 0 && !aborted(s)), 0) != 0;
     const int cq = warp & 3, chh = (warp >> 2) & 1, bsel = warp >> 3;
     const int crow = 32 * cq + lane;                 // channel within a block
-    float *recv = reinterpret_cast<float *>(&s.kv[0][0]);
+    float *send = reinterpret_cast<float *>(&s.kv[0][0]);
+    float *recv = reinterpret_cast<float *>(&s.kv[2][0]);
+    const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)chh;
     {
-        const int blk = 2 * (int)peer + bsel;
         float o[32];
         if (have) {
-            tmem_ld32(tmem + ((uint32_t)(32 * cq) << 16) + 64u * (uint32_t)blk + 32u * (uint32_t)chh, o);
+            tmem_ld32(taddr + 64u * (uint32_t)(2 * (int)peer + bsel), o);
         } else {
 #pragma unroll
             for (int h = 0; h < 32; ++h) o[h] = 0.0f;
         }
-        const uint32_t dst = peer_addr(recv + (bsel * kTK + crow) * kHeads, peer);
+        float4 *dst = reinterpret_cast<float4 *>(send + (bsel * kTK + crow) * kHeads);
 #pragma unroll
         for (int f = 0; f < 8; ++f) {                // float4 f of this half = heads 32 chh + 4 f ..
             const int h = 32 * chh + 4 * f;
-            const int fs = (8 * chh + f) ^ (crow & 7);   // swizzled float4 slot of the row
-            st_peer4(dst + 16u * (uint32_t)fs, o[4 * f] * s.wself[h], o[4 * f + 1] * s.wself[h + 1],
-                     o[4 * f + 2] * s.wself[h + 2], o[4 * f + 3] * s.wself[h + 3]);
+            dst[(8 * chh + f) ^ (crow & 7)] = make_float4(o[4 * f] * s.wself[h], o[4 * f + 1] * s.wself[h + 1],
+                                                          o[4 * f + 2] * s.wself[h + 2], o[4 * f + 3] * s.wself[h + 3]);
         }
     }
-    cluster_sync();                        // the peer's part has landed in `recv`
+    fence_async_smem();                    // generic-proxy writes of `send` -> the bulk copy
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t dst = peer_addr(recv, peer), bar = peer_addr(&s.xfer, peer);
+        bulk_copy_to_peer(dst, send, kXfer / 2, bar);
+        bulk_copy_to_peer(dst + kXfer / 2, reinterpret_cast<uint8_t *>(send) + kXfer / 2, kXfer / 2, bar);
+    }
+    float own[32];
+    if (have) {
+        tmem_ld32(taddr + 64u * (uint32_t)(2 * (int)rank + bsel), own);
+    } else {
+#pragma unroll
+        for (int h = 0; h < 32; ++h) own[h] = 0.0f;
+    }
+    const bool got = __syncthreads_and(mbar_wait<false>(&s.xfer, 0, kDrainLimitNs, s)) != 0;
+    if (!got && threadIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
     {
         const int blk = 2 * (int)rank + bsel;
-        float o[32];
-        if (have) {
-            tmem_ld32(tmem + ((uint32_t)(32 * cq) << 16) + 64u * (uint32_t)blk + 32u * (uint32_t)chh, o);
-        } else {
-#pragma unroll
-            for (int h = 0; h < 32; ++h) o[h] = 0.0f;
-        }
-        const float *src = recv + (bsel * kTK + crow) * kHeads;
+        const float4 *src = reinterpret_cast<const float4 *>(recv + (bsel * kTK + crow) * kHeads);
         float *obase = a.out + ((int64_t)qi * a.H + h0) * kDim + 128 * blk + crow;
 #pragma unroll
         for (int f = 0; f < 8; ++f) {
             const int h = 32 * chh + 4 * f;
-            const int fs = (8 * chh + f) ^ (crow & 7);
-            const float4 pr = reinterpret_cast<const float4 *>(src)[fs];
+            const float4 pr = got ? src[(8 * chh + f) ^ (crow & 7)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             const float pv[4] = {pr.x, pr.y, pr.z, pr.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-                if (h + k < hcta) obase[(int64_t)(h + k) * kDim] = fmaf(o[4 * f + k], s.wself[h + k], pv[k]);
+                if (h + k < hcta) obase[(int64_t)(h + k) * kDim] = fmaf(own[4 * f + k], s.wself[h + k], pv[k]);
         }
     }
+    // Both CTAs have seen their incoming copy land, so both outgoing copies have finished
+    // reading `send`: only now may either CTA leave (and its shared memory be reused).
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));

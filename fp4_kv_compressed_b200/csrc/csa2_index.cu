@@ -24,11 +24,12 @@ namespace csa2 {
 // ------------------------------------------------------------------------------
 // Scoring core (score_rows_at): a group of NT threads scores a tile of NT * R rows
 // staged in shared memory (thread t: rows t + NT r, r < R).  The Full scan runs it in
-// small CTAs (kScoreThreads) that keep many tiles in flight per SM; the fused Reindex
-// in 8 warps of a larger CTA behind a cp.async ring.
+// small CTAs (kScoreThreads) that keep many tiles in flight per SM; so does the Reindex
+// scoring, with the smaller tile.
 // ------------------------------------------------------------------------------
 constexpr int kScoreThreads = 64;
 constexpr int kScanRows = 4;       // rows per thread, Full scan (256-row, 32 KB tiles)
+constexpr int kReindexRows = 2;    // rows per thread, Reindex gather (128-row, 16 KB tiles)
 
 // 16-byte unit u of row r lives at unit swz(r, u): a quarter-warp reading unit
 // u of 8 consecutive rows hits 8 different 16-byte bank groups.
@@ -75,10 +76,6 @@ __device__ __forceinline__ void load_query(ScoreSmem<D, HI, R> &s, const uint16_
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem));
-}
-__device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
-    uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(sa), "l"(gmem));
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
@@ -224,6 +221,74 @@ index_scan_kernel(IndexArgs a) {
         if (threadIdx.x < R && 64 * (int)threadIdx.x < rows)
             a.bmax64[(int64_t)qi * a.bmax64_stride + p0 / 64 + threadIdx.x] =
                 fmaxf(s.m64[0][threadIdx.x], s.m64[1][threadIdx.x]);
+    }
+}
+
+// ------------------------------------------------------------------------------
+// a6: Reindex scoring of the pool.  grid (ceil(8 pool_blocks / kTileRows), B*Tq),
+// kScoreThreads threads, kTileRows = kScoreThreads * kReindexRows (16 pool blocks).
+// Candidate c = 8 * slot + r of the pool (slot < pool_blocks, r < 8) is position
+// 8 * pool[slot] + r; its score goes to scores[qi][c] and the maximum of the slot's
+// visible positions to bmax[qi][slot] (for the selection's block lemma).  Many small
+// CTAs keep many scattered 1 KB blocks in flight per SM.
+// ------------------------------------------------------------------------------
+template <int D, int HI>
+__global__ void __launch_bounds__(kScoreThreads)
+reindex_score_kernel(IndexArgs a) {
+    constexpr int R = kReindexRows, kTileRows = kScoreThreads * R;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    ScoreSmem<D, HI, R> &s = *reinterpret_cast<ScoreSmem<D, HI, R> *>(smem_raw);
+    __shared__ int64_t row_of[kTileRows];   // cache row of each candidate, -1: not scored
+    grid_dep_wait();
+    const int qi = blockIdx.y;
+    const int b = qi / a.Tq;
+    int64_t N = visible_entries(a.q_pos[qi], a.ratio);
+    N = min64(N, a.cap);
+    const int slot0 = blockIdx.x * (kTileRows / 8);
+    const int32_t *pool = a.pool + (int64_t)qi * a.pool_blocks;
+    float sgv[R];   // row threadIdx.x + kScoreThreads i is handled by this thread below
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        const int r = threadIdx.x + kScoreThreads * i;
+        const int slot = slot0 + r / 8;
+        int blk = __ldg(pool + min(slot, a.pool_blocks - 1));
+        if (slot >= a.pool_blocks) blk = -1;
+        const int64_t p = (int64_t)blk * 8 + (r & 7);
+        if (blk >= 0 && (int64_t)blk * 8 >= N && (r & 7) == 0) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
+        int64_t row = blk >= 0 && p < N ? cache_row(a.pm, a.cap, b, p) : -1;
+        if (blk >= 0 && p < N && row < 0) set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
+        row_of[r] = row;
+        sgv[i] = __ldg(a.idx_scale + (row >= 0 ? row : 0));   // branch-free (row 0 always exists)
+    }
+    __syncthreads();
+    constexpr int U = D / 16;
+    for (int e = threadIdx.x; e < kTileRows * U; e += kScoreThreads) {
+        const int r = e / U, u = e % U;
+        if (row_of[r] >= 0)
+            cp_async16(s.rows + r * D + 16 * swz<D>(r, u), a.idx_codes + row_of[r] * D + 16 * u);
+    }
+    cp_async_commit();
+    load_query<D, HI>(s, a.q_idx + (int64_t)qi * HI * D, a.w + (int64_t)qi * HI);
+    cp_async_wait_all();
+    __syncthreads();
+
+    float sc[R];
+    score_rows<D, HI, R>(s, sc);
+    grid_dep_launch();
+    float *out = a.scores + (int64_t)qi * a.score_stride + (int64_t)slot0 * 8;
+    float *bm = a.bmax + (int64_t)qi * a.bmax_stride + slot0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int row = threadIdx.x + kScoreThreads * r;
+        const bool valid = row_of[row] >= 0;
+        const float v = valid ? __fmul_rn(sc[r], sgv[r]) : -INFINITY;
+        if (slot0 + row / 8 < a.pool_blocks) out[row] = valid ? v : 0.0f;
+        // the slot's 8 candidates are 8 consecutive lanes
+        float m = v;
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+        if ((row & 7) == 0 && slot0 + row / 8 < a.pool_blocks) bm[row / 8] = m;
     }
 }
 
@@ -608,6 +673,54 @@ select_full_kernel(IndexArgs a) {
     if (threadIdx.x == 0 && a.topk_count) a.topk_count[qi] = cnt;
 }
 
+// a6 selection: Top-K of the scored pool candidates.  By the block lemma, the Top-K lies
+// in the top_k best pool slots by their maxima: select those slots (<= 2048 keys), then
+// the Top-K over their <= 8 top_k positions.  Slots are in pool order = position order.
+__global__ void __launch_bounds__(kSelThreads)
+select_reindex_kernel(IndexArgs a) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    SelSmem &s = *reinterpret_cast<SelSmem *>(smem_raw);
+    __shared__ int sel_out[CSA2_TOPK_MAX];
+    __shared__ int sub[CSA2_TOPK_MAX];
+    grid_dep_wait();
+    const int qi = blockIdx.x;
+    const int64_t N = min64(visible_entries(a.q_pos[qi], a.ratio), a.cap);
+    const int32_t *pool = a.pool + (int64_t)qi * a.pool_blocks;
+    const float *sc = a.scores + (int64_t)qi * a.score_stride;
+    const float *bm = a.bmax + (int64_t)qi * a.bmax_stride;
+    const int P = a.pool_blocks;
+    for (int i = threadIdx.x; i < P; i += kSelThreads) {
+        const int blk = __ldg(pool + i);
+        s.pool[i] = blk;
+        s.keys[i] = blk >= 0 && (int64_t)blk * 8 < N ? score_key(__ldg(bm + i)) : 0u;
+        if (i > 0 && blk >= 0 && __ldg(pool + i - 1) >= blk) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
+    }
+    __syncthreads();
+    auto skey = [&](int i) -> uint32_t { return s.keys[i]; };
+    auto sid = [&](int i) -> int { return i; };
+    const int ns = block_topk(skey, sid, P, a.top_k, sub, s);
+    __syncthreads();
+    // the chosen slots' 8 scores each (32 bytes, 16-byte aligned rows), then their keys
+    for (int c = threadIdx.x; c < 2 * ns; c += kSelThreads)
+        cp_async16(s.keys + 4 * c, sc + (int64_t)sub[c >> 1] * 8 + 4 * (c & 1));
+    cp_async_commit();
+    cp_async_wait_all();
+    __syncthreads();
+    for (int i = threadIdx.x; i < 8 * ns; i += kSelThreads) {
+        const int64_t p = (int64_t)s.pool[sub[i >> 3]] * 8 + (i & 7);
+        s.keys[i] = p < N ? score_key(__uint_as_float(s.keys[i])) : 0u;
+    }
+    __syncthreads();
+    auto key = [&](int i) -> uint32_t { return s.keys[i]; };
+    auto id = [&](int i) -> int { return s.pool[sub[i >> 3]] * 8 + (i & 7); };
+    const int cnt = block_topk(key, id, 8 * ns, a.top_k, sel_out, s);
+    __syncthreads();
+    grid_dep_launch();
+    int32_t *topk = a.topk_out + (int64_t)qi * a.top_k;
+    for (int i = threadIdx.x; i < a.top_k; i += blockDim.x) topk[i] = i < cnt ? sel_out[i] : -1;
+    if (threadIdx.x == 0) a.topk_count[qi] = cnt;
+}
+
 // ------------------------------------------------------------------------------
 // Context parallel: merge of the shards' candidate lists.  One CTA per query; the lists
 // [n_lists][BT][list_len] of candidate keys (order key << 32 | ~global id, 0 = empty;
@@ -657,207 +770,6 @@ cudaError_t launch_index_merge(const uint64_t *lists, int BT, int n_lists, int l
     cudaError_t e = launch_pdl(index_merge_kernel, dim3(BT), dim3(kSelThreads), smem, st, lists, n_lists,
                                list_len, k, lo, hi, ids_out, count_out, local_out);
     return e != cudaSuccess ? e : cudaGetLastError();
-}
-
-// ------------------------------------------------------------------------------
-// a6 fused: Reindex scoring and selection in one launch.  A cluster of C CTAs per
-// query (C = 2, 4 or 8, chosen at launch so that the grid fills the GPU); CTA c takes
-// the pool slots [c Pc, (c + 1) Pc), Pc = ceil(pool_blocks / C), in pool order:
-//   1. scores its 8 Pc candidates into order keys in shared memory: 8 warps stream
-//      the candidates' index-K rows through a two-stage cp.async ring (up to 512
-//      rows, i.e. 64 pool blocks, per stage) and score them with the same core and the
-//      same fixed fp32 order as the Full scan;
-//   2. selects a local Top-K (the exact key order, all 1024 threads);
-//   3. CTA 0 gathers the C local lists from the other CTAs' shared memory and
-//      selects the final Top-K among them.
-// Every position of the global Top-K is in its own CTA's local Top-K, so the result
-// is the exact Top-K over the pool.  The slices are contiguous runs of the ascending
-// pool, so concatenating the lists in rank order keeps positions ascending and the
-// compaction's index order is the position order.
-// ------------------------------------------------------------------------------
-constexpr int kRfScoreThreads = 256;                     // scoring warps 0-7
-constexpr int kRfStageRows = 512;                        // ring stage capacity: 64 pool blocks
-// rows per scoring thread per stage: the 1024-thread CTA has 64 registers a thread
-template <int HI>
-constexpr int rf_rows() { return HI <= 4 ? 2 : 1; }
-constexpr int kRfMaxCand = 8192;                         // candidates of one CTA (C >= 2)
-constexpr int kRfMaxC = 8;
-
-template <int D, int HI>
-struct RfSmem {
-    // scoring ring; after scoring, the merge lists of CTA 0 live here
-    alignas(128) uint8_t rows[2][kRfStageRows * D];
-    float sig[2][kRfStageRows];
-    float2 q[D / 2][HI];
-    float w[HI];
-    int32_t pool[kRfMaxCand / 8];
-    int64_t prow[kRfMaxCand / 8];                        // first cache row of each pool block
-    // selection state (block_topk)
-    uint32_t hist[1 << kSelDigit];
-    int wa[kSelWarps], wb[kSelWarps];
-    uint32_t wmin[kSelWarps], wmax[kSelWarps];
-    int bcast[4];
-    alignas(16) uint32_t keys[kRfMaxCand];
-    int32_t loc_idx[CSA2_TOPK_MAX];                      // local Top-K: candidate indices
-    uint32_t loc_key[CSA2_TOPK_MAX];                     // ... their keys and positions
-    int32_t loc_pos[CSA2_TOPK_MAX];
-    int32_t loc_cnt;
-    int32_t out[CSA2_TOPK_MAX];
-};
-
-__device__ __forceinline__ uint32_t rf_cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void rf_cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t rf_peer(const void *local, uint32_t rank) {
-    uint32_t r, a = (uint32_t)__cvta_generic_to_shared(local);
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ uint32_t rf_ld_peer(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ void rf_score_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
-template <int D, int HI>
-__global__ void __launch_bounds__(kSelThreads, 1)
-reindex_fused_kernel(IndexArgs a, int C) {
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    RfSmem<D, HI> &s = *reinterpret_cast<RfSmem<D, HI> *>(smem_raw);
-    const uint32_t rank = rf_cluster_rank();
-    const int qi = blockIdx.x / C;
-    const int b = qi / a.Tq;
-    const int Pc = (a.pool_blocks + C - 1) / C;
-    const int slot0 = min(a.pool_blocks, (int)rank * Pc);
-    const int nslot = min(a.pool_blocks, slot0 + Pc) - slot0;
-    const int ncand = 8 * nslot;
-    grid_dep_wait();
-    int64_t N = visible_entries(a.q_pos[qi], a.ratio);
-    N = min64(N, a.cap);
-    const int32_t *pool = a.pool + (int64_t)qi * a.pool_blocks + slot0;
-    for (int i = threadIdx.x; i < nslot; i += kSelThreads) {
-        const int blk = __ldg(pool + i);
-        if (blk >= 0 && (int64_t)blk * 8 >= N) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
-        if (i > 0 && blk >= 0 && __ldg(pool + i - 1) >= blk) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
-        s.pool[i] = blk >= 0 && (int64_t)blk * 8 < N ? blk : -1;
-        // the block's first cache row (a page holds whole blocks); -1: not scored
-        int64_t row = -1;
-        if (s.pool[i] >= 0) {
-            row = cache_row(a.pm, a.cap, b, (int64_t)s.pool[i] * 8);
-            if (row < 0) set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
-        }
-        s.prow[i] = row;
-    }
-    if (threadIdx.x < kSelThreads / 2) {
-        // q and w of the query (the scoring core's layout)
-        const uint16_t *qp = a.q_idx + (int64_t)qi * HI * D;
-        for (int e = threadIdx.x; e < HI * D / 2; e += kSelThreads / 2) {
-            const uint32_t two = __ldg(reinterpret_cast<const uint32_t *>(qp) + e);
-            const int h = e / (D / 2), j = e % (D / 2);
-            s.q[j][h] = make_float2(bf16_bits_to_f32(two & 0xFFFFu), bf16_bits_to_f32(two >> 16));
-        }
-        if (threadIdx.x < HI) s.w[threadIdx.x] = __ldg(a.w + (int64_t)qi * HI + threadIdx.x);
-    }
-    __syncthreads();
-
-    // ---- 1. scoring (warps 0-7), two-stage cp.async ring ----
-    constexpr int R = rf_rows<HI>(), SR = kRfScoreThreads * R;   // rows per stage
-    const int n_stages = (ncand + SR - 1) / SR;
-    if (threadIdx.x < kRfScoreThreads) {
-        const int t = threadIdx.x;
-        auto issue = [&](int st) {
-            const int buf = st & 1;
-            constexpr int U = D / 16;
-            for (int e = t; e < SR * U; e += kRfScoreThreads) {
-                const int r = e / U, u = e % U, c = st * SR + r;
-                if (c < ncand) {
-                    const int blk = s.prow[c >> 3] >= 0 ? s.pool[c >> 3] : -1;
-                    const int64_t p = (int64_t)blk * 8 + (c & 7);
-                    if (blk >= 0 && p < N)
-                        cp_async16(s.rows[buf] + r * D + 16 * swz<D>(r, u),
-                                   a.idx_codes + (s.prow[c >> 3] + (c & 7)) * D + 16 * u);
-                }
-            }
-            // the entries' scales (4 bytes each; visible positions only)
-            for (int r = t; r < SR; r += kRfScoreThreads) {
-                const int c = st * SR + r;
-                if (c < ncand) {
-                    const int blk = s.prow[c >> 3] >= 0 ? s.pool[c >> 3] : -1;
-                    const int64_t p = (int64_t)blk * 8 + (c & 7);
-                    if (blk >= 0 && p < N) cp_async4(&s.sig[buf][r], a.idx_scale + s.prow[c >> 3] + (c & 7));
-                }
-            }
-            cp_async_commit();
-        };
-        if (n_stages > 0) issue(0);
-        if (n_stages > 1) issue(1);
-        for (int st = 0; st < n_stages; ++st) {
-            const int buf = st & 1;
-            if (st + 1 < n_stages)
-                asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-            else
-                asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-            rf_score_sync();
-            float sc[R];
-            score_rows_at<D, HI, R, kRfScoreThreads>(s.rows[buf], s.q, s.w, t, sc);
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const int row = t + kRfScoreThreads * r, c = st * SR + row;
-                if (c < ncand) {
-                    const int blk = s.prow[c >> 3] >= 0 ? s.pool[c >> 3] : -1;
-                    const int64_t p = (int64_t)blk * 8 + (c & 7);
-                    s.keys[c] = (blk >= 0 && p < N) ? score_key(__fmul_rn(sc[r], s.sig[buf][row])) : 0u;
-                }
-            }
-            rf_score_sync();                                 // the buffer is free again
-            if (st + 2 < n_stages) issue(st + 2);
-        }
-    }
-    __syncthreads();
-    grid_dep_launch();
-
-    // ---- 2. local Top-K over this CTA's candidates ----
-    auto key = [&](int i) -> uint32_t { return s.keys[i]; };
-    auto idx = [&](int i) -> int { return i; };
-    const int cnt = block_topk(key, idx, ncand, a.top_k, s.loc_idx, s);
-    for (int j = threadIdx.x; j < cnt; j += kSelThreads) {
-        const int c = s.loc_idx[j];
-        s.loc_key[j] = s.keys[c];
-        s.loc_pos[j] = s.pool[c >> 3] * 8 + (c & 7);
-    }
-    if (threadIdx.x == 0) s.loc_cnt = cnt;
-    rf_cluster_sync();                                       // every local list is ready
-
-    // ---- 3. CTA 0 merges the C lists (rank order = position order) ----
-    if (rank == 0) {
-        uint32_t *mkey = reinterpret_cast<uint32_t *>(&s.rows[0][0]);
-        int32_t *mpos = reinterpret_cast<int32_t *>(&s.rows[0][0] + kRfMaxC * CSA2_TOPK_MAX * 4);
-        int off = 0;
-        for (int c = 0; c < C; ++c) {
-            const int n = (int)rf_ld_peer(rf_peer(&s.loc_cnt, (uint32_t)c));
-            const uint32_t kb = rf_peer(s.loc_key, (uint32_t)c), pb = rf_peer(s.loc_pos, (uint32_t)c);
-            for (int j = threadIdx.x; j < n; j += kSelThreads) {
-                mkey[off + j] = rf_ld_peer(kb + 4u * (uint32_t)j);
-                mpos[off + j] = (int32_t)rf_ld_peer(pb + 4u * (uint32_t)j);
-            }
-            off += n;
-        }
-        __syncthreads();
-        auto mk = [&](int i) -> uint32_t { return mkey[i]; };
-        auto mp = [&](int i) -> int { return mpos[i]; };
-        const int fin = block_topk(mk, mp, off, a.top_k, s.out, s);
-        __syncthreads();
-        int32_t *topk = a.topk_out + (int64_t)qi * a.top_k;
-        for (int i = threadIdx.x; i < a.top_k; i += kSelThreads) topk[i] = i < fin ? s.out[i] : -1;
-        if (threadIdx.x == 0) a.topk_count[qi] = fin;
-    }
-    rf_cluster_sync();                                       // no CTA leaves while CTA 0 reads it
 }
 
 // ------------------------------------------------------------------------------
@@ -913,47 +825,35 @@ cudaError_t launch_select_full(const IndexArgs &a, int BT, cudaStream_t st) {
     return launch_select_full_t<kSelStageMax>(a, BT, st);
 }
 
-// CTAs per query of the fused Reindex: enough clusters to fill the GPU in one wave
-// (one CTA per SM), at least 2 (so that a CTA holds at most 8192 candidates), at most 8.
-static int reindex_cluster_size(int BT) {
-    const int sms = device_sm_count();
-    int c = 2;
-    while (c < kRfMaxC && (int64_t)2 * c * BT <= sms) c *= 2;
-    return c;
-}
 
 template <int D, int HI>
-static cudaError_t launch_reindex_fused_t(const IndexArgs &a, int BT, cudaStream_t st) {
-    const size_t smem = sizeof(RfSmem<D, HI>);
+static cudaError_t launch_reindex_t(const IndexArgs &a, int BT, cudaStream_t st) {
+    size_t smem = sizeof(ScoreSmem<D, HI, kReindexRows>);
     static std::atomic<uint64_t> configured{0};   // per device
     {
-        cudaError_t e = config_kernel_once(reindex_fused_kernel<D, HI>, smem, configured);
+        cudaError_t e = config_kernel_once(reindex_score_kernel<D, HI>, smem, configured);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(reindex_fused_kernel<D, HI>, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
-        (void)e;
     }
-    const int C = reindex_cluster_size(BT);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(C * BT));
-    cfg.blockDim = dim3(kSelThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = (unsigned)C;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, reindex_fused_kernel<D, HI>, a, C);
+    constexpr int kBlocksPerTile = kScoreThreads * kReindexRows / 8;
+    int gx = (a.pool_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
+    cudaError_t e = launch_pdl(reindex_score_kernel<D, HI>, dim3(gx, BT), dim3(kScoreThreads), smem, st, a);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_reindex_fused(const IndexArgs &a, int BT, cudaStream_t st) {
-    if (a.d_idx == 128) { CSA2_DISPATCH_HI(128, launch_reindex_fused_t, a, BT, st) }
-    CSA2_DISPATCH_HI(64, launch_reindex_fused_t, a, BT, st)
+cudaError_t launch_reindex_score(const IndexArgs &a, int BT, cudaStream_t st) {
+    if (a.d_idx == 128) { CSA2_DISPATCH_HI(128, launch_reindex_t, a, BT, st) }
+    CSA2_DISPATCH_HI(64, launch_reindex_t, a, BT, st)
+}
+
+cudaError_t launch_select_reindex(const IndexArgs &a, int BT, cudaStream_t st) {
+    size_t smem = sizeof(SelSmem);
+    static std::atomic<uint64_t> configured{0};   // per device
+    {
+        cudaError_t e = config_kernel_once(select_reindex_kernel, smem, configured);
+        if (e != cudaSuccess) return e;
+    }
+    cudaError_t e = launch_pdl(select_reindex_kernel, dim3(BT), dim3(kSelThreads), smem, st, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace csa2

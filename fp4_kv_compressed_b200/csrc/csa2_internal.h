@@ -189,7 +189,8 @@ cudaError_t launch_quantize_append(const QuantArgs &a, cudaStream_t st);
 cudaError_t launch_index_scan(const IndexArgs &a, int BT, cudaStream_t st);
 cudaError_t launch_index_scan_tc(const IndexArgs &a, int B, cudaStream_t st);
 cudaError_t launch_select_full(const IndexArgs &a, int BT, cudaStream_t st);
-cudaError_t launch_reindex_fused(const IndexArgs &a, int BT, cudaStream_t st);
+cudaError_t launch_reindex_score(const IndexArgs &a, int BT, cudaStream_t st);
+cudaError_t launch_select_reindex(const IndexArgs &a, int BT, cudaStream_t st);
 cudaError_t launch_sparse_attn(const AttnArgs &a, int BT, cudaStream_t st);
 cudaError_t launch_index_merge(const uint64_t *lists, int BT, int n_lists, int list_len, int k,
                                int64_t lo, int64_t hi, int32_t *ids_out, int32_t *count_out,

@@ -249,7 +249,7 @@ class DecodeStack:
         for lp in self.plan:
             if lp.layer == first[lp.group] or not self._fuse_swa(self.Tq):
                 n += 1                 # quantise-append (the group's entry and/or SWA rows)
-            n += {"F": 2, "X": 1, "U": 0}[lp.mode]
+            n += {"F": 2, "X": 2, "U": 0}[lp.mode]
             n += 1                     # attention (with the fused SWA append in decode)
         return n
 

@@ -334,11 +334,9 @@ CSA2_API csa2_status csa2_attn_combine(const float *o_parts, const float *lse_pa
  * a6 Reindex layer: the same score with this layer's own q_idx / w, over the
  * visible positions of the pool's blocks only, then Top-K (same order, same
  * output form).  pool [B][Tq][pool_blocks] as written by csa2_index_full
- * (-1 = unused slot; the used slots ascending).  One launch: a cluster of CTAs
- * per query scores its share of the pool into shared memory, selects a local
- * Top-K, and the cluster merges the local lists.  No workspace is needed:
- * csa2_workspace_size(CSA2_OP_INDEX_REINDEX, ...) is 0 and `workspace` may be
- * NULL (it is ignored).
+ * (-1 = unused slot; the used slots ascending).  Workspace:
+ * csa2_workspace_size(CSA2_OP_INDEX_REINDEX, B, Tq, 0, 0, top_k, pool_blocks)
+ * bytes, 256-byte aligned (the candidates' scores and each slot's maximum).
  */
 CSA2_API csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16, const float *w,
                                const int32_t *q_pos, int32_t Tq, int32_t H_I,
@@ -447,12 +445,13 @@ CSA2_API csa2_status csa2_index_full_paged(const csa2_paged_kv *kv, const void *
                                            int32_t *topk_count, void *workspace, size_t ws_bytes,
                                            int32_t *dev_err, csa2_stream_t stream);
 
-/* csa2_index_reindex on a paged cache (no workspace). */
+/* csa2_index_reindex on a paged cache (same workspace). */
 CSA2_API csa2_status csa2_index_reindex_paged(const csa2_paged_kv *kv, const void *q_idx_bf16,
                                               const float *w, const int32_t *q_pos, int32_t Tq,
                                               int32_t H_I, const int32_t *pool,
                                               int32_t pool_blocks, int32_t top_k,
                                               int32_t *topk_out, int32_t *topk_count,
+                                              void *workspace, size_t ws_bytes,
                                               int32_t *dev_err, csa2_stream_t stream);
 
 /* csa2_sparse_attn_decode on a paged cache.  swa_bf16 non-NULL = the fused decode

@@ -42,7 +42,7 @@ def test_workspace_sizes(pkg):
     assert flat >= 64 * 131072 * 4 + 64 * 16384 * 4 + 64 * 2048 * 4 and flat == full
     short = ws(pkg.CSA2_OP_INDEX_FULL, 64, 1, 16384, 64, 512, 0)
     assert 64 * 16384 * 4 <= short < ws(pkg.CSA2_OP_INDEX_FULL, 64, 1, 16384, 64, 512, 2048)
-    assert ws(pkg.CSA2_OP_INDEX_REINDEX, 64, 1, 0, 64, 512, 2048) == 0   # scores on chip
+    assert ws(pkg.CSA2_OP_INDEX_REINDEX, 64, 1, 0, 64, 512, 2048) >= 64 * 2048 * (8 + 1) * 4
     assert ws(pkg.CSA2_OP_SPARSE_ATTN, 64, 1, 0, 64, 512, 0) == 0
     assert ws(99, 1, 1, 1, 1, 1, 1) == 0
 

@@ -80,10 +80,12 @@ def test_paged_bytes_and_index_calls(pkg):
         full(st, q_idx, w, qp, 1, H_I, N, 2048, 512, pool, topk, cnt, ws, err)
         rt = torch.full((B, 1, 512), -7, dtype=torch.int32, device="cuda")
         rc = torch.zeros(B, 1, dtype=torch.int32, device="cuda")
+        rws = torch.empty(pkg.csa2_workspace_size(pkg.CSA2_OP_INDEX_REINDEX, B, 1, 0, 0, 512, 2048),
+                          dtype=torch.uint8, device="cuda")
         if reidx is not None:
-            reidx(st, q_idx, w, qp, 1, H_I, pool, 2048, 512, rt, rc, None, err)
+            reidx(st, q_idx, w, qp, 1, H_I, pool, 2048, 512, rt, rc, rws, err)
         else:
-            pkg.csa2_index_reindex_paged(st, q_idx, w, qp, 1, H_I, pool, 2048, 512, rt, rc, err)
+            pkg.csa2_index_reindex_paged(st, q_idx, w, qp, 1, H_I, pool, 2048, 512, rt, rc, rws, err)
         out[name] = [x.cpu() for x in (pool, topk, cnt, rt, rc)]
     assert pkg.csa2_read_device_error(err) == 0
     for a, b in zip(out["flat"], out["paged"]):
