@@ -24,16 +24,17 @@
 // in fp32, to the logit and folded into P.  Q (the K-major B operand of S^T) is
 // converted to fp16 after an exact power-of-two scaling that keeps max|q| below 2^15.
 //
-// 16 warps, specialised:
+// 12 warps, specialised:
 //   warp 0       TMEM allocation + the MMA issue loop (one elected lane issues);
 //   warp 1       fused append only: quantises the query token's new SWA row;
 //   warp 2       prefetches the entries of this CTA's later tiles into L2 (bulk prefetch;
 //                the set-up prefetches the request's SWA ring);
-//   warps 4-11   softmax: warp w reads TMEM lane quadrant w % 4 (32 keys) and the
-//                32 heads of half (w - 4) / 4;
-//   warps 12-15  producers: thread = key of the tile; dequantise one 128-channel stage
-//                at a time into shared memory, the next stage's raw bytes already in
-//                registers.
+//   warps 4-11   workers, two roles in turn.  Producer: thread = (key r of the tile,
+//                channel half hh of every 128-channel stage); the raw bytes of its half
+//                of the next tile's key are loaded into registers (one round trip for
+//                all four stages) before the softmax of this tile, and dequantised into
+//                stage j as soon as O^T of this tile has read it.  Softmax: warp w reads
+//                TMEM lane quadrant w % 4 (32 keys) and the 32 heads of half (w - 4) / 4.
 // TMEM (512 columns): O^T block j (channels 128 j .. 128 j + 127) at columns
 // 64 j .. 64 j + 63 (column = head); the two S^T buffers at columns 256 and 320.
 // Online softmax in the log2 domain with lazy rescaling: the running max of a head
@@ -55,7 +56,9 @@
 namespace csa2 {
 namespace attn {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 384;
+constexpr int kWarps = kThreads / 32;
+constexpr int kQChunks = (64 * 64 + kThreads - 1) / kThreads;   // 16-byte Q chunks per thread
 constexpr int kTK = 128;                       // keys per tile (S^T M, TMEM lanes)
 constexpr int kHeads = 64;                     // heads per CTA (MMA N)
 constexpr int kStages = 4;                     // 128-channel quarters of a tile
@@ -64,8 +67,8 @@ constexpr int kCbBytes = kTK * 128;            // one 64-channel block of a stag
 constexpr int kQCbBytes = kHeads * 128;        // one 64-channel block of Q
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol = 256;                // S^T buffer b at columns 256 + 64 b
-constexpr int kSoftWarp0 = 4;                  // softmax warps 4..11
-constexpr int kProdWarp0 = 12;                 // producer warps 12..15
+constexpr int kWorkWarp0 = 4;                  // softmax + producer warps 4..11
+constexpr int kWorkWarps = kWarps - kWorkWarp0;
 constexpr float kLazy = 8.0f;                  // rescale threshold (log2 units)
 
 struct __align__(1024) Smem {
@@ -73,7 +76,6 @@ struct __align__(1024) Smem {
     uint8_t kv[kStages][kStageBytes];          // stage j: [2 cb][128 keys][128 B] swizzled
     uint8_t pt[kTK * 128];                     // P^T fp16, [128 keys][64 heads] swizzled
     int32_t ids[CSA2_TOPK_MAX];                // compacted selected entry ids
-    float ksig[kTK];                           // per key of the tile: 1 FP4, sigma SWA, -1 none
     alignas(16) uint8_t swa_new[kDim];         // fused append: the new SWA row (E4M3 codes)
     float swa_new_sigma;
     alignas(16) float red[2][4][32];           // softmax half hh: per quadrant warp, 32 heads
@@ -87,8 +89,8 @@ struct __align__(1024) Smem {
     uint64_t xfer;                             // combine: the peer's part has landed
     uint32_t tmem_base;
     int32_t abort;
-    float wred[16];
-    int32_t wcnt[16];
+    float wred[kWarps];
+    int32_t wcnt[2 * kWarps];
 };
 
 // ---- small PTX wrappers ---------------------------------------------------------------
@@ -190,22 +192,23 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v) {
+// 32 lanes x 16 columns, in place: v *= f (per column), read and written back.
+__device__ __forceinline__ void tmem_scale16(uint32_t taddr, const float *f) {
+    uint32_t r[16];
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
-        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
-        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
-        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
-        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f[i]);
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
@@ -280,13 +283,14 @@ __device__ __forceinline__ uint32_t swz(int row, int c) {
     return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4));
 }
 
-// ---- producer: one stage (128 channels) of one key -------------------------------------
-// The raw bytes of stage j of a key, gathered into registers one stage ahead.
+// ---- producer: a worker thread's channel half of one key, a whole tile ahead -----------
+// Worker thread (key r, half hh) owns channels 64 hh .. 64 hh + 63 of every 128-channel
+// stage of key r, i.e. the 128-byte row r of block hh of each stage.
 struct Raw {
-    uint4 c[8];      // FP4: c[0..3] = the stage's 64 code bytes; SWA / new row: c[0..7] = 128 codes
-    uint2 sc;        // FP4: the stage's 8 scale bytes (E4M3, one per 16 channels)
-    float sigma;     // SWA scale (stage 0)
-    int kind;        // 1 FP4 entry, 2 SWA row (ring or the fused new row), 0 zero row, -1 nothing
+    uint4 c[kStages][4];   // FP4: c[j][0..1] = the 64 codes of stage j; SWA: c[j][0..3] = 64 E4M3 codes
+    uint32_t sc[kStages];  // FP4: the stage's 4 scale bytes (E4M3, one per 16 channels)
+    float sigma;           // 1 for an FP4 entry, the row scale of an SWA row, -1 for no key
+    int kind;              // 1 FP4 entry, 2 SWA row (ring or the fused new row), 0 zero row, -1 nothing
 };
 
 struct KeyMap {      // this CTA's keys and where each comes from
@@ -300,63 +304,68 @@ struct KeyMap {      // this CTA's keys and where each comes from
     const uint8_t *new_row;   // fused append: the newest window key is this row (smem)
     const float *new_sigma;
     uint64_t *new_ready;      // ... written once this completes
-    bool *new_ok;
     const Smem *smem;
 };
 
-__device__ __forceinline__ void load_stage(Raw &r, const AttnArgs &a, const KeyMap &km, int kg, bool zrow,
-                                           int j) {
+// Issue every load of key kg's channel half for all four stages (one memory round trip).
+__device__ __forceinline__ void load_key(Raw &r, const AttnArgs &a, const KeyMap &km, int kg, bool zrow, int hh,
+                                         bool &new_ok) {
     r.kind = zrow ? 0 : -1;
-    if (kg < km.k_end) {
-        if (kg < km.n_sel) {
-            const int64_t off = cache_row(a.pm, a.cap, km.b, km.ids[kg]);   // checked when compacted
-            const uint4 *src = reinterpret_cast<const uint4 *>(a.codes + off * kCodeBytes + 64 * j);
+    r.sigma = -1.0f;
+    if (kg >= km.k_end) return;
+    if (kg < km.n_sel) {
+        const int64_t off = cache_row(a.pm, a.cap, km.b, km.ids[kg]);   // checked when compacted
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.codes + off * kCodeBytes + 32 * hh);
+        const uint32_t *sc = reinterpret_cast<const uint32_t *>(a.scales + off * kScaleBytes + 4 * hh);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) r.c[u] = __ldg(src + u);
-            r.sc = __ldg(reinterpret_cast<const uint2 *>(a.scales + off * kScaleBytes + 8 * j));
-            r.kind = 1;
-        } else if (km.new_row != nullptr && kg == km.n_keys - 1) {
-            if (!*km.new_ok) {
-                *km.new_ok = mbar_wait(km.new_ready, 0, a.wait.limit_ns, *km.smem);
-                if (!*km.new_ok) {
-                    set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
-                    r.kind = 0;
-                    return;
-                }
-            }
-            const uint4 *src = reinterpret_cast<const uint4 *>(km.new_row + 128 * j);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) r.c[u] = src[u];
-            r.sigma = *km.new_sigma;
-            r.kind = 2;
-        } else {
-            const int64_t pos = km.w0 + (kg - km.n_sel);
-            const int64_t slot = km.ring_base + pos % a.wcap;
-            const uint4 *src = reinterpret_cast<const uint4 *>(a.swa_codes + slot * kDim + 128 * j);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) r.c[u] = __ldg(src + u);
-            r.sigma = j == 0 ? __ldg(a.swa_scale + slot) : 0.0f;
-            r.kind = 2;
+        for (int j = 0; j < kStages; ++j) {
+            r.c[j][0] = __ldg(src + 4 * j);
+            r.c[j][1] = __ldg(src + 4 * j + 1);
+            r.sc[j] = __ldg(sc + 2 * j);
         }
+        r.kind = 1;
+        r.sigma = 1.0f;
+    } else if (km.new_row != nullptr && kg == km.n_keys - 1) {
+        if (!new_ok) {
+            new_ok = mbar_wait(km.new_ready, 0, a.wait.limit_ns, *km.smem);
+            if (!new_ok) {
+                set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+                r.kind = 0;
+                return;
+            }
+        }
+        const uint4 *src = reinterpret_cast<const uint4 *>(km.new_row + 64 * hh);
+#pragma unroll
+        for (int j = 0; j < kStages; ++j)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) r.c[j][u] = src[8 * j + u];
+        r.sigma = *km.new_sigma;
+        r.kind = 2;
+    } else {
+        const int64_t pos = km.w0 + (kg - km.n_sel);
+        const int64_t slot = km.ring_base + pos % a.wcap;
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.swa_codes + slot * kDim + 64 * hh);
+#pragma unroll
+        for (int j = 0; j < kStages; ++j)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) r.c[j][u] = __ldg(src + 8 * j + u);
+        r.sigma = __ldg(a.swa_scale + slot);
+        r.kind = 2;
     }
 }
 
-// Dequantise the thread's key row of one stage into shared memory (fp16, swizzled).
-__device__ __forceinline__ void store_stage(const Raw &r, uint8_t *stage, int row) {
+// Dequantise stage j of the thread's key half into row `row` of block hh (fp16, swizzled).
+__device__ __forceinline__ void store_half(const Raw &r, int j, uint8_t *stage, int row, int hh) {
+    uint8_t *blk = stage + hh * kCbBytes;
     if (r.kind == 1) {
-        uint32_t scale2[8];                            // f16x2 scale of each 16 channels
+        const uint32_t lo = cvt_e4m3x2_f16x2(r.sc[j] & 0xFFFFu), hi = cvt_e4m3x2_f16x2(r.sc[j] >> 16);
+        const uint32_t scale2[4] = {(lo & 0xFFFFu) * 0x10001u, (lo >> 16) * 0x10001u, (hi & 0xFFFFu) * 0x10001u,
+                                    (hi >> 16) * 0x10001u};   // f16x2 scale of each 16 channels
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-            const uint32_t sw = g < 2 ? r.sc.x : r.sc.y;
-            const uint32_t hh = cvt_e4m3x2_f16x2((sw >> (16 * (g & 1))) & 0xFFFFu);
-            scale2[2 * g] = (hh & 0xFFFFu) * 0x10001u;
-            scale2[2 * g + 1] = (hh >> 16) * 0x10001u;
-        }
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {                 // 8 channels per 32-bit code word
-            const uint4 cv = r.c[u >> 2];
-            const uint32_t w = (u & 3) == 0 ? cv.x : (u & 3) == 1 ? cv.y : (u & 3) == 2 ? cv.z : cv.w;
-            const __half2 sv = *reinterpret_cast<const __half2 *>(&scale2[u >> 1]);
+        for (int c = 0; c < 8; ++c) {                  // 8 channels per 32-bit code word
+            const uint4 cv = r.c[j][c >> 2];
+            const uint32_t w = (c & 3) == 0 ? cv.x : (c & 3) == 1 ? cv.y : (c & 3) == 2 ? cv.z : cv.w;
+            const __half2 sv = *reinterpret_cast<const __half2 *>(&scale2[c >> 1]);
             uint32_t v[4];
             cvt_e2m1x8_f16x2(w, v);
 #pragma unroll
@@ -364,23 +373,22 @@ __device__ __forceinline__ void store_stage(const Raw &r, uint8_t *stage, int ro
                 __half2 x = __hmul2(*reinterpret_cast<__half2 *>(&v[k]), sv);
                 v[k] = *reinterpret_cast<uint32_t *>(&x);
             }
-            *reinterpret_cast<uint4 *>(stage + (u >> 3) * kCbBytes + swz(row, u & 7)) =
-                make_uint4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<uint4 *>(blk + swz(row, c)) = make_uint4(v[0], v[1], v[2], v[3]);
         }
     } else if (r.kind == 2) {
         // exact E4M3 codes; the row scale is applied in fp32 on the logit and on P
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {                 // 8 channels = 8 code bytes
-            const uint4 cv = r.c[u >> 1];
-            const uint32_t w0 = (u & 1) ? cv.z : cv.x, w1 = (u & 1) ? cv.w : cv.y;
-            *reinterpret_cast<uint4 *>(stage + (u >> 3) * kCbBytes + swz(row, u & 7)) =
+        for (int c = 0; c < 8; ++c) {                  // 8 channels = 8 code bytes
+            const uint4 cv = r.c[j][c >> 1];
+            const uint32_t w0 = (c & 1) ? cv.z : cv.x, w1 = (c & 1) ? cv.w : cv.y;
+            *reinterpret_cast<uint4 *>(blk + swz(row, c)) =
                 make_uint4(cvt_e4m3x2_f16x2(w0 & 0xFFFFu), cvt_e4m3x2_f16x2(w0 >> 16),
                            cvt_e4m3x2_f16x2(w1 & 0xFFFFu), cvt_e4m3x2_f16x2(w1 >> 16));
         }
     } else if (r.kind == 0) {
         const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) *reinterpret_cast<uint4 *>(stage + (u >> 3) * kCbBytes + swz(row, u & 7)) = z;
+        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(blk + swz(row, c)) = z;
     }
 }
 
@@ -427,12 +435,12 @@ attn_kernel(AttnArgs a) {
     // ---- set-up -----------------------------------------------------------------------------
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&s.kv_full[i], 4);
+            mbar_init(&s.kv_full[i], kWorkWarps);
             mbar_init(&s.kv_empty[i], 1);
         }
         mbar_init(&s.s_full[0], 1);
         mbar_init(&s.s_full[1], 1);
-        mbar_init(&s.p_full, 8);
+        mbar_init(&s.p_full, kWorkWarps);
         mbar_init(&s.pv_done, 1);
         mbar_init(&s.drain, 1);
         mbar_init(&s.never, 1);
@@ -451,15 +459,18 @@ attn_kernel(AttnArgs a) {
     // previous kernel of the stream wrote
     grid_dep_wait();
     // every independent global load first (one memory round trip): the position, this
-    // thread's Top-K entry, its Q chunks and (warp 1, fused append) the new SWA row
+    // thread's two Top-K slots, its Q chunks and (warp 1, fused append) the new SWA row
     const int32_t t32 = a.q_pos[qi];
-    const int e_id = (int)threadIdx.x < a.top_k ? a.topk[(int64_t)qi * a.top_k + threadIdx.x] : -1;
+    const int *tk = a.topk + (int64_t)qi * a.top_k;
+    const int e_id0 = (int)threadIdx.x < a.top_k ? tk[threadIdx.x] : -1;
+    const int e_id1 = (int)threadIdx.x + kThreads < a.top_k ? tk[threadIdx.x + kThreads] : -1;
     const uint16_t *q = a.q + ((int64_t)qi * a.H + h0) * kDim;
-    uint4 qv[8];        // chunk i = threadIdx.x + 512 k: head i / 64, channels 8 (i % 64) .. + 7
+    uint4 qv[kQChunks];   // chunk i = threadIdx.x + kThreads k: head i / 64, channels 8 (i % 64) .. + 7
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < kQChunks; ++k) {
         const int i = threadIdx.x + kThreads * k;
-        qv[k] = (i / 64 < hcta) ? __ldg(reinterpret_cast<const uint4 *>(q) + i) : make_uint4(0u, 0u, 0u, 0u);
+        qv[k] = (i < kHeads * 64 && i / 64 < hcta) ? __ldg(reinterpret_cast<const uint4 *>(q) + i)
+                                                   : make_uint4(0u, 0u, 0u, 0u);
     }
     uint4 xraw[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
     if (a.swa_new != nullptr && warp == 1) {
@@ -471,15 +482,16 @@ attn_kernel(AttnArgs a) {
     const int64_t w0 = max64(0, t - a.swa_len + 1);
     const int n_win = a.swa_len > 0 ? (int)(t - w0 + 1) : 0;
     const int64_t n_vis = min64(visible_entries((int32_t)t, a.ratio), a.cap);
-    bool e_ok = e_id >= 0 && e_id < n_vis;
-    if (e_id >= 0 && !e_ok) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
-    if (e_ok) {
-        const int64_t row = cache_row(a.pm, a.cap, b, e_id);
-        if (row < 0) {
+    auto entry_ok = [&](int e) {
+        bool ok = e >= 0 && e < n_vis;
+        if (e >= 0 && !ok) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
+        if (ok && cache_row(a.pm, a.cap, b, e) < 0) {
             set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
-            e_ok = false;
+            ok = false;
         }
-    }
+        return ok;
+    };
+    const bool e_ok0 = entry_ok(e_id0), e_ok1 = entry_ok(e_id1);
     if (threadIdx.x == 32 * 3 && a.swa_len > 0 && rank == 0) {
         // the request's whole SWA ring (rows are contiguous) and its scales
         prefetch_l2(a.swa_codes + (int64_t)b * a.wcap * kDim, (uint32_t)a.wcap * kDim);
@@ -487,10 +499,10 @@ attn_kernel(AttnArgs a) {
         if ((reinterpret_cast<uintptr_t>(sg) & 15) == 0 && (a.wcap & 3) == 0)
             prefetch_l2(sg, (uint32_t)a.wcap * 4);
     }
-    const uint32_t bal = __ballot_sync(0xFFFFFFFFu, e_ok);
+    const uint32_t bal0 = __ballot_sync(0xFFFFFFFFu, e_ok0), bal1 = __ballot_sync(0xFFFFFFFFu, e_ok1);
     float qm = 0.0f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < kQChunks; ++k) {
         const uint32_t w[4] = {qv[k].x, qv[k].y, qv[k].z, qv[k].w};
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -498,19 +510,27 @@ attn_kernel(AttnArgs a) {
     }
     qm = warp_max(qm);
     if (lane == 0) {
-        s.wcnt[warp] = __popc(bal);
+        s.wcnt[warp] = __popc(bal0);
+        s.wcnt[kWarps + warp] = __popc(bal1);
         s.wred[warp] = qm;
     }
     __syncthreads();
-    int base = 0, n_sel = 0;
+    // compaction in Top-K slot order: slots [0, kThreads) by warp, then [kThreads, 2 kThreads)
+    int base0 = 0, base1 = 0, n_sel = 0;
     float qmax = 0.0f;
 #pragma unroll
-    for (int w = 0; w < 16; ++w) {
-        base += w < warp ? s.wcnt[w] : 0;
+    for (int w = 0; w < kWarps; ++w) {
+        base0 += w < warp ? s.wcnt[w] : 0;
+        base1 += w < warp ? s.wcnt[kWarps + w] : 0;
         n_sel += s.wcnt[w];
         qmax = fmaxf(qmax, s.wred[w]);
     }
-    if (e_ok) s.ids[base + __popc(bal & ((1u << lane) - 1u))] = e_id;
+    base1 += n_sel;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) n_sel += s.wcnt[kWarps + w];
+    const uint32_t below = (1u << lane) - 1u;
+    if (e_ok0) s.ids[base0 + __popc(bal0 & below)] = e_id0;
+    if (e_ok1) s.ids[base1 + __popc(bal1 & below)] = e_id1;
     // this CTA's key range: the query's keys cut in two at a multiple of 16
     const int n_keys = n_sel + n_win;
     const int k_split = min(n_keys, ((n_keys + 1) / 2 + 15) / 16 * 16);
@@ -519,11 +539,33 @@ attn_kernel(AttnArgs a) {
     const bool fuse = a.swa_new != nullptr && n_win > 0;
     const uint32_t owner = (n_keys - 1) < k_split ? 0u : 1u;   // the CTA holding the newest key
     const int qexp = qmax > 0.0f ? max(0, ilogbf(qmax) - 14) : 0;   // max|q| * 2^-qexp < 2^15
+    KeyMap km;
+    km.ids = s.ids;
+    km.n_sel = n_sel;
+    km.w0 = w0;
+    km.n_keys = n_keys;
+    km.k_end = k1;
+    km.b = b;
+    km.ring_base = (int64_t)b * a.wcap;
+    km.new_row = fuse && rank == owner ? s.swa_new : nullptr;
+    km.new_sigma = &s.swa_new_sigma;
+    km.new_ready = &s.new_ready;
+    km.smem = &s;
+    const bool worker = warp >= kWorkWarp0;
+    const int qd = warp & 3, hh = (warp - kWorkWarp0) >> 2;   // worker: key quadrant, head / channel half
+    const int r = 32 * qd + lane;                              // worker: key of the tile
+    // rows of the tile's last 16-key group of valid keys are read by the output MMAs
+    // and so written (zeros past the keys); rows after that group are not written
+    auto zrow_of = [&](int i) { return r < ((min(kTK, k1 - k0 - i * kTK) + 15) / 16) * 16; };
+    bool new_ok = false;
+    Raw raw;
+    __syncthreads();                       // s.ids complete
     {
         const float inv = exp2f((float)-qexp);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < kQChunks; ++k) {
             const int i = threadIdx.x + kThreads * k;
+            if (i >= kHeads * 64) break;
             const int hd = i / 64, ch8 = i % 64;
             const uint32_t w[4] = {qv[k].x, qv[k].y, qv[k].z, qv[k].w};
             uint32_t h[4];
@@ -534,6 +576,7 @@ attn_kernel(AttnArgs a) {
                 make_uint4(h[0], h[1], h[2], h[3]);
         }
     }
+    if (worker && nt > 0) load_key(raw, a, km, k0 + r, zrow_of(0), hh, new_ok);   // tile 0, in flight
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -549,7 +592,7 @@ attn_kernel(AttnArgs a) {
             // O^T = V^T P^T: A = stage (MN-major, 128 channels), B = P^T (MN-major, 64 heads)
             const uint32_t idesc_o = (1u << 4) | (1u << 15) | (1u << 16) | ((uint32_t)(kHeads >> 3) << 17) |
                                      ((uint32_t)(kTK >> 4) << 24);
-            const uint64_t qd = sw128_desc(smem_u32(s.q), 16, 1024);
+            const uint64_t qd_desc = sw128_desc(smem_u32(s.q), 16, 1024);
             const uint64_t pd = sw128_desc(smem_u32(s.pt), 8192, 1024);
             for (int i = 0; ok && i < nt; ++i) {
                 const uint32_t sd = tmem + kSCol + 64u * (uint32_t)(i & 1);
@@ -564,7 +607,7 @@ attn_kernel(AttnArgs a) {
                         for (int k = 0; k < 8; ++k) {       // K-steps of 16 channels
                             const uint64_t aoff = (uint64_t)((k >> 2) * (kCbBytes >> 4) + (k & 3) * 2);
                             const uint64_t boff = (uint64_t)((2 * j + (k >> 2)) * (kQCbBytes >> 4) + (k & 3) * 2);
-                            mma_f16(sd, kd + aoff, qd + boff, idesc_s, (j | k) != 0 ? 1u : 0u);
+                            mma_f16(sd, kd + aoff, qd_desc + boff, idesc_s, (j | k) != 0 ? 1u : 0u);
                         }
                         if (j == kStages - 1) mma_commit(&s.s_full[i & 1]);
                     }
@@ -604,7 +647,7 @@ attn_kernel(AttnArgs a) {
     } else if (warp == 1) {
         if (fuse && rank == owner) {
             // The same FP8 row quantiser as csa2_quantize_append: codes and sigma go to
-            // shared memory (this CTA's producers read the window's newest key from there,
+            // shared memory (this CTA's workers read the window's newest key from there,
             // after new_ready) and, from head group 0, to the ring slot t % wcap.
             float xnew[16];
             unpack_bf16x8(xraw[0], xnew);
@@ -625,39 +668,52 @@ attn_kernel(AttnArgs a) {
             }
         }
     } else if (warp == 2) {
-        // L2 prefetch of the entries of this CTA's later tiles (tile 0 the producers fetch
-        // at once)
+        // L2 prefetch of the entries of this CTA's later tiles (tile 0 is already in flight)
         for (int kg = k0 + kTK + lane; kg < min(k1, n_sel); kg += 32) {
             const int64_t row = cache_row(a.pm, a.cap, b, s.ids[kg]);
             prefetch_l2(a.codes + row * kCodeBytes, kCodeBytes);
             prefetch_l2(a.scales + row * kScaleBytes, kScaleBytes);
         }
-    } else if (warp >= kSoftWarp0 && warp < kProdWarp0) {
-        // ---------------- softmax: keys 32 qd .. (TMEM lanes), heads 32 hh .. ----------------
-        const int qd = warp & 3, hh = (warp - kSoftWarp0) >> 2;
-        const int r = 32 * qd + lane;                           // key of the tile
+    } else if (worker) {
+        // ---------------- workers: produce tile i + 1 after the softmax of tile i ----------------
+        // Softmax: keys 32 qd .. (TMEM lanes), heads 32 hh .. .  Producer: key r, channel
+        // half hh of every stage; the raw bytes of the next tile are in registers while the
+        // softmax of this one runs.
         const float c0 = a.softmax_scale * 1.4426950408889634f * exp2f((float)qexp);
         const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
-        // the running max lives in shared memory (s.mrun, identical for the four warps
-        // of the half); the partial sums per head in registers
-        float l[32];
-#pragma unroll
-        for (int h = 0; h < 32; ++h) l[h] = 0.0f;
         const float4 *mrun4 = reinterpret_cast<const float4 *>(&s.mrun[32 * hh]);
-        bool stop = false;
+        float lsum = 0.0f;   // head 32 hh + lane: partial sum over this warp's keys
+        float sig = -1.0f;   // the current tile's key: 1 FP4, sigma SWA, -1 none
+        bool ok = true, stop = false;
         for (int i = 0; i < nt; ++i) {
-            // every wait of the tile first; the four warps of the half then agree
-            const bool w_ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.s_full[i & 1], (i >> 1) & 1, lim, s) &&
-                                                          mbar_wait(&s.kv_full[0], i & 1, lim, s) &&
-                                                          (i == 0 || mbar_wait(&s.pv_done, (i - 1) & 1, lim, s)));
+            // ---- produce tile i (its stages are free once O^T(i - 1) has read them) ----
+            if (ok) {
+#pragma unroll
+                for (int j = 0; j < kStages; ++j) {   // unrolled: raw.c[j] stays in registers
+                    if (i > 0) {
+                        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.kv_empty[j], (i - 1) & 1, lim, s));
+                        if (!ok) break;
+                    }
+                    store_half(raw, j, s.kv[j], r, hh);
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.kv_full[j]);
+                }
+                sig = raw.sigma;
+                // P carries sigma in fp16: p <= 2^8 needs sigma <= 65504 / 256
+                if (raw.kind == 2 && hh == 0 && sig * 256.0f > 65504.0f) set_dev_err(a.dev_err, CSA2_DEVERR_RANGE);
+                if (ok && i + 1 < nt) load_key(raw, a, km, k0 + (i + 1) * kTK + r, zrow_of(i + 1), hh, new_ok);
+            }
+            // ---- softmax of tile i: every wait first; the four warps of the half agree ----
+            const bool w_ok = ok && __all_sync(0xFFFFFFFFu, mbar_wait(&s.s_full[i & 1], (i >> 1) & 1, lim, s) &&
+                                                                (i == 0 || mbar_wait(&s.pv_done, (i - 1) & 1, lim, s)));
             stop = group_any(hh, !w_ok || aborted(s));
             if (stop) break;
             tc_fence_after();
             float x[32];
             tmem_ld32(tmem + lane_base + kSCol + 64u * (uint32_t)(i & 1) + 32u * (uint32_t)hh, x);
-            const float sg = s.ksig[r];
-            const bool valid = sg >= 0.0f;
-            const float ck = c0 * sg;
+            const bool valid = sig >= 0.0f;
+            const float ck = c0 * sig;
             float dmax = -INFINITY;
 #pragma unroll
             for (int h = 0; h < 32; ++h) x[h] = valid ? x[h] * ck : -INFINITY;
@@ -684,24 +740,20 @@ attn_kernel(AttnArgs a) {
                     s.alpha[32 * hh + lane] = old == -INFINITY ? 0.0f : ex2(old - mn);
                 }
                 group_sync(hh);
-#pragma unroll
-                for (int h4 = 0; h4 < 8; ++h4) {
-                    const float4 av = reinterpret_cast<const float4 *>(&s.alpha[32 * hh])[h4];
-                    l[4 * h4] *= av.x; l[4 * h4 + 1] *= av.y; l[4 * h4 + 2] *= av.z; l[4 * h4 + 3] *= av.w;
-                }
+                lsum *= s.alpha[32 * hh + lane];
             }
             // p = 2^(x - m); P^T carries the key's scale (V holds SWA codes, not values)
-            const float sv = valid ? sg : 0.0f;
+            const float sv = valid ? sig : 0.0f;
             uint32_t pk[16];
 #pragma unroll
             for (int h4 = 0; h4 < 8; ++h4) {
                 const float4 mv = mrun4[h4];
                 const float p0 = ex2(x[4 * h4] - mv.x), p1 = ex2(x[4 * h4 + 1] - mv.y);
                 const float p2 = ex2(x[4 * h4 + 2] - mv.z), p3 = ex2(x[4 * h4 + 3] - mv.w);
-                l[4 * h4] += p0;
-                l[4 * h4 + 1] += p1;
-                l[4 * h4 + 2] += p2;
-                l[4 * h4 + 3] += p3;
+                x[4 * h4] = p0;
+                x[4 * h4 + 1] = p1;
+                x[4 * h4 + 2] = p2;
+                x[4 * h4 + 3] = p3;
                 pk[2 * h4] = pack_h2(p0 * sv, p1 * sv);
                 pk[2 * h4 + 1] = pack_h2(p2 * sv, p3 * sv);
             }
@@ -709,20 +761,16 @@ attn_kernel(AttnArgs a) {
             for (int c = 0; c < 4; ++c)
                 *reinterpret_cast<uint4 *>(s.pt + swz(r, 4 * hh + c)) =
                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            lsum += reduce_scatter32<false>(x, lane);   // this tile's 32 keys, head 32 hh + lane
             if (upd && i > 0) {
                 // the running max moved: O^T(i - 1) has landed (pv_done above); scale this
                 // warp's 32 head columns of every block before O^T(i) accumulates on them
 #pragma unroll 1
-                for (int j = 0; j < kStages; ++j) {
-                    float o[32];
-                    const uint32_t oa = tmem + lane_base + 64u * (uint32_t)j + 32u * (uint32_t)hh;
-                    tmem_ld32(oa, o);
+                for (int j = 0; j < 2 * kStages; ++j) {    // 16 head columns at a time
+                    float f[16];
 #pragma unroll
-                    for (int h4 = 0; h4 < 8; ++h4) {
-                        const float4 av = reinterpret_cast<const float4 *>(&s.alpha[32 * hh])[h4];
-                        o[4 * h4] *= av.x; o[4 * h4 + 1] *= av.y; o[4 * h4 + 2] *= av.z; o[4 * h4 + 3] *= av.w;
-                    }
-                    tmem_st32(oa, o);
+                    for (int h = 0; h < 16; ++h) f[h] = s.alpha[32 * hh + 16 * (j & 1) + h];
+                    tmem_scale16(tmem + lane_base + 64u * (uint32_t)(j >> 1) + 32u * (uint32_t)hh + 16u * (uint32_t)(j & 1), f);
                 }
                 asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             }
@@ -731,7 +779,7 @@ attn_kernel(AttnArgs a) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.p_full);
         }
-        bool ok = !stop;
+        ok = ok && !stop;
         if (ok && nt > 0) {
             ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.pv_done, (nt - 1) & 1, lim, s));
             tc_fence_after();
@@ -740,10 +788,9 @@ attn_kernel(AttnArgs a) {
             atomicExch(&s.abort, 1);
             set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
         }
-        // this CTA's partial sum per head: over the warp's keys, then the four quadrants
-        // (the group barrier is taken by all four warps of the half, aborted or not)
-        const float ls = reduce_scatter32<false>(l, lane);
-        s.red[hh][qd][lane] = ls;
+        // this CTA's partial sum per head: the four quadrants' sums (the group barrier is
+        // taken by all four warps of the half, aborted or not)
+        s.red[hh][qd][lane] = lsum;
         group_sync(hh);
         if (qd == 0) {
             const bool have = nt > 0 && !aborted(s);
@@ -751,59 +798,6 @@ attn_kernel(AttnArgs a) {
                                               s.red[hh][3][lane]
                                         : 0.0f;
             s.cm[32 * hh + lane] = have ? s.mrun[32 * hh + lane] : -INFINITY;
-        }
-    } else if (warp >= kProdWarp0) {
-        // ---------------- producers: thread = key row r of the tile ----------------
-        const int r = threadIdx.x - 32 * kProdWarp0;
-        KeyMap km;
-        km.ids = s.ids;
-        km.n_sel = n_sel;
-        km.w0 = w0;
-        km.n_keys = n_keys;
-        km.k_end = k1;
-        km.b = b;
-        km.ring_base = (int64_t)b * a.wcap;
-        bool new_ok = false;
-        km.new_row = fuse && rank == owner ? s.swa_new : nullptr;
-        km.new_sigma = &s.swa_new_sigma;
-        km.new_ready = &s.new_ready;
-        km.new_ok = &new_ok;
-        km.smem = &s;
-        // rows of the tile's last 16-key group of valid keys are read by the output MMAs
-        // and so written (zeros past the keys); rows after that group are not written
-        auto zrow_of = [&](int i) { return r < ((min(kTK, k1 - k0 - i * kTK) + 15) / 16) * 16; };
-        Raw cur, nxt;
-        if (nt > 0) load_stage(nxt, a, km, k0 + r, zrow_of(0), 0);
-        bool ok = true;
-        for (int i = 0; ok && i < nt; ++i) {
-            const int kg = k0 + i * kTK + r;
-            float sig = -1.0f;
-#pragma unroll 1
-            for (int j = 0; j < kStages; ++j) {
-                cur = nxt;
-                if (j + 1 < kStages)
-                    load_stage(nxt, a, km, kg, zrow_of(i), j + 1);
-                else if (i + 1 < nt)
-                    load_stage(nxt, a, km, kg + kTK, zrow_of(i + 1), 0);
-                if (j == 0) sig = cur.kind == 1 ? 1.0f : cur.kind == 2 ? cur.sigma : -1.0f;
-                if (i > 0) {
-                    ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.kv_empty[j], (i - 1) & 1, lim, s));
-                    if (!ok) break;
-                }
-                store_stage(cur, s.kv[j], r);
-                if (j == 0) {
-                    // P carries sigma in fp16: p <= 2^8 needs sigma <= 65504 / 256
-                    if (cur.kind == 2 && sig * 256.0f > 65504.0f) set_dev_err(a.dev_err, CSA2_DEVERR_RANGE);
-                    s.ksig[r] = sig;
-                }
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s.kv_full[j]);
-            }
-        }
-        if (!ok && lane == 0) {
-            atomicExch(&s.abort, 1);
-            set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
         }
     }
 
@@ -839,18 +833,19 @@ attn_kernel(AttnArgs a) {
             a.lse[(int64_t)qi * a.H + h0 + h] = valid ? (m_all + log2f(l_all)) * 0.6931471805599453f : -INFINITY;
     }
     __syncthreads();
-    // Warp w: TMEM lane quadrant w % 4 (channels 32 (w % 4) .. of a block), head half
-    // (w >> 2) & 1, block pair member w >> 3.  The peer's blocks, scaled, are staged in
-    // local shared memory (`send`, [2 blocks][128 channels][64 heads] fp32, float4 slots
-    // swizzled by channel) and moved by one bulk copy into the peer's `recv`; own blocks
-    // wait in registers.
+    // Combine task u (16 of them, warp u % 12 takes u; TMEM lane quadrant u % 4 = warp % 4):
+    // channels 32 (u % 4) .. of a block, head half (u >> 2) & 1, block pair member u >> 3.
+    // The peer's blocks, scaled, are staged in local shared memory (`send`, [2 blocks][128
+    // channels][64 heads] fp32, float4 slots swizzled by channel) and moved by one bulk
+    // copy into the peer's `recv`.
     const bool have = __shfl_sync(0xFFFFFFFFu, (int)(nt > 0 && !aborted(s)), 0) != 0;
-    const int cq = warp & 3, chh = (warp >> 2) & 1, bsel = warp >> 3;
-    const int crow = 32 * cq + lane;                 // channel within a block
     float *send = reinterpret_cast<float *>(&s.kv[0][0]);
     float *recv = reinterpret_cast<float *>(&s.kv[2][0]);
-    const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)chh;
-    {
+#pragma unroll 1
+    for (int u = warp; u < 16; u += kWarps) {
+        const int cq = u & 3, chh = (u >> 2) & 1, bsel = u >> 3;
+        const int crow = 32 * cq + lane;             // channel within a block
+        const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)chh;
         float o[32];
         if (have) {
             tmem_ld32(taddr + 64u * (uint32_t)(2 * (int)peer + bsel), o);
@@ -873,16 +868,20 @@ attn_kernel(AttnArgs a) {
         bulk_copy_to_peer(dst, send, kXfer / 2, bar);
         bulk_copy_to_peer(dst + kXfer / 2, reinterpret_cast<uint8_t *>(send) + kXfer / 2, kXfer / 2, bar);
     }
-    float own[32];
-    if (have) {
-        tmem_ld32(taddr + 64u * (uint32_t)(2 * (int)rank + bsel), own);
-    } else {
-#pragma unroll
-        for (int h = 0; h < 32; ++h) own[h] = 0.0f;
-    }
     const bool got = __syncthreads_and(mbar_wait<false>(&s.xfer, 0, kDrainLimitNs, s)) != 0;
     if (!got && threadIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
-    {
+#pragma unroll 1
+    for (int u = warp; u < 16; u += kWarps) {
+        const int cq = u & 3, chh = (u >> 2) & 1, bsel = u >> 3;
+        const int crow = 32 * cq + lane;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)chh;
+        float own[32];
+        if (have) {
+            tmem_ld32(taddr + 64u * (uint32_t)(2 * (int)rank + bsel), own);
+        } else {
+#pragma unroll
+            for (int h = 0; h < 32; ++h) own[h] = 0.0f;
+        }
         const int blk = 2 * (int)rank + bsel;
         const float4 *src = reinterpret_cast<const float4 *>(recv + (bsel * kTK + crow) * kHeads);
         float *obase = a.out + ((int64_t)qi * a.H + h0) * kDim + 128 * blk + crow;
