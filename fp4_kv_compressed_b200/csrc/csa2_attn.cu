@@ -290,7 +290,8 @@ struct Raw {
     uint4 c[kStages][4];   // FP4: c[j][0..1] = the 64 codes of stage j; SWA: c[j][0..3] = 64 E4M3 codes
     uint32_t sc[kStages];  // FP4: the stage's 4 scale bytes (E4M3, one per 16 channels)
     float sigma;           // 1 for an FP4 entry, the row scale of an SWA row, -1 for no key
-    int kind;              // 1 FP4 entry, 2 SWA row (ring or the fused new row), 0 zero row, -1 nothing
+    int kind;              // 1 FP4 entry, 2 SWA row, 3 the fused new SWA row (not yet read), 0 zero row,
+                           // -1 nothing
 };
 
 struct KeyMap {      // this CTA's keys and where each comes from
@@ -308,8 +309,8 @@ struct KeyMap {      // this CTA's keys and where each comes from
 };
 
 // Issue every load of key kg's channel half for all four stages (one memory round trip).
-__device__ __forceinline__ void load_key(Raw &r, const AttnArgs &a, const KeyMap &km, int kg, bool zrow, int hh,
-                                         bool &new_ok) {
+// The fused new SWA row is only marked here (kind 3): see take_new_row.
+__device__ __forceinline__ void load_key(Raw &r, const AttnArgs &a, const KeyMap &km, int kg, bool zrow, int hh) {
     r.kind = zrow ? 0 : -1;
     r.sigma = -1.0f;
     if (kg >= km.k_end) return;
@@ -326,21 +327,7 @@ __device__ __forceinline__ void load_key(Raw &r, const AttnArgs &a, const KeyMap
         r.kind = 1;
         r.sigma = 1.0f;
     } else if (km.new_row != nullptr && kg == km.n_keys - 1) {
-        if (!new_ok) {
-            new_ok = mbar_wait(km.new_ready, 0, a.wait.limit_ns, *km.smem);
-            if (!new_ok) {
-                set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
-                r.kind = 0;
-                return;
-            }
-        }
-        const uint4 *src = reinterpret_cast<const uint4 *>(km.new_row + 64 * hh);
-#pragma unroll
-        for (int j = 0; j < kStages; ++j)
-#pragma unroll
-            for (int u = 0; u < 4; ++u) r.c[j][u] = src[8 * j + u];
-        r.sigma = *km.new_sigma;
-        r.kind = 2;
+        r.kind = 3;   // read from shared memory when stored, once warp 1 has written it
     } else {
         const int64_t pos = km.w0 + (kg - km.n_sel);
         const int64_t slot = km.ring_base + pos % a.wcap;
@@ -352,6 +339,25 @@ __device__ __forceinline__ void load_key(Raw &r, const AttnArgs &a, const KeyMap
         r.sigma = __ldg(a.swa_scale + slot);
         r.kind = 2;
     }
+}
+
+// Kind 3 -> 2: the fused new SWA row, once warp 1 has quantised it into shared memory
+// (bounded wait; on timeout the key is dropped as a zero row and flagged).
+__device__ __forceinline__ void take_new_row(Raw &r, const AttnArgs &a, const KeyMap &km, int hh, bool &new_ok) {
+    if (!new_ok) new_ok = mbar_wait(km.new_ready, 0, a.wait.limit_ns, *km.smem);
+    if (!new_ok) {
+        set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+        r.kind = 0;
+        r.sigma = -1.0f;
+        return;
+    }
+    const uint4 *src = reinterpret_cast<const uint4 *>(km.new_row + 64 * hh);
+#pragma unroll
+    for (int j = 0; j < kStages; ++j)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) r.c[j][u] = src[8 * j + u];
+    r.sigma = *km.new_sigma;
+    r.kind = 2;
 }
 
 // Dequantise stage j of the thread's key half into row `row` of block hh (fp16, swizzled).
@@ -576,7 +582,7 @@ attn_kernel(AttnArgs a) {
                 make_uint4(h[0], h[1], h[2], h[3]);
         }
     }
-    if (worker && nt > 0) load_key(raw, a, km, k0 + r, zrow_of(0), hh, new_ok);   // tile 0, in flight
+    if (worker && nt > 0) load_key(raw, a, km, k0 + r, zrow_of(0), hh);   // tile 0, in flight
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -688,6 +694,7 @@ attn_kernel(AttnArgs a) {
         for (int i = 0; i < nt; ++i) {
             // ---- produce tile i (its stages are free once O^T(i - 1) has read them) ----
             if (ok) {
+                if (raw.kind == 3) take_new_row(raw, a, km, hh, new_ok);
 #pragma unroll
                 for (int j = 0; j < kStages; ++j) {   // unrolled: raw.c[j] stays in registers
                     if (i > 0) {
@@ -702,7 +709,7 @@ attn_kernel(AttnArgs a) {
                 sig = raw.sigma;
                 // P carries sigma in fp16: p <= 2^8 needs sigma <= 65504 / 256
                 if (raw.kind == 2 && hh == 0 && sig * 256.0f > 65504.0f) set_dev_err(a.dev_err, CSA2_DEVERR_RANGE);
-                if (ok && i + 1 < nt) load_key(raw, a, km, k0 + (i + 1) * kTK + r, zrow_of(i + 1), hh, new_ok);
+                if (ok && i + 1 < nt) load_key(raw, a, km, k0 + (i + 1) * kTK + r, zrow_of(i + 1), hh);
             }
             // ---- softmax of tile i: every wait first; the four warps of the half agree ----
             const bool w_ok = ok && __all_sync(0xFFFFFFFFu, mbar_wait(&s.s_full[i & 1], (i >> 1) & 1, lim, s) &&
