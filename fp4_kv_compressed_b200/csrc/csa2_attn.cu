@@ -29,12 +29,12 @@
 //   warp 1       fused append only: quantises the query token's new SWA row;
 //   warp 2       prefetches the entries of this CTA's later tiles into L2 (bulk prefetch;
 //                the set-up prefetches the request's SWA ring);
-//   warps 4-11   workers, two roles in turn.  Producer: thread = (key r of the tile,
-//                channel half hh of every 128-channel stage); the raw bytes of its half
-//                of the next tile's key are loaded into registers (one round trip for
-//                all four stages) before the softmax of this tile, and dequantised into
-//                stage j as soon as O^T of this tile has read it.  Softmax: warp w reads
-//                TMEM lane quadrant w % 4 (32 keys) and the 32 heads of half (w - 4) / 4.
+//   warps 4-11   workers, two roles in turn.  Producer: warp wi = w - 4 gathers keys
+//                16 wi .. 16 wi + 15 of the next tile warp-cooperatively (one load
+//                instruction = one 64-byte stage slice of 8 keys), all four stages in
+//                registers before the softmax of this tile, and dequantises stage j as
+//                soon as O^T of this tile has read it.  Softmax: warp w reads TMEM lane
+//                quadrant w % 4 (32 keys) and the 32 heads of half (w - 4) / 4.
 // TMEM (512 columns): O^T block j (channels 128 j .. 128 j + 127) at columns
 // 64 j .. 64 j + 63 (column = head); the two S^T buffers at columns 256 and 320.
 // Online softmax in the log2 domain with lazy rescaling: the running max of a head
@@ -76,6 +76,7 @@ struct __align__(1024) Smem {
     uint8_t kv[kStages][kStageBytes];          // stage j: [2 cb][128 keys][128 B] swizzled
     uint8_t pt[kTK * 128];                     // P^T fp16, [128 keys][64 heads] swizzled
     int32_t ids[CSA2_TOPK_MAX];                // compacted selected entry ids
+    float ksig[kTK];                           // per key of the tile: 1 FP4, sigma SWA, -1 none
     alignas(16) uint8_t swa_new[kDim];         // fused append: the new SWA row (E4M3 codes)
     float swa_new_sigma;
     alignas(16) float red[2][4][32];           // softmax half hh: per quadrant warp, 32 heads
@@ -283,15 +284,26 @@ __device__ __forceinline__ uint32_t swz(int row, int c) {
     return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4));
 }
 
-// ---- producer: a worker thread's channel half of one key, a whole tile ahead -----------
-// Worker thread (key r, half hh) owns channels 64 hh .. 64 hh + 63 of every 128-channel
-// stage of key r, i.e. the 128-byte row r of block hh of each stage.
+// ---- producer: warp-cooperative gather, a whole tile ahead ------------------------------
+// Worker warp wi (0..7) produces keys 16 wi .. 16 wi + 15 of a tile, as two groups of 8.
+// Lane l of a group handles key 4 ((l >> 3) & 1) + ((l & 7) >> 1) of the group and piece
+// p = 2 (l >> 4) + (l & 1) of every 128-channel stage: channels 32 p .. 32 p + 31, i.e.
+// chunks 4 (p & 1) .. + 3 of block p >> 1.  So one load instruction reads one 64-byte
+// stage slice of 8 keys (8 cache lines, not 32), and a quarter-warp's 16-byte shared
+// stores hit 4 consecutive rows x 2 chunk halves: 8 distinct bank groups.
+constexpr int kGroups = 2;         // key groups of 8 per worker warp and tile
+
+__device__ __forceinline__ int prod_key(int wi, int g, int lane) {   // key of the tile
+    return 16 * wi + 8 * g + 4 * ((lane >> 3) & 1) + ((lane & 7) >> 1);
+}
+__device__ __forceinline__ int prod_piece(int lane) { return 2 * (lane >> 4) + (lane & 1); }
+
 struct Raw {
-    uint4 c[kStages][4];   // FP4: c[j][0..1] = the 64 codes of stage j; SWA: c[j][0..3] = 64 E4M3 codes
-    uint32_t sc[kStages];  // FP4: the stage's 4 scale bytes (E4M3, one per 16 channels)
-    float sigma;           // 1 for an FP4 entry, the row scale of an SWA row, -1 for no key
-    int kind;              // 1 FP4 entry, 2 SWA row, 3 the fused new SWA row (not yet read), 0 zero row,
-                           // -1 nothing
+    uint4 c[kGroups][kStages][2];   // FP4: c[g][j][0] = 32 codes of stage j; SWA: 32 E4M3 codes
+    uint32_t sc[kGroups][2];        // FP4: the 2 scale bytes of stage j at bits 16 (j & 1) of sc[g][j >> 1]
+    float sigma[kGroups];           // 1 for an FP4 entry, the row scale of an SWA row, -1 for no key
+    int kind[kGroups];              // 1 FP4 entry, 2 SWA row, 3 the fused new SWA row (not yet read),
+                                    // 0 zero row, -1 nothing
 };
 
 struct KeyMap {      // this CTA's keys and where each comes from
@@ -308,69 +320,80 @@ struct KeyMap {      // this CTA's keys and where each comes from
     const Smem *smem;
 };
 
-// Issue every load of key kg's channel half for all four stages (one memory round trip).
-// The fused new SWA row is only marked here (kind 3): see take_new_row.
-__device__ __forceinline__ void load_key(Raw &r, const AttnArgs &a, const KeyMap &km, int kg, bool zrow, int hh) {
-    r.kind = zrow ? 0 : -1;
-    r.sigma = -1.0f;
-    if (kg >= km.k_end) return;
-    if (kg < km.n_sel) {
-        const int64_t off = cache_row(a.pm, a.cap, km.b, km.ids[kg]);   // checked when compacted
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.codes + off * kCodeBytes + 32 * hh);
-        const uint32_t *sc = reinterpret_cast<const uint32_t *>(a.scales + off * kScaleBytes + 4 * hh);
+// Issue every load of the lane's two keys (all four stages: one memory round trip).
+// kg0: the tile's first key; zlim: keys of the tile below zlim are written (zero rows
+// past the valid keys).  The fused new SWA row is only marked here (kind 3).
+__device__ __forceinline__ void load_keys(Raw &r, const AttnArgs &a, const KeyMap &km, int kg0, int zlim,
+                                          int wi, int lane) {
+    const int p = prod_piece(lane);
 #pragma unroll
-        for (int j = 0; j < kStages; ++j) {
-            r.c[j][0] = __ldg(src + 4 * j);
-            r.c[j][1] = __ldg(src + 4 * j + 1);
-            r.sc[j] = __ldg(sc + 2 * j);
+    for (int g = 0; g < kGroups; ++g) {
+        const int kt = prod_key(wi, g, lane), kg = kg0 + kt;
+        r.kind[g] = kt < zlim ? 0 : -1;
+        r.sigma[g] = -1.0f;
+        if (kg >= km.k_end) continue;
+        if (kg < km.n_sel) {
+            const int64_t off = cache_row(a.pm, a.cap, km.b, km.ids[kg]);   // checked when compacted
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.codes + off * kCodeBytes + 16 * p);
+            const uint16_t *sc = reinterpret_cast<const uint16_t *>(a.scales + off * kScaleBytes + 2 * p);
+#pragma unroll
+            for (int j = 0; j < kStages; ++j) r.c[g][j][0] = __ldg(src + 4 * j);
+            r.sc[g][0] = (uint32_t)__ldg(sc) | ((uint32_t)__ldg(sc + 4) << 16);
+            r.sc[g][1] = (uint32_t)__ldg(sc + 8) | ((uint32_t)__ldg(sc + 12) << 16);
+            r.kind[g] = 1;
+            r.sigma[g] = 1.0f;
+        } else if (km.new_row != nullptr && kg == km.n_keys - 1) {
+            r.kind[g] = 3;
+        } else {
+            const int64_t pos = km.w0 + (kg - km.n_sel);
+            const int64_t slot = km.ring_base + pos % a.wcap;
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.swa_codes + slot * kDim + 32 * p);
+#pragma unroll
+            for (int j = 0; j < kStages; ++j) {
+                r.c[g][j][0] = __ldg(src + 8 * j);
+                r.c[g][j][1] = __ldg(src + 8 * j + 1);
+            }
+            r.sigma[g] = __ldg(a.swa_scale + slot);
+            r.kind[g] = 2;
         }
-        r.kind = 1;
-        r.sigma = 1.0f;
-    } else if (km.new_row != nullptr && kg == km.n_keys - 1) {
-        r.kind = 3;   // read from shared memory when stored, once warp 1 has written it
-    } else {
-        const int64_t pos = km.w0 + (kg - km.n_sel);
-        const int64_t slot = km.ring_base + pos % a.wcap;
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.swa_codes + slot * kDim + 64 * hh);
-#pragma unroll
-        for (int j = 0; j < kStages; ++j)
-#pragma unroll
-            for (int u = 0; u < 4; ++u) r.c[j][u] = __ldg(src + 8 * j + u);
-        r.sigma = __ldg(a.swa_scale + slot);
-        r.kind = 2;
     }
 }
 
 // Kind 3 -> 2: the fused new SWA row, once warp 1 has quantised it into shared memory
 // (bounded wait; on timeout the key is dropped as a zero row and flagged).
-__device__ __forceinline__ void take_new_row(Raw &r, const AttnArgs &a, const KeyMap &km, int hh, bool &new_ok) {
+__device__ __forceinline__ void take_new_row(Raw &r, int g, const AttnArgs &a, const KeyMap &km, int lane,
+                                             bool &new_ok) {
     if (!new_ok) new_ok = mbar_wait(km.new_ready, 0, a.wait.limit_ns, *km.smem);
     if (!new_ok) {
         set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
-        r.kind = 0;
-        r.sigma = -1.0f;
+        r.kind[g] = 0;
+        r.sigma[g] = -1.0f;
         return;
     }
-    const uint4 *src = reinterpret_cast<const uint4 *>(km.new_row + 64 * hh);
+    const uint4 *src = reinterpret_cast<const uint4 *>(km.new_row + 32 * prod_piece(lane));
 #pragma unroll
-    for (int j = 0; j < kStages; ++j)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) r.c[j][u] = src[8 * j + u];
-    r.sigma = *km.new_sigma;
-    r.kind = 2;
+    for (int j = 0; j < kStages; ++j) {
+        r.c[g][j][0] = src[8 * j];
+        r.c[g][j][1] = src[8 * j + 1];
+    }
+    r.sigma[g] = *km.new_sigma;
+    r.kind[g] = 2;
 }
 
-// Dequantise stage j of the thread's key half into row `row` of block hh (fp16, swizzled).
-__device__ __forceinline__ void store_half(const Raw &r, int j, uint8_t *stage, int row, int hh) {
-    uint8_t *blk = stage + hh * kCbBytes;
-    if (r.kind == 1) {
-        const uint32_t lo = cvt_e4m3x2_f16x2(r.sc[j] & 0xFFFFu), hi = cvt_e4m3x2_f16x2(r.sc[j] >> 16);
-        const uint32_t scale2[4] = {(lo & 0xFFFFu) * 0x10001u, (lo >> 16) * 0x10001u, (hi & 0xFFFFu) * 0x10001u,
-                                    (hi >> 16) * 0x10001u};   // f16x2 scale of each 16 channels
+// Dequantise stage j of the lane's piece of key row `row` (fp16, swizzled).
+__device__ __forceinline__ void store_piece(const Raw &r, int g, int j, uint8_t *stage, int row, int lane) {
+    const int p = prod_piece(lane);
+    uint8_t *blk = stage + (p >> 1) * kCbBytes;
+    const int c0 = 4 * (p & 1);
+    const int kind = r.kind[g];
+    if (kind == 1) {
+        const uint32_t two = (r.sc[g][j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+        const uint32_t hs = cvt_e4m3x2_f16x2(two);
+        const uint32_t scale2[2] = {(hs & 0xFFFFu) * 0x10001u, (hs >> 16) * 0x10001u};   // per 16 channels
+        const uint4 cv = r.c[g][j][0];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {                  // 8 channels per 32-bit code word
-            const uint4 cv = r.c[j][c >> 2];
-            const uint32_t w = (c & 3) == 0 ? cv.x : (c & 3) == 1 ? cv.y : (c & 3) == 2 ? cv.z : cv.w;
+        for (int c = 0; c < 4; ++c) {                  // 8 channels per 32-bit code word
+            const uint32_t w = c == 0 ? cv.x : c == 1 ? cv.y : c == 2 ? cv.z : cv.w;
             const __half2 sv = *reinterpret_cast<const __half2 *>(&scale2[c >> 1]);
             uint32_t v[4];
             cvt_e2m1x8_f16x2(w, v);
@@ -379,22 +402,22 @@ __device__ __forceinline__ void store_half(const Raw &r, int j, uint8_t *stage, 
                 __half2 x = __hmul2(*reinterpret_cast<__half2 *>(&v[k]), sv);
                 v[k] = *reinterpret_cast<uint32_t *>(&x);
             }
-            *reinterpret_cast<uint4 *>(blk + swz(row, c)) = make_uint4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<uint4 *>(blk + swz(row, c0 + c)) = make_uint4(v[0], v[1], v[2], v[3]);
         }
-    } else if (r.kind == 2) {
+    } else if (kind == 2) {
         // exact E4M3 codes; the row scale is applied in fp32 on the logit and on P
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {                  // 8 channels = 8 code bytes
-            const uint4 cv = r.c[j][c >> 1];
+        for (int c = 0; c < 4; ++c) {                  // 8 channels = 8 code bytes
+            const uint4 cv = r.c[g][j][c >> 1];
             const uint32_t w0 = (c & 1) ? cv.z : cv.x, w1 = (c & 1) ? cv.w : cv.y;
-            *reinterpret_cast<uint4 *>(blk + swz(row, c)) =
+            *reinterpret_cast<uint4 *>(blk + swz(row, c0 + c)) =
                 make_uint4(cvt_e4m3x2_f16x2(w0 & 0xFFFFu), cvt_e4m3x2_f16x2(w0 >> 16),
                            cvt_e4m3x2_f16x2(w1 & 0xFFFFu), cvt_e4m3x2_f16x2(w1 >> 16));
         }
-    } else if (r.kind == 0) {
+    } else if (kind == 0) {
         const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(blk + swz(row, c)) = z;
+        for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4 *>(blk + swz(row, c0 + c)) = z;
     }
 }
 
@@ -559,10 +582,11 @@ attn_kernel(AttnArgs a) {
     km.smem = &s;
     const bool worker = warp >= kWorkWarp0;
     const int qd = warp & 3, hh = (warp - kWorkWarp0) >> 2;   // worker: key quadrant, head / channel half
-    const int r = 32 * qd + lane;                              // worker: key of the tile
+    const int r = 32 * qd + lane;                              // worker softmax: key of the tile
+    const int wi = warp - kWorkWarp0;                          // worker producer: keys 16 wi ..
     // rows of the tile's last 16-key group of valid keys are read by the output MMAs
     // and so written (zeros past the keys); rows after that group are not written
-    auto zrow_of = [&](int i) { return r < ((min(kTK, k1 - k0 - i * kTK) + 15) / 16) * 16; };
+    auto zlim_of = [&](int i) { return ((min(kTK, k1 - k0 - i * kTK) + 15) / 16) * 16; };
     bool new_ok = false;
     Raw raw;
     __syncthreads();                       // s.ids complete
@@ -582,7 +606,7 @@ attn_kernel(AttnArgs a) {
                 make_uint4(h[0], h[1], h[2], h[3]);
         }
     }
-    if (worker && nt > 0) load_key(raw, a, km, k0 + r, zrow_of(0), hh);   // tile 0, in flight
+    if (worker && nt > 0) load_keys(raw, a, km, k0, zlim_of(0), wi, lane);   // tile 0, in flight
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -682,43 +706,54 @@ attn_kernel(AttnArgs a) {
         }
     } else if (worker) {
         // ---------------- workers: produce tile i + 1 after the softmax of tile i ----------------
-        // Softmax: keys 32 qd .. (TMEM lanes), heads 32 hh .. .  Producer: key r, channel
-        // half hh of every stage; the raw bytes of the next tile are in registers while the
-        // softmax of this one runs.
+        // Softmax: keys 32 qd .. (TMEM lanes), heads 32 hh .. .  Producer: keys 16 wi ..
+        // (prod_key); the raw bytes of the next tile are in registers while the softmax of
+        // this one runs.
         const float c0 = a.softmax_scale * 1.4426950408889634f * exp2f((float)qexp);
         const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
         const float4 *mrun4 = reinterpret_cast<const float4 *>(&s.mrun[32 * hh]);
         float lsum = 0.0f;   // head 32 hh + lane: partial sum over this warp's keys
-        float sig = -1.0f;   // the current tile's key: 1 FP4, sigma SWA, -1 none
         bool ok = true, stop = false;
         for (int i = 0; i < nt; ++i) {
             // ---- produce tile i (its stages are free once O^T(i - 1) has read them) ----
             if (ok) {
-                if (raw.kind == 3) take_new_row(raw, a, km, hh, new_ok);
 #pragma unroll
-                for (int j = 0; j < kStages; ++j) {   // unrolled: raw.c[j] stays in registers
+                for (int g = 0; g < kGroups; ++g)
+                    if (raw.kind[g] == 3) take_new_row(raw, g, a, km, lane, new_ok);
+#pragma unroll
+                for (int j = 0; j < kStages; ++j) {   // unrolled: raw.c[.][j] stays in registers
                     if (i > 0) {
                         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.kv_empty[j], (i - 1) & 1, lim, s));
                         if (!ok) break;
                     }
-                    store_half(raw, j, s.kv[j], r, hh);
+#pragma unroll
+                    for (int g = 0; g < kGroups; ++g) {
+                        const int kt = prod_key(wi, g, lane);
+                        store_piece(raw, g, j, s.kv[j], kt, lane);
+                        if (j == 0 && prod_piece(lane) == 0) {
+                            const float sg = raw.sigma[g];
+                            s.ksig[kt] = sg;
+                            // P carries sigma in fp16: p <= 2^8 needs sigma <= 65504 / 256
+                            if (raw.kind[g] == 2 && sg * 256.0f > 65504.0f) set_dev_err(a.dev_err, CSA2_DEVERR_RANGE);
+                        }
+                    }
                     fence_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&s.kv_full[j]);
                 }
-                sig = raw.sigma;
-                // P carries sigma in fp16: p <= 2^8 needs sigma <= 65504 / 256
-                if (raw.kind == 2 && hh == 0 && sig * 256.0f > 65504.0f) set_dev_err(a.dev_err, CSA2_DEVERR_RANGE);
-                if (ok && i + 1 < nt) load_key(raw, a, km, k0 + (i + 1) * kTK + r, zrow_of(i + 1), hh);
+                if (ok && i + 1 < nt) load_keys(raw, a, km, k0 + (i + 1) * kTK, zlim_of(i + 1), wi, lane);
             }
             // ---- softmax of tile i: every wait first; the four warps of the half agree ----
+            // (kv_full[0] of tile i: every worker's s.ksig of the tile is written)
             const bool w_ok = ok && __all_sync(0xFFFFFFFFu, mbar_wait(&s.s_full[i & 1], (i >> 1) & 1, lim, s) &&
+                                                                mbar_wait(&s.kv_full[0], i & 1, lim, s) &&
                                                                 (i == 0 || mbar_wait(&s.pv_done, (i - 1) & 1, lim, s)));
             stop = group_any(hh, !w_ok || aborted(s));
             if (stop) break;
             tc_fence_after();
             float x[32];
             tmem_ld32(tmem + lane_base + kSCol + 64u * (uint32_t)(i & 1) + 32u * (uint32_t)hh, x);
+            const float sig = s.ksig[r];
             const bool valid = sig >= 0.0f;
             const float ck = c0 * sig;
             float dmax = -INFINITY;
