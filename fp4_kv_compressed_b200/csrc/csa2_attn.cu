@@ -87,7 +87,7 @@ struct __align__(1024) Smem {
     float wself[kHeads];                       // combine: weight of this CTA's partial
     uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], p_full, pv_done, drain, never;
     uint64_t new_ready;                        // fused append: the new SWA row is in smem
-    uint64_t xfer;                             // combine: the peer's part has landed
+    uint64_t xfer[2];                          // combine: the peer's part of head half h has landed
     uint32_t tmem_base;
     int32_t abort;
     float wred[kWarps];
@@ -474,7 +474,8 @@ attn_kernel(AttnArgs a) {
         mbar_init(&s.drain, 1);
         mbar_init(&s.never, 1);
         mbar_init(&s.new_ready, 1);
-        mbar_init(&s.xfer, 1);
+        mbar_init(&s.xfer[0], 1);
+        mbar_init(&s.xfer[1], 1);
         s.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -484,15 +485,10 @@ attn_kernel(AttnArgs a) {
                      "r"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
-    // barriers and TMEM above touch no global memory; everything below may read what the
-    // previous kernel of the stream wrote
-    grid_dep_wait();
-    // every independent global load first (one memory round trip): the position, this
-    // thread's two Top-K slots, its Q chunks and (warp 1, fused append) the new SWA row
+    // The caller's inputs q, q_pos and swa_new are read before the dependency wait (no
+    // kernel of this library writes them; see the header): Q is loaded, scaled and
+    // staged while the previous kernel of the stream finishes.
     const int32_t t32 = a.q_pos[qi];
-    const int *tk = a.topk + (int64_t)qi * a.top_k;
-    const int e_id0 = (int)threadIdx.x < a.top_k ? tk[threadIdx.x] : -1;
-    const int e_id1 = (int)threadIdx.x + kThreads < a.top_k ? tk[threadIdx.x + kThreads] : -1;
     const uint16_t *q = a.q + ((int64_t)qi * a.H + h0) * kDim;
     uint4 qv[kQChunks];   // chunk i = threadIdx.x + kThreads k: head i / 64, channels 8 (i % 64) .. + 7
 #pragma unroll
@@ -507,6 +503,44 @@ attn_kernel(AttnArgs a) {
         xraw[0] = __ldg(src);
         xraw[1] = __ldg(src + 1);
     }
+    {
+        float qm = 0.0f;
+#pragma unroll
+        for (int k = 0; k < kQChunks; ++k) {
+            const uint32_t w[4] = {qv[k].x, qv[k].y, qv[k].z, qv[k].w};
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                qm = fmaxf(qm, fmaxf(fabsf(bf16_bits_to_f32(w[c] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[c] >> 16))));
+        }
+        qm = warp_max(qm);
+        if (lane == 0) s.wred[warp] = qm;
+    }
+    __syncthreads();
+    float qmax = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) qmax = fmaxf(qmax, s.wred[w]);
+    const int qexp = qmax > 0.0f ? max(0, ilogbf(qmax) - 14) : 0;   // max|q| * 2^-qexp < 2^15
+    {
+        const float inv = exp2f((float)-qexp);
+#pragma unroll
+        for (int k = 0; k < kQChunks; ++k) {
+            const int i = threadIdx.x + kThreads * k;
+            if (i >= kHeads * 64) break;
+            const int hd = i / 64, ch8 = i % 64;
+            const uint32_t w[4] = {qv[k].x, qv[k].y, qv[k].z, qv[k].w};
+            uint32_t h[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                h[c] = pack_h2(bf16_bits_to_f32(w[c] & 0xFFFFu) * inv, bf16_bits_to_f32(w[c] >> 16) * inv);
+            *reinterpret_cast<uint4 *>(s.q + (ch8 >> 3) * kQCbBytes + swz(hd, ch8 & 7)) =
+                make_uint4(h[0], h[1], h[2], h[3]);
+        }
+    }
+    // everything below may read what the previous kernel of the stream wrote (the Top-K)
+    grid_dep_wait();
+    const int *tk = a.topk + (int64_t)qi * a.top_k;
+    const int e_id0 = (int)threadIdx.x < a.top_k ? tk[threadIdx.x] : -1;
+    const int e_id1 = (int)threadIdx.x + kThreads < a.top_k ? tk[threadIdx.x + kThreads] : -1;
     const int64_t t = t32;
     const int64_t w0 = max64(0, t - a.swa_len + 1);
     const int n_win = a.swa_len > 0 ? (int)(t - w0 + 1) : 0;
@@ -529,30 +563,18 @@ attn_kernel(AttnArgs a) {
             prefetch_l2(sg, (uint32_t)a.wcap * 4);
     }
     const uint32_t bal0 = __ballot_sync(0xFFFFFFFFu, e_ok0), bal1 = __ballot_sync(0xFFFFFFFFu, e_ok1);
-    float qm = 0.0f;
-#pragma unroll
-    for (int k = 0; k < kQChunks; ++k) {
-        const uint32_t w[4] = {qv[k].x, qv[k].y, qv[k].z, qv[k].w};
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-            qm = fmaxf(qm, fmaxf(fabsf(bf16_bits_to_f32(w[c] & 0xFFFFu)), fabsf(bf16_bits_to_f32(w[c] >> 16))));
-    }
-    qm = warp_max(qm);
     if (lane == 0) {
         s.wcnt[warp] = __popc(bal0);
         s.wcnt[kWarps + warp] = __popc(bal1);
-        s.wred[warp] = qm;
     }
     __syncthreads();
     // compaction in Top-K slot order: slots [0, kThreads) by warp, then [kThreads, 2 kThreads)
     int base0 = 0, base1 = 0, n_sel = 0;
-    float qmax = 0.0f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
         base0 += w < warp ? s.wcnt[w] : 0;
         base1 += w < warp ? s.wcnt[kWarps + w] : 0;
         n_sel += s.wcnt[w];
-        qmax = fmaxf(qmax, s.wred[w]);
     }
     base1 += n_sel;
 #pragma unroll
@@ -567,7 +589,6 @@ attn_kernel(AttnArgs a) {
     const int nt = (k1 - k0 + kTK - 1) / kTK;
     const bool fuse = a.swa_new != nullptr && n_win > 0;
     const uint32_t owner = (n_keys - 1) < k_split ? 0u : 1u;   // the CTA holding the newest key
-    const int qexp = qmax > 0.0f ? max(0, ilogbf(qmax) - 14) : 0;   // max|q| * 2^-qexp < 2^15
     KeyMap km;
     km.ids = s.ids;
     km.n_sel = n_sel;
@@ -590,22 +611,6 @@ attn_kernel(AttnArgs a) {
     bool new_ok = false;
     Raw raw;
     __syncthreads();                       // s.ids complete
-    {
-        const float inv = exp2f((float)-qexp);
-#pragma unroll
-        for (int k = 0; k < kQChunks; ++k) {
-            const int i = threadIdx.x + kThreads * k;
-            if (i >= kHeads * 64) break;
-            const int hd = i / 64, ch8 = i % 64;
-            const uint32_t w[4] = {qv[k].x, qv[k].y, qv[k].z, qv[k].w};
-            uint32_t h[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                h[c] = pack_h2(bf16_bits_to_f32(w[c] & 0xFFFFu) * inv, bf16_bits_to_f32(w[c] >> 16) * inv);
-            *reinterpret_cast<uint4 *>(s.q + (ch8 >> 3) * kQCbBytes + swz(hd, ch8 & 7)) =
-                make_uint4(h[0], h[1], h[2], h[3]);
-        }
-    }
     if (worker && nt > 0) load_keys(raw, a, km, k0, zlim_of(0), wi, lane);   // tile 0, in flight
     fence_async_smem();
     tc_fence_before();
@@ -758,17 +763,25 @@ attn_kernel(AttnArgs a) {
             const float ck = c0 * sig;
             float dmax = -INFINITY;
 #pragma unroll
-            for (int h = 0; h < 32; ++h) x[h] = valid ? x[h] * ck : -INFINITY;
+            for (int h = 0; h < 32; ++h) x[h] = valid ? x[h] * ck : -INFINITY;   // logits, log2 units
             if (i > 0) {
+                // x -> x - m in place: the lazy check, and (common case) the exponent of p
 #pragma unroll
                 for (int h4 = 0; h4 < 8; ++h4) {
                     const float4 mv = mrun4[h4];
-                    dmax = fmaxf(dmax, fmaxf(fmaxf(x[4 * h4] - mv.x, x[4 * h4 + 1] - mv.y),
-                                             fmaxf(x[4 * h4 + 2] - mv.z, x[4 * h4 + 3] - mv.w)));
+                    x[4 * h4] -= mv.x; x[4 * h4 + 1] -= mv.y; x[4 * h4 + 2] -= mv.z; x[4 * h4 + 3] -= mv.w;
+                    dmax = fmaxf(dmax, fmaxf(fmaxf(x[4 * h4], x[4 * h4 + 1]), fmaxf(x[4 * h4 + 2], x[4 * h4 + 3])));
                 }
             }
             const bool upd = group_any(hh, i == 0 || dmax > kLazy);
             if (upd) {
+                if (i > 0) {   // back to the logits (one rounding; p's exponent stays consistent)
+#pragma unroll
+                    for (int h4 = 0; h4 < 8; ++h4) {
+                        const float4 mv = mrun4[h4];
+                        x[4 * h4] += mv.x; x[4 * h4 + 1] += mv.y; x[4 * h4 + 2] += mv.z; x[4 * h4 + 3] += mv.w;
+                    }
+                }
                 // exact tile max per head, then the running max moves
                 const float wm = reduce_scatter32<true>(x, lane);   // head 32 hh + lane
                 s.red[hh][qd][lane] = wm;
@@ -783,21 +796,21 @@ attn_kernel(AttnArgs a) {
                 }
                 group_sync(hh);
                 lsum *= s.alpha[32 * hh + lane];
+#pragma unroll
+                for (int h4 = 0; h4 < 8; ++h4) {
+                    const float4 mv = mrun4[h4];
+                    x[4 * h4] -= mv.x; x[4 * h4 + 1] -= mv.y; x[4 * h4 + 2] -= mv.z; x[4 * h4 + 3] -= mv.w;
+                }
             }
             // p = 2^(x - m); P^T carries the key's scale (V holds SWA codes, not values)
             const float sv = valid ? sig : 0.0f;
             uint32_t pk[16];
 #pragma unroll
-            for (int h4 = 0; h4 < 8; ++h4) {
-                const float4 mv = mrun4[h4];
-                const float p0 = ex2(x[4 * h4] - mv.x), p1 = ex2(x[4 * h4 + 1] - mv.y);
-                const float p2 = ex2(x[4 * h4 + 2] - mv.z), p3 = ex2(x[4 * h4 + 3] - mv.w);
-                x[4 * h4] = p0;
-                x[4 * h4 + 1] = p1;
-                x[4 * h4 + 2] = p2;
-                x[4 * h4 + 3] = p3;
-                pk[2 * h4] = pack_h2(p0 * sv, p1 * sv);
-                pk[2 * h4 + 1] = pack_h2(p2 * sv, p3 * sv);
+            for (int h2 = 0; h2 < 16; ++h2) {
+                const float p0 = ex2(x[2 * h2]), p1 = ex2(x[2 * h2 + 1]);
+                x[2 * h2] = p0;
+                x[2 * h2 + 1] = p1;
+                pk[h2] = pack_h2(p0 * sv, p1 * sv);
             }
 #pragma unroll
             for (int c = 0; c < 4; ++c)
@@ -851,12 +864,15 @@ attn_kernel(AttnArgs a) {
     __syncthreads();                       // stats written; this CTA's MMAs have completed
     tc_fence_after();
     const uint32_t peer = rank ^ 1u;
-    constexpr uint32_t kXfer = 2 * kTK * kHeads * 4;    // the peer's two blocks, fp32
+    constexpr uint32_t kXferHalf = 2 * kTK * (kHeads / 2) * 4;   // the peer's two blocks, 32 heads, fp32
     if (threadIdx.x < kHeads) {
         st_peer(peer_addr(&s.pm[threadIdx.x], peer), s.cm[threadIdx.x]);
         st_peer(peer_addr(&s.pl[threadIdx.x], peer), s.cl[threadIdx.x]);
     }
-    if (threadIdx.x == 0) mbar_expect_tx(&s.xfer, kXfer);   // armed before the peer can send
+    if (threadIdx.x == 0) {                // armed before the peer can send
+        mbar_expect_tx(&s.xfer[0], kXferHalf);
+        mbar_expect_tx(&s.xfer[1], kXferHalf);
+    }
     cluster_sync();                        // stats exchanged; both CTAs' tiles are free
     grid_dep_launch();
     if (threadIdx.x < kHeads) {
@@ -875,19 +891,21 @@ attn_kernel(AttnArgs a) {
             a.lse[(int64_t)qi * a.H + h0 + h] = valid ? (m_all + log2f(l_all)) * 0.6931471805599453f : -INFINITY;
     }
     __syncthreads();
-    // Combine task u (16 of them, warp u % 12 takes u; TMEM lane quadrant u % 4 = warp % 4):
-    // channels 32 (u % 4) .. of a block, head half (u >> 2) & 1, block pair member u >> 3.
-    // The peer's blocks, scaled, are staged in local shared memory (`send`, [2 blocks][128
-    // channels][64 heads] fp32, float4 slots swizzled by channel) and moved by one bulk
-    // copy into the peer's `recv`.
+    // Combine task u (16 of them; warp u % 12 takes u, so the TMEM lane quadrant u % 4 is
+    // the warp's): head half hp = u >> 3, block pair member bsel = (u >> 2) & 1, channels
+    // 32 (u % 4) .. of that block.  The peer's blocks, scaled, are staged in local shared
+    // memory (`send`, [2 head halves][2 blocks][128 channels][32 heads] fp32, float4
+    // slots swizzled by channel) and moved by one bulk copy per head half into the
+    // peer's `recv`; the half-0 tasks add and write while half 1 is still in flight.
     const bool have = __shfl_sync(0xFFFFFFFFu, (int)(nt > 0 && !aborted(s)), 0) != 0;
     float *send = reinterpret_cast<float *>(&s.kv[0][0]);
     float *recv = reinterpret_cast<float *>(&s.kv[2][0]);
+    constexpr int kHalfF = 2 * kTK * (kHeads / 2);   // floats per head half
 #pragma unroll 1
     for (int u = warp; u < 16; u += kWarps) {
-        const int cq = u & 3, chh = (u >> 2) & 1, bsel = u >> 3;
+        const int cq = u & 3, bsel = (u >> 2) & 1, hp = u >> 3;
         const int crow = 32 * cq + lane;             // channel within a block
-        const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)chh;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)hp;
         float o[32];
         if (have) {
             tmem_ld32(taddr + 64u * (uint32_t)(2 * (int)peer + bsel), o);
@@ -895,28 +913,27 @@ attn_kernel(AttnArgs a) {
 #pragma unroll
             for (int h = 0; h < 32; ++h) o[h] = 0.0f;
         }
-        float4 *dst = reinterpret_cast<float4 *>(send + (bsel * kTK + crow) * kHeads);
+        float4 *dst = reinterpret_cast<float4 *>(send + hp * kHalfF + (bsel * kTK + crow) * (kHeads / 2));
 #pragma unroll
-        for (int f = 0; f < 8; ++f) {                // float4 f of this half = heads 32 chh + 4 f ..
-            const int h = 32 * chh + 4 * f;
-            dst[(8 * chh + f) ^ (crow & 7)] = make_float4(o[4 * f] * s.wself[h], o[4 * f + 1] * s.wself[h + 1],
-                                                          o[4 * f + 2] * s.wself[h + 2], o[4 * f + 3] * s.wself[h + 3]);
+        for (int f = 0; f < 8; ++f) {                // float4 f = heads 32 hp + 4 f ..
+            const int h = 32 * hp + 4 * f;
+            dst[f ^ (crow & 7)] = make_float4(o[4 * f] * s.wself[h], o[4 * f + 1] * s.wself[h + 1],
+                                              o[4 * f + 2] * s.wself[h + 2], o[4 * f + 3] * s.wself[h + 3]);
         }
     }
     fence_async_smem();                    // generic-proxy writes of `send` -> the bulk copy
     __syncthreads();
     if (threadIdx.x == 0) {
-        const uint32_t dst = peer_addr(recv, peer), bar = peer_addr(&s.xfer, peer);
-        bulk_copy_to_peer(dst, send, kXfer / 2, bar);
-        bulk_copy_to_peer(dst + kXfer / 2, reinterpret_cast<uint8_t *>(send) + kXfer / 2, kXfer / 2, bar);
+        const uint32_t dst = peer_addr(recv, peer);
+        bulk_copy_to_peer(dst, send, kXferHalf, peer_addr(&s.xfer[0], peer));
+        bulk_copy_to_peer(dst + kXferHalf, send + kHalfF, kXferHalf, peer_addr(&s.xfer[1], peer));
     }
-    const bool got = __syncthreads_and(mbar_wait<false>(&s.xfer, 0, kDrainLimitNs, s)) != 0;
-    if (!got && threadIdx.x == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+    bool got_all = true;
 #pragma unroll 1
     for (int u = warp; u < 16; u += kWarps) {
-        const int cq = u & 3, chh = (u >> 2) & 1, bsel = u >> 3;
+        const int cq = u & 3, bsel = (u >> 2) & 1, hp = u >> 3;
         const int crow = 32 * cq + lane;
-        const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)chh;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)hp;
         float own[32];
         if (have) {
             tmem_ld32(taddr + 64u * (uint32_t)(2 * (int)rank + bsel), own);
@@ -924,19 +941,28 @@ attn_kernel(AttnArgs a) {
 #pragma unroll
             for (int h = 0; h < 32; ++h) own[h] = 0.0f;
         }
+        const bool got = __all_sync(0xFFFFFFFFu, mbar_wait<false>(&s.xfer[hp], 0, kDrainLimitNs, s));
+        got_all = got_all && got;
         const int blk = 2 * (int)rank + bsel;
-        const float4 *src = reinterpret_cast<const float4 *>(recv + (bsel * kTK + crow) * kHeads);
+        const float4 *src = reinterpret_cast<const float4 *>(recv + hp * kHalfF + (bsel * kTK + crow) * (kHeads / 2));
         float *obase = a.out + ((int64_t)qi * a.H + h0) * kDim + 128 * blk + crow;
 #pragma unroll
         for (int f = 0; f < 8; ++f) {
-            const int h = 32 * chh + 4 * f;
-            const float4 pr = got ? src[(8 * chh + f) ^ (crow & 7)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            const int h = 32 * hp + 4 * f;
+            const float4 pr = got ? src[f ^ (crow & 7)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             const float pv[4] = {pr.x, pr.y, pr.z, pr.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 if (h + k < hcta) obase[(int64_t)(h + k) * kDim] = fmaf(own[4 * f + k], s.wself[h + k], pv[k]);
         }
     }
+    if (!got_all && lane == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+    // A warp with no half-1 task still waits for it, so that both incoming copies have
+    // landed before the closing barrier.
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait<false>(&s.xfer[0], 0, kDrainLimitNs, s) &&
+                                     mbar_wait<false>(&s.xfer[1], 0, kDrainLimitNs, s)) &&
+        lane == 0)
+        set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
     // Both CTAs have seen their incoming copy land, so both outgoing copies have finished
     // reading `send`: only now may either CTA leave (and its shared memory be reused).
     tc_fence_before();

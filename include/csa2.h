@@ -30,7 +30,12 @@
  *  - Kernels are launched with programmatic dependent launch: each may be
  *    scheduled while the previous kernel of the stream finishes, but waits for it
  *    (completion and memory visibility) before its first global memory access, so
- *    results are stream-ordered exactly as with ordinary launches.
+ *    results are stream-ordered exactly as with ordinary launches.  One exception:
+ *    the sparse attention calls read the caller's q, q_pos and new SWA row before
+ *    that wait (no kernel of this library writes them).  Those three must not be
+ *    written by the immediately preceding kernel of the stream if that kernel
+ *    itself triggers programmatic launch completion before its writes; ordinary
+ *    kernels and copies (which trigger only at completion) are fine.
  *  - bf16 inputs are row-major and contiguous; "B" is the request count, "Tq"
  *    the number of query tokens per request (1 = decode, >1 = prefill chunk).
  *  - Numbers are finite: NaN/Inf inputs are outside the contract.
