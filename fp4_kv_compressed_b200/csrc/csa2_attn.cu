@@ -9,10 +9,9 @@
 //
 // Work split: a 2-CTA cluster per (query, group of 64 heads).  The query's keys
 // (selected entries first, then the window) are cut in two halves at a multiple of
-// 16; each CTA runs an independent online softmax over its half.  At the end the
-// partial maxima and sums are exchanged through distributed shared memory and the
-// partial outputs through the output rows (L2): each CTA finalises half of the
-// output channels.
+// 16; each CTA runs an independent online softmax over its half and the two partial
+// results are merged through distributed shared memory at the end (each CTA writes
+// half of the output channels).
 //
 // Transposed tiles.  A tile is 128 keys.  The scores are S^T = K Q^T with the keys
 // as the MMA's M = 128 (one TMEM lane per key) and the 64 heads as N, so the score
@@ -88,6 +87,7 @@ struct __align__(1024) Smem {
     float wself[kHeads];                       // combine: weight of this CTA's partial
     uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], p_full, pv_done, drain, never;
     uint64_t new_ready;                        // fused append: the new SWA row is in smem
+    uint64_t xfer[2];                          // combine: the peer's part of head half h has landed
     uint32_t tmem_base;
     int32_t abort;
     float wred[kWarps];
@@ -238,6 +238,18 @@ __device__ __forceinline__ bool group_any(int hh, bool pred) {
         : "r"((uint32_t)pred), "r"(1 + hh)
         : "memory");
     return r != 0;
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+                 : "memory");
+}
+// Bulk copy from this CTA's shared memory into the peer CTA's (dst and bar are
+// shared::cluster addresses; completes as bytes on bar).  No multicast.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "r"(smem_u32(src)), "r"(bytes), "r"(bar)
+        : "memory");
 }
 // L2 prefetch of [p, p + bytes) (p 16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
@@ -462,6 +474,8 @@ attn_kernel(AttnArgs a) {
         mbar_init(&s.drain, 1);
         mbar_init(&s.never, 1);
         mbar_init(&s.new_ready, 1);
+        mbar_init(&s.xfer[0], 1);
+        mbar_init(&s.xfer[1], 1);
         s.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -842,25 +856,24 @@ attn_kernel(AttnArgs a) {
         }
     }
 
-    // ---- combine the two key halves of the query --------------------------------------------
-    // CTA r finalises channels [256 r, 256 r + 256) = O^T blocks 2 r, 2 r + 1.  The
-    // partial maxima and sums go to the peer through distributed shared memory; the
-    // partial outputs go through the output rows themselves: each CTA first writes its
-    // scaled partial for the PEER's channels there, and after the cluster barrier
-    // (release / acquire at cluster scope) the owner reads it back from L2, adds its
-    // own and overwrites it with the final value.  Exactly one partial per element
-    // passes through memory, so the sum is exact fp32 a + b in a fixed order.  Every
-    // thread of both CTAs takes both cluster barriers, whatever happened above.
+    // ---- combine the two key halves of the query through distributed shared memory ----
+    // CTA r writes channels [256 r, 256 r + 256) = O^T blocks 2 r, 2 r + 1.  Every thread
+    // of both CTAs takes every cluster barrier, whatever happened above.
     __syncwarp();
     tc_fence_before();
     __syncthreads();                       // stats written; this CTA's MMAs have completed
     tc_fence_after();
     const uint32_t peer = rank ^ 1u;
+    constexpr uint32_t kXferHalf = 2 * kTK * (kHeads / 2) * 4;   // the peer's two blocks, 32 heads, fp32
     if (threadIdx.x < kHeads) {
         st_peer(peer_addr(&s.pm[threadIdx.x], peer), s.cm[threadIdx.x]);
         st_peer(peer_addr(&s.pl[threadIdx.x], peer), s.cl[threadIdx.x]);
     }
-    cluster_sync();                        // stats exchanged
+    if (threadIdx.x == 0) {                // armed before the peer can send
+        mbar_expect_tx(&s.xfer[0], kXferHalf);
+        mbar_expect_tx(&s.xfer[1], kXferHalf);
+    }
+    cluster_sync();                        // stats exchanged; both CTAs' tiles are free
     grid_dep_launch();
     if (threadIdx.x < kHeads) {
         const int h = threadIdx.x;
@@ -878,55 +891,82 @@ attn_kernel(AttnArgs a) {
             a.lse[(int64_t)qi * a.H + h0 + h] = valid ? (m_all + log2f(l_all)) * 0.6931471805599453f : -INFINITY;
     }
     __syncthreads();
-    // Task u (16; warp u % 12 takes u, so the TMEM lane quadrant u % 4 is the warp's):
-    // channels 32 (u % 4) .. of block 2 c + ((u >> 2) & 1) (c the CTA whose channels are
-    // written), heads 32 (u >> 3) .. .  A thread holds one channel of 32 heads; a warp
-    // store covers 32 consecutive channels of one head (128 bytes).
+    // Combine task u (16 of them; warp u % 12 takes u, so the TMEM lane quadrant u % 4 is
+    // the warp's): head half hp = u >> 3, block pair member bsel = (u >> 2) & 1, channels
+    // 32 (u % 4) .. of that block.  The peer's blocks, scaled, are staged in local shared
+    // memory (`send`, [2 head halves][2 blocks][128 channels][32 heads] fp32, float4
+    // slots swizzled by channel) and moved by one bulk copy per head half into the
+    // peer's `recv`; the half-0 tasks add and write while half 1 is still in flight.
     const bool have = __shfl_sync(0xFFFFFFFFu, (int)(nt > 0 && !aborted(s)), 0) != 0;
-    float *orow = a.out + ((int64_t)qi * a.H + h0) * kDim;
+    float *send = reinterpret_cast<float *>(&s.kv[0][0]);
+    float *recv = reinterpret_cast<float *>(&s.kv[2][0]);
+    constexpr int kHalfF = 2 * kTK * (kHeads / 2);   // floats per head half
 #pragma unroll 1
-    for (int u = warp; u < 16; u += kWarps) {      // the peer's channels: this CTA's partial
-        const int cq = u & 3, blk = 2 * (int)peer + ((u >> 2) & 1), hp = u >> 3;
+    for (int u = warp; u < 16; u += kWarps) {
+        const int cq = u & 3, bsel = (u >> 2) & 1, hp = u >> 3;
+        const int crow = 32 * cq + lane;             // channel within a block
+        const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)hp;
         float o[32];
         if (have) {
-            tmem_ld32(tmem + ((uint32_t)(32 * cq) << 16) + 64u * (uint32_t)blk + 32u * (uint32_t)hp, o);
+            tmem_ld32(taddr + 64u * (uint32_t)(2 * (int)peer + bsel), o);
         } else {
 #pragma unroll
             for (int h = 0; h < 32; ++h) o[h] = 0.0f;
         }
-        float *dst = orow + 128 * blk + 32 * cq + lane;
+        float4 *dst = reinterpret_cast<float4 *>(send + hp * kHalfF + (bsel * kTK + crow) * (kHeads / 2));
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const int h = 32 * hp + k;
-            if (h < hcta) dst[(int64_t)h * kDim] = o[k] * s.wself[h];
+        for (int f = 0; f < 8; ++f) {                // float4 f = heads 32 hp + 4 f ..
+            const int h = 32 * hp + 4 * f;
+            dst[f ^ (crow & 7)] = make_float4(o[4 * f] * s.wself[h], o[4 * f + 1] * s.wself[h + 1],
+                                              o[4 * f + 2] * s.wself[h + 2], o[4 * f + 3] * s.wself[h + 3]);
         }
     }
-    cluster_sync();                        // the partials are in L2 for their owners
+    fence_async_smem();                    // generic-proxy writes of `send` -> the bulk copy
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t dst = peer_addr(recv, peer);
+        bulk_copy_to_peer(dst, send, kXferHalf, peer_addr(&s.xfer[0], peer));
+        bulk_copy_to_peer(dst + kXferHalf, send + kHalfF, kXferHalf, peer_addr(&s.xfer[1], peer));
+    }
+    bool got_all = true;
 #pragma unroll 1
-    for (int u = warp; u < 16; u += kWarps) {      // own channels: own partial + the peer's
-        const int cq = u & 3, blk = 2 * (int)rank + ((u >> 2) & 1), hp = u >> 3;
-        float o[32];
+    for (int u = warp; u < 16; u += kWarps) {
+        const int cq = u & 3, bsel = (u >> 2) & 1, hp = u >> 3;
+        const int crow = 32 * cq + lane;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)hp;
+        float own[32];
         if (have) {
-            tmem_ld32(tmem + ((uint32_t)(32 * cq) << 16) + 64u * (uint32_t)blk + 32u * (uint32_t)hp, o);
+            tmem_ld32(taddr + 64u * (uint32_t)(2 * (int)rank + bsel), own);
         } else {
 #pragma unroll
-            for (int h = 0; h < 32; ++h) o[h] = 0.0f;
+            for (int h = 0; h < 32; ++h) own[h] = 0.0f;
         }
-        float *dst = orow + 128 * blk + 32 * cq + lane;
-        float pv[32];
+        const bool got = __all_sync(0xFFFFFFFFu, mbar_wait<false>(&s.xfer[hp], 0, kDrainLimitNs, s));
+        got_all = got_all && got;
+        const int blk = 2 * (int)rank + bsel;
+        const float4 *src = reinterpret_cast<const float4 *>(recv + hp * kHalfF + (bsel * kTK + crow) * (kHeads / 2));
+        float *obase = a.out + ((int64_t)qi * a.H + h0) * kDim + 128 * blk + crow;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const int h = 32 * hp + k;
-            pv[k] = h < hcta ? __ldcg(dst + (int64_t)h * kDim) : 0.0f;
-        }
+        for (int f = 0; f < 8; ++f) {
+            const int h = 32 * hp + 4 * f;
+            const float4 pr = got ? src[f ^ (crow & 7)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            const float pv[4] = {pr.x, pr.y, pr.z, pr.w};
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const int h = 32 * hp + k;
-            if (h < hcta) dst[(int64_t)h * kDim] = fmaf(o[k], s.wself[h], pv[k]);
+            for (int k = 0; k < 4; ++k)
+                if (h + k < hcta) obase[(int64_t)(h + k) * kDim] = fmaf(own[4 * f + k], s.wself[h + k], pv[k]);
         }
     }
+    if (!got_all && lane == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+    // A warp with no half-1 task still waits for it, so that both incoming copies have
+    // landed before the closing barrier.
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait<false>(&s.xfer[0], 0, kDrainLimitNs, s) &&
+                                     mbar_wait<false>(&s.xfer[1], 0, kDrainLimitNs, s)) &&
+        lane == 0)
+        set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+    // Both CTAs have seen their incoming copy land, so both outgoing copies have finished
+    // reading `send`: only now may either CTA leave (and its shared memory be reused).
     tc_fence_before();
-    __syncthreads();                       // every TMEM load of the CTA has completed
+    cluster_sync();
     tc_fence_after();
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
