@@ -29,7 +29,7 @@ namespace csa2 {
 // ------------------------------------------------------------------------------
 constexpr int kScoreThreads = 64;
 constexpr int kScanRows = 4;       // rows per thread, Full scan (256-row, 32 KB tiles)
-constexpr int kReindexRows = 4;    // rows per thread, Reindex gather (256-row, 32 KB tiles)
+constexpr int kReindexRows = 2;    // rows per thread, Reindex gather (128-row, 16 KB tiles)
 
 // 16-byte unit u of row r lives at unit swz(r, u): a quarter-warp reading unit
 // u of 8 consecutive rows hits 8 different 16-byte bank groups.
@@ -44,7 +44,7 @@ __device__ __forceinline__ int swz(int r, int u) {
 template <int D, int HI, int R>
 struct ScoreSmem {
     uint8_t rows[kScoreThreads * R * D];
-    alignas(16) float2 q[D / 2][HI];     // q pairs (q[h][2j], q[h][2j+1]) as fp32
+    float2 q[D / 2][HI];     // q pairs (q[h][2j], q[h][2j+1]) as fp32
     float w[HI];
     float m64[kScoreThreads / 32][R];   // per warp and row group: max of its 32 rows
 };
@@ -104,23 +104,10 @@ __device__ __forceinline__ void score_rows_at(const uint8_t *rows, const float2 
 #pragma unroll
         for (int i = 0; i < 4; ++i) {           // one 32-bit word = channel pairs 2i, 2i+1 of the unit
             float2 qa[HI], qb[HI];              // q is read per word: few live registers
-            if constexpr (HI % 2 == 0) {        // 16-byte loads: two heads' pairs at a time
-                const float4 *qa4 = reinterpret_cast<const float4 *>(q[8 * u + 2 * i]);
-                const float4 *qb4 = reinterpret_cast<const float4 *>(q[8 * u + 2 * i + 1]);
 #pragma unroll
-                for (int h2 = 0; h2 < HI / 2; ++h2) {
-                    const float4 va = qa4[h2], vb = qb4[h2];
-                    qa[2 * h2] = make_float2(va.x, va.y);
-                    qa[2 * h2 + 1] = make_float2(va.z, va.w);
-                    qb[2 * h2] = make_float2(vb.x, vb.y);
-                    qb[2 * h2 + 1] = make_float2(vb.z, vb.w);
-                }
-            } else {
-#pragma unroll
-                for (int h = 0; h < HI; ++h) {
-                    qa[h] = q[8 * u + 2 * i][h];
-                    qb[h] = q[8 * u + 2 * i + 1][h];
-                }
+            for (int h = 0; h < HI; ++h) {
+                qa[h] = q[8 * u + 2 * i][h];
+                qb[h] = q[8 * u + 2 * i + 1][h];
             }
 #pragma unroll
             for (int r = 0; r < R; ++r) {
@@ -239,7 +226,7 @@ index_scan_kernel(IndexArgs a) {
 
 // ------------------------------------------------------------------------------
 // a6: Reindex scoring of the pool.  grid (ceil(8 pool_blocks / kTileRows), B*Tq),
-// kScoreThreads threads, kTileRows = kScoreThreads * kReindexRows (32 pool blocks).
+// kScoreThreads threads, kTileRows = kScoreThreads * kReindexRows (16 pool blocks).
 // Candidate c = 8 * slot + r of the pool (slot < pool_blocks, r < 8) is position
 // 8 * pool[slot] + r; its score goes to scores[qi][c] and the maximum of the slot's
 // visible positions to bmax[qi][slot] (for the selection's block lemma).  Many small
