@@ -7,11 +7,13 @@
 // together with its own 128-token FP8 SWA window; one softmax over the union.
 // K = V = the 512-channel entry (MQA, fixed for this build).
 //
-// Work split: a 2-CTA cluster per (query, group of 64 heads).  The query's keys
-// (selected entries first, then the window) are cut in two halves at a multiple of
-// 16; each CTA runs an independent online softmax over its half and the two partial
-// results are merged through distributed shared memory at the end (each CTA writes
-// half of the output channels).
+// Work split: a cluster of CS CTAs per (query, group of 64 heads), CS = 4 when the
+// grid still fits the SMs (small batches), else 2.  The query's keys (selected entries
+// first, then the window) are cut in CS chunks of a multiple of 16; each CTA runs an
+// independent online softmax over its chunk.  At the end the partial maxima and sums
+// are exchanged through distributed shared memory, and each CTA finalises 4 / CS of
+// the four 128-channel output blocks from its own partial and the others' (bulk
+// copies between the CTAs' shared memories).
 //
 // Transposed tiles.  A tile is 128 keys.  The scores are S^T = K Q^T with the keys
 // as the MMA's M = 128 (one TMEM lane per key) and the 64 heads as N, so the score
@@ -70,6 +72,7 @@ constexpr uint32_t kSCol = 256;                // S^T buffer b at columns 256 + 
 constexpr int kWorkWarp0 = 4;                  // softmax + producer warps 4..11
 constexpr int kWorkWarps = kWarps - kWorkWarp0;
 constexpr float kLazy = 8.0f;                  // rescale threshold (log2 units)
+constexpr int kMaxCS = 4;                      // CTAs per query (cluster size): 2 or 4
 
 struct __align__(1024) Smem {
     uint8_t q[8 * kQCbBytes];                  // Q fp16, [8 cb][64 heads][128 B] swizzled
@@ -83,11 +86,11 @@ struct __align__(1024) Smem {
     alignas(16) float mrun[kHeads];            // running max per head (log2 domain)
     alignas(16) float alpha[kHeads];           // factor of the last move of the running max
     float cm[kHeads], cl[kHeads];              // this CTA's partial max / sum per head
-    float pm[kHeads], pl[kHeads];              // the peer's, written by the peer
+    float pm[kMaxCS][kHeads], pl[kMaxCS][kHeads];   // every CTA's partial max / sum, by rank
     float wself[kHeads];                       // combine: weight of this CTA's partial
     uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], p_full, pv_done, drain, never;
     uint64_t new_ready;                        // fused append: the new SWA row is in smem
-    uint64_t xfer[2];                          // combine: the peer's part of head half h has landed
+    uint64_t xfer[2];                          // combine: the peers' parts of head half h have landed
     uint32_t tmem_base;
     int32_t abort;
     float wred[kWarps];
@@ -448,15 +451,16 @@ __device__ __forceinline__ float reduce_scatter32(const float *x, int lane) {
 
 // ---------------------------------------------------------------------------------------
 // kRope: the fused append rotates the new SWA row first (a separate instantiation, so
-// that the plain kernel carries none of its code).
-template <bool kRope>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+// that the plain kernel carries none of its code).  CS: CTAs per query (the cluster,
+// set at launch), 2 or 4.
+template <bool kRope, int CS>
+__global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(AttnArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem &s = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
-    const int qi = blockIdx.x >> 1;
+    const int qi = blockIdx.x / CS;
     const int b = qi / a.Tq;
     const int h0 = blockIdx.y * kHeads;
     const int hcta = min(kHeads, a.H - h0);
@@ -582,13 +586,13 @@ attn_kernel(AttnArgs a) {
     const uint32_t below = (1u << lane) - 1u;
     if (e_ok0) s.ids[base0 + __popc(bal0 & below)] = e_id0;
     if (e_ok1) s.ids[base1 + __popc(bal1 & below)] = e_id1;
-    // this CTA's key range: the query's keys cut in two at a multiple of 16
+    // this CTA's key range: the query's keys cut in CS chunks of a multiple of 16
     const int n_keys = n_sel + n_win;
-    const int k_split = min(n_keys, ((n_keys + 1) / 2 + 15) / 16 * 16);
-    const int k0 = rank == 0 ? 0 : k_split, k1 = rank == 0 ? k_split : n_keys;
+    const int chunk = ((n_keys + CS - 1) / CS + 15) / 16 * 16;
+    const int k0 = min(n_keys, (int)rank * chunk), k1 = min(n_keys, k0 + chunk);
     const int nt = (k1 - k0 + kTK - 1) / kTK;
     const bool fuse = a.swa_new != nullptr && n_win > 0;
-    const uint32_t owner = (n_keys - 1) < k_split ? 0u : 1u;   // the CTA holding the newest key
+    const uint32_t owner = n_keys > 0 ? (uint32_t)((n_keys - 1) / chunk) : 0u;   // holds the newest key
     KeyMap km;
     km.ids = s.ids;
     km.n_sel = n_sel;
@@ -863,57 +867,77 @@ attn_kernel(AttnArgs a) {
     tc_fence_before();
     __syncthreads();                       // stats written; this CTA's MMAs have completed
     tc_fence_after();
-    const uint32_t peer = rank ^ 1u;
-    constexpr uint32_t kXferHalf = 2 * kTK * (kHeads / 2) * 4;   // the peer's two blocks, 32 heads, fp32
-    if (threadIdx.x < kHeads) {
-        st_peer(peer_addr(&s.pm[threadIdx.x], peer), s.cm[threadIdx.x]);
-        st_peer(peer_addr(&s.pl[threadIdx.x], peer), s.cl[threadIdx.x]);
+    // Every CTA owns NB = 4 / CS of the four 128-channel blocks (blocks NB r ..): it sends
+    // its partial of every other CTA's blocks (scaled by its weight) into that CTA's
+    // shared memory and adds what the others sent it to its own.
+    constexpr int NB = 4 / CS;
+    constexpr uint32_t kPiece = NB * kTK * (kHeads / 2) * 4;   // one peer's blocks, one head half, fp32
+    constexpr int kPieceF = (int)(kPiece / 4);
+    for (int i = threadIdx.x; i < CS * kHeads; i += kThreads) {   // stats to every CTA, own slot `rank`
+        const int r2 = i / kHeads, h = i % kHeads;
+        if (r2 == (int)rank) {
+            s.pm[rank][h] = s.cm[h];
+            s.pl[rank][h] = s.cl[h];
+        } else {
+            st_peer(peer_addr(&s.pm[rank][h], (uint32_t)r2), s.cm[h]);
+            st_peer(peer_addr(&s.pl[rank][h], (uint32_t)r2), s.cl[h]);
+        }
     }
-    if (threadIdx.x == 0) {                // armed before the peer can send
-        mbar_expect_tx(&s.xfer[0], kXferHalf);
-        mbar_expect_tx(&s.xfer[1], kXferHalf);
+    if (threadIdx.x == 0) {                // armed before any peer can send
+        mbar_expect_tx(&s.xfer[0], (CS - 1) * kPiece);
+        mbar_expect_tx(&s.xfer[1], (CS - 1) * kPiece);
     }
-    cluster_sync();                        // stats exchanged; both CTAs' tiles are free
+    cluster_sync();                        // stats exchanged; every CTA's tiles are free
     grid_dep_launch();
     if (threadIdx.x < kHeads) {
         const int h = threadIdx.x;
-        const float m_self = s.cm[h], l_self = s.cl[h], m_peer = s.pm[h], l_peer = s.pl[h];
-        const float m_all = fmaxf(m_self, m_peer);
-        float f_self = 0.0f, f_peer = 0.0f;
+        float m_all = -INFINITY;
+#pragma unroll
+        for (int r2 = 0; r2 < CS; ++r2) m_all = fmaxf(m_all, s.pm[r2][h]);
+        float l_all = 0.0f, f_self = 0.0f;
         if (m_all != -INFINITY) {
-            f_self = m_self == -INFINITY ? 0.0f : ex2(m_self - m_all);
-            f_peer = m_peer == -INFINITY ? 0.0f : ex2(m_peer - m_all);
+#pragma unroll
+            for (int r2 = 0; r2 < CS; ++r2) {
+                const float f = s.pm[r2][h] == -INFINITY ? 0.0f : ex2(s.pm[r2][h] - m_all);
+                l_all += s.pl[r2][h] * f;
+                if (r2 == (int)rank) f_self = f;
+            }
         }
-        const float l_all = l_self * f_self + l_peer * f_peer;
         const bool valid = h < hcta && l_all > 0.0f;
         s.wself[h] = valid ? f_self / l_all : 0.0f;
         if (rank == 0 && h < hcta)
             a.lse[(int64_t)qi * a.H + h0 + h] = valid ? (m_all + log2f(l_all)) * 0.6931471805599453f : -INFINITY;
     }
     __syncthreads();
-    // Combine task u (16 of them; warp u % 12 takes u, so the TMEM lane quadrant u % 4 is
-    // the warp's): head half hp = u >> 3, block pair member bsel = (u >> 2) & 1, channels
-    // 32 (u % 4) .. of that block.  The peer's blocks, scaled, are staged in local shared
-    // memory (`send`, [2 head halves][2 blocks][128 channels][32 heads] fp32, float4
-    // slots swizzled by channel) and moved by one bulk copy per head half into the
-    // peer's `recv`; the half-0 tasks add and write while half 1 is still in flight.
+    // Send slot j (0 .. CS - 2) holds the part for peer (rank + 1 + j) % CS; it lands in
+    // that peer's receive slot CS - 2 - j (so receive slot i holds what CTA
+    // (peer + 1 + i) % CS sent).  A slot is [2 head halves][NB blocks][128 channels][32
+    // heads] fp32, float4 units swizzled by channel; receive slots fill s.kv from the
+    // start, send slots follow them in s.kv and then s.q (both free by now).
+    // Task u (warp u % 12 takes u, so the TMEM lane quadrant u % 4 is the warp's):
+    // channels 32 (u % 4) .., head half (u >> 2) & 1, block bsel / send slot from u >> 3.
     const bool have = __shfl_sync(0xFFFFFFFFu, (int)(nt > 0 && !aborted(s)), 0) != 0;
-    float *send = reinterpret_cast<float *>(&s.kv[0][0]);
-    float *recv = reinterpret_cast<float *>(&s.kv[2][0]);
-    constexpr int kHalfF = 2 * kTK * (kHeads / 2);   // floats per head half
+    auto recv_slot = [&](int i) { return reinterpret_cast<float *>(&s.kv[0][0]) + i * 2 * kPieceF; };
+    auto send_slot = [&](int j) {
+        const int k = (CS - 1) + j;        // slot index in the sequence s.kv, then s.q
+        return k * 2 * kPieceF < (int)(sizeof(s.kv) / 4)
+                   ? reinterpret_cast<float *>(&s.kv[0][0]) + k * 2 * kPieceF
+                   : reinterpret_cast<float *>(s.q) + (k * 2 * kPieceF - (int)(sizeof(s.kv) / 4));
+    };
 #pragma unroll 1
-    for (int u = warp; u < 16; u += kWarps) {
-        const int cq = u & 3, bsel = (u >> 2) & 1, hp = u >> 3;
+    for (int u = warp; u < 8 * NB * (CS - 1); u += kWarps) {
+        const int cq = u & 3, hp = (u >> 2) & 1, bsel = (u >> 3) % NB, j = (u >> 3) / NB;
+        const int pr = ((int)rank + 1 + j) % CS;
         const int crow = 32 * cq + lane;             // channel within a block
         const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)hp;
         float o[32];
         if (have) {
-            tmem_ld32(taddr + 64u * (uint32_t)(2 * (int)peer + bsel), o);
+            tmem_ld32(taddr + 64u * (uint32_t)(NB * pr + bsel), o);
         } else {
 #pragma unroll
             for (int h = 0; h < 32; ++h) o[h] = 0.0f;
         }
-        float4 *dst = reinterpret_cast<float4 *>(send + hp * kHalfF + (bsel * kTK + crow) * (kHeads / 2));
+        float4 *dst = reinterpret_cast<float4 *>(send_slot(j) + hp * kPieceF + (bsel * kTK + crow) * (kHeads / 2));
 #pragma unroll
         for (int f = 0; f < 8; ++f) {                // float4 f = heads 32 hp + 4 f ..
             const int h = 32 * hp + 4 * f;
@@ -923,48 +947,57 @@ attn_kernel(AttnArgs a) {
     }
     fence_async_smem();                    // generic-proxy writes of `send` -> the bulk copy
     __syncthreads();
-    if (threadIdx.x == 0) {
-        const uint32_t dst = peer_addr(recv, peer);
-        bulk_copy_to_peer(dst, send, kXferHalf, peer_addr(&s.xfer[0], peer));
-        bulk_copy_to_peer(dst + kXferHalf, send + kHalfF, kXferHalf, peer_addr(&s.xfer[1], peer));
+    if (threadIdx.x < 2 * (CS - 1)) {      // one copy per (peer, head half)
+        const int j = threadIdx.x >> 1, hp = threadIdx.x & 1;
+        const uint32_t pr = (uint32_t)(((int)rank + 1 + j) % CS);
+        const uint32_t dst = peer_addr(recv_slot(CS - 2 - j) + hp * kPieceF, pr);
+        bulk_copy_to_peer(dst, send_slot(j) + hp * kPieceF, kPiece, peer_addr(&s.xfer[hp], pr));
     }
     bool got_all = true;
 #pragma unroll 1
-    for (int u = warp; u < 16; u += kWarps) {
-        const int cq = u & 3, bsel = (u >> 2) & 1, hp = u >> 3;
+    for (int u = warp; u < 8 * NB; u += kWarps) {
+        const int cq = u & 3, hp = (u >> 2) & 1, bsel = u >> 3;
         const int crow = 32 * cq + lane;
         const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)hp;
         float own[32];
         if (have) {
-            tmem_ld32(taddr + 64u * (uint32_t)(2 * (int)rank + bsel), own);
+            tmem_ld32(taddr + 64u * (uint32_t)(NB * (int)rank + bsel), own);
         } else {
 #pragma unroll
             for (int h = 0; h < 32; ++h) own[h] = 0.0f;
         }
         const bool got = __all_sync(0xFFFFFFFFu, mbar_wait<false>(&s.xfer[hp], 0, kDrainLimitNs, s));
         got_all = got_all && got;
-        const int blk = 2 * (int)rank + bsel;
-        const float4 *src = reinterpret_cast<const float4 *>(recv + hp * kHalfF + (bsel * kTK + crow) * (kHeads / 2));
-        float *obase = a.out + ((int64_t)qi * a.H + h0) * kDim + 128 * blk + crow;
 #pragma unroll
         for (int f = 0; f < 8; ++f) {
             const int h = 32 * hp + 4 * f;
-            const float4 pr = got ? src[f ^ (crow & 7)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            const float pv[4] = {pr.x, pr.y, pr.z, pr.w};
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                if (h + k < hcta) obase[(int64_t)(h + k) * kDim] = fmaf(own[4 * f + k], s.wself[h + k], pv[k]);
+            for (int k = 0; k < 4; ++k) own[4 * f + k] *= s.wself[h + k];
         }
+#pragma unroll 1
+        for (int i = 0; i < CS - 1; ++i) {           // the senders in a fixed order
+            const float4 *src = reinterpret_cast<const float4 *>(recv_slot(i) + hp * kPieceF +
+                                                                 (bsel * kTK + crow) * (kHeads / 2));
+#pragma unroll
+            for (int f = 0; f < 8; ++f) {
+                const float4 pr = got ? src[f ^ (crow & 7)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                own[4 * f] += pr.x; own[4 * f + 1] += pr.y; own[4 * f + 2] += pr.z; own[4 * f + 3] += pr.w;
+            }
+        }
+        float *obase = a.out + ((int64_t)qi * a.H + h0) * kDim + 128 * (NB * (int)rank + bsel) + crow;
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+            if (32 * hp + k < hcta) obase[(int64_t)(32 * hp + k) * kDim] = own[k];
     }
     if (!got_all && lane == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
-    // A warp with no half-1 task still waits for it, so that both incoming copies have
-    // landed before the closing barrier.
+    // A warp with no task for a head half still waits for it, so that every incoming
+    // copy has landed before the closing barrier.
     if (!__all_sync(0xFFFFFFFFu, mbar_wait<false>(&s.xfer[0], 0, kDrainLimitNs, s) &&
                                      mbar_wait<false>(&s.xfer[1], 0, kDrainLimitNs, s)) &&
         lane == 0)
         set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
-    // Both CTAs have seen their incoming copy land, so both outgoing copies have finished
-    // reading `send`: only now may either CTA leave (and its shared memory be reused).
+    // Every CTA has seen its incoming copies land, so every outgoing copy has finished
+    // reading its send slot: only now may a CTA leave (and its shared memory be reused).
     tc_fence_before();
     cluster_sync();
     tc_fence_after();
@@ -976,22 +1009,40 @@ attn_kernel(AttnArgs a) {
 
 size_t attn_smem_bytes() { return sizeof(attn::Smem) + 1024; }
 
-template <bool kRope>
-static cudaError_t launch_attn_t(const AttnArgs &a, int BT, cudaStream_t st) {
+template <bool kRope, int CS>
+static cudaError_t launch_attn_t(const AttnArgs &a, int BT, int hg, cudaStream_t st) {
     const size_t smem = attn_smem_bytes();
     static std::atomic<uint64_t> configured{0};   // per device
     {
-        cudaError_t e = config_kernel_once(attn::attn_kernel<kRope>, smem, configured);
+        cudaError_t e = config_kernel_once(attn::attn_kernel<kRope, CS>, smem, configured);
         if (e != cudaSuccess) return e;
     }
-    dim3 grid(2 * BT, (a.H + attn::kHeads - 1) / attn::kHeads);   // 2-CTA clusters
-    cudaError_t e = launch_pdl(attn::attn_kernel<kRope>, grid, dim3(attn::kThreads), smem, st, a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(CS * BT, hg);
+    cfg.blockDim = dim3(attn::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;   // the CS CTAs of a query
+    attr[1].val.clusterDim.x = CS;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, attn::attn_kernel<kRope, CS>, a);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+// 4 CTAs per query when the whole grid still fits the SMs once (small batches: shorter
+// per-query latency), else 2.
 cudaError_t launch_sparse_attn(const AttnArgs &a, int BT, cudaStream_t st) {
-    return a.swa_new != nullptr && a.rope.cs != nullptr ? launch_attn_t<true>(a, BT, st)
-                                                         : launch_attn_t<false>(a, BT, st);
+    const int hg = (a.H + attn::kHeads - 1) / attn::kHeads;
+    const bool four = (int64_t)4 * BT * hg <= device_sm_count();
+    const bool rope = a.swa_new != nullptr && a.rope.cs != nullptr;
+    if (four) return rope ? launch_attn_t<true, 4>(a, BT, hg, st) : launch_attn_t<false, 4>(a, BT, hg, st);
+    return rope ? launch_attn_t<true, 2>(a, BT, hg, st) : launch_attn_t<false, 2>(a, BT, hg, st);
 }
 
 }  // namespace csa2
