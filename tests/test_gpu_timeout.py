@@ -70,9 +70,10 @@ def test_tc_scan_wait_runs_out_then_recovers(pkg):
 
 
 def test_attention_wait_runs_out_then_recovers(pkg):
-    """The same for the sparse attention: a stuck wait in every CTA (after the first
-    score MMAs were issued) must end the call with the timeout bit and leave the tensor
-    memory free for the next call."""
+    """The same for the sparse attention: a stuck wait in every CTA of every
+    cluster (after the first score MMAs were issued) must end the call with the timeout
+    bit, every CTA still meeting at the cluster barriers of the combine, and leave the
+    tensor memory free for the next call."""
     import math
     B, cap, H, W = 3, 1500, 64, 128
     kv = pkg.GlobalKV(B, cap, 128, 1, "cuda")
