@@ -820,7 +820,6 @@ attn_kernel(AttnArgs a) {
             for (int c = 0; c < 4; ++c)
                 *reinterpret_cast<uint4 *>(s.pt + swz(r, 4 * hh + c)) =
                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            lsum += reduce_scatter32<false>(x, lane);   // this tile's 32 keys, head 32 hh + lane
             if (upd && i > 0) {
                 // the running max moved: O^T(i - 1) has landed (pv_done above); scale this
                 // warp's 32 head columns of every block before O^T(i) accumulates on them
@@ -837,6 +836,8 @@ attn_kernel(AttnArgs a) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.p_full);
+            // l after P is released: the sum is off the output MMAs' critical path
+            lsum += reduce_scatter32<false>(x, lane);   // this tile's 32 keys, head 32 hh + lane
         }
         ok = ok && !stop;
         if (ok && nt > 0) {
