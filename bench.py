@@ -91,11 +91,14 @@ def attn_flops(wl) -> int:
 # kernel sources, code_hash of those sources at capture time).  Reported, each kernel
 # scaled to the batch, only for decode workloads and while the code is unchanged.
 NCU_TRAFFIC = {
-    "csa2_sparse_attn_decode": ([], ("csa2_attn.cu",), ""),
-    "csa2_sparse_attn_decode_append": ([], ("csa2_attn.cu",), ""),
-    "csa2_index_full": ([(138_466_304 + 4_205_312, 8), (2_321_920, 8)], ("csa2_index.cu",),
-                        "c6711e4c46445f50"),
-    "csa2_index_reindex": ([], ("csa2_index.cu",), ""),
+    # attention: attn_kernel<0, 2> (2 CTAs per query) at batch 40, one launch
+    "csa2_sparse_attn_decode": ([(13_224_448, 40)], ("csa2_attn.cu",), "4045433ab704ea1f"),
+    "csa2_sparse_attn_decode_append": ([(13_224_448, 40)], ("csa2_attn.cu",), "4045433ab704ea1f"),
+    # Full: index_scan_kernel + select_full_kernel at batch 8
+    "csa2_index_full": ([(138_484_224 + 4_782_592, 8), (1_133_824, 8)], ("csa2_index.cu",),
+                        "db4b2a2e98873967"),
+    # Reindex: reindex_score_kernel + select_reindex_kernel at batch 8
+    "csa2_index_reindex": ([(18_608_640, 8), (551_168, 8)], ("csa2_index.cu",), "db4b2a2e98873967"),
 }
 
 
@@ -439,6 +442,19 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     if st.dev_err.item() != 0:
         raise RuntimeError(f"device error bits {st.dev_err.item()} in the warm-up step")
+    if args.profile_steps:
+        # for profilers: warm-up steps, then the requested eager steps inside one NVTX
+        # range named "step" (e.g. ncu --nvtx --nvtx-include "step/"); no timing
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                st.step(**inputs)
+            torch.cuda.synchronize(dev)
+            torch.cuda.nvtx.range_push("step")
+            for _ in range(args.profile_steps):
+                st.step(**inputs)
+            torch.cuda.synchronize(dev)
+            torch.cuda.nvtx.range_pop()
+        return None, wl
 
     S = max(1, min(10, args.steps))
     import fp4_kv_compressed_b200.stack as stack_mod
@@ -655,6 +671,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (small cases for profiling)")
+    ap.add_argument("--profile-steps", type=int, default=0,
+                    help="run this many eager steps inside an NVTX range 'step' and exit (for ncu)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -675,6 +693,8 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     try:
         line, wl = run_ours(args, rank, world, local_rank)
+        if line is None:
+            return
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline(wl, [0, wl.B - 1])
