@@ -37,9 +37,8 @@
 //                heads.  Per tile: wait for S^T(i); write K(i + 1) to TMEM; the softmax
 //                of tile i -> P^T; V(i + 1), copied from K(i + 1) in TMEM, into the
 //                shared stages as O^T(i) releases them.  The raw bytes of tile i + 2
-//                are loaded right after K(i + 1) is written: FP4 entries by a coalesced
-//                copy of the warp's 32 half rows into shared memory (4 cache lines per
-//                instruction), SWA rows into registers.
+//                are loaded right after K(i + 1) is written (one thread per key, one
+//                memory round trip for its two stages).
 // TMEM (512 columns): O^T block j (channels 128 j .. 128 j + 127) at columns
 // 32 j .. 32 j + 31 (column = head); the two S^T buffers at columns 128 and 160; K at
 // columns 256 + channel / 2 (lane = key).
@@ -81,10 +80,6 @@ struct __align__(1024) Smem {
     uint8_t q[8 * kQCbBytes];                  // Q fp16, [8 cb][32 heads][128 B] swizzled
     uint8_t kv[kStages][kStageBytes];          // stage j: [2 cb][128 keys][128 B] swizzled
     uint8_t pt[kTK * kHeads * 2];              // P^T fp16, [128 keys][32 heads], 64-byte swizzle
-    // worker warp w: the raw FP4 bytes of its 32 keys' channel half for the next tile
-    // (128 code bytes + 16 scale bytes per key; 144-byte rows keep a thread-per-row read
-    // conflict-free)
-    alignas(16) uint8_t raw[8][32][144];
     int32_t ids[CSA2_TOPK_MAX];                // compacted selected entry ids
     float ksig[kTK];                           // per key of the tile: 1 FP4, sigma SWA, -1 none
     alignas(16) uint8_t swa_new[kDim];         // fused append: the new SWA row (E4M3 codes)
@@ -295,18 +290,22 @@ struct KeyMap {      // the query's keys and where each comes from
     const Smem *smem;
 };
 
-// Key kg of the thread (its two stages): the kind and scale; an SWA row's bytes are
-// loaded into registers here (one memory round trip), an FP4 entry's cache row is
-// returned in `off` for the warp's coalesced copy (fp4_copy).  The fused new SWA row is
-// only marked here (kind 3): see take_new_row.
-__device__ __forceinline__ void load_key(Raw &r, const AttnArgs &a, const KeyMap &km, int kg, bool zrow, int h,
-                                         int64_t &off) {
+// Issue every load of key kg's two stages (one memory round trip).  The fused new SWA
+// row is only marked here (kind 3): see take_new_row.
+__device__ __forceinline__ void load_key(Raw &r, const AttnArgs &a, const KeyMap &km, int kg, bool zrow, int h) {
     r.kind = zrow ? 0 : -1;
     r.sigma = -1.0f;
-    off = -1;
     if (kg >= km.n_keys) return;
     if (kg < km.n_sel) {
-        off = cache_row(a.pm, a.cap, km.b, km.ids[kg]);   // checked when compacted
+        const int64_t off = cache_row(a.pm, a.cap, km.b, km.ids[kg]);   // checked when compacted
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.codes + off * kCodeBytes + 128 * h);
+        const uint2 *sc = reinterpret_cast<const uint2 *>(a.scales + off * kScaleBytes + 16 * h);
+#pragma unroll
+        for (int st = 0; st < 2; ++st) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) r.c[st][u] = __ldg(src + 4 * st + u);
+            r.sc[st] = __ldg(sc + st);
+        }
         r.kind = 1;
         r.sigma = 1.0f;
     } else if (km.new_row != nullptr && kg == km.n_keys - 1) {
@@ -322,26 +321,6 @@ __device__ __forceinline__ void load_key(Raw &r, const AttnArgs &a, const KeyMap
         r.sigma = __ldg(a.swa_scale + slot);
         r.kind = 2;
     }
-}
-
-// 16-byte global -> shared copy (cp.async, L1 bypassed).
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
-}
-
-// The warp's coalesced copy of its FP4 keys' half rows into `buf` ([32 keys][144 B]):
-// instruction m copies the 8 code chunks of keys 4 m .. 4 m + 3 (4 cache lines), then
-// one instruction the 16 scale bytes of every key.  off: the thread's own key's cache
-// row (-1: not an FP4 entry).
-__device__ __forceinline__ void fp4_copy(uint8_t (*buf)[144], const AttnArgs &a, int64_t off, int h, int lane) {
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const int kk = 4 * m + (lane >> 3), c = lane & 7;
-        const int64_t o = __shfl_sync(0xFFFFFFFFu, off, kk);
-        if (o >= 0) cp_async16(buf[kk] + 16 * c, a.codes + o * kCodeBytes + 128 * h + 16 * c);
-    }
-    if (off >= 0) cp_async16(buf[lane] + 128, a.scales + off * kScaleBytes + 16 * h);
-    asm volatile("cp.async.commit_group;\n" ::: "memory");
 }
 
 // Kind 3 -> 2: the fused new SWA row, once warp 1 has quantised it into shared memory
@@ -615,11 +594,7 @@ attn_kernel(AttnArgs a, int n32) {
     bool new_ok = false;
     Raw raw;
     __syncthreads();                       // s.ids complete
-    if (worker && nt > 0) {                // tile 0, in flight
-        int64_t off;
-        load_key(raw, a, km, r, r < zlim_of(0), hh, off);
-        fp4_copy(s.raw[warp - kWorkWarp0], a, off, hh, lane);
-    }
+    if (worker && nt > 0) load_key(raw, a, km, r, r < zlim_of(0), hh);   // tile 0, in flight
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -744,17 +719,6 @@ attn_kernel(AttnArgs a, int n32) {
         int kind_next = -1;
         auto put_k = [&]() {
             if (raw.kind == 3) take_new_row(raw, a, km, hh, new_ok);
-            asm volatile("cp.async.wait_all;\n" ::: "memory");   // the warp's FP4 rows are in s.raw
-            __syncwarp();
-            if (raw.kind == 1) {
-                const uint8_t *row = s.raw[warp - kWorkWarp0][lane];
-#pragma unroll
-                for (int st = 0; st < 2; ++st) {
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) raw.c[st][u] = *reinterpret_cast<const uint4 *>(row + 64 * st + 16 * u);
-                    raw.sc[st] = *reinterpret_cast<const uint2 *>(row + 128 + 8 * st);
-                }
-            }
 #pragma unroll
             for (int st = 0; st < 2; ++st)
                 store_k(raw, st, tmem + lane_base + kKCol + 64u * (uint32_t)(2 * hh + st));
@@ -790,11 +754,7 @@ attn_kernel(AttnArgs a, int n32) {
         };
         if (nt > 0) {
             put_k();
-            if (nt > 1) {
-                int64_t off;
-                load_key(raw, a, km, kTK + r, r < zlim_of(1), hh, off);
-                fp4_copy(s.raw[warp - kWorkWarp0], a, off, hh, lane);
-            }
+            if (nt > 1) load_key(raw, a, km, kTK + r, r < zlim_of(1), hh);
             ok = put_v(0);
         }
         for (int i = 0; i < nt; ++i) {
@@ -813,11 +773,7 @@ attn_kernel(AttnArgs a, int n32) {
             tc_fence_before();
             if (i + 1 < nt) {
                 put_k();
-                if (i + 2 < nt) {
-                    int64_t off;
-                    load_key(raw, a, km, (i + 2) * kTK + r, r < zlim_of(i + 2), hh, off);
-                    fp4_copy(s.raw[warp - kWorkWarp0], a, off, hh, lane);
-                }
+                if (i + 2 < nt) load_key(raw, a, km, (i + 2) * kTK + r, r < zlim_of(i + 2), hh);
             }
             // ---- softmax of tile i ----
             const float sig = s.ksig[r];
