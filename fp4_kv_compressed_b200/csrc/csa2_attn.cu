@@ -35,10 +35,9 @@
 //   warps 4-11   workers: warp w handles keys 32 (w % 4) .. (its TMEM lane quadrant) and
 //                half hh = (w - 4) / 4: the producer's 256 channels, the softmax's 16
 //                heads.  Per tile: wait for S^T(i); write K(i + 1) to TMEM; the softmax
-//                of tile i -> P^T; V(i + 1), copied from K(i + 1) in TMEM, into the
-//                shared stages as O^T(i) releases them.  The raw bytes of tile i + 2
-//                are loaded right after K(i + 1) is written (one thread per key, one
-//                memory round trip for its two stages).
+//                of tile i -> P^T; V(i + 1) into the shared stages as O^T(i) releases
+//                them; load the raw bytes of tile i + 2 (one thread per key, one memory
+//                round trip for its two stages).
 // TMEM (512 columns): O^T block j (channels 128 j .. 128 j + 127) at columns
 // 32 j .. 32 j + 31 (column = head); the two S^T buffers at columns 128 and 160; K at
 // columns 256 + channel / 2 (lane = key).
@@ -388,24 +387,13 @@ __device__ __forceinline__ void store_k(const Raw &r, int st, uint32_t taddr) {
     }
 }
 
-// The thread's V row of stage j into row `row` of the shared-memory stage (fp16,
-// swizzled), copied from its K row in TMEM (taddr: lane 32 q, column of the stage's
-// channel 0 of this channel half): the same values, so the raw bytes are free as soon
-// as K is written.
-__device__ __forceinline__ void store_v_from_k(uint32_t taddr, uint8_t *stage, int row, bool write) {
+// The thread's V row of stage st into row `row` of the shared-memory stage (fp16, swizzled).
+__device__ __forceinline__ void store_v(const Raw &r, int st, uint8_t *stage, int row) {
 #pragma unroll
-    for (int qq = 0; qq < 4; ++qq) {
-        float f[16];
-        tmem_ld16(taddr + 16u * (uint32_t)qq, f);
-        if (write) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int u = 4 * qq + c;
-                *reinterpret_cast<uint4 *>(stage + (u >> 3) * kCbBytes + swz(row, u & 7)) =
-                    make_uint4(__float_as_uint(f[4 * c]), __float_as_uint(f[4 * c + 1]),
-                               __float_as_uint(f[4 * c + 2]), __float_as_uint(f[4 * c + 3]));
-            }
-        }
+    for (int u = 0; u < 16; ++u) {
+        uint32_t v[4];
+        dq8(r, st, u, v);
+        *reinterpret_cast<uint4 *>(stage + (u >> 3) * kCbBytes + swz(row, u & 7)) = make_uint4(v[0], v[1], v[2], v[3]);
     }
 }
 
@@ -713,10 +701,7 @@ attn_kernel(AttnArgs a, int n32) {
         const float4 *mrun4 = reinterpret_cast<const float4 *>(&s.mrun[16 * hh]);
         float lsum = 0.0f;   // head 16 hh + lane % 16: this warp's keys' share of l
         bool ok = true, stop = false;
-        // K of the thread's key and channel half into TMEM; arrive k_full.  The tile's
-        // key scale and kind are kept for put_v, and the raw bytes are free afterwards.
-        float sig_next = -1.0f;
-        int kind_next = -1;
+        // K of the thread's key and channel half into TMEM; arrive k_full
         auto put_k = [&]() {
             if (raw.kind == 3) take_new_row(raw, a, km, hh, new_ok);
 #pragma unroll
@@ -726,24 +711,19 @@ attn_kernel(AttnArgs a, int n32) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.k_full);
-            sig_next = raw.sigma;
-            kind_next = raw.kind;
         };
         // V of the thread's key and channel half into stages 2 hh, 2 hh + 1 of tile i (after
-        // O^T(i - 1) has released them), copied from K in TMEM; s.ksig of the tile; arrive
-        // kv_full
+        // O^T(i - 1) has released them); s.ksig of the tile; arrive kv_full
         auto put_v = [&](int i) -> bool {
 #pragma unroll
             for (int st = 0; st < 2; ++st) {
                 const int j = 2 * hh + st;
                 if (i > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&s.kv_empty[j], (i - 1) & 1, lim, s))) return false;
-                tc_fence_after();
-                // (TMEM loads by the whole warp; rows past the tile's last 16-key group skipped)
-                store_v_from_k(tmem + lane_base + kKCol + 64u * (uint32_t)j, s.kv[j], r, kind_next >= 0);
+                if (raw.kind >= 0) store_v(raw, st, s.kv[j], r);
                 if (st == 0 && hh == 0) {
-                    s.ksig[r] = sig_next;
+                    s.ksig[r] = raw.sigma;
                     // P carries sigma in fp16: p <= 2^8 needs sigma <= 65504 / 256
-                    if (kind_next == 2 && sig_next * 256.0f > 65504.0f && hgrp == 0)
+                    if (raw.kind == 2 && raw.sigma * 256.0f > 65504.0f && hgrp == 0)
                         set_dev_err(a.dev_err, CSA2_DEVERR_RANGE);
                 }
                 fence_async_smem();
@@ -754,8 +734,8 @@ attn_kernel(AttnArgs a, int n32) {
         };
         if (nt > 0) {
             put_k();
-            if (nt > 1) load_key(raw, a, km, kTK + r, r < zlim_of(1), hh);
             ok = put_v(0);
+            if (ok && nt > 1) load_key(raw, a, km, kTK + r, r < zlim_of(1), hh);
         }
         for (int i = 0; i < nt; ++i) {
             // ---- S^T(i) and the tile's key scales; the four warps of the half agree ----
@@ -771,10 +751,7 @@ attn_kernel(AttnArgs a, int n32) {
             // ---- K(i + 1) into TMEM: every lane of this warp has read S^T(i), which was
             // the last reader of K(i) ----
             tc_fence_before();
-            if (i + 1 < nt) {
-                put_k();
-                if (i + 2 < nt) load_key(raw, a, km, (i + 2) * kTK + r, r < zlim_of(i + 2), hh);
-            }
+            if (i + 1 < nt) put_k();
             // ---- softmax of tile i ----
             const float sig = s.ksig[r];
             const bool valid = sig >= 0.0f;
@@ -858,7 +835,10 @@ attn_kernel(AttnArgs a, int n32) {
             if (lane == 0) mbar_arrive(&s.p_full);
             lsum += reduce_scatter16<false>(x, lane);   // this tile's 32 keys, after P^T is released
             // ---- V(i + 1) into the stages as O^T(i) releases them; raw bytes of tile i + 2 ----
-            if (ok && i + 1 < nt) ok = put_v(i + 1);
+            if (ok && i + 1 < nt) {
+                ok = put_v(i + 1);
+                if (ok && i + 2 < nt) load_key(raw, a, km, (i + 2) * kTK + r, r < zlim_of(i + 2), hh);
+            }
         }
         ok = ok && !stop;
         if (ok && nt > 0) {
