@@ -7,49 +7,48 @@
 // together with its own 128-token FP8 SWA window; one softmax over the union.
 // K = V = the 512-channel entry (MQA, fixed for this build).
 //
-// Work split: one CTA per (query, group of 32 heads), over all of the query's keys, so
-// no two CTAs share a softmax and nothing is combined: each CTA writes its heads' rows
-// of the output directly.  (The other split, keys over several CTAs, needs their
-// partial outputs moved between SMs at the end; on this part that exchange cost more
-// than the extra dequantisation of every key by both head groups of a query.)
+// Work split: a cluster of CS CTAs per (query, group of 64 heads), CS = 4 when the
+// grid still fits the SMs (small batches), else 2.  The query's keys (selected entries
+// first, then the window) are cut in CS chunks of a multiple of 16; each CTA runs an
+// independent online softmax over its chunk.  At the end the partial maxima and sums
+// are exchanged through distributed shared memory, and each CTA finalises 4 / CS of
+// the four 128-channel output blocks from its own partial and the others' (bulk
+// copies between the CTAs' shared memories).
 //
 // Transposed tiles.  A tile is 128 keys.  The scores are S^T = K Q^T with the keys
-// as the MMA's M = 128 (one TMEM lane per key) and the 32 heads as N; the output is
-// O^T = V^T P^T with the channels as M (four 128-channel blocks) and the heads as N.
-// K and V are the same dequantised fp16 values: K is written into TMEM, where it is the
-// A operand of S^T (so the score MMAs read no shared memory but Q, and the next tile's
-// scores can run while this tile's softmax does), and V into a shared-memory tile of
-// four stages of 128 channels x 128 keys, the MN-major A operand of O^T.  fp16 holds
-// the FP4 values exactly (e2m1 x e4m3 has at most 6 significant bits); an SWA row is
-// stored as its exact E4M3 codes and its scale sigma is applied in fp32, to the logit
-// and folded into P.  Q (the K-major B operand of S^T) is converted to fp16 after an
-// exact power-of-two scaling that keeps max|q| below 2^15.  P^T (the MN-major B
-// operand of O^T) is [128 keys][32 heads] with the 64-byte swizzle.
+// as the MMA's M = 128 (one TMEM lane per key) and the 64 heads as N, so the score
+// MMAs run at the full M = 128 shape; the output is O^T = V^T P^T with the channels
+// as M (four 128-channel blocks) and the heads as N.  One fp16 tile in shared memory
+// serves both: four stages of 128 channels x 128 keys, each the K-major A operand of
+// S^T (rows = keys) and the MN-major A operand of O^T (M = channels contiguous in a
+// row).  fp16 holds the FP4 values exactly (e2m1 x e4m3 has at most 6 significant
+// bits); an SWA row is stored as its exact E4M3 codes and its scale sigma is applied
+// in fp32, to the logit and folded into P.  Q (the K-major B operand of S^T) is
+// converted to fp16 after an exact power-of-two scaling that keeps max|q| below 2^15.
 //
 // 12 warps, specialised:
-//   warp 0       TMEM allocation + the MMA issue loop (one elected lane issues): S^T of
-//                the next tile as soon as its K is in TMEM, then O^T of this tile;
+//   warp 0       TMEM allocation + the MMA issue loop (one elected lane issues);
 //   warp 1       fused append only: quantises the query token's new SWA row;
-//   warp 2       prefetches the entries of the later tiles into L2 (bulk prefetch; the
-//                set-up prefetches the request's SWA ring);
-//   warps 4-11   workers: warp w handles keys 32 (w % 4) .. (its TMEM lane quadrant) and
-//                half hh = (w - 4) / 4: the producer's 256 channels, the softmax's 16
-//                heads.  Per tile: wait for S^T(i); write K(i + 1) to TMEM; the softmax
-//                of tile i -> P^T; V(i + 1) into the shared stages as O^T(i) releases
-//                them; load the raw bytes of tile i + 2 (one thread per key, one memory
-//                round trip for its two stages).
+//   warp 2       prefetches the entries of this CTA's later tiles into L2 (bulk prefetch;
+//                the set-up prefetches the request's SWA ring);
+//   warps 4-11   workers, two roles in turn.  Producer: warp wi = w - 4 gathers keys
+//                16 wi .. 16 wi + 15 of the next tile warp-cooperatively (one load
+//                instruction = one 64-byte stage slice of 8 keys), all four stages in
+//                registers before the softmax of this tile, and dequantises stage j as
+//                soon as O^T of this tile has read it.  Softmax: warp w reads TMEM lane
+//                quadrant w % 4 (32 keys) and the 32 heads of half (w - 4) / 4.
 // TMEM (512 columns): O^T block j (channels 128 j .. 128 j + 127) at columns
-// 32 j .. 32 j + 31 (column = head); the two S^T buffers at columns 128 and 160; K at
-// columns 256 + channel / 2 (lane = key).
+// 64 j .. 64 j + 63 (column = head); the two S^T buffers at columns 256 and 320.
 // Online softmax in the log2 domain with lazy rescaling: the running max of a head
 // moves (and O, l are rescaled) only when a tile's logit exceeds it by more than 8,
 // so p <= 2^8 stays safe in fp16.  The check is per tile and per head half; the exact
 // tile max (a shuffle reduce-scatter within a warp, then across the four warps that
 // share the heads) is formed only when it fires, and always on the first tile.
 // Every wait is bounded (WaitCfg): on timeout the kernel flags CSA2_DEVERR_TIMEOUT,
-// waits (bounded) for the MMAs it issued, frees TMEM and returns.  The four softmax
-// warps of a head half agree on leaving the tile loop through a barrier reduction, so
-// that no named barrier is ever left waiting for a warp that has gone.
+// waits (bounded) for the MMAs it issued, still takes part in both cluster barriers
+// of the combine, frees TMEM and returns.  The four softmax warps of a head half
+// agree on leaving the tile loop through a barrier reduction, so that no named
+// barrier is ever left waiting for a warp that has gone.
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -61,34 +60,37 @@ namespace attn {
 
 constexpr int kThreads = 384;
 constexpr int kWarps = kThreads / 32;
-constexpr int kQChunks = (32 * 64 + kThreads - 1) / kThreads;   // 16-byte Q chunks per thread
+constexpr int kQChunks = (64 * 64 + kThreads - 1) / kThreads;   // 16-byte Q chunks per thread
 constexpr int kTK = 128;                       // keys per tile (S^T M, TMEM lanes)
-constexpr int kHeads = 32;                     // heads per CTA (MMA N)
+constexpr int kHeads = 64;                     // heads per CTA (MMA N)
 constexpr int kStages = 4;                     // 128-channel quarters of a tile
 constexpr int kStageBytes = kTK * 128 * 2;     // 128 keys x 128 channels fp16
 constexpr int kCbBytes = kTK * 128;            // one 64-channel block of a stage
 constexpr int kQCbBytes = kHeads * 128;        // one 64-channel block of Q
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSCol = 128;                // S^T buffer b at columns 128 + 32 b
-constexpr uint32_t kKCol = 256;                // K of the tile (A of S^T): channel c at column 256 + c / 2
+constexpr uint32_t kSCol = 256;                // S^T buffer b at columns 256 + 64 b
 constexpr int kWorkWarp0 = 4;                  // softmax + producer warps 4..11
 constexpr int kWorkWarps = kWarps - kWorkWarp0;
 constexpr float kLazy = 8.0f;                  // rescale threshold (log2 units)
+constexpr int kMaxCS = 4;                      // CTAs per query (cluster size): 2 or 4
 
 struct __align__(1024) Smem {
-    uint8_t q[8 * kQCbBytes];                  // Q fp16, [8 cb][32 heads][128 B] swizzled
+    uint8_t q[8 * kQCbBytes];                  // Q fp16, [8 cb][64 heads][128 B] swizzled
     uint8_t kv[kStages][kStageBytes];          // stage j: [2 cb][128 keys][128 B] swizzled
-    uint8_t pt[kTK * kHeads * 2];              // P^T fp16, [128 keys][32 heads], 64-byte swizzle
+    uint8_t pt[kTK * 128];                     // P^T fp16, [128 keys][64 heads] swizzled
     int32_t ids[CSA2_TOPK_MAX];                // compacted selected entry ids
     float ksig[kTK];                           // per key of the tile: 1 FP4, sigma SWA, -1 none
     alignas(16) uint8_t swa_new[kDim];         // fused append: the new SWA row (E4M3 codes)
     float swa_new_sigma;
-    alignas(16) float red[2][4][16];           // softmax half hh: per quadrant warp, 16 heads
+    alignas(16) float red[2][4][32];           // softmax half hh: per quadrant warp, 32 heads
     alignas(16) float mrun[kHeads];            // running max per head (log2 domain)
     alignas(16) float alpha[kHeads];           // factor of the last move of the running max
-    float wfin[kHeads];                        // 1 / l per head (0: no key)
-    uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], k_full, p_full, pv_done, drain, never;
+    float cm[kHeads], cl[kHeads];              // this CTA's partial max / sum per head
+    float pm[kMaxCS][kHeads], pl[kMaxCS][kHeads];   // every CTA's partial max / sum, by rank
+    float wself[kHeads];                       // combine: weight of this CTA's partial
+    uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], p_full, pv_done, drain, never;
     uint64_t new_ready;                        // fused append: the new SWA row is in smem
+    uint64_t xfer[2];                          // combine: the peers' parts of head half h have landed
     uint32_t tmem_base;
     int32_t abort;
     float wred[kWarps];
@@ -153,10 +155,6 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
     d |= (uint64_t)2 << 61;
     return d;
 }
-// The same descriptor with the 64-byte swizzle (layout type 4).
-__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    return (sw128_desc(saddr, lbo, sbo) & ~((uint64_t)7 << 61)) | ((uint64_t)4 << 61);
-}
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                         uint32_t accumulate) {
     asm volatile(
@@ -164,15 +162,6 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
         "setp.ne.b32 p, %4, 0;\n"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
         "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
-}
-// The same with A read from TMEM (a_tmem: lane 0, first column of the K-step).
-__device__ __forceinline__ void mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                           uint32_t accumulate) {
-    asm volatile(
-        "{\n.reg .pred p;\n"
-        "setp.ne.b32 p, %4, 0;\n"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
 }
 // One lane of a converged warp (the same lane on every call).
 __device__ __forceinline__ bool elect_one() {
@@ -189,18 +178,23 @@ __device__ __forceinline__ void mma_commit(uint64_t *b) {
                      smem_u32(b))
                  : "memory");
 }
-// 32 lanes x 16 columns: thread t of the warp reads TMEM lane (base + t), 16 columns.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
-    uint32_t r[16];
+// 32 lanes x 32 columns: thread t of the warp reads TMEM lane (base + t), 32 columns.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
+    uint32_t r[32];
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 // 32 lanes x 16 columns, in place: v *= f (per column), read and written back.
 __device__ __forceinline__ void tmem_scale16(uint32_t taddr, const float *f) {
@@ -248,39 +242,79 @@ __device__ __forceinline__ bool group_any(int hh, bool pred) {
         : "memory");
     return r != 0;
 }
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+                 : "memory");
+}
+// Bulk copy from this CTA's shared memory into the peer CTA's (dst and bar are
+// shared::cluster addresses; completes as bytes on bar).  No multicast.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "r"(smem_u32(src)), "r"(bytes), "r"(bar)
+        : "memory");
+}
 // L2 prefetch of [p, p + bytes) (p 16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// ---- cluster helpers (2 CTAs per query split its keys; partials combine via DSMEM) ----
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t peer_addr(const void *local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_peer(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_peer4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c),
+                 "f"(d)
+                 : "memory");
 }
 
 // Byte offset of (row, 16-byte chunk c of a 128-byte row) in a 128B-swizzled block.
 __device__ __forceinline__ uint32_t swz(int row, int c) {
     return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4));
 }
-// The same for 64-byte rows with the 64-byte swizzle (chunk c of row r at c ^ (r / 2 % 4)).
-__device__ __forceinline__ uint32_t swz64(int row, int c) {
-    return (uint32_t)(row * 64 + ((c ^ ((row >> 1) & 3)) << 4));
-}
 
-// ---- producer: one thread per key of the tile -------------------------------------------
-// Worker warp w (quadrant q = w % 4, half h = (w - 4) / 4): thread t handles key 32 q + t
-// of the tile and channels 256 h .. 256 h + 255 (stages 2 h and 2 h + 1).  The key's
-// row of K goes to TMEM lane 32 q + t (the A operand of S^T, columns kKCol + channel / 2)
-// and its row of V to the shared-memory tile (the A operand of O^T); both come from the
-// same raw bytes, held in registers a whole tile ahead and dequantised twice.
+// ---- producer: warp-cooperative gather, a whole tile ahead ------------------------------
+// Worker warp wi (0..7) produces keys 16 wi .. 16 wi + 15 of a tile, as two groups of 8.
+// Lane l of a group handles key 4 ((l >> 3) & 1) + ((l & 7) >> 1) of the group and piece
+// p = 2 (l >> 4) + (l & 1) of every 128-channel stage: channels 32 p .. 32 p + 31, i.e.
+// chunks 4 (p & 1) .. + 3 of block p >> 1.  So one load instruction reads one 64-byte
+// stage slice of 8 keys (8 cache lines, not 32), and a quarter-warp's 16-byte shared
+// stores hit 4 consecutive rows x 2 chunk halves: 8 distinct bank groups.
+constexpr int kGroups = 2;         // key groups of 8 per worker warp and tile
+
+__device__ __forceinline__ int prod_key(int wi, int g, int lane) {   // key of the tile
+    return 16 * wi + 8 * g + 4 * ((lane >> 3) & 1) + ((lane & 7) >> 1);
+}
+__device__ __forceinline__ int prod_piece(int lane) { return 2 * (lane >> 4) + (lane & 1); }
+
 struct Raw {
-    uint4 c[2][8];   // stage 2 h + s: FP4: c[s][0..3] = the 64 code bytes; SWA: c[s][0..7] = 128 codes
-    uint2 sc[2];     // FP4: the stage's 8 scale bytes (E4M3, one per 16 channels)
-    float sigma;     // 1 for an FP4 entry, the row scale of an SWA row, -1 for no key
-    int kind;        // 1 FP4 entry, 2 SWA row, 3 the fused new SWA row (not yet read), 0 zero row,
-                     // -1 nothing
+    uint4 c[kGroups][kStages][2];   // FP4: c[g][j][0] = 32 codes of stage j; SWA: 32 E4M3 codes
+    uint32_t sc[kGroups][2];        // FP4: the 2 scale bytes of stage j at bits 16 (j & 1) of sc[g][j >> 1]
+    float sigma[kGroups];           // 1 for an FP4 entry, the row scale of an SWA row, -1 for no key
+    int kind[kGroups];              // 1 FP4 entry, 2 SWA row, 3 the fused new SWA row (not yet read),
+                                    // 0 zero row, -1 nothing
 };
 
-struct KeyMap {      // the query's keys and where each comes from
+struct KeyMap {      // this CTA's keys and where each comes from
     const int32_t *ids;
     int n_sel;
     int64_t w0;      // first window position
     int n_keys;      // keys of the query (selection + window)
+    int k_end;       // end of this CTA's key range
     int64_t b;
     int64_t ring_base;
     const uint8_t *new_row;   // fused append: the newest window key is this row (smem)
@@ -289,129 +323,121 @@ struct KeyMap {      // the query's keys and where each comes from
     const Smem *smem;
 };
 
-// Issue every load of key kg's two stages (one memory round trip).  The fused new SWA
-// row is only marked here (kind 3): see take_new_row.
-__device__ __forceinline__ void load_key(Raw &r, const AttnArgs &a, const KeyMap &km, int kg, bool zrow, int h) {
-    r.kind = zrow ? 0 : -1;
-    r.sigma = -1.0f;
-    if (kg >= km.n_keys) return;
-    if (kg < km.n_sel) {
-        const int64_t off = cache_row(a.pm, a.cap, km.b, km.ids[kg]);   // checked when compacted
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.codes + off * kCodeBytes + 128 * h);
-        const uint2 *sc = reinterpret_cast<const uint2 *>(a.scales + off * kScaleBytes + 16 * h);
+// Issue every load of the lane's two keys (all four stages: one memory round trip).
+// kg0: the tile's first key; zlim: keys of the tile below zlim are written (zero rows
+// past the valid keys).  The fused new SWA row is only marked here (kind 3).
+__device__ __forceinline__ void load_keys(Raw &r, const AttnArgs &a, const KeyMap &km, int kg0, int zlim,
+                                          int wi, int lane) {
+    const int p = prod_piece(lane);
 #pragma unroll
-        for (int st = 0; st < 2; ++st) {
+    for (int g = 0; g < kGroups; ++g) {
+        const int kt = prod_key(wi, g, lane), kg = kg0 + kt;
+        r.kind[g] = kt < zlim ? 0 : -1;
+        r.sigma[g] = -1.0f;
+        if (kg >= km.k_end) continue;
+        if (kg < km.n_sel) {
+            const int64_t off = cache_row(a.pm, a.cap, km.b, km.ids[kg]);   // checked when compacted
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.codes + off * kCodeBytes + 16 * p);
+            const uint16_t *sc = reinterpret_cast<const uint16_t *>(a.scales + off * kScaleBytes + 2 * p);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) r.c[st][u] = __ldg(src + 4 * st + u);
-            r.sc[st] = __ldg(sc + st);
+            for (int j = 0; j < kStages; ++j) r.c[g][j][0] = __ldg(src + 4 * j);
+            r.sc[g][0] = (uint32_t)__ldg(sc) | ((uint32_t)__ldg(sc + 4) << 16);
+            r.sc[g][1] = (uint32_t)__ldg(sc + 8) | ((uint32_t)__ldg(sc + 12) << 16);
+            r.kind[g] = 1;
+            r.sigma[g] = 1.0f;
+        } else if (km.new_row != nullptr && kg == km.n_keys - 1) {
+            r.kind[g] = 3;
+        } else {
+            const int64_t pos = km.w0 + (kg - km.n_sel);
+            const int64_t slot = km.ring_base + pos % a.wcap;
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.swa_codes + slot * kDim + 32 * p);
+#pragma unroll
+            for (int j = 0; j < kStages; ++j) {
+                r.c[g][j][0] = __ldg(src + 8 * j);
+                r.c[g][j][1] = __ldg(src + 8 * j + 1);
+            }
+            r.sigma[g] = __ldg(a.swa_scale + slot);
+            r.kind[g] = 2;
         }
-        r.kind = 1;
-        r.sigma = 1.0f;
-    } else if (km.new_row != nullptr && kg == km.n_keys - 1) {
-        r.kind = 3;
-    } else {
-        const int64_t pos = km.w0 + (kg - km.n_sel);
-        const int64_t slot = km.ring_base + pos % a.wcap;
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.swa_codes + slot * kDim + 256 * h);
-#pragma unroll
-        for (int st = 0; st < 2; ++st)
-#pragma unroll
-            for (int u = 0; u < 8; ++u) r.c[st][u] = __ldg(src + 8 * st + u);
-        r.sigma = __ldg(a.swa_scale + slot);
-        r.kind = 2;
     }
 }
 
 // Kind 3 -> 2: the fused new SWA row, once warp 1 has quantised it into shared memory
 // (bounded wait; on timeout the key is dropped as a zero row and flagged).
-__device__ __forceinline__ void take_new_row(Raw &r, const AttnArgs &a, const KeyMap &km, int h, bool &new_ok) {
+__device__ __forceinline__ void take_new_row(Raw &r, int g, const AttnArgs &a, const KeyMap &km, int lane,
+                                             bool &new_ok) {
     if (!new_ok) new_ok = mbar_wait(km.new_ready, 0, a.wait.limit_ns, *km.smem);
     if (!new_ok) {
         set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
-        r.kind = 0;
-        r.sigma = -1.0f;
+        r.kind[g] = 0;
+        r.sigma[g] = -1.0f;
         return;
     }
-    const uint4 *src = reinterpret_cast<const uint4 *>(km.new_row + 256 * h);
+    const uint4 *src = reinterpret_cast<const uint4 *>(km.new_row + 32 * prod_piece(lane));
 #pragma unroll
-    for (int st = 0; st < 2; ++st)
-#pragma unroll
-        for (int u = 0; u < 8; ++u) r.c[st][u] = src[8 * st + u];
-    r.sigma = *km.new_sigma;
-    r.kind = 2;
+    for (int j = 0; j < kStages; ++j) {
+        r.c[g][j][0] = src[8 * j];
+        r.c[g][j][1] = src[8 * j + 1];
+    }
+    r.sigma[g] = *km.new_sigma;
+    r.kind[g] = 2;
 }
 
-// Channels 8 u .. 8 u + 7 of the thread's stage st as four f16x2 words (zeros for no key).
-__device__ __forceinline__ void dq8(const Raw &r, int st, int u, uint32_t v[4]) {
-    if (r.kind == 1) {
-        const uint4 cv = r.c[st][u >> 2];
-        const uint32_t w = (u & 3) == 0 ? cv.x : (u & 3) == 1 ? cv.y : (u & 3) == 2 ? cv.z : cv.w;
-        // scale byte u / 2 (one per 16 channels): byte pair (u / 4) % 2 of word u / 8
-        const uint32_t sw = (u >> 3) == 0 ? r.sc[st].x : r.sc[st].y;
-        const uint32_t hs = cvt_e4m3x2_f16x2((sw >> (16 * ((u >> 2) & 1))) & 0xFFFFu);
-        const uint32_t s2 = (((u >> 1) & 1) ? (hs >> 16) : (hs & 0xFFFFu)) * 0x10001u;
-        const __half2 sv = *reinterpret_cast<const __half2 *>(&s2);
-        cvt_e2m1x8_f16x2(w, v);
+// Dequantise stage j of the lane's piece of key row `row` (fp16, swizzled).
+__device__ __forceinline__ void store_piece(const Raw &r, int g, int j, uint8_t *stage, int row, int lane) {
+    const int p = prod_piece(lane);
+    uint8_t *blk = stage + (p >> 1) * kCbBytes;
+    const int c0 = 4 * (p & 1);
+    const int kind = r.kind[g];
+    if (kind == 1) {
+        const uint32_t two = (r.sc[g][j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+        const uint32_t hs = cvt_e4m3x2_f16x2(two);
+        const uint32_t scale2[2] = {(hs & 0xFFFFu) * 0x10001u, (hs >> 16) * 0x10001u};   // per 16 channels
+        const uint4 cv = r.c[g][j][0];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            __half2 x = __hmul2(*reinterpret_cast<__half2 *>(&v[k]), sv);
-            v[k] = *reinterpret_cast<uint32_t *>(&x);
+        for (int c = 0; c < 4; ++c) {                  // 8 channels per 32-bit code word
+            const uint32_t w = c == 0 ? cv.x : c == 1 ? cv.y : c == 2 ? cv.z : cv.w;
+            const __half2 sv = *reinterpret_cast<const __half2 *>(&scale2[c >> 1]);
+            uint32_t v[4];
+            cvt_e2m1x8_f16x2(w, v);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                __half2 x = __hmul2(*reinterpret_cast<__half2 *>(&v[k]), sv);
+                v[k] = *reinterpret_cast<uint32_t *>(&x);
+            }
+            *reinterpret_cast<uint4 *>(blk + swz(row, c0 + c)) = make_uint4(v[0], v[1], v[2], v[3]);
         }
-    } else if (r.kind == 2) {
+    } else if (kind == 2) {
         // exact E4M3 codes; the row scale is applied in fp32 on the logit and on P
-        const uint4 cv = r.c[st][u >> 1];
-        const uint32_t w0 = (u & 1) ? cv.z : cv.x, w1 = (u & 1) ? cv.w : cv.y;
-        v[0] = cvt_e4m3x2_f16x2(w0 & 0xFFFFu);
-        v[1] = cvt_e4m3x2_f16x2(w0 >> 16);
-        v[2] = cvt_e4m3x2_f16x2(w1 & 0xFFFFu);
-        v[3] = cvt_e4m3x2_f16x2(w1 >> 16);
-    } else {
-        v[0] = v[1] = v[2] = v[3] = 0u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {                  // 8 channels = 8 code bytes
+            const uint4 cv = r.c[g][j][c >> 1];
+            const uint32_t w0 = (c & 1) ? cv.z : cv.x, w1 = (c & 1) ? cv.w : cv.y;
+            *reinterpret_cast<uint4 *>(blk + swz(row, c0 + c)) =
+                make_uint4(cvt_e4m3x2_f16x2(w0 & 0xFFFFu), cvt_e4m3x2_f16x2(w0 >> 16),
+                           cvt_e4m3x2_f16x2(w1 & 0xFFFFu), cvt_e4m3x2_f16x2(w1 >> 16));
+        }
+    } else if (kind == 0) {
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4 *>(blk + swz(row, c0 + c)) = z;
     }
 }
 
-// The thread's K row of stage st into TMEM (taddr: lane 32 q, column of the stage's
-// channel 0): 64 columns in four 16-column stores.
-__device__ __forceinline__ void store_k(const Raw &r, int st, uint32_t taddr) {
-#pragma unroll
-    for (int qq = 0; qq < 4; ++qq) {
-        uint32_t v[16];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) dq8(r, st, 4 * qq + c, v + 4 * c);
-        asm volatile(
-            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-            "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr + 16u * (uint32_t)qq),
-            "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-            "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-            : "memory");
-    }
-}
-
-// The thread's V row of stage st into row `row` of the shared-memory stage (fp16, swizzled).
-__device__ __forceinline__ void store_v(const Raw &r, int st, uint8_t *stage, int row) {
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-        uint32_t v[4];
-        dq8(r, st, u, v);
-        *reinterpret_cast<uint4 *>(stage + (u >> 3) * kCbBytes + swz(row, u & 7)) = make_uint4(v[0], v[1], v[2], v[3]);
-    }
-}
-
-// Max (kMax) or sum over the warp's 32 lanes of each of 16 values; lane l ends with the
-// reduction of value l % 16 (a butterfly reduce-scatter over 16 lanes, then one more
-// exchange with the other half-warp).
+// Max (kMax) or sum over the warp's 32 lanes of each of 32 values; lane l ends with
+// the reduction of value l (a butterfly reduce-scatter: 31 shuffles).
 template <bool kMax>
-__device__ __forceinline__ float reduce_scatter16(const float *x, int lane) {
-    float a[8];
+__device__ __forceinline__ float reduce_scatter32(const float *x, int lane) {
+    float a[16];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const bool hi = lane & 8;
-        const float mine = hi ? x[8 + k] : x[k], other = hi ? x[k] : x[8 + k];
-        const float o = __shfl_xor_sync(0xFFFFFFFFu, other, 8);
+    for (int k = 0; k < 16; ++k) {
+        const bool hi = lane & 16;
+        const float mine = hi ? x[16 + k] : x[k], other = hi ? x[k] : x[16 + k];
+        const float o = __shfl_xor_sync(0xFFFFFFFFu, other, 16);
         a[k] = kMax ? fmaxf(mine, o) : mine + o;
     }
 #pragma unroll
-    for (int st = 4; st >= 1; st >>= 1) {
+    for (int st = 8; st >= 1; st >>= 1) {
 #pragma unroll
         for (int k = 0; k < st; ++k) {
             const bool hi = lane & st;
@@ -420,38 +446,40 @@ __device__ __forceinline__ float reduce_scatter16(const float *x, int lane) {
             a[k] = kMax ? fmaxf(mine, o) : mine + o;
         }
     }
-    const float o = __shfl_xor_sync(0xFFFFFFFFu, a[0], 16);
-    return kMax ? fmaxf(a[0], o) : a[0] + o;
+    return a[0];
 }
 
 // ---------------------------------------------------------------------------------------
 // kRope: the fused append rotates the new SWA row first (a separate instantiation, so
-// that the plain kernel carries none of its code).  Grid: (n32 * BT), n32 = ceil(H / 32).
-template <bool kRope>
+// that the plain kernel carries none of its code).  CS: CTAs per query (the cluster,
+// set at launch), 2 or 4.
+template <bool kRope, int CS>
 __global__ void __launch_bounds__(kThreads, 1)
-attn_kernel(AttnArgs a, int n32) {
+attn_kernel(AttnArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem &s = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qi = blockIdx.x / n32, hgrp = blockIdx.x % n32;
+    const uint32_t rank = cluster_rank();
+    const int qi = blockIdx.x / CS;
     const int b = qi / a.Tq;
-    const int h0 = hgrp * kHeads;
+    const int h0 = blockIdx.y * kHeads;
     const int hcta = min(kHeads, a.H - h0);
     const uint64_t lim = a.wait.limit_ns;
     // ---- set-up -----------------------------------------------------------------------------
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&s.kv_full[i], kWorkWarps / 2);   // stage j: the 4 warps of channel half j / 2
+            mbar_init(&s.kv_full[i], kWorkWarps);
             mbar_init(&s.kv_empty[i], 1);
         }
         mbar_init(&s.s_full[0], 1);
         mbar_init(&s.s_full[1], 1);
-        mbar_init(&s.k_full, kWorkWarps);
         mbar_init(&s.p_full, kWorkWarps);
         mbar_init(&s.pv_done, 1);
         mbar_init(&s.drain, 1);
         mbar_init(&s.never, 1);
         mbar_init(&s.new_ready, 1);
+        mbar_init(&s.xfer[0], 1);
+        mbar_init(&s.xfer[1], 1);
         s.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -523,15 +551,15 @@ attn_kernel(AttnArgs a, int n32) {
     const int64_t n_vis = min64(visible_entries((int32_t)t, a.ratio), a.cap);
     auto entry_ok = [&](int e) {
         bool ok = e >= 0 && e < n_vis;
-        if (e >= 0 && !ok && hgrp == 0) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
+        if (e >= 0 && !ok) set_dev_err(a.dev_err, CSA2_DEVERR_INDEX);
         if (ok && cache_row(a.pm, a.cap, b, e) < 0) {
-            if (hgrp == 0) set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
+            set_dev_err(a.dev_err, CSA2_DEVERR_PAGE);
             ok = false;
         }
         return ok;
     };
     const bool e_ok0 = entry_ok(e_id0), e_ok1 = entry_ok(e_id1);
-    if (threadIdx.x == 32 * 3 && a.swa_len > 0 && hgrp == 0) {
+    if (threadIdx.x == 32 * 3 && a.swa_len > 0 && rank == 0) {
         // the request's whole SWA ring (rows are contiguous) and its scales
         prefetch_l2(a.swa_codes + (int64_t)b * a.wcap * kDim, (uint32_t)a.wcap * kDim);
         const float *sg = a.swa_scale + (int64_t)b * a.wcap;   // only whole 16-byte units
@@ -558,31 +586,36 @@ attn_kernel(AttnArgs a, int n32) {
     const uint32_t below = (1u << lane) - 1u;
     if (e_ok0) s.ids[base0 + __popc(bal0 & below)] = e_id0;
     if (e_ok1) s.ids[base1 + __popc(bal1 & below)] = e_id1;
-    const int n_keys = n_sel + n_win;         // the selected entries, then the window
-    const int nt = (n_keys + kTK - 1) / kTK;
+    // this CTA's key range: the query's keys cut in CS chunks of a multiple of 16
+    const int n_keys = n_sel + n_win;
+    const int chunk = ((n_keys + CS - 1) / CS + 15) / 16 * 16;
+    const int k0 = min(n_keys, (int)rank * chunk), k1 = min(n_keys, k0 + chunk);
+    const int nt = (k1 - k0 + kTK - 1) / kTK;
     const bool fuse = a.swa_new != nullptr && n_win > 0;
+    const uint32_t owner = n_keys > 0 ? (uint32_t)((n_keys - 1) / chunk) : 0u;   // holds the newest key
     KeyMap km;
     km.ids = s.ids;
     km.n_sel = n_sel;
     km.w0 = w0;
     km.n_keys = n_keys;
+    km.k_end = k1;
     km.b = b;
     km.ring_base = (int64_t)b * a.wcap;
-    km.new_row = fuse ? s.swa_new : nullptr;
+    km.new_row = fuse && rank == owner ? s.swa_new : nullptr;
     km.new_sigma = &s.swa_new_sigma;
     km.new_ready = &s.new_ready;
     km.smem = &s;
     const bool worker = warp >= kWorkWarp0;
-    // worker: key quadrant, and half (the softmax's 16 heads, the producer's 256 channels)
-    const int qd = warp & 3, hh = (warp - kWorkWarp0) >> 2;
-    const int r = 32 * qd + lane;                              // worker: key of the tile
+    const int qd = warp & 3, hh = (warp - kWorkWarp0) >> 2;   // worker: key quadrant, head / channel half
+    const int r = 32 * qd + lane;                              // worker softmax: key of the tile
+    const int wi = warp - kWorkWarp0;                          // worker producer: keys 16 wi ..
     // rows of the tile's last 16-key group of valid keys are read by the output MMAs
     // and so written (zeros past the keys); rows after that group are not written
-    auto zlim_of = [&](int i) { return ((min(kTK, n_keys - i * kTK) + 15) / 16) * 16; };
+    auto zlim_of = [&](int i) { return ((min(kTK, k1 - k0 - i * kTK) + 15) / 16) * 16; };
     bool new_ok = false;
     Raw raw;
     __syncthreads();                       // s.ids complete
-    if (worker && nt > 0) load_key(raw, a, km, r, r < zlim_of(0), hh);   // tile 0, in flight
+    if (worker && nt > 0) load_keys(raw, a, km, k0, zlim_of(0), wi, lane);   // tile 0, in flight
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -593,59 +626,52 @@ attn_kernel(AttnArgs a, int n32) {
         // ---------------- MMA issuer (whole warp runs the loop; one lane issues) ----------------
         if (nt > 0) {
             bool ok = true;
-            // S^T = K Q^T: A = stage (K-major, 128 keys), B = Q (K-major, 32 heads), M 128 N 32
+            // S^T = K Q^T: A = stage (K-major, 128 keys), B = Q (K-major, 64 heads), M 128 N 64
             const uint32_t idesc_s = (1u << 4) | ((uint32_t)(kHeads >> 3) << 17) | ((uint32_t)(kTK >> 4) << 24);
-            // O^T = V^T P^T: A = stage (MN-major, 128 channels), B = P^T (MN-major, 32 heads)
+            // O^T = V^T P^T: A = stage (MN-major, 128 channels), B = P^T (MN-major, 64 heads)
             const uint32_t idesc_o = (1u << 4) | (1u << 15) | (1u << 16) | ((uint32_t)(kHeads >> 3) << 17) |
                                      ((uint32_t)(kTK >> 4) << 24);
             const uint64_t qd_desc = sw128_desc(smem_u32(s.q), 16, 1024);
-            // P^T rows are 64 bytes (32 heads): 8-row groups 512 bytes apart
-            const uint64_t pd = sw64_desc(smem_u32(s.pt), 4096, 512);
-            // S^T(i) once K(i) is in TMEM (A from TMEM: the 8 columns of 16 channels per step)
-            auto issue_s = [&](int i) -> bool {
-                const bool got = __shfl_sync(0xFFFFFFFFu, (int)mbar_wait(&s.k_full, i & 1, lim, s), 0) != 0;
-                if (!got) return false;
-                tc_fence_after();
-                if (elect_one()) {
-                    const uint32_t sd = tmem + kSCol + (uint32_t)kHeads * (uint32_t)(i & 1);
-#pragma unroll 4
-                    for (int k = 0; k < 32; ++k) {      // K-steps of 16 channels
-                        const uint64_t boff = (uint64_t)((k >> 2) * (kQCbBytes >> 4) + (k & 3) * 2);
-                        mma_f16_ta(sd, tmem + kKCol + 8u * (uint32_t)k, qd_desc + boff, idesc_s, k != 0 ? 1u : 0u);
-                    }
-                    mma_commit(&s.s_full[i & 1]);
-                }
-                __syncwarp();
-                return true;
-            };
-            ok = issue_s(0);
+            const uint64_t pd = sw128_desc(smem_u32(s.pt), 8192, 1024);
             for (int i = 0; ok && i < nt; ++i) {
-                // the next tile's scores first: they run while the softmax of this tile does
-                if (i + 1 < nt && !(ok = issue_s(i + 1))) break;
-                // P^T(i) from the softmax (the test hook makes the first of these waits stuck)
-                const bool got = a.wait.stuck && i == 0 ? mbar_wait(&s.never, 0, lim, s)
-                                                        : mbar_wait(&s.p_full, i & 1, lim, s);
-                ok = __shfl_sync(0xFFFFFFFFu, (int)got, 0) != 0;
-                if (!ok) break;
-                tc_fence_after();
-                const int nk = (min(kTK, n_keys - i * kTK) + 15) / 16;   // K-steps of valid keys
+                const uint32_t sd = tmem + kSCol + 64u * (uint32_t)(i & 1);
 #pragma unroll 1
                 for (int j = 0; j < kStages; ++j) {
                     ok = __shfl_sync(0xFFFFFFFFu, (int)mbar_wait(&s.kv_full[j], i & 1, lim, s), 0) != 0;
                     if (!ok) break;
                     tc_fence_after();
                     if (elect_one()) {
-                        const uint64_t vd = sw128_desc(smem_u32(s.kv[j]), kCbBytes, 1024);
+                        const uint64_t kd = sw128_desc(smem_u32(s.kv[j]), 16, 1024);
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)    // 16 keys per step: 2048 B of V^T, 1024 B of P^T
-                            if (kk < nk)
-                                mma_f16(tmem + (uint32_t)kHeads * (uint32_t)j, vd + (uint64_t)(kk * 128),
-                                        pd + (uint64_t)(kk * 64), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-                        mma_commit(&s.kv_empty[j]);
-                        if (j == kStages - 1) mma_commit(&s.pv_done);
+                        for (int k = 0; k < 8; ++k) {       // K-steps of 16 channels
+                            const uint64_t aoff = (uint64_t)((k >> 2) * (kCbBytes >> 4) + (k & 3) * 2);
+                            const uint64_t boff = (uint64_t)((2 * j + (k >> 2)) * (kQCbBytes >> 4) + (k & 3) * 2);
+                            mma_f16(sd, kd + aoff, qd_desc + boff, idesc_s, (j | k) != 0 ? 1u : 0u);
+                        }
+                        if (j == kStages - 1) mma_commit(&s.s_full[i & 1]);
                     }
                     __syncwarp();
                 }
+                if (!ok) break;
+                // P^T(i) from the softmax (the test hook makes the first of these waits stuck)
+                const bool got = a.wait.stuck && i == 0 ? mbar_wait(&s.never, 0, lim, s)
+                                                        : mbar_wait(&s.p_full, i & 1, lim, s);
+                ok = __shfl_sync(0xFFFFFFFFu, (int)got, 0) != 0;
+                if (!ok) break;
+                tc_fence_after();
+                const int nk = (min(kTK, k1 - k0 - i * kTK) + 15) / 16;   // K-steps of valid keys
+                if (elect_one()) {
+#pragma unroll 1
+                    for (int j = 0; j < kStages; ++j) {
+                        const uint64_t vd = sw128_desc(smem_u32(s.kv[j]), kCbBytes, 1024);
+                        for (int kk = 0; kk < nk; ++kk)
+                            mma_f16(tmem + 64u * (uint32_t)j, vd + (uint64_t)(kk * 128), pd + (uint64_t)(kk * 128),
+                                    idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(&s.kv_empty[j]);
+                    }
+                    mma_commit(&s.pv_done);
+                }
+                __syncwarp();
             }
             if (!ok && lane == 0) {
                 atomicExch(&s.abort, 1);
@@ -658,22 +684,22 @@ attn_kernel(AttnArgs a, int n32) {
             (void)drained;
         }
     } else if (warp == 1) {
-        if (fuse) {
+        if (fuse && rank == owner) {
             // The same FP8 row quantiser as csa2_quantize_append: codes and sigma go to
-            // shared memory (the workers read the window's newest key from there, after
-            // new_ready) and, from head group 0, to the ring slot t % wcap.
+            // shared memory (this CTA's workers read the window's newest key from there,
+            // after new_ready) and, from head group 0, to the ring slot t % wcap.
             float xnew[16];
             unpack_bf16x8(xraw[0], xnew);
             unpack_bf16x8(xraw[1], xnew + 8);
             if constexpr (kRope) {
                 if (!rope_lane16(xnew, lane, a.rope.cs, a.rope.n_pos, a.rope.start, a.rope.pairs, t) &&
-                    lane == 0 && hgrp == 0)
+                    lane == 0)
                     set_dev_err(a.dev_err, CSA2_DEVERR_ROPE);
             }
             quant_fp8_lanes<kDim>(xnew, s.swa_new, &s.swa_new_sigma, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.new_ready);
-            if (hgrp == 0) {
+            if (blockIdx.y == 0) {
                 const int64_t slot = (int64_t)b * a.wcap + t % a.wcap;
                 reinterpret_cast<uint4 *>(a.swa_codes + slot * kDim)[lane] =
                     reinterpret_cast<const uint4 *>(s.swa_new)[lane];
@@ -681,88 +707,71 @@ attn_kernel(AttnArgs a, int n32) {
             }
         }
     } else if (warp == 2) {
-        // L2 prefetch of the entries of the later tiles (tile 0 is already in flight), by
-        // one head group (the others read the same rows)
-        if (hgrp == 0) {
-            for (int kg = kTK + lane; kg < n_sel; kg += 32) {
-                const int64_t row = cache_row(a.pm, a.cap, b, s.ids[kg]);
-                prefetch_l2(a.codes + row * kCodeBytes, kCodeBytes);
-                prefetch_l2(a.scales + row * kScaleBytes, kScaleBytes);
-            }
+        // L2 prefetch of the entries of this CTA's later tiles (tile 0 is already in flight)
+        for (int kg = k0 + kTK + lane; kg < min(k1, n_sel); kg += 32) {
+            const int64_t row = cache_row(a.pm, a.cap, b, s.ids[kg]);
+            prefetch_l2(a.codes + row * kCodeBytes, kCodeBytes);
+            prefetch_l2(a.scales + row * kScaleBytes, kScaleBytes);
         }
     } else if (worker) {
-        // ---------------- workers ----------------
-        // Tile i: wait for S^T(i); write K(i + 1) into TMEM (S^T(i) no longer reads it), so
-        // that S^T(i + 1) runs during this softmax; the softmax of tile i (keys 32 qd ..,
-        // heads 16 hh ..) -> P^T(i); V(i + 1) into the shared-memory stages as O^T(i)
-        // releases them; then the raw bytes of tile i + 2.
+        // ---------------- workers: produce tile i + 1 after the softmax of tile i ----------------
+        // Softmax: keys 32 qd .. (TMEM lanes), heads 32 hh .. .  Producer: keys 16 wi ..
+        // (prod_key); the raw bytes of the next tile are in registers while the softmax of
+        // this one runs.
         const float c0 = a.softmax_scale * 1.4426950408889634f * exp2f((float)qexp);
         const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
-        const float4 *mrun4 = reinterpret_cast<const float4 *>(&s.mrun[16 * hh]);
-        float lsum = 0.0f;   // head 16 hh + lane % 16: this warp's keys' share of l
+        const float4 *mrun4 = reinterpret_cast<const float4 *>(&s.mrun[32 * hh]);
+        float lsum = 0.0f;   // head 32 hh + lane: partial sum over this warp's keys
         bool ok = true, stop = false;
-        // K of the thread's key and channel half into TMEM; arrive k_full
-        auto put_k = [&]() {
-            if (raw.kind == 3) take_new_row(raw, a, km, hh, new_ok);
-#pragma unroll
-            for (int st = 0; st < 2; ++st)
-                store_k(raw, st, tmem + lane_base + kKCol + 64u * (uint32_t)(2 * hh + st));
-            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.k_full);
-        };
-        // V of the thread's key and channel half into stages 2 hh, 2 hh + 1 of tile i (after
-        // O^T(i - 1) has released them); s.ksig of the tile; arrive kv_full
-        auto put_v = [&](int i) -> bool {
-#pragma unroll
-            for (int st = 0; st < 2; ++st) {
-                const int j = 2 * hh + st;
-                if (i > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&s.kv_empty[j], (i - 1) & 1, lim, s))) return false;
-                if (raw.kind >= 0) store_v(raw, st, s.kv[j], r);
-                if (st == 0 && hh == 0) {
-                    s.ksig[r] = raw.sigma;
-                    // P carries sigma in fp16: p <= 2^8 needs sigma <= 65504 / 256
-                    if (raw.kind == 2 && raw.sigma * 256.0f > 65504.0f && hgrp == 0)
-                        set_dev_err(a.dev_err, CSA2_DEVERR_RANGE);
-                }
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s.kv_full[j]);
-            }
-            return true;
-        };
-        if (nt > 0) {
-            put_k();
-            ok = put_v(0);
-            if (ok && nt > 1) load_key(raw, a, km, kTK + r, r < zlim_of(1), hh);
-        }
         for (int i = 0; i < nt; ++i) {
-            // ---- S^T(i) and the tile's key scales; the four warps of the half agree ----
-            // (kv_full[2 hh] of tile i: the ksig writes of this half's... every h = 0 warp;
-            // kv_full[0] covers them)
+            // ---- produce tile i (its stages are free once O^T(i - 1) has read them) ----
+            if (ok) {
+#pragma unroll
+                for (int g = 0; g < kGroups; ++g)
+                    if (raw.kind[g] == 3) take_new_row(raw, g, a, km, lane, new_ok);
+#pragma unroll
+                for (int j = 0; j < kStages; ++j) {   // unrolled: raw.c[.][j] stays in registers
+                    if (i > 0) {
+                        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.kv_empty[j], (i - 1) & 1, lim, s));
+                        if (!ok) break;
+                    }
+#pragma unroll
+                    for (int g = 0; g < kGroups; ++g) {
+                        const int kt = prod_key(wi, g, lane);
+                        store_piece(raw, g, j, s.kv[j], kt, lane);
+                        if (j == 0 && prod_piece(lane) == 0) {
+                            const float sg = raw.sigma[g];
+                            s.ksig[kt] = sg;
+                            // P carries sigma in fp16: p <= 2^8 needs sigma <= 65504 / 256
+                            if (raw.kind[g] == 2 && sg * 256.0f > 65504.0f) set_dev_err(a.dev_err, CSA2_DEVERR_RANGE);
+                        }
+                    }
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.kv_full[j]);
+                }
+                if (ok && i + 1 < nt) load_keys(raw, a, km, k0 + (i + 1) * kTK, zlim_of(i + 1), wi, lane);
+            }
+            // ---- softmax of tile i: every wait first; the four warps of the half agree ----
+            // (kv_full[0] of tile i: every worker's s.ksig of the tile is written)
             const bool w_ok = ok && __all_sync(0xFFFFFFFFu, mbar_wait(&s.s_full[i & 1], (i >> 1) & 1, lim, s) &&
-                                                                mbar_wait(&s.kv_full[0], i & 1, lim, s));
+                                                                mbar_wait(&s.kv_full[0], i & 1, lim, s) &&
+                                                                (i == 0 || mbar_wait(&s.pv_done, (i - 1) & 1, lim, s)));
             stop = group_any(hh, !w_ok || aborted(s));
             if (stop) break;
             tc_fence_after();
-            float x[16];
-            tmem_ld16(tmem + lane_base + kSCol + (uint32_t)kHeads * (uint32_t)(i & 1) + 16u * (uint32_t)hh, x);
-            // ---- K(i + 1) into TMEM: every lane of this warp has read S^T(i), which was
-            // the last reader of K(i) ----
-            tc_fence_before();
-            if (i + 1 < nt) put_k();
-            // ---- softmax of tile i ----
+            float x[32];
+            tmem_ld32(tmem + lane_base + kSCol + 64u * (uint32_t)(i & 1) + 32u * (uint32_t)hh, x);
             const float sig = s.ksig[r];
             const bool valid = sig >= 0.0f;
             const float ck = c0 * sig;
             float dmax = -INFINITY;
 #pragma unroll
-            for (int h = 0; h < 16; ++h) x[h] = valid ? x[h] * ck : -INFINITY;   // logits, log2 units
+            for (int h = 0; h < 32; ++h) x[h] = valid ? x[h] * ck : -INFINITY;   // logits, log2 units
             if (i > 0) {
                 // x -> x - m in place: the lazy check, and (common case) the exponent of p
 #pragma unroll
-                for (int h4 = 0; h4 < 4; ++h4) {
+                for (int h4 = 0; h4 < 8; ++h4) {
                     const float4 mv = mrun4[h4];
                     x[4 * h4] -= mv.x; x[4 * h4 + 1] -= mv.y; x[4 * h4 + 2] -= mv.z; x[4 * h4 + 3] -= mv.w;
                     dmax = fmaxf(dmax, fmaxf(fmaxf(x[4 * h4], x[4 * h4 + 1]), fmaxf(x[4 * h4 + 2], x[4 * h4 + 3])));
@@ -772,73 +781,63 @@ attn_kernel(AttnArgs a, int n32) {
             if (upd) {
                 if (i > 0) {   // back to the logits (one rounding; p's exponent stays consistent)
 #pragma unroll
-                    for (int h4 = 0; h4 < 4; ++h4) {
+                    for (int h4 = 0; h4 < 8; ++h4) {
                         const float4 mv = mrun4[h4];
                         x[4 * h4] += mv.x; x[4 * h4 + 1] += mv.y; x[4 * h4 + 2] += mv.z; x[4 * h4 + 3] += mv.w;
                     }
                 }
                 // exact tile max per head, then the running max moves
-                const float wm = reduce_scatter16<true>(x, lane);   // head 16 hh + lane % 16
-                if (lane < 16) s.red[hh][qd][lane] = wm;
+                const float wm = reduce_scatter32<true>(x, lane);   // head 32 hh + lane
+                s.red[hh][qd][lane] = wm;
                 group_sync(hh);
-                if (qd == 0 && lane < 16) {
+                if (qd == 0) {
                     const float tm = fmaxf(fmaxf(s.red[hh][0][lane], s.red[hh][1][lane]),
                                            fmaxf(s.red[hh][2][lane], s.red[hh][3][lane]));
-                    const float old = i > 0 ? s.mrun[16 * hh + lane] : -INFINITY;
+                    const float old = i > 0 ? s.mrun[32 * hh + lane] : -INFINITY;
                     const float mn = fmaxf(old, tm);
-                    s.mrun[16 * hh + lane] = mn;
-                    s.alpha[16 * hh + lane] = old == -INFINITY ? 0.0f : ex2(old - mn);
+                    s.mrun[32 * hh + lane] = mn;
+                    s.alpha[32 * hh + lane] = old == -INFINITY ? 0.0f : ex2(old - mn);
                 }
                 group_sync(hh);
-                lsum *= s.alpha[16 * hh + (lane & 15)];
+                lsum *= s.alpha[32 * hh + lane];
 #pragma unroll
-                for (int h4 = 0; h4 < 4; ++h4) {
+                for (int h4 = 0; h4 < 8; ++h4) {
                     const float4 mv = mrun4[h4];
                     x[4 * h4] -= mv.x; x[4 * h4 + 1] -= mv.y; x[4 * h4 + 2] -= mv.z; x[4 * h4 + 3] -= mv.w;
                 }
             }
             // p = 2^(x - m); P^T carries the key's scale (V holds SWA codes, not values)
             const float sv = valid ? sig : 0.0f;
-            uint32_t pk[8];
+            uint32_t pk[16];
 #pragma unroll
-            for (int h2 = 0; h2 < 8; ++h2) {
+            for (int h2 = 0; h2 < 16; ++h2) {
                 const float p0 = ex2(x[2 * h2]), p1 = ex2(x[2 * h2 + 1]);
                 x[2 * h2] = p0;
                 x[2 * h2 + 1] = p1;
                 pk[h2] = pack_h2(p0 * sv, p1 * sv);
             }
 #pragma unroll
-            for (int c = 0; c < 2; ++c)   // heads 16 hh + 8 c .. : chunk 2 hh + c of the key's row
-                *reinterpret_cast<uint4 *>(s.pt + swz64(r, 2 * hh + c)) =
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<uint4 *>(s.pt + swz(r, 4 * hh + c)) =
                     make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
             if (upd && i > 0) {
-                // the running max moved: wait for O^T(i - 1) (issued after S^T(i + 1), so not
-                // implied by s_full(i)), then scale this warp's 16 head columns of every block
-                // before O^T(i) accumulates on them
-                const bool pv = __all_sync(0xFFFFFFFFu, mbar_wait(&s.pv_done, (i - 1) & 1, lim, s));
-                if (!pv && lane == 0) {
-                    atomicExch(&s.abort, 1);
-                    set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
-                }
-                tc_fence_after();
-                float f[16];
-#pragma unroll
-                for (int h = 0; h < 16; ++h) f[h] = s.alpha[16 * hh + h];
+                // the running max moved: O^T(i - 1) has landed (pv_done above); scale this
+                // warp's 32 head columns of every block before O^T(i) accumulates on them
 #pragma unroll 1
-                for (int j = 0; j < kStages; ++j)
-                    tmem_scale16(tmem + lane_base + (uint32_t)kHeads * (uint32_t)j + 16u * (uint32_t)hh, f);
+                for (int j = 0; j < 2 * kStages; ++j) {    // 16 head columns at a time
+                    float f[16];
+#pragma unroll
+                    for (int h = 0; h < 16; ++h) f[h] = s.alpha[32 * hh + 16 * (j & 1) + h];
+                    tmem_scale16(tmem + lane_base + 64u * (uint32_t)(j >> 1) + 32u * (uint32_t)hh + 16u * (uint32_t)(j & 1), f);
+                }
                 asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             }
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s.p_full);
-            lsum += reduce_scatter16<false>(x, lane);   // this tile's 32 keys, after P^T is released
-            // ---- V(i + 1) into the stages as O^T(i) releases them; raw bytes of tile i + 2 ----
-            if (ok && i + 1 < nt) {
-                ok = put_v(i + 1);
-                if (ok && i + 2 < nt) load_key(raw, a, km, (i + 2) * kTK + r, r < zlim_of(i + 2), hh);
-            }
+            // l after P is released: the sum is off the output MMAs' critical path
+            lsum += reduce_scatter32<false>(x, lane);   // this tile's 32 keys, head 32 hh + lane
         }
         ok = ok && !stop;
         if (ok && nt > 0) {
@@ -849,52 +848,159 @@ attn_kernel(AttnArgs a, int n32) {
             atomicExch(&s.abort, 1);
             set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
         }
-        // the sum per head over the four quadrants; 1 / l and the log-sum-exp (the group
-        // barrier is taken by all four warps of the half, aborted or not)
-        if (lane < 16) s.red[hh][qd][lane] = lsum;
+        // this CTA's partial sum per head: the four quadrants' sums (the group barrier is
+        // taken by all four warps of the half, aborted or not)
+        s.red[hh][qd][lane] = lsum;
         group_sync(hh);
-        if (qd == 0 && lane < 16) {
-            const int h = 16 * hh + lane;
+        if (qd == 0) {
             const bool have = nt > 0 && !aborted(s);
-            const float l = have ? s.red[hh][0][lane] + s.red[hh][1][lane] + s.red[hh][2][lane] + s.red[hh][3][lane]
-                                 : 0.0f;
-            const bool valid = h < hcta && l > 0.0f;
-            s.wfin[h] = valid ? 1.0f / l : 0.0f;
-            if (h < hcta)
-                a.lse[(int64_t)qi * a.H + h0 + h] =
-                    valid ? (s.mrun[h] + log2f(l)) * 0.6931471805599453f : -INFINITY;
+            s.cl[32 * hh + lane] = have ? s.red[hh][0][lane] + s.red[hh][1][lane] + s.red[hh][2][lane] +
+                                              s.red[hh][3][lane]
+                                        : 0.0f;
+            s.cm[32 * hh + lane] = have ? s.mrun[32 * hh + lane] : -INFINITY;
         }
     }
 
-    // ---- output: O^T / l, straight from TMEM --------------------------------------------------
+    // ---- combine the two key halves of the query through distributed shared memory ----
+    // CTA r writes channels [256 r, 256 r + 256) = O^T blocks 2 r, 2 r + 1.  Every thread
+    // of both CTAs takes every cluster barrier, whatever happened above.
     __syncwarp();
     tc_fence_before();
-    __syncthreads();                       // 1 / l written; every MMA of the CTA has completed
+    __syncthreads();                       // stats written; this CTA's MMAs have completed
     tc_fence_after();
-    grid_dep_launch();
-    // Task u (32; warp u % 12 takes u, so the TMEM lane quadrant u % 4 is the warp's):
-    // channels 32 (u % 4) .. of block (u >> 2) & 3, heads 16 (u >> 4) .. .  A thread holds
-    // one channel of 16 heads; a warp store covers 32 consecutive channels of one head.
-    const bool have = __shfl_sync(0xFFFFFFFFu, (int)(nt > 0 && !aborted(s)), 0) != 0;
-#pragma unroll 1
-    for (int u = warp; u < 32; u += kWarps) {
-        const int cq = u & 3, blk = (u >> 2) & 3, hp = u >> 4;
-        float o[16];
-        if (have) {
-            tmem_ld16(tmem + ((uint32_t)(32 * cq) << 16) + (uint32_t)kHeads * (uint32_t)blk + 16u * (uint32_t)hp, o);
+    // Every CTA owns NB = 4 / CS of the four 128-channel blocks (blocks NB r ..): it sends
+    // its partial of every other CTA's blocks (scaled by its weight) into that CTA's
+    // shared memory and adds what the others sent it to its own.
+    constexpr int NB = 4 / CS;
+    constexpr uint32_t kPiece = NB * kTK * (kHeads / 2) * 4;   // one peer's blocks, one head half, fp32
+    constexpr int kPieceF = (int)(kPiece / 4);
+    for (int i = threadIdx.x; i < CS * kHeads; i += kThreads) {   // stats to every CTA, own slot `rank`
+        const int r2 = i / kHeads, h = i % kHeads;
+        if (r2 == (int)rank) {
+            s.pm[rank][h] = s.cm[h];
+            s.pl[rank][h] = s.cl[h];
         } else {
-#pragma unroll
-            for (int h = 0; h < 16; ++h) o[h] = 0.0f;
-        }
-        float *dst = a.out + ((int64_t)qi * a.H + h0) * kDim + 128 * blk + 32 * cq + lane;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const int h = 16 * hp + k;
-            if (h < hcta) dst[(int64_t)h * kDim] = o[k] * s.wfin[h];
+            st_peer(peer_addr(&s.pm[rank][h], (uint32_t)r2), s.cm[h]);
+            st_peer(peer_addr(&s.pl[rank][h], (uint32_t)r2), s.cl[h]);
         }
     }
+    if (threadIdx.x == 0) {                // armed before any peer can send
+        mbar_expect_tx(&s.xfer[0], (CS - 1) * kPiece);
+        mbar_expect_tx(&s.xfer[1], (CS - 1) * kPiece);
+    }
+    cluster_sync();                        // stats exchanged; every CTA's tiles are free
+    grid_dep_launch();
+    if (threadIdx.x < kHeads) {
+        const int h = threadIdx.x;
+        float m_all = -INFINITY;
+#pragma unroll
+        for (int r2 = 0; r2 < CS; ++r2) m_all = fmaxf(m_all, s.pm[r2][h]);
+        float l_all = 0.0f, f_self = 0.0f;
+        if (m_all != -INFINITY) {
+#pragma unroll
+            for (int r2 = 0; r2 < CS; ++r2) {
+                const float f = s.pm[r2][h] == -INFINITY ? 0.0f : ex2(s.pm[r2][h] - m_all);
+                l_all += s.pl[r2][h] * f;
+                if (r2 == (int)rank) f_self = f;
+            }
+        }
+        const bool valid = h < hcta && l_all > 0.0f;
+        s.wself[h] = valid ? f_self / l_all : 0.0f;
+        if (rank == 0 && h < hcta)
+            a.lse[(int64_t)qi * a.H + h0 + h] = valid ? (m_all + log2f(l_all)) * 0.6931471805599453f : -INFINITY;
+    }
+    __syncthreads();
+    // Send slot j (0 .. CS - 2) holds the part for peer (rank + 1 + j) % CS; it lands in
+    // that peer's receive slot CS - 2 - j (so receive slot i holds what CTA
+    // (peer + 1 + i) % CS sent).  A slot is [2 head halves][NB blocks][128 channels][32
+    // heads] fp32, float4 units swizzled by channel; receive slots fill s.kv from the
+    // start, send slots follow them in s.kv and then s.q (both free by now).
+    // Task u (warp u % 12 takes u, so the TMEM lane quadrant u % 4 is the warp's):
+    // channels 32 (u % 4) .., head half (u >> 2) & 1, block bsel / send slot from u >> 3.
+    const bool have = __shfl_sync(0xFFFFFFFFu, (int)(nt > 0 && !aborted(s)), 0) != 0;
+    auto recv_slot = [&](int i) { return reinterpret_cast<float *>(&s.kv[0][0]) + i * 2 * kPieceF; };
+    auto send_slot = [&](int j) {
+        const int k = (CS - 1) + j;        // slot index in the sequence s.kv, then s.q
+        return k * 2 * kPieceF < (int)(sizeof(s.kv) / 4)
+                   ? reinterpret_cast<float *>(&s.kv[0][0]) + k * 2 * kPieceF
+                   : reinterpret_cast<float *>(s.q) + (k * 2 * kPieceF - (int)(sizeof(s.kv) / 4));
+    };
+#pragma unroll 1
+    for (int u = warp; u < 8 * NB * (CS - 1); u += kWarps) {
+        const int cq = u & 3, hp = (u >> 2) & 1, bsel = (u >> 3) % NB, j = (u >> 3) / NB;
+        const int pr = ((int)rank + 1 + j) % CS;
+        const int crow = 32 * cq + lane;             // channel within a block
+        const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)hp;
+        float o[32];
+        if (have) {
+            tmem_ld32(taddr + 64u * (uint32_t)(NB * pr + bsel), o);
+        } else {
+#pragma unroll
+            for (int h = 0; h < 32; ++h) o[h] = 0.0f;
+        }
+        float4 *dst = reinterpret_cast<float4 *>(send_slot(j) + hp * kPieceF + (bsel * kTK + crow) * (kHeads / 2));
+#pragma unroll
+        for (int f = 0; f < 8; ++f) {                // float4 f = heads 32 hp + 4 f ..
+            const int h = 32 * hp + 4 * f;
+            dst[f ^ (crow & 7)] = make_float4(o[4 * f] * s.wself[h], o[4 * f + 1] * s.wself[h + 1],
+                                              o[4 * f + 2] * s.wself[h + 2], o[4 * f + 3] * s.wself[h + 3]);
+        }
+    }
+    fence_async_smem();                    // generic-proxy writes of `send` -> the bulk copy
+    __syncthreads();
+    if (threadIdx.x < 2 * (CS - 1)) {      // one copy per (peer, head half)
+        const int j = threadIdx.x >> 1, hp = threadIdx.x & 1;
+        const uint32_t pr = (uint32_t)(((int)rank + 1 + j) % CS);
+        const uint32_t dst = peer_addr(recv_slot(CS - 2 - j) + hp * kPieceF, pr);
+        bulk_copy_to_peer(dst, send_slot(j) + hp * kPieceF, kPiece, peer_addr(&s.xfer[hp], pr));
+    }
+    bool got_all = true;
+#pragma unroll 1
+    for (int u = warp; u < 8 * NB; u += kWarps) {
+        const int cq = u & 3, hp = (u >> 2) & 1, bsel = u >> 3;
+        const int crow = 32 * cq + lane;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)hp;
+        float own[32];
+        if (have) {
+            tmem_ld32(taddr + 64u * (uint32_t)(NB * (int)rank + bsel), own);
+        } else {
+#pragma unroll
+            for (int h = 0; h < 32; ++h) own[h] = 0.0f;
+        }
+        const bool got = __all_sync(0xFFFFFFFFu, mbar_wait<false>(&s.xfer[hp], 0, kDrainLimitNs, s));
+        got_all = got_all && got;
+#pragma unroll
+        for (int f = 0; f < 8; ++f) {
+            const int h = 32 * hp + 4 * f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) own[4 * f + k] *= s.wself[h + k];
+        }
+#pragma unroll 1
+        for (int i = 0; i < CS - 1; ++i) {           // the senders in a fixed order
+            const float4 *src = reinterpret_cast<const float4 *>(recv_slot(i) + hp * kPieceF +
+                                                                 (bsel * kTK + crow) * (kHeads / 2));
+#pragma unroll
+            for (int f = 0; f < 8; ++f) {
+                const float4 pr = got ? src[f ^ (crow & 7)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                own[4 * f] += pr.x; own[4 * f + 1] += pr.y; own[4 * f + 2] += pr.z; own[4 * f + 3] += pr.w;
+            }
+        }
+        float *obase = a.out + ((int64_t)qi * a.H + h0) * kDim + 128 * (NB * (int)rank + bsel) + crow;
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+            if (32 * hp + k < hcta) obase[(int64_t)(32 * hp + k) * kDim] = own[k];
+    }
+    if (!got_all && lane == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+    // A warp with no task for a head half still waits for it, so that every incoming
+    // copy has landed before the closing barrier.
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait<false>(&s.xfer[0], 0, kDrainLimitNs, s) &&
+                                     mbar_wait<false>(&s.xfer[1], 0, kDrainLimitNs, s)) &&
+        lane == 0)
+        set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+    // Every CTA has seen its incoming copies land, so every outgoing copy has finished
+    // reading its send slot: only now may a CTA leave (and its shared memory be reused).
     tc_fence_before();
-    __syncthreads();                       // every TMEM load of the CTA has completed
+    cluster_sync();
     tc_fence_after();
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
@@ -904,22 +1010,40 @@ attn_kernel(AttnArgs a, int n32) {
 
 size_t attn_smem_bytes() { return sizeof(attn::Smem) + 1024; }
 
-template <bool kRope>
-static cudaError_t launch_attn_t(const AttnArgs &a, int BT, cudaStream_t st) {
+template <bool kRope, int CS>
+static cudaError_t launch_attn_t(const AttnArgs &a, int BT, int hg, cudaStream_t st) {
     const size_t smem = attn_smem_bytes();
     static std::atomic<uint64_t> configured{0};   // per device
     {
-        cudaError_t e = config_kernel_once(attn::attn_kernel<kRope>, smem, configured);
+        cudaError_t e = config_kernel_once(attn::attn_kernel<kRope, CS>, smem, configured);
         if (e != cudaSuccess) return e;
     }
-    const int n32 = (a.H + attn::kHeads - 1) / attn::kHeads;
-    cudaError_t e = launch_pdl(attn::attn_kernel<kRope>, dim3(n32 * BT), dim3(attn::kThreads), smem, st, a, n32);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(CS * BT, hg);
+    cfg.blockDim = dim3(attn::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;   // the CS CTAs of a query
+    attr[1].val.clusterDim.x = CS;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, attn::attn_kernel<kRope, CS>, a);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+// 4 CTAs per query when the whole grid still fits the SMs once (small batches: shorter
+// per-query latency), else 2.
 cudaError_t launch_sparse_attn(const AttnArgs &a, int BT, cudaStream_t st) {
-    return a.swa_new != nullptr && a.rope.cs != nullptr ? launch_attn_t<true>(a, BT, st)
-                                                         : launch_attn_t<false>(a, BT, st);
+    const int hg = (a.H + attn::kHeads - 1) / attn::kHeads;
+    const bool four = (int64_t)4 * BT * hg <= device_sm_count();
+    const bool rope = a.swa_new != nullptr && a.rope.cs != nullptr;
+    if (four) return rope ? launch_attn_t<true, 4>(a, BT, hg, st) : launch_attn_t<false, 4>(a, BT, hg, st);
+    return rope ? launch_attn_t<true, 2>(a, BT, hg, st) : launch_attn_t<false, 2>(a, BT, hg, st);
 }
 
 }  // namespace csa2
