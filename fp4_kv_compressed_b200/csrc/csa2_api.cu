@@ -35,9 +35,12 @@ bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 // Workspace layout of csa2_index_full: scores [BT][score_stride] fp32, then block
 // maxima of 8 positions [BT][bmax_stride] (hierarchical rows, and flat rows longer than
-// kFlatDirect), then maxima of 64 positions [BT][bmax64_stride] (rows longer than
-// kFlatDirect).  The selection of a long row goes through the block maxima.
+// kFlatDirect), then maxima of 64 positions [BT][bmax64_stride] (flat rows longer than
+// kFlatDirect; hierarchical rows of more than kPoolDirect blocks).  The selection of a
+// long row goes through the block maxima; the select stages up to kPoolDirect block
+// maxima directly.
 constexpr int64_t kFlatDirect = 16384;
+constexpr int64_t kPoolDirect = 16384;
 
 struct FullLayout {
     int64_t score_stride, bmax_stride, bmax64_stride;
@@ -51,7 +54,7 @@ FullLayout full_layout(int64_t BT, int64_t n_max, int32_t pool_blocks) {
     L.bmax_stride = (int64_t)align_up((size_t)((n_max + 7) / 8 > 0 ? (n_max + 7) / 8 : 1), 64);
     L.bmax64_stride = (int64_t)align_up((size_t)((n_max + 63) / 64 > 0 ? (n_max + 63) / 64 : 1), 64);
     L.bmax = pool_blocks > 0 || n_max > kFlatDirect;
-    L.bmax64 = n_max > kFlatDirect;
+    L.bmax64 = pool_blocks > 0 ? (n_max + 7) / 8 > kPoolDirect : n_max > kFlatDirect;
     L.bmax_off = align_up((size_t)BT * L.score_stride * sizeof(float), kAlign);
     L.bmax64_off = L.bmax_off + (L.bmax ? align_up((size_t)BT * L.bmax_stride * sizeof(float), kAlign) : 0);
     L.total = L.bmax64_off + (L.bmax64 ? align_up((size_t)BT * L.bmax64_stride * sizeof(float), kAlign) : 0);

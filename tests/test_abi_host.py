@@ -37,9 +37,13 @@ def test_workspace_sizes(pkg):
     ws = pkg.csa2_workspace_size
     full = ws(pkg.CSA2_OP_INDEX_FULL, 64, 1, 131072, 64, 512, 2048)
     assert full >= 64 * 131072 * 4 + 64 * 16384 * 4 and full % 256 == 0
-    # long rows (flat or hierarchical) also hold the 8- and 64-position maxima
+    # long flat rows also hold the 8- and 64-position maxima; hierarchical rows hold the
+    # 64-position maxima only beyond 16384 blocks
     flat = ws(pkg.CSA2_OP_INDEX_FULL, 64, 1, 131072, 64, 512, 0)
-    assert flat >= 64 * 131072 * 4 + 64 * 16384 * 4 + 64 * 2048 * 4 and flat == full
+    assert flat >= 64 * 131072 * 4 + 64 * 16384 * 4 + 64 * 2048 * 4 and flat > full
+    assert full == 64 * 131072 * 4 + 64 * 16384 * 4
+    big = ws(pkg.CSA2_OP_INDEX_FULL, 4, 1, 1 << 20, 64, 512, 2048)
+    assert big == 4 * (1 << 20) * 4 + 4 * (1 << 17) * 4 + 4 * (1 << 14) * 4
     short = ws(pkg.CSA2_OP_INDEX_FULL, 64, 1, 16384, 64, 512, 0)
     assert 64 * 16384 * 4 <= short < ws(pkg.CSA2_OP_INDEX_FULL, 64, 1, 16384, 64, 512, 2048)
     assert ws(pkg.CSA2_OP_INDEX_REINDEX, 64, 1, 0, 64, 512, 2048) >= 64 * 2048 * (8 + 1) * 4
