@@ -547,6 +547,10 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device error bits {st.dev_err.item()} in the timed steps")
 
     # ---- e2e: inputs from pinned host memory, last layer's output back to the host ----
+    # Every step copies its inputs host -> device and its result device -> host.  The
+    # inputs are double-buffered: while step k computes on one device buffer, a copy
+    # stream fills the other with step k + 1's inputs (the way a serving loop overlaps
+    # its transfers), so the step costs max(copy, compute) rather than their sum.
     last = len(st.plan) - 1
     out_h = torch.empty_like(st.out[last], device="cpu").pin_memory()
     lse_h = torch.empty_like(st.lse[last], device="cpu").pin_memory()
@@ -554,26 +558,42 @@ def run_ours(args, rank, world, local_rank):
     Ke = 0 if args.no_e2e else max(3, min(K, args.e2e_steps))
     e2e_ms = None
     if Ke:
+        inputs_b, dbuf_b, _, _ = pack_inputs(dw.inputs, dev)
+        g1b = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1b, stream=stream):
+            st.step(**inputs_b)
+        bufs, graphs = (dbuf, dbuf_b), (g1, g1b)
+        copy_stream = torch.cuda.Stream(device=dev)
+        copied = [torch.cuda.Event(), torch.cuda.Event()]
+        free = [torch.cuda.Event(), torch.cuda.Event()]
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
 
-        def e2e_step():
-            dbuf.copy_(hbuf, non_blocking=True)          # this step's inputs, host -> device
-            g1.replay()
-            out_h.copy_(st.out[last], non_blocking=True)  # the step's result, device -> host
-            lse_h.copy_(st.lse[last], non_blocking=True)
-        with torch.cuda.stream(stream):
-            for _ in range(2):
-                e2e_step()
+        def run(n, timed):
+            for e in free:                                # both buffers free at the start
+                e.record(stream)
+            if timed:
+                e0.record(copy_stream)
+            for k in range(n):
+                j = k % 2
+                with torch.cuda.stream(copy_stream):      # step k's inputs, host -> device
+                    copy_stream.wait_event(free[j])
+                    bufs[j].copy_(hbuf, non_blocking=True)
+                    copied[j].record(copy_stream)
+                with torch.cuda.stream(stream):
+                    stream.wait_event(copied[j])
+                    graphs[j].replay()
+                    out_h.copy_(st.out[last], non_blocking=True)   # the step's result, device -> host
+                    lse_h.copy_(st.lse[last], non_blocking=True)
+                    free[j].record(stream)
+            if timed:
+                e1.record(stream)
+        run(2, False)
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
-        with torch.cuda.stream(stream):
-            e0.record()
-            for _ in range(Ke):
-                e2e_step()
-            e1.record()
+        run(Ke, True)
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
