@@ -884,10 +884,7 @@ attn_kernel(AttnArgs a) {
             st_peer(peer_addr(&s.pl[rank][h], (uint32_t)r2), s.cl[h]);
         }
     }
-    // Two CTAs with a full head group exchange their partials through L2 (the output
-    // rows themselves, see below); otherwise through shared memory.
-    const bool via_l2 = CS == 2 && hcta == kHeads;
-    if (threadIdx.x == 0 && !via_l2) {     // armed before any peer can send
+    if (threadIdx.x == 0) {                // armed before any peer can send
         mbar_expect_tx(&s.xfer[0], (CS - 1) * kPiece);
         mbar_expect_tx(&s.xfer[1], (CS - 1) * kPiece);
     }
@@ -913,174 +910,98 @@ attn_kernel(AttnArgs a) {
             a.lse[(int64_t)qi * a.H + h0 + h] = valid ? (m_all + log2f(l_all)) * 0.6931471805599453f : -INFINITY;
     }
     __syncthreads();
+    // Send slot j (0 .. CS - 2) holds the part for peer (rank + 1 + j) % CS; it lands in
+    // that peer's receive slot CS - 2 - j (so receive slot i holds what CTA
+    // (peer + 1 + i) % CS sent).  A slot is [2 head halves][NB blocks][128 channels][32
+    // heads] fp32, float4 units swizzled by channel; receive slots fill s.kv from the
+    // start, send slots follow them in s.kv and then s.q (both free by now).
+    // Task u (warp u % 12 takes u, so the TMEM lane quadrant u % 4 is the warp's):
+    // channels 32 (u % 4) .., head half (u >> 2) & 1, block bsel / send slot from u >> 3.
     const bool have = __shfl_sync(0xFFFFFFFFu, (int)(nt > 0 && !aborted(s)), 0) != 0;
-    if (via_l2) {
-        // The peer's 256 output channels of this query's 64 head rows are the scratch for
-        // this CTA's partial of them: task u (16; warp u % 12, TMEM lane quadrant u % 4)
-        // stores channel 32 (u % 4) + lane of block 2 peer + bsel, heads 32 hp .., as 128
-        // contiguous bytes at float (bsel 128 + channel) 64 + 32 hp of the half.  After
-        // the cluster barrier (release / acquire) the owner reads its half back from L2,
-        // adds its own partial and overwrites it with the final rows, once every thread
-        // of the CTA has read its share.
-        float *oq = a.out + ((int64_t)qi * a.H + h0) * kDim;
-        auto scratch = [&](float *half, int bsel, int crow, int hp) {
-            const int f = (bsel * kTK + crow) * kHeads + 32 * hp;
-            return half + (f >> 8) * kDim + (f & 255);
-        };
-        const uint32_t peer = rank ^ 1u;
+    auto recv_slot = [&](int i) { return reinterpret_cast<float *>(&s.kv[0][0]) + i * 2 * kPieceF; };
+    auto send_slot = [&](int j) {
+        const int k = (CS - 1) + j;        // slot index in the sequence s.kv, then s.q
+        return k * 2 * kPieceF < (int)(sizeof(s.kv) / 4)
+                   ? reinterpret_cast<float *>(&s.kv[0][0]) + k * 2 * kPieceF
+                   : reinterpret_cast<float *>(s.q) + (k * 2 * kPieceF - (int)(sizeof(s.kv) / 4));
+    };
 #pragma unroll 1
-        for (int u = warp; u < 16; u += kWarps) {
-            const int cq = u & 3, hp = (u >> 2) & 1, bsel = u >> 3;
-            const int crow = 32 * cq + lane;
-            float o[32];
-            if (have) {
-                tmem_ld32(tmem + ((uint32_t)(32 * cq) << 16) + 64u * (uint32_t)(2 * (int)peer + bsel) + 32u * (uint32_t)hp, o);
-            } else {
+    for (int u = warp; u < 8 * NB * (CS - 1); u += kWarps) {
+        const int cq = u & 3, hp = (u >> 2) & 1, bsel = (u >> 3) % NB, j = (u >> 3) / NB;
+        const int pr = ((int)rank + 1 + j) % CS;
+        const int crow = 32 * cq + lane;             // channel within a block
+        const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)hp;
+        float o[32];
+        if (have) {
+            tmem_ld32(taddr + 64u * (uint32_t)(NB * pr + bsel), o);
+        } else {
 #pragma unroll
-                for (int h = 0; h < 32; ++h) o[h] = 0.0f;
-            }
-            float4 *dst = reinterpret_cast<float4 *>(scratch(oq + 256 * peer, bsel, crow, hp));
-#pragma unroll
-            for (int f = 0; f < 8; ++f) {
-                const int h = 32 * hp + 4 * f;
-                dst[f] = make_float4(o[4 * f] * s.wself[h], o[4 * f + 1] * s.wself[h + 1],
-                                     o[4 * f + 2] * s.wself[h + 2], o[4 * f + 3] * s.wself[h + 3]);
-            }
+            for (int h = 0; h < 32; ++h) o[h] = 0.0f;
         }
-        tc_fence_before();
-        cluster_sync();                    // each half holds the other CTA's partial
-        tc_fence_after();
-        // own tasks: u = warp (and warp + 12 for warps 0..3)
-        float part[2][32];
+        float4 *dst = reinterpret_cast<float4 *>(send_slot(j) + hp * kPieceF + (bsel * kTK + crow) * (kHeads / 2));
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const int u = warp + kWarps * t;
-            if (u < 16) {
-                const int cq = u & 3, hp = (u >> 2) & 1, bsel = u >> 3;
-                const float4 *src = reinterpret_cast<const float4 *>(scratch(oq + 256 * rank, bsel, 32 * cq + lane, hp));
-#pragma unroll
-                for (int f = 0; f < 8; ++f) {
-                    const float4 v = __ldcg(src + f);
-                    part[t][4 * f] = v.x; part[t][4 * f + 1] = v.y; part[t][4 * f + 2] = v.z; part[t][4 * f + 3] = v.w;
-                }
-            }
+        for (int f = 0; f < 8; ++f) {                // float4 f = heads 32 hp + 4 f ..
+            const int h = 32 * hp + 4 * f;
+            dst[f ^ (crow & 7)] = make_float4(o[4 * f] * s.wself[h], o[4 * f + 1] * s.wself[h + 1],
+                                              o[4 * f + 2] * s.wself[h + 2], o[4 * f + 3] * s.wself[h + 3]);
         }
-        __syncthreads();                   // every thread's share of the scratch is read
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const int u = warp + kWarps * t;
-            if (u < 16) {
-                const int cq = u & 3, hp = (u >> 2) & 1, bsel = u >> 3;
-                const int crow = 32 * cq + lane;
-                float own[32];
-                if (have) {
-                    tmem_ld32(tmem + ((uint32_t)(32 * cq) << 16) + 64u * (uint32_t)(2 * (int)rank + bsel) + 32u * (uint32_t)hp, own);
-                } else {
-#pragma unroll
-                    for (int h = 0; h < 32; ++h) own[h] = 0.0f;
-                }
-                float *obase = oq + 128 * (2 * (int)rank + bsel) + crow;
-#pragma unroll
-                for (int k = 0; k < 32; ++k)
-                    obase[(int64_t)(32 * hp + k) * kDim] = own[k] * s.wself[32 * hp + k] + part[t][k];
-            }
-        }
-        tc_fence_before();
-        __syncthreads();                   // every TMEM load of the CTA has completed
-        tc_fence_after();
-    } else {
-        // Send slot j (0 .. CS - 2) holds the part for peer (rank + 1 + j) % CS; it lands in
-        // that peer's receive slot CS - 2 - j (so receive slot i holds what CTA
-        // (peer + 1 + i) % CS sent).  A slot is [2 head halves][NB blocks][128 channels][32
-        // heads] fp32, float4 units swizzled by channel; receive slots fill s.kv from the
-        // start, send slots follow them in s.kv and then s.q (both free by now).
-        // Task u (warp u % 12 takes u, so the TMEM lane quadrant u % 4 is the warp's):
-        // channels 32 (u % 4) .., head half (u >> 2) & 1, block bsel / send slot from u >> 3.
-        auto recv_slot = [&](int i) { return reinterpret_cast<float *>(&s.kv[0][0]) + i * 2 * kPieceF; };
-        auto send_slot = [&](int j) {
-            const int k = (CS - 1) + j;        // slot index in the sequence s.kv, then s.q
-            return k * 2 * kPieceF < (int)(sizeof(s.kv) / 4)
-                       ? reinterpret_cast<float *>(&s.kv[0][0]) + k * 2 * kPieceF
-                       : reinterpret_cast<float *>(s.q) + (k * 2 * kPieceF - (int)(sizeof(s.kv) / 4));
-        };
-    #pragma unroll 1
-        for (int u = warp; u < 8 * NB * (CS - 1); u += kWarps) {
-            const int cq = u & 3, hp = (u >> 2) & 1, bsel = (u >> 3) % NB, j = (u >> 3) / NB;
-            const int pr = ((int)rank + 1 + j) % CS;
-            const int crow = 32 * cq + lane;             // channel within a block
-            const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)hp;
-            float o[32];
-            if (have) {
-                tmem_ld32(taddr + 64u * (uint32_t)(NB * pr + bsel), o);
-            } else {
-    #pragma unroll
-                for (int h = 0; h < 32; ++h) o[h] = 0.0f;
-            }
-            float4 *dst = reinterpret_cast<float4 *>(send_slot(j) + hp * kPieceF + (bsel * kTK + crow) * (kHeads / 2));
-    #pragma unroll
-            for (int f = 0; f < 8; ++f) {                // float4 f = heads 32 hp + 4 f ..
-                const int h = 32 * hp + 4 * f;
-                dst[f ^ (crow & 7)] = make_float4(o[4 * f] * s.wself[h], o[4 * f + 1] * s.wself[h + 1],
-                                                  o[4 * f + 2] * s.wself[h + 2], o[4 * f + 3] * s.wself[h + 3]);
-            }
-        }
-        fence_async_smem();                    // generic-proxy writes of `send` -> the bulk copy
-        __syncthreads();
-        if (threadIdx.x < 2 * (CS - 1)) {      // one copy per (peer, head half)
-            const int j = threadIdx.x >> 1, hp = threadIdx.x & 1;
-            const uint32_t pr = (uint32_t)(((int)rank + 1 + j) % CS);
-            const uint32_t dst = peer_addr(recv_slot(CS - 2 - j) + hp * kPieceF, pr);
-            bulk_copy_to_peer(dst, send_slot(j) + hp * kPieceF, kPiece, peer_addr(&s.xfer[hp], pr));
-        }
-        bool got_all = true;
-    #pragma unroll 1
-        for (int u = warp; u < 8 * NB; u += kWarps) {
-            const int cq = u & 3, hp = (u >> 2) & 1, bsel = u >> 3;
-            const int crow = 32 * cq + lane;
-            const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)hp;
-            float own[32];
-            if (have) {
-                tmem_ld32(taddr + 64u * (uint32_t)(NB * (int)rank + bsel), own);
-            } else {
-    #pragma unroll
-                for (int h = 0; h < 32; ++h) own[h] = 0.0f;
-            }
-            const bool got = __all_sync(0xFFFFFFFFu, mbar_wait<false>(&s.xfer[hp], 0, kDrainLimitNs, s));
-            got_all = got_all && got;
-    #pragma unroll
-            for (int f = 0; f < 8; ++f) {
-                const int h = 32 * hp + 4 * f;
-    #pragma unroll
-                for (int k = 0; k < 4; ++k) own[4 * f + k] *= s.wself[h + k];
-            }
-    #pragma unroll 1
-            for (int i = 0; i < CS - 1; ++i) {           // the senders in a fixed order
-                const float4 *src = reinterpret_cast<const float4 *>(recv_slot(i) + hp * kPieceF +
-                                                                     (bsel * kTK + crow) * (kHeads / 2));
-    #pragma unroll
-                for (int f = 0; f < 8; ++f) {
-                    const float4 pr = got ? src[f ^ (crow & 7)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                    own[4 * f] += pr.x; own[4 * f + 1] += pr.y; own[4 * f + 2] += pr.z; own[4 * f + 3] += pr.w;
-                }
-            }
-            float *obase = a.out + ((int64_t)qi * a.H + h0) * kDim + 128 * (NB * (int)rank + bsel) + crow;
-    #pragma unroll
-            for (int k = 0; k < 32; ++k)
-                if (32 * hp + k < hcta) obase[(int64_t)(32 * hp + k) * kDim] = own[k];
-        }
-        if (!got_all && lane == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
-        // A warp with no task for a head half still waits for it, so that every incoming
-        // copy has landed before the closing barrier.
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait<false>(&s.xfer[0], 0, kDrainLimitNs, s) &&
-                                         mbar_wait<false>(&s.xfer[1], 0, kDrainLimitNs, s)) &&
-            lane == 0)
-            set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
-        // Every CTA has seen its incoming copies land, so every outgoing copy has finished
-        // reading its send slot: only now may a CTA leave (and its shared memory be reused).
-        tc_fence_before();
-        cluster_sync();
-        tc_fence_after();
     }
+    fence_async_smem();                    // generic-proxy writes of `send` -> the bulk copy
+    __syncthreads();
+    if (threadIdx.x < 2 * (CS - 1)) {      // one copy per (peer, head half)
+        const int j = threadIdx.x >> 1, hp = threadIdx.x & 1;
+        const uint32_t pr = (uint32_t)(((int)rank + 1 + j) % CS);
+        const uint32_t dst = peer_addr(recv_slot(CS - 2 - j) + hp * kPieceF, pr);
+        bulk_copy_to_peer(dst, send_slot(j) + hp * kPieceF, kPiece, peer_addr(&s.xfer[hp], pr));
+    }
+    bool got_all = true;
+#pragma unroll 1
+    for (int u = warp; u < 8 * NB; u += kWarps) {
+        const int cq = u & 3, hp = (u >> 2) & 1, bsel = u >> 3;
+        const int crow = 32 * cq + lane;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * cq) << 16) + 32u * (uint32_t)hp;
+        float own[32];
+        if (have) {
+            tmem_ld32(taddr + 64u * (uint32_t)(NB * (int)rank + bsel), own);
+        } else {
+#pragma unroll
+            for (int h = 0; h < 32; ++h) own[h] = 0.0f;
+        }
+        const bool got = __all_sync(0xFFFFFFFFu, mbar_wait<false>(&s.xfer[hp], 0, kDrainLimitNs, s));
+        got_all = got_all && got;
+#pragma unroll
+        for (int f = 0; f < 8; ++f) {
+            const int h = 32 * hp + 4 * f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) own[4 * f + k] *= s.wself[h + k];
+        }
+#pragma unroll 1
+        for (int i = 0; i < CS - 1; ++i) {           // the senders in a fixed order
+            const float4 *src = reinterpret_cast<const float4 *>(recv_slot(i) + hp * kPieceF +
+                                                                 (bsel * kTK + crow) * (kHeads / 2));
+#pragma unroll
+            for (int f = 0; f < 8; ++f) {
+                const float4 pr = got ? src[f ^ (crow & 7)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                own[4 * f] += pr.x; own[4 * f + 1] += pr.y; own[4 * f + 2] += pr.z; own[4 * f + 3] += pr.w;
+            }
+        }
+        float *obase = a.out + ((int64_t)qi * a.H + h0) * kDim + 128 * (NB * (int)rank + bsel) + crow;
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+            if (32 * hp + k < hcta) obase[(int64_t)(32 * hp + k) * kDim] = own[k];
+    }
+    if (!got_all && lane == 0) set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+    // A warp with no task for a head half still waits for it, so that every incoming
+    // copy has landed before the closing barrier.
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait<false>(&s.xfer[0], 0, kDrainLimitNs, s) &&
+                                     mbar_wait<false>(&s.xfer[1], 0, kDrainLimitNs, s)) &&
+        lane == 0)
+        set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+    // Every CTA has seen its incoming copies land, so every outgoing copy has finished
+    // reading its send slot: only now may a CTA leave (and its shared memory be reused).
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
