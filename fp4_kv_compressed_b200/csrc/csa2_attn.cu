@@ -15,40 +15,49 @@
 // the four 128-channel output blocks from its own partial and the others' (bulk
 // copies between the CTAs' shared memories).
 //
-// Transposed tiles.  A tile is 128 keys.  The scores are S^T = K Q^T with the keys
-// as the MMA's M = 128 (one TMEM lane per key) and the 64 heads as N, so the score
-// MMAs run at the full M = 128 shape; the output is O^T = V^T P^T with the channels
-// as M (four 128-channel blocks) and the heads as N.  One fp16 tile in shared memory
-// serves both: four stages of 128 channels x 128 keys, each the K-major A operand of
-// S^T (rows = keys) and the MN-major A operand of O^T (M = channels contiguous in a
-// row).  fp16 holds the FP4 values exactly (e2m1 x e4m3 has at most 6 significant
-// bits); an SWA row is stored as its exact E4M3 codes and its scale sigma is applied
-// in fp32, to the logit and folded into P.  Q (the K-major B operand of S^T) is
-// converted to fp16 after an exact power-of-two scaling that keeps max|q| below 2^15.
+// Transposed tiles.  A tile is 64 keys.  The scores are S^T = K Q^T with the keys as
+// the MMA's M = 64 (TMEM lanes 32 q .. 32 q + 15 hold keys 16 q .. 16 q + 15) and the
+// 64 heads as N; the output is O^T = V^T P^T with the channels as M (four 128-channel
+// blocks, M = 128) and the heads as N.  One fp16 tile in shared memory serves both:
+// four stages of 128 channels x 64 keys, each the K-major A operand of S^T (rows =
+// keys) and the MN-major A operand of O^T (M = channels contiguous in a row).  fp16
+// holds the FP4 values exactly (e2m1 x e4m3 has at most 6 significant bits); an SWA
+// row is stored as its exact E4M3 codes and its scale sigma is applied in fp32, to the
+// logit and folded into P.  Q (the K-major B operand of S^T) is converted to fp16
+// after an exact power-of-two scaling that keeps max|q| below 2^15.
+//
+// Two tiles in flight.  The worker warps form two sets of four; set s owns the tiles
+// h with h % 2 == s and its own tile buffer, S^T accumulator and P^T buffer.  The MMA
+// warp issues S^T(h) and then O^T(h - 1), so the score MMAs of one set's tile run
+// while the other set takes the softmax of its own, and the output MMAs of a tile run
+// while the next tile is being written.  The running max is handed from tile to tile
+// (an mbarrier per set); each thread keeps its row-sum partial against the max it last
+// saw, so neither set ever rescales the other's sums.
 //
 // 12 warps, specialised:
 //   warp 0       TMEM allocation + the MMA issue loop (one elected lane issues);
 //   warp 1       fused append only: quantises the query token's new SWA row;
 //   warp 2       prefetches the entries of this CTA's later tiles into L2 (bulk prefetch;
 //                the set-up prefetches the request's SWA ring);
-//   warps 4-11   workers, two roles in turn.  Producer: warp wi = w - 4 gathers keys
-//                16 wi .. 16 wi + 15 of the next tile warp-cooperatively (one load
-//                instruction = one 64-byte stage slice of 8 keys), all four stages in
-//                registers before the softmax of this tile, and dequantises stage j as
-//                soon as O^T of this tile has read it.  Softmax: warp w reads TMEM lane
-//                quadrant w % 4 (32 keys) and the 32 heads of half (w - 4) / 4.
+//   warps 4-11   workers: set (w - 4) / 4, TMEM lane quadrant w % 4.  Producer: the warp
+//                gathers keys 16 (w % 4) .. + 15 of its set's next tile warp-cooperatively
+//                (one load instruction = one 64-byte stage slice of 8 keys), all four
+//                stages in registers before the softmax of the set's current tile, and
+//                dequantises stage j as soon as O^T of the set's previous tile has read
+//                it.  Softmax: the warp reads its 16 keys x 64 heads with one
+//                tcgen05.ld.16x256b.x8 (a thread: 2 keys x 16 heads).
 // TMEM (512 columns): O^T block j (channels 128 j .. 128 j + 127) at columns
-// 64 j .. 64 j + 63 (column = head); the two S^T buffers at columns 256 and 320.
+// 64 j .. 64 j + 63 (column = head); the two sets' S^T at columns 256 and 320.
 // Online softmax in the log2 domain with lazy rescaling: the running max of a head
-// moves (and O, l are rescaled) only when a tile's logit exceeds it by more than 8,
-// so p <= 2^8 stays safe in fp16.  The check is per tile and per head half; the exact
-// tile max (a shuffle reduce-scatter within a warp, then across the four warps that
-// share the heads) is formed only when it fires, and always on the first tile.
+// moves (and O is rescaled) only when a tile's logit exceeds it by more than 8, so
+// p <= 2^8 stays safe in fp16.  The check is per tile; the exact tile max (a shuffle
+// reduce-scatter within a warp, then across the set's four warps) is formed only when
+// it fires, and always on the first tile.
 // Every wait is bounded (WaitCfg): on timeout the kernel flags CSA2_DEVERR_TIMEOUT,
 // waits (bounded) for the MMAs it issued, still takes part in both cluster barriers
-// of the combine, frees TMEM and returns.  The four softmax warps of a head half
-// agree on leaving the tile loop through a barrier reduction, so that no named
-// barrier is ever left waiting for a warp that has gone.
+// of the combine, frees TMEM and returns.  The four warps of a set agree on leaving
+// the tile loop through a barrier reduction, so that no named barrier is ever left
+// waiting for a warp that has gone.
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -61,34 +70,38 @@ namespace attn {
 constexpr int kThreads = 384;
 constexpr int kWarps = kThreads / 32;
 constexpr int kQChunks = (64 * 64 + kThreads - 1) / kThreads;   // 16-byte Q chunks per thread
-constexpr int kTK = 128;                       // keys per tile (S^T M, TMEM lanes)
+constexpr int kTK = 64;                        // keys per tile (S^T M)
+constexpr int kSets = 2;                       // worker sets = tiles in flight
+constexpr int kCh = 128;                       // channels per O^T block (its M, TMEM lanes)
 constexpr int kHeads = 64;                     // heads per CTA (MMA N)
 constexpr int kStages = 4;                     // 128-channel quarters of a tile
-constexpr int kStageBytes = kTK * 128 * 2;     // 128 keys x 128 channels fp16
+constexpr int kStageBytes = kTK * 128 * 2;     // 64 keys x 128 channels fp16
 constexpr int kCbBytes = kTK * 128;            // one 64-channel block of a stage
 constexpr int kQCbBytes = kHeads * 128;        // one 64-channel block of Q
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSCol = 256;                // S^T buffer b at columns 256 + 64 b
+constexpr uint32_t kSCol = 256;                // S^T of set s at columns 256 + 64 s
 constexpr int kWorkWarp0 = 4;                  // softmax + producer warps 4..11
-constexpr int kWorkWarps = kWarps - kWorkWarp0;
+constexpr int kSetWarps = 4;                   // warps per set (one per TMEM lane quadrant)
 constexpr float kLazy = 8.0f;                  // rescale threshold (log2 units)
 constexpr int kMaxCS = 4;                      // CTAs per query (cluster size): 2 or 4
 
 struct __align__(1024) Smem {
     uint8_t q[8 * kQCbBytes];                  // Q fp16, [8 cb][64 heads][128 B] swizzled
-    uint8_t kv[kStages][kStageBytes];          // stage j: [2 cb][128 keys][128 B] swizzled
-    uint8_t pt[kTK * 128];                     // P^T fp16, [128 keys][64 heads] swizzled
+    uint8_t kv[kSets][kStages][kStageBytes];   // set s, stage j: [2 cb][64 keys][128 B] swizzled
+    uint8_t pt[kSets][kTK * 128];              // P^T fp16 of set s, [64 keys][64 heads] swizzled
     int32_t ids[CSA2_TOPK_MAX];                // compacted selected entry ids
-    float ksig[kTK];                           // per key of the tile: 1 FP4, sigma SWA, -1 none
+    float ksig[kSets][kTK];                    // per key of the tile: 1 FP4, sigma SWA, -1 none
     alignas(16) uint8_t swa_new[kDim];         // fused append: the new SWA row (E4M3 codes)
     float swa_new_sigma;
-    alignas(16) float red[2][4][32];           // softmax half hh: per quadrant warp, 32 heads
+    alignas(16) float red[kSets][kSetWarps][kHeads];    // per set and warp: tile max / row sums
+    alignas(16) float mref[kSets][kSetWarps][kHeads];   // the max the row sums are taken against
     alignas(16) float mrun[kHeads];            // running max per head (log2 domain)
-    alignas(16) float alpha[kHeads];           // factor of the last move of the running max
+    alignas(16) float alpha[kSets][kHeads];    // factor of the last move of the running max
     float cm[kHeads], cl[kHeads];              // this CTA's partial max / sum per head
     float pm[kMaxCS][kHeads], pl[kMaxCS][kHeads];   // every CTA's partial max / sum, by rank
     float wself[kHeads];                       // combine: weight of this CTA's partial
-    uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], p_full, pv_done, drain, never;
+    uint64_t kv_full[kSets][kStages], kv_empty[kSets][kStages];
+    uint64_t s_full[kSets], p_full[kSets], pv_done[kSets], m_ready[kSets], drain, never;
     uint64_t new_ready;                        // fused append: the new SWA row is in smem
     uint64_t xfer[2];                          // combine: the peers' parts of head half h have landed
     uint32_t tmem_base;
@@ -96,6 +109,8 @@ struct __align__(1024) Smem {
     float wred[kWarps];
     int32_t wcnt[2 * kWarps];
 };
+
+static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "one CTA per SM: at most 227 KB of shared memory");
 
 // ---- small PTX wrappers ---------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -196,6 +211,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+// 16 lanes x 64 columns (16x256b, 8 repeats): thread t reads lanes base + t / 4 and
+// base + t / 4 + 8, columns 8 r + 2 (t % 4) and + 1 of repeat r, as
+// v[4 r] v[4 r + 1] (first lane) and v[4 r + 2] v[4 r + 3] (second lane).
+__device__ __forceinline__ void tmem_ld16x64(uint32_t taddr, float *v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
 // 32 lanes x 16 columns, in place: v *= f (per column), read and written back.
 __device__ __forceinline__ void tmem_scale16(uint32_t taddr, const float *f) {
     uint32_t r[16];
@@ -224,13 +259,13 @@ __device__ __forceinline__ float ex2(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-// Named barrier of the four softmax warps that share head half hh (ids 1, 2).
-__device__ __forceinline__ void group_sync(int hh) {
-    asm volatile("bar.sync %0, 128;" ::"r"(1 + hh) : "memory");
+// Named barrier of the four warps of worker set `set` (ids 1, 2).
+__device__ __forceinline__ void group_sync(int set) {
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + set) : "memory");
 }
 // The same barrier with an OR over the four warps' predicates: every thread of the
-// group receives the same answer.
-__device__ __forceinline__ bool group_any(int hh, bool pred) {
+// set receives the same answer.
+__device__ __forceinline__ bool group_any(int set, bool pred) {
     uint32_t r;
     asm volatile(
         "{\n.reg .pred p, q;\n"
@@ -238,7 +273,7 @@ __device__ __forceinline__ bool group_any(int hh, bool pred) {
         "bar.red.or.pred q, %2, 128, p;\n"
         "selp.u32 %0, 1, 0, q;\n}"
         : "=r"(r)
-        : "r"((uint32_t)pred), "r"(1 + hh)
+        : "r"((uint32_t)pred), "r"(1 + set)
         : "memory");
     return r != 0;
 }
@@ -424,29 +459,37 @@ __device__ __forceinline__ void store_piece(const Raw &r, int g, int j, uint8_t 
     }
 }
 
-// Max (kMax) or sum over the warp's 32 lanes of each of 32 values; lane l ends with
-// the reduction of value l (a butterfly reduce-scatter: 31 shuffles).
+// Max (kMax) or sum over the 16 keys of a softmax warp, per head.  A thread holds
+// x[4 r + e] (its first key) and x[4 r + 2 + e] (its second key) of head 8 r + 2 (lane
+// % 4) + e; value i = 2 r + e is the reduction of that head over the thread's two keys,
+// then over the eight lanes that share lane % 4.  The lane ends with values 2 (lane / 4)
+// and 2 (lane / 4) + 1 (a butterfly reduce-scatter over lane bits 4, 3, 2: 14 shuffles).
 template <bool kMax>
-__device__ __forceinline__ float reduce_scatter32(const float *x, int lane) {
-    float a[16];
+__device__ __forceinline__ float2 reduce_keys16(const float *x, int lane) {
+    auto val = [&](int i) {
+        const float p = x[4 * (i >> 1) + (i & 1)], q = x[4 * (i >> 1) + 2 + (i & 1)];
+        return kMax ? fmaxf(p, q) : p + q;
+    };
+    float a[8];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
+    for (int k = 0; k < 8; ++k) {
         const bool hi = lane & 16;
-        const float mine = hi ? x[16 + k] : x[k], other = hi ? x[k] : x[16 + k];
+        const float lo_v = val(k), hi_v = val(8 + k);
+        const float mine = hi ? hi_v : lo_v, other = hi ? lo_v : hi_v;
         const float o = __shfl_xor_sync(0xFFFFFFFFu, other, 16);
         a[k] = kMax ? fmaxf(mine, o) : mine + o;
     }
 #pragma unroll
-    for (int st = 8; st >= 1; st >>= 1) {
+    for (int st = 4; st >= 2; st >>= 1) {
 #pragma unroll
         for (int k = 0; k < st; ++k) {
-            const bool hi = lane & st;
+            const bool hi = lane & (2 * st);
             const float mine = hi ? a[st + k] : a[k], other = hi ? a[k] : a[st + k];
-            const float o = __shfl_xor_sync(0xFFFFFFFFu, other, st);
+            const float o = __shfl_xor_sync(0xFFFFFFFFu, other, 2 * st);
             a[k] = kMax ? fmaxf(mine, o) : mine + o;
         }
     }
-    return a[0];
+    return make_float2(a[0], a[1]);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -467,14 +510,16 @@ attn_kernel(AttnArgs a) {
     const uint64_t lim = a.wait.limit_ns;
     // ---- set-up -----------------------------------------------------------------------------
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(&s.kv_full[i], kWorkWarps);
-            mbar_init(&s.kv_empty[i], 1);
+        for (int st = 0; st < kSets; ++st) {
+            for (int i = 0; i < kStages; ++i) {
+                mbar_init(&s.kv_full[st][i], kSetWarps);
+                mbar_init(&s.kv_empty[st][i], 1);
+            }
+            mbar_init(&s.s_full[st], 1);
+            mbar_init(&s.p_full[st], kSetWarps);
+            mbar_init(&s.pv_done[st], 1);
+            mbar_init(&s.m_ready[st], kSetWarps);
         }
-        mbar_init(&s.s_full[0], 1);
-        mbar_init(&s.s_full[1], 1);
-        mbar_init(&s.p_full, kWorkWarps);
-        mbar_init(&s.pv_done, 1);
         mbar_init(&s.drain, 1);
         mbar_init(&s.never, 1);
         mbar_init(&s.new_ready, 1);
@@ -590,7 +635,7 @@ attn_kernel(AttnArgs a) {
     const int n_keys = n_sel + n_win;
     const int chunk = ((n_keys + CS - 1) / CS + 15) / 16 * 16;
     const int k0 = min(n_keys, (int)rank * chunk), k1 = min(n_keys, k0 + chunk);
-    const int nt = (k1 - k0 + kTK - 1) / kTK;
+    const int nt = (k1 - k0 + kTK - 1) / kTK;   // tiles; tile h belongs to worker set h % 2
     const bool fuse = a.swa_new != nullptr && n_win > 0;
     const uint32_t owner = n_keys > 0 ? (uint32_t)((n_keys - 1) / chunk) : 0u;   // holds the newest key
     KeyMap km;
@@ -606,16 +651,15 @@ attn_kernel(AttnArgs a) {
     km.new_ready = &s.new_ready;
     km.smem = &s;
     const bool worker = warp >= kWorkWarp0;
-    const int qd = warp & 3, hh = (warp - kWorkWarp0) >> 2;   // worker: key quadrant, head / channel half
-    const int r = 32 * qd + lane;                              // worker softmax: key of the tile
-    const int wi = warp - kWorkWarp0;                          // worker producer: keys 16 wi ..
+    const int set = (warp - kWorkWarp0) >> 2;   // worker: set, its tiles h = set, set + 2, ..
+    const int qd = warp & 3;                     // worker: TMEM lane quadrant, keys 16 qd .. of a tile
     // rows of the tile's last 16-key group of valid keys are read by the output MMAs
     // and so written (zeros past the keys); rows after that group are not written
     auto zlim_of = [&](int i) { return ((min(kTK, k1 - k0 - i * kTK) + 15) / 16) * 16; };
     bool new_ok = false;
     Raw raw;
     __syncthreads();                       // s.ids complete
-    if (worker && nt > 0) load_keys(raw, a, km, k0, zlim_of(0), wi, lane);   // tile 0, in flight
+    if (worker && set < nt) load_keys(raw, a, km, k0 + set * kTK, zlim_of(set), qd, lane);   // in flight
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -624,52 +668,60 @@ attn_kernel(AttnArgs a) {
     const uint32_t tmem = s.tmem_base;
     if (warp == 0) {
         // ---------------- MMA issuer (whole warp runs the loop; one lane issues) ----------------
+        // Issue order S^T(0), S^T(1), O^T(0), S^T(2), O^T(1), ..: the scores of the next
+        // tile go ahead of the output of this one.
         if (nt > 0) {
             bool ok = true;
-            // S^T = K Q^T: A = stage (K-major, 128 keys), B = Q (K-major, 64 heads), M 128 N 64
+            // S^T = K Q^T: A = stage (K-major, 64 keys), B = Q (K-major, 64 heads), M 64 N 64
             const uint32_t idesc_s = (1u << 4) | ((uint32_t)(kHeads >> 3) << 17) | ((uint32_t)(kTK >> 4) << 24);
             // O^T = V^T P^T: A = stage (MN-major, 128 channels), B = P^T (MN-major, 64 heads)
             const uint32_t idesc_o = (1u << 4) | (1u << 15) | (1u << 16) | ((uint32_t)(kHeads >> 3) << 17) |
-                                     ((uint32_t)(kTK >> 4) << 24);
+                                     ((uint32_t)(kCh >> 4) << 24);
             const uint64_t qd_desc = sw128_desc(smem_u32(s.q), 16, 1024);
-            const uint64_t pd = sw128_desc(smem_u32(s.pt), 8192, 1024);
-            for (int i = 0; ok && i < nt; ++i) {
-                const uint32_t sd = tmem + kSCol + 64u * (uint32_t)(i & 1);
+            for (int h = 0; ok && h <= nt; ++h) {
+                if (h < nt) {
+                    const int bs = h & 1;
+                    const uint32_t sd = tmem + kSCol + 64u * (uint32_t)bs;
 #pragma unroll 1
-                for (int j = 0; j < kStages; ++j) {
-                    ok = __shfl_sync(0xFFFFFFFFu, (int)mbar_wait(&s.kv_full[j], i & 1, lim, s), 0) != 0;
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (elect_one()) {
-                        const uint64_t kd = sw128_desc(smem_u32(s.kv[j]), 16, 1024);
+                    for (int j = 0; j < kStages; ++j) {
+                        ok = __shfl_sync(0xFFFFFFFFu, (int)mbar_wait(&s.kv_full[bs][j], (h >> 1) & 1, lim, s), 0) != 0;
+                        if (!ok) break;
+                        tc_fence_after();
+                        if (elect_one()) {
+                            const uint64_t kd = sw128_desc(smem_u32(s.kv[bs][j]), 16, 1024);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {       // K-steps of 16 channels
-                            const uint64_t aoff = (uint64_t)((k >> 2) * (kCbBytes >> 4) + (k & 3) * 2);
-                            const uint64_t boff = (uint64_t)((2 * j + (k >> 2)) * (kQCbBytes >> 4) + (k & 3) * 2);
-                            mma_f16(sd, kd + aoff, qd_desc + boff, idesc_s, (j | k) != 0 ? 1u : 0u);
+                            for (int k = 0; k < 8; ++k) {       // K-steps of 16 channels
+                                const uint64_t aoff = (uint64_t)((k >> 2) * (kCbBytes >> 4) + (k & 3) * 2);
+                                const uint64_t boff = (uint64_t)((2 * j + (k >> 2)) * (kQCbBytes >> 4) + (k & 3) * 2);
+                                mma_f16(sd, kd + aoff, qd_desc + boff, idesc_s, (j | k) != 0 ? 1u : 0u);
+                            }
+                            if (j == kStages - 1) mma_commit(&s.s_full[bs]);
                         }
-                        if (j == kStages - 1) mma_commit(&s.s_full[i & 1]);
+                        __syncwarp();
                     }
-                    __syncwarp();
+                    if (!ok) break;
                 }
-                if (!ok) break;
-                // P^T(i) from the softmax (the test hook makes the first of these waits stuck)
-                const bool got = a.wait.stuck && i == 0 ? mbar_wait(&s.never, 0, lim, s)
-                                                        : mbar_wait(&s.p_full, i & 1, lim, s);
+                if (h == 0) continue;
+                // O^T(h - 1) once its P^T is written (the test hook makes the first of these
+                // waits stuck)
+                const int ho = h - 1, bo = ho & 1;
+                const bool got = a.wait.stuck && ho == 0 ? mbar_wait(&s.never, 0, lim, s)
+                                                         : mbar_wait(&s.p_full[bo], (ho >> 1) & 1, lim, s);
                 ok = __shfl_sync(0xFFFFFFFFu, (int)got, 0) != 0;
                 if (!ok) break;
                 tc_fence_after();
-                const int nk = (min(kTK, k1 - k0 - i * kTK) + 15) / 16;   // K-steps of valid keys
+                const int nk = (min(kTK, k1 - k0 - ho * kTK) + 15) / 16;   // K-steps of valid keys
                 if (elect_one()) {
+                    const uint64_t pd = sw128_desc(smem_u32(s.pt[bo]), 8192, 1024);
 #pragma unroll 1
                     for (int j = 0; j < kStages; ++j) {
-                        const uint64_t vd = sw128_desc(smem_u32(s.kv[j]), kCbBytes, 1024);
+                        const uint64_t vd = sw128_desc(smem_u32(s.kv[bo][j]), kCbBytes, 1024);
                         for (int kk = 0; kk < nk; ++kk)
                             mma_f16(tmem + 64u * (uint32_t)j, vd + (uint64_t)(kk * 128), pd + (uint64_t)(kk * 128),
-                                    idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-                        mma_commit(&s.kv_empty[j]);
+                                    idesc_o, (ho > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(&s.kv_empty[bo][j]);
                     }
-                    mma_commit(&s.pv_done);
+                    mma_commit(&s.pv_done[bo]);
                 }
                 __syncwarp();
             }
@@ -707,158 +759,196 @@ attn_kernel(AttnArgs a) {
             }
         }
     } else if (warp == 2) {
-        // L2 prefetch of the entries of this CTA's later tiles (tile 0 is already in flight)
-        for (int kg = k0 + kTK + lane; kg < min(k1, n_sel); kg += 32) {
+        // L2 prefetch of the entries of this CTA's later tiles (tiles 0 and 1 are in flight)
+        for (int kg = k0 + kSets * kTK + lane; kg < min(k1, n_sel); kg += 32) {
             const int64_t row = cache_row(a.pm, a.cap, b, s.ids[kg]);
             prefetch_l2(a.codes + row * kCodeBytes, kCodeBytes);
             prefetch_l2(a.scales + row * kScaleBytes, kScaleBytes);
         }
     } else if (worker) {
-        // ---------------- workers: produce tile i + 1 after the softmax of tile i ----------------
-        // Softmax: keys 32 qd .. (TMEM lanes), heads 32 hh .. .  Producer: keys 16 wi ..
-        // (prod_key); the raw bytes of the next tile are in registers while the softmax of
-        // this one runs.
+        // ---------------- workers: produce tile h, take its softmax, load tile h + 2 ----------------
+        // Softmax: thread (ii, cc) = (lane / 4, lane % 4) holds keys kA = 16 qd + ii and
+        // kA + 8 of the tile and heads 8 r + 2 cc + e (r < 8, e < 2): x[4 r + e] (kA) and
+        // x[4 r + 2 + e] (kA + 8).  Its row sums are for heads 8 ii + 2 cc + e.
         const float c0 = a.softmax_scale * 1.4426950408889634f * exp2f((float)qexp);
         const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
-        const float4 *mrun4 = reinterpret_cast<const float4 *>(&s.mrun[32 * hh]);
-        float lsum = 0.0f;   // head 32 hh + lane: partial sum over this warp's keys
+        const int ii = lane >> 2, cc = lane & 3;
+        const int kA = 16 * qd + ii;
+        // row sums of this warp's keys of this set's tiles, heads 8 ii + 2 cc + e, as sums of
+        // 2^(x - mref) with mref in the thread's own slot of s.mref
+        float lsum[2] = {0.0f, 0.0f};
+        float2 *mref = reinterpret_cast<float2 *>(&s.mref[set][qd][8 * ii + 2 * cc]);
+        *mref = make_float2(-INFINITY, -INFINITY);
         bool ok = true, stop = false;
-        for (int i = 0; i < nt; ++i) {
-            // ---- produce tile i (its stages are free once O^T(i - 1) has read them) ----
+        for (int h = set; h < nt; h += kSets) {
+            // ---- produce tile h (its stages are free once O^T(h - 2) has read them) ----
             if (ok) {
 #pragma unroll
                 for (int g = 0; g < kGroups; ++g)
                     if (raw.kind[g] == 3) take_new_row(raw, g, a, km, lane, new_ok);
 #pragma unroll
                 for (int j = 0; j < kStages; ++j) {   // unrolled: raw.c[.][j] stays in registers
-                    if (i > 0) {
-                        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.kv_empty[j], (i - 1) & 1, lim, s));
+                    if (h >= kSets) {
+                        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.kv_empty[set][j], ((h - kSets) >> 1) & 1, lim, s));
                         if (!ok) break;
                     }
 #pragma unroll
                     for (int g = 0; g < kGroups; ++g) {
-                        const int kt = prod_key(wi, g, lane);
-                        store_piece(raw, g, j, s.kv[j], kt, lane);
+                        const int kt = prod_key(qd, g, lane);
+                        store_piece(raw, g, j, s.kv[set][j], kt, lane);
                         if (j == 0 && prod_piece(lane) == 0) {
                             const float sg = raw.sigma[g];
-                            s.ksig[kt] = sg;
+                            s.ksig[set][kt] = sg;
                             // P carries sigma in fp16: p <= 2^8 needs sigma <= 65504 / 256
                             if (raw.kind[g] == 2 && sg * 256.0f > 65504.0f) set_dev_err(a.dev_err, CSA2_DEVERR_RANGE);
                         }
                     }
                     fence_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&s.kv_full[j]);
+                    if (lane == 0) mbar_arrive(&s.kv_full[set][j]);
                 }
-                if (ok && i + 1 < nt) load_keys(raw, a, km, k0 + (i + 1) * kTK, zlim_of(i + 1), wi, lane);
+                if (ok && h + kSets < nt) load_keys(raw, a, km, k0 + (h + kSets) * kTK, zlim_of(h + kSets), qd, lane);
             }
-            // ---- softmax of tile i: every wait first; the four warps of the half agree ----
-            // (kv_full[0] of tile i: every worker's s.ksig of the tile is written)
-            const bool w_ok = ok && __all_sync(0xFFFFFFFFu, mbar_wait(&s.s_full[i & 1], (i >> 1) & 1, lim, s) &&
-                                                                mbar_wait(&s.kv_full[0], i & 1, lim, s) &&
-                                                                (i == 0 || mbar_wait(&s.pv_done, (i - 1) & 1, lim, s)));
-            stop = group_any(hh, !w_ok || aborted(s));
+            // ---- softmax of tile h: every wait first; the four warps of the set agree ----
+            // (kv_full[set][0]: every warp's s.ksig of the tile is written; m_ready: the
+            // previous tile has fixed the running max)
+            const bool w_ok =
+                ok && __all_sync(0xFFFFFFFFu, mbar_wait(&s.s_full[set], (h >> 1) & 1, lim, s) &&
+                                                  mbar_wait(&s.kv_full[set][0], (h >> 1) & 1, lim, s) &&
+                                                  (h == 0 || mbar_wait(&s.m_ready[set ^ 1], ((h - 1) >> 1) & 1, lim, s)));
+            stop = group_any(set, !w_ok || aborted(s));
             if (stop) break;
             tc_fence_after();
             float x[32];
-            tmem_ld32(tmem + lane_base + kSCol + 64u * (uint32_t)(i & 1) + 32u * (uint32_t)hh, x);
-            const float sig = s.ksig[r];
-            const bool valid = sig >= 0.0f;
-            const float ck = c0 * sig;
-            float dmax = -INFINITY;
+            tmem_ld16x64(tmem + lane_base + kSCol + 64u * (uint32_t)set, x);
+            const float sgA = s.ksig[set][kA], sgB = s.ksig[set][kA + 8];
+            const bool vA = sgA >= 0.0f, vB = sgB >= 0.0f;
+            const float ckA = c0 * sgA, ckB = c0 * sgB;
 #pragma unroll
-            for (int h = 0; h < 32; ++h) x[h] = valid ? x[h] * ck : -INFINITY;   // logits, log2 units
-            if (i > 0) {
+            for (int r = 0; r < 8; ++r) {   // logits, log2 units
+                x[4 * r] = vA ? x[4 * r] * ckA : -INFINITY;
+                x[4 * r + 1] = vA ? x[4 * r + 1] * ckA : -INFINITY;
+                x[4 * r + 2] = vB ? x[4 * r + 2] * ckB : -INFINITY;
+                x[4 * r + 3] = vB ? x[4 * r + 3] * ckB : -INFINITY;
+            }
+            float dmax = -INFINITY;
+            if (h > 0) {
                 // x -> x - m in place: the lazy check, and (common case) the exponent of p
 #pragma unroll
-                for (int h4 = 0; h4 < 8; ++h4) {
-                    const float4 mv = mrun4[h4];
-                    x[4 * h4] -= mv.x; x[4 * h4 + 1] -= mv.y; x[4 * h4 + 2] -= mv.z; x[4 * h4 + 3] -= mv.w;
-                    dmax = fmaxf(dmax, fmaxf(fmaxf(x[4 * h4], x[4 * h4 + 1]), fmaxf(x[4 * h4 + 2], x[4 * h4 + 3])));
+                for (int r = 0; r < 8; ++r) {
+                    const float2 mv = *reinterpret_cast<const float2 *>(&s.mrun[8 * r + 2 * cc]);
+                    x[4 * r] -= mv.x; x[4 * r + 1] -= mv.y; x[4 * r + 2] -= mv.x; x[4 * r + 3] -= mv.y;
+                    dmax = fmaxf(dmax, fmaxf(fmaxf(x[4 * r], x[4 * r + 1]), fmaxf(x[4 * r + 2], x[4 * r + 3])));
                 }
             }
-            const bool upd = group_any(hh, i == 0 || dmax > kLazy);
+            const bool upd = group_any(set, h == 0 || dmax > kLazy);
             if (upd) {
-                if (i > 0) {   // back to the logits (one rounding; p's exponent stays consistent)
+                if (h > 0) {   // back to the logits (one rounding; p's exponent stays consistent)
 #pragma unroll
-                    for (int h4 = 0; h4 < 8; ++h4) {
-                        const float4 mv = mrun4[h4];
-                        x[4 * h4] += mv.x; x[4 * h4 + 1] += mv.y; x[4 * h4 + 2] += mv.z; x[4 * h4 + 3] += mv.w;
+                    for (int r = 0; r < 8; ++r) {
+                        const float2 mv = *reinterpret_cast<const float2 *>(&s.mrun[8 * r + 2 * cc]);
+                        x[4 * r] += mv.x; x[4 * r + 1] += mv.y; x[4 * r + 2] += mv.x; x[4 * r + 3] += mv.y;
                     }
                 }
                 // exact tile max per head, then the running max moves
-                const float wm = reduce_scatter32<true>(x, lane);   // head 32 hh + lane
-                s.red[hh][qd][lane] = wm;
-                group_sync(hh);
+                const float2 wm = reduce_keys16<true>(x, lane);   // heads 8 ii + 2 cc, + 1
+                *reinterpret_cast<float2 *>(&s.red[set][qd][8 * ii + 2 * cc]) = wm;
+                group_sync(set);
                 if (qd == 0) {
-                    const float tm = fmaxf(fmaxf(s.red[hh][0][lane], s.red[hh][1][lane]),
-                                           fmaxf(s.red[hh][2][lane], s.red[hh][3][lane]));
-                    const float old = i > 0 ? s.mrun[32 * hh + lane] : -INFINITY;
-                    const float mn = fmaxf(old, tm);
-                    s.mrun[32 * hh + lane] = mn;
-                    s.alpha[32 * hh + lane] = old == -INFINITY ? 0.0f : ex2(old - mn);
-                }
-                group_sync(hh);
-                lsum *= s.alpha[32 * hh + lane];
 #pragma unroll
-                for (int h4 = 0; h4 < 8; ++h4) {
-                    const float4 mv = mrun4[h4];
-                    x[4 * h4] -= mv.x; x[4 * h4 + 1] -= mv.y; x[4 * h4 + 2] -= mv.z; x[4 * h4 + 3] -= mv.w;
+                    for (int e = 0; e < 2; ++e) {
+                        const int hd = 2 * lane + e;
+                        const float tm = fmaxf(fmaxf(s.red[set][0][hd], s.red[set][1][hd]),
+                                               fmaxf(s.red[set][2][hd], s.red[set][3][hd]));
+                        const float old = h > 0 ? s.mrun[hd] : -INFINITY;
+                        const float mn = fmaxf(old, tm);
+                        s.mrun[hd] = mn;
+                        s.alpha[set][hd] = old == -INFINITY ? 0.0f : ex2(old - mn);
+                    }
+                }
+                group_sync(set);
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const float2 mv = *reinterpret_cast<const float2 *>(&s.mrun[8 * r + 2 * cc]);
+                    x[4 * r] -= mv.x; x[4 * r + 1] -= mv.y; x[4 * r + 2] -= mv.x; x[4 * r + 3] -= mv.y;
                 }
             }
-            // p = 2^(x - m); P^T carries the key's scale (V holds SWA codes, not values)
-            const float sv = valid ? sig : 0.0f;
-            uint32_t pk[16];
-#pragma unroll
-            for (int h2 = 0; h2 < 16; ++h2) {
-                const float p0 = ex2(x[2 * h2]), p1 = ex2(x[2 * h2 + 1]);
-                x[2 * h2] = p0;
-                x[2 * h2 + 1] = p1;
-                pk[h2] = pack_h2(p0 * sv, p1 * sv);
+            // bring the row sums to this tile's running max; then the next tile may move it
+            {
+                const float2 mt = *reinterpret_cast<const float2 *>(&s.mrun[8 * ii + 2 * cc]);
+                const float2 mr = *mref;
+                if (mt.x != mr.x) lsum[0] = lsum[0] > 0.0f ? lsum[0] * ex2(mr.x - mt.x) : 0.0f;   // the max only grows
+                if (mt.y != mr.y) lsum[1] = lsum[1] > 0.0f ? lsum[1] * ex2(mr.y - mt.y) : 0.0f;
+                *mref = mt;
             }
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                *reinterpret_cast<uint4 *>(s.pt + swz(r, 4 * hh + c)) =
-                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            if (upd && i > 0) {
-                // the running max moved: O^T(i - 1) has landed (pv_done above); scale this
-                // warp's 32 head columns of every block before O^T(i) accumulates on them
-#pragma unroll 1
-                for (int j = 0; j < 2 * kStages; ++j) {    // 16 head columns at a time
-                    float f[16];
-#pragma unroll
-                    for (int h = 0; h < 16; ++h) f[h] = s.alpha[32 * hh + 16 * (j & 1) + h];
-                    tmem_scale16(tmem + lane_base + 64u * (uint32_t)(j >> 1) + 32u * (uint32_t)hh + 16u * (uint32_t)(j & 1), f);
-                }
-                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-            }
-            fence_async_smem();
-            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s.p_full);
-            // l after P is released: the sum is off the output MMAs' critical path
-            lsum += reduce_scatter32<false>(x, lane);   // this tile's 32 keys, head 32 hh + lane
+            if (lane == 0) mbar_arrive(&s.m_ready[set]);
+            // p = 2^(x - m); P^T carries the key's scale (V holds SWA codes, not values).
+            // Row kA (and kA + 8) of P^T, 16-byte chunk r: word cc = heads 8 r + 2 cc, + 1.
+            const float svA = vA ? sgA : 0.0f, svB = vB ? sgB : 0.0f;
+            uint8_t *pt = s.pt[set];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) x[4 * r + k] = ex2(x[4 * r + k]);
+                const uint32_t off = (uint32_t)(((r ^ ii) << 4) + 4 * cc);
+                *reinterpret_cast<uint32_t *>(pt + kA * 128 + off) = pack_h2(x[4 * r] * svA, x[4 * r + 1] * svA);
+                *reinterpret_cast<uint32_t *>(pt + (kA + 8) * 128 + off) =
+                    pack_h2(x[4 * r + 2] * svB, x[4 * r + 3] * svB);
+            }
+            // The row sums are taken after P is released (off the output MMAs' critical
+            // path), except when O must be rescaled first: then before, so that x is no
+            // longer live during the rescale.
+            float2 ls;
+            if (upd && h > 0) {
+                ls = reduce_keys16<false>(x, lane);   // heads 8 ii + 2 cc, + 1
+                // the running max moved: once O^T(h - 1) has landed, scale this warp's lanes
+                // (32 channels of every block) before O^T(h) accumulates on them
+                const bool landed =
+                    __all_sync(0xFFFFFFFFu, mbar_wait(&s.pv_done[set ^ 1], ((h - 1) >> 1) & 1, lim, s));
+                if (landed) {
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int j = 0; j < 4 * kStages; ++j) {    // block j / 4, 16 head columns at a time
+                        float f[16];
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) f[k] = s.alpha[set][16 * (j & 3) + k];
+                        tmem_scale16(tmem + lane_base + 64u * (uint32_t)(j >> 2) + 16u * (uint32_t)(j & 3), f);
+                    }
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                } else if (lane == 0) {
+                    atomicExch(&s.abort, 1);
+                    set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
+                }
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.p_full[set]);
+            } else {
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s.p_full[set]);
+                ls = reduce_keys16<false>(x, lane);
+            }
+            lsum[0] += ls.x;
+            lsum[1] += ls.y;
         }
         ok = ok && !stop;
-        if (ok && nt > 0) {
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.pv_done, (nt - 1) & 1, lim, s));
+        if (ok && set < nt) {
+            // O^T of this set's last tile has landed.  (Only the set's own pv_done: its
+            // previous phase is known complete, so the parity wait cannot alias; the MMA
+            // warp's drain covers every MMA before the combine.)
+            const int hl = nt - 1 - (((nt - 1) ^ set) & 1);
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.pv_done[set], (hl >> 1) & 1, lim, s));
             tc_fence_after();
         }
         if (!ok && lane == 0) {
             atomicExch(&s.abort, 1);
             set_dev_err(a.dev_err, CSA2_DEVERR_TIMEOUT);
         }
-        // this CTA's partial sum per head: the four quadrants' sums (the group barrier is
-        // taken by all four warps of the half, aborted or not)
-        s.red[hh][qd][lane] = lsum;
-        group_sync(hh);
-        if (qd == 0) {
-            const bool have = nt > 0 && !aborted(s);
-            s.cl[32 * hh + lane] = have ? s.red[hh][0][lane] + s.red[hh][1][lane] + s.red[hh][2][lane] +
-                                              s.red[hh][3][lane]
-                                        : 0.0f;
-            s.cm[32 * hh + lane] = have ? s.mrun[32 * hh + lane] : -INFINITY;
-        }
+        // this warp's row sums (the max they are taken against is in s.mref)
+        *reinterpret_cast<float2 *>(&s.red[set][qd][8 * ii + 2 * cc]) = make_float2(lsum[0], lsum[1]);
     }
 
     // ---- combine the two key halves of the query through distributed shared memory ----
@@ -866,13 +956,31 @@ attn_kernel(AttnArgs a) {
     // of both CTAs takes every cluster barrier, whatever happened above.
     __syncwarp();
     tc_fence_before();
-    __syncthreads();                       // stats written; this CTA's MMAs have completed
+    __syncthreads();                       // row sums written; this CTA's MMAs have completed
     tc_fence_after();
+    const bool have = __shfl_sync(0xFFFFFFFFu, (int)(nt > 0 && !aborted(s)), 0) != 0;
+    if (threadIdx.x < kHeads) {
+        // this CTA's partial max and sum per head: the eight warps' sums brought to the
+        // final running max, in a fixed order
+        const int h = threadIdx.x;
+        const float m = s.mrun[h];
+        float l = 0.0f;
+#pragma unroll
+        for (int st = 0; st < kSets; ++st)
+#pragma unroll
+            for (int w = 0; w < kSetWarps; ++w) {
+                const float ls = s.red[st][w][h];
+                if (ls > 0.0f) l += ls * ex2(s.mref[st][w][h] - m);
+            }
+        s.cl[h] = have ? l : 0.0f;
+        s.cm[h] = have ? m : -INFINITY;
+    }
+    __syncthreads();
     // Every CTA owns NB = 4 / CS of the four 128-channel blocks (blocks NB r ..): it sends
     // its partial of every other CTA's blocks (scaled by its weight) into that CTA's
     // shared memory and adds what the others sent it to its own.
     constexpr int NB = 4 / CS;
-    constexpr uint32_t kPiece = NB * kTK * (kHeads / 2) * 4;   // one peer's blocks, one head half, fp32
+    constexpr uint32_t kPiece = NB * kCh * (kHeads / 2) * 4;   // one peer's blocks, one head half, fp32
     constexpr int kPieceF = (int)(kPiece / 4);
     for (int i = threadIdx.x; i < CS * kHeads; i += kThreads) {   // stats to every CTA, own slot `rank`
         const int r2 = i / kHeads, h = i % kHeads;
@@ -917,12 +1025,11 @@ attn_kernel(AttnArgs a) {
     // start, send slots follow them in s.kv and then s.q (both free by now).
     // Task u (warp u % 12 takes u, so the TMEM lane quadrant u % 4 is the warp's):
     // channels 32 (u % 4) .., head half (u >> 2) & 1, block bsel / send slot from u >> 3.
-    const bool have = __shfl_sync(0xFFFFFFFFu, (int)(nt > 0 && !aborted(s)), 0) != 0;
-    auto recv_slot = [&](int i) { return reinterpret_cast<float *>(&s.kv[0][0]) + i * 2 * kPieceF; };
+    auto recv_slot = [&](int i) { return reinterpret_cast<float *>(&s.kv[0][0][0]) + i * 2 * kPieceF; };
     auto send_slot = [&](int j) {
         const int k = (CS - 1) + j;        // slot index in the sequence s.kv, then s.q
         return k * 2 * kPieceF < (int)(sizeof(s.kv) / 4)
-                   ? reinterpret_cast<float *>(&s.kv[0][0]) + k * 2 * kPieceF
+                   ? reinterpret_cast<float *>(&s.kv[0][0][0]) + k * 2 * kPieceF
                    : reinterpret_cast<float *>(s.q) + (k * 2 * kPieceF - (int)(sizeof(s.kv) / 4));
     };
 #pragma unroll 1
@@ -938,7 +1045,7 @@ attn_kernel(AttnArgs a) {
 #pragma unroll
             for (int h = 0; h < 32; ++h) o[h] = 0.0f;
         }
-        float4 *dst = reinterpret_cast<float4 *>(send_slot(j) + hp * kPieceF + (bsel * kTK + crow) * (kHeads / 2));
+        float4 *dst = reinterpret_cast<float4 *>(send_slot(j) + hp * kPieceF + (bsel * kCh + crow) * (kHeads / 2));
 #pragma unroll
         for (int f = 0; f < 8; ++f) {                // float4 f = heads 32 hp + 4 f ..
             const int h = 32 * hp + 4 * f;
@@ -978,7 +1085,7 @@ attn_kernel(AttnArgs a) {
 #pragma unroll 1
         for (int i = 0; i < CS - 1; ++i) {           // the senders in a fixed order
             const float4 *src = reinterpret_cast<const float4 *>(recv_slot(i) + hp * kPieceF +
-                                                                 (bsel * kTK + crow) * (kHeads / 2));
+                                                                 (bsel * kCh + crow) * (kHeads / 2));
 #pragma unroll
             for (int f = 0; f < 8; ++f) {
                 const float4 pr = got ? src[f ^ (crow & 7)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -1047,3 +1154,4 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, int BT, cudaStream_t st) {
 }
 
 }  // namespace csa2
+
