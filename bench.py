@@ -92,8 +92,8 @@ def attn_flops(wl) -> int:
 # scaled to the batch, only for decode workloads and while the code is unchanged.
 NCU_TRAFFIC = {
     # attention: attn_kernel<0, 2> (2 CTAs per query) at batch 40, one launch
-    "csa2_sparse_attn_decode": ([(13_225_216, 40)], ("csa2_attn.cu",), "4045433ab704ea1f"),
-    "csa2_sparse_attn_decode_append": ([(13_225_216, 40)], ("csa2_attn.cu",), "4045433ab704ea1f"),
+    "csa2_sparse_attn_decode": ([(13_228_032, 40)], ("csa2_attn.cu",), "7fbe922818180b08"),
+    "csa2_sparse_attn_decode_append": ([(13_228_032, 40)], ("csa2_attn.cu",), "7fbe922818180b08"),
     # Full: index_scan_kernel + select_full_kernel at batch 8
     "csa2_index_full": ([(138_491_392 + 5_009_408, 8), (1_134_080, 8)], ("csa2_index.cu",),
                         "db4b2a2e98873967"),

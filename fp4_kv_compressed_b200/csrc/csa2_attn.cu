@@ -939,7 +939,7 @@ attn_kernel(AttnArgs a) {
             // O^T of this set's last tile has landed.  (Only the set's own pv_done: its
             // previous phase is known complete, so the parity wait cannot alias; the MMA
             // warp's drain covers every MMA before the combine.)
-            const int hl = nt - 1 - (((nt - 1) ^ set) & 1);
+            const int hl = set + ((nt - 1 - set) / kSets) * kSets;
             ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s.pv_done[set], (hl >> 1) & 1, lim, s));
             tc_fence_after();
         }
