@@ -101,6 +101,41 @@ def test_attention_edges(pkg, orc):
     assert bits & pkg.DEVERR_INDEX
 
 
+@pytest.mark.parametrize("B,top_k", [(1, 384), (1, 512), (38, 512)])
+def test_attention_running_max_moves_every_tile(pkg, orc, B, top_k):
+    """Entry e is c_e times head 0 of the query, c_e growing along the key order, so the
+    logits of every later 64-key tile exceed the running max by more than 8 (log2 units):
+    the max moves and O is rescaled on every tile, by each worker set in turn (after the
+    other set's output MMAs of the previous tile).  B = 1: 4 CTAs per query, 2 or 3 tiles
+    each; B = 38: 2 CTAs per query, 5 tiles each.  Within the tolerance of the oracle."""
+    H, cap, W = 64, 700, 128
+    q_pos = torch.full((B, 1), 699, dtype=torch.int32)
+    q = torch.stack([synth.rows_normal_bf16(9, "q", b, 0, H, 512, stride=synth.Q_STRIDE)
+                     for b in range(B)]).view(B, 1, H, 512)
+    c = torch.arange(cap, dtype=torch.float32) * 0.006
+    x = (c.view(1, cap, 1) * q[:, 0, 0].float().view(B, 1, 512)).to(torch.bfloat16)
+    sw = torch.stack([synth.rows_normal_bf16(9, "swa", b, 0, W, 512) for b in range(B)])
+    kv = pkg.GlobalKV(B, cap, 128, 1, "cuda")
+    ring = pkg.SwaRing(B, W, "cuda")
+    z = torch.zeros(B, dtype=torch.int32, device="cuda")
+    pkg.csa2_quantize_append(kv.struct, x.cuda(), None, cap, z, ring.struct, sw.cuda(), W, z)
+    topk = torch.arange(top_k, dtype=torch.int32).view(1, 1, top_k).expand(B, 1, top_k).contiguous()
+    out = torch.zeros(B, 1, H, 512, device="cuda")
+    lse = torch.zeros(B, 1, H, device="cuda")
+    dev_err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkg.csa2_sparse_attn_decode(kv.struct, ring.struct, q.cuda(), q_pos.cuda(), 1, H, topk.cuda(), top_k,
+                                128, 1 / math.sqrt(512), out, lse, None, dev_err)
+    assert pkg.csa2_read_device_error(dev_err) == 0
+    mc, ms = orc.quantize_fp4(x)
+    sc, ss = orc.quantize_fp8(sw)
+    o_ref, l_ref = orc.attention(mc, ms, sc, ss, q, q_pos.numpy(), topk.numpy(), 128, 1 / math.sqrt(512))
+    # the premise: head 0's logits (log2 units) rise by more than 8 per 64 entries
+    qq = q[0, 0, 0].double()
+    step = float((qq * qq).sum()) * 0.006 * 64 / math.sqrt(512) / math.log(2)
+    assert step > 8
+    _assert_close(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref)
+
+
 def _stack_check(wl, requests, layers=None):
     import csa2_harness
     dw = csa2_harness.DeviceWorkload(wl)
