@@ -36,7 +36,7 @@ EXPORTS = ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_workspace_
            "csa2_status_string", "csa2_abi_version", "csa2_debug_set_waits",
            "csa2_index_full_slice", "csa2_index_merge", "csa2_attn_combine",
            "csa2_quantize_append_paged", "csa2_index_full_paged", "csa2_index_reindex_paged",
-           "csa2_sparse_attn_decode_paged")
+           "csa2_sparse_attn_decode_paged", "csa2_sparse_attn_decode_reuse")
 
 
 class Csa2Error(RuntimeError):
@@ -123,8 +123,9 @@ def load_library(path: str = LIB_PATH):
     L.csa2_index_reindex_paged.argtypes = [P, P, P, P, i32, i32, P, i32, i32, P, P, P, sz, P, P]
     L.csa2_sparse_attn_decode_paged.argtypes = [P, P, P, P, P, i32, i32, P, i32, i32, C.c_float,
                                                 P, P, P, P, P]
+    L.csa2_sparse_attn_decode_reuse.argtypes = L.csa2_sparse_attn_decode_paged.argtypes
     for fn in ("csa2_quantize_append_paged", "csa2_index_full_paged", "csa2_index_reindex_paged",
-               "csa2_sparse_attn_decode_paged"):
+               "csa2_sparse_attn_decode_paged", "csa2_sparse_attn_decode_reuse"):
         getattr(L, fn).restype = C.c_int
     for fn in ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_index_full",
                "csa2_index_full_tc", "csa2_index_reindex", "csa2_sparse_attn_decode",
@@ -275,6 +276,19 @@ def csa2_index_reindex_paged(kv: CSA2PagedKV, q_idx, w, q_pos, Tq: int, H_I: int
                                     _ptr(topk_count), _ptr(workspace), ws_bytes, _ptr(dev_err),
                                     _stream(stream))
     _check("csa2_index_reindex_paged", st)
+
+
+def csa2_sparse_attn_decode_reuse(kv: CSA2GlobalKV, swa: CSA2SWA | None, swa_bf16, q, q_pos,
+                                  Tq: int, H: int, topk, top_k: int, swa_len: int,
+                                  softmax_scale: float, rope, out, lse, dev_err=None, stream=None):
+    """The sparse attention of a Reuse layer (swa_bf16 None: no fused append), whose
+    inputs were all written two or more launches earlier on the stream."""
+    L = load_library()
+    st = L.csa2_sparse_attn_decode_reuse(
+        C.byref(kv), C.byref(swa) if swa is not None else None, _ptr(swa_bf16), _ptr(q), _ptr(q_pos),
+        Tq, H, _ptr(topk), top_k, swa_len, softmax_scale, C.byref(rope) if rope is not None else None,
+        _ptr(out), _ptr(lse), _ptr(dev_err), _stream(stream))
+    _check("csa2_sparse_attn_decode_reuse", st)
 
 
 def csa2_sparse_attn_decode_paged(kv: CSA2PagedKV, swa: CSA2SWA | None, swa_bf16, q, q_pos,

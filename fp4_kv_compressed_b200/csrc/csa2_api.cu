@@ -136,7 +136,7 @@ bool hi_supported(int32_t H_I) {
 
 extern "C" {
 
-int32_t csa2_abi_version(void) { return 104; }
+int32_t csa2_abi_version(void) { return 105; }
 
 void csa2_debug_set_waits(uint64_t limit_ns, int32_t stuck_wait) {
     g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
@@ -443,7 +443,8 @@ static csa2_status sparse_attn(const KvView *kv, const csa2_swa *swa, const void
                                const void *q_bf16, const int32_t *q_pos, int32_t Tq, int32_t H,
                                const int32_t *topk, int32_t top_k, int32_t swa_len,
                                float softmax_scale, const csa2_rope *rope, float *out,
-                               float *lse, int32_t *dev_err, csa2_stream_t stream) {
+                               float *lse, int32_t *dev_err, csa2_stream_t stream,
+                               bool settled = false) {
     csa2_status st = check_kv(kv, false);
     if (st != CSA2_OK) return st;
     if (!q_bf16 || !q_pos || !out || !lse) return CSA2_ERR_INVALID_ARG;
@@ -489,6 +490,7 @@ static csa2_status sparse_attn(const KvView *kv, const csa2_swa *swa, const void
     a.lse = lse;
     a.dev_err = dev_err;
     a.wait = current_wait_cfg();
+    a.settled = settled ? 1 : 0;
     return launched(launch_sparse_attn(a, (int)BT, (cudaStream_t)stream));
 }
 
@@ -530,6 +532,23 @@ csa2_status csa2_sparse_attn_decode_append_rope(
     KvView v;
     return sparse_attn(view_of(kv, &v), swa, swa_bf16, q_bf16, q_pos, Tq, H, topk, top_k, swa_len,
                        softmax_scale, rope, out, lse, dev_err, stream);
+}
+
+csa2_status csa2_sparse_attn_decode_reuse(const csa2_global_kv *kv, const csa2_swa *swa,
+                                          const void *swa_bf16, const void *q_bf16,
+                                          const int32_t *q_pos, int32_t Tq, int32_t H,
+                                          const int32_t *topk, int32_t top_k, int32_t swa_len,
+                                          float softmax_scale, const csa2_rope *rope, float *out,
+                                          float *lse, int32_t *dev_err, csa2_stream_t stream) {
+    if (swa_bf16) {
+        if (Tq != 1) return CSA2_ERR_UNSUPPORTED;
+        if (swa_len <= 0 || !swa || !aligned(swa_bf16, 16)) return CSA2_ERR_INVALID_ARG;
+    } else if (rope) {
+        return CSA2_ERR_INVALID_ARG;
+    }
+    KvView v;
+    return sparse_attn(view_of(kv, &v), swa, swa_bf16, q_bf16, q_pos, Tq, H, topk, top_k, swa_len,
+                       softmax_scale, rope, out, lse, dev_err, stream, true);
 }
 
 // ---- paged cache: the same calls over a csa2_paged_kv ----------------------------------

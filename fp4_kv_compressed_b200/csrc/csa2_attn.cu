@@ -585,8 +585,11 @@ attn_kernel(AttnArgs a) {
                 make_uint4(h[0], h[1], h[2], h[3]);
         }
     }
-    // everything below may read what the previous kernel of the stream wrote (the Top-K)
-    grid_dep_wait();
+    // everything below may read what the previous kernel of the stream wrote (the Top-K),
+    // unless the caller settled every input two or more launches earlier: then the wait
+    // moves to just before the next launch is let go (each kernel of the library waits
+    // before it does that, so whatever was written two launches back is complete here)
+    if (!a.settled) grid_dep_wait();
     const int *tk = a.topk + (int64_t)qi * a.top_k;
     const int e_id0 = (int)threadIdx.x < a.top_k ? tk[threadIdx.x] : -1;
     const int e_id1 = (int)threadIdx.x + kThreads < a.top_k ? tk[threadIdx.x + kThreads] : -1;
@@ -997,6 +1000,7 @@ attn_kernel(AttnArgs a) {
         mbar_expect_tx(&s.xfer[1], (CS - 1) * kPiece);
     }
     cluster_sync();                        // stats exchanged; every CTA's tiles are free
+    if (a.settled) grid_dep_wait();
     grid_dep_launch();
     if (threadIdx.x < kHeads) {
         const int h = threadIdx.x;

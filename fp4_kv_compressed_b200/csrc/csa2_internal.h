@@ -125,6 +125,10 @@ struct AttnArgs {
     int32_t *dev_err;
     WaitCfg wait;
     PageMap pm;
+    // 1: every input was written at least two launches earlier on the stream (a Reuse
+    // layer), so the kernel reads them before its dependency wait and waits only before
+    // it lets the next launch start
+    int32_t settled;
 };
 
 // Every kernel of the library asks for the largest shared-memory carveout, so that

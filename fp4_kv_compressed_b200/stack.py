@@ -130,6 +130,9 @@ class DecodeStack:
         # "exact": the fixed fp32 score order (reproducible Top-K); "tc": the tensor-core
         # scan for prefill chunks (relaxed summation order, see csa2_index_full_tc)
         self.index_scan = index_scan
+        # Reuse layers launch with csa2_sparse_attn_decode_reuse (overlapping the previous
+        # launch); False: the ordinary calls (same results, bit for bit)
+        self.reuse_launch = True
         # a _binding.Rope: the main-KV and SWA rows are passed before RoPE and rotated
         # inside the append launches (csa2_quantize_append_rope and the fused attention)
         self.rope = rope
@@ -219,7 +222,15 @@ class DecodeStack:
                                      self.count[l], self.workspace, self.dev_err, stream)
             fused = (l != first_of_group[g] or kv_bf16 is None or kv_bf16[g] is None) \
                 and swa_bf16[l] is not None and self._fuse_swa(T_swa)
-            if fused and rope is not None:
+            if fused and lp.mode == "U" and self.reuse_launch:
+                # a Reuse layer: its Top-K and every other input were written two or more
+                # launches back (the source layer's attention launched in between), so
+                # the launch overlaps the previous one
+                bind.csa2_sparse_attn_decode_reuse(
+                    kv.struct, self.swa[l].struct, swa_bf16[l], q[l], q_pos, self.Tq, self.H,
+                    self.topk_of(l), self.top_k, self.swa_len, self.softmax_scale, rope,
+                    self.out[l], self.lse[l], self.dev_err, stream)
+            elif fused and rope is not None:
                 bind.csa2_sparse_attn_decode_append_rope(
                     kv.struct, self.swa[l].struct, swa_bf16[l], q[l], q_pos, self.Tq, self.H,
                     self.topk_of(l), self.top_k, self.swa_len, self.softmax_scale, rope,

@@ -403,6 +403,30 @@ CSA2_API csa2_status csa2_sparse_attn_decode_append_rope(
     void *workspace, size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream);
 
 /*
+ * The sparse attention of a Reuse layer (study notes section 2: a Reuse layer attends
+ * over the selection of an earlier layer), launched so that it overlaps the previous
+ * launch on the stream.  swa_bf16 non-NULL = the fused decode append of
+ * csa2_sparse_attn_decode_append (Tq = 1), rope non-NULL (with swa_bf16) = its RoPE
+ * form; both NULL = csa2_sparse_attn_decode.  Same arguments, checks and results, bit
+ * for bit.
+ *   Precondition (the caller's): no input of the call (kv, swa, q_bf16, q_pos, topk,
+ *   swa_bf16, rope) is written, and no output (out, lse, the layer's ring row) read, by
+ *   the launch that immediately precedes it on `stream` (a Reuse layer: its topk comes
+ *   from a Full or Reindex layer whose own attention launched in between).  The kernel then reads them before it waits for the previous
+ *   launch (every launch of the library waits for its predecessor before it lets the
+ *   next one start, so whatever was written two launches back is complete), and waits
+ *   before it lets the next launch start.  A kernel outside the library that lets its
+ *   dependents start early (programmatic dependent launch) must not write the inputs.
+ */
+CSA2_API csa2_status csa2_sparse_attn_decode_reuse(const csa2_global_kv *kv, const csa2_swa *swa,
+                                                   const void *swa_bf16, const void *q_bf16,
+                                                   const int32_t *q_pos, int32_t Tq, int32_t H,
+                                                   const int32_t *topk, int32_t top_k,
+                                                   int32_t swa_len, float softmax_scale,
+                                                   const csa2_rope *rope, float *out, float *lse,
+                                                   int32_t *dev_err, csa2_stream_t stream);
+
+/*
  * Paged global KV (serving: requests of different lengths share one pool of pages;
  * the pages' cache is the one global KV of study notes section 5 / myzaker "cache
  * precision and tiering", here laid out in fixed-size pages).  The planes hold

@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol(pkg):
     assert set(names) == set(pkg.EXPORTS)
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.csa2_abi_version() == 104      # 1.4: the paged cache
+    assert lib.csa2_abi_version() == 105      # 1.5: the Reuse-layer attention launch
     for st in range(7):
         assert lib.csa2_status_string(st)
 

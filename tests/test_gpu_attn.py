@@ -136,6 +136,30 @@ def test_attention_running_max_moves_every_tile(pkg, orc, B, top_k):
     _assert_close(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref)
 
 
+@pytest.mark.parametrize("name", ["decode_128k", "decode_1m"])
+def test_reuse_launch_matches_ordinary_calls(pkg, name):
+    """Reuse layers launched with csa2_sparse_attn_decode_reuse (inputs read before the
+    dependency wait, the launch overlapping the previous one) give the same outputs and
+    lse on every layer, bit for bit, as the ordinary calls: whole decode stacks, so that
+    every Reuse layer follows another layer's launch on the stream."""
+    import csa2_harness
+    wl = small_variant(WORKLOADS[name], B=4, ctx=6000)
+    res = []
+    for reuse in (False, True):
+        dw = csa2_harness.DeviceWorkload(wl)
+        dw.stack.reuse_launch = reuse
+        st = torch.cuda.Stream()      # a real stream, where launches may overlap
+        st.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(st):
+            dw.step(stream=st)
+        torch.cuda.synchronize()
+        assert dw.stack.dev_err.item() == 0
+        res.append([t.clone() for t in dw.stack.out] + [t.clone() for t in dw.stack.lse])
+    assert len(res[0]) > 0
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
+
+
 def _stack_check(wl, requests, layers=None):
     import csa2_harness
     dw = csa2_harness.DeviceWorkload(wl)
