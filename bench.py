@@ -92,13 +92,15 @@ def attn_flops(wl) -> int:
 # scaled to the batch, only for decode workloads and while the code is unchanged.
 NCU_TRAFFIC = {
     # attention: attn_kernel<0, 2> (2 CTAs per query) at batch 40, one launch
-    "csa2_sparse_attn_decode": ([(13_228_032, 40)], ("csa2_attn.cu",), "7fbe922818180b08"),
-    "csa2_sparse_attn_decode_append": ([(13_228_032, 40)], ("csa2_attn.cu",), "7fbe922818180b08"),
+    "csa2_sparse_attn_decode": ([(13_244_160, 40)], ("csa2_attn.cu",), "0533d212713e8e2b"),
+    "csa2_sparse_attn_decode_append": ([(13_244_160, 40)], ("csa2_attn.cu",), "0533d212713e8e2b"),
+    "csa2_sparse_attn_decode_reuse": ([(13_244_160, 40)], ("csa2_attn.cu",), "0533d212713e8e2b"),
     # Full: index_scan_kernel + select_full_kernel at batch 8
-    "csa2_index_full": ([(138_491_392 + 5_009_408, 8), (1_134_080, 8)], ("csa2_index.cu",),
-                        "db4b2a2e98873967"),
+    "csa2_index_full": ([(138_471_424 + 4_538_624, 8), (1_134_336, 8)], ("csa2_index.cu",),
+                        "2c19ef68d42489bf"),
     # Reindex: reindex_score_kernel + select_reindex_kernel at batch 8
-    "csa2_index_reindex": ([(18_609_920, 8), (550_144, 8)], ("csa2_index.cu",), "db4b2a2e98873967"),
+    "csa2_index_reindex": ([(18_609_408, 8), (553_472, 8)], ("csa2_index.cu",), "2c19ef68d42489bf"),
+    "csa2_index_reindex_settled": ([(18_609_408, 8), (553_472, 8)], ("csa2_index.cu",), "2c19ef68d42489bf"),
 }
 
 
@@ -137,15 +139,18 @@ OP_KERNELS = {
     "csa2_index_full": "index_scan_kernel + select_full_kernel",
     "csa2_index_full_tc": "index_scan_tc_kernel + select_full_kernel",
     "csa2_index_reindex": "reindex_score_kernel + select_reindex_kernel",
+    "csa2_index_reindex_settled": "reindex_score_kernel (overlapping the previous launch) + select_reindex_kernel",
     "csa2_sparse_attn_decode": "attn_kernel",
+    "csa2_sparse_attn_decode_reuse": "attn_kernel (Reuse layer, with the SWA append, overlapping the previous launch)",
     "csa2_sparse_attn_decode_append": "attn_kernel (with the SWA append)",
     "csa2_sparse_attn_decode_append_rope": "attn_kernel (with the RoPE + SWA append)",
 }
 
 
-def op_step_bytes(wl, plan, rope: bool = False, index_scan: str = "exact") -> dict:
+def op_step_bytes(wl, plan, rope: bool = False, index_scan: str = "exact", reuse: bool = True) -> dict:
     """Per library call name: (algorithmic bytes per step, launches per step), walking the
-    layer plan the way DecodeStack.step issues its calls."""
+    layer plan the way DecodeStack.step issues its calls (reuse: DecodeStack.reuse_launch,
+    the Reuse and Reindex layers' overlapping calls)."""
     ob = op_bytes(wl)
     fused = wl.Tq == 1 and wl.swa_len > 0          # decode: SWA append inside the attention
     first = {}
@@ -167,9 +172,12 @@ def op_step_bytes(wl, plan, rope: bool = False, index_scan: str = "exact") -> di
         if lp.mode == "F":
             add(full, ob[f"index_full_g{g}"])
         elif lp.mode == "X":
-            add("csa2_index_reindex", ob[f"index_reindex_g{g}"])
+            add("csa2_index_reindex_settled" if reuse else "csa2_index_reindex", ob[f"index_reindex_g{g}"])
         if fused and lp.layer != first[g]:
-            name = "csa2_sparse_attn_decode_append" + ("_rope" if rope else "")
+            if reuse and lp.mode == "U":
+                name = "csa2_sparse_attn_decode_reuse"
+            else:
+                name = "csa2_sparse_attn_decode_append" + ("_rope" if rope else "")
             add(name, ob["attn"] + ob["swa_append"] + (ob["rope_row"] if rope else 0))
         else:
             add("csa2_sparse_attn_decode", ob["attn"])
@@ -177,11 +185,11 @@ def op_step_bytes(wl, plan, rope: bool = False, index_scan: str = "exact") -> di
 
 
 def op_rooflines(wl, plan, op_ms: dict, ms_step: float, rope: bool = False,
-                 index_scan: str = "exact") -> dict:
+                 index_scan: str = "exact", reuse: bool = True) -> dict:
     """Per library call: algorithmic bytes (and flops) per step over its measured time per
     step.  op_ms[name] = (total ms per step of the calls of that name, calls per step)."""
     pk = measured_peaks()
-    per = op_step_bytes(wl, plan, rope, index_scan)
+    per = op_step_bytes(wl, plan, rope, index_scan, reuse)
     modes = [lp.mode for lp in plan]
     out = {}
     for name, (tot_ms, n) in op_ms.items():
@@ -473,8 +481,9 @@ def run_ours(args, rank, world, local_rank):
     with torch.cuda.graph(g1, stream=stream):
         st.step(**inputs)
     op_names = [n for n in ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_index_full",
-                            "csa2_index_full_tc", "csa2_index_reindex", "csa2_sparse_attn_decode",
-                            "csa2_sparse_attn_decode_append", "csa2_sparse_attn_decode_append_rope")
+                            "csa2_index_full_tc", "csa2_index_reindex", "csa2_index_reindex_settled",
+                            "csa2_sparse_attn_decode", "csa2_sparse_attn_decode_append",
+                            "csa2_sparse_attn_decode_append_rope", "csa2_sparse_attn_decode_reuse")
                 if hasattr(stack_mod.bind, n)]
     originals = {name: getattr(stack_mod.bind, name) for name in op_names}
     marks = []                       # (op name, event after the call)
@@ -605,7 +614,8 @@ def run_ours(args, rank, world, local_rank):
     sb = step_bytes(wl)
     ob = op_bytes(wl)
     g_full = st.plan[full_layers[0]].group
-    ops = op_rooflines(wl, st.plan, op_ms, ops_step_ms, rope=args.rope, index_scan=args.index_scan)
+    ops = op_rooflines(wl, st.plan, op_ms, ops_step_ms, rope=args.rope, index_scan=args.index_scan,
+                       reuse=st.reuse_launch)
     dominant = max(ops, key=lambda n: ops[n]["share_of_step"])
     launches = st.launches_per_step() * K
     line = {

@@ -36,7 +36,8 @@ EXPORTS = ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_workspace_
            "csa2_status_string", "csa2_abi_version", "csa2_debug_set_waits",
            "csa2_index_full_slice", "csa2_index_merge", "csa2_attn_combine",
            "csa2_quantize_append_paged", "csa2_index_full_paged", "csa2_index_reindex_paged",
-           "csa2_sparse_attn_decode_paged", "csa2_sparse_attn_decode_reuse")
+           "csa2_sparse_attn_decode_paged", "csa2_sparse_attn_decode_reuse",
+           "csa2_index_reindex_settled")
 
 
 class Csa2Error(RuntimeError):
@@ -124,8 +125,10 @@ def load_library(path: str = LIB_PATH):
     L.csa2_sparse_attn_decode_paged.argtypes = [P, P, P, P, P, i32, i32, P, i32, i32, C.c_float,
                                                 P, P, P, P, P]
     L.csa2_sparse_attn_decode_reuse.argtypes = L.csa2_sparse_attn_decode_paged.argtypes
+    L.csa2_index_reindex_settled.argtypes = L.csa2_index_reindex.argtypes
     for fn in ("csa2_quantize_append_paged", "csa2_index_full_paged", "csa2_index_reindex_paged",
-               "csa2_sparse_attn_decode_paged", "csa2_sparse_attn_decode_reuse"):
+               "csa2_sparse_attn_decode_paged", "csa2_sparse_attn_decode_reuse",
+               "csa2_index_reindex_settled"):
         getattr(L, fn).restype = C.c_int
     for fn in ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_index_full",
                "csa2_index_full_tc", "csa2_index_reindex", "csa2_sparse_attn_decode",
@@ -313,6 +316,19 @@ def csa2_index_reindex(kv: CSA2GlobalKV, q_idx, w, q_pos, Tq: int, H_I: int, poo
                               _ptr(pool), pool_blocks, top_k, _ptr(topk_out), _ptr(topk_count),
                               _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream))
     _check("csa2_index_reindex", st)
+
+
+def csa2_index_reindex_settled(kv: CSA2GlobalKV, q_idx, w, q_pos, Tq: int, H_I: int, pool,
+                               pool_blocks: int, top_k: int, topk_out, topk_count, workspace,
+                               dev_err=None, stream=None):
+    """csa2_index_reindex whose scoring overlaps the previous launch on the stream (every
+    input written two or more launches earlier)."""
+    L = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = L.csa2_index_reindex_settled(C.byref(kv), _ptr(q_idx), _ptr(w), _ptr(q_pos), Tq, H_I,
+                                      _ptr(pool), pool_blocks, top_k, _ptr(topk_out), _ptr(topk_count),
+                                      _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream))
+    _check("csa2_index_reindex_settled", st)
 
 
 def csa2_sparse_attn_decode(kv: CSA2GlobalKV, swa: CSA2SWA | None, q, q_pos, Tq: int, H: int,

@@ -385,7 +385,8 @@ static csa2_status index_reindex(const KvView *kv, const void *q_idx_bf16, const
                                  const int32_t *q_pos, int32_t Tq, int32_t H_I,
                                  const int32_t *pool, int32_t pool_blocks, int32_t top_k,
                                  int32_t *topk_out, int32_t *topk_count, void *workspace,
-                                 size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream) {
+                                 size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream,
+                                 bool settled = false) {
     csa2_status st = check_kv(kv, true);
     if (st != CSA2_OK) return st;
     if (!q_idx_bf16 || !w || !q_pos || !pool || !topk_out || !topk_count) return CSA2_ERR_INVALID_ARG;
@@ -423,6 +424,7 @@ static csa2_status index_reindex(const KvView *kv, const void *q_idx_bf16, const
     a.dev_err = dev_err;
     a.wait = current_wait_cfg();
     a.pm = kv->pm;
+    a.settled = settled ? 1 : 0;
     cudaStream_t s = (cudaStream_t)stream;
     st = launched(launch_reindex_score(a, (int)BT, s));
     if (st != CSA2_OK) return st;
@@ -437,6 +439,17 @@ csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_idx_bf16,
     KvView v;
     return index_reindex(view_of(kv, &v), q_idx_bf16, w, q_pos, Tq, H_I, pool, pool_blocks, top_k,
                          topk_out, topk_count, workspace, ws_bytes, dev_err, stream);
+}
+
+csa2_status csa2_index_reindex_settled(const csa2_global_kv *kv, const void *q_idx_bf16,
+                                       const float *w, const int32_t *q_pos, int32_t Tq,
+                                       int32_t H_I, const int32_t *pool, int32_t pool_blocks,
+                                       int32_t top_k, int32_t *topk_out, int32_t *topk_count,
+                                       void *workspace, size_t ws_bytes, int32_t *dev_err,
+                                       csa2_stream_t stream) {
+    KvView v;
+    return index_reindex(view_of(kv, &v), q_idx_bf16, w, q_pos, Tq, H_I, pool, pool_blocks, top_k,
+                         topk_out, topk_count, workspace, ws_bytes, dev_err, stream, true);
 }
 
 static csa2_status sparse_attn(const KvView *kv, const csa2_swa *swa, const void *swa_new_bf16,

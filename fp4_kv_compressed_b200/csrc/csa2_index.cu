@@ -239,7 +239,10 @@ reindex_score_kernel(IndexArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     ScoreSmem<D, HI, R> &s = *reinterpret_cast<ScoreSmem<D, HI, R> *>(smem_raw);
     __shared__ int64_t row_of[kTileRows];   // cache row of each candidate, -1: not scored
-    grid_dep_wait();
+    // settled inputs (written two or more launches back): the wait moves to just before
+    // the next launch is let go (the scores go to a workspace the previous launch does
+    // not read)
+    if (!a.settled) grid_dep_wait();
     const int qi = blockIdx.y;
     const int b = qi / a.Tq;
     int64_t N = visible_entries(a.q_pos[qi], a.ratio);
@@ -274,6 +277,7 @@ reindex_score_kernel(IndexArgs a) {
 
     float sc[R];
     score_rows<D, HI, R>(s, sc);
+    if (a.settled) grid_dep_wait();
     grid_dep_launch();
     float *out = a.scores + (int64_t)qi * a.score_stride + (int64_t)slot0 * 8;
     float *bm = a.bmax + (int64_t)qi * a.bmax_stride + slot0;

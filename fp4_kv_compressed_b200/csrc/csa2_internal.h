@@ -100,6 +100,10 @@ struct IndexArgs {
     uint64_t *pool_keys_out;   // [BT][pool_blocks] or null
     uint64_t *topk_keys_out;   // [BT][top_k] or null
     PageMap pm;
+    // Reindex scoring: 1 when every input was written at least two launches earlier on
+    // the stream; the kernel then waits for the previous launch only before it lets the
+    // next one start
+    int32_t settled;
 };
 
 struct AttnArgs {

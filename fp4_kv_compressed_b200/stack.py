@@ -130,8 +130,9 @@ class DecodeStack:
         # "exact": the fixed fp32 score order (reproducible Top-K); "tc": the tensor-core
         # scan for prefill chunks (relaxed summation order, see csa2_index_full_tc)
         self.index_scan = index_scan
-        # Reuse layers launch with csa2_sparse_attn_decode_reuse (overlapping the previous
-        # launch); False: the ordinary calls (same results, bit for bit)
+        # Reuse layers launch with csa2_sparse_attn_decode_reuse and Reindex layers with
+        # csa2_index_reindex_settled (overlapping the previous launch); False: the
+        # ordinary calls (same results, bit for bit)
         self.reuse_launch = True
         # a _binding.Rope: the main-KV and SWA rows are passed before RoPE and rotated
         # inside the append launches (csa2_quantize_append_rope and the fused attention)
@@ -217,9 +218,13 @@ class DecodeStack:
                      spec.pool_blocks, self.top_k, self.pool[g] if spec.pool_blocks else None,
                      self.topk[l], self.count[l], self.workspace, self.dev_err, stream)
             elif lp.mode == "X":
-                bind.csa2_index_reindex(kv.struct, q_idx[l], w[l], q_pos, self.Tq, self.H_I,
-                                     self.pool[g], spec.pool_blocks, self.top_k, self.topk[l],
-                                     self.count[l], self.workspace, self.dev_err, stream)
+                # the pool comes from the group's Full layer, whose attention launched in
+                # between: the scoring may overlap the previous launch (unless this layer's
+                # own SWA append was just launched, which the scoring does not read either)
+                reindex = bind.csa2_index_reindex_settled if self.reuse_launch else bind.csa2_index_reindex
+                reindex(kv.struct, q_idx[l], w[l], q_pos, self.Tq, self.H_I, self.pool[g],
+                        spec.pool_blocks, self.top_k, self.topk[l], self.count[l], self.workspace,
+                        self.dev_err, stream)
             fused = (l != first_of_group[g] or kv_bf16 is None or kv_bf16[g] is None) \
                 and swa_bf16[l] is not None and self._fuse_swa(T_swa)
             if fused and lp.mode == "U" and self.reuse_launch:

@@ -350,6 +350,23 @@ CSA2_API csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_
                                size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream);
 
 /*
+ * csa2_index_reindex whose scoring overlaps the previous launch on the stream (same
+ * arguments, workspace and results, bit for bit).  Precondition (the caller's): no
+ * input (kv, q_idx_bf16, w, q_pos, pool) is written, and the workspace not read, by the
+ * launch that immediately precedes it on `stream` (a Reindex layer: its pool comes from
+ * the Full layer, whose attention, at least, launched in between).  The scoring kernel
+ * then reads its inputs before it waits for the previous launch (as
+ * csa2_sparse_attn_decode_reuse does); the selection waits for the scoring as usual.
+ */
+CSA2_API csa2_status csa2_index_reindex_settled(const csa2_global_kv *kv, const void *q_idx_bf16,
+                                                const float *w, const int32_t *q_pos, int32_t Tq,
+                                                int32_t H_I, const int32_t *pool,
+                                                int32_t pool_blocks, int32_t top_k,
+                                                int32_t *topk_out, int32_t *topk_count,
+                                                void *workspace, size_t ws_bytes,
+                                                int32_t *dev_err, csa2_stream_t stream);
+
+/*
  * a8 sparse attention.  For each query (request b, token position t = q_pos)
  * and head h:
  *   o_h = sum_j softmax_j(softmax_scale * q_h . v_j) v_j,  K = V = the entry,

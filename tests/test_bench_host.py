@@ -107,16 +107,24 @@ def test_op_rooflines_dominant_and_traffic():
     from fp4_kv_compressed_b200.stack import plan_layers
     wl = WORKLOADS["decode_128k"]
     plan = plan_layers([g.schedule for g in wl.groups])
-    per = bench.op_step_bytes(wl, plan)
+    # the ordinary calls: 19 fused attention launches, 4 Reindex ops
+    per = bench.op_step_bytes(wl, plan, reuse=False)
     assert per["csa2_quantize_append"][1] == 1 and per["csa2_index_full"][1] == 1
     assert per["csa2_index_reindex"][1] == 4 and per["csa2_sparse_attn_decode"][1] == 1
     assert per["csa2_sparse_attn_decode_append"][1] == 19
     assert sum(b for b, _ in per.values()) == bench.step_bytes(wl)
+    # the stack's default: the 15 Reuse layers and the 4 Reindex ops overlap their
+    # predecessors through their own calls; the same bytes in all
+    per_r = bench.op_step_bytes(wl, plan)
+    assert per_r["csa2_sparse_attn_decode_reuse"][1] == 15 and per_r["csa2_sparse_attn_decode_append"][1] == 4
+    assert per_r["csa2_index_reindex_settled"][1] == 4 and "csa2_index_reindex" not in per_r
+    assert per_r["csa2_sparse_attn_decode_reuse"][0] == 15 * per["csa2_sparse_attn_decode_append"][0] // 19
+    assert sum(b for b, _ in per_r.values()) == bench.step_bytes(wl)
     op_ms = {"csa2_quantize_append": (0.005, 1), "csa2_index_full": (0.4, 1),
              "csa2_index_reindex": (0.4, 4), "csa2_sparse_attn_decode": (0.03, 1),
              "csa2_sparse_attn_decode_append": (0.665, 19)}
     ms_step = sum(t for t, _ in op_ms.values())
-    ops = bench.op_rooflines(wl, plan, op_ms, ms_step=ms_step)
+    ops = bench.op_rooflines(wl, plan, op_ms, ms_step=ms_step, reuse=False)
     assert abs(sum(e["share_of_step"] for e in ops.values()) - 1.0) < 1e-12
     f = ops["csa2_index_full"]
     assert f["launches_per_step"] == 1 and f["bound"] == "hbm"
@@ -167,7 +175,7 @@ def test_prefill_and_rope_op_rooflines():
     dec = WORKLOADS["decode_128k"]
     plan = plan_layers([g.schedule for g in dec.groups])
     r = bench.op_rooflines(dec, plan, {"csa2_sparse_attn_decode_append_rope": (19 * 0.033, 19)}, 1.12,
-                           rope=True)
+                           rope=True, reuse=False)
     e = r["csa2_sparse_attn_decode_append_rope"]
     assert e["algorithmic_bytes_per_launch"] == (bench.op_bytes(dec)["attn"] + 64 * (1024 + 516)
                                                  + 64 * ROPE_PAIRS * 8)
