@@ -92,15 +92,15 @@ def attn_flops(wl) -> int:
 # scaled to the batch, only for decode workloads and while the code is unchanged.
 NCU_TRAFFIC = {
     # attention: attn_kernel<0, 2> (2 CTAs per query) at batch 40, one launch
-    "csa2_sparse_attn_decode": ([(13_244_160, 40)], ("csa2_attn.cu",), "0533d212713e8e2b"),
-    "csa2_sparse_attn_decode_append": ([(13_244_160, 40)], ("csa2_attn.cu",), "0533d212713e8e2b"),
-    "csa2_sparse_attn_decode_reuse": ([(13_244_160, 40)], ("csa2_attn.cu",), "0533d212713e8e2b"),
+    "csa2_sparse_attn_decode": ([(13_241_344, 40)], ("csa2_attn.cu",), "2fc388cfd0f29445"),
+    "csa2_sparse_attn_decode_append": ([(13_241_344, 40)], ("csa2_attn.cu",), "2fc388cfd0f29445"),
+    "csa2_sparse_attn_decode_reuse": ([(13_241_344, 40)], ("csa2_attn.cu",), "2fc388cfd0f29445"),
     # Full: index_scan_kernel + select_full_kernel at batch 8
-    "csa2_index_full": ([(138_471_424 + 4_538_624, 8), (1_134_336, 8)], ("csa2_index.cu",),
-                        "2c19ef68d42489bf"),
+    "csa2_index_full": ([(138_469_120 + 4_143_872, 8), (1_132_288, 8)], ("csa2_index.cu",),
+                        "516e9707365416eb"),
     # Reindex: reindex_score_kernel + select_reindex_kernel at batch 8
-    "csa2_index_reindex": ([(18_609_408, 8), (553_472, 8)], ("csa2_index.cu",), "2c19ef68d42489bf"),
-    "csa2_index_reindex_settled": ([(18_609_408, 8), (553_472, 8)], ("csa2_index.cu",), "2c19ef68d42489bf"),
+    "csa2_index_reindex": ([(18_610_432, 8), (552_960, 8)], ("csa2_index.cu",), "516e9707365416eb"),
+    "csa2_index_reindex_settled": ([(18_610_432, 8), (552_960, 8)], ("csa2_index.cu",), "516e9707365416eb"),
 }
 
 

@@ -502,6 +502,10 @@ attn_kernel(AttnArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem &s = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // Settled: the next launch may start at once; it computes from its queries only after
+    // this kernel has completed, and this kernel completes only after its MMA warp has
+    // waited for the previous launch (below), so the layers' compute stays in order.
+    if (a.settled) grid_dep_launch();
     const uint32_t rank = cluster_rank();
     const int qi = blockIdx.x / CS;
     const int b = qi / a.Tq;
@@ -585,11 +589,18 @@ attn_kernel(AttnArgs a) {
                 make_uint4(h[0], h[1], h[2], h[3]);
         }
     }
-    // everything below may read what the previous kernel of the stream wrote (the Top-K),
-    // unless the caller settled every input two or more launches earlier: then the wait
-    // moves to just before the next launch is let go (each kernel of the library waits
-    // before it does that, so whatever was written two launches back is complete here)
-    if (!a.settled) grid_dep_wait();
+    // Everything below may read what the previous kernel of the stream wrote (the
+    // Top-K), unless the caller settled every input before the most recent ordinary
+    // launch (an ordinary launch waits for its predecessor before it lets the next one
+    // start, so whatever was written before it is complete here).  Settled, the set-up
+    // and the first tiles' gathers and dequantisation run at once and the wait moves to
+    // the MMA warp, before the first score MMA: nothing computed from this layer's
+    // queries starts before the previous launch has completed (in the model a layer's
+    // queries come from the previous layer's output).
+    if (!a.settled) {
+        grid_dep_wait();
+        grid_dep_launch();   // the previous launch has completed: the next may start
+    }
     const int *tk = a.topk + (int64_t)qi * a.top_k;
     const int e_id0 = (int)threadIdx.x < a.top_k ? tk[threadIdx.x] : -1;
     const int e_id1 = (int)threadIdx.x + kThreads < a.top_k ? tk[threadIdx.x + kThreads] : -1;
@@ -681,6 +692,7 @@ attn_kernel(AttnArgs a) {
             const uint32_t idesc_o = (1u << 4) | (1u << 15) | (1u << 16) | ((uint32_t)(kHeads >> 3) << 17) |
                                      ((uint32_t)(kCh >> 4) << 24);
             const uint64_t qd_desc = sw128_desc(smem_u32(s.q), 16, 1024);
+            if (a.settled) grid_dep_wait();
             for (int h = 0; ok && h <= nt; ++h) {
                 if (h < nt) {
                     const int bs = h & 1;
@@ -1000,8 +1012,7 @@ attn_kernel(AttnArgs a) {
         mbar_expect_tx(&s.xfer[1], (CS - 1) * kPiece);
     }
     cluster_sync();                        // stats exchanged; every CTA's tiles are free
-    if (a.settled) grid_dep_wait();
-    grid_dep_launch();
+    if (a.settled && nt == 0) grid_dep_wait();   // (a CTA without keys did not wait above)
     if (threadIdx.x < kHeads) {
         const int h = threadIdx.x;
         float m_all = -INFINITY;

@@ -239,9 +239,10 @@ reindex_score_kernel(IndexArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     ScoreSmem<D, HI, R> &s = *reinterpret_cast<ScoreSmem<D, HI, R> *>(smem_raw);
     __shared__ int64_t row_of[kTileRows];   // cache row of each candidate, -1: not scored
-    // settled inputs (written two or more launches back): the wait moves to just before
-    // the next launch is let go (the scores go to a workspace the previous launch does
-    // not read)
+    // Settled inputs (written before the most recent ordinary launch): the pool ids are
+    // resolved and the rows staged at once, and the wait moves to just before the scoring,
+    // so that nothing is computed from this layer's query before the previous launch has
+    // completed (the scores go to a workspace the previous launch does not read).
     if (!a.settled) grid_dep_wait();
     const int qi = blockIdx.y;
     const int b = qi / a.Tq;
@@ -274,10 +275,10 @@ reindex_score_kernel(IndexArgs a) {
     load_query<D, HI>(s, a.q_idx + (int64_t)qi * HI * D, a.w + (int64_t)qi * HI);
     cp_async_wait_all();
     __syncthreads();
+    if (a.settled) grid_dep_wait();
 
     float sc[R];
     score_rows<D, HI, R>(s, sc);
-    if (a.settled) grid_dep_wait();
     grid_dep_launch();
     float *out = a.scores + (int64_t)qi * a.score_stride + (int64_t)slot0 * 8;
     float *bm = a.bmax + (int64_t)qi * a.bmax_stride + slot0;

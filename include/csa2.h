@@ -350,13 +350,14 @@ CSA2_API csa2_status csa2_index_reindex(const csa2_global_kv *kv, const void *q_
                                size_t ws_bytes, int32_t *dev_err, csa2_stream_t stream);
 
 /*
- * csa2_index_reindex whose scoring overlaps the previous launch on the stream (same
- * arguments, workspace and results, bit for bit).  Precondition (the caller's): no
- * input (kv, q_idx_bf16, w, q_pos, pool) is written, and the workspace not read, by the
- * launch that immediately precedes it on `stream` (a Reindex layer: its pool comes from
- * the Full layer, whose attention, at least, launched in between).  The scoring kernel
- * then reads its inputs before it waits for the previous launch (as
- * csa2_sparse_attn_decode_reuse does); the selection waits for the scoring as usual.
+ * csa2_index_reindex whose loads overlap the previous launch on the stream (same
+ * arguments, workspace and results, bit for bit).  Precondition (the caller's), as for
+ * csa2_sparse_attn_decode_reuse: no input (kv, q_idx_bf16, w, q_pos, pool) is written,
+ * and the workspace not read, by the most recent ordinary launch of the library on
+ * `stream` or by any launch since (a Reindex layer: its pool comes from the Full layer,
+ * whose attention, at least, came in between).  The scoring kernel resolves the pool
+ * and stages its rows without waiting for the previous launch, and waits for it before
+ * it scores; the selection waits for the scoring as usual.
  */
 CSA2_API csa2_status csa2_index_reindex_settled(const csa2_global_kv *kv, const void *q_idx_bf16,
                                                 const float *w, const int32_t *q_pos, int32_t Tq,
@@ -428,12 +429,17 @@ CSA2_API csa2_status csa2_sparse_attn_decode_append_rope(
  * for bit.
  *   Precondition (the caller's): no input of the call (kv, swa, q_bf16, q_pos, topk,
  *   swa_bf16, rope) is written, and no output (out, lse, the layer's ring row) read, by
- *   the launch that immediately precedes it on `stream` (a Reuse layer: its topk comes
- *   from a Full or Reindex layer whose own attention launched in between).  The kernel then reads them before it waits for the previous
- *   launch (every launch of the library waits for its predecessor before it lets the
- *   next one start, so whatever was written two launches back is complete), and waits
- *   before it lets the next launch start.  A kernel outside the library that lets its
- *   dependents start early (programmatic dependent launch) must not write the inputs.
+ *   the most recent ordinary launch of the library on `stream` (any launch but this call
+ *   and csa2_index_reindex_settled) or by any launch since (a Reuse layer: its topk comes
+ *   from a Full or Reindex selection, and that layer's own attention, an ordinary
+ *   launch, came in between).  The kernel lets the next launch start at once and reads
+ *   its inputs, compacts the selection, and gathers and dequantises its first keys
+ *   without waiting for the previous launch (an ordinary launch waits for its
+ *   predecessor before it lets the next one start, so whatever was written before it is
+ *   complete); its first score MMA waits for the previous launch to complete, so that
+ *   the layers' compute stays in stream order.  A kernel outside the library that lets
+ *   its dependents start early (programmatic dependent launch) must not write the
+ *   inputs.
  */
 CSA2_API csa2_status csa2_sparse_attn_decode_reuse(const csa2_global_kv *kv, const csa2_swa *swa,
                                                    const void *swa_bf16, const void *q_bf16,
