@@ -323,7 +323,7 @@ constexpr int kSelFlatDirect = 16384;
 template <int kCap>
 struct SelSmemT {
     uint32_t hist[1 << kSelDigit];
-    int wa[kSelWarps], wb[kSelWarps];
+    int wa[kSelWarps], wb[kSelWarps], wc[kSelWarps];
     uint32_t wmin[kSelWarps], wmax[kSelWarps];
     int bcast[4];
     alignas(16) int pool[CSA2_POOL_MAX];
@@ -332,8 +332,6 @@ struct SelSmemT {
 };
 using SelSmem = SelSmemT<kSelStageMax>;
 
-// Exclusive scans (in warp order) of s.wa and s.wb; totals in s.bcast[0], s.bcast[1].
-// Call with every warp's entry written; ends with a barrier.
 // dst[0..n) = the raw 32-bit words src[0..n), copied into shared memory with 16-byte
 // cp.async (src 16-byte aligned, as every workspace row is) so that no register or
 // dependent round trip is involved; the caller converts in place after a barrier.
@@ -346,27 +344,20 @@ __device__ __forceinline__ void stage_raw(uint32_t *dst, const void *src, int n)
     cp_async_wait_all();
 }
 
-template <class S>
-__device__ __forceinline__ void sel_scan_warps(S &s) {
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        const int a = s.wa[lane], b = s.wb[lane];
-        int ia = a, ib = b;
+// Inclusive scan over the warp's lanes.
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int ta = __shfl_up_sync(0xFFFFFFFFu, ia, o), tb = __shfl_up_sync(0xFFFFFFFFu, ib, o);
-            if (lane >= o) { ia += ta; ib += tb; }
-        }
-        s.wa[lane] = ia - a;
-        s.wb[lane] = ib - b;
-        if (lane == 31) { s.bcast[0] = ia; s.bcast[1] = ib; }
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xFFFFFFFFu, v, o);
+        if (lane >= o) v += t;
     }
-    __syncthreads();
+    return v;
 }
 
 // The bin (of nbins, visited from the top) holding the rem-th largest counted key:
-// bin, number of counted keys in higher bins, population of the bin.
+// bin, number of counted keys in higher bins, population of the bin.  Each thread reads
+// its bins and zeroes them for the next pass.  Every warp derives its own prefix from
+// the warps' totals (no broadcast step): two barriers.
 template <class S>
 __device__ __forceinline__ void sel_find_bin(S &s, int nbins, int rem, int &bin, int &above,
                                              int &cnt) {
@@ -376,40 +367,41 @@ __device__ __forceinline__ void sel_find_bin(S &s, int nbins, int rem, int &bin,
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
         const int bb = nbins - 1 - (threadIdx.x * per + j);
-        if (j < per && bb >= 0) c[j] = (int)s.hist[bb];
+        if (j < per && bb >= 0) {
+            c[j] = (int)s.hist[bb];
+            s.hist[bb] = 0u;
+        }
         sum += c[j];
     }
-    int incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += t;
-    }
+    const int incl = warp_incl_scan(sum, lane);
     if (lane == 31) s.wa[warp] = incl;
-    s.wb[warp] = 0;
-    sel_scan_warps(s);
-    int run = s.wa[warp] + incl - sum;
+    __syncthreads();
+    const int wt = s.wa[lane];
+    const int wprefix = __shfl_sync(0xFFFFFFFFu, warp_incl_scan(wt, lane) - wt, warp);
+    int run = wprefix + incl - sum;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
         if (c[j] > 0 && run < rem && rem <= run + c[j]) {
-            s.bcast[2] = nbins - 1 - (threadIdx.x * per + j);
-            s.bcast[3] = run;
-            s.wmin[0] = (uint32_t)c[j];
+            s.bcast[0] = nbins - 1 - (threadIdx.x * per + j);
+            s.bcast[1] = run;
+            s.bcast[2] = c[j];
         }
         run += c[j];
     }
     __syncthreads();
-    bin = s.bcast[2];
-    above = s.bcast[3];
-    cnt = (int)s.wmin[0];
-    __syncthreads();
+    bin = s.bcast[0];
+    above = s.bcast[1];
+    cnt = s.bcast[2];
 }
 
 // Top-k of n candidates (keys from key_at, 0 = not a candidate) -> ascending ids in
-// out[0..cnt), cnt = min(k, #valid) returned.
+// out[0..cnt), cnt = min(k, #valid) returned.  Block barriers: one for the statistics,
+// three per radix pass, two for the compaction.
 template <class KeyAt, class IdAt, class S>
 __device__ int block_topk(KeyAt key_at, IdAt id_at, int n, int k, int *out, S &s) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // the first radix pass's bins start at zero (each pass's readers zero them for the next)
+    for (int i = threadIdx.x; i < (1 << kSelDigit); i += kSelThreads) s.hist[i] = 0u;
     // valid count, smallest and largest valid key
     int nv = 0;
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
@@ -425,28 +417,20 @@ __device__ int block_topk(KeyAt key_at, IdAt id_at, int n, int k, int *out, S &s
     kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
     kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
     if (lane == 0) {
-        s.wa[warp] = nv;
+        s.wc[warp] = nv;
         s.wmin[warp] = kmin;
         s.wmax[warp] = kmax;
     }
     __syncthreads();
-    if (warp == 0) {
-        const int v = __reduce_add_sync(0xFFFFFFFFu, s.wa[lane]);
-        const uint32_t mn = __reduce_min_sync(0xFFFFFFFFu, s.wmin[lane]);
-        const uint32_t mx = __reduce_max_sync(0xFFFFFFFFu, s.wmax[lane]);
-        if (lane == 0) {
-            s.bcast[0] = v;
-            s.bcast[1] = (int)mn;
-            s.bcast[2] = (int)mx;
-        }
-    }
-    __syncthreads();
-    const int nvalid = s.bcast[0];
-    kmin = (uint32_t)s.bcast[1];
-    kmax = (uint32_t)s.bcast[2];
-    __syncthreads();
+    // every warp reduces the warps' figures itself
+    const int nvalid = __reduce_add_sync(0xFFFFFFFFu, s.wc[lane]);
+    kmin = __reduce_min_sync(0xFFFFFFFFu, s.wmin[lane]);
+    kmax = __reduce_max_sync(0xFFFFFFFFu, s.wmax[lane]);
     const int kk = min(k, nvalid);
-    if (kk == 0) return 0;
+    if (kk == 0) {
+        __syncthreads();   // every warp has read the figures before the next selection writes them
+        return 0;
+    }
 
     // ---- threshold ----
     uint32_t T, mask;
@@ -466,8 +450,6 @@ __device__ int block_topk(KeyAt key_at, IdAt id_at, int n, int k, int *out, S &s
         int rem = kk, lo_bit = hi + 1;
         while (lo_bit > 0) {
             const int bits = min(kSelDigit, lo_bit), shift = lo_bit - bits, nbins = 1 << bits;
-            for (int i = threadIdx.x; i < nbins; i += kSelThreads) s.hist[i] = 0u;
-            __syncthreads();
             for (int i = threadIdx.x; i < n; i += kSelThreads) {
                 const uint32_t key = key_at(i);
                 if (key != 0u && (key & pmask) == prefix)
@@ -502,9 +484,12 @@ __device__ int block_topk(KeyAt key_at, IdAt id_at, int n, int k, int *out, S &s
         s.wa[warp] = ngt;
         s.wb[warp] = neq;
     }
-    sel_scan_warps(s);
-    int gt_run = s.wa[warp], eq_run = s.wb[warp];
-    const int total = s.bcast[0] + min(take, s.bcast[1]);
+    __syncthreads();
+    // this warp's exclusive prefixes and the totals, from the warps' counts
+    const int a_w = s.wa[lane], b_w = s.wb[lane];
+    const int ia = warp_incl_scan(a_w, lane), ib = warp_incl_scan(b_w, lane);
+    int gt_run = __shfl_sync(0xFFFFFFFFu, ia - a_w, warp), eq_run = __shfl_sync(0xFFFFFFFFu, ib - b_w, warp);
+    const int total = __shfl_sync(0xFFFFFFFFu, ia, 31) + min(take, __shfl_sync(0xFFFFFFFFu, ib, 31));
     const uint32_t lt = (1u << lane) - 1u;
     for (int i0 = lo; i0 < hi_i; i0 += 32) {
         const int i = i0 + lane;
