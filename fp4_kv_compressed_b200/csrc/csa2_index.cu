@@ -544,6 +544,10 @@ select_full_kernel(IndexArgs a) {
     __shared__ int sel_out[CSA2_TOPK_MAX];
     __shared__ int sub[CSA2_TOPK_MAX];
     grid_dep_wait();
+    // The next launch (the layer's attention) may start now: its CTAs take the SMs this
+    // selection leaves free and stage their queries; they read the Top-K only after
+    // this kernel has completed.
+    grid_dep_launch();
     const int qi = blockIdx.x;
     int64_t N64 = max64(0, visible_entries(a.q_pos[qi], a.ratio) - a.entry_lo);
     N64 = min64(min64(N64, a.n_max), a.cap);
@@ -647,7 +651,6 @@ select_full_kernel(IndexArgs a) {
         cnt = block_topk(key, id, N, a.top_k, sel_out, s);
     }
     __syncthreads();
-    grid_dep_launch();
     if (a.topk_keys_out) {
         // slice form: the selected entries' candidate keys, global ids
         uint64_t *tk = a.topk_keys_out + (int64_t)qi * a.top_k;
@@ -673,6 +676,7 @@ select_reindex_kernel(IndexArgs a) {
     __shared__ int sel_out[CSA2_TOPK_MAX];
     __shared__ int sub[CSA2_TOPK_MAX];
     grid_dep_wait();
+    grid_dep_launch();   // as in select_full_kernel: the layer's attention may start
     const int qi = blockIdx.x;
     const int64_t N = min64(visible_entries(a.q_pos[qi], a.ratio), a.cap);
     const int32_t *pool = a.pool + (int64_t)qi * a.pool_blocks;
@@ -705,7 +709,6 @@ select_reindex_kernel(IndexArgs a) {
     auto id = [&](int i) -> int { return s.pool[sub[i >> 3]] * 8 + (i & 7); };
     const int cnt = block_topk(key, id, 8 * ns, a.top_k, sel_out, s);
     __syncthreads();
-    grid_dep_launch();
     int32_t *topk = a.topk_out + (int64_t)qi * a.top_k;
     for (int i = threadIdx.x; i < a.top_k; i += blockDim.x) topk[i] = i < cnt ? sel_out[i] : -1;
     if (threadIdx.x == 0) a.topk_count[qi] = cnt;
