@@ -92,15 +92,15 @@ def attn_flops(wl) -> int:
 # scaled to the batch, only for decode workloads and while the code is unchanged.
 NCU_TRAFFIC = {
     # attention: attn_kernel<0, 2> (2 CTAs per query) at batch 40, one launch
-    "csa2_sparse_attn_decode": ([(13_241_344, 40)], ("csa2_attn.cu",), "2fc388cfd0f29445"),
-    "csa2_sparse_attn_decode_append": ([(13_241_344, 40)], ("csa2_attn.cu",), "2fc388cfd0f29445"),
-    "csa2_sparse_attn_decode_reuse": ([(13_241_344, 40)], ("csa2_attn.cu",), "2fc388cfd0f29445"),
+    "csa2_sparse_attn_decode": ([(13_242_112, 40)], ("csa2_attn.cu",), "2fc388cfd0f29445"),
+    "csa2_sparse_attn_decode_append": ([(13_242_112, 40)], ("csa2_attn.cu",), "2fc388cfd0f29445"),
+    "csa2_sparse_attn_decode_reuse": ([(13_242_112, 40)], ("csa2_attn.cu",), "2fc388cfd0f29445"),
     # Full: index_scan_kernel + select_full_kernel at batch 8
-    "csa2_index_full": ([(138_469_120 + 4_143_872, 8), (1_132_288, 8)], ("csa2_index.cu",),
-                        "516e9707365416eb"),
+    "csa2_index_full": ([(138_471_936 + 4_568_064, 8), (1_127_680, 8)], ("csa2_index.cu",),
+                        "c796ebf0ae6d4c2b"),
     # Reindex: reindex_score_kernel + select_reindex_kernel at batch 8
-    "csa2_index_reindex": ([(18_610_432, 8), (552_960, 8)], ("csa2_index.cu",), "516e9707365416eb"),
-    "csa2_index_reindex_settled": ([(18_610_432, 8), (552_960, 8)], ("csa2_index.cu",), "516e9707365416eb"),
+    "csa2_index_reindex": ([(18_616_832, 8), (542_208, 8)], ("csa2_index.cu",), "c796ebf0ae6d4c2b"),
+    "csa2_index_reindex_settled": ([(18_616_832, 8), (542_208, 8)], ("csa2_index.cu",), "c796ebf0ae6d4c2b"),
 }
 
 
