@@ -136,17 +136,18 @@ def test_attention_running_max_moves_every_tile(pkg, orc, B, top_k):
     _assert_close(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref)
 
 
-@pytest.mark.parametrize("name", ["decode_128k", "decode_1m"])
-def test_reuse_launch_matches_ordinary_calls(pkg, name):
-    """Reuse layers launched with csa2_sparse_attn_decode_reuse (inputs read before the
-    dependency wait, the launch overlapping the previous one) give the same outputs and
-    lse on every layer, bit for bit, as the ordinary calls: whole decode stacks, so that
-    every Reuse layer follows another layer's launch on the stream."""
+@pytest.mark.parametrize("name,rope", [("decode_128k", False), ("decode_1m", False), ("decode_128k", True)])
+def test_reuse_launch_matches_ordinary_calls(pkg, name, rope):
+    """Reuse layers launched with csa2_sparse_attn_decode_reuse and Reindex layers with
+    csa2_index_reindex_settled (loads before the wait for the previous launch) give the
+    same outputs and lse on every layer, bit for bit, as the ordinary calls: whole decode
+    stacks, so that every such launch follows another layer's launch on the stream; with
+    RoPE, the fused append's rotation goes through the same call."""
     import csa2_harness
     wl = small_variant(WORKLOADS[name], B=4, ctx=6000)
     res = []
     for reuse in (False, True):
-        dw = csa2_harness.DeviceWorkload(wl)
+        dw = csa2_harness.DeviceWorkload(wl, rope=rope)
         dw.stack.reuse_launch = reuse
         st = torch.cuda.Stream()      # a real stream, where launches may overlap
         st.wait_stream(torch.cuda.current_stream())
