@@ -92,9 +92,9 @@ def attn_flops(wl) -> int:
 # scaled to the batch, only for decode workloads and while the code is unchanged.
 NCU_TRAFFIC = {
     # attention: attn_kernel<0, 2> (2 CTAs per query) at batch 40, one launch
-    "csa2_sparse_attn_decode": ([(13_242_112, 40)], ("csa2_attn.cu",), "2fc388cfd0f29445"),
-    "csa2_sparse_attn_decode_append": ([(13_242_112, 40)], ("csa2_attn.cu",), "2fc388cfd0f29445"),
-    "csa2_sparse_attn_decode_reuse": ([(13_242_112, 40)], ("csa2_attn.cu",), "2fc388cfd0f29445"),
+    "csa2_sparse_attn_decode": ([(13_242_112, 40)], ("csa2_attn.cu",), "cf0d443258f3fd02"),
+    "csa2_sparse_attn_decode_append": ([(13_242_112, 40)], ("csa2_attn.cu",), "cf0d443258f3fd02"),
+    "csa2_sparse_attn_decode_reuse": ([(13_242_112, 40)], ("csa2_attn.cu",), "cf0d443258f3fd02"),
     # Full: index_scan_kernel + select_full_kernel at batch 8
     "csa2_index_full": ([(138_471_936 + 4_568_064, 8), (1_127_680, 8)], ("csa2_index.cu",),
                         "c796ebf0ae6d4c2b"),

@@ -311,11 +311,6 @@ __device__ __forceinline__ uint32_t peer_addr(const void *local, uint32_t rank) 
 __device__ __forceinline__ void st_peer(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
-__device__ __forceinline__ void st_peer4(uint32_t addr, float a, float b, float c, float d) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c),
-                 "f"(d)
-                 : "memory");
-}
 
 // Byte offset of (row, 16-byte chunk c of a 128-byte row) in a 128B-swizzled block.
 __device__ __forceinline__ uint32_t swz(int row, int c) {
