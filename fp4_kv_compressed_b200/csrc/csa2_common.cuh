@@ -92,11 +92,6 @@ __device__ __forceinline__ uint32_t score_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ float key_to_score(uint32_t k) {
-    uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
-    return __uint_as_float(u);
-}
-
 __device__ __forceinline__ void unpack_bf16x8(uint4 v, float *x) {
     uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
