@@ -242,3 +242,55 @@ def test_ratio2_earliest_positions(harness, orc):
     topk, cnt, _ = _index_case(pkg, orc, rows, 2, [0, 1, 2, 3], 0, 16)
     assert cnt[:, 0].tolist() == [0, 1, 1, 2]
     assert (topk[0, 0] == -1).all() and (topk[3, 0, 2:] == -1).all()
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_reindex_many_pool_tiles(harness, orc, paged):
+    """24 queries x 128 pool tiles of 128 positions: more scoring CTAs than the SMs hold
+    at once.  The query positions are ragged (some pool blocks only partly visible) and
+    each pool is a random set of 2048 visible blocks, the last one included; Top-K and
+    counts bit-exact against the oracle, on the contiguous and on a paged layout with
+    shuffled pages."""
+    import fp4_kv_compressed_b200 as pkg
+    import synth
+    B, cap, d, H_I, P, K, page = 24, 20480, 128, 4, 2048, 512, 256
+    rng = np.random.default_rng(81)
+    codes = rng.integers(0, 256, size=(B, cap, d), dtype=np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x3C                  # E4M3 NaN codes -> 1.5
+    sigma = rng.uniform(0.01, 2.0, size=(B, cap)).astype(np.float32)
+    q_pos = np.array([cap - 1 - 13 * b - (b % 3) for b in range(B)], np.int32)
+    pool = np.zeros((B, 1, P), np.int32)
+    for b in range(B):
+        nb = (int(q_pos[b]) + 8) // 8                     # blocks with a visible position
+        blocks = rng.choice(nb - 1, size=P - 1, replace=False)
+        pool[b, 0] = np.sort(np.append(blocks, nb - 1))   # the last, partly visible block too
+    q = torch.stack([synth.rows_normal_bf16(82, "qi", b, 0, H_I, d) for b in range(B)]).view(B, 1, H_I, d)
+    w = torch.stack([synth.rows_uniform_f32(82, "w", b, 0, 1, H_I) for b in range(B)]).view(B, 1, H_I)
+    if paged:
+        max_pages = cap // page
+        n_pages = B * max_pages + 5
+        perm = torch.randperm(n_pages, generator=torch.Generator().manual_seed(83)).to(torch.int32)
+        table = perm[:B * max_pages].view(B, max_pages).contiguous()
+        kv = pkg.PagedKV(B, max_pages, page, n_pages, d, 1, table, "cuda")
+        for b in range(B):
+            r = kv.rows_of(b, cap)
+            kv.idx_codes[r] = torch.from_numpy(codes[b]).cuda()
+            kv.idx_scale[r] = torch.from_numpy(sigma[b]).cuda()
+        call = pkg.csa2_index_reindex_paged
+    else:
+        kv = pkg.GlobalKV(B, cap, d, 1, "cuda")
+        kv.idx_codes.copy_(torch.from_numpy(codes))
+        kv.idx_scale.copy_(torch.from_numpy(sigma))
+        call = pkg.csa2_index_reindex
+    topk = torch.full((B, 1, K), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(B, 1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(pkg.csa2_workspace_size(pkg.CSA2_OP_INDEX_REINDEX, B, 1, 0, 0, K, P),
+                     dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    call(kv.struct, q.cuda(), w.cuda(), torch.from_numpy(q_pos).view(B, 1).cuda(), 1, H_I,
+         torch.from_numpy(pool).cuda(), P, K, topk, cnt, ws, err)
+    torch.cuda.synchronize()
+    assert pkg.csa2_read_device_error(err) == 0
+    t_ref, c_ref = orc.index_reindex(codes, sigma, 1, q, w.numpy(), q_pos.reshape(B, 1), pool, K)
+    assert np.array_equal(cnt.cpu().numpy(), c_ref)
+    assert np.array_equal(topk.cpu().numpy(), t_ref)
