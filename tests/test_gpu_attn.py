@@ -101,13 +101,14 @@ def test_attention_edges(pkg, orc):
     assert bits & pkg.DEVERR_INDEX
 
 
-@pytest.mark.parametrize("B,top_k", [(1, 384), (1, 512), (38, 512)])
+@pytest.mark.parametrize("B,top_k", [(1, 384), (1, 512), (12, 512), (38, 512)])
 def test_attention_running_max_moves_every_tile(pkg, orc, B, top_k):
     """Entry e is c_e times head 0 of the query, c_e growing along the key order, so the
     logits of every later 64-key tile exceed the running max by more than 8 (log2 units):
     the max moves and O is rescaled on every tile, by each worker set in turn (after the
-    other set's output MMAs of the previous tile).  B = 1: 4 CTAs per query, 2 or 3 tiles
-    each; B = 38: 2 CTAs per query, 5 tiles each.  Within the tolerance of the oracle."""
+    other set's output MMAs of the previous tile).  B = 1 and 12: 4 CTAs per query, 2 or
+    3 tiles each; B = 38: 2 CTAs per query, 5 tiles each.  Within the tolerance of the
+    oracle."""
     H, cap, W = 64, 700, 128
     q_pos = torch.full((B, 1), 699, dtype=torch.int32)
     q = torch.stack([synth.rows_normal_bf16(9, "q", b, 0, H, 512, stride=synth.Q_STRIDE)
