@@ -95,6 +95,24 @@ def test_validation_rejects_before_launch(pkg):
     assert lib.csa2_sparse_attn_decode_append(C.byref(kv), C.byref(swa), C.c_void_p(4100), qbuf,
                                               qbuf, 1, 64, qbuf, 8, 128, C.c_float(0.04), qbuf,
                                               qbuf, None, 0, None, None) == 1
+    # the overlapping forms take the same checks: the settled Reindex (bad d_idx), the
+    # Reuse attention (H not a multiple of 16; with the fused append: decode only, needs
+    # the ring and a 16-byte aligned row; RoPE only with the append)
+    assert lib.csa2_index_reindex_settled(C.byref(kv2), qbuf, qbuf, qbuf, 1, 4, qbuf, 64, 64, qbuf,
+                                          qbuf, qbuf, 1 << 20, None, None) == 4
+    assert lib.csa2_sparse_attn_decode_reuse(C.byref(kv), C.byref(swa), None, qbuf, qbuf, 1, 24, qbuf,
+                                             8, 128, C.c_float(0.04), None, qbuf, qbuf, None, None) == 4
+    assert lib.csa2_sparse_attn_decode_reuse(C.byref(kv), C.byref(swa), qbuf, qbuf, qbuf, 2, 64, qbuf,
+                                             8, 128, C.c_float(0.04), None, qbuf, qbuf, None, None) == 4
+    assert lib.csa2_sparse_attn_decode_reuse(C.byref(kv), None, qbuf, qbuf, qbuf, 1, 64, qbuf,
+                                             8, 128, C.c_float(0.04), None, qbuf, qbuf, None, None) == 1
+    assert lib.csa2_sparse_attn_decode_reuse(C.byref(kv), C.byref(swa), C.c_void_p(4100), qbuf, qbuf, 1,
+                                             64, qbuf, 8, 128, C.c_float(0.04), None, qbuf, qbuf, None,
+                                             None) == 1
+    rope_ok = pkg.CSA2Rope(4096, 8, 0, 4)
+    assert lib.csa2_sparse_attn_decode_reuse(C.byref(kv), C.byref(swa), None, qbuf, qbuf, 1, 64, qbuf,
+                                             8, 128, C.c_float(0.04), C.byref(rope_ok), qbuf, qbuf, None,
+                                             None) == 1
     # RoPE descriptors: null table, odd start, range past channel 511, no pairs, no rows,
     # misaligned table -- each rejected before any launch, in both _rope calls
     for bad in [(0, 8, 0, 4), (4096, 8, 3, 4), (4096, 8, 500, 8), (4096, 8, 0, 0),
