@@ -641,6 +641,153 @@ def run_ours(args, rank, world, local_rank):
     return line, wl
 
 
+def run_cp(args) -> dict:
+    """Context parallel (one long request's entries split over shards), its S shards
+    emulated in turn on one GPU: one decode step's Full layer and attention of the
+    workload's hierarchical (decoder) group.  Device times (CUDA events around a CUDA
+    graph of each call, median of --steps replays after --warmup) of each shard's slice
+    scan with its local selections, of the merge, of each shard's partial attention and
+    of the combine, beside the unsplit csa2_index_full and csa2_sparse_attn_decode on the
+    same cache.  The two all-gathers between the steps need several GPUs and are not
+    run; their bytes per step are reported."""
+    import statistics
+    import torch
+    from synth.workloads import WORKLOADS
+    import csa2_harness
+    import fp4_kv_compressed_b200 as pkg
+    from fp4_kv_compressed_b200 import _binding as bind
+    from fp4_kv_compressed_b200.context_parallel import LibraryBackend as LB, slice_bounds
+
+    S = args.cp_shards
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload]
+    if args.batch:
+        from synth.workloads import small_variant
+        wl = small_variant(wl, B=args.batch, name=f"{wl.name}_b{args.batch}")
+    dw = csa2_harness.DeviceWorkload(wl, device=dev)
+    st = dw.stack
+    dw.step()                                   # this step's entries and rows appended
+    torch.cuda.synchronize(dev)
+    lp = next(lp for lp in st.plan if lp.mode == "F" and dw.groups[lp.group].pool_blocks > 0)
+    g, L = lp.group, lp.layer
+    kv = st.kv[g]
+    inp = dw.inputs
+    B, Tq, H, H_I, K, W = wl.B, wl.Tq, wl.H, wl.H_I, wl.top_k, wl.swa_len
+    P = dw.groups[g].pool_blocks
+    N = wl.entries(g)
+    q_pos, q_idx, w, q = inp["q_pos"], inp["q_idx"][L], inp["w"][L], inp["q"][L]
+    ring = st.swa[L]
+    scale = 1 / math.sqrt(512)
+    err = st.dev_err
+    stream = torch.cuda.Stream(device=dev)
+    i32 = dict(dtype=torch.int32, device=dev)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > L2: written before every replay
+
+    def timed(fn) -> float:
+        with torch.cuda.stream(stream):
+            fn()                                # eager once (kernel attributes)
+        torch.cuda.synchronize(dev)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            fn()
+        for _ in range(max(args.warmup, 3)):
+            gr.replay()
+        torch.cuda.synchronize(dev)
+        ev = []
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                flush.zero_()
+                e0.record(stream)
+                gr.replay()
+                e1.record(stream)
+                ev.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+    # the unsplit calls
+    pool = torch.empty(B, Tq, P, **i32)
+    topk = torch.empty(B, Tq, K, **i32)
+    cnt = torch.empty(B, Tq, **i32)
+    ws = torch.empty(pkg.csa2_workspace_size(pkg.CSA2_OP_INDEX_FULL, B, Tq, N, 0, K, P), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty(B, Tq, H, 512, dtype=torch.float32, device=dev)
+    lse = torch.empty(B, Tq, H, dtype=torch.float32, device=dev)
+    t_full = timed(lambda: bind.csa2_index_full(kv.struct, q_idx, w, q_pos, Tq, H_I, N, P, K, pool, topk, cnt,
+                                                ws, err, stream))
+    t_attn = timed(lambda: bind.csa2_sparse_attn_decode(kv.struct, ring.struct, q, q_pos, Tq, H, topk, K, W,
+                                                        scale, out, lse, None, err, stream))
+    # the shards: copies of the slices of the cache
+    bounds = slice_bounds(N, S)
+    pool_lists = torch.zeros(S, B, Tq, P, dtype=torch.int64, device=dev)
+    topk_lists = torch.zeros(S, B, Tq, K, dtype=torch.int64, device=dev)
+    o_parts = torch.empty(S, B, Tq, H, 512, dtype=torch.float32, device=dev)
+    l_parts = torch.empty(S, B, Tq, H, dtype=torch.float32, device=dev)
+    t_slice, t_part, merged_ok = [], [], True
+    t_merge = t_combine = 0.0
+    shards = []
+    for r, (lo, hi) in enumerate(bounds):
+        kv_s = pkg.GlobalKV(B, max(hi - lo, 1), wl.d_I, kv.ratio, dev)
+        for src, dst in ((kv.codes, kv_s.codes), (kv.scales, kv_s.scales), (kv.idx_codes, kv_s.idx_codes),
+                         (kv.idx_scale, kv_s.idx_scale)):
+            dst[:, :hi - lo].copy_(src[:, lo:hi])
+        n_max = max(0, min(hi, (int(q_pos.max()) + 1) // kv.ratio) - lo)
+        ws_s = torch.empty(max(256, pkg.csa2_workspace_size(pkg.CSA2_OP_INDEX_FULL, B, Tq, max(n_max, 1), 0,
+                                                            K, P)), dtype=torch.uint8, device=dev)
+        shards.append((kv_s, lo, hi, n_max, ws_s))
+        t_slice.append(timed(lambda kv_s=kv_s, lo=lo, n_max=n_max, ws_s=ws_s, r=r: LB.index_full_slice(
+            kv_s, lo, q_idx, w, q_pos, Tq, H_I, n_max, P, K, pool_lists[r], topk_lists[r], ws_s, err, stream))
+            if n_max > 0 else 0.0)
+    # the merge (every shard runs the same; shard 0's local range) and each shard's part
+    gpool = torch.empty(B, Tq, P, **i32)
+    gpool_loc = torch.empty(B, Tq, P, **i32)
+    gtopk = torch.empty(B, Tq, K, **i32)
+    gcnt = torch.empty(B, Tq, **i32)
+    locs = [torch.empty(B, Tq, K, **i32) for _ in range(S)]
+    BT = B * Tq
+
+    def merge_calls(r):
+        lo, hi = bounds[r]
+        LB.index_merge(pool_lists, BT, S, P, P, lo // 8, -(-hi // 8), gpool, None, gpool_loc, stream)
+        LB.index_merge(topk_lists, BT, S, K, K, lo, hi, gtopk, gcnt, locs[r], stream)
+
+    t_merge = timed(lambda: merge_calls(0))
+    for r in range(1, S):
+        with torch.cuda.stream(stream):
+            merge_calls(r)
+    torch.cuda.synchronize(dev)
+    merged_ok = bool(torch.equal(gtopk, topk) and torch.equal(gcnt, cnt) and torch.equal(gpool, pool))
+    for r, (kv_s, lo, hi, n_max, ws_s) in enumerate(shards):
+        win = r == S - 1
+        t_part.append(timed(lambda kv_s=kv_s, r=r, win=win: LB.attention(
+            kv_s, ring if win else None, q, q_pos, Tq, H, locs[r], K, W if win else 0, scale, o_parts[r],
+            l_parts[r], err, stream)))
+    out_c = torch.empty_like(out)
+    lse_c = torch.empty_like(lse)
+    t_combine = timed(lambda: LB.combine(o_parts, l_parts, S, B * Tq * H, out_c, lse_c, stream))
+    torch.cuda.synchronize(dev)
+    if st.dev_err.item() != 0:
+        raise RuntimeError(f"device error bits {st.dev_err.item()}")
+    diff = float(((out_c - out).norm(dim=-1) / out.norm(dim=-1).clamp_min(1e-30)).max())
+    proj = max(t_slice) + t_merge + max(t_part) + t_combine
+    return {
+        "metric": "context-parallel Full layer + attention of one decode step, shards emulated on one GPU",
+        "unit": "ms", "workload": wl.name, "group": g, "layer": L, "shards": S,
+        "config": {"batch": B, "entries": N, "pool": P, "top_k": K, "heads": H, "swa": W,
+                   "slices": [list(b) for b in bounds]},
+        "unsplit_ms": {"csa2_index_full": t_full, "csa2_sparse_attn_decode": t_attn, "sum": t_full + t_attn},
+        "slice_scan_ms": t_slice, "merge_ms": t_merge, "attention_part_ms": t_part, "combine_ms": t_combine,
+        "projected_ms_per_gpu": proj,
+        "all_gather_bytes_per_step": {"candidate_keys": S * B * Tq * (P + K) * 8,
+                                      "partials": S * B * Tq * H * (512 + 1) * 4},
+        "all_gathers": "not run: one GPU",
+        "merged_equals_unsplit": merged_ok, "combined_max_row_diff_vs_unsplit": diff,
+        "l2": "flushed (256 MB written) before every replay",
+    }
+
+
 def workload_config(wl, args, world: int) -> dict:
     """The `config` of a bench line: the workload and how it is run (the same for
     both arms)."""
@@ -703,7 +850,12 @@ def main():
                     help="override the workload's batch (small cases for profiling)")
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run this many eager steps inside an NVTX range 'step' and exit (for ncu)")
+    ap.add_argument("--cp-shards", type=int, default=0,
+                    help="time the context-parallel calls with this many shards emulated on one GPU")
     args = ap.parse_args()
+    if args.cp_shards:
+        print(json.dumps(run_cp(args)), flush=True)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
