@@ -144,13 +144,39 @@ OP_KERNELS = {
     "csa2_sparse_attn_decode_reuse": "attn_kernel (Reuse layer, with the SWA append, overlapping the previous launch)",
     "csa2_sparse_attn_decode_append": "attn_kernel (with the SWA append)",
     "csa2_sparse_attn_decode_append_rope": "attn_kernel (with the RoPE + SWA append)",
+    "csa2_quantize_append_paged": "quantize_append_kernel (paged cache)",
+    "csa2_index_full_paged": "index_scan_kernel + select_full_kernel (paged cache)",
+    "csa2_index_reindex_paged": "reindex_score_kernel + select_reindex_kernel (paged cache)",
+    "csa2_sparse_attn_decode_paged": "attn_kernel (paged cache; with the SWA append in decode)",
+    "csa2_index_reindex_paged_settled": "reindex_score_kernel (paged cache, overlapping the previous launch) + "
+                                        "select_reindex_kernel",
+    "csa2_sparse_attn_decode_paged_reuse": "attn_kernel (paged cache, Reuse layer, with the SWA append, "
+                                           "overlapping the previous launch)",
 }
 
 
-def op_step_bytes(wl, plan, rope: bool = False, index_scan: str = "exact", reuse: bool = True) -> dict:
+def op_step_bytes(wl, plan, rope: bool = False, index_scan: str = "exact", reuse: bool = True,
+                  paged: bool = False) -> dict:
     """Per library call name: (algorithmic bytes per step, launches per step), walking the
     layer plan the way DecodeStack.step issues its calls (reuse: DecodeStack.reuse_launch,
-    the Reuse and Reindex layers' overlapping calls)."""
+    the Reuse and Reindex layers' overlapping calls; paged: the caches in pages, every
+    call in its _paged form, the same bytes)."""
+    if paged:
+        out = {}
+        for name, v in op_step_bytes(wl, plan, rope, index_scan, reuse).items():
+            if name == "csa2_sparse_attn_decode_reuse":
+                name = "csa2_sparse_attn_decode_paged_reuse"
+            elif name.startswith("csa2_sparse_attn_decode"):
+                name = "csa2_sparse_attn_decode_paged"
+            elif name.startswith("csa2_quantize_append"):
+                name = "csa2_quantize_append_paged"
+            elif name == "csa2_index_reindex_settled":
+                name = "csa2_index_reindex_paged_settled"
+            else:
+                name += "_paged"
+            b, n = out.get(name, (0, 0))
+            out[name] = (b + v[0], n + v[1])
+        return out
     ob = op_bytes(wl)
     fused = wl.Tq == 1 and wl.swa_len > 0          # decode: SWA append inside the attention
     first = {}
@@ -185,11 +211,11 @@ def op_step_bytes(wl, plan, rope: bool = False, index_scan: str = "exact", reuse
 
 
 def op_rooflines(wl, plan, op_ms: dict, ms_step: float, rope: bool = False,
-                 index_scan: str = "exact", reuse: bool = True) -> dict:
+                 index_scan: str = "exact", reuse: bool = True, paged: bool = False) -> dict:
     """Per library call: algorithmic bytes (and flops) per step over its measured time per
     step.  op_ms[name] = (total ms per step of the calls of that name, calls per step)."""
     pk = measured_peaks()
-    per = op_step_bytes(wl, plan, rope, index_scan, reuse)
+    per = op_step_bytes(wl, plan, rope, index_scan, reuse, paged)
     modes = [lp.mode for lp in plan]
     out = {}
     for name, (tot_ms, n) in op_ms.items():
@@ -438,7 +464,8 @@ def run_ours(args, rank, world, local_rank):
         from synth.workloads import small_variant
         wl = small_variant(wl, B=args.batch, name=f"{wl.name}_b{args.batch}")
     wl = rank_workload(wl, rank)
-    dw = csa2_harness.DeviceWorkload(wl, device=dev, index_scan=args.index_scan, rope=args.rope)
+    dw = csa2_harness.DeviceWorkload(wl, device=dev, index_scan=args.index_scan, rope=args.rope,
+                                     page_size=args.page_size)
     st = dw.stack
     inputs, dbuf, hbuf, in_bytes = pack_inputs(dw.inputs, dev)
     full_layers = [lp.layer for lp in st.plan if lp.mode == "F"]
@@ -483,7 +510,10 @@ def run_ours(args, rank, world, local_rank):
     op_names = [n for n in ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_index_full",
                             "csa2_index_full_tc", "csa2_index_reindex", "csa2_index_reindex_settled",
                             "csa2_sparse_attn_decode", "csa2_sparse_attn_decode_append",
-                            "csa2_sparse_attn_decode_append_rope", "csa2_sparse_attn_decode_reuse")
+                            "csa2_sparse_attn_decode_append_rope", "csa2_sparse_attn_decode_reuse",
+                            "csa2_quantize_append_paged", "csa2_index_full_paged", "csa2_index_reindex_paged",
+                            "csa2_sparse_attn_decode_paged", "csa2_index_reindex_paged_settled",
+                            "csa2_sparse_attn_decode_paged_reuse")
                 if hasattr(stack_mod.bind, n)]
     originals = {name: getattr(stack_mod.bind, name) for name in op_names}
     marks = []                       # (op name, event after the call)
@@ -615,7 +645,7 @@ def run_ours(args, rank, world, local_rank):
     ob = op_bytes(wl)
     g_full = st.plan[full_layers[0]].group
     ops = op_rooflines(wl, st.plan, op_ms, ops_step_ms, rope=args.rope, index_scan=args.index_scan,
-                       reuse=st.reuse_launch)
+                       reuse=st.reuse_launch, paged=st.page_size > 0)
     dominant = max(ops, key=lambda n: ops[n]["share_of_step"])
     launches = st.launches_per_step() * K
     line = {
@@ -802,6 +832,8 @@ def workload_config(wl, args, world: int) -> dict:
             "rope": ({"start": ROPE_START, "pairs": ROPE_PAIRS,
                       "rows": "main KV and SWA, rotated inside the append launches"}
                      if args.rope else None),
+            "paged": ({"page_size": args.page_size, "pages": "each group's pool, handed to the requests "
+                       "in a seeded random order"} if getattr(args, "page_size", 0) else None),
             "parallelism": f"replicas x{world} (requests sharded, no collective)",
             "l2": "inputs larger than L2: the Full scan streams "
                   f"{ob[f'index_full_g{g_full}'] / 1e9:.2f} GB per step"}
@@ -850,6 +882,8 @@ def main():
                     help="override the workload's batch (small cases for profiling)")
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run this many eager steps inside an NVTX range 'step' and exit (for ncu)")
+    ap.add_argument("--page-size", type=int, default=0,
+                    help="the caches in pages of this many entries (a power of two >= 256), shuffled")
     ap.add_argument("--cp-shards", type=int, default=0,
                     help="time the context-parallel calls with this many shards emulated on one GPU")
     args = ap.parse_args()

@@ -19,13 +19,13 @@ import torch
 
 import synth
 from fp4_kv_compressed_b200 import (DecodeStack, GroupSpec, Rope, csa2_quantize_append,
-                                    csa2_quantize_append_rope)
+                                    csa2_quantize_append_paged, csa2_quantize_append_rope)
 from synth.workloads import ROPE_PAIRS, ROPE_START, Workload
 
 
 class DeviceWorkload:
     def __init__(self, wl: Workload, device="cuda", chunk_elems: int = 1 << 25, fill=True,
-                 index_scan: str = "exact", rope: bool = False):
+                 index_scan: str = "exact", rope: bool = False, page_size: int = 0):
         self.wl = wl
         self.device = torch.device(device)
         self.rope = (Rope(synth.rope_table(wl.ctx, ROPE_PAIRS), ROPE_START, ROPE_PAIRS, device)
@@ -34,7 +34,7 @@ class DeviceWorkload:
                        for i, g in enumerate(wl.groups)]
         self.stack = DecodeStack(wl.B, wl.H, wl.H_I, wl.d_I, wl.top_k, wl.swa_len, self.groups,
                                  Tq=wl.Tq, window_cap=wl.window_cap, device=device,
-                                 index_scan=index_scan, rope=self.rope)
+                                 index_scan=index_scan, rope=self.rope, page_size=page_size)
         self.t0 = wl.first_q_pos
         self.chunk_elems = chunk_elems
         if fill:
@@ -63,7 +63,10 @@ class DeviceWorkload:
         torch.cuda.synchronize(dev)
 
     def _append(self, *args):
-        if self.rope is None:
+        if self.stack.page_size and args[0] is not None:
+            csa2_quantize_append_paged(*args, self.rope.struct if self.rope is not None else None,
+                                       self.stack.dev_err)
+        elif self.rope is None:
             csa2_quantize_append(*args, self.stack.dev_err)
         else:
             csa2_quantize_append_rope(*args, self.rope.struct, self.stack.dev_err)
@@ -104,7 +107,10 @@ class DeviceWorkload:
 
     # ---------------------------------------------------------------------------------------
     def request_state(self, b: int) -> dict:
-        """Host copies of request b's caches and every layer's outputs (after a step)."""
+        """Host copies of request b's caches and every layer's outputs (after a step);
+        contiguous caches only."""
+        if self.stack.page_size:
+            raise ValueError("request_state reads the contiguous cache layout")
         st = self.stack
         out = {"kv": [], "swa": [], "topk": {}, "count": {}, "pool": {}, "out": [], "lse": []}
         for g in st.kv:

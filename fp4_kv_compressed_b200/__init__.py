@@ -13,7 +13,8 @@ from ._binding import (CSA2_OP_INDEX_FULL, CSA2_OP_INDEX_REINDEX, CSA2_OP_SPARSE
                        csa2_index_merge, csa2_index_reindex, csa2_quantize_append_paged,
                        csa2_index_full_paged, csa2_index_reindex_paged,
                        csa2_sparse_attn_decode_paged, csa2_sparse_attn_decode_reuse,
-                       csa2_index_reindex_settled,
+                       csa2_index_reindex_settled, csa2_index_reindex_paged_settled,
+                       csa2_sparse_attn_decode_paged_reuse,
                        csa2_quantize_append, csa2_quantize_append_rope, csa2_read_device_error,
                        csa2_sparse_attn_decode, csa2_sparse_attn_decode_append,
                        csa2_sparse_attn_decode_append_rope, csa2_workspace_size, load_library)
@@ -29,7 +30,7 @@ __all__ = [
     "csa2_index_full_tc", "csa2_index_reindex", "csa2_attn_combine", "csa2_index_full_slice",
     "csa2_index_merge", "CSA2PagedKV", "csa2_quantize_append_paged", "csa2_index_full_paged",
     "csa2_index_reindex_paged", "csa2_sparse_attn_decode_paged", "csa2_sparse_attn_decode_reuse",
-    "csa2_index_reindex_settled",
+    "csa2_index_reindex_settled", "csa2_index_reindex_paged_settled", "csa2_sparse_attn_decode_paged_reuse",
     "PagedKV", "csa2_quantize_append",
     "csa2_quantize_append_rope", "csa2_read_device_error", "csa2_sparse_attn_decode",
     "csa2_sparse_attn_decode_append", "csa2_sparse_attn_decode_append_rope",

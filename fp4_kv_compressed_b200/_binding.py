@@ -37,7 +37,8 @@ EXPORTS = ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_workspace_
            "csa2_index_full_slice", "csa2_index_merge", "csa2_attn_combine",
            "csa2_quantize_append_paged", "csa2_index_full_paged", "csa2_index_reindex_paged",
            "csa2_sparse_attn_decode_paged", "csa2_sparse_attn_decode_reuse",
-           "csa2_index_reindex_settled")
+           "csa2_index_reindex_settled", "csa2_index_reindex_paged_settled",
+           "csa2_sparse_attn_decode_paged_reuse")
 
 
 class Csa2Error(RuntimeError):
@@ -126,9 +127,12 @@ def load_library(path: str = LIB_PATH):
                                                 P, P, P, P, P]
     L.csa2_sparse_attn_decode_reuse.argtypes = L.csa2_sparse_attn_decode_paged.argtypes
     L.csa2_index_reindex_settled.argtypes = L.csa2_index_reindex.argtypes
+    L.csa2_index_reindex_paged_settled.argtypes = L.csa2_index_reindex_paged.argtypes
+    L.csa2_sparse_attn_decode_paged_reuse.argtypes = L.csa2_sparse_attn_decode_paged.argtypes
     for fn in ("csa2_quantize_append_paged", "csa2_index_full_paged", "csa2_index_reindex_paged",
                "csa2_sparse_attn_decode_paged", "csa2_sparse_attn_decode_reuse",
-               "csa2_index_reindex_settled"):
+               "csa2_index_reindex_settled", "csa2_index_reindex_paged_settled",
+               "csa2_sparse_attn_decode_paged_reuse"):
         getattr(L, fn).restype = C.c_int
     for fn in ("csa2_quantize_append", "csa2_quantize_append_rope", "csa2_index_full",
                "csa2_index_full_tc", "csa2_index_reindex", "csa2_sparse_attn_decode",
@@ -316,6 +320,31 @@ def csa2_index_reindex(kv: CSA2GlobalKV, q_idx, w, q_pos, Tq: int, H_I: int, poo
                               _ptr(pool), pool_blocks, top_k, _ptr(topk_out), _ptr(topk_count),
                               _ptr(workspace), ws_bytes, _ptr(dev_err), _stream(stream))
     _check("csa2_index_reindex", st)
+
+
+def csa2_index_reindex_paged_settled(kv: CSA2PagedKV, q_idx, w, q_pos, Tq: int, H_I: int, pool,
+                                     pool_blocks: int, top_k: int, topk_out, topk_count, workspace,
+                                     dev_err=None, stream=None):
+    """csa2_index_reindex_settled on a paged cache."""
+    L = load_library()
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = L.csa2_index_reindex_paged_settled(C.byref(kv), _ptr(q_idx), _ptr(w), _ptr(q_pos), Tq, H_I,
+                                            _ptr(pool), pool_blocks, top_k, _ptr(topk_out),
+                                            _ptr(topk_count), _ptr(workspace), ws_bytes, _ptr(dev_err),
+                                            _stream(stream))
+    _check("csa2_index_reindex_paged_settled", st)
+
+
+def csa2_sparse_attn_decode_paged_reuse(kv: CSA2PagedKV, swa: CSA2SWA | None, swa_bf16, q, q_pos,
+                                        Tq: int, H: int, topk, top_k: int, swa_len: int,
+                                        softmax_scale: float, rope, out, lse, dev_err=None, stream=None):
+    """csa2_sparse_attn_decode_reuse on a paged cache."""
+    L = load_library()
+    st = L.csa2_sparse_attn_decode_paged_reuse(
+        C.byref(kv), C.byref(swa) if swa is not None else None, _ptr(swa_bf16), _ptr(q), _ptr(q_pos),
+        Tq, H, _ptr(topk), top_k, swa_len, softmax_scale, C.byref(rope) if rope is not None else None,
+        _ptr(out), _ptr(lse), _ptr(dev_err), _stream(stream))
+    _check("csa2_sparse_attn_decode_paged_reuse", st)
 
 
 def csa2_index_reindex_settled(kv: CSA2GlobalKV, q_idx, w, q_pos, Tq: int, H_I: int, pool,

@@ -136,7 +136,7 @@ bool hi_supported(int32_t H_I) {
 
 extern "C" {
 
-int32_t csa2_abi_version(void) { return 105; }
+int32_t csa2_abi_version(void) { return 106; }
 
 void csa2_debug_set_waits(uint64_t limit_ns, int32_t stuck_wait) {
     g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
@@ -591,25 +591,43 @@ csa2_status csa2_index_full_paged(const csa2_paged_kv *kv, const void *q_idx_bf1
                       topk_count, workspace, ws_bytes, dev_err, stream, false);
 }
 
-csa2_status csa2_index_reindex_paged(const csa2_paged_kv *kv, const void *q_idx_bf16, const float *w,
-                                     const int32_t *q_pos, int32_t Tq, int32_t H_I, const int32_t *pool,
-                                     int32_t pool_blocks, int32_t top_k, int32_t *topk_out,
-                                     int32_t *topk_count, void *workspace, size_t ws_bytes,
-                                     int32_t *dev_err, csa2_stream_t stream) {
+static csa2_status reindex_paged(const csa2_paged_kv *kv, const void *q_idx_bf16, const float *w,
+                                 const int32_t *q_pos, int32_t Tq, int32_t H_I, const int32_t *pool,
+                                 int32_t pool_blocks, int32_t top_k, int32_t *topk_out,
+                                 int32_t *topk_count, void *workspace, size_t ws_bytes,
+                                 int32_t *dev_err, csa2_stream_t stream, bool settled) {
     KvView v;
     const KvView *pv;
     csa2_status st = paged_view(kv, &v, &pv);
     if (st != CSA2_OK) return st;
     return index_reindex(pv, q_idx_bf16, w, q_pos, Tq, H_I, pool, pool_blocks, top_k, topk_out,
-                         topk_count, workspace, ws_bytes, dev_err, stream);
+                         topk_count, workspace, ws_bytes, dev_err, stream, settled);
 }
 
-csa2_status csa2_sparse_attn_decode_paged(const csa2_paged_kv *kv, const csa2_swa *swa,
-                                          const void *swa_bf16, const void *q_bf16,
-                                          const int32_t *q_pos, int32_t Tq, int32_t H,
-                                          const int32_t *topk, int32_t top_k, int32_t swa_len,
-                                          float softmax_scale, const csa2_rope *rope, float *out,
-                                          float *lse, int32_t *dev_err, csa2_stream_t stream) {
+csa2_status csa2_index_reindex_paged(const csa2_paged_kv *kv, const void *q_idx_bf16, const float *w,
+                                     const int32_t *q_pos, int32_t Tq, int32_t H_I, const int32_t *pool,
+                                     int32_t pool_blocks, int32_t top_k, int32_t *topk_out,
+                                     int32_t *topk_count, void *workspace, size_t ws_bytes,
+                                     int32_t *dev_err, csa2_stream_t stream) {
+    return reindex_paged(kv, q_idx_bf16, w, q_pos, Tq, H_I, pool, pool_blocks, top_k, topk_out, topk_count,
+                         workspace, ws_bytes, dev_err, stream, false);
+}
+
+csa2_status csa2_index_reindex_paged_settled(const csa2_paged_kv *kv, const void *q_idx_bf16,
+                                             const float *w, const int32_t *q_pos, int32_t Tq,
+                                             int32_t H_I, const int32_t *pool, int32_t pool_blocks,
+                                             int32_t top_k, int32_t *topk_out, int32_t *topk_count,
+                                             void *workspace, size_t ws_bytes, int32_t *dev_err,
+                                             csa2_stream_t stream) {
+    return reindex_paged(kv, q_idx_bf16, w, q_pos, Tq, H_I, pool, pool_blocks, top_k, topk_out, topk_count,
+                         workspace, ws_bytes, dev_err, stream, true);
+}
+
+static csa2_status attn_paged(const csa2_paged_kv *kv, const csa2_swa *swa, const void *swa_bf16,
+                              const void *q_bf16, const int32_t *q_pos, int32_t Tq, int32_t H,
+                              const int32_t *topk, int32_t top_k, int32_t swa_len, float softmax_scale,
+                              const csa2_rope *rope, float *out, float *lse, int32_t *dev_err,
+                              csa2_stream_t stream, bool settled) {
     KvView v;
     const KvView *pv;
     csa2_status st = paged_view(kv, &v, &pv);
@@ -622,7 +640,27 @@ csa2_status csa2_sparse_attn_decode_paged(const csa2_paged_kv *kv, const csa2_sw
         return CSA2_ERR_INVALID_ARG;
     }
     return sparse_attn(pv, swa, swa_bf16, q_bf16, q_pos, Tq, H, topk, top_k, swa_len, softmax_scale,
-                       rope, out, lse, dev_err, stream);
+                       rope, out, lse, dev_err, stream, settled);
+}
+
+csa2_status csa2_sparse_attn_decode_paged(const csa2_paged_kv *kv, const csa2_swa *swa,
+                                          const void *swa_bf16, const void *q_bf16,
+                                          const int32_t *q_pos, int32_t Tq, int32_t H,
+                                          const int32_t *topk, int32_t top_k, int32_t swa_len,
+                                          float softmax_scale, const csa2_rope *rope, float *out,
+                                          float *lse, int32_t *dev_err, csa2_stream_t stream) {
+    return attn_paged(kv, swa, swa_bf16, q_bf16, q_pos, Tq, H, topk, top_k, swa_len, softmax_scale, rope, out,
+                      lse, dev_err, stream, false);
+}
+
+csa2_status csa2_sparse_attn_decode_paged_reuse(const csa2_paged_kv *kv, const csa2_swa *swa,
+                                                const void *swa_bf16, const void *q_bf16,
+                                                const int32_t *q_pos, int32_t Tq, int32_t H,
+                                                const int32_t *topk, int32_t top_k, int32_t swa_len,
+                                                float softmax_scale, const csa2_rope *rope, float *out,
+                                                float *lse, int32_t *dev_err, csa2_stream_t stream) {
+    return attn_paged(kv, swa, swa_bf16, q_bf16, q_pos, Tq, H, topk, top_k, swa_len, softmax_scale, rope, out,
+                      lse, dev_err, stream, true);
 }
 
 csa2_status csa2_read_device_error(int32_t *dev_err, int32_t *bits_out, csa2_stream_t stream) {

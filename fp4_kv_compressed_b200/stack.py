@@ -103,6 +103,10 @@ class PagedKV:
                                        self.block_table.data_ptr(), B, max_pages, page_size,
                                        n_pages, d_idx, ratio)
 
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in
+                   (self.codes, self.scales, self.idx_codes, self.idx_scale, self.block_table))
+
     def rows_of(self, b: int, n: int) -> torch.Tensor:
         """Pool rows of entries 0..n-1 of request b."""
         e = torch.arange(n, device=self.block_table.device)
@@ -124,9 +128,16 @@ class DecodeStack:
 
     def __init__(self, B: int, H: int, H_I: int, d_idx: int, top_k: int, swa_len: int,
                  groups: list[GroupSpec], Tq: int = 1, window_cap: int | None = None,
-                 device="cuda", index_scan: str = "exact", rope=None):
+                 device="cuda", index_scan: str = "exact", rope=None, page_size: int = 0,
+                 page_seed: int = 0):
         if index_scan not in ("exact", "tc"):
             raise ValueError(f"index_scan must be 'exact' or 'tc', not {index_scan!r}")
+        if page_size and index_scan != "exact":
+            raise ValueError("the paged calls take the exact Full scan")
+        # page_size > 0: each group's cache lives in pages of page_size entries (a pool of
+        # B * ceil(cap / page_size) pages per group, handed to the requests in a seeded
+        # random order through block tables) and every call takes its _paged form
+        self.page_size = page_size
         # "exact": the fixed fp32 score order (reproducible Top-K); "tc": the tensor-core
         # scan for prefill chunks (relaxed summation order, see csa2_index_full_tc)
         self.index_scan = index_scan
@@ -143,7 +154,15 @@ class DecodeStack:
         self.device = torch.device(device)
         self.window_cap = window_cap or (swa_len + Tq - 1)
         self.plan = plan_layers([g.schedule for g in groups])
-        self.kv = [GlobalKV(B, g.cap, d_idx, g.ratio, device) for g in groups]
+        if page_size:
+            self.kv = []
+            for i, g in enumerate(groups):
+                max_pages = -(-g.cap // page_size)
+                perm = torch.randperm(B * max_pages, generator=torch.Generator().manual_seed(page_seed + i))
+                self.kv.append(PagedKV(B, max_pages, page_size, B * max_pages, d_idx, g.ratio,
+                                       perm.to(torch.int32).view(B, max_pages), device))
+        else:
+            self.kv = [GlobalKV(B, g.cap, d_idx, g.ratio, device) for g in groups]
         self.swa = [SwaRing(B, self.window_cap, device) for _ in self.plan]
         BT = B * Tq
         dev = self.device
@@ -196,8 +215,12 @@ class DecodeStack:
         T_swa = swa_bf16[0].shape[1] if swa_bf16[0] is not None else 0
         rope = self.rope.struct if self.rope is not None else None
 
+        paged = self.page_size > 0
+
         def append(*args):
-            if rope is None:
+            if paged and args[0] is not None:
+                bind.csa2_quantize_append_paged(*args, rope, self.dev_err, stream)
+            elif rope is None:
                 bind.csa2_quantize_append(*args, self.dev_err, stream)
             else:
                 bind.csa2_quantize_append_rope(*args, rope, self.dev_err, stream)
@@ -214,6 +237,8 @@ class DecodeStack:
             spec = self.groups[g]
             if lp.mode == "F":
                 full = bind.csa2_index_full_tc if self.index_scan == "tc" else bind.csa2_index_full
+                if paged:
+                    full = bind.csa2_index_full_paged
                 full(kv.struct, q_idx[l], w[l], q_pos, self.Tq, self.H_I, n_max[g],
                      spec.pool_blocks, self.top_k, self.pool[g] if spec.pool_blocks else None,
                      self.topk[l], self.count[l], self.workspace, self.dev_err, stream)
@@ -221,13 +246,24 @@ class DecodeStack:
                 # the pool comes from the group's Full layer, whose attention launched in
                 # between: the scoring may overlap the previous launch (unless this layer's
                 # own SWA append was just launched, which the scoring does not read either)
-                reindex = bind.csa2_index_reindex_settled if self.reuse_launch else bind.csa2_index_reindex
+                if paged:
+                    reindex = bind.csa2_index_reindex_paged_settled if self.reuse_launch \
+                        else bind.csa2_index_reindex_paged
+                else:
+                    reindex = bind.csa2_index_reindex_settled if self.reuse_launch else bind.csa2_index_reindex
                 reindex(kv.struct, q_idx[l], w[l], q_pos, self.Tq, self.H_I, self.pool[g],
                         spec.pool_blocks, self.top_k, self.topk[l], self.count[l], self.workspace,
                         self.dev_err, stream)
             fused = (l != first_of_group[g] or kv_bf16 is None or kv_bf16[g] is None) \
                 and swa_bf16[l] is not None and self._fuse_swa(T_swa)
-            if fused and lp.mode == "U" and self.reuse_launch:
+            if paged:
+                attn = bind.csa2_sparse_attn_decode_paged_reuse if fused and lp.mode == "U" and self.reuse_launch \
+                    else bind.csa2_sparse_attn_decode_paged
+                attn(
+                    kv.struct, self.swa[l].struct, swa_bf16[l] if fused else None, q[l], q_pos, self.Tq,
+                    self.H, self.topk_of(l), self.top_k, self.swa_len, self.softmax_scale,
+                    rope if fused else None, self.out[l], self.lse[l], self.dev_err, stream)
+            elif fused and lp.mode == "U" and self.reuse_launch:
                 # a Reuse layer: its Top-K and every other input were written two or more
                 # launches back (the source layer's attention launched in between), so
                 # the launch overlaps the previous one

@@ -517,6 +517,26 @@ CSA2_API csa2_status csa2_sparse_attn_decode_paged(const csa2_paged_kv *kv, cons
                                                    const csa2_rope *rope, float *out, float *lse,
                                                    int32_t *dev_err, csa2_stream_t stream);
 
+/* The overlapping launches of the Reindex and Reuse layers on a paged cache: as
+ * csa2_index_reindex_settled and csa2_sparse_attn_decode_reuse (same arguments as the
+ * two calls above, the same preconditions, and results bit for bit equal to those
+ * calls; the block table counts among the inputs that the previous launch must not
+ * write). */
+CSA2_API csa2_status csa2_index_reindex_paged_settled(const csa2_paged_kv *kv, const void *q_idx_bf16,
+                                                      const float *w, const int32_t *q_pos, int32_t Tq,
+                                                      int32_t H_I, const int32_t *pool,
+                                                      int32_t pool_blocks, int32_t top_k,
+                                                      int32_t *topk_out, int32_t *topk_count,
+                                                      void *workspace, size_t ws_bytes,
+                                                      int32_t *dev_err, csa2_stream_t stream);
+CSA2_API csa2_status csa2_sparse_attn_decode_paged_reuse(const csa2_paged_kv *kv, const csa2_swa *swa,
+                                                         const void *swa_bf16, const void *q_bf16,
+                                                         const int32_t *q_pos, int32_t Tq, int32_t H,
+                                                         const int32_t *topk, int32_t top_k,
+                                                         int32_t swa_len, float softmax_scale,
+                                                         const csa2_rope *rope, float *out, float *lse,
+                                                         int32_t *dev_err, csa2_stream_t stream);
+
 /* Synchronise `stream`, read *dev_err (device int32) into *bits_out (host),
  * reset it to 0, and return CSA2_ERR_DEVICE_BOUNDS if any bit was set. */
 CSA2_API csa2_status csa2_read_device_error(int32_t *dev_err, int32_t *bits_out, csa2_stream_t stream);

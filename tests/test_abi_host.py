@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol(pkg):
     assert set(names) == set(pkg.EXPORTS)
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.csa2_abi_version() == 105      # 1.5: the Reuse-layer attention launch
+    assert lib.csa2_abi_version() == 106      # 1.6: the paged forms of the overlapping launches
     for st in range(7):
         assert lib.csa2_status_string(st)
 
@@ -113,6 +113,14 @@ def test_validation_rejects_before_launch(pkg):
     assert lib.csa2_sparse_attn_decode_reuse(C.byref(kv), C.byref(swa), None, qbuf, qbuf, 1, 64, qbuf,
                                              8, 128, C.c_float(0.04), C.byref(rope_ok), qbuf, qbuf, None,
                                              None) == 1
+    # their paged forms: a page size that is not a power of two >= 256 is refused first
+    pk = pkg.CSA2PagedKV(256, 256, 256, 256, 4096, 1, 4, 100, 8, 128, 1)
+    assert lib.csa2_index_reindex_paged_settled(C.byref(pk), qbuf, qbuf, qbuf, 1, 4, qbuf, 64, 64, qbuf,
+                                                qbuf, qbuf, 1 << 20, None, None) == 4
+    assert lib.csa2_sparse_attn_decode_paged_reuse(C.byref(pk), C.byref(swa), None, qbuf, qbuf, 1, 64, qbuf,
+                                                   8, 128, C.c_float(0.04), None, qbuf, qbuf, None, None) == 4
+    assert lib.csa2_sparse_attn_decode_paged_reuse(None, C.byref(swa), None, qbuf, qbuf, 1, 64, qbuf,
+                                                   8, 128, C.c_float(0.04), None, qbuf, qbuf, None, None) == 1
     # RoPE descriptors: null table, odd start, range past channel 511, no pairs, no rows,
     # misaligned table -- each rejected before any launch, in both _rope calls
     for bad in [(0, 8, 0, 4), (4096, 8, 3, 4), (4096, 8, 500, 8), (4096, 8, 0, 0),

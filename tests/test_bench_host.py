@@ -120,6 +120,15 @@ def test_op_rooflines_dominant_and_traffic():
     assert per_r["csa2_index_reindex_settled"][1] == 4 and "csa2_index_reindex" not in per_r
     assert per_r["csa2_sparse_attn_decode_reuse"][0] == 15 * per["csa2_sparse_attn_decode_append"][0] // 19
     assert sum(b for b, _ in per_r.values()) == bench.step_bytes(wl)
+    # paged caches: every call in its _paged form, the same bytes and launches
+    per_p = bench.op_step_bytes(wl, plan, paged=True)
+    assert set(per_p) == {"csa2_quantize_append_paged", "csa2_index_full_paged", "csa2_index_reindex_paged_settled",
+                          "csa2_sparse_attn_decode_paged", "csa2_sparse_attn_decode_paged_reuse"}
+    assert per_p["csa2_sparse_attn_decode_paged_reuse"][1] == 15 and per_p["csa2_sparse_attn_decode_paged"][1] == 5
+    assert per_p["csa2_index_reindex_paged_settled"][1] == 4
+    assert bench.op_step_bytes(wl, plan, reuse=False, paged=True)["csa2_index_reindex_paged"][1] == 4
+    assert sum(b for b, _ in per_p.values()) == bench.step_bytes(wl)
+    assert sum(n for _, n in per_p.values()) == sum(n for _, n in per.values())
     op_ms = {"csa2_quantize_append": (0.005, 1), "csa2_index_full": (0.4, 1),
              "csa2_index_reindex": (0.4, 4), "csa2_sparse_attn_decode": (0.03, 1),
              "csa2_sparse_attn_decode_append": (0.665, 19)}

@@ -155,3 +155,31 @@ def test_bad_page_is_flagged_not_read(pkg):
     pkg.csa2_sparse_attn_decode_paged(pk.struct, None, None, q, t, 1, 16, topk, 512, 0, 0.05, None, o, l, err)
     assert pkg.csa2_read_device_error(err) & pkg.DEVERR_PAGE
     assert torch.isfinite(o).all() and torch.isfinite(l).all()
+
+
+@pytest.mark.parametrize("name,B,ctx,page", [("decoder_group_32k", 3, 20005, 256), ("decode_1m", 2, 6001, 1024)])
+def test_paged_stack_equals_contiguous(pkg, name, B, ctx, page):
+    """One decode step of the whole layer loop on paged caches (each group's pages handed
+    to the requests in a shuffled order) equals the same step on contiguous caches, bit
+    for bit: every layer's Top-K, counts, outputs and lse, and every group's pool."""
+    import csa2_harness
+    from synth.workloads import WORKLOADS, small_variant
+    wl = small_variant(WORKLOADS[name], B=B, ctx=ctx)
+    res = []
+    for page_size in (0, page):
+        dw = csa2_harness.DeviceWorkload(wl, page_size=page_size)
+        dw.step()
+        torch.cuda.synchronize()
+        st = dw.stack
+        assert st.dev_err.item() == 0
+        res.append(({l: t.cpu() for l, t in st.topk.items()}, {l: c.cpu() for l, c in st.count.items()},
+                    {g: p.cpu() for g, p in st.pool.items()}, [o.cpu() for o in st.out],
+                    [x.cpu() for x in st.lse]))
+        del dw, st
+    (t0, c0, p0, o0, l0), (t1, c1, p1, o1, l1) = res
+    for l in t0:
+        assert torch.equal(t0[l], t1[l]) and torch.equal(c0[l], c1[l]), f"layer {l}"
+    for g in p0:
+        assert torch.equal(p0[g], p1[g]), f"group {g}"
+    for l in range(len(o0)):
+        assert torch.equal(o0[l], o1[l]) and torch.equal(l0[l], l1[l]), f"layer {l} output"
