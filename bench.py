@@ -680,7 +680,6 @@ def run_cp(args) -> dict:
     of the combine, beside the unsplit csa2_index_full and csa2_sparse_attn_decode on the
     same cache.  The two all-gathers between the steps need several GPUs and are not
     run; their bytes per step are reported."""
-    import statistics
     import torch
     from synth.workloads import WORKLOADS
     import csa2_harness
